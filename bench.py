@@ -1,0 +1,421 @@
+#!/usr/bin/env python
+"""Throughput of one mHC layer, forward + backward, on B200.
+
+A step is one pass of the whole hot path over one batch of synthetic tokens:
+  mhc_pre -> mhc_post (with a supplied f_out standing in for F's output) ->
+  mhc_backward_map -> mhc_backward_apply
+at T = 16384 tokens per GPU, n = 4 streams, C = 7168 channels, bf16
+activations, Sinkhorn t_max = 20.  Under torchrun each rank runs its own
+16384 tokens (data parallel over tokens, weak scaling) and the step ends with
+the one exchange the backward has: an all-reduce of grad_phi / grad_b /
+grad_alpha (2.75 MB).
+
+Timing: W warm-up steps, then exactly K steps between a barrier +
+synchronize on each side, CUDA events on the launching stream, max over
+ranks.  Every input tensor (x, grad_x_next: 940 MB each) is larger than the
+126 MB L2, so no flush is needed between steps.  CUDA events recorded
+between the calls give each call's device time; the roofline line is taken
+for the longest single-kernel call.
+
+``--impl reference`` times the fp64 CPU oracle (the reference arm of this
+library) on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "mHC layer tokens/s (fwd+bwd, n=4, C=7168) and achieved HBM GB/s vs B200 peak"
+T_TOK, N_STR, C_CH, T_MAX = 16384, 4, 7168, 20
+FALLBACK_HBM_GBS = 6650.0
+
+
+def per_token_bytes(n=N_STR, C=C_CH, act=2):
+    """Algorithmic bytes per token of each call (bf16 activations, fp32 maps)."""
+    M = n * n + 2 * n
+    nC = n * C
+    coef = ((n * n + 2 * n + M + 1) + 3) // 4 * 4 * 4  # per-token record of the split backward
+    return {
+        "pre": nC * act + C * act + 4 * (2 * n + n * n),                  # x in; h_in, H out
+        "post": nC * act + C * act + 4 * (n + n * n) + nC * act,           # x, f, H in; x_next out
+        "bwd_map": 2 * nC * act + 2 * C * act + coef,                      # x, G, g, f in; records out
+        "bwd_apply": 2 * nC * act + C * act + coef + nC * act + C * act,   # x, G, g, records in; grads out
+        "bwd_min": 2 * nC * act + 2 * C * act + nC * act + C * act,        # one pass: x, G, g, f in; grads out
+    }
+
+
+def per_call_param_bytes(n=N_STR, C=C_CH):
+    K, M = n * C, n * n + 2 * n
+    phi = K * M * 4
+    return {"pre": phi, "post": 0, "bwd_map": phi, "bwd_apply": 2 * phi}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_sha(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "manifold_constrained_hyper_token_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+# kernels behind each single-kernel call, for matching ncu traffic to sources
+CALL_SOURCES = {
+    "post": ["k_post.cu", "mhc_common.cuh"],
+    "bwd_map": ["k_map.cu", "mhc_common.cuh"],
+    "bwd_apply": ["k_bwd.cu", "mhc_common.cuh"],
+    "pre": ["k_map.cu", "k_post.cu", "mhc_common.cuh"],
+}
+
+
+def ncu_traffic(call):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current source of that kernel; else None."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d[call]
+        if e.get("source_sha") != kernel_source_sha(CALL_SOURCES[call]):
+            return None
+        return float(e["bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) >= 9]
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for k, v in zip(names, r[5:9]):
+                if v.strip().lower().startswith("active"):
+                    reasons.add(k)
+        sm.sort()
+        med = sm[len(sm) // 2] if sm else None
+        return {"sm_mhz": med, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_reference(seconds: float, seed: int = 0):
+    """The fp64 oracle, as it stands, on the first S tokens of the same workload:
+    pre + post + backward.  S is grown until one pass takes about `seconds`."""
+    import torch
+
+    import oracle
+    from manifold_constrained_hyper_token_b200 import synth
+
+    params = synth.layer_params(N_STR, C_CH, seed)
+    alpha = float(params["alpha"][0])
+
+    def run(S):
+        d = synth.activations(S, N_STR, C_CH, seed, torch.bfloat16, backward=True)
+        t0 = time.perf_counter()
+        o = oracle.pre(d["x"], params["phi"], params["b"], alpha, iters=T_MAX)
+        oracle.post(d["x"], d["f_out"], o["H_post"], o["H_res"])
+        oracle.backward(d["x"], params["phi"], params["b"], alpha, d["f_out"], d["grad_x_next"],
+                        d["grad_h_in"], iters=T_MAX)
+        return time.perf_counter() - t0
+
+    S = 32
+    dt = run(S)
+    while dt < seconds / 4 and S < 8192:
+        S = min(8192, int(S * max(2.0, min(8.0, seconds / max(dt, 1e-3) / 2))))
+        dt = run(S)
+    return {"value": S / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"first {S} tokens of the T={T_TOK}, n={N_STR}, C={C_CH} bf16 workload, "
+                      f"pre+post+backward in fp64, {dt:.2f} s"}
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the fp64 oracle on the host cores.  Each step runs
+    pre + post + backward on a bounded sample of S tokens of the same
+    workload; S is chosen from a short calibration so that the whole
+    W + K step run takes about two minutes."""
+    if rank != 0:
+        return
+    import torch
+
+    import oracle
+    from manifold_constrained_hyper_token_b200 import synth
+
+    params = synth.layer_params(N_STR, C_CH, 0)
+    alpha = float(params["alpha"][0])
+    pool = synth.activations(256, N_STR, C_CH, 0, torch.bfloat16, backward=True)
+
+    def one(S):
+        d = {k: v[:S] for k, v in pool.items()}
+        t0 = time.perf_counter()
+        o = oracle.pre(d["x"], params["phi"], params["b"], alpha, iters=T_MAX)
+        oracle.post(d["x"], d["f_out"], o["H_post"], o["H_res"])
+        oracle.backward(d["x"], params["phi"], params["b"], alpha, d["f_out"], d["grad_x_next"],
+                        d["grad_h_in"], iters=T_MAX)
+        return time.perf_counter() - t0
+
+    rate = 32 / one(32)
+    S = int(max(1, min(256, 120.0 * rate / (args.warmup + args.steps))))
+    for _ in range(args.warmup):
+        one(S)
+    total = sum(one(S) for _ in range(args.steps))
+    val = args.steps * S / total
+    cb = {"value": val, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+          "sample": f"{S} tokens per step of the T={T_TOK}, n={N_STR}, C={C_CH} bf16 workload, "
+                    f"pre+post+backward in fp64"}
+    line = {"metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1000.0 * T_TOK / val, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": f"mHC layer fwd+bwd per GPU: T={T_TOK} tokens, n={N_STR}, "
+                                   f"C={C_CH}, t_max={T_MAX}, bf16 activations, fp32 maps",
+                       "T_per_gpu": T_TOK, "n": N_STR, "C": C_CH, "t_max": T_MAX,
+                       "parallelism": "host cores (oracle)"},
+            "cpu_baseline": cb,
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-sample-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import manifold_constrained_hyper_token_b200 as mhc
+    from manifold_constrained_hyper_token_b200 import synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    T, n, C = T_TOK, N_STR, C_CH
+    K, M = n * C, n * n + 2 * n
+    prm = synth.layer_params(n, C, seed=0)
+    act = synth.activations(T, n, C, seed=rank, dtype=torch.bfloat16, backward=True)
+    phi, b, alpha = (prm["phi"].to(dev), prm["b"].to(dev), prm["alpha"].to(dev))
+    x, f_out = act["x"].to(dev), act["f_out"].to(dev)
+    G, g = act["grad_x_next"].to(dev), act["grad_h_in"].to(dev)
+    h_in = torch.empty(T, C, dtype=torch.bfloat16, device=dev)
+    Hpre = torch.empty(T, n, dtype=torch.float32, device=dev)
+    Hpost = torch.empty(T, n, dtype=torch.float32, device=dev)
+    Hres = torch.empty(T, n, n, dtype=torch.float32, device=dev)
+    x_next = torch.empty_like(x)
+    gx = torch.empty_like(x)
+    gf = torch.empty_like(f_out)
+    pgrads = torch.empty(K * M + M + 1, dtype=torch.float32, device=dev)  # one all-reduce buffer
+    gphi, gb, ga = pgrads[:K * M].view(K, M), pgrads[K * M:K * M + M], pgrads[K * M + M:]
+    ws = torch.empty(mhc.mhc_backward_workspace_size(n, T, C, torch.bfloat16), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream()
+    calls = ["pre", "post", "bwd_map", "bwd_apply"]
+    launches_per_call = {"pre": 2, "post": 1, "bwd_map": 1, "bwd_apply": 1}
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record(stream)
+        mhc.mhc_pre(x, phi, b, alpha, t_max=T_MAX, out=(h_in, Hpre, Hpost, Hres), stream=stream)
+        if evs is not None:
+            evs[1].record(stream)
+        mhc.mhc_post(x, f_out, Hpost, Hres, out=x_next, stream=stream)
+        if evs is not None:
+            evs[2].record(stream)
+        mhc.mhc_backward_map(x, phi, b, alpha, f_out, G, g, ws, t_max=T_MAX, stream=stream)
+        if evs is not None:
+            evs[3].record(stream)
+        mhc.mhc_backward_apply(x, phi, G, g, ws, t_max=T_MAX, out=(gx, gphi, gb, ga, gf),
+                               stream=stream)
+        if evs is not None:
+            evs[4].record(stream)
+        if world > 1:
+            dist.all_reduce(pgrads)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)  # let the sampler come up before the timed region
+    t_start.record(stream)
+    for s in range(args.steps):
+        step(evs[s])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    per_call = {c: 0.0 for c in calls}
+    for s in range(args.steps):
+        for i, c in enumerate(calls):
+            per_call[c] += evs[s][i].elapsed_time(evs[s][i + 1])
+    per_call = {c: v / args.steps for c, v in per_call.items()}
+    if world > 1:
+        tt = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(tt.item())
+    ms_per_step = elapsed_ms / args.steps
+    tokens_per_s = T * world / (ms_per_step / 1000.0)
+
+    # ---- roofline of the longest single-kernel call, and the whole step
+    peak, peak_kind = load_peaks()
+    tb = per_token_bytes(n, C)
+    pb = per_call_param_bytes(n, C)
+    call_bytes = {c: T * tb[c] + pb[c] for c in calls}
+    single = [c for c in calls if launches_per_call[c] == 1]
+    dom = max(single, key=lambda c: per_call[c])
+    achieved = call_bytes[dom] / (per_call[dom] / 1000.0) / 1e9
+    traffic = ncu_traffic(dom)
+    step_alg_bytes = T * (tb["pre"] + tb["post"] + tb["bwd_min"]) + pb["pre"] + pb["bwd_apply"]
+    step_gbs = step_alg_bytes / (ms_per_step / 1000.0) / 1e9
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        hx, hf = act["x"].pin_memory(), act["f_out"].pin_memory()
+        hG, hg = act["grad_x_next"].pin_memory(), act["grad_h_in"].pin_memory()
+        hout = torch.empty(K * M + M + 1, dtype=torch.float32).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (hx, hf, hG, hg))
+        d2h = hout.numel() * hout.element_size()
+
+        def e2e_step():
+            x.copy_(hx, non_blocking=True)
+            f_out.copy_(hf, non_blocking=True)
+            G.copy_(hG, non_blocking=True)
+            g.copy_(hg, non_blocking=True)
+            step()
+            hout.copy_(pgrads, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1) / args.e2e_steps
+        if world > 1:
+            tt = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        e2e = {"value": T * world / (e_ms / 1000.0), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+               "ms_per_step": e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_reference(args.cpu_sample_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": f"mHC layer fwd+bwd per GPU: T={T} tokens, n={n}, C={C}, "
+                                   f"t_max={T_MAX}, bf16 activations, fp32 maps",
+                       "T_per_gpu": T, "n": n, "C": C, "t_max": T_MAX,
+                       "parallelism": f"dp{world} over tokens",
+                       "l2": "inputs larger than L2 (x and grad_x_next are 940 MB each); no flush"},
+            "hbm": {"achieved_gbs": step_gbs, "peak_gbs": peak, "frac": step_gbs / peak,
+                    "peak_kind": peak_kind,
+                    "alg_bytes_per_step": step_alg_bytes},
+            "per_call_ms": per_call,
+            "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
+                         "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                         "alg_bytes_per_launch": call_bytes[dom], "peak_kind": peak_kind},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": args.steps * sum(launches_per_call.values()),
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

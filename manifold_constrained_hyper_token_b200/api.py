@@ -1,0 +1,188 @@
+"""Thin Python binding of libmhc.so (include/mhc.h).
+
+Each function has the name of the C entry point it calls and only marshals
+arguments: tensors become device pointers, shapes become an ``mhc_params``,
+the stream is the current torch stream unless one is given.  Output tensors
+are allocated with torch when the caller does not pass them.  Every step of
+the computation runs in the library's CUDA kernels; a non-zero status raises
+``MhcError``.  Tensors must be contiguous CUDA tensors.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+
+DTYPE_CODE = {torch.float32: 0, torch.bfloat16: 1}
+
+
+class MhcError(RuntimeError):
+    """A libmhc entry point returned a non-zero mhc_status."""
+
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {mhc_status_string(status)}")
+
+
+def mhc_version() -> int:
+    return int(_lib.load().mhc_version())
+
+
+def mhc_status_string(status: int) -> str:
+    return _lib.load().mhc_status_string(int(status)).decode()
+
+
+def _check(st: int, where: str) -> None:
+    if st != 0:
+        raise MhcError(st, where)
+
+
+def _p(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libmhc takes CUDA tensors only")
+    if not t.is_contiguous():
+        raise ValueError("libmhc takes contiguous tensors only")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def params(n: int, T: int, C: int, dtype: torch.dtype, t_max: int = 20, eps: float = 1e-6):
+    """Build an ``mhc_params`` struct."""
+    if dtype not in DTYPE_CODE:
+        raise ValueError(f"unsupported activation dtype {dtype}")
+    return _lib.MhcParams(n=int(n), t_max=int(t_max), T=int(T), C=int(C), eps=float(eps),
+                          dtype=DTYPE_CODE[dtype])
+
+
+def mhc_pre_workspace_size(n: int, T: int, C: int, dtype: torch.dtype, t_max: int = 20,
+                           eps: float = 1e-6) -> int:
+    p = params(n, T, C, dtype, t_max, eps)
+    return int(_lib.load().mhc_pre_workspace_size(ctypes.byref(p)))
+
+
+def mhc_backward_workspace_size(n: int, T: int, C: int, dtype: torch.dtype, t_max: int = 20,
+                                eps: float = 1e-6) -> int:
+    p = params(n, T, C, dtype, t_max, eps)
+    return int(_lib.load().mhc_backward_workspace_size(ctypes.byref(p)))
+
+
+def _workspace(nbytes: int, device, ws):
+    if nbytes == 0:
+        return None, 0
+    if ws is None:
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return ws, ws.numel() * ws.element_size()
+
+
+def mhc_pre(x, phi, b, alpha, *, t_max: int = 20, eps: float = 1e-6, out=None, workspace=None,
+            dev_status=None, stream=None):
+    """x [T,n,C] -> (h_in [T,C], H_pre [T,n], H_post [T,n], H_res [T,n,n])."""
+    T, n, C = x.shape
+    p = params(n, T, C, x.dtype, t_max, eps)
+    if out is None:
+        out = (torch.empty(T, C, dtype=x.dtype, device=x.device),
+               torch.empty(T, n, dtype=torch.float32, device=x.device),
+               torch.empty(T, n, dtype=torch.float32, device=x.device),
+               torch.empty(T, n, n, dtype=torch.float32, device=x.device))
+    h_in, H_pre, H_post, H_res = out
+    lib = _lib.load()
+    ws, wsb = _workspace(int(lib.mhc_pre_workspace_size(ctypes.byref(p))), x.device, workspace)
+    st = lib.mhc_pre(ctypes.byref(p), _p(x), _p(phi), _p(b), _p(alpha), _p(h_in), _p(H_pre),
+                     _p(H_post), _p(H_res), _p(ws), wsb, _p(dev_status), _stream(stream))
+    _check(st, "mhc_pre")
+    return h_in, H_pre, H_post, H_res
+
+
+def mhc_post(x, f_out, H_post, H_res, *, out=None, dev_status=None, stream=None):
+    """x [T,n,C], f_out [T,C], H_post [T,n], H_res [T,n,n] -> x_next [T,n,C]."""
+    T, n, C = x.shape
+    p = params(n, T, C, x.dtype)
+    x_next = torch.empty_like(x) if out is None else out
+    st = _lib.load().mhc_post(ctypes.byref(p), _p(x), _p(f_out), _p(H_post), _p(H_res),
+                              _p(x_next), _p(dev_status), _stream(stream))
+    _check(st, "mhc_post")
+    return x_next
+
+
+def mhc_backward(x, phi, b, alpha, f_out, grad_x_next, grad_h_in, *, t_max: int = 20,
+                 eps: float = 1e-6, out=None, workspace=None, dev_status=None, stream=None):
+    """Gradients of pre+post with recompute.
+    Returns (grad_x, grad_phi, grad_b, grad_alpha, grad_f_out)."""
+    T, n, C = x.shape
+    p = params(n, T, C, x.dtype, t_max, eps)
+    if out is None:
+        out = (torch.empty_like(x), torch.empty_like(phi), torch.empty_like(b),
+               torch.empty_like(alpha), torch.empty_like(f_out))
+    gx, gphi, gb, ga, gf = out
+    lib = _lib.load()
+    ws, wsb = _workspace(int(lib.mhc_backward_workspace_size(ctypes.byref(p))), x.device,
+                         workspace)
+    st = lib.mhc_backward(ctypes.byref(p), _p(x), _p(phi), _p(b), _p(alpha), _p(f_out),
+                          _p(grad_x_next), _p(grad_h_in), _p(gx), _p(gphi), _p(gb), _p(ga),
+                          _p(gf), _p(ws), wsb, _p(dev_status), _stream(stream))
+    _check(st, "mhc_backward")
+    return gx, gphi, gb, ga, gf
+
+
+def mhc_backward_map(x, phi, b, alpha, f_out, grad_x_next, grad_h_in, workspace, *,
+                     t_max: int = 20, eps: float = 1e-6, dev_status=None, stream=None):
+    """Phase 1 of mhc_backward: per-token records into ``workspace`` (uint8 tensor of at
+    least mhc_backward_workspace_size bytes)."""
+    T, n, C = x.shape
+    p = params(n, T, C, x.dtype, t_max, eps)
+    st = _lib.load().mhc_backward_map(ctypes.byref(p), _p(x), _p(phi), _p(b), _p(alpha), _p(f_out),
+                                      _p(grad_x_next), _p(grad_h_in), _p(workspace),
+                                      workspace.numel(), _p(dev_status), _stream(stream))
+    _check(st, "mhc_backward_map")
+
+
+def mhc_backward_apply(x, phi, grad_x_next, grad_h_in, workspace, *, t_max: int = 20,
+                       eps: float = 1e-6, out=None, dev_status=None, stream=None):
+    """Phase 2 of mhc_backward.  Returns (grad_x, grad_phi, grad_b, grad_alpha, grad_f_out)."""
+    T, n, C = x.shape
+    p = params(n, T, C, x.dtype, t_max, eps)
+    M = n * n + 2 * n
+    if out is None:
+        out = (torch.empty_like(x), torch.empty_like(phi),
+               torch.empty(M, dtype=torch.float32, device=x.device),
+               torch.empty(1, dtype=torch.float32, device=x.device),
+               torch.empty(T, C, dtype=x.dtype, device=x.device))
+    gx, gphi, gb, ga, gf = out
+    st = _lib.load().mhc_backward_apply(ctypes.byref(p), _p(x), _p(phi), _p(grad_x_next),
+                                        _p(grad_h_in), _p(gx), _p(gphi), _p(gb), _p(ga), _p(gf),
+                                        _p(workspace), workspace.numel(), _p(dev_status),
+                                        _stream(stream))
+    _check(st, "mhc_backward_apply")
+    return gx, gphi, gb, ga, gf
+
+
+def mhc_sinkhorn_knopp(logits, iters: int = 20, *, out=None, dev_status=None, stream=None):
+    """logits [..., n, n] fp32 -> Sinkhorn-Knopp estimate, same shape."""
+    n = logits.shape[-1]
+    B = logits.numel() // (n * n)
+    res = torch.empty_like(logits) if out is None else out
+    st = _lib.load().mhc_sinkhorn_knopp(int(n), int(iters), int(B), _p(logits), _p(res),
+                                        _p(dev_status), _stream(stream))
+    _check(st, "mhc_sinkhorn_knopp")
+    return res
+
+
+def mhc_depth_amax(H, *, out=None, dev_status=None, stream=None):
+    """H [T, L, n, n] fp32 -> (gain_fwd [T], gain_bwd [T]) of P = H[L-1] ... H[0]."""
+    T, L, n, _ = H.shape
+    if out is None:
+        out = (torch.empty(T, dtype=torch.float32, device=H.device),
+               torch.empty(T, dtype=torch.float32, device=H.device))
+    gf, gb = out
+    st = _lib.load().mhc_depth_amax(int(n), int(T), int(L), _p(H), _p(gf), _p(gb),
+                                    _p(dev_status), _stream(stream))
+    _check(st, "mhc_depth_amax")
+    return gf, gb

@@ -1,0 +1,234 @@
+// mhc_api.cu -- the extern "C" boundary of libmhc.so: argument validation,
+// workspace carving and kernel launches.  No entry point allocates,
+// synchronises or keeps state between calls.
+#include <math.h>
+
+#include "mhc_common.cuh"
+
+namespace mhc {
+// k_sinkhorn.cu
+cudaError_t sinkhorn_dispatch(int n, int iters, int64_t B, const float* logits, float* out,
+                              int* st, cudaStream_t s);
+cudaError_t depth_amax_dispatch(int n, int64_t T, int L, const float* H, float* gf, float* gb,
+                                cudaStream_t s);
+// k_post.cu
+cudaError_t post_dispatch(int n, int dtype, int64_t T, int64_t C, const void* x, const void* f,
+                          const float* Hpost, const float* Hres, void* xn, cudaStream_t s);
+cudaError_t hin_dispatch(int n, int dtype, int64_t T, int64_t C, const void* x, const float* Hpre,
+                         void* h_in, cudaStream_t s);
+// k_map.cu
+cudaError_t map_fwd_dispatch(int n, int dtype, int64_t T, int64_t C, int iters, float eps,
+                             const void* x, const float* phi, const float* b, const float* alpha,
+                             float* Hpre, float* Hpost, float* Hres, int* st, cudaStream_t s);
+cudaError_t map_bwd_dispatch(int n, int dtype, int64_t T, int64_t C, int iters, float eps,
+                             const void* x, const float* phi, const float* b, const float* alpha,
+                             const void* G, const void* g, const void* f, float* coef, float* dzr,
+                             int* st, cudaStream_t s);
+// k_bwd.cu
+cudaError_t apply_dispatch(int n, int dtype, int64_t T, int64_t C, const void* x, const float* phi,
+                           const void* G, const void* g, const float* coef, const float* part,
+                           int nparts, void* gx, void* gf, float* gphi, float* gb, float* ga,
+                           cudaStream_t s);
+}  // namespace mhc
+
+namespace {
+
+constexpr int kVersionMajor = 0;
+constexpr int kVersionMinor = 1;
+
+bool aligned16(const void* p) { return p != nullptr && ((uintptr_t)p & 15u) == 0; }
+
+mhc_status check_params(const mhc_params* p) {
+  if (!p) return MHC_ERR_INVALID_ARG;
+  if (p->T < 1 || p->C < 8 || (p->C % 8) != 0 || p->t_max < 0) return MHC_ERR_INVALID_ARG;
+  if (!(p->eps >= 0.0f) || !isfinite(p->eps)) return MHC_ERR_INVALID_ARG;
+  if (p->n != 1 && p->n != 2 && p->n != 4) return MHC_ERR_UNSUPPORTED;
+  if (p->dtype != MHC_DTYPE_F32 && p->dtype != MHC_DTYPE_BF16) return MHC_ERR_UNSUPPORTED;
+  // token count is bounded by the 1-D grid of the mapping kernel (64 tokens per CTA)
+  if (p->T > (int64_t)64 * 0x7fffffffLL) return MHC_ERR_INVALID_ARG;
+  return MHC_OK;
+}
+
+mhc_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MHC_OK : MHC_ERR_CUDA; }
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+int coef_size(int n) {
+  switch (n) {
+    case 1: return mhc::Coef<1>::SIZE;
+    case 2: return mhc::Coef<2>::SIZE;
+    default: return mhc::Coef<4>::SIZE;
+  }
+}
+int dz_size(int n) {
+  switch (n) {
+    case 1: return mhc::Coef<1>::DZ_SIZE;
+    case 2: return mhc::Coef<2>::DZ_SIZE;
+    default: return mhc::Coef<4>::DZ_SIZE;
+  }
+}
+
+// Backward workspace: per-token coefficient records, then one partial-sum
+// record (dz, dz . y) per 64-token CTA of the mapping kernel.
+constexpr int kMapTokens = 64;
+
+struct BwdWorkspace {
+  size_t coef_off, part_off, total;
+  int nparts;
+};
+
+BwdWorkspace bwd_layout(const mhc_params* p) {
+  BwdWorkspace w;
+  w.nparts = (int)((p->T + kMapTokens - 1) / kMapTokens);
+  w.coef_off = 0;
+  w.part_off = round_up(w.coef_off + (size_t)p->T * coef_size(p->n) * 4, 256);
+  w.total = round_up(w.part_off + (size_t)w.nparts * dz_size(p->n) * 4, 256);
+  return w;
+}
+
+mhc_status check_workspace(const BwdWorkspace& w, void* workspace, size_t bytes) {
+  if (workspace == nullptr || bytes < w.total || ((uintptr_t)workspace & 255u) != 0)
+    return MHC_ERR_WORKSPACE;
+  return MHC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mhc_version(void) { return (kVersionMajor << 16) | kVersionMinor; }
+
+const char* mhc_status_string(int status) {
+  switch (status) {
+    case MHC_OK: return "MHC_OK: success";
+    case MHC_ERR_INVALID_ARG:
+      return "MHC_ERR_INVALID_ARG: null or misaligned pointer, or a size/iteration/eps out of range";
+    case MHC_ERR_UNSUPPORTED: return "MHC_ERR_UNSUPPORTED: stream count n or dtype not built";
+    case MHC_ERR_CUDA: return "MHC_ERR_CUDA: a CUDA runtime call or kernel launch failed";
+    case MHC_ERR_NONFINITE: return "MHC_ERR_NONFINITE: a kernel saw a non-finite RMS or logit";
+    case MHC_ERR_TIMEOUT: return "MHC_ERR_TIMEOUT: a bounded device-side wait gave up";
+    case MHC_ERR_WORKSPACE: return "MHC_ERR_WORKSPACE: workspace missing or too small";
+    default: return "unknown mhc_status";
+  }
+}
+
+size_t mhc_pre_workspace_size(const mhc_params* p) {
+  (void)p;
+  return 0;
+}
+
+mhc_status mhc_pre(const mhc_params* p, const void* x, const float* phi, const float* b,
+                   const float* alpha, void* h_in, float* H_pre, float* H_post, float* H_res,
+                   void* workspace, size_t workspace_bytes, int* dev_status, mhc_stream_t stream) {
+  mhc_status st = check_params(p);
+  if (st != MHC_OK) return st;
+  if (!aligned16(x) || !aligned16(phi) || !aligned16(b) || !aligned16(alpha) || !aligned16(h_in) ||
+      !aligned16(H_pre) || !aligned16(H_post) || !aligned16(H_res))
+    return MHC_ERR_INVALID_ARG;
+  (void)workspace;
+  (void)workspace_bytes;
+  cudaStream_t s = (cudaStream_t)stream;
+  st = from_cuda(mhc::map_fwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
+                                       alpha, H_pre, H_post, H_res, dev_status, s));
+  if (st != MHC_OK) return st;
+  return from_cuda(mhc::hin_dispatch(p->n, p->dtype, p->T, p->C, x, H_pre, h_in, s));
+}
+
+mhc_status mhc_post(const mhc_params* p, const void* x, const void* f_out, const float* H_post,
+                    const float* H_res, void* x_next, int* dev_status, mhc_stream_t stream) {
+  (void)dev_status;
+  mhc_status st = check_params(p);
+  if (st != MHC_OK) return st;
+  if (!aligned16(x) || !aligned16(f_out) || !aligned16(H_post) || !aligned16(H_res) ||
+      !aligned16(x_next))
+    return MHC_ERR_INVALID_ARG;
+  if (x_next == x || x_next == f_out) return MHC_ERR_INVALID_ARG;
+  return from_cuda(mhc::post_dispatch(p->n, p->dtype, p->T, p->C, x, f_out, H_post, H_res, x_next,
+                                      (cudaStream_t)stream));
+}
+
+size_t mhc_backward_workspace_size(const mhc_params* p) {
+  if (check_params(p) != MHC_OK) return 0;
+  return bwd_layout(p).total;
+}
+
+mhc_status mhc_backward_map(const mhc_params* p, const void* x, const float* phi, const float* b,
+                            const float* alpha, const void* f_out, const void* grad_x_next,
+                            const void* grad_h_in, void* workspace, size_t workspace_bytes,
+                            int* dev_status, mhc_stream_t stream) {
+  mhc_status st = check_params(p);
+  if (st != MHC_OK) return st;
+  if (!aligned16(x) || !aligned16(phi) || !aligned16(b) || !aligned16(alpha) ||
+      !aligned16(f_out) || !aligned16(grad_x_next) || !aligned16(grad_h_in))
+    return MHC_ERR_INVALID_ARG;
+  const BwdWorkspace w = bwd_layout(p);
+  st = check_workspace(w, workspace, workspace_bytes);
+  if (st != MHC_OK) return st;
+  char* ws = (char*)workspace;
+  return from_cuda(mhc::map_bwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
+                                         alpha, grad_x_next, grad_h_in, f_out,
+                                         (float*)(ws + w.coef_off), (float*)(ws + w.part_off),
+                                         dev_status, (cudaStream_t)stream));
+}
+
+mhc_status mhc_backward_apply(const mhc_params* p, const void* x, const float* phi,
+                              const void* grad_x_next, const void* grad_h_in, void* grad_x,
+                              float* grad_phi, float* grad_b, float* grad_alpha, void* grad_f_out,
+                              const void* workspace, size_t workspace_bytes, int* dev_status,
+                              mhc_stream_t stream) {
+  (void)dev_status;
+  mhc_status st = check_params(p);
+  if (st != MHC_OK) return st;
+  if (!aligned16(x) || !aligned16(phi) || !aligned16(grad_x_next) || !aligned16(grad_h_in) ||
+      !aligned16(grad_x) || !aligned16(grad_phi) || !aligned16(grad_b) ||
+      !aligned16(grad_alpha) || !aligned16(grad_f_out))
+    return MHC_ERR_INVALID_ARG;
+  const BwdWorkspace w = bwd_layout(p);
+  st = check_workspace(w, (void*)workspace, workspace_bytes);
+  if (st != MHC_OK) return st;
+  const char* ws = (const char*)workspace;
+  return from_cuda(mhc::apply_dispatch(p->n, p->dtype, p->T, p->C, x, phi, grad_x_next, grad_h_in,
+                                       (const float*)(ws + w.coef_off),
+                                       (const float*)(ws + w.part_off), w.nparts, grad_x,
+                                       grad_f_out, grad_phi, grad_b, grad_alpha,
+                                       (cudaStream_t)stream));
+}
+
+mhc_status mhc_backward(const mhc_params* p, const void* x, const float* phi, const float* b,
+                        const float* alpha, const void* f_out, const void* grad_x_next,
+                        const void* grad_h_in, void* grad_x, float* grad_phi, float* grad_b,
+                        float* grad_alpha, void* grad_f_out, void* workspace,
+                        size_t workspace_bytes, int* dev_status, mhc_stream_t stream) {
+  mhc_status st = check_params(p);
+  if (st != MHC_OK) return st;
+  if (!aligned16(grad_x) || !aligned16(grad_phi) || !aligned16(grad_b) ||
+      !aligned16(grad_alpha) || !aligned16(grad_f_out))
+    return MHC_ERR_INVALID_ARG;
+  st = mhc_backward_map(p, x, phi, b, alpha, f_out, grad_x_next, grad_h_in, workspace,
+                        workspace_bytes, dev_status, stream);
+  if (st != MHC_OK) return st;
+  return mhc_backward_apply(p, x, phi, grad_x_next, grad_h_in, grad_x, grad_phi, grad_b,
+                            grad_alpha, grad_f_out, workspace, workspace_bytes, dev_status, stream);
+}
+
+mhc_status mhc_sinkhorn_knopp(int n, int iters, int64_t B, const float* logits, float* out,
+                              int* dev_status, mhc_stream_t stream) {
+  if (n != 1 && n != 2 && n != 4 && n != 8 && n != 16) return MHC_ERR_UNSUPPORTED;
+  if (B < 1 || iters < 0 || !aligned16(logits) || !aligned16(out)) return MHC_ERR_INVALID_ARG;
+  if (B > (int64_t)0x7fffffffLL * 64) return MHC_ERR_INVALID_ARG;
+  return from_cuda(mhc::sinkhorn_dispatch(n, iters, B, logits, out, dev_status,
+                                          (cudaStream_t)stream));
+}
+
+mhc_status mhc_depth_amax(int n, int64_t T, int L, const float* H, float* gain_fwd,
+                          float* gain_bwd, int* dev_status, mhc_stream_t stream) {
+  (void)dev_status;
+  if (n != 1 && n != 2 && n != 4 && n != 8 && n != 16) return MHC_ERR_UNSUPPORTED;
+  if (T < 1 || L < 0 || !aligned16(gain_fwd) || !aligned16(gain_bwd)) return MHC_ERR_INVALID_ARG;
+  if (L > 0 && !aligned16(H)) return MHC_ERR_INVALID_ARG;
+  if (T > (int64_t)0x7fffffffLL * 16) return MHC_ERR_INVALID_ARG;
+  return from_cuda(
+      mhc::depth_amax_dispatch(n, T, L, H, gain_fwd, gain_bwd, (cudaStream_t)stream));
+}
+
+}  // extern "C"

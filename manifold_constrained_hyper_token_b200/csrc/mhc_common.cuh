@@ -1,0 +1,196 @@
+// mhc_common.cuh -- device helpers shared by the mHC kernels: 16-byte vector
+// I/O for the two activation dtypes, status reporting, and the per-token
+// mapping arithmetic (gates and Sinkhorn-Knopp with its adjoint) that the
+// forward and backward kernels both run in registers.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/mhc.h"
+
+namespace mhc {
+
+// ---------------------------------------------------------------- vector I/O
+// One 16-byte vector of the activation dtype, widened to fp32.
+template <typename T> struct Vec;
+
+template <> struct Vec<float> {
+  static constexpr int N = 4;
+  __device__ __forceinline__ static void load(const float* p, float (&v)[4]) {
+    float4 q = *reinterpret_cast<const float4*>(p);
+    v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+  }
+  __device__ __forceinline__ static void load_stream(const float* p, float (&v)[4]) {
+    float4 q = __ldcs(reinterpret_cast<const float4*>(p));
+    v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+  }
+  __device__ __forceinline__ static void store_stream(float* p, const float (&v)[4]) {
+    __stcs(reinterpret_cast<float4*>(p), make_float4(v[0], v[1], v[2], v[3]));
+  }
+};
+
+template <> struct Vec<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ __forceinline__ static void unpack(const uint4 q, float (&v)[8]) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+  __device__ __forceinline__ static uint4 pack(const float (&v)[8]) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+      w[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  __device__ __forceinline__ static void load(const __nv_bfloat16* p, float (&v)[8]) {
+    unpack(*reinterpret_cast<const uint4*>(p), v);
+  }
+  __device__ __forceinline__ static void load_stream(const __nv_bfloat16* p, float (&v)[8]) {
+    unpack(__ldcs(reinterpret_cast<const uint4*>(p)), v);
+  }
+  __device__ __forceinline__ static void store_stream(__nv_bfloat16* p, const float (&v)[8]) {
+    __stcs(reinterpret_cast<uint4*>(p), pack(v));
+  }
+};
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// ------------------------------------------------------------------- status
+// Record the first run-time error code in the caller's status word.
+__device__ __forceinline__ void flag_status(int* st, int code) {
+  if (st) atomicCAS(st, 0, code);
+}
+
+// -------------------------------------------------------- per-token mapping
+__device__ __forceinline__ float sigmoidf_(float v) { return 1.0f / (1.0f + expf(-v)); }
+
+// Sinkhorn-Knopp for one N x N matrix held by one thread.  On entry A holds
+// the logits; on exit the estimate after `iters` iterations of (row pass,
+// column pass).  With iters >= 1 the row maximum is subtracted before exp;
+// the first row pass cancels that factor exactly in real arithmetic.
+template <int N>
+__device__ __forceinline__ void sk_init(float (&A)[N * N], int iters) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    float mx = 0.0f;
+    if (iters > 0) {
+      mx = A[i * N];
+#pragma unroll
+      for (int j = 1; j < N; ++j) mx = fmaxf(mx, A[i * N + j]);
+    }
+#pragma unroll
+    for (int j = 0; j < N; ++j) A[i * N + j] = expf(A[i * N + j] - mx);
+  }
+}
+
+// Normalisation number q (1-based): odd q = row pass, even q = column pass.
+// `s` receives the sums that were divided out.
+template <int N>
+__device__ __forceinline__ void sk_step(float (&A)[N * N], int q, float (&s)[N]) {
+  if (q & 1) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      float acc = 0.0f;
+#pragma unroll
+      for (int j = 0; j < N; ++j) acc += A[i * N + j];
+      s[i] = acc;
+      const float inv = 1.0f / acc;
+#pragma unroll
+      for (int j = 0; j < N; ++j) A[i * N + j] *= inv;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+      float acc = 0.0f;
+#pragma unroll
+      for (int i = 0; i < N; ++i) acc += A[i * N + j];
+      s[j] = acc;
+      const float inv = 1.0f / acc;
+#pragma unroll
+      for (int i = 0; i < N; ++i) A[i * N + j] *= inv;
+    }
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void sk_forward(float (&A)[N * N], int iters) {
+  sk_init<N>(A, iters);
+  float s[N];
+  for (int q = 1; q <= 2 * iters; ++q) sk_step<N>(A, q, s);
+}
+
+// Adjoint of sk_forward.  z holds the logits, dA the gradient with respect
+// to the output; on exit dz holds the gradient with respect to the logits.
+// Every intermediate iterate is recomputed from the start with the same
+// instructions as the forward pass, so the backward sees the forward's exact
+// fp32 iterates (O(iters^2) work on 16 registers, no stored iterates).
+template <int N>
+__device__ __forceinline__ void sk_adjoint(const float (&z)[N * N], float (&dA)[N * N],
+                                           float (&dz)[N * N], int iters) {
+  float M0[N * N];
+#pragma unroll
+  for (int e = 0; e < N * N; ++e) M0[e] = z[e];
+  sk_init<N>(M0, iters);
+  for (int step = 2 * iters; step >= 1; --step) {
+    float A[N * N];
+#pragma unroll
+    for (int e = 0; e < N * N; ++e) A[e] = M0[e];
+    float s[N];
+    for (int q = 1; q < step; ++q) sk_step<N>(A, q, s);
+    sk_step<N>(A, step, s);  // A is now the output of this step, s its sums
+    if (step & 1) {
+#pragma unroll
+      for (int i = 0; i < N; ++i) {
+        float d = 0.0f;
+#pragma unroll
+        for (int j = 0; j < N; ++j) d += dA[i * N + j] * A[i * N + j];
+        const float inv = 1.0f / s[i];
+#pragma unroll
+        for (int j = 0; j < N; ++j) dA[i * N + j] = (dA[i * N + j] - d) * inv;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < N; ++j) {
+        float d = 0.0f;
+#pragma unroll
+        for (int i = 0; i < N; ++i) d += dA[i * N + j] * A[i * N + j];
+        const float inv = 1.0f / s[j];
+#pragma unroll
+        for (int i = 0; i < N; ++i) dA[i * N + j] = (dA[i * N + j] - d) * inv;
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < N * N; ++e) dz[e] = dA[e] * M0[e];
+}
+
+// Per-token coefficient record written by the backward mapping kernel and
+// read by the backward apply kernel (floats):
+//   [0, N*N)            H_res
+//   [N*N, N*N+N)        H_pre
+//   [.., +N)            H_post
+//   [.., +M)            u = alpha * dz / r     (M = N*N + 2N)
+//   [.., +1)            kappa = alpha * (dz . y) / (K r^2)
+// padded to a multiple of 4 floats.
+template <int N> struct Coef {
+  static constexpr int M = N * N + 2 * N;
+  static constexpr int RES = 0;
+  static constexpr int PRE = N * N;
+  static constexpr int POST = N * N + N;
+  static constexpr int U = N * N + 2 * N;
+  static constexpr int KAPPA = U + M;
+  static constexpr int SIZE = ((KAPPA + 1) + 3) / 4 * 4;
+  // dz record for the bias / alpha sums: [0, M) dz, [M] dz . y, padded.
+  static constexpr int DZ_SIZE = ((M + 1) + 3) / 4 * 4;
+};
+
+}  // namespace mhc

@@ -1,0 +1,304 @@
+"""GPU parity: every libmhc entry point against the fp64 oracle, element by
+element, on the same seeded inputs.
+
+Tolerances (norm-wise, per output tensor: max|gpu - ref| / max|ref|):
+  fp32 I/O  1e-5
+  bf16 I/O  2e-2   (bf16 inputs widen exactly on both sides; the gap is fp32
+                    accumulation, bf16 rounding of the outputs and, for the
+                    tensor-core projection, bf16 operands)
+Standalone Sinkhorn and depth gain (fp32): 1e-5.
+"""
+import numpy as np
+import pytest
+import torch
+
+from conftest import rel_err
+
+pytestmark = pytest.mark.gpu
+
+TOL = {torch.float32: 1e-5, torch.bfloat16: 2e-2}
+
+
+@pytest.fixture(scope="module")
+def mhc():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from manifold_constrained_hyper_token_b200 import build
+    build.build()
+    import manifold_constrained_hyper_token_b200 as m
+    return m
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def _inputs(T, n, C, dtype, seed=0, alpha=0.01):
+    from manifold_constrained_hyper_token_b200 import synth
+    d = synth.layer_inputs(T, n, C, seed=seed, dtype=dtype, backward=True)
+    d["alpha"] = torch.tensor([alpha], dtype=torch.float32)
+    return d
+
+
+def _dev(d):
+    return {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in d.items()}
+
+
+def _status():
+    return torch.zeros(1, dtype=torch.int32, device="cuda")
+
+
+# --------------------------------------------------------------- Sinkhorn
+@pytest.mark.parametrize("n", [1, 2, 4, 8, 16])
+@pytest.mark.parametrize("iters", [0, 1, 20])
+@pytest.mark.parametrize("B", [1, 1000, 1003])
+def test_sinkhorn_parity(mhc, oracle_mod, n, iters, B):
+    from manifold_constrained_hyper_token_b200 import synth
+    lg = synth.sinkhorn_logits(B, n, seed=n * 7 + iters)
+    st = _status()
+    out = mhc.mhc_sinkhorn_knopp(lg.cuda(), iters, dev_status=st)
+    ref = oracle_mod.sinkhorn(lg, iters)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert rel_err(_np(out), ref) < 1e-5
+
+
+@pytest.mark.parametrize("n", [4, 8, 16])
+def test_sinkhorn_full_batch(mhc, oracle_mod, n):
+    """2^22 matrices, logits N(0, 2), 20 iterations: sampled parity plus the
+    column sums of every matrix (exact after the closing column pass)."""
+    from manifold_constrained_hyper_token_b200 import synth
+    B = 1 << 22
+    lg = synth.sinkhorn_logits(B, n, seed=100 + n)
+    out = mhc.mhc_sinkhorn_knopp(lg.cuda(), 20)
+    idx = synth.token_sample(B, 2048, seed=n)
+    ref = oracle_mod.sinkhorn(lg[idx], 20)
+    assert rel_err(_np(out[idx.cuda()]), ref) < 1e-5
+    assert float(out.min()) >= 0.0
+    assert float((out.sum(dim=1) - 1).abs().max()) < 1e-5
+    del out
+
+
+def test_sinkhorn_nonfinite_status(mhc):
+    lg = torch.zeros(64, 4, 4)
+    lg[5, 1, 2] = float("inf")
+    st = _status()
+    mhc.mhc_sinkhorn_knopp(lg.cuda(), 20, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 4
+
+
+# ------------------------------------------------------------ depth gain
+@pytest.mark.parametrize("n", [1, 2, 4, 8, 16])
+@pytest.mark.parametrize("L", [0, 1, 64])
+def test_depth_amax_parity(mhc, oracle_mod, n, L):
+    from manifold_constrained_hyper_token_b200 import synth
+    T = 301
+    lg = synth.sinkhorn_logits(T * max(L, 1), n, seed=200 + n + L)
+    H = oracle_mod.sinkhorn(lg, 20).reshape(T, max(L, 1), n, n)[:, :L]
+    Ht = torch.from_numpy(np.ascontiguousarray(H)).float()
+    gf, gb = mhc.mhc_depth_amax(Ht.cuda() if L > 0 else torch.empty(T, 0, n, n, device="cuda"))
+    rf, rb = oracle_mod.depth_amax(Ht)
+    assert rel_err(_np(gf), rf) < 1e-5 and rel_err(_np(gb), rb) < 1e-5
+
+
+def test_depth_amax_non_doubly_stochastic(mhc, oracle_mod):
+    H = torch.randn(257, 8, 4, 4, generator=torch.Generator().manual_seed(5)) * 0.7
+    gf, gb = mhc.mhc_depth_amax(H.cuda())
+    rf, rb = oracle_mod.depth_amax(H)
+    assert rel_err(_np(gf), rf) < 1e-5 and rel_err(_np(gb), rb) < 1e-5
+
+
+def test_depth_amax_sinkhorn_batch(mhc, oracle_mod):
+    """2^16 tokens x 64 layers of 20-iteration Sinkhorn outputs (N(0,2) logits)."""
+    from manifold_constrained_hyper_token_b200 import synth
+    T, L, n = 1 << 16, 64, 4
+    lg = synth.sinkhorn_logits(T * L, n, seed=300)
+    H = mhc.mhc_sinkhorn_knopp(lg.cuda(), 20).view(T, L, n, n)
+    gf, gb = mhc.mhc_depth_amax(H)
+    idx = synth.token_sample(T, 1024, seed=3)
+    rf, rb = oracle_mod.depth_amax(H[idx.cuda()].cpu())
+    assert rel_err(_np(gf[idx.cuda()]), rf) < 1e-5 and rel_err(_np(gb[idx.cuda()]), rb) < 1e-5
+    print(f"Amax gain over {T} tokens x {L} layers: fwd max {float(gf.max()):.6f} "
+          f"bwd max {float(gb.max()):.6f}")
+
+
+# ----------------------------------------------------------------- post
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("n", [1, 2, 4])
+@pytest.mark.parametrize("T,C", [(1, 8), (67, 24), (130, 256)])
+def test_post_parity(mhc, oracle_mod, dtype, n, T, C):
+    d = _inputs(T, n, C, dtype, seed=T + C)
+    g = torch.Generator().manual_seed(T * 3 + n)
+    Hpost = torch.rand(T, n, generator=g) * 2
+    Hres = torch.rand(T, n, n, generator=g)
+    out = mhc.mhc_post(d["x"].cuda(), d["f_out"].cuda(), Hpost.cuda(), Hres.cuda())
+    ref = oracle_mod.post(d["x"], d["f_out"], Hpost, Hres)
+    assert rel_err(_np(out), ref) < TOL[dtype]
+
+
+def test_post_standard_residual_exact(mhc):
+    x = torch.randn(33, 1, 64)
+    f = torch.randn(33, 64)
+    out = mhc.mhc_post(x.cuda(), f.cuda(), torch.ones(33, 1).cuda(), torch.ones(33, 1, 1).cuda())
+    assert torch.equal(out.cpu()[:, 0], x[:, 0] + f)
+
+
+# ------------------------------------------------------------------ pre
+def _check_pre(mhc, oracle_mod, d, iters, dtype, eps=1e-6):
+    dd = _dev(d)
+    st = _status()
+    h_in, Hpre, Hpost, Hres = mhc.mhc_pre(dd["x"], dd["phi"], dd["b"], dd["alpha"], t_max=iters,
+                                          eps=eps, dev_status=st)
+    ref = oracle_mod.pre(d["x"], d["phi"], d["b"], float(d["alpha"][0]), iters=iters, eps=eps)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    tol = TOL[dtype]
+    errs = dict(H_pre=rel_err(_np(Hpre), ref["H_pre"]), H_post=rel_err(_np(Hpost), ref["H_post"]),
+                H_res=rel_err(_np(Hres), ref["H_res"]), h_in=rel_err(_np(h_in), ref["h_in"]))
+    assert all(v < tol for v in errs.values()), errs
+    return errs
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("n", [1, 2, 4])
+@pytest.mark.parametrize("T,C", [(1, 8), (65, 24), (130, 256)])
+@pytest.mark.parametrize("iters", [0, 1, 20])
+def test_pre_parity(mhc, oracle_mod, dtype, n, T, C, iters):
+    d = _inputs(T, n, C, dtype, seed=T * 11 + C + n)
+    _check_pre(mhc, oracle_mod, d, iters, dtype)
+
+
+def test_pre_large_alpha_parity(mhc, oracle_mod):
+    """alpha = 1 so that the projection, not the bias, dominates the logits."""
+    d = _inputs(200, 4, 512, torch.float32, seed=9, alpha=1.0)
+    _check_pre(mhc, oracle_mod, d, 20, torch.float32)
+
+
+def test_pre_nonfinite_status(mhc):
+    d = _dev(_inputs(70, 4, 64, torch.bfloat16, seed=1))
+    d["x"][3, 1, 5] = float("nan")
+    st = _status()
+    mhc.mhc_pre(d["x"], d["phi"], d["b"], d["alpha"], dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 4
+
+
+def test_tiny_forward_with_linear_F(mhc, oracle_mod):
+    """T=64, n=4, C=256 fp32, F = fixed random linear map W [256, 256]."""
+    from manifold_constrained_hyper_token_b200 import synth
+    d = synth.tiny_forward(0)
+    dd = _dev(d)
+    h_in, Hpre, Hpost, Hres = mhc.mhc_pre(dd["x"], dd["phi"], dd["b"], dd["alpha"])
+    f_out = (h_in.double() @ dd["W"].double().T).float().contiguous()
+    x_next = mhc.mhc_post(dd["x"], f_out, Hpost, Hres)
+    ref = oracle_mod.pre(d["x"], d["phi"], d["b"], float(d["alpha"][0]))
+    f_ref = ref["h_in"] @ _np(d["W"]).T
+    xn_ref = oracle_mod.post(d["x"], f_ref, ref["H_post"], ref["H_res"])
+    assert rel_err(_np(h_in), ref["h_in"]) < 1e-5
+    assert rel_err(_np(f_out), f_ref) < 1e-5
+    assert rel_err(_np(x_next), xn_ref) < 1e-5
+
+
+# -------------------------------------------------------------- backward
+def _check_bwd(mhc, oracle_mod, d, iters, dtype, eps=1e-6, idx=None, chunk=None):
+    dd = _dev(d)
+    st = _status()
+    gx, gphi, gb, ga, gf = mhc.mhc_backward(dd["x"], dd["phi"], dd["b"], dd["alpha"], dd["f_out"],
+                                            dd["grad_x_next"], dd["grad_h_in"], t_max=iters,
+                                            eps=eps, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ref = oracle_mod.backward(d["x"], d["phi"], d["b"], float(d["alpha"][0]), d["f_out"],
+                              d["grad_x_next"], d["grad_h_in"], iters=iters, eps=eps, chunk=chunk)
+    tol = TOL[dtype]
+    errs = dict(grad_x=rel_err(_np(gx), ref["grad_x"]), grad_f_out=rel_err(_np(gf), ref["grad_f_out"]),
+                grad_phi=rel_err(_np(gphi), ref["grad_phi"]), grad_b=rel_err(_np(gb), ref["grad_b"]),
+                grad_alpha=rel_err(_np(ga), np.array([ref["grad_alpha"]])))
+    assert all(v < tol for v in errs.values()), errs
+    return errs, (gx, gphi, gb, ga, gf)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("n", [1, 2, 4])
+@pytest.mark.parametrize("T,C", [(1, 8), (65, 24), (130, 256)])
+@pytest.mark.parametrize("iters", [0, 1, 20])
+def test_backward_parity(mhc, oracle_mod, dtype, n, T, C, iters):
+    d = _inputs(T, n, C, dtype, seed=T * 13 + C + n + iters)
+    _check_bwd(mhc, oracle_mod, d, iters, dtype)
+
+
+def test_backward_large_alpha_parity(mhc, oracle_mod):
+    d = _inputs(150, 4, 512, torch.float32, seed=19, alpha=1.0)
+    _check_bwd(mhc, oracle_mod, d, 20, torch.float32)
+
+
+def test_backward_is_deterministic(mhc):
+    d = _dev(_inputs(300, 4, 512, torch.bfloat16, seed=4))
+    a = mhc.mhc_backward(d["x"], d["phi"], d["b"], d["alpha"], d["f_out"], d["grad_x_next"],
+                         d["grad_h_in"])
+    b = mhc.mhc_backward(d["x"], d["phi"], d["b"], d["alpha"], d["f_out"], d["grad_x_next"],
+                         d["grad_h_in"])
+    for u, v in zip(a, b):
+        assert torch.equal(u, v)
+
+
+def test_backward_small_workspace_rejected(mhc):
+    d = _dev(_inputs(64, 4, 64, torch.bfloat16))
+    need = mhc.mhc_backward_workspace_size(4, 64, 64, torch.bfloat16)
+    ws = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(mhc.MhcError) as e:
+        mhc.mhc_backward(d["x"], d["phi"], d["b"], d["alpha"], d["f_out"], d["grad_x_next"],
+                         d["grad_h_in"], workspace=ws)
+    assert e.value.status == 6
+
+
+# ------------------------------------------------------ full-size configs
+@pytest.mark.slow
+def test_forward_bf16_full_size(mhc, oracle_mod):
+    """T=8192, n=4, C=4096 bf16 forward (pre + post with a supplied f_out):
+    a seeded sample of tokens against the oracle."""
+    from manifold_constrained_hyper_token_b200 import synth
+    T, n, C = 8192, 4, 4096
+    d = synth.layer_inputs(T, n, C, seed=0, dtype=torch.bfloat16, backward=False)
+    dd = _dev(d)
+    h_in, Hpre, Hpost, Hres = mhc.mhc_pre(dd["x"], dd["phi"], dd["b"], dd["alpha"])
+    x_next = mhc.mhc_post(dd["x"], dd["f_out"], Hpost, Hres)
+    idx = synth.token_sample(T, 256, seed=1)
+    ref = oracle_mod.pre(d["x"][idx], d["phi"], d["b"], float(d["alpha"][0]))
+    xn = oracle_mod.post(d["x"][idx], d["f_out"][idx], ref["H_post"], ref["H_res"])
+    ic = idx.cuda()
+    for got, r in ((h_in[ic], ref["h_in"]), (Hpre[ic], ref["H_pre"]), (Hpost[ic], ref["H_post"]),
+                   (Hres[ic], ref["H_res"]), (x_next[ic], xn)):
+        assert rel_err(_np(got), r) < 2e-2
+
+
+@pytest.mark.slow
+def test_forward_backward_full_size(mhc, oracle_mod):
+    """T=16384, n=4, C=7168 bf16 forward + backward: per-token outputs on a seeded
+    sample of tokens; grad_phi / grad_b / grad_alpha against the full-T oracle."""
+    from manifold_constrained_hyper_token_b200 import synth
+    T, n, C = 16384, 4, 7168
+    d = synth.layer_inputs(T, n, C, seed=0, dtype=torch.bfloat16, backward=True)
+    dd = _dev(d)
+    alpha = float(d["alpha"][0])
+    h_in, Hpre, Hpost, Hres = mhc.mhc_pre(dd["x"], dd["phi"], dd["b"], dd["alpha"])
+    x_next = mhc.mhc_post(dd["x"], dd["f_out"], Hpost, Hres)
+    gx, gphi, gb, ga, gf = mhc.mhc_backward(dd["x"], dd["phi"], dd["b"], dd["alpha"], dd["f_out"],
+                                            dd["grad_x_next"], dd["grad_h_in"])
+    torch.cuda.synchronize()
+    idx = synth.token_sample(T, 256, seed=2)
+    ic = idx.cuda()
+    ref = oracle_mod.pre(d["x"][idx], d["phi"], d["b"], alpha)
+    xn = oracle_mod.post(d["x"][idx], d["f_out"][idx], ref["H_post"], ref["H_res"])
+    for got, r in ((h_in[ic], ref["h_in"]), (Hres[ic], ref["H_res"]), (x_next[ic], xn)):
+        assert rel_err(_np(got), r) < 2e-2
+    rs = oracle_mod.backward(d["x"][idx], d["phi"], d["b"], alpha, d["f_out"][idx],
+                             d["grad_x_next"][idx], d["grad_h_in"][idx])
+    assert rel_err(_np(gx[ic]), rs["grad_x"]) < 2e-2
+    assert rel_err(_np(gf[ic]), rs["grad_f_out"]) < 2e-2
+    full = oracle_mod.backward(d["x"], d["phi"], d["b"], alpha, d["f_out"], d["grad_x_next"],
+                               d["grad_h_in"], chunk=1024)
+    assert rel_err(_np(gphi), full["grad_phi"]) < 2e-2
+    assert rel_err(_np(gb), full["grad_b"]) < 2e-2
+    assert rel_err(_np(ga), np.array([full["grad_alpha"]])) < 2e-2
