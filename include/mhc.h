@@ -198,6 +198,38 @@ MHC_API mhc_status mhc_backward_apply(const mhc_params *p, const void *x, const 
                                       mhc_stream_t stream);
 
 /*
+ * mhc_backward_noalloc -- mhc_backward for callers that cannot allocate
+ * device memory where they run the backward: runtimes that plan every device
+ * buffer at start-up and forbid allocation afterwards, plugins that a host
+ * framework hands only their input and output buffers, or processes whose
+ * framework allocator already holds the whole device (cudaMalloc can also
+ * synchronise the device and has no latency bound).  The pages have no
+ * counterpart: this is a deployment variant of mhc_backward, not part of the
+ * method.
+ *
+ * Arguments, layouts, results and errors are those of mhc_backward, minus
+ * the workspace.  The scratch is a library-owned device array of
+ * MHC_NOALLOC_SCRATCH_BYTES that every GPU loading this library holds until
+ * the process exits.  A problem whose mhc_backward_workspace_size() exceeds
+ * MHC_NOALLOC_SCRATCH_BYTES is rejected with MHC_ERR_WORKSPACE before any
+ * launch (n = 4: up to about 20,000 tokens per call).  The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress) with
+ * that device current and caches it; make that first call before any stream
+ * capture.  All calls share the one array and it keeps the last call's
+ * contents (nothing in it needs to start at zero): calls whose work can
+ * overlap on the GPU (on different streams, or from several threads without
+ * ordering) race on it and must be serialised by the caller.  Allocates
+ * nothing: no cudaMalloc, cudaFree or allocating library routine.
+ */
+#define MHC_NOALLOC_SCRATCH_BYTES (4u * 1024u * 1024u)
+MHC_API mhc_status mhc_backward_noalloc(const mhc_params *p, const void *x, const float *phi,
+                                        const float *b, const float *alpha, const void *f_out,
+                                        const void *grad_x_next, const void *grad_h_in,
+                                        void *grad_x, float *grad_phi, float *grad_b,
+                                        float *grad_alpha, void *grad_f_out, int *dev_status,
+                                        mhc_stream_t stream);
+
+/*
  * mhc_sinkhorn_knopp -- standalone batched Sinkhorn-Knopp (source: section
  * "Vielfaeltig eingeschraenkte Hyperverbindungen": alternate row and column
  * normalisation, the classical 1967 algorithm; reportify.cn [16]).

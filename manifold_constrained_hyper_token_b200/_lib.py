@@ -11,7 +11,7 @@ LIB_PATH = os.path.join(_PKG, "libmhc.so")
 # mhc.h symbols this binding requires
 SYMBOLS = ("mhc_version", "mhc_status_string", "mhc_pre_workspace_size", "mhc_pre", "mhc_post",
            "mhc_backward_workspace_size", "mhc_backward", "mhc_backward_map", "mhc_backward_apply",
-           "mhc_sinkhorn_knopp", "mhc_depth_amax")
+           "mhc_backward_noalloc", "mhc_sinkhorn_knopp", "mhc_depth_amax")
 
 
 class MhcParams(ctypes.Structure):
@@ -51,6 +51,8 @@ def load() -> ctypes.CDLL:
     lib.mhc_backward_map.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
     lib.mhc_backward_apply.restype = i32
     lib.mhc_backward_apply.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
+    lib.mhc_backward_noalloc.restype = i32
+    lib.mhc_backward_noalloc.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.mhc_sinkhorn_knopp.restype = i32
     lib.mhc_sinkhorn_knopp.argtypes = [i32, i32, i64, vp, vp, vp, vp]
     lib.mhc_depth_amax.restype = i32

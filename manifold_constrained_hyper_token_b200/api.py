@@ -132,6 +132,26 @@ def mhc_backward(x, phi, b, alpha, f_out, grad_x_next, grad_h_in, *, t_max: int 
     return gx, gphi, gb, ga, gf
 
 
+def mhc_backward_noalloc(x, phi, b, alpha, f_out, grad_x_next, grad_h_in, *, t_max: int = 20,
+                         eps: float = 1e-6, out=None, dev_status=None, stream=None):
+    """mhc_backward without a workspace: the library's fixed device scratch array is used
+    (for callers that cannot allocate device memory).  Output tensors must be passed in
+    ``out`` by callers that cannot allocate; they are created here only as a convenience.
+    Returns (grad_x, grad_phi, grad_b, grad_alpha, grad_f_out)."""
+    T, n, C = x.shape
+    p = params(n, T, C, x.dtype, t_max, eps)
+    if out is None:
+        out = (torch.empty_like(x), torch.empty_like(phi), torch.empty_like(b),
+               torch.empty_like(alpha), torch.empty_like(f_out))
+    gx, gphi, gb, ga, gf = out
+    st = _lib.load().mhc_backward_noalloc(ctypes.byref(p), _p(x), _p(phi), _p(b), _p(alpha),
+                                          _p(f_out), _p(grad_x_next), _p(grad_h_in), _p(gx),
+                                          _p(gphi), _p(gb), _p(ga), _p(gf), _p(dev_status),
+                                          _stream(stream))
+    _check(st, "mhc_backward_noalloc")
+    return gx, gphi, gb, ga, gf
+
+
 def mhc_backward_map(x, phi, b, alpha, f_out, grad_x_next, grad_h_in, workspace, *,
                      t_max: int = 20, eps: float = 1e-6, dev_status=None, stream=None):
     """Phase 1 of mhc_backward: per-token records into ``workspace`` (uint8 tensor of at
