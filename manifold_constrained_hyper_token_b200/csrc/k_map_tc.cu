@@ -1,0 +1,485 @@
+// k_map_tc.cu -- per-token mapping on the 5th-generation tensor cores
+// (bf16 activations, n = 4): the logit projection y = x . phi runs as
+// tcgen05.mma (bf16 operands, fp32 accumulation in TMEM) while the CUDA cores
+// take the sum of squares (and, for the backward, the C-reductions) from the
+// same shared-memory tiles.  Sources: the fused RMSNorm / projection / gating
+// operator of the chatgpz.de explainer (section "Systemarbeit und
+// Schulungsaufwand") and reportify.cn [17]-[19], [21] (RMS applied after the
+// projection, Sinkhorn and its custom backward in the same operator,
+// recompute in the backward).
+//
+// One CTA = 128 tokens (the MMA M).  The token's n*C inputs stream through a
+// TMA ring in chunks of 32 channels x 4 streams (64-byte rows, 64-byte
+// swizzle): per stream an x tile [128 x 32] (the MMA A operand, K-major) and
+// the matching rows of phi^T as a [48 x 32] B operand, whose 48 rows are the
+// 24 logit columns split into a bf16 high part and a bf16 low part
+// (phi = hi + lo), so y = D[:, m] + D[:, 24 + m] carries phi to ~16 bits.
+// x itself is bf16, so the products are exact and only the fp32
+// accumulation order differs from the oracle.
+//
+// Warp roles: warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs, warps
+// 2..9 (two per TMEM lane quarter, one per channel half) reduce the sum of
+// squares -- and in the backward the 24 C-reductions <G_i, x_j>, <g, x_i>,
+// <G_i, f> -- from the same stages, then run the per-token epilogue (gates,
+// Sinkhorn, adjoint) with one thread per token.  Every wait is bounded; on
+// timeout the kernel records MHC_ERR_TIMEOUT, drains what it issued, frees
+// TMEM and returns.
+#include "mhc_common.cuh"
+#include "tc_sm100.cuh"
+
+namespace mhc {
+
+namespace tcmap {
+constexpr int N = 4;
+constexpr int M = N * N + 2 * N;     // 24 logits
+constexpr int TM = 128;              // tokens per CTA (MMA M)
+constexpr int CH = 32;               // channels per chunk: 64-byte rows
+constexpr int NL = 48;               // MMA N: 24 high + 24 low logit columns
+constexpr int NWARPS = 10;
+constexpr int NT = NWARPS * 32;
+constexpr int XBOX = TM * CH * 2;    // one stream's x tile, 8 KB
+constexpr int PBOX = NL * CH * 2;    // one stream's phi^T tile, 3 KB
+constexpr uint32_t TMEM_COLS = 64;
+constexpr uint64_t WAIT_NS = 2000000000ull;  // 2 s per wait before giving up
+
+template <bool BWD> struct Cfg {
+  static constexpr int NS = BWD ? 2 : 4;        // pipeline stages
+  static constexpr int X_OFF = 0;
+  static constexpr int P_OFF = N * XBOX;
+  static constexpr int G_OFF = P_OFF + N * PBOX;
+  static constexpr int GG_OFF = G_OFF + N * XBOX;  // grad_h_in tile
+  static constexpr int F_OFF = GG_OFF + XBOX;      // f_out tile
+  static constexpr int STAGE = BWD ? F_OFF + XBOX : G_OFF;
+  static constexpr int DATA = NS * STAGE;
+  static constexpr int SMEM = DATA + 1024 /*align*/ + 256 /*barriers, flags*/;
+};
+}  // namespace tcmap
+
+// phi [K][24] fp32 -> phi^T split [48][K] bf16: rows 0..23 high parts, 24..47
+// the bf16 rounding of the remainder.
+__global__ void k_phi_split(int64_t K, const float* __restrict__ phi, __nv_bfloat16* __restrict__ out) {
+  const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= K) return;
+#pragma unroll 4
+  for (int m = 0; m < tcmap::M; ++m) {
+    const float v = __ldg(phi + k * tcmap::M + m);
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+    out[(int64_t)m * K + k] = hi;
+    out[(int64_t)(tcmap::M + m) * K + k] = lo;
+  }
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(uint4 q, float (&v)[8]) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+// Row `tok` of a [128 x 32] bf16 tile stored with the 64-byte swizzle: the
+// 16-byte chunk c of the row sits at chunk position c ^ ((tok >> 1) & 3).
+__device__ __forceinline__ uint4 ld_sw64(const uint8_t* tile, int tok, int chunk) {
+  const int phys = chunk ^ ((tok >> 1) & 3);
+  return *reinterpret_cast<const uint4*>(tile + tok * 64 + phys * 16);
+}
+
+__device__ __forceinline__ void named_bar(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+template <bool BWD>
+__global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
+    const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_phi,
+    const __grid_constant__ CUtensorMap tm_G, const __grid_constant__ CUtensorMap tm_g,
+    const __grid_constant__ CUtensorMap tm_f, int64_t T, int64_t C, int iters, float eps,
+    int ck_period, const float* __restrict__ bias, const float* __restrict__ alpha_p,
+    float* __restrict__ Hpre_o, float* __restrict__ Hpost_o, float* __restrict__ Hres_o,
+    float* __restrict__ coef_o, float* __restrict__ part_o, int* status) {
+  using namespace tcmap;
+  using CFG = Cfg<BWD>;
+  constexpr int NS = CFG::NS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~(uintptr_t)1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + CFG::DATA);  // full[NS] empty[NS] done fin
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  auto full = [&](int s) { return tc::smem_u32(bars + s); };
+  auto empty = [&](int s) { return tc::smem_u32(bars + NS + s); };
+  const uint32_t done_bar = tc::smem_u32(bars + 2 * NS);
+  const uint32_t fin_bar = tc::smem_u32(bars + 2 * NS + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int64_t t0 = (int64_t)blockIdx.x * TM;
+  const int nch = (int)((C + CH - 1) / CH);
+  const int64_t K = (int64_t)N * C;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      tc::mbar_init(full(s), 1);
+      tc::mbar_init(empty(s), 1 + 8);  // the MMA commit + one arrive per math warp
+    }
+    tc::mbar_init(done_bar, 1);
+    tc::mbar_init(fin_bar, 1);
+    *abort_flag = 0;
+    tc::mbar_fence_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tc::tma_prefetch_desc(&tm_x);
+    tc::tma_prefetch_desc(&tm_phi);
+    if constexpr (BWD) {
+      tc::tma_prefetch_desc(&tm_G);
+      tc::tma_prefetch_desc(&tm_g);
+      tc::tma_prefetch_desc(&tm_f);
+    }
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tc::smem_u32(tmem_slot), TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto give_up = [&]() {
+    *abort_flag = 1;
+    flag_status(status, MHC_ERR_TIMEOUT);
+  };
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA
+    if (lane == 0) {
+      const uint64_t pol_stream = tc::policy_evict_first();
+      const uint64_t pol_keep = tc::policy_evict_last();
+      int issued = 0;
+      for (int cc = 0; cc < nch; ++cc) {
+        const int s = cc % NS;
+        const uint32_t ph = (uint32_t)(cc / NS) & 1u;
+        if (cc >= NS && !tc::mbar_wait(empty(s), ph ^ 1u, abort_flag, WAIT_NS)) {
+          give_up();
+          break;
+        }
+        const uint32_t base = tc::smem_u32(smem + s * CFG::STAGE);
+        tc::mbar_arrive_expect_tx(full(s), CFG::STAGE);
+        const int c0 = cc * CH;
+        for (int i = 0; i < N; ++i) {
+          tc::tma_load_3d(base + CFG::X_OFF + i * XBOX, &tm_x, full(s), c0, i, (int)t0, pol_stream);
+          tc::tma_load_3d(base + CFG::P_OFF + i * PBOX, &tm_phi, full(s), c0, i, 0, pol_keep);
+          if constexpr (BWD)
+            tc::tma_load_3d(base + CFG::G_OFF + i * XBOX, &tm_G, full(s), c0, i, (int)t0,
+                            pol_stream);
+        }
+        if constexpr (BWD) {
+          tc::tma_load_2d(base + CFG::GG_OFF, &tm_g, full(s), c0, (int)t0, pol_stream);
+          tc::tma_load_2d(base + CFG::F_OFF, &tm_f, full(s), c0, (int)t0, pol_stream);
+        }
+        ++issued;
+      }
+      if (*abort_flag) {
+        // drain: the last min(NS, issued) loads may still be landing
+        for (int cc = (issued > NS ? issued - NS : 0); cc < issued; ++cc)
+          tc::mbar_wait(full(cc % NS), (uint32_t)(cc / NS) & 1u, nullptr, WAIT_NS / 4);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t idesc = tc::idesc_bf16(TM, NL);
+      bool any = false;
+      for (int cc = 0; cc < nch; ++cc) {
+        const int s = cc % NS;
+        const uint32_t ph = (uint32_t)(cc / NS) & 1u;
+        if (!tc::mbar_wait(full(s), ph, abort_flag, WAIT_NS)) {
+          give_up();
+          break;
+        }
+        tc::tc_fence_after();
+        const uint32_t base = tc::smem_u32(smem + s * CFG::STAGE);
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+#pragma unroll
+          for (int kk = 0; kk < CH / 16; ++kk) {
+            const uint64_t a = tc::smem_desc(base + CFG::X_OFF + i * XBOX + kk * 32, 16, 512, tc::SWZ_64B);
+            const uint64_t b = tc::smem_desc(base + CFG::P_OFF + i * PBOX + kk * 32, 16, 512, tc::SWZ_64B);
+            tc::mma_bf16(tmem, a, b, idesc, (cc | i | kk) != 0 ? 1u : 0u);
+          }
+        }
+        any = true;
+        tc::mma_commit(empty(s));
+      }
+      if (!*abort_flag) {
+        tc::mma_commit(done_bar);
+      } else if (any) {
+        tc::mma_commit(fin_bar);
+        tc::mbar_wait(fin_bar, 0, nullptr, WAIT_NS / 4);
+      }
+    }
+  } else {
+    // -------------------------------------------------- CUDA-core reductions
+    const int q = warp & 3;            // TMEM lane quarter this warp may read
+    const int h = (warp - 2) >> 2;     // channel half of each chunk
+    const int tok = 32 * q + lane;
+    float ss = 0.0f;
+    float dots[BWD ? M : 1];
+#pragma unroll
+    for (int m = 0; m < (BWD ? M : 1); ++m) dots[m] = 0.0f;
+    for (int cc = 0; cc < nch; ++cc) {
+      const int s = cc % NS;
+      const uint32_t ph = (uint32_t)(cc / NS) & 1u;
+      if (!tc::mbar_wait(full(s), ph, abort_flag, WAIT_NS)) {
+        give_up();
+        break;
+      }
+      const uint8_t* st = smem + s * CFG::STAGE;
+#pragma unroll
+      for (int qq = 0; qq < 2; ++qq) {
+        const int chunk = 2 * h + qq;
+        float xv[N][8];
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+          bf16x8_to_f32(ld_sw64(st + CFG::X_OFF + i * XBOX, tok, chunk), xv[i]);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ss = fmaf(xv[i][e], xv[i][e], ss);
+        }
+        if constexpr (BWD) {
+          float gv[8], fv[8];
+          bf16x8_to_f32(ld_sw64(st + CFG::GG_OFF, tok, chunk), gv);
+          bf16x8_to_f32(ld_sw64(st + CFG::F_OFF, tok, chunk), fv);
+#pragma unroll
+          for (int i = 0; i < N; ++i) {
+            float Gv[8];
+            bf16x8_to_f32(ld_sw64(st + CFG::G_OFF + i * XBOX, tok, chunk), Gv);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+#pragma unroll
+              for (int j = 0; j < N; ++j) dots[i * N + j] = fmaf(Gv[e], xv[j][e], dots[i * N + j]);
+              dots[N * N + i] = fmaf(gv[e], xv[i][e], dots[N * N + i]);
+              dots[N * N + N + i] = fmaf(Gv[e], fv[e], dots[N * N + N + i]);
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(empty(s));
+    }
+
+    // all MMAs (and so all reads of the stage buffers) finished before the
+    // stage memory is reused for the epilogue
+    bool ok = !*abort_flag && tc::mbar_wait(done_bar, 0, abort_flag, WAIT_NS);
+    if (!ok && !*abort_flag) give_up();
+    float* red_ss = reinterpret_cast<float*>(smem);       // [2][TM]
+    float* red_dt = red_ss + 2 * TM;                      // [2][M][TM]
+    float* dzs = red_dt + 2 * M * TM;                     // [M + 1][TM]
+    float* ck = dzs + (M + 1) * TM;                       // checkpoints [nck][16][TM]
+    if (ok) {
+      red_ss[h * TM + tok] = ss;
+      if constexpr (BWD) {
+#pragma unroll
+        for (int m = 0; m < M; ++m) red_dt[(h * M + m) * TM + tok] = dots[m];
+      }
+    }
+    named_bar(1, 256);
+    if (ok && h == 0) {
+      // ------------------------------------------------- per-token epilogue
+      tc::tc_fence_after();
+      float d[NL];
+      const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+      float v16[16];
+      tc::tmem_ld16(lane_base + 0, v16);
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int e = 0; e < 16; ++e) d[e] = v16[e];
+      tc::tmem_ld16(lane_base + 16, v16);
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int e = 0; e < 16; ++e) d[16 + e] = v16[e];
+      tc::tmem_ld16(lane_base + 32, v16);
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int e = 0; e < 16; ++e) d[32 + e] = v16[e];
+
+      const int64_t t = t0 + tok;
+      const float sst = red_ss[tok] + red_ss[TM + tok];
+      const float r = sqrtf(sst / (float)K + eps);
+      const float alpha = __ldg(alpha_p);
+      float y[M], z[M];
+#pragma unroll
+      for (int m = 0; m < M; ++m) {
+        y[m] = (d[m] + d[M + m]) / r;
+        z[m] = fmaf(alpha, y[m], __ldg(bias + m));
+      }
+      float spre[N], spost[N];
+#pragma unroll
+      for (int i = 0; i < N; ++i) {
+        spre[i] = sigmoidf_(z[i]);
+        spost[i] = sigmoidf_(z[N + i]);
+      }
+      float H[N * N];
+#pragma unroll
+      for (int e = 0; e < N * N; ++e) H[e] = z[2 * N + e];
+      if (t < T) {
+        bool bad = !isfinite(r);
+#pragma unroll
+        for (int m = 0; m < M; ++m) bad |= !isfinite(z[m]);
+        if (bad) flag_status(status, MHC_ERR_NONFINITE);
+      }
+      if constexpr (!BWD) {
+        sk_forward<N>(H, iters);
+        if (t < T) {
+#pragma unroll
+          for (int i = 0; i < N; ++i) {
+            Hpre_o[t * N + i] = spre[i];
+            Hpost_o[t * N + i] = 2.0f * spost[i];
+          }
+#pragma unroll
+          for (int e = 0; e < N * N; e += 4)
+            *reinterpret_cast<float4*>(Hres_o + t * N * N + e) =
+                make_float4(H[e], H[e + 1], H[e + 2], H[e + 3]);
+        }
+      } else {
+        sk_forward_ckpt<N>(H, iters, ck + tok, TM, ck_period);
+        float dA[N * N], dz[M], dzres[N * N];
+#pragma unroll
+        for (int e = 0; e < N * N; ++e)
+          dA[e] = red_dt[(0 * M + e) * TM + tok] + red_dt[(1 * M + e) * TM + tok];
+        sk_adjoint_ckpt<N>(dA, dzres, iters, ck + tok, TM, ck_period);
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+          const float dpre = red_dt[(0 * M + N * N + i) * TM + tok] + red_dt[(1 * M + N * N + i) * TM + tok];
+          const float dpost = red_dt[(0 * M + N * N + N + i) * TM + tok] +
+                              red_dt[(1 * M + N * N + N + i) * TM + tok];
+          dz[i] = dpre * spre[i] * (1.0f - spre[i]);
+          dz[N + i] = dpost * 2.0f * spost[i] * (1.0f - spost[i]);
+        }
+#pragma unroll
+        for (int e = 0; e < N * N; ++e) dz[2 * N + e] = dzres[e];
+        float dzy = 0.0f;
+#pragma unroll
+        for (int m = 0; m < M; ++m) dzy = fmaf(dz[m], y[m], dzy);
+        const bool live = t < T;
+        if (live) {
+          using CF = Coef<N>;
+          float rec[CF::SIZE];
+#pragma unroll
+          for (int e = 0; e < N * N; ++e) rec[CF::RES + e] = H[e];
+#pragma unroll
+          for (int i = 0; i < N; ++i) {
+            rec[CF::PRE + i] = spre[i];
+            rec[CF::POST + i] = 2.0f * spost[i];
+          }
+          const float ar = alpha / r;
+#pragma unroll
+          for (int m = 0; m < M; ++m) rec[CF::U + m] = ar * dz[m];
+          rec[CF::KAPPA] = alpha * dzy / ((float)K * r * r);
+#pragma unroll
+          for (int e = CF::KAPPA + 1; e < CF::SIZE; ++e) rec[e] = 0.0f;
+          float4* dst = reinterpret_cast<float4*>(coef_o + t * CF::SIZE);
+#pragma unroll
+          for (int e = 0; e < CF::SIZE / 4; ++e)
+            dst[e] = make_float4(rec[4 * e], rec[4 * e + 1], rec[4 * e + 2], rec[4 * e + 3]);
+        }
+#pragma unroll
+        for (int m = 0; m < M; ++m) dzs[m * TM + tok] = live ? dz[m] : 0.0f;
+        dzs[M * TM + tok] = live ? dzy : 0.0f;
+      }
+    }
+    if constexpr (BWD) {
+      named_bar(1, 256);
+      if (ok && h == 0 && q == 0 && lane <= M) {
+        // this CTA's share of grad_b / grad_alpha, summed in token order
+        float a = 0.0f;
+        for (int k = 0; k < TM; ++k) a += dzs[lane * TM + k];
+        part_o[(int64_t)blockIdx.x * Coef<N>::DZ_SIZE + lane] = a;
+      }
+    }
+  }
+
+  __syncwarp();
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host
+static cudaError_t encode_maps(int64_t T, int64_t C, const void* x, const void* phiT, const void* G,
+                               const void* g, const void* f, CUtensorMap* mx, CUtensorMap* mp,
+                               CUtensorMap* mG, CUtensorMap* mg, CUtensorMap* mf) {
+  using namespace tcmap;
+  const uint64_t dx[3] = {(uint64_t)C, (uint64_t)N, (uint64_t)T};
+  const uint64_t sx[2] = {(uint64_t)C * 2, (uint64_t)N * C * 2};
+  const uint32_t bx[3] = {CH, 1, TM};
+  cudaError_t e = make_tmap_bf16(mx, x, 3, dx, sx, bx, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (e != cudaSuccess) return e;
+  const uint64_t dp[3] = {(uint64_t)C, (uint64_t)N, (uint64_t)NL};
+  const uint32_t bp[3] = {CH, 1, NL};
+  e = make_tmap_bf16(mp, phiT, 3, dp, sx, bp, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (e != cudaSuccess) return e;
+  if (G == nullptr) {
+    *mG = *mx;
+    *mg = *mx;
+    *mf = *mx;
+    return cudaSuccess;
+  }
+  e = make_tmap_bf16(mG, G, 3, dx, sx, bx, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (e != cudaSuccess) return e;
+  const uint64_t d2[2] = {(uint64_t)C, (uint64_t)T};
+  const uint64_t s2[1] = {(uint64_t)C * 2};
+  const uint32_t b2[2] = {CH, TM};
+  e = make_tmap_bf16(mg, g, 2, d2, s2, b2, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (e != cudaSuccess) return e;
+  return make_tmap_bf16(mf, f, 2, d2, s2, b2, CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+// Smallest checkpoint period whose checkpoints fit beside the epilogue
+// scratch in the freed stage memory.
+static int ck_period_for(int iters, size_t stage_bytes) {
+  using namespace tcmap;
+  const size_t scratch = (size_t)(2 * TM + 2 * M * TM + (M + 1) * TM) * 4;
+  const size_t per_ck = (size_t)N * N * TM * 4;
+  const int max_ck = (int)((stage_bytes - scratch) / per_ck);  // >= 2 for the sizes used here
+  const int steps = 2 * iters;
+  int P = 1;
+  while (steps / P + 1 > max_ck) ++P;
+  return P;
+}
+
+size_t map_tc_phi_bytes(int64_t C) { return (size_t)tcmap::NL * tcmap::N * C * 2; }
+
+cudaError_t map_tc_dispatch(bool bwd, int64_t T, int64_t C, int iters, float eps, const void* x,
+                            const float* phi, void* phi_split, const float* b, const float* alpha,
+                            float* Hpre, float* Hpost, float* Hres, const void* G, const void* g,
+                            const void* f, float* coef, float* part, int* st, cudaStream_t s) {
+  using namespace tcmap;
+  const int64_t K = (int64_t)N * C;
+  k_phi_split<<<(unsigned)((K + 255) / 256), 256, 0, s>>>(K, phi, (__nv_bfloat16*)phi_split);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  CUtensorMap mx, mp, mG, mg, mf;
+  e = encode_maps(T, C, x, phi_split, bwd ? G : nullptr, g, f, &mx, &mp, &mG, &mg, &mf);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = (unsigned)((T + TM - 1) / TM);
+  if (bwd) {
+    auto kern = k_map_tc<true>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<true>::SMEM);
+    if (e != cudaSuccess) return e;
+    const int P = ck_period_for(iters, Cfg<true>::DATA);
+    kern<<<grid, NT, Cfg<true>::SMEM, s>>>(mx, mp, mG, mg, mf, T, C, iters, eps, P, b, alpha,
+                                           nullptr, nullptr, nullptr, coef, part, st);
+  } else {
+    auto kern = k_map_tc<false>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<false>::SMEM);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, NT, Cfg<false>::SMEM, s>>>(mx, mp, mG, mg, mf, T, C, iters, eps, 1, b, alpha,
+                                            Hpre, Hpost, Hres, nullptr, nullptr, st);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace mhc

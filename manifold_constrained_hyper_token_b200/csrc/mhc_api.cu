@@ -24,6 +24,12 @@ cudaError_t map_bwd_dispatch(int n, int dtype, int64_t T, int64_t C, int iters, 
                              const void* x, const float* phi, const float* b, const float* alpha,
                              const void* G, const void* g, const void* f, float* coef, float* dzr,
                              int* st, cudaStream_t s);
+// k_map_tc.cu (bf16, n = 4: projection on the tensor cores)
+cudaError_t map_tc_dispatch(bool bwd, int64_t T, int64_t C, int iters, float eps, const void* x,
+                            const float* phi, void* phi_split, const float* b, const float* alpha,
+                            float* Hpre, float* Hpost, float* Hres, const void* G, const void* g,
+                            const void* f, float* coef, float* part, int* st, cudaStream_t s);
+size_t map_tc_phi_bytes(int64_t C);
 // k_bwd.cu
 cudaError_t apply_dispatch(int n, int dtype, int64_t T, int64_t C, const void* x, const float* phi,
                            const void* G, const void* g, const float* coef, const float* part,
@@ -68,21 +74,26 @@ int dz_size(int n) {
   }
 }
 
-// Backward workspace: per-token coefficient records, then one partial-sum
-// record (dz, dz . y) per 64-token CTA of the mapping kernel.
-constexpr int kMapTokens = 64;
+// bf16 activations with n = 4 take the tensor-core mapping kernel (128 tokens
+// per CTA); every other case the CUDA-core one (64 tokens per CTA).
+bool use_tc(const mhc_params* p) { return p->dtype == MHC_DTYPE_BF16 && p->n == 4; }
 
+// Backward workspace: per-token coefficient records, one partial-sum record
+// (dz, dz . y) per mapping CTA, then (tensor-core path) the bf16 split copy
+// of phi^T that the MMA reads.
 struct BwdWorkspace {
-  size_t coef_off, part_off, total;
+  size_t coef_off, part_off, phi_off, total;
   int nparts;
 };
 
 BwdWorkspace bwd_layout(const mhc_params* p) {
   BwdWorkspace w;
-  w.nparts = (int)((p->T + kMapTokens - 1) / kMapTokens);
+  const int tokens_per_cta = use_tc(p) ? 128 : 64;
+  w.nparts = (int)((p->T + tokens_per_cta - 1) / tokens_per_cta);
   w.coef_off = 0;
   w.part_off = round_up(w.coef_off + (size_t)p->T * coef_size(p->n) * 4, 256);
-  w.total = round_up(w.part_off + (size_t)w.nparts * dz_size(p->n) * 4, 256);
+  w.phi_off = round_up(w.part_off + (size_t)w.nparts * dz_size(p->n) * 4, 256);
+  w.total = round_up(w.phi_off + (use_tc(p) ? mhc::map_tc_phi_bytes(p->C) : 0), 256);
   return w;
 }
 
@@ -113,8 +124,8 @@ const char* mhc_status_string(int status) {
 }
 
 size_t mhc_pre_workspace_size(const mhc_params* p) {
-  (void)p;
-  return 0;
+  if (check_params(p) != MHC_OK) return 0;
+  return use_tc(p) ? round_up(mhc::map_tc_phi_bytes(p->C), 256) : 0;
 }
 
 mhc_status mhc_pre(const mhc_params* p, const void* x, const float* phi, const float* b,
@@ -125,11 +136,18 @@ mhc_status mhc_pre(const mhc_params* p, const void* x, const float* phi, const f
   if (!aligned16(x) || !aligned16(phi) || !aligned16(b) || !aligned16(alpha) || !aligned16(h_in) ||
       !aligned16(H_pre) || !aligned16(H_post) || !aligned16(H_res))
     return MHC_ERR_INVALID_ARG;
-  (void)workspace;
-  (void)workspace_bytes;
   cudaStream_t s = (cudaStream_t)stream;
-  st = from_cuda(mhc::map_fwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
-                                       alpha, H_pre, H_post, H_res, dev_status, s));
+  if (use_tc(p)) {
+    const size_t need = mhc_pre_workspace_size(p);
+    if (workspace == nullptr || workspace_bytes < need || ((uintptr_t)workspace & 255u) != 0)
+      return MHC_ERR_WORKSPACE;
+    st = from_cuda(mhc::map_tc_dispatch(false, p->T, p->C, p->t_max, p->eps, x, phi, workspace, b,
+                                        alpha, H_pre, H_post, H_res, nullptr, nullptr, nullptr,
+                                        nullptr, nullptr, dev_status, s));
+  } else {
+    st = from_cuda(mhc::map_fwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
+                                         alpha, H_pre, H_post, H_res, dev_status, s));
+  }
   if (st != MHC_OK) return st;
   return from_cuda(mhc::hin_dispatch(p->n, p->dtype, p->T, p->C, x, H_pre, h_in, s));
 }
@@ -165,6 +183,12 @@ mhc_status mhc_backward_map(const mhc_params* p, const void* x, const float* phi
   st = check_workspace(w, workspace, workspace_bytes);
   if (st != MHC_OK) return st;
   char* ws = (char*)workspace;
+  if (use_tc(p))
+    return from_cuda(mhc::map_tc_dispatch(true, p->T, p->C, p->t_max, p->eps, x, phi,
+                                          ws + w.phi_off, b, alpha, nullptr, nullptr, nullptr,
+                                          grad_x_next, grad_h_in, f_out,
+                                          (float*)(ws + w.coef_off), (float*)(ws + w.part_off),
+                                          dev_status, (cudaStream_t)stream));
   return from_cuda(mhc::map_bwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
                                          alpha, grad_x_next, grad_h_in, f_out,
                                          (float*)(ws + w.coef_off), (float*)(ws + w.part_off),

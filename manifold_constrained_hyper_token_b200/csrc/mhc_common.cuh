@@ -173,6 +173,66 @@ __device__ __forceinline__ void sk_adjoint(const float (&z)[N * N], float (&dA)[
   for (int e = 0; e < N * N; ++e) dz[e] = dA[e] * M0[e];
 }
 
+// Checkpointed variants for the tensor-core kernels: the forward stores the
+// iterate after every P-th normalisation (and the start) in shared memory,
+// ck[(j * N * N + e) * stride]; the adjoint rebuilds each iterate from the
+// nearest checkpoint with the forward's own instructions (bitwise the same
+// iterates), at O(iters * P) instead of O(iters^2) work.
+template <int N>
+__device__ __forceinline__ void sk_forward_ckpt(float (&A)[N * N], int iters, float* ck, int stride,
+                                                int P) {
+  sk_init<N>(A, iters);
+#pragma unroll
+  for (int e = 0; e < N * N; ++e) ck[e * stride] = A[e];
+  float s[N];
+  for (int q = 1; q <= 2 * iters; ++q) {
+    sk_step<N>(A, q, s);
+    if (q % P == 0) {
+      float* c = ck + (q / P) * N * N * stride;
+#pragma unroll
+      for (int e = 0; e < N * N; ++e) c[e * stride] = A[e];
+    }
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void sk_adjoint_ckpt(float (&dA)[N * N], float (&dz)[N * N], int iters,
+                                                const float* ck, int stride, int P) {
+  for (int step = 2 * iters; step >= 1; --step) {
+    const int c = (step - 1) / P;
+    float A[N * N];
+    const float* cp = ck + c * N * N * stride;
+#pragma unroll
+    for (int e = 0; e < N * N; ++e) A[e] = cp[e * stride];
+    float s[N];
+    for (int q = c * P + 1; q < step; ++q) sk_step<N>(A, q, s);
+    sk_step<N>(A, step, s);
+    if (step & 1) {
+#pragma unroll
+      for (int i = 0; i < N; ++i) {
+        float d = 0.0f;
+#pragma unroll
+        for (int j = 0; j < N; ++j) d += dA[i * N + j] * A[i * N + j];
+        const float inv = 1.0f / s[i];
+#pragma unroll
+        for (int j = 0; j < N; ++j) dA[i * N + j] = (dA[i * N + j] - d) * inv;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < N; ++j) {
+        float d = 0.0f;
+#pragma unroll
+        for (int i = 0; i < N; ++i) d += dA[i * N + j] * A[i * N + j];
+        const float inv = 1.0f / s[j];
+#pragma unroll
+        for (int i = 0; i < N; ++i) dA[i * N + j] = (dA[i * N + j] - d) * inv;
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < N * N; ++e) dz[e] = dA[e] * ck[e * stride];
+}
+
 // Per-token coefficient record written by the backward mapping kernel and
 // read by the backward apply kernel (floats):
 //   [0, N*N)            H_res
