@@ -30,6 +30,12 @@ cudaError_t map_tc_dispatch(bool bwd, int64_t T, int64_t C, int iters, float eps
                             float* Hpre, float* Hpost, float* Hres, const void* G, const void* g,
                             const void* f, float* coef, float* part, int* st, cudaStream_t s);
 size_t map_tc_phi_bytes(int64_t C);
+// k_apply_tc.cu (bf16, n = 4: phi u and grad_phi on the tensor cores)
+cudaError_t apply_tc_dispatch(int64_t T, int64_t C, const void* x, const float* phi, const void* G,
+                              const void* g, const float* coef, const float* part, int nparts,
+                              void* gx, void* gf, float* gphi, float* gb, float* ga,
+                              void* scratch, int* st, cudaStream_t s);
+size_t apply_tc_scratch_bytes(int64_t C);
 // k_bwd.cu
 cudaError_t apply_dispatch(int n, int dtype, int64_t T, int64_t C, const void* x, const float* phi,
                            const void* G, const void* g, const float* coef, const float* part,
@@ -80,9 +86,10 @@ bool use_tc(const mhc_params* p) { return p->dtype == MHC_DTYPE_BF16 && p->n == 
 
 // Backward workspace: per-token coefficient records, one partial-sum record
 // (dz, dz . y) per mapping CTA, then (tensor-core path) the bf16 split copy
-// of phi^T that the MMA reads.
+// of phi^T that the mapping MMA reads and the apply kernel's grad_phi
+// partials and slice counters.
 struct BwdWorkspace {
-  size_t coef_off, part_off, phi_off, total;
+  size_t coef_off, part_off, phi_off, apply_off, total;
   int nparts;
 };
 
@@ -93,7 +100,8 @@ BwdWorkspace bwd_layout(const mhc_params* p) {
   w.coef_off = 0;
   w.part_off = round_up(w.coef_off + (size_t)p->T * coef_size(p->n) * 4, 256);
   w.phi_off = round_up(w.part_off + (size_t)w.nparts * dz_size(p->n) * 4, 256);
-  w.total = round_up(w.phi_off + (use_tc(p) ? mhc::map_tc_phi_bytes(p->C) : 0), 256);
+  w.apply_off = round_up(w.phi_off + (use_tc(p) ? mhc::map_tc_phi_bytes(p->C) : 0), 256);
+  w.total = round_up(w.apply_off + (use_tc(p) ? mhc::apply_tc_scratch_bytes(p->C) : 0), 256);
   return w;
 }
 
@@ -211,6 +219,13 @@ mhc_status mhc_backward_apply(const mhc_params* p, const void* x, const float* p
   st = check_workspace(w, (void*)workspace, workspace_bytes);
   if (st != MHC_OK) return st;
   const char* ws = (const char*)workspace;
+  if (use_tc(p))
+    return from_cuda(mhc::apply_tc_dispatch(p->T, p->C, x, phi, grad_x_next, grad_h_in,
+                                            (const float*)(ws + w.coef_off),
+                                            (const float*)(ws + w.part_off), w.nparts, grad_x,
+                                            grad_f_out, grad_phi, grad_b, grad_alpha,
+                                            (void*)(ws + w.apply_off), dev_status,
+                                            (cudaStream_t)stream));
   return from_cuda(mhc::apply_dispatch(p->n, p->dtype, p->T, p->C, x, phi, grad_x_next, grad_h_in,
                                        (const float*)(ws + w.coef_off),
                                        (const float*)(ws + w.part_off), w.nparts, grad_x,
