@@ -235,6 +235,8 @@ def main():
     ap.add_argument("--cpu-sample-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--tokens", type=int, default=T_TOK,
+                    help="tokens per GPU (default 16384; smaller values for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -260,7 +262,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
-    T, n, C = T_TOK, N_STR, C_CH
+    T, n, C = args.tokens, N_STR, C_CH
     K, M = n * C, n * n + 2 * n
     prm = synth.layer_params(n, C, seed=0)
     act = synth.activations(T, n, C, seed=rank, dtype=torch.bfloat16, backward=True)

@@ -18,9 +18,12 @@
 // U holds u as a bf16 high part and low part (m' = 0..23 and 32..55), so
 // MMA2 carries u to ~16 bits and x is exact; PHI holds phi's bf16 high part
 // in both halves, so D1 = (u_hi + u_lo) . phi_hi -- phi u is a small term of
-// grad_x.  X (TMA, 64-byte swizzle) is the MN-major A operand of MMA2; U is
-// written by the epilogue threads with the 128-byte swizzle and serves as the
-// K-major A of MMA1 and the MN-major B of MMA2.
+// grad_x.  Everything an item reads arrives by TMA into one pipeline stage:
+// the x, grad_x_next and grad_h_in tiles (64-byte swizzle, 64-byte L2 fills:
+// the neighbouring half-lines belong to another slice that is read much
+// later), the item's U rows as written by the mapping kernel (128-byte
+// swizzle; the K-major A of MMA1 and the MN-major B of MMA2) and its H
+// records (a contiguous bulk copy).  X is the MN-major A operand of MMA2.
 //
 // grad_phi: a CTA accumulates D2 in TMEM over the consecutive items of one
 // slice ("segment") and flushes it at the segment's end.  A slice is covered
@@ -40,20 +43,26 @@ constexpr int TT = 128;               // tokens per item (MMA1 M, MMA2 K)
 constexpr int CS = 32;                // channels per slice
 constexpr int KR = N * CS;            // 128 phi rows per slice (MMA2 M, MMA1 N)
 constexpr int NU = 64;                // U width: 24 hi + 8 pad + 24 lo + 8 pad
-constexpr int NWARPS = 10;
+constexpr int NEPI = 8;               // epilogue warps: 2 per TMEM lane quarter
+constexpr int CPT = CS / (NEPI / 4);  // channels per epilogue thread (16)
+constexpr int VPT = CPT / 8;          // 16-byte vectors per thread per stream row
+constexpr int NWARPS = 2 + NEPI;
+constexpr int NEPI_T = NEPI * 32;
 constexpr int NT = NWARPS * 32;
 constexpr int XB = TT * CS * 2;       // one stream's x (or G) tile: 8 KB
 constexpr int X_OFF = 0, G_OFF = N * XB, GG_OFF = 2 * N * XB;
-constexpr int STAGE = GG_OFF + XB;    // 72 KB
+constexpr int U_OFF = GG_OFF + XB;              // 73728: U rows of the item, 16 KB
+constexpr int U_BYTES = TT * NU * 2;
+constexpr int H_OFF = U_OFF + U_BYTES;          // 90112: H records, 14 KB
+constexpr int H_BYTES = TT * TcRec::H_BYTES;
+constexpr int STAGE = 104448;                   // 102 KB, 1024-aligned
+static_assert(H_OFF + H_BYTES <= STAGE, "stage layout");
 constexpr int NS = 2;
-constexpr int U_BYTES = TT * NU * 2;  // 16 KB
-constexpr int PHI_BYTES = KR * NU * 2;  // 16 KB
-constexpr int STAGES_OFF = 0;
-constexpr int U_OFF = NS * STAGE;             // 147456
-constexpr int PHI_OFF = U_OFF + 2 * U_BYTES;  // 180224
-constexpr int XCH_OFF = PHI_OFF + PHI_BYTES;  // 196608: D2 exchange [KR][M] floats
-constexpr int DATA = XCH_OFF + KR * M * 4;    // 208896
+constexpr int PHI_BYTES = KR * NU * 2;          // 16 KB
+constexpr int PHI_OFF = NS * STAGE;             // 208896
+constexpr int DATA = PHI_OFF + PHI_BYTES;       // 225280
 constexpr int SMEM = DATA + 1024 + 256;
+static_assert(KR * M * 4 <= H_BYTES, "the D2 exchange reuses a stage's H region");
 constexpr uint32_t TMEM_COLS = 512;           // D1 x2 (256) + D2 (64)
 constexpr uint32_t D2_COL = 256;
 constexpr uint64_t WAIT_NS = 2000000000ull;
@@ -84,10 +93,11 @@ struct ApplyArgs {
   int64_t T, C;
   int S;          // slices = ceil(C / 32)
   int NTT;        // token tiles = ceil(T / 128)
-  int64_t items;  // S * NTT
-  int64_t per;    // items per CTA
+  int paired;     // 1: CTAs 2c and 2c+1 take slices 2v and 2v+1 of the same items
+  int64_t items;  // (paired ? S / 2 : S) * NTT virtual items
+  int64_t per;    // virtual items per CTA (per CTA pair when paired)
   const float* phi;     // [nC][24]
-  const float* coef;    // [T][Coef<4>::SIZE]
+  const float* hrec;    // [T][TcRec::H_FLOATS]
   const float* part;    // bias / alpha partials of the mapping kernel
   int nparts;
   __nv_bfloat16* grad_x;
@@ -102,7 +112,8 @@ struct ApplyArgs {
 
 __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_G,
-    const __grid_constant__ CUtensorMap tm_g, const ApplyArgs a) {
+    const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_u,
+    const ApplyArgs a) {
   using namespace tcap;
   using CF = Coef<N>;
   extern __shared__ uint8_t smem_raw[];
@@ -110,28 +121,32 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
                                              ~(uintptr_t)1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DATA);
   // barrier slots
-  enum { B_FULL = 0, B_SFREE = 2, B_UREADY = 4, B_UFREE = 6, B_D1READY = 8, B_D1FREE = 10,
-         B_SEGREADY = 12, B_SEGDONE = 13, B_FIN = 14, NBARS = 15 };
+  enum { B_FULL = 0, B_SFREE = 2, B_D1READY = 4, B_D1FREE = 6, B_SEGREADY = 8, B_SEGDONE = 9,
+         B_FIN = 10, NBARS = 11 };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* bcast = reinterpret_cast<int*>(tmem_slot + 2);
   auto bar = [&](int i) { return tc::smem_u32(bars + i); };
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int64_t it0 = (int64_t)blockIdx.x * a.per;
+  // Virtual item v = (virtual slice v / NTT, tile v % NTT).  Paired CTAs share
+  // the virtual items and take the even / odd real slice, so the two 64-byte
+  // halves of every 128-byte row are requested at about the same time (one
+  // DRAM fetch with 128-byte L2 fills).
+  const int cta_slot = a.paired ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int half = a.paired ? (int)(blockIdx.x & 1) : 0;
+  const int64_t it0 = (int64_t)cta_slot * a.per;
   const int64_t it1 = (it0 + a.per < a.items) ? it0 + a.per : a.items;
   const int nit = (int)(it1 > it0 ? it1 - it0 : 0);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(bar(B_FULL + s), 1);
-      tc::mbar_init(bar(B_SFREE + s), 1 + 8);
-      tc::mbar_init(bar(B_UREADY + s), 8);
-      tc::mbar_init(bar(B_UFREE + s), 1);
+      tc::mbar_init(bar(B_SFREE + s), 1 + NEPI);
       tc::mbar_init(bar(B_D1READY + s), 1);
-      tc::mbar_init(bar(B_D1FREE + s), 8);
+      tc::mbar_init(bar(B_D1FREE + s), NEPI);
     }
-    tc::mbar_init(bar(B_SEGREADY), 8);
+    tc::mbar_init(bar(B_SEGREADY), NEPI);
     tc::mbar_init(bar(B_SEGDONE), 1);
     tc::mbar_init(bar(B_FIN), 1);
     *abort_flag = 0;
@@ -141,6 +156,7 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
     tc::tma_prefetch_desc(&tm_x);
     tc::tma_prefetch_desc(&tm_G);
     tc::tma_prefetch_desc(&tm_g);
+    tc::tma_prefetch_desc(&tm_u);
   }
   if (warp == 1) {
     tc::tmem_alloc(tc::smem_u32(tmem_slot), TMEM_COLS);
@@ -155,7 +171,10 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
     *abort_flag = 1;
     flag_status(a.status, MHC_ERR_TIMEOUT);
   };
-  auto item_slice = [&](int64_t it) { return (int)(it / a.NTT); };
+  auto item_slice = [&](int64_t it) {
+    const int vs = (int)(it / a.NTT);
+    return a.paired ? 2 * vs + half : vs;
+  };
   auto item_tile = [&](int64_t it) { return (int)(it % a.NTT); };
   auto seg_first = [&](int64_t it) { return it == it0 || item_tile(it) == 0; };
   auto seg_last = [&](int64_t it) { return it == it1 - 1 || item_tile(it) == a.NTT - 1; };
@@ -164,6 +183,7 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
     // ---------------------------------------------------------------- TMA
     if (lane == 0 && nit > 0) {
       const uint64_t pol = tc::policy_evict_first();
+      const uint64_t pol_keep = tc::policy_evict_last();  // records: read by every slice
       int issued = 0;
       for (int i = 0; i < nit; ++i) {
         const int s = i & 1;
@@ -175,13 +195,18 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
         const int64_t it = it0 + i;
         const int c0 = item_slice(it) * CS;
         const int tt0 = item_tile(it) * TT;
-        const uint32_t base = tc::smem_u32(smem + STAGES_OFF + s * STAGE);
-        tc::mbar_arrive_expect_tx(bar(B_FULL + s), STAGE);
+        const uint32_t base = tc::smem_u32(smem + s * STAGE);
+        const int64_t nvalid = (a.T - tt0) < TT ? (a.T - tt0) : TT;
+        const uint32_t hbytes = (uint32_t)nvalid * TcRec::H_BYTES;
+        tc::mbar_arrive_expect_tx(bar(B_FULL + s), (uint32_t)U_OFF + (uint32_t)U_BYTES + hbytes);
         for (int j = 0; j < N; ++j) {
           tc::tma_load_3d(base + X_OFF + j * XB, &tm_x, bar(B_FULL + s), c0, j, tt0, pol);
           tc::tma_load_3d(base + G_OFF + j * XB, &tm_G, bar(B_FULL + s), c0, j, tt0, pol);
         }
         tc::tma_load_2d(base + GG_OFF, &tm_g, bar(B_FULL + s), c0, tt0, pol);
+        tc::tma_load_2d(base + U_OFF, &tm_u, bar(B_FULL + s), 0, tt0, pol_keep);
+        tc::bulk_load(base + H_OFF, a.hrec + (int64_t)tt0 * TcRec::H_FLOATS, hbytes, bar(B_FULL + s),
+                      pol_keep);
         ++issued;
       }
       if (*abort_flag)
@@ -200,8 +225,7 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
         const int64_t it = it0 + i;
         const int s = i & 1, b = i & 1;
         const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-        bool ok = tc::mbar_wait(bar(B_FULL + s), ph, abort_flag, WAIT_NS) &&
-                  tc::mbar_wait(bar(B_UREADY + b), ph, abort_flag, WAIT_NS);
+        bool ok = tc::mbar_wait(bar(B_FULL + s), ph, abort_flag, WAIT_NS);
         if (ok && i >= 2) ok = tc::mbar_wait(bar(B_D1FREE + b), ph ^ 1u, abort_flag, WAIT_NS);
         const bool first = seg_first(it);
         if (ok && first) ok = tc::mbar_wait(bar(B_SEGREADY), (uint32_t)seg & 1u, abort_flag, WAIT_NS);
@@ -210,8 +234,8 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
           break;
         }
         tc::tc_fence_after();
-        const uint32_t xs = tc::smem_u32(smem + STAGES_OFF + s * STAGE + X_OFF);
-        const uint32_t us = tc::smem_u32(smem + U_OFF + b * U_BYTES);
+        const uint32_t xs = tc::smem_u32(smem + s * STAGE + X_OFF);
+        const uint32_t us = tc::smem_u32(smem + s * STAGE + U_OFF);
         // MMA1: D1[b] = U . PHI^T   (K = 64 over m', 128-byte swizzle, K-major)
 #pragma unroll
         for (int k = 0; k < NU / 16; ++k) {
@@ -229,7 +253,6 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
         }
         any = true;
         tc::mma_commit(bar(B_D1READY + b));
-        tc::mma_commit(bar(B_UFREE + b));
         tc::mma_commit(bar(B_SFREE + s));
         if (seg_last(it)) {
           tc::mma_commit(bar(B_SEGDONE));
@@ -244,33 +267,33 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;           // TMEM lane quarter
-    const int h = (warp - 2) >> 2;    // channel half (16 of the slice's 32)
+    const int hq = (warp - 2) >> 2;   // channel group: channels CPT*hq .. CPT*hq+CPT-1 of the slice
     const int tok = 32 * q + lane;    // token row within the tile / phi row in D2
-    const int etid = threadIdx.x - 64;  // 0..255
+    const int etid = threadIdx.x - 64;  // 0 .. NEPI_T-1
 
     if (blockIdx.x == 0) {
       // grad_b / grad_alpha from the mapping kernel's per-CTA partials, in a fixed order
-      float* wsum = reinterpret_cast<float*>(smem + XCH_OFF);
+      float* wsum = reinterpret_cast<float*>(smem + PHI_OFF);  // before PHI is loaded
       const int ew = etid / 32;
       float sacc = 0.0f;
       if (lane <= M)
-        for (int p = ew; p < a.nparts; p += 8) sacc += __ldg(a.part + (int64_t)p * CF::DZ_SIZE + lane);
+        for (int p = ew; p < a.nparts; p += NEPI) sacc += __ldg(a.part + (int64_t)p * CF::DZ_SIZE + lane);
       if (lane <= M) wsum[ew * (M + 1) + lane] = sacc;
-      named_bar_sync(1, 256);
+      named_bar_sync(1, NEPI_T);
       if (etid <= M) {
         float acc = 0.0f;
-        for (int w = 0; w < 8; ++w) acc += wsum[w * (M + 1) + etid];
+        for (int w = 0; w < NEPI; ++w) acc += wsum[w * (M + 1) + etid];
         if (etid < M) a.grad_b[etid] = acc;
         else *a.grad_alpha = acc;
       }
-      named_bar_sync(1, 256);
+      named_bar_sync(1, NEPI_T);
     }
 
     // PHI for a slice: row r = j*32 + c holds phi_hi[j*C + c0 + c][0..23] in m' 0..23
     // and again in m' 32..55 (zeros elsewhere), 128-byte swizzle.
     auto load_phi = [&](int slice) {
       uint8_t* ps = smem + PHI_OFF;
-      for (int e = etid; e < KR * 8; e += 256) {
+      for (int e = etid; e < KR * 8; e += NEPI_T) {
         const int r = e >> 3, chunk = e & 7;
         const int j = r / CS, cl = r % CS;
         const int64_t c = (int64_t)slice * CS + cl;
@@ -289,211 +312,147 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
       if (lane == 0) tc::mbar_arrive(bar(B_SEGREADY));
     };
 
-    // coefficient record of token row `tok` of item i; writes this thread's half of
-    // the U row (h = 0: u_hi, h = 1: u_lo) into U buffer i & 1.
-    float hres[N * N], hpre[N], hpost[N], kap;      // for the item being finished
-    float nres[N * N], npre[N], npost[N], nkap;     // for the item whose U was written
-    auto write_u = [&](int i) {
-      const int64_t it = it0 + i;
-      const int64_t t = (int64_t)item_tile(it) * TT + tok;
-      float rec[CF::SIZE];
-      if (t < a.T) {
-        const float4* src = reinterpret_cast<const float4*>(a.coef + t * CF::SIZE);
-#pragma unroll
-        for (int e = 0; e < CF::SIZE / 4; ++e) {
-          const float4 v = __ldg(src + e);
-          rec[4 * e] = v.x; rec[4 * e + 1] = v.y; rec[4 * e + 2] = v.z; rec[4 * e + 3] = v.w;
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < CF::SIZE; ++e) rec[e] = 0.0f;
-      }
-#pragma unroll
-      for (int e = 0; e < N * N; ++e) nres[e] = rec[CF::RES + e];
-#pragma unroll
-      for (int e = 0; e < N; ++e) {
-        npre[e] = rec[CF::PRE + e];
-        npost[e] = rec[CF::POST + e];
-      }
-      nkap = rec[CF::KAPPA];
-      float uv[32];
-#pragma unroll
-      for (int m = 0; m < 32; ++m) {
-        float u = m < M ? rec[CF::U + m] : 0.0f;
-        const float hi = __bfloat162float(__float2bfloat16_rn(u));
-        uv[m] = h == 0 ? hi : u - hi;
-      }
-      const int b = i & 1;
-      if (i >= 2 &&
-          !tc::mbar_wait(bar(B_UFREE + b), (uint32_t)((i >> 1) - 1) & 1u, abort_flag, WAIT_NS)) {
-        give_up();
-        return;
-      }
-      uint8_t* us = smem + U_OFF + b * U_BYTES;
-#pragma unroll
-      for (int cch = 0; cch < 4; ++cch)
-        *reinterpret_cast<uint4*>(us + sw128(tok, 4 * h + cch)) =
-            make_uint4(pack2(uv[8 * cch], uv[8 * cch + 1]), pack2(uv[8 * cch + 2], uv[8 * cch + 3]),
-                       pack2(uv[8 * cch + 4], uv[8 * cch + 5]), pack2(uv[8 * cch + 6], uv[8 * cch + 7]));
-      tc::fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(bar(B_UREADY + b));
-    };
-    auto rotate = [&]() {
-#pragma unroll
-      for (int e = 0; e < N * N; ++e) hres[e] = nres[e];
-#pragma unroll
-      for (int e = 0; e < N; ++e) {
-        hpre[e] = npre[e];
-        hpost[e] = npost[e];
-      }
-      kap = nkap;
-    };
-
     int seg = 0;
-    if (nit > 0) {
-      load_phi(item_slice(it0));
-      write_u(0);
-      rotate();
-    }
-    float* xch = reinterpret_cast<float*>(smem + XCH_OFF);
+    if (nit > 0) load_phi(item_slice(it0));
     // The loop never breaks: after a failed wait it keeps walking the items
     // without touching memory, so all eight warps meet every named barrier.
     for (int i = 0; i < nit; ++i) {
       const int64_t it = it0 + i;
       const int s = i & 1, b = i & 1;
       const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-      if (i + 1 < nit && !*abort_flag) write_u(i + 1);
       bool live = !*abort_flag;
       if (live && (!tc::mbar_wait(bar(B_FULL + s), ph, abort_flag, WAIT_NS) ||
                    !tc::mbar_wait(bar(B_D1READY + b), ph, abort_flag, WAIT_NS))) {
         give_up();
         live = false;
       }
+      live = __all_sync(0xffffffffu, live);  // TMEM loads below are warp-collective
       tc::tc_fence_after();
       const int slice = item_slice(it);
       const int64_t t = (int64_t)item_tile(it) * TT + tok;
-      const int64_t cbase = (int64_t)slice * CS + 16 * h;
-      const uint8_t* st = smem + STAGES_OFF + s * STAGE;
-      // G and g for this thread's 16 channels, all four streams
-      float Gv[N][16], gv[16];
-#pragma unroll
-      for (int i2 = 0; i2 < N; ++i2) {
-        float tmp[8];
-        unpack8(*reinterpret_cast<const uint4*>(st + G_OFF + i2 * XB + sw64(tok, 2 * h)), tmp);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) Gv[i2][e] = tmp[e];
-        unpack8(*reinterpret_cast<const uint4*>(st + G_OFF + i2 * XB + sw64(tok, 2 * h + 1)), tmp);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) Gv[i2][8 + e] = tmp[e];
-      }
-      {
-        float tmp[8];
-        unpack8(*reinterpret_cast<const uint4*>(st + GG_OFF + sw64(tok, 2 * h)), tmp);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) gv[e] = tmp[e];
-        unpack8(*reinterpret_cast<const uint4*>(st + GG_OFF + sw64(tok, 2 * h + 1)), tmp);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) gv[8 + e] = tmp[e];
-      }
+      const int64_t cbase = (int64_t)slice * CS + CPT * hq;   // this thread's channels
+      const uint8_t* st = smem + s * STAGE;
       const bool tvalid = live && t < a.T;
-      // grad_f_out
-      if (tvalid) {
-        float o[16];
+      // this token's H record
+      float hres[N * N], hpre[N], hpost[N], kap;
+      {
+        const float4* hr = reinterpret_cast<const float4*>(st + H_OFF + tok * TcRec::H_BYTES);
+        float rec[TcRec::H_FLOATS];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
+        for (int e = 0; e < TcRec::H_FLOATS / 4; ++e) {
+          const float4 v = hr[e];
+          rec[4 * e] = v.x; rec[4 * e + 1] = v.y; rec[4 * e + 2] = v.z; rec[4 * e + 3] = v.w;
+        }
+#pragma unroll
+        for (int e = 0; e < N * N; ++e) hres[e] = rec[TcRec::H_RES + e];
+#pragma unroll
+        for (int e = 0; e < N; ++e) {
+          hpre[e] = rec[TcRec::H_PRE + e];
+          hpost[e] = rec[TcRec::H_POST + e];
+        }
+        kap = rec[TcRec::H_KAPPA];
+      }
+#pragma unroll
+      for (int v = 0; v < VPT; ++v) {
+        const int chunk = VPT * hq + v;            // 16-byte chunk of the 64-byte tile row
+        const int64_t c8 = cbase + 8 * v;
+        const bool ok8 = tvalid && c8 < a.C;
+        // phi u of the four output streams for these 8 channels: four TMEM loads,
+        // one wait (warp-collective: every lane takes part, whatever its token)
+        float d1[N][8];
+        if (live) {
+#pragma unroll
+          for (int jj = 0; jj < N; ++jj)
+            tc::tmem_ld8(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * KR + jj * CS + 8 * chunk),
+                         d1[jj]);
+        }
+        float Gv[N][8], gv[8], xv[N][8];
+#pragma unroll
+        for (int i2 = 0; i2 < N; ++i2) {
+          unpack8(*reinterpret_cast<const uint4*>(st + G_OFF + i2 * XB + sw64(tok, chunk)), Gv[i2]);
+          unpack8(*reinterpret_cast<const uint4*>(st + X_OFF + i2 * XB + sw64(tok, chunk)), xv[i2]);
+        }
+        unpack8(*reinterpret_cast<const uint4*>(st + GG_OFF + sw64(tok, chunk)), gv);
+        if (live) tc::tmem_ld_wait();
+        float o[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
           float acc = 0.0f;
 #pragma unroll
           for (int i2 = 0; i2 < N; ++i2) acc = fmaf(hpost[i2], Gv[i2][e], acc);
           o[e] = acc;
         }
+        if (ok8)
+          __stcs(reinterpret_cast<uint4*>(a.grad_f + t * a.C + c8),
+                 make_uint4(pack2(o[0], o[1]), pack2(o[2], o[3]), pack2(o[4], o[5]), pack2(o[6], o[7])));
 #pragma unroll
-        for (int v8 = 0; v8 < 2; ++v8) {
-          if (cbase + 8 * v8 < a.C) {
-            uint4 pk = make_uint4(pack2(o[8 * v8], o[8 * v8 + 1]), pack2(o[8 * v8 + 2], o[8 * v8 + 3]),
-                                  pack2(o[8 * v8 + 4], o[8 * v8 + 5]), pack2(o[8 * v8 + 6], o[8 * v8 + 7]));
-            __stcs(reinterpret_cast<uint4*>(a.grad_f + t * a.C + cbase + 8 * v8), pk);
-          }
-        }
-      }
-      // grad_x, one output stream at a time
+        for (int jj = 0; jj < N; ++jj) {
 #pragma unroll
-      for (int jj = 0; jj < N; ++jj) {
-        float d1[16];
-        if (live)
-          tc::tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * KR + jj * CS + 16 * h), d1);
-        float xv[16];
-        {
-          float tmp[8];
-          unpack8(*reinterpret_cast<const uint4*>(st + X_OFF + jj * XB + sw64(tok, 2 * h)), tmp);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) xv[e] = tmp[e];
-          unpack8(*reinterpret_cast<const uint4*>(st + X_OFF + jj * XB + sw64(tok, 2 * h + 1)), tmp);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) xv[8 + e] = tmp[e];
-        }
-        if (live) tc::tmem_ld_wait();
-        if (tvalid) {
-          float o[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            float acc = fmaf(hpre[jj], gv[e], d1[e]);
+          for (int e = 0; e < 8; ++e) {
+            float acc = fmaf(hpre[jj], gv[e], d1[jj][e]);
 #pragma unroll
             for (int i2 = 0; i2 < N; ++i2) acc = fmaf(hres[i2 * N + jj], Gv[i2][e], acc);
-            o[e] = fmaf(-kap, xv[e], acc);
+            o[e] = fmaf(-kap, xv[jj][e], acc);
           }
-#pragma unroll
-          for (int v8 = 0; v8 < 2; ++v8) {
-            if (cbase + 8 * v8 < a.C) {
-              uint4 pk = make_uint4(pack2(o[8 * v8], o[8 * v8 + 1]), pack2(o[8 * v8 + 2], o[8 * v8 + 3]),
-                                    pack2(o[8 * v8 + 4], o[8 * v8 + 5]), pack2(o[8 * v8 + 6], o[8 * v8 + 7]));
-              __stcs(reinterpret_cast<uint4*>(a.grad_x + (t * N + jj) * a.C + cbase + 8 * v8), pk);
-            }
-          }
+          if (ok8)
+            __stcs(reinterpret_cast<uint4*>(a.grad_x + (t * N + jj) * a.C + c8),
+                   make_uint4(pack2(o[0], o[1]), pack2(o[2], o[3]), pack2(o[4], o[5]), pack2(o[6], o[7])));
         }
       }
       tc::tc_fence_before();
       __syncwarp();
+      const bool last = seg_last(it);
       if (lane == 0 && live) {
         tc::mbar_arrive(bar(B_D1FREE + b));
-        tc::mbar_arrive(bar(B_SFREE + s));
+        // the stage of a segment's last item is released after the flush, which
+        // uses its H region as scratch
+        if (!last) tc::mbar_arrive(bar(B_SFREE + s));
       }
-      rotate();
 
-      if (seg_last(it)) {
-        // ---- flush this segment's grad_phi rows
+      if (last) {
+        // ---- flush this segment's grad_phi rows.  Every warp has finished
+        // reading this stage's H records before any overwrites them.
+        named_bar_sync(1, NEPI_T);
+        float* xch = reinterpret_cast<float*>(smem + s * STAGE + H_OFF);  // [KR][M]: the u_lo part
         if (live && !tc::mbar_wait(bar(B_SEGDONE), (uint32_t)seg & 1u, abort_flag, WAIT_NS)) {
           give_up();
           live = false;
         }
+        live = __all_sync(0xffffffffu, live);
         tc::tc_fence_after();
-        // D2 row tok (phi row j*32 + c of the slice); h = 0 reads m' 0..31 (u_hi),
-        // h = 1 reads m' 32..63 (u_lo); the two halves meet in shared memory.
-        float dd[16], dd2[16];
+        // D2 row tok (phi row j*32 + c of the slice): hq = 0 reads m' 0..31 (the
+        // u_hi part), hq = 1 reads m' 32..63 (the u_lo part); they meet in smem.
+        float dd[32];
         if (live) {
-          tc::tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + D2_COL + 32 * h, dd);
-          tc::tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + D2_COL + 32 * h + 16, dd2);
+          float t16[16];
+          tc::tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + D2_COL + 32 * hq, t16);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) dd[e] = t16[e];
+          tc::tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + D2_COL + 32 * hq + 16, t16);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) dd[16 + e] = t16[e];
           tc::tmem_ld_wait();
         }
-        if (live && h == 1) {
+        if (live && hq == 1) {
 #pragma unroll
-          for (int m = 0; m < M; ++m) xch[tok * M + m] = m < 16 ? dd[m] : dd2[m - 16];
+          for (int m = 0; m < M; ++m) xch[tok * M + m] = dd[m];
         }
-        named_bar_sync(1, 256);
+        named_bar_sync(1, NEPI_T);
         const int j = tok / CS, cl = tok % CS;
         const int64_t c = (int64_t)slice * CS + cl;
         // part 0: this CTA holds the slice's first item; part 1: its last items
         const int part_idx = (it - item_tile(it) >= it0) ? 0 : 1;
-        const bool whole = (it - item_tile(it) >= it0) && (it == (int64_t)slice * a.NTT + a.NTT - 1);
+        const bool whole = (it - item_tile(it) >= it0) && (item_tile(it) == a.NTT - 1);
         float* dst_row = a.grad_phi + ((int64_t)j * a.C + c) * M;
-        if (live && h == 0) {
+        if (live && hq == 0) {
           float sum[M];
 #pragma unroll
-          for (int m = 0; m < M; ++m) sum[m] = (m < 16 ? dd[m] : dd2[m - 16]) + xch[tok * M + m];
+          for (int m = 0; m < M; ++m) sum[m] = dd[m] + xch[tok * M + m];
           if (whole) {
-            if (c < a.C)
+            if (c < a.C) {
 #pragma unroll
               for (int m = 0; m < M; ++m) dst_row[m] = sum[m];
+            }
           } else {
             float* pr = a.gphi_part + (((int64_t)slice * 2 + part_idx) * KR + tok) * M;
 #pragma unroll
@@ -502,13 +461,13 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
         }
         if (!whole) {
           __threadfence();
-          named_bar_sync(1, 256);
+          named_bar_sync(1, NEPI_T);
           if (etid == 0) *bcast = live ? atomicAdd(a.gphi_cnt + slice, 1) : -1;
-          named_bar_sync(1, 256);
+          named_bar_sync(1, NEPI_T);
           if (*bcast == 1) {
             // both parts are in memory: add them in part order
             __threadfence();
-            if (h == 0 && c < a.C) {
+            if (hq == 0 && c < a.C) {
               const float* p0 = a.gphi_part + (((int64_t)slice * 2 + 0) * KR + tok) * M;
               const float* p1 = a.gphi_part + (((int64_t)slice * 2 + 1) * KR + tok) * M;
 #pragma unroll
@@ -518,7 +477,8 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
           }
         }
         tc::tc_fence_before();
-        named_bar_sync(1, 256);
+        named_bar_sync(1, NEPI_T);
+        if (lane == 0 && live) tc::mbar_arrive(bar(B_SFREE + s));
         ++seg;
         if (i + 1 < nit && live) load_phi(item_slice(it + 1));
       }
@@ -541,8 +501,8 @@ size_t apply_tc_scratch_bytes(int64_t C) {
 }
 
 cudaError_t apply_tc_dispatch(int64_t T, int64_t C, const void* x, const float* phi, const void* G,
-                              const void* g, const float* coef, const float* part, int nparts,
-                              void* gx, void* gf, float* gphi, float* gb, float* ga,
+                              const void* g, const void* urec, const float* hrec, const float* part,
+                              int nparts, void* gx, void* gf, float* gphi, float* gb, float* ga,
                               void* scratch, int* st, cudaStream_t s) {
   using namespace tcap;
   int dev = 0, num_sms = 0;
@@ -550,31 +510,45 @@ cudaError_t apply_tc_dispatch(int64_t T, int64_t C, const void* x, const float* 
   if (e != cudaSuccess) return e;
   e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  CUtensorMap mx, mG, mg;
+  CUtensorMap mx, mG, mg, mu;
   const uint64_t dx[3] = {(uint64_t)C, (uint64_t)N, (uint64_t)T};
   const uint64_t sx[2] = {(uint64_t)C * 2, (uint64_t)N * C * 2};
   const uint32_t bx[3] = {CS, 1, TT};
-  e = make_tmap_bf16(&mx, x, 3, dx, sx, bx, CU_TENSOR_MAP_SWIZZLE_64B);
+  const int S = (int)((C + CS - 1) / CS);
+  const bool paired = (S % 2 == 0) && num_sms >= 2;
+  // paired CTAs read both halves of each 128-byte row: fetch it whole
+  const CUtensorMapL2promotion promo =
+      paired ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B : CU_TENSOR_MAP_L2_PROMOTION_L2_64B;
+  e = make_tmap_bf16(&mx, x, 3, dx, sx, bx, CU_TENSOR_MAP_SWIZZLE_64B, promo);
   if (e != cudaSuccess) return e;
-  e = make_tmap_bf16(&mG, G, 3, dx, sx, bx, CU_TENSOR_MAP_SWIZZLE_64B);
+  e = make_tmap_bf16(&mG, G, 3, dx, sx, bx, CU_TENSOR_MAP_SWIZZLE_64B, promo);
   if (e != cudaSuccess) return e;
   const uint64_t d2[2] = {(uint64_t)C, (uint64_t)T};
   const uint64_t s2[1] = {(uint64_t)C * 2};
   const uint32_t b2[2] = {CS, TT};
-  e = make_tmap_bf16(&mg, g, 2, d2, s2, b2, CU_TENSOR_MAP_SWIZZLE_64B);
+  e = make_tmap_bf16(&mg, g, 2, d2, s2, b2, CU_TENSOR_MAP_SWIZZLE_64B, promo);
+  if (e != cudaSuccess) return e;
+  const uint64_t du[2] = {(uint64_t)NU, (uint64_t)T};
+  const uint64_t su[1] = {(uint64_t)NU * 2};
+  const uint32_t bu[2] = {NU, TT};
+  e = make_tmap_bf16(&mu, urec, 2, du, su, bu, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
 
   ApplyArgs a;
   a.T = T;
   a.C = C;
-  a.S = (int)((C + CS - 1) / CS);
+  a.S = S;
   a.NTT = (int)((T + TT - 1) / TT);
-  a.items = (int64_t)a.S * a.NTT;
-  // at most one CTA per slice so that every slice meets at most two CTAs
-  const int grid = a.S < num_sms ? a.S : num_sms;
-  a.per = (a.items + grid - 1) / grid;
+  a.paired = paired ? 1 : 0;
+  const int vslices = paired ? S / 2 : S;
+  a.items = (int64_t)vslices * a.NTT;
+  // at most one CTA (pair) per virtual slice, so every slice meets at most two CTAs
+  const int slots_max = paired ? num_sms / 2 : num_sms;
+  const int slots = vslices < slots_max ? vslices : slots_max;
+  a.per = (a.items + slots - 1) / slots;
+  const int grid = paired ? 2 * slots : slots;
   a.phi = phi;
-  a.coef = coef;
+  a.hrec = hrec;
   a.part = part;
   a.nparts = nparts;
   a.grad_x = (__nv_bfloat16*)gx;
@@ -590,7 +564,7 @@ cudaError_t apply_tc_dispatch(int64_t T, int64_t C, const void* x, const float* 
   // slice counters start at zero (the combining CTA resets its counter too)
   e = cudaMemsetAsync(a.gphi_cnt, 0, (size_t)a.S * sizeof(int), s);
   if (e != cudaSuccess) return e;
-  k_apply_tc<<<grid, NT, SMEM, s>>>(mx, mG, mg, a);
+  k_apply_tc<<<grid, NT, SMEM, s>>>(mx, mG, mg, mu, a);
   return cudaGetLastError();
 }
 

@@ -97,7 +97,8 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
     const __grid_constant__ CUtensorMap tm_f, int64_t T, int64_t C, int iters, float eps,
     int ck_period, const float* __restrict__ bias, const float* __restrict__ alpha_p,
     float* __restrict__ Hpre_o, float* __restrict__ Hpost_o, float* __restrict__ Hres_o,
-    float* __restrict__ coef_o, float* __restrict__ part_o, int* status) {
+    __nv_bfloat16* __restrict__ urec_o, float* __restrict__ hrec_o, float* __restrict__ part_o,
+    int* status) {
   using namespace tcmap;
   using CFG = Cfg<BWD>;
   constexpr int NS = CFG::NS;
@@ -271,6 +272,7 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
     // stage memory is reused for the epilogue
     bool ok = !*abort_flag && tc::mbar_wait(done_bar, 0, abort_flag, WAIT_NS);
     if (!ok && !*abort_flag) give_up();
+    ok = __all_sync(0xffffffffu, ok);  // the TMEM loads below are warp-collective
     float* red_ss = reinterpret_cast<float*>(smem);       // [2][TM]
     float* red_dt = red_ss + 2 * TM;                      // [2][M][TM]
     float* dzs = red_dt + 2 * M * TM;                     // [M + 1][TM]
@@ -362,25 +364,35 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
         for (int m = 0; m < M; ++m) dzy = fmaf(dz[m], y[m], dzy);
         const bool live = t < T;
         if (live) {
-          using CF = Coef<N>;
-          float rec[CF::SIZE];
+          float rec[TcRec::H_FLOATS];
 #pragma unroll
-          for (int e = 0; e < N * N; ++e) rec[CF::RES + e] = H[e];
+          for (int e = 0; e < N * N; ++e) rec[TcRec::H_RES + e] = H[e];
 #pragma unroll
           for (int i = 0; i < N; ++i) {
-            rec[CF::PRE + i] = spre[i];
-            rec[CF::POST + i] = 2.0f * spost[i];
+            rec[TcRec::H_PRE + i] = spre[i];
+            rec[TcRec::H_POST + i] = 2.0f * spost[i];
           }
+          rec[TcRec::H_KAPPA] = alpha * dzy / ((float)K * r * r);
+          rec[25] = rec[26] = rec[27] = 0.0f;
+          float4* hd = reinterpret_cast<float4*>(hrec_o + t * TcRec::H_FLOATS);
+#pragma unroll
+          for (int e = 0; e < TcRec::H_FLOATS / 4; ++e)
+            hd[e] = make_float4(rec[4 * e], rec[4 * e + 1], rec[4 * e + 2], rec[4 * e + 3]);
           const float ar = alpha / r;
+          uint32_t w[32];
 #pragma unroll
-          for (int m = 0; m < M; ++m) rec[CF::U + m] = ar * dz[m];
-          rec[CF::KAPPA] = alpha * dzy / ((float)K * r * r);
+          for (int m2 = 0; m2 < 12; ++m2) {
+            const float u0 = ar * dz[2 * m2], u1 = ar * dz[2 * m2 + 1];
+            const __nv_bfloat162 hi = __floats2bfloat162_rn(u0, u1);
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(u0 - __low2float(hi), u1 - __high2float(hi));
+            w[m2] = *reinterpret_cast<const uint32_t*>(&hi);
+            w[16 + m2] = *reinterpret_cast<const uint32_t*>(&lo);
+          }
 #pragma unroll
-          for (int e = CF::KAPPA + 1; e < CF::SIZE; ++e) rec[e] = 0.0f;
-          float4* dst = reinterpret_cast<float4*>(coef_o + t * CF::SIZE);
+          for (int m2 = 12; m2 < 16; ++m2) w[m2] = w[16 + m2] = 0u;
+          uint4* ud = reinterpret_cast<uint4*>(urec_o + t * TcRec::U_ELEMS);
 #pragma unroll
-          for (int e = 0; e < CF::SIZE / 4; ++e)
-            dst[e] = make_float4(rec[4 * e], rec[4 * e + 1], rec[4 * e + 2], rec[4 * e + 3]);
+          for (int e = 0; e < 8; ++e) ud[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
         }
 #pragma unroll
         for (int m = 0; m < M; ++m) dzs[m * TM + tok] = live ? dz[m] : 0.0f;
@@ -455,7 +467,8 @@ size_t map_tc_phi_bytes(int64_t C) { return (size_t)tcmap::NL * tcmap::N * C * 2
 cudaError_t map_tc_dispatch(bool bwd, int64_t T, int64_t C, int iters, float eps, const void* x,
                             const float* phi, void* phi_split, const float* b, const float* alpha,
                             float* Hpre, float* Hpost, float* Hres, const void* G, const void* g,
-                            const void* f, float* coef, float* part, int* st, cudaStream_t s) {
+                            const void* f, void* urec, float* hrec, float* part, int* st,
+                            cudaStream_t s) {
   using namespace tcmap;
   const int64_t K = (int64_t)N * C;
   k_phi_split<<<(unsigned)((K + 255) / 256), 256, 0, s>>>(K, phi, (__nv_bfloat16*)phi_split);
@@ -471,13 +484,14 @@ cudaError_t map_tc_dispatch(bool bwd, int64_t T, int64_t C, int iters, float eps
     if (e != cudaSuccess) return e;
     const int P = ck_period_for(iters, Cfg<true>::DATA);
     kern<<<grid, NT, Cfg<true>::SMEM, s>>>(mx, mp, mG, mg, mf, T, C, iters, eps, P, b, alpha,
-                                           nullptr, nullptr, nullptr, coef, part, st);
+                                           nullptr, nullptr, nullptr, (__nv_bfloat16*)urec, hrec,
+                                           part, st);
   } else {
     auto kern = k_map_tc<false>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<false>::SMEM);
     if (e != cudaSuccess) return e;
     kern<<<grid, NT, Cfg<false>::SMEM, s>>>(mx, mp, mG, mg, mf, T, C, iters, eps, 1, b, alpha,
-                                            Hpre, Hpost, Hres, nullptr, nullptr, st);
+                                            Hpre, Hpost, Hres, nullptr, nullptr, nullptr, st);
   }
   return cudaGetLastError();
 }

@@ -28,12 +28,13 @@ cudaError_t map_bwd_dispatch(int n, int dtype, int64_t T, int64_t C, int iters, 
 cudaError_t map_tc_dispatch(bool bwd, int64_t T, int64_t C, int iters, float eps, const void* x,
                             const float* phi, void* phi_split, const float* b, const float* alpha,
                             float* Hpre, float* Hpost, float* Hres, const void* G, const void* g,
-                            const void* f, float* coef, float* part, int* st, cudaStream_t s);
+                            const void* f, void* urec, float* hrec, float* part, int* st,
+                            cudaStream_t s);
 size_t map_tc_phi_bytes(int64_t C);
 // k_apply_tc.cu (bf16, n = 4: phi u and grad_phi on the tensor cores)
 cudaError_t apply_tc_dispatch(int64_t T, int64_t C, const void* x, const float* phi, const void* G,
-                              const void* g, const float* coef, const float* part, int nparts,
-                              void* gx, void* gf, float* gphi, float* gb, float* ga,
+                              const void* g, const void* urec, const float* hrec, const float* part,
+                              int nparts, void* gx, void* gf, float* gphi, float* gb, float* ga,
                               void* scratch, int* st, cudaStream_t s);
 size_t apply_tc_scratch_bytes(int64_t C);
 // k_bwd.cu
@@ -84,24 +85,38 @@ int dz_size(int n) {
 // per CTA); every other case the CUDA-core one (64 tokens per CTA).
 bool use_tc(const mhc_params* p) { return p->dtype == MHC_DTYPE_BF16 && p->n == 4; }
 
-// Backward workspace: per-token coefficient records, one partial-sum record
-// (dz, dz . y) per mapping CTA, then (tensor-core path) the bf16 split copy
-// of phi^T that the mapping MMA reads and the apply kernel's grad_phi
-// partials and slice counters.
+// Backward workspace.  CUDA-core path: per-token coefficient records, then one
+// partial-sum record (dz, dz . y) per 64-token mapping CTA.  Tensor-core path:
+// per-token U rows (bf16) and H records, the partial sums per 128-token CTA,
+// the bf16 split copy of phi^T that the mapping MMA reads, and the apply
+// kernel's grad_phi partials and slice counters.
 struct BwdWorkspace {
-  size_t coef_off, part_off, phi_off, apply_off, total;
+  size_t coef_off, urec_off, hrec_off, part_off, phi_off, apply_off, total;
   int nparts;
 };
 
 BwdWorkspace bwd_layout(const mhc_params* p) {
-  BwdWorkspace w;
-  const int tokens_per_cta = use_tc(p) ? 128 : 64;
+  BwdWorkspace w{};
+  const bool tc = use_tc(p);
+  const int tokens_per_cta = tc ? 128 : 64;
   w.nparts = (int)((p->T + tokens_per_cta - 1) / tokens_per_cta);
-  w.coef_off = 0;
-  w.part_off = round_up(w.coef_off + (size_t)p->T * coef_size(p->n) * 4, 256);
-  w.phi_off = round_up(w.part_off + (size_t)w.nparts * dz_size(p->n) * 4, 256);
-  w.apply_off = round_up(w.phi_off + (use_tc(p) ? mhc::map_tc_phi_bytes(p->C) : 0), 256);
-  w.total = round_up(w.apply_off + (use_tc(p) ? mhc::apply_tc_scratch_bytes(p->C) : 0), 256);
+  size_t off = 0;
+  if (tc) {
+    w.urec_off = off;
+    off = round_up(off + (size_t)p->T * mhc::TcRec::U_BYTES, 256);
+    w.hrec_off = off;
+    off = round_up(off + (size_t)p->T * mhc::TcRec::H_BYTES, 256);
+  } else {
+    w.coef_off = off;
+    off = round_up(off + (size_t)p->T * coef_size(p->n) * 4, 256);
+  }
+  w.part_off = off;
+  off = round_up(off + (size_t)w.nparts * dz_size(p->n) * 4, 256);
+  w.phi_off = off;
+  off = round_up(off + (tc ? mhc::map_tc_phi_bytes(p->C) : 0), 256);
+  w.apply_off = off;
+  off = round_up(off + (tc ? mhc::apply_tc_scratch_bytes(p->C) : 0), 256);
+  w.total = off;
   return w;
 }
 
@@ -151,7 +166,7 @@ mhc_status mhc_pre(const mhc_params* p, const void* x, const float* phi, const f
       return MHC_ERR_WORKSPACE;
     st = from_cuda(mhc::map_tc_dispatch(false, p->T, p->C, p->t_max, p->eps, x, phi, workspace, b,
                                         alpha, H_pre, H_post, H_res, nullptr, nullptr, nullptr,
-                                        nullptr, nullptr, dev_status, s));
+                                        nullptr, nullptr, nullptr, dev_status, s));
   } else {
     st = from_cuda(mhc::map_fwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
                                          alpha, H_pre, H_post, H_res, dev_status, s));
@@ -194,8 +209,8 @@ mhc_status mhc_backward_map(const mhc_params* p, const void* x, const float* phi
   if (use_tc(p))
     return from_cuda(mhc::map_tc_dispatch(true, p->T, p->C, p->t_max, p->eps, x, phi,
                                           ws + w.phi_off, b, alpha, nullptr, nullptr, nullptr,
-                                          grad_x_next, grad_h_in, f_out,
-                                          (float*)(ws + w.coef_off), (float*)(ws + w.part_off),
+                                          grad_x_next, grad_h_in, f_out, ws + w.urec_off,
+                                          (float*)(ws + w.hrec_off), (float*)(ws + w.part_off),
                                           dev_status, (cudaStream_t)stream));
   return from_cuda(mhc::map_bwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
                                          alpha, grad_x_next, grad_h_in, f_out,
@@ -221,7 +236,7 @@ mhc_status mhc_backward_apply(const mhc_params* p, const void* x, const float* p
   const char* ws = (const char*)workspace;
   if (use_tc(p))
     return from_cuda(mhc::apply_tc_dispatch(p->T, p->C, x, phi, grad_x_next, grad_h_in,
-                                            (const float*)(ws + w.coef_off),
+                                            ws + w.urec_off, (const float*)(ws + w.hrec_off),
                                             (const float*)(ws + w.part_off), w.nparts, grad_x,
                                             grad_f_out, grad_phi, grad_b, grad_alpha,
                                             (void*)(ws + w.apply_off), dev_status,

@@ -253,4 +253,17 @@ template <int N> struct Coef {
   static constexpr int DZ_SIZE = ((M + 1) + 3) / 4 * 4;
 };
 
+// Per-token records of the tensor-core backward (n = 4), written by the
+// mapping kernel and streamed by the apply kernel's TMA:
+//   U row  [64] bf16: u_hi (24) | 0 (8) | u_lo (24) | 0 (8), u = alpha dz / r,
+//          u_lo = bf16(u - u_hi) -- the MMA operand row, 128 bytes
+//   H rec  [28] fp32: H_res (16) | H_pre (4) | H_post (4) | kappa | 0 0 0
+struct TcRec {
+  static constexpr int U_ELEMS = 64;
+  static constexpr int U_BYTES = U_ELEMS * 2;
+  static constexpr int H_FLOATS = 28;
+  static constexpr int H_BYTES = H_FLOATS * 4;
+  static constexpr int H_RES = 0, H_PRE = 16, H_POST = 20, H_KAPPA = 24;
+};
+
 }  // namespace mhc

@@ -17,7 +17,7 @@ std::once_flag g_encode_once;
 
 cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                            const uint64_t* strides_bytes, const uint32_t* box,
-                           CUtensorMapSwizzle swz) {
+                           CUtensorMapSwizzle swz, CUtensorMapL2promotion promo) {
   std::call_once(g_encode_once, [] {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
@@ -38,8 +38,7 @@ cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const u
   }
   const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank,
                               const_cast<void*>(base), gdim, gstr, bdim, estr,
-                              CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, promo,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
