@@ -93,9 +93,9 @@ struct ApplyArgs {
   int64_t T, C;
   int S;          // slices = ceil(C / 32)
   int NTT;        // token tiles = ceil(T / 128)
-  int paired;     // 1: CTAs 2c and 2c+1 take slices 2v and 2v+1 of the same items
-  int64_t items;  // (paired ? S / 2 : S) * NTT virtual items
-  int64_t per;    // virtual items per CTA (per CTA pair when paired)
+  int group;      // CTAs g*c .. g*c+g-1 take slices g*v .. g*v+g-1 of the same items
+  int64_t items;  // (S / group) * NTT virtual items
+  int64_t per;    // virtual items per CTA group
   const float* phi;     // [nC][24]
   const float* hrec;    // [T][TcRec::H_FLOATS]
   const float* part;    // bias / alpha partials of the mapping kernel
@@ -129,12 +129,13 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
   auto bar = [&](int i) { return tc::smem_u32(bars + i); };
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  // Virtual item v = (virtual slice v / NTT, tile v % NTT).  Paired CTAs share
-  // the virtual items and take the even / odd real slice, so the two 64-byte
-  // halves of every 128-byte row are requested at about the same time (one
-  // DRAM fetch with 128-byte L2 fills).
-  const int cta_slot = a.paired ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
-  const int half = a.paired ? (int)(blockIdx.x & 1) : 0;
+  // Virtual item v = (virtual slice v / NTT, tile v % NTT).  The `group` CTAs
+  // of a slot share the virtual items and take adjacent real slices, so the
+  // group's 64-byte pieces of each row (group * 64 bytes in all) are requested
+  // at about the same time and reach DRAM as one wide fetch (L2 fills of
+  // group * 64 bytes).
+  const int cta_slot = (int)(blockIdx.x / a.group);
+  const int member = (int)(blockIdx.x % a.group);
   const int64_t it0 = (int64_t)cta_slot * a.per;
   const int64_t it1 = (it0 + a.per < a.items) ? it0 + a.per : a.items;
   const int nit = (int)(it1 > it0 ? it1 - it0 : 0);
@@ -173,7 +174,7 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
   };
   auto item_slice = [&](int64_t it) {
     const int vs = (int)(it / a.NTT);
-    return a.paired ? 2 * vs + half : vs;
+    return a.group * vs + member;
   };
   auto item_tile = [&](int64_t it) { return (int)(it % a.NTT); };
   auto seg_first = [&](int64_t it) { return it == it0 || item_tile(it) == 0; };
@@ -515,10 +516,12 @@ cudaError_t apply_tc_dispatch(int64_t T, int64_t C, const void* x, const float* 
   const uint64_t sx[2] = {(uint64_t)C * 2, (uint64_t)N * C * 2};
   const uint32_t bx[3] = {CS, 1, TT};
   const int S = (int)((C + CS - 1) / CS);
-  const bool paired = (S % 2 == 0) && num_sms >= 2;
-  // paired CTAs read both halves of each 128-byte row: fetch it whole
-  const CUtensorMapL2promotion promo =
-      paired ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B : CU_TENSOR_MAP_L2_PROMOTION_L2_64B;
+  int group = 1;
+  for (int gsz : {2})
+    if (S % gsz == 0 && num_sms >= gsz && group == 1) group = gsz;
+  const CUtensorMapL2promotion promo = group == 4   ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+                                       : group == 2 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
+                                                    : CU_TENSOR_MAP_L2_PROMOTION_L2_64B;
   e = make_tmap_bf16(&mx, x, 3, dx, sx, bx, CU_TENSOR_MAP_SWIZZLE_64B, promo);
   if (e != cudaSuccess) return e;
   e = make_tmap_bf16(&mG, G, 3, dx, sx, bx, CU_TENSOR_MAP_SWIZZLE_64B, promo);
@@ -539,14 +542,14 @@ cudaError_t apply_tc_dispatch(int64_t T, int64_t C, const void* x, const float* 
   a.C = C;
   a.S = S;
   a.NTT = (int)((T + TT - 1) / TT);
-  a.paired = paired ? 1 : 0;
-  const int vslices = paired ? S / 2 : S;
+  a.group = group;
+  const int vslices = S / group;
   a.items = (int64_t)vslices * a.NTT;
-  // at most one CTA (pair) per virtual slice, so every slice meets at most two CTAs
-  const int slots_max = paired ? num_sms / 2 : num_sms;
+  // at most one CTA group per virtual slice, so every slice meets at most two CTAs
+  const int slots_max = num_sms / group;
   const int slots = vslices < slots_max ? vslices : slots_max;
   a.per = (a.items + slots - 1) / slots;
-  const int grid = paired ? 2 * slots : slots;
+  const int grid = group * slots;
   a.phi = phi;
   a.hrec = hrec;
   a.part = part;
