@@ -253,7 +253,7 @@ def main():
     import torch.distributed as dist
 
     import manifold_constrained_hyper_token_b200 as mhc
-    from manifold_constrained_hyper_token_b200 import synth
+    from manifold_constrained_hyper_token_b200 import parallel, synth
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -276,8 +276,7 @@ def main():
     x_next = torch.empty_like(x)
     gx = torch.empty_like(x)
     gf = torch.empty_like(f_out)
-    pgrads = torch.empty(K * M + M + 1, dtype=torch.float32, device=dev)  # one all-reduce buffer
-    gphi, gb, ga = pgrads[:K * M].view(K, M), pgrads[K * M:K * M + M], pgrads[K * M + M:]
+    pgrads, gphi, gb, ga = parallel.param_grad_buffer(n, C, dev)  # one all-reduce buffer
     ws = torch.empty(mhc.mhc_backward_workspace_size(n, T, C, torch.bfloat16), dtype=torch.uint8,
                      device=dev)
     stream = torch.cuda.current_stream()
@@ -301,7 +300,7 @@ def main():
         if evs is not None:
             evs[4].record(stream)
         if world > 1:
-            dist.all_reduce(pgrads)
+            parallel.allreduce_param_grads(pgrads)
 
     for _ in range(args.warmup):
         step()
@@ -329,10 +328,7 @@ def main():
         for i, c in enumerate(calls):
             per_call[c] += evs[s][i].elapsed_time(evs[s][i + 1])
     per_call = {c: v / args.steps for c, v in per_call.items()}
-    if world > 1:
-        tt = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(tt.item())
+    elapsed_ms = parallel.max_over_ranks(elapsed_ms, dev)
     ms_per_step = elapsed_ms / args.steps
     tokens_per_s = T * world / (ms_per_step / 1000.0)
 
@@ -376,11 +372,7 @@ def main():
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e_ms = e0.elapsed_time(e1) / args.e2e_steps
-        if world > 1:
-            tt = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt.item())
+        e_ms = parallel.max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dev)
         e2e = {"value": T * world / (e_ms / 1000.0), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
                "ms_per_step": e_ms}
