@@ -32,11 +32,11 @@ cudaError_t map_tc_dispatch(bool bwd, int64_t T, int64_t C, int iters, float eps
                             cudaStream_t s);
 size_t map_tc_phi_bytes(int64_t C);
 // k_apply_tc.cu (bf16, n = 4: phi u and grad_phi on the tensor cores)
-cudaError_t apply_tc_dispatch(int64_t T, int64_t C, const void* x, const float* phi, const void* G,
-                              const void* g, const void* urec, const float* hrec, const float* part,
-                              int nparts, void* gx, void* gf, float* gphi, float* gb, float* ga,
-                              void* scratch, int* st, cudaStream_t s);
-size_t apply_tc_scratch_bytes(int64_t C);
+cudaError_t apply_tc_dispatch(int64_t T, int64_t C, const void* x, const void* phi_split,
+                              const void* G, const void* g, const void* urec, const float* hrec,
+                              const float* part, int nparts, void* gx, void* gf, float* gphi,
+                              float* gb, float* ga, void* scratch, int* st, cudaStream_t s);
+size_t apply_tc_scratch_bytes(int64_t T, int64_t C);
 // k_bwd.cu
 cudaError_t apply_dispatch(int n, int dtype, int64_t T, int64_t C, const void* x, const float* phi,
                            const void* G, const void* g, const float* coef, const float* part,
@@ -115,7 +115,7 @@ BwdWorkspace bwd_layout(const mhc_params* p) {
   w.phi_off = off;
   off = round_up(off + (tc ? mhc::map_tc_phi_bytes(p->C) : 0), 256);
   w.apply_off = off;
-  off = round_up(off + (tc ? mhc::apply_tc_scratch_bytes(p->C) : 0), 256);
+  off = round_up(off + (tc ? mhc::apply_tc_scratch_bytes(p->T, p->C) : 0), 256);
   w.total = off;
   return w;
 }
@@ -235,7 +235,7 @@ mhc_status mhc_backward_apply(const mhc_params* p, const void* x, const float* p
   if (st != MHC_OK) return st;
   const char* ws = (const char*)workspace;
   if (use_tc(p))
-    return from_cuda(mhc::apply_tc_dispatch(p->T, p->C, x, phi, grad_x_next, grad_h_in,
+    return from_cuda(mhc::apply_tc_dispatch(p->T, p->C, x, ws + w.phi_off, grad_x_next, grad_h_in,
                                             ws + w.urec_off, (const float*)(ws + w.hrec_off),
                                             (const float*)(ws + w.part_off), w.nparts, grad_x,
                                             grad_f_out, grad_phi, grad_b, grad_alpha,
