@@ -420,88 +420,92 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
       const int s = i % NS, d = i & 1;
       const uint32_t sph = (uint32_t)(i / NS) & 1u, dph = (uint32_t)(i >> 1) & 1u;
       bool live = !*abort_flag;
-      if (live && (!tc::mbar_wait(bar(B_FULL + s), sph, abort_flag, WAIT_NS) ||
-                   !tc::mbar_wait(bar(B_D1READY + d), dph, abort_flag, WAIT_NS))) {
+      if (live && !tc::mbar_wait(bar(B_FULL + s), sph, abort_flag, WAIT_NS)) {
         give_up();
         live = false;
       }
-      live = __all_sync(0xffffffffu, live);  // TMEM loads below are warp-collective
-      tc::tc_fence_after();
       const int slice = cur.slice(a, b);
       uint8_t* st = smem + s * STAGE;
-      // this token's H record
-      float hres[N * N], hpre[N], hpost[N], kap;
+      const int chunk = hq;  // 16-byte chunk of the 32-byte tile row
+      // Everything but phi u comes from the stage: compute it while the MMA for
+      // this item may still run, then add phi u from TMEM at the end.
+      uint64_t acc[N][4];
       {
-        const float4* hr = reinterpret_cast<const float4*>(st + H_OFF + tok * TcRec::H_BYTES);
-        float rec[TcRec::H_FLOATS];
+        uint64_t hres2[N * N], hpre2[N], hpost2[N], nkap2;
+        {
+          const float4* hr = reinterpret_cast<const float4*>(st + H_OFF + tok * TcRec::H_BYTES);
+          float rec[TcRec::H_FLOATS];
 #pragma unroll
-        for (int e = 0; e < TcRec::H_FLOATS / 4; ++e) {
-          const float4 v = hr[e];
-          rec[4 * e] = v.x; rec[4 * e + 1] = v.y; rec[4 * e + 2] = v.z; rec[4 * e + 3] = v.w;
+          for (int e = 0; e < TcRec::H_FLOATS / 4; ++e) {
+            const float4 v = hr[e];
+            rec[4 * e] = v.x; rec[4 * e + 1] = v.y; rec[4 * e + 2] = v.z; rec[4 * e + 3] = v.w;
+          }
+#pragma unroll
+          for (int e = 0; e < N * N; ++e)
+            hres2[e] = f2pack(rec[TcRec::H_RES + e], rec[TcRec::H_RES + e]);
+#pragma unroll
+          for (int e = 0; e < N; ++e) {
+            hpre2[e] = f2pack(rec[TcRec::H_PRE + e], rec[TcRec::H_PRE + e]);
+            hpost2[e] = f2pack(rec[TcRec::H_POST + e], rec[TcRec::H_POST + e]);
+          }
+          nkap2 = f2pack(-rec[TcRec::H_KAPPA], -rec[TcRec::H_KAPPA]);
         }
+        uint64_t Gp[N][4], gp[4];
 #pragma unroll
-        for (int e = 0; e < N * N; ++e) hres[e] = rec[TcRec::H_RES + e];
+        for (int i2 = 0; i2 < N; ++i2)
+          unpack_pairs(*reinterpret_cast<const uint4*>(st + G_OFF + i2 * XB + sw32(tok, chunk)), Gp[i2]);
+        unpack_pairs(*reinterpret_cast<const uint4*>(st + GG_OFF + sw32(tok, chunk)), gp);
+        // grad_f_out = sum_i H_post[i] G_i; it replaces this thread's grad_h_in
+        // piece in the stage (same swizzled position) for the tile store
+        {
+          uint32_t w[4];
 #pragma unroll
-        for (int e = 0; e < N; ++e) {
-          hpre[e] = rec[TcRec::H_PRE + e];
-          hpost[e] = rec[TcRec::H_POST + e];
+          for (int pr = 0; pr < 4; ++pr) {
+            uint64_t f = f2pack(0.0f, 0.0f);
+#pragma unroll
+            for (int i2 = 0; i2 < N; ++i2) f = f2fma(hpost2[i2], Gp[i2][pr], f);
+            w[pr] = f2_to_bf2(f);
+          }
+          *reinterpret_cast<uint4*>(st + GG_OFF + sw32(tok, chunk)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        kap = rec[TcRec::H_KAPPA];
+        // grad_x_j without phi u: H_pre[j] g + sum_i H_res[i][j] G_i - kappa x_j
+#pragma unroll
+        for (int jj = 0; jj < N; ++jj) {
+          uint64_t xp[4];
+          unpack_pairs(*reinterpret_cast<const uint4*>(st + X_OFF + jj * XB + sw32(tok, chunk)), xp);
+#pragma unroll
+          for (int pr = 0; pr < 4; ++pr) {
+            uint64_t v = f2fma(hpre2[jj], gp[pr], f2pack(0.0f, 0.0f));
+#pragma unroll
+            for (int i2 = 0; i2 < N; ++i2) v = f2fma(hres2[i2 * N + jj], Gp[i2][pr], v);
+            acc[jj][pr] = f2fma(nkap2, xp[pr], v);
+          }
+        }
       }
+      if (live && !tc::mbar_wait(bar(B_D1READY + d), dph, abort_flag, WAIT_NS)) {
+        give_up();
+        live = false;
+      }
+      live = __all_sync(0xffffffffu, live);  // the TMEM loads below are warp-collective
+      tc::tc_fence_after();
       {
-        const int chunk = hq;  // 16-byte chunk of the 32-byte tile row
-        // phi u of the four output streams for these 8 channels: four TMEM loads,
-        // one wait (warp-collective: every lane takes part, whatever its token)
+        // phi u of the four output streams for these 8 channels
         float d1[N][8];
         if (live) {
 #pragma unroll
           for (int jj = 0; jj < N; ++jj)
             tc::tmem_ld8(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(d * KR + jj * CS + 8 * chunk),
                          d1[jj]);
+          tc::tmem_ld_wait();
         }
-        // the token's coefficients as broadcast pairs
-        uint64_t hres2[N * N], hpre2[N], hpost2[N];
-#pragma unroll
-        for (int e = 0; e < N * N; ++e) hres2[e] = f2pack(hres[e], hres[e]);
-#pragma unroll
-        for (int e = 0; e < N; ++e) {
-          hpre2[e] = f2pack(hpre[e], hpre[e]);
-          hpost2[e] = f2pack(hpost[e], hpost[e]);
-        }
-        const uint64_t nkap2 = f2pack(-kap, -kap);
-        uint64_t Gp[N][4], gp[4];
-#pragma unroll
-        for (int i2 = 0; i2 < N; ++i2)
-          unpack_pairs(*reinterpret_cast<const uint4*>(st + G_OFF + i2 * XB + sw32(tok, chunk)), Gp[i2]);
-        unpack_pairs(*reinterpret_cast<const uint4*>(st + GG_OFF + sw32(tok, chunk)), gp);
-        if (live) tc::tmem_ld_wait();
-        // grad_f_out = sum_i H_post[i] G_i; it replaces this thread's grad_h_in piece
-        // in the stage (same swizzled position) for the tile store below
-        {
-          uint32_t w[4];
-#pragma unroll
-          for (int pr = 0; pr < 4; ++pr) {
-            uint64_t acc = f2pack(0.0f, 0.0f);
-#pragma unroll
-            for (int i2 = 0; i2 < N; ++i2) acc = f2fma(hpost2[i2], Gp[i2][pr], acc);
-            w[pr] = f2_to_bf2(acc);
-          }
-          *reinterpret_cast<uint4*>(st + GG_OFF + sw32(tok, chunk)) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        // grad_x_j = phi u + H_pre[j] g + sum_i H_res[i][j] G_i - kappa x_j; it
-        // replaces this thread's x piece of stream j
 #pragma unroll
         for (int jj = 0; jj < N; ++jj) {
-          uint64_t xp[4];
-          unpack_pairs(*reinterpret_cast<const uint4*>(st + X_OFF + jj * XB + sw32(tok, chunk)), xp);
           uint32_t w[4];
 #pragma unroll
           for (int pr = 0; pr < 4; ++pr) {
-            uint64_t acc = f2fma(hpre2[jj], gp[pr], f2pack(d1[jj][2 * pr], d1[jj][2 * pr + 1]));
-#pragma unroll
-            for (int i2 = 0; i2 < N; ++i2) acc = f2fma(hres2[i2 * N + jj], Gp[i2][pr], acc);
-            acc = f2fma(nkap2, xp[pr], acc);
-            w[pr] = f2_to_bf2(acc);
+            float lo, hi;
+            asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(acc[jj][pr]));
+            w[pr] = pack2(lo + d1[jj][2 * pr], hi + d1[jj][2 * pr + 1]);
           }
           *reinterpret_cast<uint4*>(st + X_OFF + jj * XB + sw32(tok, chunk)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
