@@ -81,9 +81,9 @@ def kernel_source_sha(files):
 # kernels behind each single-kernel call, for matching ncu traffic to sources
 CALL_SOURCES = {
     "post": ["k_post.cu", "mhc_common.cuh"],
-    "bwd_map": ["k_map.cu", "mhc_common.cuh"],
-    "bwd_apply": ["k_bwd.cu", "mhc_common.cuh"],
-    "pre": ["k_map.cu", "k_post.cu", "mhc_common.cuh"],
+    "bwd_map": ["k_map_tc.cu", "tc_sm100.cuh", "mhc_common.cuh"],
+    "bwd_apply": ["k_apply_tc.cu", "tc_sm100.cuh", "mhc_common.cuh"],
+    "pre": ["k_map_tc.cu", "k_post.cu", "tc_sm100.cuh", "mhc_common.cuh"],
 }
 
 
