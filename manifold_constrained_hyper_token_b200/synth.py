@@ -98,6 +98,15 @@ def depth_gain(l: int) -> float:
     return float(0.5 + torch.rand(1, generator=g).item())
 
 
+def depth_stack_chunk(T: int, n: int, C: int, chunk: int,
+                      dtype: torch.dtype = torch.bfloat16) -> dict:
+    """One token chunk of the depth-stack workload: the stack input x_0 [T,n,C] and the
+    upstream gradient of the last layer's output G_L [T,n,C], both ~ N(0,1).  Chunk k
+    draws from its own seed, so any chunk can be regenerated alone."""
+    g = _gen(chunk + 6000)
+    return dict(x0=_normal((T, n, C), 1.0, g, dtype), G_last=_normal((T, n, C), 1.0, g, dtype))
+
+
 def token_sample(T: int, k: int, seed: int = 0) -> torch.Tensor:
     """Sorted random subset of k distinct token indices in [0, T) (always includes the
     first and last token)."""
