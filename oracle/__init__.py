@@ -52,11 +52,15 @@ def _load():
         lib.orc_post.argtypes = [i32, i64, i64, _D, _D, _D, _D, _D]
         lib.orc_backward.argtypes = [i32, i64, i64, i32, dbl, _D, _D, _D, dbl, _D, _D, _D,
                                      _D, _D, _D, _D, _D]
+        lib.orc_post_backward.argtypes = [i32, i64, i64, _D, _D, _D, _D, _D, _D]
+        lib.orc_pre_backward.argtypes = [i32, i64, i64, i32, dbl, _D, _D, _D, dbl, _D, _D, _D,
+                                         _D, _D, _D, _D]
         lib.orc_depth_amax.argtypes = [i32, i64, i32, _D, _D, _D]
         lib.orc_num_threads.restype = i32
         lib.orc_set_num_threads.argtypes = [i32]
         for f in ("orc_sinkhorn", "orc_sinkhorn_backward", "orc_pre", "orc_post", "orc_backward",
-                  "orc_depth_amax", "orc_set_num_threads"):
+                  "orc_post_backward", "orc_pre_backward", "orc_depth_amax",
+                  "orc_set_num_threads"):
             getattr(lib, f).restype = None
         _lib = lib
     return _lib
@@ -152,6 +156,48 @@ def backward(x, phi, b, alpha: float, f_out, grad_x_next, grad_h_in, iters: int 
         gx[t0:t1] = gxc
         gf[t0:t1] = gfc
     return dict(grad_x=gx, grad_phi=gphi, grad_b=gb, grad_alpha=float(ga[0]), grad_f_out=gf)
+
+
+def post_backward(x, f_out, H_post, grad_x_next):
+    """First half of the layer backward in training order: the reverse of the post
+    merge with the forward's H_post.  Returns dict(grad_f_out [T,C],
+    red [T, n*n + n] = (<G_i, x_j> row-major, then <G_i, f_out>))."""
+    xd = _f64(x)
+    T, n, C = xd.shape
+    fd, hp, Gd = _f64(f_out), _f64(H_post), _f64(grad_x_next)
+    gf = np.empty((T, C))
+    red = np.empty((T, n * n + n))
+    _load().orc_post_backward(n, T, C, _p(xd), _p(fd), _p(hp), _p(Gd), _p(gf), _p(red))
+    return dict(grad_f_out=gf, red=red)
+
+
+def pre_backward(x, phi, b, alpha: float, grad_x_next, grad_h_in, red, iters: int = 20,
+                 eps: float = 1e-6, chunk: int | None = None):
+    """Second half of the layer backward in training order: recompute the mapping and
+    take grad_h_in and the post half's reductions.  Returns dict(grad_x, grad_phi,
+    grad_b, grad_alpha)."""
+    T = x.shape[0]
+    n, C = x.shape[1], x.shape[2]
+    M = n * n + 2 * n
+    ph, bd = _f64(phi).reshape(n * C, M), _f64(b).reshape(M)
+    rd = _f64(red).reshape(T, n * n + n)
+    gphi = np.zeros((n * C, M))
+    gb = np.zeros(M)
+    ga = np.zeros(1)
+    gx = np.empty((T, n, C))
+    step = T if chunk is None else int(chunk)
+    lib = _load()
+    for t0 in range(0, T, step):
+        t1 = min(T, t0 + step)
+        xd = _f64(x[t0:t1])
+        Gd, gd = _f64(grad_x_next[t0:t1]), _f64(grad_h_in[t0:t1])
+        rc = np.ascontiguousarray(rd[t0:t1])
+        gxc = np.empty((t1 - t0, n, C))
+        lib.orc_pre_backward(n, t1 - t0, C, int(iters), float(eps), _p(xd), _p(ph), _p(bd),
+                             float(alpha), _p(Gd), _p(gd), _p(rc), _p(gxc), _p(gphi), _p(gb),
+                             _p(ga))
+        gx[t0:t1] = gxc
+    return dict(grad_x=gx, grad_phi=gphi, grad_b=gb, grad_alpha=float(ga[0]))
 
 
 def depth_amax(H) -> tuple[np.ndarray, np.ndarray]:

@@ -44,6 +44,14 @@
  *   x, grad_x_next (G), grad_x : [T][n][C]      f_out, grad_h_in (g), h_in : [T][C]
  *   phi, grad_phi : [n*C][n*n+2n]   b, grad_b : [n*n+2n]
  *   H_pre, H_post : [T][n]          H_res : [T][n][n]
+ *   red (the post half's reductions, backward in training order):
+ *                   [T][n*n + n] = <G_i, x_j> (row-major i, j) then <G_i, f_out>
+ *
+ * Parity pins (tests/test_oracle_pins.py): hand-worked and closed-form
+ * Sinkhorn cases, diagonal-scaling and permutation invariants, the gate and
+ * RMS special cases, the standard residual at n = 1, finite differences of
+ * every backward gradient (the whole backward and the post half), and the
+ * split backward against the one-call backward.
  */
 #include <math.h>
 #include <stdint.h>
@@ -205,13 +213,20 @@ void orc_post(int n, int64_t T, int64_t C, const double *x, const double *f_out,
  * with G = dL/dx_next, g = dL/dh_in given.  Hand-written reverse mode of the
  * program in orc_pre / orc_post.
  *
- * Per-token outputs grad_x [T][n][C] and grad_f_out [T][C] are written.
- * grad_phi, grad_b and grad_alpha are ADDED to (the caller zeroes them), token
- * by token in increasing t, so that a caller may run T in consecutive chunks. */
-void orc_backward(int n, int64_t T, int64_t C, int iters, double eps, const double *x,
-                  const double *phi, const double *b, double alpha, const double *f_out,
-                  const double *G, const double *g, double *grad_x, double *grad_phi,
-                  double *grad_b, double *grad_alpha, double *grad_f_out) {
+ * The derivatives of L with respect to the post merge's maps,
+ *   dH_res[i][j] = <G_i, x_j>,   dH_post[i] = <G_i, f_out>,
+ * are taken from `red` ([T][n*n + n]: dH_res then dH_post) when it is given,
+ * and computed from G and f_out otherwise.  grad_f_out is written when the
+ * pointer is non-null.
+ *
+ * Per-token output grad_x [T][n][C] is written.  grad_phi, grad_b and
+ * grad_alpha are ADDED to (the caller zeroes them), token by token in
+ * increasing t, so that a caller may run T in consecutive chunks. */
+static void backward_core(int n, int64_t T, int64_t C, int iters, double eps, const double *x,
+                          const double *phi, const double *b, double alpha, const double *f_out,
+                          const double *G, const double *g, const double *red, double *grad_x,
+                          double *grad_phi, double *grad_b, double *grad_alpha,
+                          double *grad_f_out) {
   const int M = n * n + 2 * n;
   const int nn = n * n;
   const int64_t K = (int64_t)n * C;
@@ -225,7 +240,6 @@ void orc_backward(int n, int64_t T, int64_t C, int iters, double eps, const doub
     const double *xt = x + t * K;
     const double *Gt = G + t * K;
     const double *gt = g + t * C;
-    const double *ft = f_out + t * C;
     double *gx = grad_x + t * K;
     double y[16 * 16 + 32], z[16 * 16 + 32], dz[16 * 16 + 32], r;
     double hpre[16], spre[16], spost[16], hpost[16];
@@ -243,19 +257,27 @@ void orc_backward(int n, int64_t T, int64_t C, int iters, double eps, const doub
     orc_sk_forward(n, iters, z + 2 * n, hres, iterates);
 
     /* post: x_next = H_res x + H_post^T f_out */
-    for (int64_t c = 0; c < C; ++c) {
-      double acc = 0.0;
-      for (int i = 0; i < n; ++i) acc += hpost[i] * Gt[i * C + c];
-      grad_f_out[t * C + c] = acc;
+    if (grad_f_out != NULL) {
+      for (int64_t c = 0; c < C; ++c) {
+        double acc = 0.0;
+        for (int i = 0; i < n; ++i) acc += hpost[i] * Gt[i * C + c];
+        grad_f_out[t * C + c] = acc;
+      }
     }
-    for (int i = 0; i < n; ++i) {
-      double acc = 0.0;
-      for (int64_t c = 0; c < C; ++c) acc += Gt[i * C + c] * ft[c];
-      dhpost[i] = acc;
-      for (int j = 0; j < n; ++j) {
-        double a2 = 0.0;
-        for (int64_t c = 0; c < C; ++c) a2 += Gt[i * C + c] * xt[j * C + c];
-        dhres[i * n + j] = a2;
+    if (red != NULL) {
+      for (int e = 0; e < nn; ++e) dhres[e] = red[t * (nn + n) + e];
+      for (int i = 0; i < n; ++i) dhpost[i] = red[t * (nn + n) + nn + i];
+    } else {
+      const double *ft = f_out + t * C;
+      for (int i = 0; i < n; ++i) {
+        double acc = 0.0;
+        for (int64_t c = 0; c < C; ++c) acc += Gt[i * C + c] * ft[c];
+        dhpost[i] = acc;
+        for (int j = 0; j < n; ++j) {
+          double a2 = 0.0;
+          for (int64_t c = 0; c < C; ++c) a2 += Gt[i * C + c] * xt[j * C + c];
+          dhres[i * n + j] = a2;
+        }
       }
     }
     /* pre: h_in = H_pre x */
@@ -320,6 +342,59 @@ void orc_backward(int n, int64_t T, int64_t C, int iters, double eps, const doub
   free(dz_all);
   free(y_all);
   free(r_all);
+}
+
+/* The whole layer backward in one call (grad_h_in given together with
+ * grad_x_next): grad_x, grad_f_out and the parameter sums. */
+void orc_backward(int n, int64_t T, int64_t C, int iters, double eps, const double *x,
+                  const double *phi, const double *b, double alpha, const double *f_out,
+                  const double *G, const double *g, double *grad_x, double *grad_phi,
+                  double *grad_b, double *grad_alpha, double *grad_f_out) {
+  backward_core(n, T, C, iters, eps, x, phi, b, alpha, f_out, G, g, NULL, grad_x, grad_phi, grad_b,
+                grad_alpha, grad_f_out);
+}
+
+/* First half of the layer backward in training order [P5 [20]-[21]]: the
+ * reverse of the post merge x_next = H_res x + H_post^T f_out alone, with the
+ * forward's H_post given.  Writes
+ *   grad_f_out[c] = sum_i H_post[i] G_i[c]
+ *   red = [ dH_res[i][j] = <G_i, x_j>  (n*n) | dH_post[i] = <G_i, f_out>  (n) ]
+ * per token; red is what the second half needs from grad_x_next besides G. */
+void orc_post_backward(int n, int64_t T, int64_t C, const double *x, const double *f_out,
+                       const double *H_post, const double *G, double *grad_f_out, double *red) {
+  const int nn = n * n;
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; ++t) {
+    const double *xt = x + t * n * C;
+    const double *Gt = G + t * n * C;
+    const double *ft = f_out + t * C;
+    for (int64_t c = 0; c < C; ++c) {
+      double acc = 0.0;
+      for (int i = 0; i < n; ++i) acc += H_post[t * n + i] * Gt[i * C + c];
+      grad_f_out[t * C + c] = acc;
+    }
+    for (int i = 0; i < n; ++i) {
+      for (int j = 0; j < n; ++j) {
+        double acc = 0.0;
+        for (int64_t c = 0; c < C; ++c) acc += Gt[i * C + c] * xt[j * C + c];
+        red[t * (nn + n) + i * n + j] = acc;
+      }
+      double acc = 0.0;
+      for (int64_t c = 0; c < C; ++c) acc += Gt[i * C + c] * ft[c];
+      red[t * (nn + n) + nn + i] = acc;
+    }
+  }
+}
+
+/* Second half of the layer backward in training order: given grad_h_in (from
+ * F's backward), grad_x_next and the post half's reductions, recompute the
+ * mapping and write grad_x plus the parameter sums (added to, as above). */
+void orc_pre_backward(int n, int64_t T, int64_t C, int iters, double eps, const double *x,
+                      const double *phi, const double *b, double alpha, const double *G,
+                      const double *g, const double *red, double *grad_x, double *grad_phi,
+                      double *grad_b, double *grad_alpha) {
+  backward_core(n, T, C, iters, eps, x, phi, b, alpha, NULL, G, g, red, grad_x, grad_phi, grad_b,
+                grad_alpha, NULL);
 }
 
 /* Composite residual map over depth and its Amax gain [P1 "Warum

@@ -330,3 +330,60 @@ def test_backward_parameter_sums_are_token_additive(oracle_mod):
     for k in ("grad_phi", "grad_b"):
         np.testing.assert_allclose(a[k], bch[k], rtol=1e-14, atol=1e-14)
     np.testing.assert_array_equal(a["grad_x"], bch["grad_x"])
+
+
+# ------------------------------------- the backward in training order (split)
+@pytest.mark.parametrize("n", [1, 2, 4])
+def test_post_backward_finite_differences(oracle_mod, n):
+    """The post half against central differences of L = sum G . post(x, f, H_post, H_res):
+    grad_f_out = dL/df_out, red = (dL/dH_res row-major, dL/dH_post).  post is linear
+    in each argument, so the differences are exact up to rounding."""
+    T, C = 3, 5
+    rng = _rng(120 + n)
+    x = rng.normal(size=(T, n, C))
+    f = rng.normal(size=(T, C))
+    hp = rng.uniform(0, 2, size=(T, n))
+    hr = rng.uniform(0, 1, size=(T, n, n))
+    G = rng.normal(size=(T, n, C))
+    got = oracle_mod.post_backward(x, f, hp, G)
+    h = 1e-6
+
+    def L(f_=f, hp_=hp, hr_=hr):
+        return float(np.sum(G * oracle_mod.post(x, f_, hp_, hr_)))
+
+    def fd(arr, which):
+        out = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            ap, am = arr.copy(), arr.copy()
+            ap[idx] += h
+            am[idx] -= h
+            out[idx] = (L(**{which: ap}) - L(**{which: am})) / (2 * h)
+        return out
+
+    np.testing.assert_allclose(got["grad_f_out"], fd(f, "f_"), rtol=0, atol=1e-8)
+    red = got["red"].reshape(T, n * n + n)
+    np.testing.assert_allclose(red[:, :n * n].reshape(T, n, n), fd(hr, "hr_"), rtol=0, atol=1e-8)
+    np.testing.assert_allclose(red[:, n * n:], fd(hp, "hp_"), rtol=0, atol=1e-8)
+
+
+@pytest.mark.parametrize("n", [1, 2, 4])
+def test_split_backward_equals_whole(oracle_mod, n):
+    """post half -> pre half (with grad_h_in given) reproduces the one-call backward,
+    whose every gradient is pinned by finite differences above."""
+    T, C = 4, 6
+    M = n * n + 2 * n
+    rng = _rng(130 + n)
+    x = rng.normal(size=(T, n, C))
+    phi = rng.normal(0, 0.3, size=(n * C, M))
+    b = rng.normal(size=M)
+    f = rng.normal(size=(T, C))
+    G = rng.normal(size=(T, n, C))
+    g = rng.normal(size=(T, C))
+    whole = oracle_mod.backward(x, phi, b, 0.7, f, G, g, iters=20)
+    fwd = oracle_mod.pre(x, phi, b, 0.7, iters=20)
+    pb = oracle_mod.post_backward(x, f, fwd["H_post"], G)
+    qb = oracle_mod.pre_backward(x, phi, b, 0.7, G, g, pb["red"], iters=20)
+    np.testing.assert_allclose(pb["grad_f_out"], whole["grad_f_out"], rtol=1e-13, atol=1e-13)
+    for k in ("grad_x", "grad_phi", "grad_b"):
+        np.testing.assert_allclose(qb[k], whole[k], rtol=1e-12, atol=1e-12, err_msg=k)
+    assert qb["grad_alpha"] == pytest.approx(whole["grad_alpha"], rel=1e-12, abs=1e-12)
