@@ -4,7 +4,11 @@
 A step is one pass of the whole hot path over one batch of synthetic tokens:
   mhc_pre -> mhc_post (with a supplied f_out standing in for F's output) ->
   mhc_backward_map -> mhc_backward_apply
-at T = 16384 tokens per GPU, n = 4 streams, C = 7168 channels, bf16
+``--forward fused`` times one layer of a deep stack in steady state instead:
+  mhc_layer_input -> mhc_post_fused (x_next and the next layer's maps) ->
+  mhc_backward_map -> mhc_backward_apply
+(the layer's own maps then come from one mhc_pre before timing).  Both run at
+T = 16384 tokens per GPU, n = 4 streams, C = 7168 channels, bf16
 activations, Sinkhorn t_max = 20.  Under torchrun each rank runs its own
 16384 tokens (data parallel over tokens, weak scaling) and the step ends with
 the one exchange the backward has: an all-reduce of grad_phi / grad_b /
@@ -48,6 +52,8 @@ def per_token_bytes(n=N_STR, C=C_CH, act=2):
     return {
         "pre": nC * act + C * act + 4 * (2 * n + n * n),                  # x in; h_in, H out
         "post": nC * act + C * act + 4 * (n + n * n) + nC * act,           # x, f, H in; x_next out
+        "layer_input": nC * act + C * act + 4 * n,                         # x, H_pre in; h_in out
+        "post_fused": nC * act + C * act + 4 * (n + n * n) + nC * act + 4 * (2 * n + n * n),
         "bwd_map": 2 * nC * act + 2 * C * act + coef,                      # x, G, g, f in; records out
         "bwd_apply": 2 * nC * act + C * act + coef + nC * act + C * act,   # x, G, g, records in; grads out
         "bwd_min": 2 * nC * act + 2 * C * act + nC * act + C * act,        # one pass: x, G, g, f in; grads out
@@ -57,7 +63,8 @@ def per_token_bytes(n=N_STR, C=C_CH, act=2):
 def per_call_param_bytes(n=N_STR, C=C_CH):
     K, M = n * C, n * n + 2 * n
     phi = K * M * 4
-    return {"pre": phi, "post": 0, "bwd_map": phi, "bwd_apply": 2 * phi}
+    return {"pre": phi, "post": 0, "layer_input": 0, "post_fused": phi, "bwd_map": phi,
+            "bwd_apply": 2 * phi}
 
 
 def load_peaks():
@@ -84,6 +91,8 @@ CALL_SOURCES = {
     "bwd_map": ["k_map_tc.cu", "tc_sm100.cuh", "mhc_common.cuh"],
     "bwd_apply": ["k_apply_tc.cu", "tc_sm100.cuh", "mhc_common.cuh"],
     "pre": ["k_map_tc.cu", "k_post.cu", "tc_sm100.cuh", "mhc_common.cuh"],
+    "layer_input": ["k_post.cu", "mhc_common.cuh"],
+    "post_fused": ["k_map_tc.cu", "tc_sm100.cuh", "mhc_common.cuh"],
 }
 
 
@@ -237,6 +246,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--tokens", type=int, default=T_TOK,
                     help="tokens per GPU (default 16384; smaller values for profiler captures)")
+    ap.add_argument("--forward", default="unfused", choices=["fused", "unfused"],
+                    help="fused: layer input + post merge fused with the next layer's mapping; "
+                         "unfused: mhc_pre + mhc_post")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -280,16 +292,31 @@ def main():
     ws = torch.empty(mhc.mhc_backward_workspace_size(n, T, C, torch.bfloat16), dtype=torch.uint8,
                      device=dev)
     stream = torch.cuda.current_stream()
-    calls = ["pre", "post", "bwd_map", "bwd_apply"]
-    launches_per_call = {"pre": 2, "post": 1, "bwd_map": 1, "bwd_apply": 1}
+    fused = args.forward == "fused"
+    calls = (["layer_input", "post_fused"] if fused else ["pre", "post"]) + ["bwd_map", "bwd_apply"]
+    launches_per_call = {"pre": 2, "post": 1, "layer_input": 1, "post_fused": 2, "bwd_map": 1,
+                         "bwd_apply": 1}
+    # the layer's maps; in a stack the previous layer's post_fused computes them
+    mhc.mhc_pre(x, phi, b, alpha, t_max=T_MAX, out=(h_in, Hpre, Hpost, Hres), stream=stream)
+    nxt = (torch.empty_like(Hpre), torch.empty_like(Hpost), torch.empty_like(Hres))
+    pre_ws = torch.empty(max(1, mhc.mhc_pre_workspace_size(n, T, C, torch.bfloat16)),
+                         dtype=torch.uint8, device=dev)
 
     def step(evs=None):
         if evs is not None:
             evs[0].record(stream)
-        mhc.mhc_pre(x, phi, b, alpha, t_max=T_MAX, out=(h_in, Hpre, Hpost, Hres), stream=stream)
+        if fused:
+            mhc.mhc_layer_input(x, Hpre, out=h_in, stream=stream)
+        else:
+            mhc.mhc_pre(x, phi, b, alpha, t_max=T_MAX, out=(h_in, Hpre, Hpost, Hres),
+                        workspace=pre_ws, stream=stream)
         if evs is not None:
             evs[1].record(stream)
-        mhc.mhc_post(x, f_out, Hpost, Hres, out=x_next, stream=stream)
+        if fused:
+            mhc.mhc_post_fused(x, f_out, Hpost, Hres, phi, b, alpha, t_max=T_MAX,
+                               out=(x_next,) + nxt, workspace=pre_ws, stream=stream)
+        else:
+            mhc.mhc_post(x, f_out, Hpost, Hres, out=x_next, stream=stream)
         if evs is not None:
             evs[2].record(stream)
         mhc.mhc_backward_map(x, phi, b, alpha, f_out, G, g, ws, t_max=T_MAX, stream=stream)
@@ -341,7 +368,9 @@ def main():
     dom = max(single, key=lambda c: per_call[c])
     achieved = call_bytes[dom] / (per_call[dom] / 1000.0) / 1e9
     traffic = ncu_traffic(dom)
-    step_alg_bytes = T * (tb["pre"] + tb["post"] + tb["bwd_min"]) + pb["pre"] + pb["bwd_apply"]
+    fwd_calls = calls[:2]
+    step_alg_bytes = (T * (sum(tb[c] for c in fwd_calls) + tb["bwd_min"]) +
+                      sum(pb[c] for c in fwd_calls) + pb["bwd_apply"])
     step_gbs = step_alg_bytes / (ms_per_step / 1000.0) / 1e9
 
     # ---- end to end through the public API with host buffers
@@ -388,7 +417,11 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
             "config": {"workload": f"mHC layer fwd+bwd per GPU: T={T} tokens, n={n}, C={C}, "
-                                   f"t_max={T_MAX}, bf16 activations, fp32 maps",
+                                   f"t_max={T_MAX}, bf16 activations, fp32 maps; " +
+                                   ("one layer of a stack: layer input, post merge fused with "
+                                    "the next layer's mapping, backward" if fused else
+                                    "pre, post, backward (no cross-layer fusion)"),
+                       "forward": args.forward,
                        "T_per_gpu": T, "n": n, "C": C, "t_max": T_MAX,
                        "parallelism": f"dp{world} over tokens",
                        "l2": "inputs larger than L2 (x and grad_x_next are 940 MB each); no flush"},

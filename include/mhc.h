@@ -198,6 +198,80 @@ MHC_API mhc_status mhc_backward_apply(const mhc_params *p, const void *x, const 
                                       mhc_stream_t stream);
 
 /*
+ * Cross-layer fusion of the forward (sources: reportify.cn [18], the unified
+ * operator, and [20], the output map applied together with the residual
+ * merge).  In a stack, layer l's post merge writes x_{l+1}, which layer l+1's
+ * mapping reads back at once; mhc_post_fused does both in one pass over the
+ * stream buffer, so the forward of a layer costs one read of x for h_in and
+ * one pass for the merge:
+ *
+ *   mhc_post_fused(x_l, f_out_l, H_post_l, H_res_l, phi_{l+1}, b_{l+1}, alpha_{l+1})
+ *       -> x_{l+1}, H_pre_{l+1}, H_post_{l+1}, H_res_{l+1}
+ *   mhc_layer_input(x_{l+1}, H_pre_{l+1}) -> h_in_{l+1}
+ *
+ * mhc_post_fused -- x_next exactly as mhc_post writes it, and layer l+1's maps
+ *   exactly as mhc_pre would compute them from that x_next (the mapping reads
+ *   the stored, dtype-rounded x_next).  p->t_max and p->eps are layer l+1's.
+ *   phi_next [nC][n^2+2n], b_next, alpha_next as in mhc_pre.  workspace:
+ *   mhc_post_fused_workspace_size(p) bytes (may be NULL when that is 0).
+ *   x_next must not alias x or f_out.
+ * mhc_layer_input -- h_in [T][C] = sum_i H_pre[i] x[i][:] alone (the second
+ *   half of mhc_pre).
+ * Errors: as mhc_pre.
+ */
+MHC_API size_t mhc_post_fused_workspace_size(const mhc_params *p);
+MHC_API mhc_status mhc_post_fused(const mhc_params *p, const void *x, const void *f_out,
+                                  const float *H_post, const float *H_res, const float *phi_next,
+                                  const float *b_next, const float *alpha_next, void *x_next,
+                                  float *H_pre_next, float *H_post_next, float *H_res_next,
+                                  void *workspace, size_t workspace_bytes, int *dev_status,
+                                  mhc_stream_t stream);
+MHC_API mhc_status mhc_layer_input(const mhc_params *p, const void *x, const float *H_pre,
+                                   void *h_in, int *dev_status, mhc_stream_t stream);
+
+/*
+ * The layer backward in training order, split around F's backward (sources:
+ * the recompute bullet of the "Systemarbeit" section; reportify.cn [20]-[21]).
+ * In training, grad_h_in is only known after F's backward, which needs
+ * grad_f_out first:
+ *
+ *   mhc_post_backward(x, f_out, H_post, grad_x_next) -> grad_f_out, red
+ *   F's backward (caller)                            -> grad_h_in
+ *   mhc_pre_backward(x, phi, b, alpha, grad_x_next, grad_h_in, red)
+ *                                                    -> grad_x, grad_phi, grad_b, grad_alpha
+ *
+ * Together they give exactly what mhc_backward gives for the same
+ * (grad_x_next, grad_h_in).
+ *
+ * mhc_post_backward -- the reverse of the post merge alone, with the
+ *   forward's H_post [T][n] (float32, as mhc_pre wrote it):
+ *     grad_f_out[c] = sum_i H_post[i] grad_x_next[i][c]        [T][C] (dtype)
+ *     red = [ <grad_x_next_i, x_j> (row-major i, j) | <grad_x_next_i, f_out> ]
+ *                                                    [T][n*n + n] float32
+ *   red carries the derivatives of L with respect to H_res and H_post; the
+ *   per-token sums are taken in a fixed order.  grad_f_out must not alias an
+ *   input.  No workspace.
+ * mhc_pre_backward -- recomputes the mapping from (x, phi, b, alpha), takes
+ *   <grad_h_in, x_i> itself and the rest of the mapping's upstream gradient
+ *   from red, and writes grad_x [T][n][C] (dtype) and OVERWRITES grad_phi,
+ *   grad_b, grad_alpha (float32, fixed-order sums over the T tokens).
+ *   workspace: at least mhc_pre_backward_workspace_size(p) bytes, 256-byte
+ *   aligned; its contents on entry do not matter.
+ * Errors: as mhc_backward (red must be 16-byte aligned like every pointer).
+ */
+MHC_API mhc_status mhc_post_backward(const mhc_params *p, const void *x, const void *f_out,
+                                     const float *H_post, const void *grad_x_next,
+                                     void *grad_f_out, float *red, int *dev_status,
+                                     mhc_stream_t stream);
+MHC_API size_t mhc_pre_backward_workspace_size(const mhc_params *p);
+MHC_API mhc_status mhc_pre_backward(const mhc_params *p, const void *x, const float *phi,
+                                    const float *b, const float *alpha, const void *grad_x_next,
+                                    const void *grad_h_in, const float *red, void *grad_x,
+                                    float *grad_phi, float *grad_b, float *grad_alpha,
+                                    void *workspace, size_t workspace_bytes, int *dev_status,
+                                    mhc_stream_t stream);
+
+/*
  * mhc_backward_noalloc -- mhc_backward for callers that cannot allocate
  * device memory where they run the backward: runtimes that plan every device
  * buffer at start-up and forbid allocation afterwards, plugins that a host

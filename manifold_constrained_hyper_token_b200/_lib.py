@@ -11,7 +11,9 @@ LIB_PATH = os.path.join(_PKG, "libmhc.so")
 # mhc.h symbols this binding requires
 SYMBOLS = ("mhc_version", "mhc_status_string", "mhc_pre_workspace_size", "mhc_pre", "mhc_post",
            "mhc_backward_workspace_size", "mhc_backward", "mhc_backward_map", "mhc_backward_apply",
-           "mhc_backward_noalloc", "mhc_sinkhorn_knopp", "mhc_depth_amax")
+           "mhc_backward_noalloc", "mhc_post_backward", "mhc_pre_backward_workspace_size",
+           "mhc_pre_backward", "mhc_post_fused_workspace_size", "mhc_post_fused",
+           "mhc_layer_input", "mhc_sinkhorn_knopp", "mhc_depth_amax")
 
 
 class MhcParams(ctypes.Structure):
@@ -53,6 +55,19 @@ def load() -> ctypes.CDLL:
     lib.mhc_backward_apply.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
     lib.mhc_backward_noalloc.restype = i32
     lib.mhc_backward_noalloc.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.mhc_post_backward.restype = i32
+    lib.mhc_post_backward.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.mhc_pre_backward_workspace_size.restype = sz
+    lib.mhc_pre_backward_workspace_size.argtypes = [pp]
+    lib.mhc_pre_backward.restype = i32
+    lib.mhc_pre_backward.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
+                                     vp]
+    lib.mhc_post_fused_workspace_size.restype = sz
+    lib.mhc_post_fused_workspace_size.argtypes = [pp]
+    lib.mhc_post_fused.restype = i32
+    lib.mhc_post_fused.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
+    lib.mhc_layer_input.restype = i32
+    lib.mhc_layer_input.argtypes = [pp, vp, vp, vp, vp, vp]
     lib.mhc_sinkhorn_knopp.restype = i32
     lib.mhc_sinkhorn_knopp.argtypes = [i32, i32, i64, vp, vp, vp, vp]
     lib.mhc_depth_amax.restype = i32

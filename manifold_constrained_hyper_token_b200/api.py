@@ -152,6 +152,74 @@ def mhc_backward_noalloc(x, phi, b, alpha, f_out, grad_x_next, grad_h_in, *, t_m
     return gx, gphi, gb, ga, gf
 
 
+def mhc_post_fused(x, f_out, H_post, H_res, phi_next, b_next, alpha_next, *, t_max: int = 20,
+                   eps: float = 1e-6, out=None, workspace=None, dev_status=None, stream=None):
+    """Layer l's post merge fused with layer l+1's mapping.
+    Returns (x_next [T,n,C], H_pre_next [T,n], H_post_next [T,n], H_res_next [T,n,n])."""
+    T, n, C = x.shape
+    p = params(n, T, C, x.dtype, t_max, eps)
+    if out is None:
+        out = (torch.empty_like(x), torch.empty(T, n, dtype=torch.float32, device=x.device),
+               torch.empty(T, n, dtype=torch.float32, device=x.device),
+               torch.empty(T, n, n, dtype=torch.float32, device=x.device))
+    xn, hpre, hpost, hres = out
+    lib = _lib.load()
+    ws, wsb = _workspace(int(lib.mhc_post_fused_workspace_size(ctypes.byref(p))), x.device,
+                         workspace)
+    st = lib.mhc_post_fused(ctypes.byref(p), _p(x), _p(f_out), _p(H_post), _p(H_res),
+                            _p(phi_next), _p(b_next), _p(alpha_next), _p(xn), _p(hpre),
+                            _p(hpost), _p(hres), _p(ws), wsb, _p(dev_status), _stream(stream))
+    _check(st, "mhc_post_fused")
+    return xn, hpre, hpost, hres
+
+
+def mhc_layer_input(x, H_pre, *, out=None, dev_status=None, stream=None):
+    """h_in [T,C] = sum_i H_pre[i] x[i] (the second half of mhc_pre)."""
+    T, n, C = x.shape
+    p = params(n, T, C, x.dtype)
+    h_in = torch.empty(T, C, dtype=x.dtype, device=x.device) if out is None else out
+    st = _lib.load().mhc_layer_input(ctypes.byref(p), _p(x), _p(H_pre), _p(h_in),
+                                     _p(dev_status), _stream(stream))
+    _check(st, "mhc_layer_input")
+    return h_in
+
+
+def mhc_post_backward(x, f_out, H_post, grad_x_next, *, out=None, dev_status=None, stream=None):
+    """First half of the layer backward in training order (before F's backward).
+    Returns (grad_f_out [T,C], red [T, n*n + n] float32)."""
+    T, n, C = x.shape
+    p = params(n, T, C, x.dtype)
+    if out is None:
+        out = (torch.empty_like(f_out),
+               torch.empty(T, n * n + n, dtype=torch.float32, device=x.device))
+    gf, red = out
+    st = _lib.load().mhc_post_backward(ctypes.byref(p), _p(x), _p(f_out), _p(H_post),
+                                       _p(grad_x_next), _p(gf), _p(red), _p(dev_status),
+                                       _stream(stream))
+    _check(st, "mhc_post_backward")
+    return gf, red
+
+
+def mhc_pre_backward(x, phi, b, alpha, grad_x_next, grad_h_in, red, *, t_max: int = 20,
+                     eps: float = 1e-6, out=None, workspace=None, dev_status=None, stream=None):
+    """Second half of the layer backward in training order (after F's backward).
+    Returns (grad_x, grad_phi, grad_b, grad_alpha)."""
+    T, n, C = x.shape
+    p = params(n, T, C, x.dtype, t_max, eps)
+    if out is None:
+        out = (torch.empty_like(x), torch.empty_like(phi), torch.empty_like(b),
+               torch.empty_like(alpha))
+    gx, gphi, gb, ga = out
+    lib = _lib.load()
+    ws, wsb = _workspace(int(lib.mhc_pre_backward_workspace_size(ctypes.byref(p))), x.device,
+                         workspace)
+    st = lib.mhc_pre_backward(ctypes.byref(p), _p(x), _p(phi), _p(b), _p(alpha), _p(grad_x_next),
+                              _p(grad_h_in), _p(red), _p(gx), _p(gphi), _p(gb), _p(ga), _p(ws),
+                              wsb, _p(dev_status), _stream(stream))
+    _check(st, "mhc_pre_backward")
+    return gx, gphi, gb, ga
+
+
 def mhc_backward_map(x, phi, b, alpha, f_out, grad_x_next, grad_h_in, workspace, *,
                      t_max: int = 20, eps: float = 1e-6, dev_status=None, stream=None):
     """Phase 1 of mhc_backward: per-token records into ``workspace`` (uint8 tensor of at

@@ -34,6 +34,7 @@
 // with TMA.  Waits are bounded; on timeout the kernel records MHC_ERR_TIMEOUT,
 // drains, frees TMEM and returns.
 #include "mhc_common.cuh"
+#include "mhc_dispatch.h"
 #include "tc_sm100.cuh"
 
 namespace mhc {
@@ -135,6 +136,7 @@ struct ApplyArgs {
   float* xpart;   // [E][NTT][KR][M] partials of the leftover slices
   int* xcnt;      // [E]
   int* status;
+  int write_gf;   // 0: grad_f_out is not produced (pre half of the split backward)
 };
 
 // Walks one CTA's items: for every tile t its P owned slices, then the
@@ -353,7 +355,7 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
         const uint32_t sb = tc::smem_u32(smem + s * STAGE);
 #pragma unroll
         for (int jj = 0; jj < N; ++jj) tc::tma_store_3d(&tm_gx, sb + X_OFF + jj * XB, c0, jj, tt0);
-        tc::tma_store_2d(&tm_gf, sb + GG_OFF, c0, tt0);
+        if (a.write_gf) tc::tma_store_2d(&tm_gf, sb + GG_OFF, c0, tt0);
         tc::bulk_commit();
         tc::bulk_wait_read<0>();
         tc::mbar_arrive(bar(B_SFREE + s));
@@ -457,7 +459,7 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
         unpack_pairs(*reinterpret_cast<const uint4*>(st + GG_OFF + sw32(tok, chunk)), gp);
         // grad_f_out = sum_i H_post[i] G_i; it replaces this thread's grad_h_in
         // piece in the stage (same swizzled position) for the tile store
-        {
+        if (a.write_gf) {
           uint32_t w[4];
 #pragma unroll
           for (int pr = 0; pr < 4; ++pr) {
@@ -657,8 +659,12 @@ cudaError_t apply_tc_dispatch(int64_t T, int64_t C, const void* x, const void* p
   if (e != cudaSuccess) return e;
   e = make_tmap_bf16(&mgx, gx, 3, dx, sx, bx, CU_TENSOR_MAP_SWIZZLE_32B);
   if (e != cudaSuccess) return e;
-  e = make_tmap_bf16(&mgf, gf, 2, d2, s2, b2, CU_TENSOR_MAP_SWIZZLE_32B);
-  if (e != cudaSuccess) return e;
+  if (gf != nullptr) {
+    e = make_tmap_bf16(&mgf, gf, 2, d2, s2, b2, CU_TENSOR_MAP_SWIZZLE_32B);
+    if (e != cudaSuccess) return e;
+  } else {
+    mgf = mgx;  // never used: no grad_f_out store is issued
+  }
 
   ApplyArgs a;
   a.T = T;
@@ -677,6 +683,7 @@ cudaError_t apply_tc_dispatch(int64_t T, int64_t C, const void* x, const void* p
   a.xpart = (float*)scratch;
   a.xcnt = (int*)((char*)scratch + (size_t)pl.E * pl.NTT * KR * M * 4);
   a.status = st;
+  a.write_gf = gf != nullptr ? 1 : 0;
   e = cudaFuncSetAttribute(k_apply_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (e != cudaSuccess) return e;
   if (pl.E > 0) {

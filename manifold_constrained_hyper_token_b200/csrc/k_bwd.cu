@@ -5,7 +5,8 @@
 //
 //   grad_x[j][c]  = sum_i H_res[i][j] G[i][c] + H_pre[j] g[c]
 //                   + sum_m phi[jC+c][m] u[m] - kappa x[j][c]
-//   grad_f_out[c] = sum_i H_post[i] G[i][c]
+//   grad_f_out[c] = sum_i H_post[i] G[i][c]     (skipped when grad_f is null:
+//                                                 the split backward's pre half)
 //   grad_phi[k][m] = sum_t x_t[k] u_t[m]
 //
 // and finishes grad_b = sum_t dz_t, grad_alpha = sum_t dz_t . y_t from the
@@ -21,6 +22,7 @@
 // (stream, channel) pairs of one token; the other streams' G values arrive by
 // warp shuffle.
 #include "mhc_common.cuh"
+#include "mhc_dispatch.h"
 
 namespace mhc {
 
@@ -137,10 +139,10 @@ __global__ void __launch_bounds__(bwdk::NT) k_bwd_apply(
         if (cvalid[e]) {
           if constexpr (sizeof(TIO) == 2) {
             grad_x[(t * N + j) * C + c0 + e] = __float2bfloat16_rn(gx[e]);
-            if (j == 0) grad_f[t * C + c0 + e] = __float2bfloat16_rn(gf[e]);
+            if (j == 0 && grad_f != nullptr) grad_f[t * C + c0 + e] = __float2bfloat16_rn(gf[e]);
           } else {
             grad_x[(t * N + j) * C + c0 + e] = gx[e];
-            if (j == 0) grad_f[t * C + c0 + e] = gf[e];
+            if (j == 0 && grad_f != nullptr) grad_f[t * C + c0 + e] = gf[e];
           }
         }
       }

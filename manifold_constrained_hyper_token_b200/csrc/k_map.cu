@@ -22,6 +22,7 @@
 // bitwise reproducible.  This is the fp32-I/O path; bf16 I/O projects on the
 // tensor cores instead (k_map_tc.cu).
 #include "mhc_common.cuh"
+#include "mhc_dispatch.h"
 
 namespace mhc {
 
@@ -52,10 +53,12 @@ static size_t map_smem_bytes() {
   return two > red ? two : red;
 }
 
-// BWD = false: write H_pre / H_post / H_res.
-// BWD = true : write coef [T][Coef<N>::SIZE] and, per CTA, the sums over its
-//              tokens of dz and dz . y: part [gridDim.x][Coef<N>::DZ_SIZE].
-template <typename TIO, int N, bool BWD>
+// MAP_FWD      : write H_pre / H_post / H_res.
+// MAP_BWD      : write coef [T][Coef<N>::SIZE] and, per CTA, the sums over its
+//                tokens of dz and dz . y: part [gridDim.x][Coef<N>::DZ_SIZE].
+// MAP_BWD_SPLIT: as MAP_BWD, but <G_i, x_j> and <G_i, f_out> come from the
+//                post half's reductions `red` [T][n*n + n] (G and f unused).
+template <typename TIO, int N, int MODE>
 __global__ void __launch_bounds__(mapk::NT) k_map(
     int64_t T, int64_t C, int iters, float eps, const TIO* __restrict__ x,
     const float* __restrict__ phi, const float* __restrict__ bias, const float* __restrict__ alpha_p,
@@ -63,7 +66,10 @@ __global__ void __launch_bounds__(mapk::NT) k_map(
     float* __restrict__ Hpre_o, float* __restrict__ Hpost_o, float* __restrict__ Hres_o,
     // backward inputs / outputs
     const TIO* __restrict__ G, const TIO* __restrict__ g, const TIO* __restrict__ f,
-    float* __restrict__ coef_o, float* __restrict__ part_o, int* status) {
+    const float* __restrict__ red_in, float* __restrict__ coef_o, float* __restrict__ part_o,
+    int* status) {
+  constexpr bool BWD = MODE != MAP_FWD;
+  constexpr bool SPLIT = MODE == MAP_BWD_SPLIT;
   using S = MapShape<N>;
   using V = Vec<TIO>;
   using namespace mapk;
@@ -189,16 +195,21 @@ __global__ void __launch_bounds__(mapk::NT) k_map(
 #pragma unroll
             for (int i = 0; i < N; ++i) {
               xv[i] = xs[(i * CC + dsub * DCH + e) * TMP + dtok];
-              Gv[i] = to_f32(G[(t * N + i) * C + c]);
+              Gv[i] = SPLIT ? 0.0f : to_f32(G[(t * N + i) * C + c]);
             }
             const float gv = to_f32(g[t * C + c]);
-            const float fv = to_f32(f[t * C + c]);
+            const float fv = SPLIT ? 0.0f : to_f32(f[t * C + c]);
+            if constexpr (SPLIT) {
+#pragma unroll
+              for (int i = 0; i < N; ++i) dots[N * N + i] = fmaf(gv, xv[i], dots[N * N + i]);
+            } else {
 #pragma unroll
             for (int i = 0; i < N; ++i) {
 #pragma unroll
               for (int j = 0; j < N; ++j) dots[i * N + j] = fmaf(Gv[i], xv[j], dots[i * N + j]);
               dots[N * N + i] = fmaf(gv, xv[i], dots[N * N + i]);
               dots[N * N + N + i] = fmaf(Gv[i], fv, dots[N * N + N + i]);
+            }
             }
           }
         }
@@ -278,15 +289,17 @@ __global__ void __launch_bounds__(mapk::NT) k_map(
         for (int e = 0; e < N * N; ++e) Hres_o[t * N * N + e] = H[e];
       } else {
         const float* dt = ssr + TM + tid * M;
+        const float* rt = red_in + (SPLIT ? t * (N * N + N) : 0);
         float dA[N * N], dz[M];
 #pragma unroll
-        for (int e = 0; e < N * N; ++e) dA[e] = dt[e];
+        for (int e = 0; e < N * N; ++e) dA[e] = SPLIT ? __ldg(rt + e) : dt[e];
         float dzres[N * N];
         sk_adjoint<N>(zres, dA, dzres, iters);
 #pragma unroll
         for (int i = 0; i < N; ++i) {
           dz[i] = dt[N * N + i] * spre[i] * (1.0f - spre[i]);
-          dz[N + i] = dt[N * N + N + i] * 2.0f * spost[i] * (1.0f - spost[i]);
+          dz[N + i] = (SPLIT ? __ldg(rt + N * N + i) : dt[N * N + N + i]) * 2.0f * spost[i] *
+                      (1.0f - spost[i]);
         }
 #pragma unroll
         for (int e = 0; e < N * N; ++e) dz[2 * N + e] = dzres[e];
@@ -326,35 +339,36 @@ __global__ void __launch_bounds__(mapk::NT) k_map(
   }
 }
 
-template <typename TIO, int N, bool BWD>
+template <typename TIO, int N, int MODE>
 static cudaError_t launch_map_t(int64_t T, int64_t C, int iters, float eps, const void* x,
                                 const float* phi, const float* b, const float* alpha,
                                 float* Hpre, float* Hpost, float* Hres, const void* G,
-                                const void* g, const void* f, float* coef, float* part, int* st,
-                                cudaStream_t s) {
+                                const void* g, const void* f, const float* red, float* coef,
+                                float* part, int* st, cudaStream_t s) {
   const size_t smem = map_smem_bytes<TIO, N>();
-  auto kern = k_map<TIO, N, BWD>;
+  auto kern = k_map<TIO, N, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int64_t grid = (T + mapk::TM - 1) / mapk::TM;
   kern<<<(unsigned)grid, mapk::NT, smem, s>>>(T, C, iters, eps, (const TIO*)x, phi, b, alpha, Hpre,
                                              Hpost, Hres, (const TIO*)G, (const TIO*)g,
-                                             (const TIO*)f, coef, part, st);
+                                             (const TIO*)f, red, coef, part, st);
   return cudaGetLastError();
 }
 
 cudaError_t map_fwd_dispatch(int n, int dtype, int64_t T, int64_t C, int iters, float eps,
                              const void* x, const float* phi, const float* b, const float* alpha,
                              float* Hpre, float* Hpost, float* Hres, int* st, cudaStream_t s) {
-#define MHC_MAPF(NN)                                                                            \
-  case NN:                                                                                      \
-    return dtype == MHC_DTYPE_BF16                                                              \
-               ? launch_map_t<__nv_bfloat16, NN, false>(T, C, iters, eps, x, phi, b, alpha,     \
-                                                        Hpre, Hpost, Hres, nullptr, nullptr,    \
-                                                        nullptr, nullptr, nullptr, st, s)       \
-               : launch_map_t<float, NN, false>(T, C, iters, eps, x, phi, b, alpha, Hpre,       \
-                                                Hpost, Hres, nullptr, nullptr, nullptr,         \
-                                                nullptr, nullptr, st, s);
+#define MHC_MAPF(NN)                                                                             \
+  case NN:                                                                                       \
+    return dtype == MHC_DTYPE_BF16                                                               \
+               ? launch_map_t<__nv_bfloat16, NN, MAP_FWD>(T, C, iters, eps, x, phi, b, alpha,    \
+                                                          Hpre, Hpost, Hres, nullptr, nullptr,   \
+                                                          nullptr, nullptr, nullptr, nullptr,    \
+                                                          st, s)                                 \
+               : launch_map_t<float, NN, MAP_FWD>(T, C, iters, eps, x, phi, b, alpha, Hpre,      \
+                                                  Hpost, Hres, nullptr, nullptr, nullptr,        \
+                                                  nullptr, nullptr, nullptr, st, s);
   switch (n) {
     MHC_MAPF(1)
     MHC_MAPF(2)
@@ -364,18 +378,30 @@ cudaError_t map_fwd_dispatch(int n, int dtype, int64_t T, int64_t C, int iters, 
 #undef MHC_MAPF
 }
 
+template <typename TIO, int N>
+static cudaError_t map_bwd_n(int64_t T, int64_t C, int iters, float eps, const void* x,
+                             const float* phi, const float* b, const float* alpha, const void* G,
+                             const void* g, const void* f, const float* red, float* coef,
+                             float* part, int* st, cudaStream_t s) {
+  return red == nullptr
+             ? launch_map_t<TIO, N, MAP_BWD>(T, C, iters, eps, x, phi, b, alpha, nullptr, nullptr,
+                                             nullptr, G, g, f, nullptr, coef, part, st, s)
+             : launch_map_t<TIO, N, MAP_BWD_SPLIT>(T, C, iters, eps, x, phi, b, alpha, nullptr,
+                                                   nullptr, nullptr, nullptr, g, nullptr, red,
+                                                   coef, part, st, s);
+}
+
 cudaError_t map_bwd_dispatch(int n, int dtype, int64_t T, int64_t C, int iters, float eps,
                              const void* x, const float* phi, const float* b, const float* alpha,
-                             const void* G, const void* g, const void* f, float* coef, float* part,
-                             int* st, cudaStream_t s) {
-#define MHC_MAPB(NN)                                                                            \
-  case NN:                                                                                      \
-    return dtype == MHC_DTYPE_BF16                                                              \
-               ? launch_map_t<__nv_bfloat16, NN, true>(T, C, iters, eps, x, phi, b, alpha,      \
-                                                       nullptr, nullptr, nullptr, G, g, f, coef, \
-                                                       part, st, s)                              \
-               : launch_map_t<float, NN, true>(T, C, iters, eps, x, phi, b, alpha, nullptr,     \
-                                               nullptr, nullptr, G, g, f, coef, part, st, s);
+                             const void* G, const void* g, const void* f, const float* red,
+                             float* coef, float* part, int* st, cudaStream_t s) {
+#define MHC_MAPB(NN)                                                                          \
+  case NN:                                                                                    \
+    return dtype == MHC_DTYPE_BF16                                                            \
+               ? map_bwd_n<__nv_bfloat16, NN>(T, C, iters, eps, x, phi, b, alpha, G, g, f, red, \
+                                              coef, part, st, s)                              \
+               : map_bwd_n<float, NN>(T, C, iters, eps, x, phi, b, alpha, G, g, f, red, coef,   \
+                                      part, st, s);
   switch (n) {
     MHC_MAPB(1)
     MHC_MAPB(2)

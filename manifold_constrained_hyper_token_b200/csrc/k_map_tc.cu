@@ -9,9 +9,10 @@
 // recompute in the backward).
 //
 // One CTA = 128 tokens (the MMA M).  The token's n*C inputs stream through a
-// TMA ring in chunks of 32 channels x 4 streams (64-byte rows, 64-byte
-// swizzle): per stream an x tile [128 x 32] (the MMA A operand, K-major) and
-// the matching rows of phi^T as a [48 x 32] B operand, whose 48 rows are the
+// TMA ring in chunks of 32 channels x 4 streams (64-byte rows and swizzle; a
+// TMA row piece narrower than 64 bytes caps an SM's streaming rate): per
+// stream an x tile [128 x 32] (the MMA A operand, K-major) and the matching
+// rows of phi^T as a [48 x 32] B operand, whose 48 rows are the
 // 24 logit columns split into a bf16 high part and a bf16 low part
 // (phi = hi + lo), so y = D[:, m] + D[:, 24 + m] carries phi to ~16 bits.
 // x itself is bf16, so the products are exact and only the fp32
@@ -25,6 +26,7 @@
 // timeout the kernel records MHC_ERR_TIMEOUT, drains what it issued, frees
 // TMEM and returns.
 #include "mhc_common.cuh"
+#include "mhc_dispatch.h"
 #include "tc_sm100.cuh"
 
 namespace mhc {
@@ -33,23 +35,37 @@ namespace tcmap {
 constexpr int N = 4;
 constexpr int M = N * N + 2 * N;     // 24 logits
 constexpr int TM = 128;              // tokens per CTA (MMA M)
-constexpr int CH = 32;               // channels per chunk: 64-byte rows
 constexpr int NL = 48;               // MMA N: 24 high + 24 low logit columns
-constexpr int NWARPS = 10;
+constexpr int NWARPS = 11;           // TMA, MMA, 8 math warps, TMA stores (MAP_POSTFWD)
+constexpr int STORE_WARP = 10;
 constexpr int NT = NWARPS * 32;
-constexpr int XBOX = TM * CH * 2;    // one stream's x tile, 8 KB
-constexpr int PBOX = NL * CH * 2;    // one stream's phi^T tile, 3 KB
 constexpr uint32_t TMEM_COLS = 64;
 constexpr uint64_t WAIT_NS = 2000000000ull;  // 2 s per wait before giving up
 
-template <bool BWD> struct Cfg {
-  static constexpr int NS = BWD ? 2 : 4;        // pipeline stages
+// MAP_FWD: the forward mapping.  MAP_BWD: the backward's recompute with all
+// 24 C-reductions.  MAP_BWD_SPLIT: the pre half of the backward in training
+// order -- the post half already reduced <G_i, x_j> and <G_i, f_out> (the
+// `red` input), so only x and grad_h_in are staged.  MAP_POSTFWD: layer l's
+// post merge x_next = H_res x + H_post^T f_out fused with layer l+1's
+// forward mapping of x_next (the math warps form x_next in the stage, the
+// tensor cores project it, a store warp writes it out).
+template <int MODE> struct Cfg {
+  static constexpr bool FULLB = MODE == MAP_BWD;
+  static constexpr int CH = 32;                 // channels per chunk: 64-byte rows
+  static constexpr int ROW = CH * 2;            // bytes per tile row = swizzle span
+  static constexpr int XBOX = TM * CH * 2;      // one stream's x tile
+  static constexpr int PBOX = NL * CH * 2;      // one stream's phi^T tile
+  static constexpr int NS = FULLB ? 2 : 4;      // pipeline stages (MAP_BWD stages 4 tensors)
   static constexpr int X_OFF = 0;
   static constexpr int P_OFF = N * XBOX;
-  static constexpr int G_OFF = P_OFF + N * PBOX;
-  static constexpr int GG_OFF = G_OFF + N * XBOX;  // grad_h_in tile
-  static constexpr int F_OFF = GG_OFF + XBOX;      // f_out tile
-  static constexpr int STAGE = BWD ? F_OFF + XBOX : G_OFF;
+  static constexpr int G_OFF = P_OFF + N * PBOX;                 // grad_x_next tiles (MAP_BWD)
+  static constexpr int GG_OFF = FULLB ? G_OFF + N * XBOX : G_OFF;  // grad_h_in tile
+  static constexpr int F_OFF = GG_OFF + XBOX;                     // f_out tile (MAP_BWD)
+  static constexpr int FN_OFF = G_OFF;                            // f_out tile (MAP_POSTFWD)
+  static constexpr int STAGE = MODE == MAP_FWD ? G_OFF
+                               : FULLB        ? F_OFF + XBOX
+                               : MODE == MAP_BWD_SPLIT ? GG_OFF + XBOX
+                                                       : FN_OFF + XBOX;
   static constexpr int DATA = NS * STAGE;
   static constexpr int SMEM = DATA + 1024 /*align*/ + 256 /*barriers, flags*/;
 };
@@ -79,18 +95,29 @@ __device__ __forceinline__ void bf16x8_to_f32(uint4 q, float (&v)[8]) {
   }
 }
 
-// Row `tok` of a [128 x 32] bf16 tile stored with the 64-byte swizzle: the
-// 16-byte chunk c of the row sits at chunk position c ^ ((tok >> 1) & 3).
-__device__ __forceinline__ uint4 ld_sw64(const uint8_t* tile, int tok, int chunk) {
-  const int phys = chunk ^ ((tok >> 1) & 3);
-  return *reinterpret_cast<const uint4*>(tile + tok * 64 + phys * 16);
+// Row `tok`, 16-byte chunk `chunk` of a bf16 tile whose rows are ROW bytes
+// and stored with the ROW-byte swizzle: 64-byte rows put chunk c at
+// c ^ ((tok >> 1) & 3), 32-byte rows at c ^ ((tok >> 2) & 1).
+template <int ROW>
+__device__ __forceinline__ int sw_off(int tok, int chunk) {
+  static_assert(ROW == 32 || ROW == 64, "row width");
+  const int phys = ROW == 64 ? chunk ^ ((tok >> 1) & 3) : chunk ^ ((tok >> 2) & 1);
+  return tok * ROW + phys * 16;
+}
+template <int ROW>
+__device__ __forceinline__ uint4 ld_sw(const uint8_t* tile, int tok, int chunk) {
+  return *reinterpret_cast<const uint4*>(tile + sw_off<ROW>(tok, chunk));
+}
+__device__ __forceinline__ uint32_t pack_bf2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
 }
 
 __device__ __forceinline__ void named_bar(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-template <bool BWD>
+template <int MODE>
 __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_phi,
     const __grid_constant__ CUtensorMap tm_G, const __grid_constant__ CUtensorMap tm_g,
@@ -98,20 +125,29 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
     int ck_period, const float* __restrict__ bias, const float* __restrict__ alpha_p,
     float* __restrict__ Hpre_o, float* __restrict__ Hpost_o, float* __restrict__ Hres_o,
     __nv_bfloat16* __restrict__ urec_o, float* __restrict__ hrec_o, float* __restrict__ part_o,
-    int* status) {
+    const float* __restrict__ red_in, const float* __restrict__ hpost_in,
+    const float* __restrict__ hres_in, int* status) {
   using namespace tcmap;
-  using CFG = Cfg<BWD>;
+  using CFG = Cfg<MODE>;
+  constexpr bool BWD = MODE == MAP_BWD || MODE == MAP_BWD_SPLIT;
+  constexpr bool SPLIT = MODE == MAP_BWD_SPLIT;
+  constexpr bool POST = MODE == MAP_POSTFWD;
   constexpr int NS = CFG::NS;
+  constexpr int CH = CFG::CH, XBOX = CFG::XBOX, PBOX = CFG::PBOX, ROW = CFG::ROW;
+  constexpr tc::Swz SWZ = ROW == 64 ? tc::SWZ_64B : tc::SWZ_32B;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + CFG::DATA);  // full[NS] empty[NS] done fin
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + 2);
+  // full[NS] empty[NS] done fin xready[NS] sdone
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + CFG::DATA);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * NS + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   auto full = [&](int s) { return tc::smem_u32(bars + s); };
   auto empty = [&](int s) { return tc::smem_u32(bars + NS + s); };
   const uint32_t done_bar = tc::smem_u32(bars + 2 * NS);
   const uint32_t fin_bar = tc::smem_u32(bars + 2 * NS + 1);
+  auto xready = [&](int s) { return tc::smem_u32(bars + 2 * NS + 2 + s); };
+  const uint32_t sdone_bar = tc::smem_u32(bars + 3 * NS + 2);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t t0 = (int64_t)blockIdx.x * TM;
@@ -121,19 +157,27 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       tc::mbar_init(full(s), 1);
-      tc::mbar_init(empty(s), 1 + 8);  // the MMA commit + one arrive per math warp
+      // the MMA commit + one arrive per math warp; with the post merge fused,
+      // the MMA commit + the store warp once its x_next stores read the stage
+      tc::mbar_init(empty(s), POST ? 2 : 1 + 8);
+      tc::mbar_init(xready(s), 8);  // (MAP_POSTFWD) every math warp wrote x_next
     }
     tc::mbar_init(done_bar, 1);
     tc::mbar_init(fin_bar, 1);
+    tc::mbar_init(sdone_bar, 1);
     *abort_flag = 0;
     tc::mbar_fence_init();
   }
   if (warp == 0 && lane == 0) {
     tc::tma_prefetch_desc(&tm_x);
     tc::tma_prefetch_desc(&tm_phi);
-    if constexpr (BWD) {
+    if constexpr (BWD) tc::tma_prefetch_desc(&tm_g);
+    if constexpr (BWD && !SPLIT) {
       tc::tma_prefetch_desc(&tm_G);
-      tc::tma_prefetch_desc(&tm_g);
+      tc::tma_prefetch_desc(&tm_f);
+    }
+    if constexpr (POST) {
+      tc::tma_prefetch_desc(&tm_G);  // x_next (store)
       tc::tma_prefetch_desc(&tm_f);
     }
   }
@@ -170,14 +214,15 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
         for (int i = 0; i < N; ++i) {
           tc::tma_load_3d(base + CFG::X_OFF + i * XBOX, &tm_x, full(s), c0, i, (int)t0, pol_stream);
           tc::tma_load_3d(base + CFG::P_OFF + i * PBOX, &tm_phi, full(s), c0, i, 0, pol_keep);
-          if constexpr (BWD)
+          if constexpr (BWD && !SPLIT)
             tc::tma_load_3d(base + CFG::G_OFF + i * XBOX, &tm_G, full(s), c0, i, (int)t0,
                             pol_stream);
         }
-        if constexpr (BWD) {
-          tc::tma_load_2d(base + CFG::GG_OFF, &tm_g, full(s), c0, (int)t0, pol_stream);
+        if constexpr (BWD) tc::tma_load_2d(base + CFG::GG_OFF, &tm_g, full(s), c0, (int)t0, pol_stream);
+        if constexpr (BWD && !SPLIT)
           tc::tma_load_2d(base + CFG::F_OFF, &tm_f, full(s), c0, (int)t0, pol_stream);
-        }
+        if constexpr (POST)
+          tc::tma_load_2d(base + CFG::FN_OFF, &tm_f, full(s), c0, (int)t0, pol_stream);
         ++issued;
       }
       if (*abort_flag) {
@@ -194,7 +239,8 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
       for (int cc = 0; cc < nch; ++cc) {
         const int s = cc % NS;
         const uint32_t ph = (uint32_t)(cc / NS) & 1u;
-        if (!tc::mbar_wait(full(s), ph, abort_flag, WAIT_NS)) {
+        // with the post merge fused, the A operand is x_next, written by the math warps
+        if (!tc::mbar_wait(POST ? xready(s) : full(s), ph, abort_flag, WAIT_NS)) {
           give_up();
           break;
         }
@@ -204,8 +250,8 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
         for (int i = 0; i < N; ++i) {
 #pragma unroll
           for (int kk = 0; kk < CH / 16; ++kk) {
-            const uint64_t a = tc::smem_desc(base + CFG::X_OFF + i * XBOX + kk * 32, 16, 512, tc::SWZ_64B);
-            const uint64_t b = tc::smem_desc(base + CFG::P_OFF + i * PBOX + kk * 32, 16, 512, tc::SWZ_64B);
+            const uint64_t a = tc::smem_desc(base + CFG::X_OFF + i * XBOX + kk * 32, 16, 8 * ROW, SWZ);
+            const uint64_t b = tc::smem_desc(base + CFG::P_OFF + i * PBOX + kk * 32, 16, 8 * ROW, SWZ);
             tc::mma_bf16(tmem, a, b, idesc, (cc | i | kk) != 0 ? 1u : 0u);
           }
         }
@@ -219,12 +265,41 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
         tc::mbar_wait(fin_bar, 0, nullptr, WAIT_NS / 4);
       }
     }
+  } else if (warp == STORE_WARP) {
+    // ------------------------------------------- x_next stores (MAP_POSTFWD)
+    if (POST && lane == 0) {
+      for (int cc = 0; cc < nch; ++cc) {
+        const int s = cc % NS;
+        if (!tc::mbar_wait(xready(s), (uint32_t)(cc / NS) & 1u, abort_flag, WAIT_NS)) {
+          give_up();
+          break;
+        }
+        const uint32_t base = tc::smem_u32(smem + s * CFG::STAGE);
+#pragma unroll
+        for (int i = 0; i < N; ++i)
+          tc::tma_store_3d(&tm_G, base + CFG::X_OFF + i * XBOX, cc * CH, i, (int)t0);
+        tc::bulk_commit();
+        tc::bulk_wait_read<0>();
+        tc::mbar_arrive(empty(s));
+      }
+      tc::bulk_wait<0>();
+      tc::mbar_arrive(sdone_bar);  // every stage read: its memory may be reused
+    }
   } else {
     // -------------------------------------------------- CUDA-core reductions
     const int q = warp & 3;            // TMEM lane quarter this warp may read
     const int h = (warp - 2) >> 2;     // channel half of each chunk
     const int tok = 32 * q + lane;
     float ss = 0.0f;
+    // MAP_POSTFWD: this token's layer-l maps (the post merge's coefficients)
+    float hr_in[POST ? N * N : 1], hp_in[POST ? N : 1];
+    if constexpr (POST) {
+      const bool tv = t0 + tok < T;
+#pragma unroll
+      for (int e = 0; e < N * N; ++e) hr_in[e] = tv ? __ldg(hres_in + (t0 + tok) * N * N + e) : 0.0f;
+#pragma unroll
+      for (int i = 0; i < N; ++i) hp_in[i] = tv ? __ldg(hpost_in + (t0 + tok) * N + i) : 0.0f;
+    }
     float dots[BWD ? M : 1];
 #pragma unroll
     for (int m = 0; m < (BWD ? M : 1); ++m) dots[m] = 0.0f;
@@ -235,25 +310,59 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
         give_up();
         break;
       }
-      const uint8_t* st = smem + s * CFG::STAGE;
+      uint8_t* st = smem + s * CFG::STAGE;
 #pragma unroll
-      for (int qq = 0; qq < 2; ++qq) {
-        const int chunk = 2 * h + qq;
+      for (int qq = 0; qq < CH / 16; ++qq) {
+        const int chunk = (CH / 16) * h + qq;
+        if constexpr (POST) {
+          // x_next[i] = sum_j H_res[i][j] x_j + H_post[i] f_out (the k_post order),
+          // rounded to bf16 in place; the sum of squares is of the rounded values
+          float xv[N][8], fv[8];
+#pragma unroll
+          for (int i = 0; i < N; ++i) bf16x8_to_f32(ld_sw<ROW>(st + CFG::X_OFF + i * XBOX, tok, chunk), xv[i]);
+          bf16x8_to_f32(ld_sw<ROW>(st + CFG::FN_OFF, tok, chunk), fv);
+#pragma unroll
+          for (int i = 0; i < N; ++i) {
+            float o[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              float acc = hp_in[i] * fv[e];
+#pragma unroll
+              for (int j = 0; j < N; ++j) acc = fmaf(hr_in[i * N + j], xv[j][e], acc);
+              o[e] = acc;
+            }
+            const uint4 w = make_uint4(pack_bf2(o[0], o[1]), pack_bf2(o[2], o[3]),
+                                       pack_bf2(o[4], o[5]), pack_bf2(o[6], o[7]));
+            *reinterpret_cast<uint4*>(st + CFG::X_OFF + i * XBOX + sw_off<ROW>(tok, chunk)) = w;
+            float r[8];
+            bf16x8_to_f32(w, r);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ss = fmaf(r[e], r[e], ss);
+          }
+          continue;
+        }
         float xv[N][8];
 #pragma unroll
         for (int i = 0; i < N; ++i) {
-          bf16x8_to_f32(ld_sw64(st + CFG::X_OFF + i * XBOX, tok, chunk), xv[i]);
+          bf16x8_to_f32(ld_sw<ROW>(st + CFG::X_OFF + i * XBOX, tok, chunk), xv[i]);
 #pragma unroll
           for (int e = 0; e < 8; ++e) ss = fmaf(xv[i][e], xv[i][e], ss);
         }
-        if constexpr (BWD) {
+        if constexpr (SPLIT) {
+          float gv[8];
+          bf16x8_to_f32(ld_sw<ROW>(st + CFG::GG_OFF, tok, chunk), gv);
+#pragma unroll
+          for (int i = 0; i < N; ++i)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) dots[N * N + i] = fmaf(gv[e], xv[i][e], dots[N * N + i]);
+        } else if constexpr (BWD) {
           float gv[8], fv[8];
-          bf16x8_to_f32(ld_sw64(st + CFG::GG_OFF, tok, chunk), gv);
-          bf16x8_to_f32(ld_sw64(st + CFG::F_OFF, tok, chunk), fv);
+          bf16x8_to_f32(ld_sw<ROW>(st + CFG::GG_OFF, tok, chunk), gv);
+          bf16x8_to_f32(ld_sw<ROW>(st + CFG::F_OFF, tok, chunk), fv);
 #pragma unroll
           for (int i = 0; i < N; ++i) {
             float Gv[8];
-            bf16x8_to_f32(ld_sw64(st + CFG::G_OFF + i * XBOX, tok, chunk), Gv);
+            bf16x8_to_f32(ld_sw<ROW>(st + CFG::G_OFF + i * XBOX, tok, chunk), Gv);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
 #pragma unroll
@@ -264,13 +373,21 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
           }
         }
       }
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(empty(s));
+      if constexpr (POST) {
+        tc::fence_proxy_async_smem();  // x_next visible to the MMA and the TMA store
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(xready(s));
+      } else {
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(empty(s));
+      }
     }
 
     // all MMAs (and so all reads of the stage buffers) finished before the
-    // stage memory is reused for the epilogue
+    // stage memory is reused for the epilogue; with the post merge fused, the
+    // x_next stores as well
     bool ok = !*abort_flag && tc::mbar_wait(done_bar, 0, abort_flag, WAIT_NS);
+    if (POST && ok) ok = tc::mbar_wait(sdone_bar, 0, abort_flag, WAIT_NS);
     if (!ok && !*abort_flag) give_up();
     ok = __all_sync(0xffffffffu, ok);  // the TMEM loads below are warp-collective
     float* red_ss = reinterpret_cast<float*>(smem);       // [2][TM]
@@ -345,15 +462,19 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
       } else {
         sk_forward_ckpt<N>(H, iters, ck + tok, TM, ck_period);
         float dA[N * N], dz[M], dzres[N * N];
+        // dL/dH_res and dL/dH_post: this CTA's C-reductions, or the post half's
+        const float* rt = red_in + (t < T ? t : 0) * (N * N + N);
 #pragma unroll
         for (int e = 0; e < N * N; ++e)
-          dA[e] = red_dt[(0 * M + e) * TM + tok] + red_dt[(1 * M + e) * TM + tok];
+          dA[e] = SPLIT ? (t < T ? __ldg(rt + e) : 0.0f)
+                        : red_dt[(0 * M + e) * TM + tok] + red_dt[(1 * M + e) * TM + tok];
         sk_adjoint_ckpt<N>(dA, dzres, iters, ck + tok, TM, ck_period);
 #pragma unroll
         for (int i = 0; i < N; ++i) {
           const float dpre = red_dt[(0 * M + N * N + i) * TM + tok] + red_dt[(1 * M + N * N + i) * TM + tok];
-          const float dpost = red_dt[(0 * M + N * N + N + i) * TM + tok] +
-                              red_dt[(1 * M + N * N + N + i) * TM + tok];
+          const float dpost = SPLIT ? (t < T ? __ldg(rt + N * N + i) : 0.0f)
+                                    : red_dt[(0 * M + N * N + N + i) * TM + tok] +
+                                          red_dt[(1 * M + N * N + N + i) * TM + tok];
           dz[i] = dpre * spre[i] * (1.0f - spre[i]);
           dz[N + i] = dpost * 2.0f * spost[i] * (1.0f - spost[i]);
         }
@@ -420,33 +541,41 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
 }
 
 // ------------------------------------------------------------------ host
-static cudaError_t encode_maps(int64_t T, int64_t C, const void* x, const void* phiT, const void* G,
-                               const void* g, const void* f, CUtensorMap* mx, CUtensorMap* mp,
-                               CUtensorMap* mG, CUtensorMap* mg, CUtensorMap* mf) {
+static cudaError_t encode_maps(int mode, int64_t T, int64_t C, const void* x, const void* phiT,
+                               const void* G, const void* g, const void* f, CUtensorMap* mx,
+                               CUtensorMap* mp, CUtensorMap* mG, CUtensorMap* mg, CUtensorMap* mf) {
   using namespace tcmap;
+  const uint32_t CH = Cfg<MAP_FWD>::CH;
+  const CUtensorMapSwizzle SW = CU_TENSOR_MAP_SWIZZLE_64B;
+  static_assert(Cfg<MAP_FWD>::CH == Cfg<MAP_BWD>::CH && Cfg<MAP_BWD>::CH == Cfg<MAP_BWD_SPLIT>::CH,
+                "one chunk width for every mode");
   const uint64_t dx[3] = {(uint64_t)C, (uint64_t)N, (uint64_t)T};
   const uint64_t sx[2] = {(uint64_t)C * 2, (uint64_t)N * C * 2};
   const uint32_t bx[3] = {CH, 1, TM};
-  cudaError_t e = make_tmap_bf16(mx, x, 3, dx, sx, bx, CU_TENSOR_MAP_SWIZZLE_64B);
+  cudaError_t e = make_tmap_bf16(mx, x, 3, dx, sx, bx, SW);
   if (e != cudaSuccess) return e;
   const uint64_t dp[3] = {(uint64_t)C, (uint64_t)N, (uint64_t)NL};
   const uint32_t bp[3] = {CH, 1, NL};
-  e = make_tmap_bf16(mp, phiT, 3, dp, sx, bp, CU_TENSOR_MAP_SWIZZLE_64B);
+  e = make_tmap_bf16(mp, phiT, 3, dp, sx, bp, SW);
   if (e != cudaSuccess) return e;
-  if (G == nullptr) {
-    *mG = *mx;
-    *mg = *mx;
-    *mf = *mx;
-    return cudaSuccess;
-  }
-  e = make_tmap_bf16(mG, G, 3, dx, sx, bx, CU_TENSOR_MAP_SWIZZLE_64B);
-  if (e != cudaSuccess) return e;
+  // maps a mode does not read are copies of the x map (never dereferenced)
+  *mG = *mx;
+  *mg = *mx;
+  *mf = *mx;
   const uint64_t d2[2] = {(uint64_t)C, (uint64_t)T};
   const uint64_t s2[1] = {(uint64_t)C * 2};
   const uint32_t b2[2] = {CH, TM};
-  e = make_tmap_bf16(mg, g, 2, d2, s2, b2, CU_TENSOR_MAP_SWIZZLE_64B);
-  if (e != cudaSuccess) return e;
-  return make_tmap_bf16(mf, f, 2, d2, s2, b2, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (mode != MAP_FWD) {
+    e = make_tmap_bf16(mg, g, 2, d2, s2, b2, SW);
+    if (e != cudaSuccess) return e;
+  }
+  if (mode == MAP_BWD) {
+    e = make_tmap_bf16(mG, G, 3, dx, sx, bx, SW);
+    if (e != cudaSuccess) return e;
+    e = make_tmap_bf16(mf, f, 2, d2, s2, b2, SW);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 // Smallest checkpoint period whose checkpoints fit beside the epilogue
@@ -464,36 +593,85 @@ static int ck_period_for(int iters, size_t stage_bytes) {
 
 size_t map_tc_phi_bytes(int64_t C) { return (size_t)tcmap::NL * tcmap::N * C * 2; }
 
-cudaError_t map_tc_dispatch(bool bwd, int64_t T, int64_t C, int iters, float eps, const void* x,
+template <int MODE>
+static cudaError_t launch_map_tc(const CUtensorMap& mx, const CUtensorMap& mp, const CUtensorMap& mG,
+                                 const CUtensorMap& mg, const CUtensorMap& mf, int64_t T, int64_t C,
+                                 int iters, float eps, const float* b, const float* alpha,
+                                 float* Hpre, float* Hpost, float* Hres, void* urec, float* hrec,
+                                 float* part, const float* red, int* st, cudaStream_t s,
+                                 const float* hpost_in = nullptr, const float* hres_in = nullptr) {
+  using namespace tcmap;
+  auto kern = k_map_tc<MODE>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<MODE>::SMEM);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = (unsigned)((T + TM - 1) / TM);
+  const int P = (MODE == MAP_BWD || MODE == MAP_BWD_SPLIT) ? ck_period_for(iters, Cfg<MODE>::DATA) : 1;
+  kern<<<grid, NT, Cfg<MODE>::SMEM, s>>>(mx, mp, mG, mg, mf, T, C, iters, eps, P, b, alpha, Hpre,
+                                         Hpost, Hres, (__nv_bfloat16*)urec, hrec, part, red,
+                                         hpost_in, hres_in, st);
+  return cudaGetLastError();
+}
+
+cudaError_t map_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float eps, const void* x,
                             const float* phi, void* phi_split, const float* b, const float* alpha,
                             float* Hpre, float* Hpost, float* Hres, const void* G, const void* g,
-                            const void* f, void* urec, float* hrec, float* part, int* st,
-                            cudaStream_t s) {
+                            const void* f, const float* red, void* urec, float* hrec, float* part,
+                            int* st, cudaStream_t s) {
   using namespace tcmap;
   const int64_t K = (int64_t)N * C;
   k_phi_split<<<(unsigned)((K + 255) / 256), 256, 0, s>>>(K, phi, (__nv_bfloat16*)phi_split);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CUtensorMap mx, mp, mG, mg, mf;
-  e = encode_maps(T, C, x, phi_split, bwd ? G : nullptr, g, f, &mx, &mp, &mG, &mg, &mf);
+  e = encode_maps(mode, T, C, x, phi_split, G, g, f, &mx, &mp, &mG, &mg, &mf);
   if (e != cudaSuccess) return e;
-  const unsigned grid = (unsigned)((T + TM - 1) / TM);
-  if (bwd) {
-    auto kern = k_map_tc<true>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<true>::SMEM);
-    if (e != cudaSuccess) return e;
-    const int P = ck_period_for(iters, Cfg<true>::DATA);
-    kern<<<grid, NT, Cfg<true>::SMEM, s>>>(mx, mp, mG, mg, mf, T, C, iters, eps, P, b, alpha,
-                                           nullptr, nullptr, nullptr, (__nv_bfloat16*)urec, hrec,
-                                           part, st);
-  } else {
-    auto kern = k_map_tc<false>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<false>::SMEM);
-    if (e != cudaSuccess) return e;
-    kern<<<grid, NT, Cfg<false>::SMEM, s>>>(mx, mp, mG, mg, mf, T, C, iters, eps, 1, b, alpha,
-                                            Hpre, Hpost, Hres, nullptr, nullptr, nullptr, st);
+  switch (mode) {
+    case MAP_FWD:
+      return launch_map_tc<MAP_FWD>(mx, mp, mG, mg, mf, T, C, iters, eps, b, alpha, Hpre, Hpost,
+                                    Hres, nullptr, nullptr, nullptr, nullptr, st, s);
+    case MAP_BWD:
+      return launch_map_tc<MAP_BWD>(mx, mp, mG, mg, mf, T, C, iters, eps, b, alpha, nullptr,
+                                    nullptr, nullptr, urec, hrec, part, nullptr, st, s);
+    case MAP_BWD_SPLIT:
+      return launch_map_tc<MAP_BWD_SPLIT>(mx, mp, mG, mg, mf, T, C, iters, eps, b, alpha, nullptr,
+                                          nullptr, nullptr, urec, hrec, part, red, st, s);
+    default:
+      return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
+}
+
+// Layer l's post merge fused with layer l+1's forward mapping (bf16, n = 4):
+// x_next = H_res x + H_post^T f_out is written once, and its RMS, projection
+// onto phi_next, gates and Sinkhorn give layer l+1's maps.
+cudaError_t post_map_tc_dispatch(int64_t T, int64_t C, int iters, float eps, const void* x,
+                                 const void* f, const float* Hpost_in, const float* Hres_in,
+                                 const float* phi_next, void* phi_split, const float* b_next,
+                                 const float* alpha_next, void* x_next, float* Hpre, float* Hpost,
+                                 float* Hres, int* st, cudaStream_t s) {
+  using namespace tcmap;
+  const int64_t K = (int64_t)N * C;
+  k_phi_split<<<(unsigned)((K + 255) / 256), 256, 0, s>>>(K, phi_next,
+                                                          (__nv_bfloat16*)phi_split);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  CUtensorMap mx, mp, mG, mg, mf;
+  // the forward maps for x and phi, then x_next (store) and f_out
+  e = encode_maps(MAP_FWD, T, C, x, phi_split, nullptr, nullptr, nullptr, &mx, &mp, &mG, &mg, &mf);
+  if (e != cudaSuccess) return e;
+  const uint64_t dx[3] = {(uint64_t)C, (uint64_t)N, (uint64_t)T};
+  const uint64_t sx[2] = {(uint64_t)C * 2, (uint64_t)N * C * 2};
+  const uint32_t bx[3] = {(uint32_t)Cfg<MAP_POSTFWD>::CH, 1, TM};
+  e = make_tmap_bf16(&mG, x_next, 3, dx, sx, bx, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (e != cudaSuccess) return e;
+  const uint64_t d2[2] = {(uint64_t)C, (uint64_t)T};
+  const uint64_t s2[1] = {(uint64_t)C * 2};
+  const uint32_t b2[2] = {(uint32_t)Cfg<MAP_POSTFWD>::CH, TM};
+  e = make_tmap_bf16(&mf, f, 2, d2, s2, b2, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (e != cudaSuccess) return e;
+  return launch_map_tc<MAP_POSTFWD>(mx, mp, mG, mg, mf, T, C, iters, eps, b_next, alpha_next, Hpre,
+                                    Hpost, Hres, nullptr, nullptr, nullptr, nullptr, st, s,
+                                    Hpost_in, Hres_in);
 }
 
 }  // namespace mhc

@@ -11,6 +11,7 @@
 // block).  Row and column sums are reduced with warp shuffles inside the
 // group; the matrix never leaves registers between the load and the store.
 #include "mhc_common.cuh"
+#include "mhc_dispatch.h"
 
 namespace mhc {
 

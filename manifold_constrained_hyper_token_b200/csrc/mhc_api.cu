@@ -4,45 +4,8 @@
 #include <math.h>
 
 #include "mhc_common.cuh"
+#include "mhc_dispatch.h"
 
-namespace mhc {
-// k_sinkhorn.cu
-cudaError_t sinkhorn_dispatch(int n, int iters, int64_t B, const float* logits, float* out,
-                              int* st, cudaStream_t s);
-cudaError_t depth_amax_dispatch(int n, int64_t T, int L, const float* H, float* gf, float* gb,
-                                cudaStream_t s);
-// k_post.cu
-cudaError_t post_dispatch(int n, int dtype, int64_t T, int64_t C, const void* x, const void* f,
-                          const float* Hpost, const float* Hres, void* xn, cudaStream_t s);
-cudaError_t hin_dispatch(int n, int dtype, int64_t T, int64_t C, const void* x, const float* Hpre,
-                         void* h_in, cudaStream_t s);
-// k_map.cu
-cudaError_t map_fwd_dispatch(int n, int dtype, int64_t T, int64_t C, int iters, float eps,
-                             const void* x, const float* phi, const float* b, const float* alpha,
-                             float* Hpre, float* Hpost, float* Hres, int* st, cudaStream_t s);
-cudaError_t map_bwd_dispatch(int n, int dtype, int64_t T, int64_t C, int iters, float eps,
-                             const void* x, const float* phi, const float* b, const float* alpha,
-                             const void* G, const void* g, const void* f, float* coef, float* dzr,
-                             int* st, cudaStream_t s);
-// k_map_tc.cu (bf16, n = 4: projection on the tensor cores)
-cudaError_t map_tc_dispatch(bool bwd, int64_t T, int64_t C, int iters, float eps, const void* x,
-                            const float* phi, void* phi_split, const float* b, const float* alpha,
-                            float* Hpre, float* Hpost, float* Hres, const void* G, const void* g,
-                            const void* f, void* urec, float* hrec, float* part, int* st,
-                            cudaStream_t s);
-size_t map_tc_phi_bytes(int64_t C);
-// k_apply_tc.cu (bf16, n = 4: phi u and grad_phi on the tensor cores)
-cudaError_t apply_tc_dispatch(int64_t T, int64_t C, const void* x, const void* phi_split,
-                              const void* G, const void* g, const void* urec, const float* hrec,
-                              const float* part, int nparts, void* gx, void* gf, float* gphi,
-                              float* gb, float* ga, void* scratch, int* st, cudaStream_t s);
-size_t apply_tc_scratch_bytes(int64_t T, int64_t C);
-// k_bwd.cu
-cudaError_t apply_dispatch(int n, int dtype, int64_t T, int64_t C, const void* x, const float* phi,
-                           const void* G, const void* g, const float* coef, const float* part,
-                           int nparts, void* gx, void* gf, float* gphi, float* gb, float* ga,
-                           cudaStream_t s);
-}  // namespace mhc
 
 namespace {
 
@@ -164,9 +127,10 @@ mhc_status mhc_pre(const mhc_params* p, const void* x, const float* phi, const f
     const size_t need = mhc_pre_workspace_size(p);
     if (workspace == nullptr || workspace_bytes < need || ((uintptr_t)workspace & 255u) != 0)
       return MHC_ERR_WORKSPACE;
-    st = from_cuda(mhc::map_tc_dispatch(false, p->T, p->C, p->t_max, p->eps, x, phi, workspace, b,
-                                        alpha, H_pre, H_post, H_res, nullptr, nullptr, nullptr,
-                                        nullptr, nullptr, nullptr, dev_status, s));
+    st = from_cuda(mhc::map_tc_dispatch(mhc::MAP_FWD, p->T, p->C, p->t_max, p->eps, x, phi,
+                                        workspace, b, alpha, H_pre, H_post, H_res, nullptr,
+                                        nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                                        dev_status, s));
   } else {
     st = from_cuda(mhc::map_fwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
                                          alpha, H_pre, H_post, H_res, dev_status, s));
@@ -207,13 +171,13 @@ mhc_status mhc_backward_map(const mhc_params* p, const void* x, const float* phi
   if (st != MHC_OK) return st;
   char* ws = (char*)workspace;
   if (use_tc(p))
-    return from_cuda(mhc::map_tc_dispatch(true, p->T, p->C, p->t_max, p->eps, x, phi,
+    return from_cuda(mhc::map_tc_dispatch(mhc::MAP_BWD, p->T, p->C, p->t_max, p->eps, x, phi,
                                           ws + w.phi_off, b, alpha, nullptr, nullptr, nullptr,
-                                          grad_x_next, grad_h_in, f_out, ws + w.urec_off,
+                                          grad_x_next, grad_h_in, f_out, nullptr, ws + w.urec_off,
                                           (float*)(ws + w.hrec_off), (float*)(ws + w.part_off),
                                           dev_status, (cudaStream_t)stream));
   return from_cuda(mhc::map_bwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
-                                         alpha, grad_x_next, grad_h_in, f_out,
+                                         alpha, grad_x_next, grad_h_in, f_out, nullptr,
                                          (float*)(ws + w.coef_off), (float*)(ws + w.part_off),
                                          dev_status, (cudaStream_t)stream));
 }
@@ -263,6 +227,109 @@ mhc_status mhc_backward(const mhc_params* p, const void* x, const float* phi, co
   if (st != MHC_OK) return st;
   return mhc_backward_apply(p, x, phi, grad_x_next, grad_h_in, grad_x, grad_phi, grad_b,
                             grad_alpha, grad_f_out, workspace, workspace_bytes, dev_status, stream);
+}
+
+size_t mhc_post_fused_workspace_size(const mhc_params* p) { return mhc_pre_workspace_size(p); }
+
+mhc_status mhc_post_fused(const mhc_params* p, const void* x, const void* f_out,
+                          const float* H_post, const float* H_res, const float* phi_next,
+                          const float* b_next, const float* alpha_next, void* x_next,
+                          float* H_pre_next, float* H_post_next, float* H_res_next,
+                          void* workspace, size_t workspace_bytes, int* dev_status,
+                          mhc_stream_t stream) {
+  mhc_status st = check_params(p);
+  if (st != MHC_OK) return st;
+  if (!aligned16(x) || !aligned16(f_out) || !aligned16(H_post) || !aligned16(H_res) ||
+      !aligned16(phi_next) || !aligned16(b_next) || !aligned16(alpha_next) || !aligned16(x_next) ||
+      !aligned16(H_pre_next) || !aligned16(H_post_next) || !aligned16(H_res_next))
+    return MHC_ERR_INVALID_ARG;
+  if (x_next == x || x_next == f_out) return MHC_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (use_tc(p)) {
+    const size_t need = mhc_post_fused_workspace_size(p);
+    if (workspace == nullptr || workspace_bytes < need || ((uintptr_t)workspace & 255u) != 0)
+      return MHC_ERR_WORKSPACE;
+    return from_cuda(mhc::post_map_tc_dispatch(p->T, p->C, p->t_max, p->eps, x, f_out, H_post,
+                                               H_res, phi_next, workspace, b_next, alpha_next,
+                                               x_next, H_pre_next, H_post_next, H_res_next,
+                                               dev_status, s));
+  }
+  // fp32 or n != 4: the post merge, then the mapping of x_next (both on the GPU)
+  st = from_cuda(mhc::post_dispatch(p->n, p->dtype, p->T, p->C, x, f_out, H_post, H_res, x_next, s));
+  if (st != MHC_OK) return st;
+  return from_cuda(mhc::map_fwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x_next,
+                                         phi_next, b_next, alpha_next, H_pre_next, H_post_next,
+                                         H_res_next, dev_status, s));
+}
+
+mhc_status mhc_layer_input(const mhc_params* p, const void* x, const float* H_pre, void* h_in,
+                           int* dev_status, mhc_stream_t stream) {
+  (void)dev_status;
+  mhc_status st = check_params(p);
+  if (st != MHC_OK) return st;
+  if (!aligned16(x) || !aligned16(H_pre) || !aligned16(h_in)) return MHC_ERR_INVALID_ARG;
+  return from_cuda(mhc::hin_dispatch(p->n, p->dtype, p->T, p->C, x, H_pre, h_in,
+                                     (cudaStream_t)stream));
+}
+
+mhc_status mhc_post_backward(const mhc_params* p, const void* x, const void* f_out,
+                             const float* H_post, const void* grad_x_next, void* grad_f_out,
+                             float* red, int* dev_status, mhc_stream_t stream) {
+  (void)dev_status;
+  mhc_status st = check_params(p);
+  if (st != MHC_OK) return st;
+  if (!aligned16(x) || !aligned16(f_out) || !aligned16(H_post) || !aligned16(grad_x_next) ||
+      !aligned16(grad_f_out) || !aligned16(red))
+    return MHC_ERR_INVALID_ARG;
+  if (grad_f_out == x || grad_f_out == f_out || grad_f_out == grad_x_next)
+    return MHC_ERR_INVALID_ARG;
+  return from_cuda(mhc::post_bwd_dispatch(p->n, p->dtype, p->T, p->C, x, f_out, H_post,
+                                          grad_x_next, grad_f_out, red, (cudaStream_t)stream));
+}
+
+size_t mhc_pre_backward_workspace_size(const mhc_params* p) {
+  if (check_params(p) != MHC_OK) return 0;
+  return bwd_layout(p).total;
+}
+
+mhc_status mhc_pre_backward(const mhc_params* p, const void* x, const float* phi, const float* b,
+                            const float* alpha, const void* grad_x_next, const void* grad_h_in,
+                            const float* red, void* grad_x, float* grad_phi, float* grad_b,
+                            float* grad_alpha, void* workspace, size_t workspace_bytes,
+                            int* dev_status, mhc_stream_t stream) {
+  mhc_status st = check_params(p);
+  if (st != MHC_OK) return st;
+  if (!aligned16(x) || !aligned16(phi) || !aligned16(b) || !aligned16(alpha) ||
+      !aligned16(grad_x_next) || !aligned16(grad_h_in) || !aligned16(red) || !aligned16(grad_x) ||
+      !aligned16(grad_phi) || !aligned16(grad_b) || !aligned16(grad_alpha))
+    return MHC_ERR_INVALID_ARG;
+  const BwdWorkspace w = bwd_layout(p);
+  st = check_workspace(w, workspace, workspace_bytes);
+  if (st != MHC_OK) return st;
+  char* ws = (char*)workspace;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (use_tc(p)) {
+    st = from_cuda(mhc::map_tc_dispatch(mhc::MAP_BWD_SPLIT, p->T, p->C, p->t_max, p->eps, x, phi,
+                                        ws + w.phi_off, b, alpha, nullptr, nullptr, nullptr,
+                                        nullptr, grad_h_in, nullptr, red, ws + w.urec_off,
+                                        (float*)(ws + w.hrec_off), (float*)(ws + w.part_off),
+                                        dev_status, s));
+    if (st != MHC_OK) return st;
+    return from_cuda(mhc::apply_tc_dispatch(p->T, p->C, x, ws + w.phi_off, grad_x_next, grad_h_in,
+                                            ws + w.urec_off, (const float*)(ws + w.hrec_off),
+                                            (const float*)(ws + w.part_off), w.nparts, grad_x,
+                                            nullptr, grad_phi, grad_b, grad_alpha,
+                                            (void*)(ws + w.apply_off), dev_status, s));
+  }
+  st = from_cuda(mhc::map_bwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
+                                       alpha, nullptr, grad_h_in, nullptr, red,
+                                       (float*)(ws + w.coef_off), (float*)(ws + w.part_off),
+                                       dev_status, s));
+  if (st != MHC_OK) return st;
+  return from_cuda(mhc::apply_dispatch(p->n, p->dtype, p->T, p->C, x, phi, grad_x_next, grad_h_in,
+                                       (const float*)(ws + w.coef_off),
+                                       (const float*)(ws + w.part_off), w.nparts, grad_x, nullptr,
+                                       grad_phi, grad_b, grad_alpha, s));
 }
 
 mhc_status mhc_sinkhorn_knopp(int n, int iters, int64_t B, const float* logits, float* out,

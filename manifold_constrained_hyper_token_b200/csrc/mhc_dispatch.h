@@ -1,0 +1,65 @@
+// mhc_dispatch.h -- the host-side launchers behind the C ABI (internal to
+// libmhc.so).  Each kernel file defines its launchers; mhc_api.cu and
+// mhc_noalloc.cu call them.  All pointers are device pointers; every launcher
+// is asynchronous on stream `s` and returns the launch's cudaError_t.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace mhc {
+
+// Mapping kernels: the forward; the backward's recompute with every
+// C-reduction; or the pre half of the backward in training order, which takes
+// <G_i, x_j> and <G_i, f_out> from the post half (`red`, [T][n*n + n]).
+// MAP_POSTFWD: layer l's post merge fused with layer l+1's forward mapping.
+enum MapMode { MAP_FWD = 0, MAP_BWD = 1, MAP_BWD_SPLIT = 2, MAP_POSTFWD = 3 };
+
+// k_sinkhorn.cu
+cudaError_t sinkhorn_dispatch(int n, int iters, int64_t B, const float* logits, float* out,
+                              int* st, cudaStream_t s);
+cudaError_t depth_amax_dispatch(int n, int64_t T, int L, const float* H, float* gf, float* gb,
+                                cudaStream_t s);
+// k_post.cu
+cudaError_t post_dispatch(int n, int dtype, int64_t T, int64_t C, const void* x, const void* f,
+                          const float* Hpost, const float* Hres, void* xn, cudaStream_t s);
+cudaError_t hin_dispatch(int n, int dtype, int64_t T, int64_t C, const void* x, const float* Hpre,
+                         void* h_in, cudaStream_t s);
+cudaError_t post_bwd_dispatch(int n, int dtype, int64_t T, int64_t C, const void* x, const void* f,
+                              const float* Hpost, const void* G, void* gf, float* red,
+                              cudaStream_t s);
+// k_map.cu (CUDA cores; red == nullptr selects MAP_BWD, else MAP_BWD_SPLIT)
+cudaError_t map_fwd_dispatch(int n, int dtype, int64_t T, int64_t C, int iters, float eps,
+                             const void* x, const float* phi, const float* b, const float* alpha,
+                             float* Hpre, float* Hpost, float* Hres, int* st, cudaStream_t s);
+cudaError_t map_bwd_dispatch(int n, int dtype, int64_t T, int64_t C, int iters, float eps,
+                             const void* x, const float* phi, const float* b, const float* alpha,
+                             const void* G, const void* g, const void* f, const float* red,
+                             float* coef, float* part, int* st, cudaStream_t s);
+// k_map_tc.cu (bf16, n = 4: projection on the tensor cores); mode is a MapMode
+cudaError_t map_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float eps, const void* x,
+                            const float* phi, void* phi_split, const float* b, const float* alpha,
+                            float* Hpre, float* Hpost, float* Hres, const void* G, const void* g,
+                            const void* f, const float* red, void* urec, float* hrec, float* part,
+                            int* st, cudaStream_t s);
+size_t map_tc_phi_bytes(int64_t C);
+cudaError_t post_map_tc_dispatch(int64_t T, int64_t C, int iters, float eps, const void* x,
+                                 const void* f, const float* Hpost_in, const float* Hres_in,
+                                 const float* phi_next, void* phi_split, const float* b_next,
+                                 const float* alpha_next, void* x_next, float* Hpre, float* Hpost,
+                                 float* Hres, int* st, cudaStream_t s);
+// k_apply_tc.cu (bf16, n = 4: phi u and grad_phi on the tensor cores);
+// gf == nullptr skips grad_f_out
+cudaError_t apply_tc_dispatch(int64_t T, int64_t C, const void* x, const void* phi_split,
+                              const void* G, const void* g, const void* urec, const float* hrec,
+                              const float* part, int nparts, void* gx, void* gf, float* gphi,
+                              float* gb, float* ga, void* scratch, int* st, cudaStream_t s);
+size_t apply_tc_scratch_bytes(int64_t T, int64_t C);
+// k_bwd.cu (CUDA cores); gf == nullptr skips grad_f_out
+cudaError_t apply_dispatch(int n, int dtype, int64_t T, int64_t C, const void* x, const float* phi,
+                           const void* G, const void* g, const float* coef, const float* part,
+                           int nparts, void* gx, void* gf, float* gphi, float* gb, float* ga,
+                           cudaStream_t s);
+
+}  // namespace mhc

@@ -18,17 +18,8 @@
 #include <mutex>
 
 #include "mhc_common.cuh"
+#include "mhc_dispatch.h"
 
-namespace mhc {
-cudaError_t map_bwd_dispatch(int n, int dtype, int64_t T, int64_t C, int iters, float eps,
-                             const void* x, const float* phi, const float* b, const float* alpha,
-                             const void* G, const void* g, const void* f, float* coef, float* part,
-                             int* st, cudaStream_t s);
-cudaError_t apply_dispatch(int n, int dtype, int64_t T, int64_t C, const void* x, const float* phi,
-                           const void* G, const void* g, const float* coef, const float* part,
-                           int nparts, void* gx, void* gf, float* gphi, float* gb, float* ga,
-                           cudaStream_t s);
-}  // namespace mhc
 
 namespace {
 
@@ -93,8 +84,8 @@ extern "C" mhc_status mhc_backward_noalloc(const mhc_params* p, const void* x, c
 
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = mhc::map_bwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
-                                        alpha, grad_x_next, grad_h_in, f_out, coef, part,
-                                        dev_status, s);
+                                        alpha, grad_x_next, grad_h_in, f_out, nullptr, coef,
+                                        part, dev_status, s);
   if (e != cudaSuccess) return MHC_ERR_CUDA;
   e = mhc::apply_dispatch(p->n, p->dtype, p->T, p->C, x, phi, grad_x_next, grad_h_in, coef, part,
                           nparts, grad_x, grad_f_out, grad_phi, grad_b, grad_alpha, s);

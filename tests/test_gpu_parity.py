@@ -205,6 +205,20 @@ def test_tiny_forward_with_linear_F(mhc, oracle_mod):
 
 
 # -------------------------------------------------------------- backward
+def _alpha_err(ga, ref_total, per_token):
+    """grad_alpha = sum_t dz_t . y_t is a scalar sum whose terms can cancel (the
+    sum can be thousands of times smaller than sum_t |dz_t . y_t|), so its error is
+    measured against that sum of magnitudes, the scale fp32 accumulation error is
+    proportional to: |gpu - ref| / max(|ref|, sum_t |term_t|)."""
+    scale = max(abs(ref_total), float(np.sum(np.abs(per_token))))
+    return abs(float(_np(ga).reshape(-1)[0]) - ref_total) / scale if scale > 0 else 0.0
+
+
+def _alpha_terms(oracle_mod, call, T):
+    """Per-token grad_alpha terms from the oracle, one token per call."""
+    return np.array([call(slice(t, t + 1))["grad_alpha"] for t in range(T)])
+
+
 def _check_bwd(mhc, oracle_mod, d, iters, dtype, eps=1e-6, idx=None, chunk=None):
     dd = _dev(d)
     st = _status()
@@ -219,6 +233,12 @@ def _check_bwd(mhc, oracle_mod, d, iters, dtype, eps=1e-6, idx=None, chunk=None)
     errs = dict(grad_x=rel_err(_np(gx), ref["grad_x"]), grad_f_out=rel_err(_np(gf), ref["grad_f_out"]),
                 grad_phi=rel_err(_np(gphi), ref["grad_phi"]), grad_b=rel_err(_np(gb), ref["grad_b"]),
                 grad_alpha=rel_err(_np(ga), np.array([ref["grad_alpha"]])))
+    if errs["grad_alpha"] >= tol:
+        a = float(d["alpha"][0])
+        terms = _alpha_terms(oracle_mod, lambda sl: oracle_mod.backward(
+            d["x"][sl], d["phi"], d["b"], a, d["f_out"][sl], d["grad_x_next"][sl],
+            d["grad_h_in"][sl], iters=iters, eps=eps), d["x"].shape[0])
+        errs["grad_alpha"] = _alpha_err(ga, ref["grad_alpha"], terms)
     assert all(v < tol for v in errs.values()), errs
     return errs, (gx, gphi, gb, ga, gf)
 
@@ -236,6 +256,125 @@ def test_backward_parity(mhc, oracle_mod, dtype, n, T, C, iters):
 def test_backward_large_alpha_parity(mhc, oracle_mod, dtype):
     d = _inputs(150, 4, 512, dtype, seed=19, alpha=1.0)
     _check_bwd(mhc, oracle_mod, d, 20, dtype)
+
+
+# ---------------------------- cross-layer fusion: post(l) + mapping(l+1)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("n,T,C", [(1, 33, 24), (2, 70, 64), (4, 300, 520), (4, 1, 8), (4, 129, 4096)])
+def test_post_fused_parity(mhc, oracle_mod, dtype, n, T, C):
+    """x_next and layer l+1's maps against the oracle's post then pre, and bit for bit
+    against the unfused mhc_post -> mhc_pre (the fused kernel maps the stored x_next)."""
+    from manifold_constrained_hyper_token_b200 import synth
+    d = _inputs(T, n, C, dtype, seed=5 * T + C + n)
+    a = float(d["alpha"][0])
+    fwd = oracle_mod.pre(d["x"], d["phi"], d["b"], a)
+    hp = torch.from_numpy(fwd["H_post"]).float()
+    hr = torch.from_numpy(fwd["H_res"]).float()
+    nxt = synth.layer_params(n, C, seed=1000 + n)
+    dd, dn = _dev(d), _dev(nxt)
+    st = _status()
+    xn, hpre, hpost, hres = mhc.mhc_post_fused(dd["x"], dd["f_out"], hp.cuda(), hr.cuda(),
+                                               dn["phi"], dn["b"], dn["alpha"], dev_status=st)
+    xn_u = mhc.mhc_post(dd["x"], dd["f_out"], hp.cuda(), hr.cuda())
+    _, hpre_u, hpost_u, hres_u = mhc.mhc_pre(xn_u, dn["phi"], dn["b"], dn["alpha"])
+    h_in = mhc.mhc_layer_input(xn, hpre)
+    h_in_u = mhc.mhc_pre(xn_u, dn["phi"], dn["b"], dn["alpha"])[0]
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ref_xn = oracle_mod.post(d["x"], d["f_out"], hp, hr)
+    ref = oracle_mod.pre(ref_xn, nxt["phi"], nxt["b"], float(nxt["alpha"][0]))
+    tol = TOL[dtype]
+    assert rel_err(_np(xn), ref_xn) < tol
+    for got, k in ((hpre, "H_pre"), (hpost, "H_post"), (hres, "H_res")):
+        assert rel_err(_np(got), ref[k]) < tol, k
+    assert torch.equal(xn, xn_u)
+    assert torch.equal(hpre, hpre_u) and torch.equal(hpost, hpost_u) and torch.equal(hres, hres_u)
+    assert torch.equal(h_in, h_in_u)
+
+
+# ------------------------------------- the backward in training order (split)
+def _hpost(T, n, seed):
+    """Forward-style H_post values in (0, 2), float32, shared by both sides."""
+    g = torch.Generator().manual_seed(seed)
+    return (2.0 * torch.rand(T, n, generator=g)).float()
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("n,T,C", [(1, 33, 24), (2, 70, 64), (4, 300, 520), (4, 1, 8)])
+def test_post_backward_parity(mhc, oracle_mod, dtype, n, T, C):
+    """grad_f_out within the I/O tolerance; red (fp32 sums over C of exact products)
+    within 1e-5."""
+    d = _inputs(T, n, C, dtype, seed=T + 7 * C + n)
+    hp = _hpost(T, n, seed=T + n)
+    dd = _dev(d)
+    gf, red = mhc.mhc_post_backward(dd["x"], dd["f_out"], hp.cuda(), dd["grad_x_next"])
+    ref = oracle_mod.post_backward(d["x"], d["f_out"], hp, d["grad_x_next"])
+    assert rel_err(_np(gf), ref["grad_f_out"]) < TOL[dtype]
+    assert rel_err(_np(red), ref["red"]) < 1e-5
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("n,T,C", [(1, 33, 24), (2, 70, 64), (4, 300, 520), (4, 1, 8)])
+@pytest.mark.parametrize("iters", [1, 20])
+def test_pre_backward_parity(mhc, oracle_mod, dtype, n, T, C, iters):
+    """The pre half on the same red as the oracle (the oracle's post-half red,
+    rounded to float32, fed to both sides)."""
+    d = _inputs(T, n, C, dtype, seed=3 * T + C + n + iters)
+    a = float(d["alpha"][0])
+    fwd = oracle_mod.pre(d["x"], d["phi"], d["b"], a, iters=iters)
+    red = torch.from_numpy(oracle_mod.post_backward(d["x"], d["f_out"], fwd["H_post"],
+                                                    d["grad_x_next"])["red"]).float()
+    dd = _dev(d)
+    gx, gphi, gb, ga = mhc.mhc_pre_backward(dd["x"], dd["phi"], dd["b"], dd["alpha"],
+                                            dd["grad_x_next"], dd["grad_h_in"], red.cuda(),
+                                            t_max=iters)
+    ref = oracle_mod.pre_backward(d["x"], d["phi"], d["b"], a, d["grad_x_next"], d["grad_h_in"],
+                                  red, iters=iters)
+    tol = TOL[dtype]
+    terms = _alpha_terms(oracle_mod, lambda sl: oracle_mod.pre_backward(
+        d["x"][sl], d["phi"], d["b"], a, d["grad_x_next"][sl], d["grad_h_in"][sl], red[sl],
+        iters=iters), T)
+    errs = dict(grad_x=rel_err(_np(gx), ref["grad_x"]), grad_phi=rel_err(_np(gphi), ref["grad_phi"]),
+                grad_b=rel_err(_np(gb), ref["grad_b"]),
+                grad_alpha=_alpha_err(ga, ref["grad_alpha"], terms))
+    assert all(v < tol for v in errs.values()), errs
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_split_backward_chain(mhc, oracle_mod, dtype):
+    """GPU forward, then post half -> pre half on the GPU, against the oracle's one-call
+    backward and against the GPU's one-call backward."""
+    T, n, C = 260, 4, 1000
+    d = _inputs(T, n, C, dtype, seed=77)
+    dd = _dev(d)
+    _, _, Hpost, _ = mhc.mhc_pre(dd["x"], dd["phi"], dd["b"], dd["alpha"])
+    gf, red = mhc.mhc_post_backward(dd["x"], dd["f_out"], Hpost, dd["grad_x_next"])
+    gx, gphi, gb, ga = mhc.mhc_pre_backward(dd["x"], dd["phi"], dd["b"], dd["alpha"],
+                                            dd["grad_x_next"], dd["grad_h_in"], red)
+    whole = mhc.mhc_backward(dd["x"], dd["phi"], dd["b"], dd["alpha"], dd["f_out"],
+                             dd["grad_x_next"], dd["grad_h_in"])
+    ref = oracle_mod.backward(d["x"], d["phi"], d["b"], float(d["alpha"][0]), d["f_out"],
+                              d["grad_x_next"], d["grad_h_in"])
+    tol = TOL[dtype]
+    for got, w, r in ((gx, whole[0], ref["grad_x"]), (gphi, whole[1], ref["grad_phi"]),
+                      (gb, whole[2], ref["grad_b"]), (gf, whole[4], ref["grad_f_out"])):
+        assert rel_err(_np(got), r) < tol
+        assert rel_err(_np(got), _np(w)) < tol
+    a = float(d["alpha"][0])
+    terms = _alpha_terms(oracle_mod, lambda sl: oracle_mod.backward(
+        d["x"][sl], d["phi"], d["b"], a, d["f_out"][sl], d["grad_x_next"][sl],
+        d["grad_h_in"][sl]), T)
+    assert _alpha_err(ga, ref["grad_alpha"], terms) < tol
+
+
+def test_pre_backward_small_workspace_rejected(mhc):
+    d = _dev(_inputs(64, 4, 256, torch.bfloat16, seed=5))
+    red = torch.zeros(64, 20, dtype=torch.float32, device="cuda")
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(mhc.MhcError) as e:
+        mhc.mhc_pre_backward(d["x"], d["phi"], d["b"], d["alpha"], d["grad_x_next"],
+                             d["grad_h_in"], red, workspace=ws)
+    assert e.value.status == 6
 
 
 def test_backward_is_deterministic(mhc):
