@@ -18,6 +18,13 @@
 // x itself is bf16, so the products are exact and only the fp32
 // accumulation order differs from the oracle.
 //
+// Split over channels: when one CTA per 128-token tile would leave SMs idle,
+// the tile's chunks are cut into kp contiguous parts, one CTA each.  A part
+// publishes its per-token sums (sum of squares, projection, C-reductions) as a
+// 52-float record; the tile's last part to finish (an atomic count) adds the
+// kp records in part order and runs the epilogue -- a fixed order, so repeated
+// calls give identical bits.
+//
 // Warp roles: warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs, warps
 // 2..9 (two per TMEM lane quarter, one per channel half) reduce the sum of
 // squares -- and in the backward the 24 C-reductions <G_i, x_j>, <g, x_i>,
@@ -40,6 +47,7 @@ constexpr int NWARPS = 11;           // TMA, MMA, 8 math warps, TMA stores (MAP_
 constexpr int STORE_WARP = 10;
 constexpr int NT = NWARPS * 32;
 constexpr uint32_t TMEM_COLS = 64;
+constexpr int KREC = 52;             // floats per part record: y[24] | ss | dots[24] | pad
 constexpr uint64_t WAIT_NS = 2000000000ull;  // 2 s per wait before giving up
 
 // MAP_FWD: the forward mapping.  MAP_BWD: the backward's recompute with all
@@ -126,7 +134,8 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
     float* __restrict__ Hpre_o, float* __restrict__ Hpost_o, float* __restrict__ Hres_o,
     __nv_bfloat16* __restrict__ urec_o, float* __restrict__ hrec_o, float* __restrict__ part_o,
     const float* __restrict__ red_in, const float* __restrict__ hpost_in,
-    const float* __restrict__ hres_in, int* status) {
+    const float* __restrict__ hres_in, int kp, float* __restrict__ kpart, int* __restrict__ kcnt,
+    int* status) {
   using namespace tcmap;
   using CFG = Cfg<MODE>;
   constexpr bool BWD = MODE == MAP_BWD || MODE == MAP_BWD_SPLIT;
@@ -142,6 +151,7 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + CFG::DATA);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * NS + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* bcast = reinterpret_cast<volatile int*>(tmem_slot + 2);
   auto full = [&](int s) { return tc::smem_u32(bars + s); };
   auto empty = [&](int s) { return tc::smem_u32(bars + NS + s); };
   const uint32_t done_bar = tc::smem_u32(bars + 2 * NS);
@@ -150,8 +160,11 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
   const uint32_t sdone_bar = tc::smem_u32(bars + 3 * NS + 2);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int64_t t0 = (int64_t)blockIdx.x * TM;
-  const int nch = (int)((C + CH - 1) / CH);
+  const int tile = blockIdx.x / kp, part = blockIdx.x % kp;
+  const int64_t t0 = (int64_t)tile * TM;
+  const int nch_all = (int)((C + CH - 1) / CH);
+  const int cbeg = (int)((int64_t)part * nch_all / kp);     // this part's chunks
+  const int nch = (int)((int64_t)(part + 1) * nch_all / kp) - cbeg;
   const int64_t K = (int64_t)N * C;
 
   if (threadIdx.x == 0) {
@@ -210,7 +223,7 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
         }
         const uint32_t base = tc::smem_u32(smem + s * CFG::STAGE);
         tc::mbar_arrive_expect_tx(full(s), CFG::STAGE);
-        const int c0 = cc * CH;
+        const int c0 = (cbeg + cc) * CH;
         for (int i = 0; i < N; ++i) {
           tc::tma_load_3d(base + CFG::X_OFF + i * XBOX, &tm_x, full(s), c0, i, (int)t0, pol_stream);
           tc::tma_load_3d(base + CFG::P_OFF + i * PBOX, &tm_phi, full(s), c0, i, 0, pol_keep);
@@ -277,7 +290,7 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
         const uint32_t base = tc::smem_u32(smem + s * CFG::STAGE);
 #pragma unroll
         for (int i = 0; i < N; ++i)
-          tc::tma_store_3d(&tm_G, base + CFG::X_OFF + i * XBOX, cc * CH, i, (int)t0);
+          tc::tma_store_3d(&tm_G, base + CFG::X_OFF + i * XBOX, (cbeg + cc) * CH, i, (int)t0);
         tc::bulk_commit();
         tc::bulk_wait_read<0>();
         tc::mbar_arrive(empty(s));
@@ -402,8 +415,9 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
       }
     }
     named_bar(1, 256);
+    // this CTA's sums for its chunks, per token (one thread per token)
+    float sst = 0.0f, yr[M], dt[BWD ? M : 1];
     if (ok && h == 0) {
-      // ------------------------------------------------- per-token epilogue
       tc::tc_fence_after();
       float d[NL];
       const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
@@ -420,15 +434,73 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
       tc::tmem_ld_wait();
 #pragma unroll
       for (int e = 0; e < 16; ++e) d[32 + e] = v16[e];
-
+      sst = red_ss[tok] + red_ss[TM + tok];
+#pragma unroll
+      for (int m = 0; m < M; ++m) yr[m] = d[m] + d[M + m];
+      if constexpr (BWD) {
+#pragma unroll
+        for (int m = 0; m < M; ++m) dt[m] = red_dt[(0 * M + m) * TM + tok] + red_dt[(1 * M + m) * TM + tok];
+      }
+    }
+    bool epi = ok;  // this CTA runs the per-token epilogue
+    if (kp > 1) {
+      // publish this part's sums and count it; the tile's last part adds the
+      // kp records in part order
+      if (ok && h == 0) {
+        float rec[KREC];
+#pragma unroll
+        for (int m = 0; m < M; ++m) rec[m] = yr[m];
+        rec[M] = sst;
+#pragma unroll
+        for (int m = 0; m < M; ++m) rec[M + 1 + m] = BWD ? dt[BWD ? m : 0] : 0.0f;
+        rec[2 * M + 1] = rec[2 * M + 2] = rec[2 * M + 3] = 0.0f;
+        float4* dst = reinterpret_cast<float4*>(kpart + (((int64_t)tile * kp + part) * TM + tok) * KREC);
+#pragma unroll
+        for (int e = 0; e < KREC / 4; ++e)
+          __stcg(dst + e, make_float4(rec[4 * e], rec[4 * e + 1], rec[4 * e + 2], rec[4 * e + 3]));
+      }
+      __threadfence();
+      named_bar(1, 256);
+      if (threadIdx.x == 64) *bcast = ok ? atomicAdd(kcnt + tile, 1) : -1;
+      named_bar(1, 256);
+      epi = ok && *bcast == kp - 1;
+      if (epi && h == 0) {
+        __threadfence();
+        sst = 0.0f;
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+          yr[m] = 0.0f;
+          if constexpr (BWD) dt[m] = 0.0f;
+        }
+        for (int pp = 0; pp < kp; ++pp) {
+          const float4* src =
+              reinterpret_cast<const float4*>(kpart + (((int64_t)tile * kp + pp) * TM + tok) * KREC);
+          float rec[KREC];
+#pragma unroll
+          for (int e = 0; e < KREC / 4; ++e) {
+            const float4 v = __ldcg(src + e);
+            rec[4 * e] = v.x; rec[4 * e + 1] = v.y; rec[4 * e + 2] = v.z; rec[4 * e + 3] = v.w;
+          }
+#pragma unroll
+          for (int m = 0; m < M; ++m) yr[m] += rec[m];
+          sst += rec[M];
+          if constexpr (BWD) {
+#pragma unroll
+            for (int m = 0; m < M; ++m) dt[m] += rec[M + 1 + m];
+          }
+        }
+      }
+      if (epi && threadIdx.x == 64) kcnt[tile] = 0;  // ready for the next call
+    }
+    if (epi && h == 0) {
+      // ------------------------------------------------- per-token epilogue
       const int64_t t = t0 + tok;
-      const float sst = red_ss[tok] + red_ss[TM + tok];
       const float r = sqrtf(sst / (float)K + eps);
       const float alpha = __ldg(alpha_p);
       float y[M], z[M];
 #pragma unroll
       for (int m = 0; m < M; ++m) {
-        y[m] = (d[m] + d[M + m]) / r;
+        y[m] = yr[m] / r;
         z[m] = fmaf(alpha, y[m], __ldg(bias + m));
       }
       float spre[N], spost[N];
@@ -465,16 +537,12 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
         // dL/dH_res and dL/dH_post: this CTA's C-reductions, or the post half's
         const float* rt = red_in + (t < T ? t : 0) * (N * N + N);
 #pragma unroll
-        for (int e = 0; e < N * N; ++e)
-          dA[e] = SPLIT ? (t < T ? __ldg(rt + e) : 0.0f)
-                        : red_dt[(0 * M + e) * TM + tok] + red_dt[(1 * M + e) * TM + tok];
+        for (int e = 0; e < N * N; ++e) dA[e] = SPLIT ? (t < T ? __ldg(rt + e) : 0.0f) : dt[e];
         sk_adjoint_ckpt<N>(dA, dzres, iters, ck + tok, TM, ck_period);
 #pragma unroll
         for (int i = 0; i < N; ++i) {
-          const float dpre = red_dt[(0 * M + N * N + i) * TM + tok] + red_dt[(1 * M + N * N + i) * TM + tok];
-          const float dpost = SPLIT ? (t < T ? __ldg(rt + N * N + i) : 0.0f)
-                                    : red_dt[(0 * M + N * N + N + i) * TM + tok] +
-                                          red_dt[(1 * M + N * N + N + i) * TM + tok];
+          const float dpre = dt[N * N + i];
+          const float dpost = SPLIT ? (t < T ? __ldg(rt + N * N + i) : 0.0f) : dt[N * N + N + i];
           dz[i] = dpre * spre[i] * (1.0f - spre[i]);
           dz[N + i] = dpost * 2.0f * spost[i] * (1.0f - spost[i]);
         }
@@ -522,11 +590,11 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
     }
     if constexpr (BWD) {
       named_bar(1, 256);
-      if (ok && h == 0 && q == 0 && lane <= M) {
-        // this CTA's share of grad_b / grad_alpha, summed in token order
+      if (epi && h == 0 && q == 0 && lane <= M) {
+        // this tile's share of grad_b / grad_alpha, summed in token order
         float a = 0.0f;
         for (int k = 0; k < TM; ++k) a += dzs[lane * TM + k];
-        part_o[(int64_t)blockIdx.x * Coef<N>::DZ_SIZE + lane] = a;
+        part_o[(int64_t)tile * Coef<N>::DZ_SIZE + lane] = a;
       }
     }
   }
@@ -593,23 +661,85 @@ static int ck_period_for(int iters, size_t stage_bytes) {
 
 size_t map_tc_phi_bytes(int64_t C) { return (size_t)tcmap::NL * tcmap::N * C * 2; }
 
+static int map_device_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+// Parts per 128-token tile.  The time of a launch is about
+//   waves(kp) * (chunks per part + F),   waves(kp) = ceil(tiles * kp / SMs),
+// where F = 8 chunks is a CTA's fixed cost (setup, pipeline fill and drain,
+// the part records and their combine), measured at T = 16384, C = 7168: there
+// one part per tile (one wave of 128 CTAs) beats eight parts (1024 CTAs).
+// Small T is where the split pays: at T = 4096 one part per tile would leave
+// 116 of 148 SMs idle.
+static int map_tc_kp(int64_t T, int64_t C) {
+  using namespace tcmap;
+  const int64_t ntt = (T + TM - 1) / TM;
+  const int nch = (int)((C + Cfg<MAP_FWD>::CH - 1) / Cfg<MAP_FWD>::CH);
+  const int sms = map_device_sms();
+  constexpr double kFixedChunks = 8.0;
+  int kmax = nch / 4;
+  if (kmax > 32) kmax = 32;
+  if (kmax < 1) kmax = 1;
+  int best = 1;
+  double best_cost = 0.0;
+  for (int kp = 1; kp <= kmax; ++kp) {
+    const int64_t waves = (ntt * kp + sms - 1) / sms;
+    const double cost = (double)waves * ((double)nch / kp + kFixedChunks);
+    if (kp == 1 || cost < best_cost * 0.97) {  // a new split must win by 3 %
+      best_cost = cost;
+      best = kp;
+    }
+  }
+  return best;
+}
+
+static size_t round256(size_t v) { return (v + 255) / 256 * 256; }
+
+// Part records [tiles][kp][128][KREC] fp32 and per-tile counters; 0 when one
+// CTA per tile fills the SMs.
+size_t map_tc_scratch_bytes(int64_t T, int64_t C) {
+  using namespace tcmap;
+  const int kp = map_tc_kp(T, C);
+  if (kp == 1) return 0;
+  const int64_t ntt = (T + TM - 1) / TM;
+  return round256((size_t)ntt * kp * TM * KREC * 4) + round256((size_t)ntt * 4);
+}
+
 template <int MODE>
 static cudaError_t launch_map_tc(const CUtensorMap& mx, const CUtensorMap& mp, const CUtensorMap& mG,
                                  const CUtensorMap& mg, const CUtensorMap& mf, int64_t T, int64_t C,
                                  int iters, float eps, const float* b, const float* alpha,
                                  float* Hpre, float* Hpost, float* Hres, void* urec, float* hrec,
-                                 float* part, const float* red, int* st, cudaStream_t s,
-                                 const float* hpost_in = nullptr, const float* hres_in = nullptr) {
+                                 float* part, const float* red, void* kscratch, int* st,
+                                 cudaStream_t s, const float* hpost_in = nullptr,
+                                 const float* hres_in = nullptr) {
   using namespace tcmap;
   auto kern = k_map_tc<MODE>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<MODE>::SMEM);
   if (e != cudaSuccess) return e;
-  const unsigned grid = (unsigned)((T + TM - 1) / TM);
+  const int64_t ntt = (T + TM - 1) / TM;
+  const int kp = map_tc_kp(T, C);
+  float* kpart = nullptr;
+  int* kcnt = nullptr;
+  if (kp > 1) {
+    if (kscratch == nullptr) return cudaErrorInvalidValue;
+    kpart = (float*)kscratch;
+    kcnt = (int*)((char*)kscratch + round256((size_t)ntt * kp * TM * KREC * 4));
+    // per-tile part counters start at zero (each tile's last part resets its own)
+    e = cudaMemsetAsync(kcnt, 0, (size_t)ntt * sizeof(int), s);
+    if (e != cudaSuccess) return e;
+  }
+  const unsigned grid = (unsigned)(ntt * kp);
   const int P = (MODE == MAP_BWD || MODE == MAP_BWD_SPLIT) ? ck_period_for(iters, Cfg<MODE>::DATA) : 1;
   kern<<<grid, NT, Cfg<MODE>::SMEM, s>>>(mx, mp, mG, mg, mf, T, C, iters, eps, P, b, alpha, Hpre,
                                          Hpost, Hres, (__nv_bfloat16*)urec, hrec, part, red,
-                                         hpost_in, hres_in, st);
+                                         hpost_in, hres_in, kp, kpart, kcnt, st);
   return cudaGetLastError();
 }
 
@@ -617,7 +747,7 @@ cudaError_t map_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float eps
                             const float* phi, void* phi_split, const float* b, const float* alpha,
                             float* Hpre, float* Hpost, float* Hres, const void* G, const void* g,
                             const void* f, const float* red, void* urec, float* hrec, float* part,
-                            int* st, cudaStream_t s) {
+                            void* kscratch, int* st, cudaStream_t s) {
   using namespace tcmap;
   const int64_t K = (int64_t)N * C;
   k_phi_split<<<(unsigned)((K + 255) / 256), 256, 0, s>>>(K, phi, (__nv_bfloat16*)phi_split);
@@ -629,13 +759,13 @@ cudaError_t map_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float eps
   switch (mode) {
     case MAP_FWD:
       return launch_map_tc<MAP_FWD>(mx, mp, mG, mg, mf, T, C, iters, eps, b, alpha, Hpre, Hpost,
-                                    Hres, nullptr, nullptr, nullptr, nullptr, st, s);
+                                    Hres, nullptr, nullptr, nullptr, nullptr, kscratch, st, s);
     case MAP_BWD:
       return launch_map_tc<MAP_BWD>(mx, mp, mG, mg, mf, T, C, iters, eps, b, alpha, nullptr,
-                                    nullptr, nullptr, urec, hrec, part, nullptr, st, s);
+                                    nullptr, nullptr, urec, hrec, part, nullptr, kscratch, st, s);
     case MAP_BWD_SPLIT:
       return launch_map_tc<MAP_BWD_SPLIT>(mx, mp, mG, mg, mf, T, C, iters, eps, b, alpha, nullptr,
-                                          nullptr, nullptr, urec, hrec, part, red, st, s);
+                                          nullptr, nullptr, urec, hrec, part, red, kscratch, st, s);
     default:
       return cudaErrorInvalidValue;
   }
@@ -648,7 +778,7 @@ cudaError_t post_map_tc_dispatch(int64_t T, int64_t C, int iters, float eps, con
                                  const void* f, const float* Hpost_in, const float* Hres_in,
                                  const float* phi_next, void* phi_split, const float* b_next,
                                  const float* alpha_next, void* x_next, float* Hpre, float* Hpost,
-                                 float* Hres, int* st, cudaStream_t s) {
+                                 float* Hres, void* kscratch, int* st, cudaStream_t s) {
   using namespace tcmap;
   const int64_t K = (int64_t)N * C;
   k_phi_split<<<(unsigned)((K + 255) / 256), 256, 0, s>>>(K, phi_next,
@@ -670,8 +800,8 @@ cudaError_t post_map_tc_dispatch(int64_t T, int64_t C, int iters, float eps, con
   e = make_tmap_bf16(&mf, f, 2, d2, s2, b2, CU_TENSOR_MAP_SWIZZLE_64B);
   if (e != cudaSuccess) return e;
   return launch_map_tc<MAP_POSTFWD>(mx, mp, mG, mg, mf, T, C, iters, eps, b_next, alpha_next, Hpre,
-                                    Hpost, Hres, nullptr, nullptr, nullptr, nullptr, st, s,
-                                    Hpost_in, Hres_in);
+                                    Hpost, Hres, nullptr, nullptr, nullptr, nullptr, kscratch, st,
+                                    s, Hpost_in, Hres_in);
 }
 
 }  // namespace mhc

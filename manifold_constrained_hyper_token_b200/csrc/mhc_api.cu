@@ -18,7 +18,7 @@ mhc_status check_params(const mhc_params* p) {
   if (!p) return MHC_ERR_INVALID_ARG;
   if (p->T < 1 || p->C < 8 || (p->C % 8) != 0 || p->t_max < 0) return MHC_ERR_INVALID_ARG;
   if (!(p->eps >= 0.0f) || !isfinite(p->eps)) return MHC_ERR_INVALID_ARG;
-  if (p->n != 1 && p->n != 2 && p->n != 4) return MHC_ERR_UNSUPPORTED;
+  if (p->n != 1 && p->n != 2 && p->n != 4 && p->n != 8) return MHC_ERR_UNSUPPORTED;
   if (p->dtype != MHC_DTYPE_F32 && p->dtype != MHC_DTYPE_BF16) return MHC_ERR_UNSUPPORTED;
   // token count is bounded by the 1-D grid of the mapping kernel (64 tokens per CTA)
   if (p->T > (int64_t)64 * 0x7fffffffLL) return MHC_ERR_INVALID_ARG;
@@ -33,6 +33,7 @@ int coef_size(int n) {
   switch (n) {
     case 1: return mhc::Coef<1>::SIZE;
     case 2: return mhc::Coef<2>::SIZE;
+    case 8: return mhc::Coef<8>::SIZE;
     default: return mhc::Coef<4>::SIZE;
   }
 }
@@ -40,6 +41,7 @@ int dz_size(int n) {
   switch (n) {
     case 1: return mhc::Coef<1>::DZ_SIZE;
     case 2: return mhc::Coef<2>::DZ_SIZE;
+    case 8: return mhc::Coef<8>::DZ_SIZE;
     default: return mhc::Coef<4>::DZ_SIZE;
   }
 }
@@ -54,7 +56,7 @@ bool use_tc(const mhc_params* p) { return p->dtype == MHC_DTYPE_BF16 && p->n == 
 // the bf16 split copy of phi^T that the mapping MMA reads, and the apply
 // kernel's grad_phi partials and slice counters.
 struct BwdWorkspace {
-  size_t coef_off, urec_off, hrec_off, part_off, phi_off, apply_off, total;
+  size_t coef_off, urec_off, hrec_off, part_off, phi_off, apply_off, kmap_off, total;
   int nparts;
 };
 
@@ -79,6 +81,8 @@ BwdWorkspace bwd_layout(const mhc_params* p) {
   off = round_up(off + (tc ? mhc::map_tc_phi_bytes(p->C) : 0), 256);
   w.apply_off = off;
   off = round_up(off + (tc ? mhc::apply_tc_scratch_bytes(p->T, p->C) : 0), 256);
+  w.kmap_off = off;
+  off = round_up(off + (tc ? mhc::map_tc_scratch_bytes(p->T, p->C) : 0), 256);
   w.total = off;
   return w;
 }
@@ -111,7 +115,10 @@ const char* mhc_status_string(int status) {
 
 size_t mhc_pre_workspace_size(const mhc_params* p) {
   if (check_params(p) != MHC_OK) return 0;
-  return use_tc(p) ? round_up(mhc::map_tc_phi_bytes(p->C), 256) : 0;
+  // the bf16 split copy of phi, then the channel-split mapping's scratch
+  return use_tc(p) ? round_up(mhc::map_tc_phi_bytes(p->C), 256) +
+                         round_up(mhc::map_tc_scratch_bytes(p->T, p->C), 256)
+                   : 0;
 }
 
 mhc_status mhc_pre(const mhc_params* p, const void* x, const float* phi, const float* b,
@@ -127,9 +134,11 @@ mhc_status mhc_pre(const mhc_params* p, const void* x, const float* phi, const f
     const size_t need = mhc_pre_workspace_size(p);
     if (workspace == nullptr || workspace_bytes < need || ((uintptr_t)workspace & 255u) != 0)
       return MHC_ERR_WORKSPACE;
-    st = from_cuda(mhc::map_tc_dispatch(mhc::MAP_FWD, p->T, p->C, p->t_max, p->eps, x, phi,
-                                        workspace, b, alpha, H_pre, H_post, H_res, nullptr,
-                                        nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+    char* ws = (char*)workspace;
+    st = from_cuda(mhc::map_tc_dispatch(mhc::MAP_FWD, p->T, p->C, p->t_max, p->eps, x, phi, ws, b,
+                                        alpha, H_pre, H_post, H_res, nullptr, nullptr, nullptr,
+                                        nullptr, nullptr, nullptr, nullptr,
+                                        ws + round_up(mhc::map_tc_phi_bytes(p->C), 256),
                                         dev_status, s));
   } else {
     st = from_cuda(mhc::map_fwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
@@ -175,6 +184,7 @@ mhc_status mhc_backward_map(const mhc_params* p, const void* x, const float* phi
                                           ws + w.phi_off, b, alpha, nullptr, nullptr, nullptr,
                                           grad_x_next, grad_h_in, f_out, nullptr, ws + w.urec_off,
                                           (float*)(ws + w.hrec_off), (float*)(ws + w.part_off),
+                                          ws + w.kmap_off,
                                           dev_status, (cudaStream_t)stream));
   return from_cuda(mhc::map_bwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
                                          alpha, grad_x_next, grad_h_in, f_out, nullptr,
@@ -249,10 +259,11 @@ mhc_status mhc_post_fused(const mhc_params* p, const void* x, const void* f_out,
     const size_t need = mhc_post_fused_workspace_size(p);
     if (workspace == nullptr || workspace_bytes < need || ((uintptr_t)workspace & 255u) != 0)
       return MHC_ERR_WORKSPACE;
-    return from_cuda(mhc::post_map_tc_dispatch(p->T, p->C, p->t_max, p->eps, x, f_out, H_post,
-                                               H_res, phi_next, workspace, b_next, alpha_next,
-                                               x_next, H_pre_next, H_post_next, H_res_next,
-                                               dev_status, s));
+    char* ws = (char*)workspace;
+    return from_cuda(mhc::post_map_tc_dispatch(
+        p->T, p->C, p->t_max, p->eps, x, f_out, H_post, H_res, phi_next, ws, b_next, alpha_next,
+        x_next, H_pre_next, H_post_next, H_res_next,
+        ws + round_up(mhc::map_tc_phi_bytes(p->C), 256), dev_status, s));
   }
   // fp32 or n != 4: the post merge, then the mapping of x_next (both on the GPU)
   st = from_cuda(mhc::post_dispatch(p->n, p->dtype, p->T, p->C, x, f_out, H_post, H_res, x_next, s));
@@ -313,7 +324,7 @@ mhc_status mhc_pre_backward(const mhc_params* p, const void* x, const float* phi
                                         ws + w.phi_off, b, alpha, nullptr, nullptr, nullptr,
                                         nullptr, grad_h_in, nullptr, red, ws + w.urec_off,
                                         (float*)(ws + w.hrec_off), (float*)(ws + w.part_off),
-                                        dev_status, s));
+                                        ws + w.kmap_off, dev_status, s));
     if (st != MHC_OK) return st;
     return from_cuda(mhc::apply_tc_dispatch(p->T, p->C, x, ws + w.phi_off, grad_x_next, grad_h_in,
                                             ws + w.urec_off, (const float*)(ws + w.hrec_off),

@@ -42,13 +42,16 @@ cudaError_t map_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float eps
                             const float* phi, void* phi_split, const float* b, const float* alpha,
                             float* Hpre, float* Hpost, float* Hres, const void* G, const void* g,
                             const void* f, const float* red, void* urec, float* hrec, float* part,
-                            int* st, cudaStream_t s);
+                            void* kscratch, int* st, cudaStream_t s);
 size_t map_tc_phi_bytes(int64_t C);
+// scratch of the channel-split mapping (part records, counters); kscratch
+// must hold this many bytes, 256-byte aligned (may be null when it is 0)
+size_t map_tc_scratch_bytes(int64_t T, int64_t C);
 cudaError_t post_map_tc_dispatch(int64_t T, int64_t C, int iters, float eps, const void* x,
                                  const void* f, const float* Hpost_in, const float* Hres_in,
                                  const float* phi_next, void* phi_split, const float* b_next,
                                  const float* alpha_next, void* x_next, float* Hpre, float* Hpost,
-                                 float* Hres, int* st, cudaStream_t s);
+                                 float* Hres, void* kscratch, int* st, cudaStream_t s);
 // k_apply_tc.cu (bf16, n = 4: phi u and grad_phi on the tensor cores);
 // gf == nullptr skips grad_f_out
 cudaError_t apply_tc_dispatch(int64_t T, int64_t C, const void* x, const void* phi_split,
