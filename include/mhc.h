@@ -94,7 +94,7 @@ typedef enum mhc_dtype {
 
 /* Problem description shared by mhc_pre / mhc_post / mhc_backward. */
 typedef struct mhc_params {
-  int32_t n;      /* streams; this build supports n in {1, 2, 4}              */
+  int32_t n;      /* streams; this build supports n in {1, 2, 4, 8}           */
   int32_t t_max;  /* Sinkhorn-Knopp iterations (row then column pass), >= 0   */
   int64_t T;      /* tokens, >= 1                                             */
   int64_t C;      /* channels per stream, >= 8 and a multiple of 8            */

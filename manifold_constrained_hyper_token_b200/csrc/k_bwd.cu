@@ -63,16 +63,18 @@ __global__ void __launch_bounds__(bwdk::NT) k_bwd_apply(
     // grad_b and grad_alpha: add the mapping kernel's per-CTA partial sums.
     // Warp w takes partials w, w + NW, ... in order; the NW results are then
     // added in warp order -- a fixed order, so repeated calls agree bitwise.
+    // (M + 1 columns can exceed a warp's 32 lanes: n = 8 has 81)
     float* wsum = sm;  // [NW][M + 1]
-    float s = 0.0f;
-    if (lane <= M)
-      for (int q = warp; q < nparts; q += NW) s += __ldg(part + (int64_t)q * CF::DZ_SIZE + lane);
-    if (lane <= M) wsum[warp * (M + 1) + lane] = s;
+    for (int col = lane; col <= M; col += 32) {
+      float s = 0.0f;
+      for (int q = warp; q < nparts; q += NW) s += __ldg(part + (int64_t)q * CF::DZ_SIZE + col);
+      wsum[warp * (M + 1) + col] = s;
+    }
     __syncthreads();
-    if (threadIdx.x <= M) {
+    for (int col = threadIdx.x; col <= M; col += NT) {
       float a = 0.0f;
-      for (int w = 0; w < NW; ++w) a += wsum[w * (M + 1) + threadIdx.x];
-      if (threadIdx.x < M) grad_b[threadIdx.x] = a;
+      for (int w = 0; w < NW; ++w) a += wsum[w * (M + 1) + col];
+      if (col < M) grad_b[col] = a;
       else *grad_alpha = a;
     }
   }
@@ -204,6 +206,7 @@ cudaError_t apply_dispatch(int n, int dtype, int64_t T, int64_t C, const void* x
     MHC_APPLY(1)
     MHC_APPLY(2)
     MHC_APPLY(4)
+    MHC_APPLY(8)
     default: return cudaErrorInvalidValue;
   }
 #undef MHC_APPLY

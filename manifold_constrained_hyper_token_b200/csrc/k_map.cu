@@ -373,6 +373,7 @@ cudaError_t map_fwd_dispatch(int n, int dtype, int64_t T, int64_t C, int iters, 
     MHC_MAPF(1)
     MHC_MAPF(2)
     MHC_MAPF(4)
+    MHC_MAPF(8)
     default: return cudaErrorInvalidValue;
   }
 #undef MHC_MAPF
@@ -406,6 +407,7 @@ cudaError_t map_bwd_dispatch(int n, int dtype, int64_t T, int64_t C, int iters, 
     MHC_MAPB(1)
     MHC_MAPB(2)
     MHC_MAPB(4)
+    MHC_MAPB(8)
     default: return cudaErrorInvalidValue;
   }
 #undef MHC_MAPB

@@ -216,6 +216,7 @@ cudaError_t post_dispatch(int n, int dtype, int64_t T, int64_t C, const void* x,
     MHC_POST_CASE(1)
     MHC_POST_CASE(2)
     MHC_POST_CASE(4)
+    MHC_POST_CASE(8)
     default: return cudaErrorInvalidValue;
   }
 #undef MHC_POST_CASE
@@ -244,6 +245,7 @@ cudaError_t post_bwd_dispatch(int n, int dtype, int64_t T, int64_t C, const void
     MHC_PBWD_CASE(1)
     MHC_PBWD_CASE(2)
     MHC_PBWD_CASE(4)
+    MHC_PBWD_CASE(8)
     default: return cudaErrorInvalidValue;
   }
 #undef MHC_PBWD_CASE
@@ -259,6 +261,7 @@ cudaError_t hin_dispatch(int n, int dtype, int64_t T, int64_t C, const void* x, 
     MHC_HIN_CASE(1)
     MHC_HIN_CASE(2)
     MHC_HIN_CASE(4)
+    MHC_HIN_CASE(8)
     default: return cudaErrorInvalidValue;
   }
 #undef MHC_HIN_CASE

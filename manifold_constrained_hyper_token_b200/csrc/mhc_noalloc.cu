@@ -57,7 +57,7 @@ extern "C" mhc_status mhc_backward_noalloc(const mhc_params* p, const void* x, c
                                            float* grad_alpha, void* grad_f_out, int* dev_status,
                                            mhc_stream_t stream) {
   if (p == nullptr) return MHC_ERR_INVALID_ARG;
-  if (p->n != 1 && p->n != 2 && p->n != 4) return MHC_ERR_UNSUPPORTED;
+  if (p->n != 1 && p->n != 2 && p->n != 4 && p->n != 8) return MHC_ERR_UNSUPPORTED;
   if (p->dtype != MHC_DTYPE_F32 && p->dtype != MHC_DTYPE_BF16) return MHC_ERR_UNSUPPORTED;
   const size_t need = mhc_backward_workspace_size(p);
   if (need == 0) return MHC_ERR_INVALID_ARG;  // a size, t_max or eps out of range
@@ -76,6 +76,7 @@ extern "C" mhc_status mhc_backward_noalloc(const mhc_params* p, const void* x, c
   // before the second reads them, so no part of the scratch needs clearing.
   const int coef_floats = p->n == 1   ? mhc::Coef<1>::SIZE
                           : p->n == 2 ? mhc::Coef<2>::SIZE
+                          : p->n == 8 ? mhc::Coef<8>::SIZE
                                       : mhc::Coef<4>::SIZE;
   const int nparts = (int)((p->T + 63) / 64);
   char* ws = (char*)scratch;

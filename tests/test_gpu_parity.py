@@ -125,7 +125,7 @@ def test_depth_amax_sinkhorn_batch(mhc, oracle_mod):
 
 # ----------------------------------------------------------------- post
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
-@pytest.mark.parametrize("n", [1, 2, 4])
+@pytest.mark.parametrize("n", [1, 2, 4, 8])
 @pytest.mark.parametrize("T,C", [(1, 8), (67, 24), (130, 256)])
 def test_post_parity(mhc, oracle_mod, dtype, n, T, C):
     d = _inputs(T, n, C, dtype, seed=T + C)
@@ -161,7 +161,7 @@ def _check_pre(mhc, oracle_mod, d, iters, dtype, eps=1e-6):
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
-@pytest.mark.parametrize("n", [1, 2, 4])
+@pytest.mark.parametrize("n", [1, 2, 4, 8])
 @pytest.mark.parametrize("T,C", [(1, 8), (65, 24), (130, 256)])
 @pytest.mark.parametrize("iters", [0, 1, 20])
 def test_pre_parity(mhc, oracle_mod, dtype, n, T, C, iters):
@@ -244,7 +244,7 @@ def _check_bwd(mhc, oracle_mod, d, iters, dtype, eps=1e-6, idx=None, chunk=None)
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
-@pytest.mark.parametrize("n", [1, 2, 4])
+@pytest.mark.parametrize("n", [1, 2, 4, 8])
 @pytest.mark.parametrize("T,C", [(1, 8), (65, 24), (130, 256)])
 @pytest.mark.parametrize("iters", [0, 1, 20])
 def test_backward_parity(mhc, oracle_mod, dtype, n, T, C, iters):
@@ -260,7 +260,8 @@ def test_backward_large_alpha_parity(mhc, oracle_mod, dtype):
 
 # ---------------------------- cross-layer fusion: post(l) + mapping(l+1)
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
-@pytest.mark.parametrize("n,T,C", [(1, 33, 24), (2, 70, 64), (4, 300, 520), (4, 1, 8), (4, 129, 4096)])
+@pytest.mark.parametrize("n,T,C", [(1, 33, 24), (2, 70, 64), (4, 300, 520), (4, 1, 8), (4, 129, 4096),
+                                   (8, 65, 136)])
 def test_post_fused_parity(mhc, oracle_mod, dtype, n, T, C):
     """x_next and layer l+1's maps against the oracle's post then pre, and bit for bit
     against the unfused mhc_post -> mhc_pre (the fused kernel maps the stored x_next)."""
@@ -300,7 +301,7 @@ def _hpost(T, n, seed):
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
-@pytest.mark.parametrize("n,T,C", [(1, 33, 24), (2, 70, 64), (4, 300, 520), (4, 1, 8)])
+@pytest.mark.parametrize("n,T,C", [(1, 33, 24), (2, 70, 64), (4, 300, 520), (4, 1, 8), (8, 65, 136)])
 def test_post_backward_parity(mhc, oracle_mod, dtype, n, T, C):
     """grad_f_out within the I/O tolerance; red (fp32 sums over C of exact products)
     within 1e-5."""
@@ -314,7 +315,7 @@ def test_post_backward_parity(mhc, oracle_mod, dtype, n, T, C):
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
-@pytest.mark.parametrize("n,T,C", [(1, 33, 24), (2, 70, 64), (4, 300, 520), (4, 1, 8)])
+@pytest.mark.parametrize("n,T,C", [(1, 33, 24), (2, 70, 64), (4, 300, 520), (4, 1, 8), (8, 65, 136)])
 @pytest.mark.parametrize("iters", [1, 20])
 def test_pre_backward_parity(mhc, oracle_mod, dtype, n, T, C, iters):
     """The pre half on the same red as the oracle (the oracle's post-half red,
