@@ -29,7 +29,8 @@
 // 2..9 (two per TMEM lane quarter, one per channel half) reduce the sum of
 // squares -- and in the backward the 24 C-reductions <G_i, x_j>, <g, x_i>,
 // <G_i, f> -- from the same stages, then run the per-token epilogue (gates,
-// Sinkhorn, adjoint) with one thread per token.  Every wait is bounded; on
+// Sinkhorn, adjoint) with one thread per token; warp 10 stores x_next in the
+// fused post-merge mode.  Every wait is bounded; on
 // timeout the kernel records MHC_ERR_TIMEOUT, drains what it issued, frees
 // TMEM and returns.
 #include "mhc_common.cuh"
