@@ -96,7 +96,7 @@ typedef enum mhc_dtype {
 typedef struct mhc_params {
   int32_t n;      /* streams; this build supports n in {1, 2, 4, 8}           */
   int32_t t_max;  /* Sinkhorn-Knopp iterations (row then column pass), >= 0   */
-  int64_t T;      /* tokens, >= 1                                             */
+  int64_t T;      /* tokens, 1 <= T <= 2^31 - 257 (32-bit tile coordinates)    */
   int64_t C;      /* channels per stream, >= 8 and a multiple of 8            */
   float eps;      /* RMS epsilon added to the mean square, >= 0               */
   int32_t dtype;  /* mhc_dtype of x, f_out, h_in, x_next and the activation

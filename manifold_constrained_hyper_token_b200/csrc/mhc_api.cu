@@ -20,8 +20,9 @@ mhc_status check_params(const mhc_params* p) {
   if (!(p->eps >= 0.0f) || !isfinite(p->eps)) return MHC_ERR_INVALID_ARG;
   if (p->n != 1 && p->n != 2 && p->n != 4 && p->n != 8) return MHC_ERR_UNSUPPORTED;
   if (p->dtype != MHC_DTYPE_F32 && p->dtype != MHC_DTYPE_BF16) return MHC_ERR_UNSUPPORTED;
-  // token count is bounded by the 1-D grid of the mapping kernel (64 tokens per CTA)
-  if (p->T > (int64_t)64 * 0x7fffffffLL) return MHC_ERR_INVALID_ARG;
+  // tile coordinates of the TMA copies are 32-bit signed: keep T (and a tile
+  // past it) inside that range
+  if (p->T > (int64_t)0x7fffffffLL - 256) return MHC_ERR_INVALID_ARG;
   return MHC_OK;
 }
 
