@@ -48,12 +48,12 @@ def _load():
         i64, i32, dbl = ctypes.c_int64, ctypes.c_int, ctypes.c_double
         lib.orc_sinkhorn.argtypes = [i32, i32, i64, _D, _D]
         lib.orc_sinkhorn_backward.argtypes = [i32, i32, i64, _D, _D, _D]
-        lib.orc_pre.argtypes = [i32, i64, i64, i32, dbl, _D, _D, _D, dbl, _D, _D, _D, _D, _D, _D]
+        lib.orc_pre.argtypes = [i32, i64, i64, i32, dbl, _D, _D, _D, _D, _D, _D, _D, _D, _D, _D]
         lib.orc_post.argtypes = [i32, i64, i64, _D, _D, _D, _D, _D]
-        lib.orc_backward.argtypes = [i32, i64, i64, i32, dbl, _D, _D, _D, dbl, _D, _D, _D,
+        lib.orc_backward.argtypes = [i32, i64, i64, i32, dbl, _D, _D, _D, _D, _D, _D, _D,
                                      _D, _D, _D, _D, _D]
         lib.orc_post_backward.argtypes = [i32, i64, i64, _D, _D, _D, _D, _D, _D]
-        lib.orc_pre_backward.argtypes = [i32, i64, i64, i32, dbl, _D, _D, _D, dbl, _D, _D, _D,
+        lib.orc_pre_backward.argtypes = [i32, i64, i64, i32, dbl, _D, _D, _D, _D, _D, _D, _D,
                                          _D, _D, _D, _D]
         lib.orc_depth_amax.argtypes = [i32, i64, i32, _D, _D, _D]
         lib.orc_num_threads.restype = i32
@@ -74,6 +74,17 @@ def _f64(a) -> np.ndarray:
 
 def _p(a: np.ndarray):
     return a.ctypes.data_as(_D)
+
+
+def _alpha3(alpha):
+    """alpha as [alpha_pre, alpha_post, alpha_res]; a single alpha is three equal
+    entries.  Returns (array, whether alpha was a single value)."""
+    a = np.asarray(_f64(alpha), dtype=np.float64).reshape(-1)
+    if a.size == 1:
+        return np.full(3, float(a[0])), True
+    if a.size != 3:
+        raise ValueError("alpha: one value or three (pre, post, res)")
+    return np.ascontiguousarray(a), False
 
 
 def num_threads() -> int:
@@ -104,15 +115,17 @@ def sinkhorn_backward(logits, dout, iters: int) -> np.ndarray:
     return dl
 
 
-def pre(x, phi, b, alpha: float, iters: int = 20, eps: float = 1e-6):
-    """x [T,n,C] -> dict(h_in [T,C], H_pre [T,n], H_post [T,n], H_res [T,n,n], z, r)."""
+def pre(x, phi, b, alpha, iters: int = 20, eps: float = 1e-6):
+    """x [T,n,C] -> dict(h_in [T,C], H_pre [T,n], H_post [T,n], H_res [T,n,n], z, r).
+    alpha: one value, or three (pre, post, res) for per-group scales."""
     xd = _f64(x)
     T, n, C = xd.shape
     M = n * n + 2 * n
     ph, bd = _f64(phi).reshape(n * C, M), _f64(b).reshape(M)
     out = dict(h_in=np.empty((T, C)), H_pre=np.empty((T, n)), H_post=np.empty((T, n)),
                H_res=np.empty((T, n, n)), z=np.empty((T, M)), r=np.empty(T))
-    _load().orc_pre(n, T, C, int(iters), float(eps), _p(xd), _p(ph), _p(bd), float(alpha),
+    a3, _ = _alpha3(alpha)
+    _load().orc_pre(n, T, C, int(iters), float(eps), _p(xd), _p(ph), _p(bd), _p(a3),
                     _p(out["h_in"]), _p(out["H_pre"]), _p(out["H_post"]), _p(out["H_res"]),
                     _p(out["z"]), _p(out["r"]))
     return out
@@ -128,18 +141,21 @@ def post(x, f_out, H_post, H_res) -> np.ndarray:
     return out
 
 
-def backward(x, phi, b, alpha: float, f_out, grad_x_next, grad_h_in, iters: int = 20,
+def backward(x, phi, b, alpha, f_out, grad_x_next, grad_h_in, iters: int = 20,
              eps: float = 1e-6, chunk: int | None = None):
     """Backward of pre+post with recompute.  Returns dict(grad_x, grad_phi, grad_b,
-    grad_alpha, grad_f_out).  ``chunk`` runs T in consecutive token chunks (the
-    parameter sums still accumulate in increasing token order)."""
+    grad_alpha, grad_f_out).  alpha is one value (grad_alpha a float) or three, the
+    per-group scales of the pre, post and res logits (grad_alpha an array of
+    three).  ``chunk`` runs T in consecutive token chunks (the parameter sums
+    still accumulate in increasing token order)."""
     T = x.shape[0]
     n, C = x.shape[1], x.shape[2]
     M = n * n + 2 * n
     ph, bd = _f64(phi).reshape(n * C, M), _f64(b).reshape(M)
+    a3, single = _alpha3(alpha)
     gphi = np.zeros((n * C, M))
     gb = np.zeros(M)
-    ga = np.zeros(1)
+    ga = np.zeros(3)
     gx = np.empty((T, n, C))
     gf = np.empty((T, C))
     step = T if chunk is None else int(chunk)
@@ -151,11 +167,12 @@ def backward(x, phi, b, alpha: float, f_out, grad_x_next, grad_h_in, iters: int 
         gxc = np.empty((t1 - t0, n, C))
         gfc = np.empty((t1 - t0, C))
         lib.orc_backward(n, t1 - t0, C, int(iters), float(eps), _p(xd), _p(ph), _p(bd),
-                         float(alpha), _p(fd), _p(Gd), _p(gd), _p(gxc), _p(gphi), _p(gb),
+                         _p(a3), _p(fd), _p(Gd), _p(gd), _p(gxc), _p(gphi), _p(gb),
                          _p(ga), _p(gfc))
         gx[t0:t1] = gxc
         gf[t0:t1] = gfc
-    return dict(grad_x=gx, grad_phi=gphi, grad_b=gb, grad_alpha=float(ga[0]), grad_f_out=gf)
+    return dict(grad_x=gx, grad_phi=gphi, grad_b=gb, grad_f_out=gf,
+                grad_alpha=float(ga[0] + ga[1] + ga[2]) if single else ga)
 
 
 def post_backward(x, f_out, H_post, grad_x_next):
@@ -171,7 +188,7 @@ def post_backward(x, f_out, H_post, grad_x_next):
     return dict(grad_f_out=gf, red=red)
 
 
-def pre_backward(x, phi, b, alpha: float, grad_x_next, grad_h_in, red, iters: int = 20,
+def pre_backward(x, phi, b, alpha, grad_x_next, grad_h_in, red, iters: int = 20,
                  eps: float = 1e-6, chunk: int | None = None):
     """Second half of the layer backward in training order: recompute the mapping and
     take grad_h_in and the post half's reductions.  Returns dict(grad_x, grad_phi,
@@ -181,9 +198,10 @@ def pre_backward(x, phi, b, alpha: float, grad_x_next, grad_h_in, red, iters: in
     M = n * n + 2 * n
     ph, bd = _f64(phi).reshape(n * C, M), _f64(b).reshape(M)
     rd = _f64(red).reshape(T, n * n + n)
+    a3, single = _alpha3(alpha)
     gphi = np.zeros((n * C, M))
     gb = np.zeros(M)
-    ga = np.zeros(1)
+    ga = np.zeros(3)
     gx = np.empty((T, n, C))
     step = T if chunk is None else int(chunk)
     lib = _load()
@@ -194,10 +212,11 @@ def pre_backward(x, phi, b, alpha: float, grad_x_next, grad_h_in, red, iters: in
         rc = np.ascontiguousarray(rd[t0:t1])
         gxc = np.empty((t1 - t0, n, C))
         lib.orc_pre_backward(n, t1 - t0, C, int(iters), float(eps), _p(xd), _p(ph), _p(bd),
-                             float(alpha), _p(Gd), _p(gd), _p(rc), _p(gxc), _p(gphi), _p(gb),
+                             _p(a3), _p(Gd), _p(gd), _p(rc), _p(gxc), _p(gphi), _p(gb),
                              _p(ga))
         gx[t0:t1] = gxc
-    return dict(grad_x=gx, grad_phi=gphi, grad_b=gb, grad_alpha=float(ga[0]))
+    return dict(grad_x=gx, grad_phi=gphi, grad_b=gb,
+                grad_alpha=float(ga[0] + ga[1] + ga[2]) if single else ga)
 
 
 def depth_amax(H) -> tuple[np.ndarray, np.ndarray]:

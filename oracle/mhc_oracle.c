@@ -60,6 +60,11 @@
 
 static double orc_sigmoid(double v) { return 1.0 / (1.0 + exp(-v)); }
 
+/* Scale group of logit m: 0 = pre (m < n), 1 = post (m < 2n), 2 = res.
+ * alpha is always passed as [alpha_pre, alpha_post, alpha_res]; one shared
+ * alpha is the case of three equal entries. */
+static int orc_group(int n, int m) { return m < n ? 0 : (m < 2 * n ? 1 : 2); }
+
 /* Sinkhorn-Knopp [P1 "Vielfaeltig eingeschraenkte Hyperverbindungen";
  * P5 [10], [16]]: M0 = exp(logits), then `iters` times: divide each row by its
  * sum, then divide each column by its sum.  If `iterates` is non-NULL it
@@ -145,7 +150,8 @@ void orc_sinkhorn_backward(int n, int iters, int64_t B, const double *logits,
  * z = alpha * y + b.  The normalisation is applied first, as RMSNorm is
  * usually written. */
 static void orc_logits(int n, int64_t C, double eps, const double *x, const double *phi,
-                       const double *b, double alpha, double *r_out, double *y, double *z) {
+                       const double *b, const double *alpha, double *r_out, double *y,
+                       double *z) {
   const int64_t K = (int64_t)n * C;
   const int M = n * n + 2 * n;
   double ss = 0.0;
@@ -156,7 +162,7 @@ static void orc_logits(int n, int64_t C, double eps, const double *x, const doub
     const double xh = x[k] / r;
     for (int m = 0; m < M; ++m) y[m] += xh * phi[k * M + m];
   }
-  for (int m = 0; m < M; ++m) z[m] = alpha * y[m] + b[m];
+  for (int m = 0; m < M; ++m) z[m] = alpha[orc_group(n, m)] * y[m] + b[m];
   *r_out = r;
 }
 
@@ -167,7 +173,7 @@ static void orc_logits(int n, int64_t C, double eps, const double *x, const doub
  *   h_in[c] = sum_i H_pre[i] x[i][c].
  * z_out ([T][n*n+2n]) and r_out ([T]) may be NULL. */
 void orc_pre(int n, int64_t T, int64_t C, int iters, double eps, const double *x,
-             const double *phi, const double *b, double alpha, double *h_in, double *H_pre,
+             const double *phi, const double *b, const double *alpha, double *h_in, double *H_pre,
              double *H_post, double *H_res, double *z_out, double *r_out) {
   const int M = n * n + 2 * n;
 #pragma omp parallel for schedule(static)
@@ -220,10 +226,12 @@ void orc_post(int n, int64_t T, int64_t C, const double *x, const double *f_out,
  * pointer is non-null.
  *
  * Per-token output grad_x [T][n][C] is written.  grad_phi, grad_b and
- * grad_alpha are ADDED to (the caller zeroes them), token by token in
+ * grad_alpha (per scale group: pre, post, res) are ADDED to (the caller
+ * zeroes them), token by token in
  * increasing t, so that a caller may run T in consecutive chunks. */
 static void backward_core(int n, int64_t T, int64_t C, int iters, double eps, const double *x,
-                          const double *phi, const double *b, double alpha, const double *f_out,
+                          const double *phi, const double *b, const double *alpha,
+                          const double *f_out,
                           const double *G, const double *g, const double *red, double *grad_x,
                           double *grad_phi, double *grad_b, double *grad_alpha,
                           double *grad_f_out) {
@@ -303,7 +311,7 @@ static void backward_core(int n, int64_t T, int64_t C, int iters, double eps, co
     }
     /* z = alpha * y + b;  y = xhat . phi;  xhat = x / r */
     double dy[16 * 16 + 32];
-    for (int m = 0; m < M; ++m) dy[m] = alpha * dz[m];
+    for (int m = 0; m < M; ++m) dy[m] = alpha[orc_group(n, m)] * dz[m];
     double dot = 0.0; /* sum_k dxhat_k x_k */
     for (int64_t k = 0; k < K; ++k) {
       double dxh = 0.0;
@@ -324,12 +332,12 @@ static void backward_core(int n, int64_t T, int64_t C, int iters, double eps, co
 
   /* parameter gradients: sums over tokens, in increasing t */
   for (int64_t t = 0; t < T; ++t) {
-    double ga = 0.0;
+    double ga[3] = {0.0, 0.0, 0.0};
     for (int m = 0; m < M; ++m) {
       grad_b[m] += dz_all[t * M + m];
-      ga += dz_all[t * M + m] * y_all[t * M + m];
+      ga[orc_group(n, m)] += dz_all[t * M + m] * y_all[t * M + m];
     }
-    *grad_alpha += ga;
+    for (int g = 0; g < 3; ++g) grad_alpha[g] += ga[g];
   }
 #pragma omp parallel for schedule(static)
   for (int64_t k = 0; k < K; ++k) {
@@ -347,9 +355,9 @@ static void backward_core(int n, int64_t T, int64_t C, int iters, double eps, co
 /* The whole layer backward in one call (grad_h_in given together with
  * grad_x_next): grad_x, grad_f_out and the parameter sums. */
 void orc_backward(int n, int64_t T, int64_t C, int iters, double eps, const double *x,
-                  const double *phi, const double *b, double alpha, const double *f_out,
-                  const double *G, const double *g, double *grad_x, double *grad_phi,
-                  double *grad_b, double *grad_alpha, double *grad_f_out) {
+                  const double *phi, const double *b, const double *alpha,
+                  const double *f_out, const double *G, const double *g, double *grad_x,
+                  double *grad_phi, double *grad_b, double *grad_alpha, double *grad_f_out) {
   backward_core(n, T, C, iters, eps, x, phi, b, alpha, f_out, G, g, NULL, grad_x, grad_phi, grad_b,
                 grad_alpha, grad_f_out);
 }
@@ -390,7 +398,7 @@ void orc_post_backward(int n, int64_t T, int64_t C, const double *x, const doubl
  * F's backward), grad_x_next and the post half's reductions, recompute the
  * mapping and write grad_x plus the parameter sums (added to, as above). */
 void orc_pre_backward(int n, int64_t T, int64_t C, int iters, double eps, const double *x,
-                      const double *phi, const double *b, double alpha, const double *G,
+                      const double *phi, const double *b, const double *alpha, const double *G,
                       const double *g, const double *red, double *grad_x, double *grad_phi,
                       double *grad_b, double *grad_alpha) {
   backward_core(n, T, C, iters, eps, x, phi, b, alpha, NULL, G, g, red, grad_x, grad_phi, grad_b,

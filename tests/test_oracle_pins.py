@@ -387,3 +387,53 @@ def test_split_backward_equals_whole(oracle_mod, n):
     for k in ("grad_x", "grad_phi", "grad_b"):
         np.testing.assert_allclose(qb[k], whole[k], rtol=1e-12, atol=1e-12, err_msg=k)
     assert qb["grad_alpha"] == pytest.approx(whole["grad_alpha"], rel=1e-12, abs=1e-12)
+
+
+# ------------------------------------------------- per-group alpha (pre/post/res)
+def test_per_group_alpha_finite_differences(oracle_mod):
+    """With alpha = (a_pre, a_post, a_res) each logit group has its own scale:
+    grad_alpha[g] against central differences of L in a_g, and grad_x / grad_phi
+    against differences too (the groups enter the logits, u and kappa)."""
+    n, T, C, iters, eps = 4, 2, 6, 20, 1e-6
+    M = n * n + 2 * n
+    rng = _rng(140)
+    x = rng.normal(size=(T, n, C))
+    phi = rng.normal(0, 0.3, size=(n * C, M))
+    b = rng.normal(size=M)
+    a3 = np.array([0.6, -0.4, 0.9])
+    f = rng.normal(size=(T, C))
+    G = rng.normal(size=(T, n, C))
+    g = rng.normal(size=(T, C))
+    got = oracle_mod.backward(x, phi, b, a3, f, G, g, iters=iters, eps=eps)
+    assert np.shape(got["grad_alpha"]) == (3,)
+    h = 1e-6
+    for k in range(3):
+        ap, am = a3.copy(), a3.copy()
+        ap[k] += h
+        am[k] -= h
+        fd = (_loss(oracle_mod, x, phi, b, ap, f, G, g, iters, eps) -
+              _loss(oracle_mod, x, phi, b, am, f, G, g, iters, eps)) / (2 * h)
+        assert got["grad_alpha"][k] == pytest.approx(fd, rel=1e-6, abs=1e-7), k
+    for idx in [(0, 1, 2), (1, 3, 5)]:
+        xp, xm = x.copy(), x.copy()
+        xp[idx] += h
+        xm[idx] -= h
+        fd = (_loss(oracle_mod, xp, phi, b, a3, f, G, g, iters, eps) -
+              _loss(oracle_mod, xm, phi, b, a3, f, G, g, iters, eps)) / (2 * h)
+        assert got["grad_x"][idx] == pytest.approx(fd, rel=1e-6, abs=1e-7)
+
+
+def test_three_equal_alphas_reproduce_one(oracle_mod):
+    """alpha = (a, a, a) is the single-alpha layer; its grad_alpha entries add up to
+    the single-alpha gradient."""
+    n, T, C = 2, 3, 5
+    M = n * n + 2 * n
+    rng = _rng(141)
+    x, phi, b = rng.normal(size=(T, n, C)), rng.normal(0, 0.3, size=(n * C, M)), rng.normal(size=M)
+    f, G, g = rng.normal(size=(T, C)), rng.normal(size=(T, n, C)), rng.normal(size=(T, C))
+    one = oracle_mod.backward(x, phi, b, 0.7, f, G, g)
+    three = oracle_mod.backward(x, phi, b, np.array([0.7, 0.7, 0.7]), f, G, g)
+    np.testing.assert_array_equal(one["grad_x"], three["grad_x"])
+    assert one["grad_alpha"] == pytest.approx(float(np.sum(three["grad_alpha"])), rel=1e-14)
+    p1, p3 = oracle_mod.pre(x, phi, b, 0.7), oracle_mod.pre(x, phi, b, np.array([0.7, 0.7, 0.7]))
+    np.testing.assert_array_equal(p1["H_res"], p3["H_res"])
