@@ -101,6 +101,9 @@ typedef struct mhc_params {
   float eps;      /* RMS epsilon added to the mean square, >= 0               */
   int32_t dtype;  /* mhc_dtype of x, f_out, h_in, x_next and the activation
                      gradients                                                */
+  int32_t alpha_groups; /* 0 or 1: one alpha scales all n^2+2n logits;
+                           3: alpha = (alpha_pre, alpha_post, alpha_res), one
+                           scale per logit group, and grad_alpha has 3 entries */
 } mhc_params;
 
 /* Library version, (major << 16) | minor. */
@@ -118,7 +121,7 @@ MHC_API size_t mhc_pre_workspace_size(const mhc_params *p);
  * RMS/projection/gating operator of the "Systemarbeit" section and
  * reportify.cn [17]-[18]; Sinkhorn-Knopp with t_max iterations, [16]).
  *
- *   in : x [T][n][C] (dtype), phi [nC][n^2+2n], b [n^2+2n], alpha [1]
+ *   in : x [T][n][C] (dtype), phi [nC][n^2+2n], b [n^2+2n], alpha [1 or 3]
  *   out: h_in [T][C] (dtype) = sum_i H_pre[i] x[i][:]
  *        H_pre [T][n], H_post [T][n], H_res [T][n][n]   (float32)
  *   workspace: mhc_pre_workspace_size(p) bytes (may be NULL when that is 0).
@@ -158,7 +161,7 @@ MHC_API size_t mhc_backward_workspace_size(const mhc_params *p);
  *   in : x [T][n][C], phi, b, alpha, f_out [T][C], grad_x_next [T][n][C],
  *        grad_h_in [T][C]
  *   out: grad_x [T][n][C] (dtype), grad_f_out [T][C] (dtype),
- *        grad_phi [nC][n^2+2n], grad_b [n^2+2n], grad_alpha [1]   (float32)
+ *        grad_phi [nC][n^2+2n], grad_b [n^2+2n], grad_alpha [1 or 3]   (float32)
  * grad_phi / grad_b / grad_alpha are OVERWRITTEN (not accumulated) with sums
  * over the T tokens taken in a fixed order: repeated calls give identical
  * bits.  workspace: at least mhc_backward_workspace_size(p) bytes, 256-byte

@@ -54,12 +54,18 @@ def _stream(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def params(n: int, T: int, C: int, dtype: torch.dtype, t_max: int = 20, eps: float = 1e-6):
-    """Build an ``mhc_params`` struct."""
+def params(n: int, T: int, C: int, dtype: torch.dtype, t_max: int = 20, eps: float = 1e-6,
+           alpha_groups: int = 1):
+    """Build an ``mhc_params`` struct (alpha_groups 3: per-group alpha)."""
     if dtype not in DTYPE_CODE:
         raise ValueError(f"unsupported activation dtype {dtype}")
     return _lib.MhcParams(n=int(n), t_max=int(t_max), T=int(T), C=int(C), eps=float(eps),
-                          dtype=DTYPE_CODE[dtype])
+                          dtype=DTYPE_CODE[dtype], alpha_groups=int(alpha_groups))
+
+
+def _ag(alpha) -> int:
+    """3 when alpha holds the pre, post and res scales, else 1 (one shared alpha)."""
+    return 3 if alpha.numel() == 3 else 1
 
 
 def mhc_pre_workspace_size(n: int, T: int, C: int, dtype: torch.dtype, t_max: int = 20,
@@ -86,7 +92,7 @@ def mhc_pre(x, phi, b, alpha, *, t_max: int = 20, eps: float = 1e-6, out=None, w
             dev_status=None, stream=None):
     """x [T,n,C] -> (h_in [T,C], H_pre [T,n], H_post [T,n], H_res [T,n,n])."""
     T, n, C = x.shape
-    p = params(n, T, C, x.dtype, t_max, eps)
+    p = params(n, T, C, x.dtype, t_max, eps, _ag(alpha))
     if out is None:
         out = (torch.empty(T, C, dtype=x.dtype, device=x.device),
                torch.empty(T, n, dtype=torch.float32, device=x.device),
@@ -117,7 +123,7 @@ def mhc_backward(x, phi, b, alpha, f_out, grad_x_next, grad_h_in, *, t_max: int 
     """Gradients of pre+post with recompute.
     Returns (grad_x, grad_phi, grad_b, grad_alpha, grad_f_out)."""
     T, n, C = x.shape
-    p = params(n, T, C, x.dtype, t_max, eps)
+    p = params(n, T, C, x.dtype, t_max, eps, _ag(alpha))
     if out is None:
         out = (torch.empty_like(x), torch.empty_like(phi), torch.empty_like(b),
                torch.empty_like(alpha), torch.empty_like(f_out))
@@ -139,7 +145,7 @@ def mhc_backward_noalloc(x, phi, b, alpha, f_out, grad_x_next, grad_h_in, *, t_m
     ``out`` by callers that cannot allocate; they are created here only as a convenience.
     Returns (grad_x, grad_phi, grad_b, grad_alpha, grad_f_out)."""
     T, n, C = x.shape
-    p = params(n, T, C, x.dtype, t_max, eps)
+    p = params(n, T, C, x.dtype, t_max, eps, _ag(alpha))
     if out is None:
         out = (torch.empty_like(x), torch.empty_like(phi), torch.empty_like(b),
                torch.empty_like(alpha), torch.empty_like(f_out))
@@ -157,7 +163,7 @@ def mhc_post_fused(x, f_out, H_post, H_res, phi_next, b_next, alpha_next, *, t_m
     """Layer l's post merge fused with layer l+1's mapping.
     Returns (x_next [T,n,C], H_pre_next [T,n], H_post_next [T,n], H_res_next [T,n,n])."""
     T, n, C = x.shape
-    p = params(n, T, C, x.dtype, t_max, eps)
+    p = params(n, T, C, x.dtype, t_max, eps, _ag(alpha_next))
     if out is None:
         out = (torch.empty_like(x), torch.empty(T, n, dtype=torch.float32, device=x.device),
                torch.empty(T, n, dtype=torch.float32, device=x.device),
@@ -205,7 +211,7 @@ def mhc_pre_backward(x, phi, b, alpha, grad_x_next, grad_h_in, red, *, t_max: in
     """Second half of the layer backward in training order (after F's backward).
     Returns (grad_x, grad_phi, grad_b, grad_alpha)."""
     T, n, C = x.shape
-    p = params(n, T, C, x.dtype, t_max, eps)
+    p = params(n, T, C, x.dtype, t_max, eps, _ag(alpha))
     if out is None:
         out = (torch.empty_like(x), torch.empty_like(phi), torch.empty_like(b),
                torch.empty_like(alpha))
@@ -225,7 +231,7 @@ def mhc_backward_map(x, phi, b, alpha, f_out, grad_x_next, grad_h_in, workspace,
     """Phase 1 of mhc_backward: per-token records into ``workspace`` (uint8 tensor of at
     least mhc_backward_workspace_size bytes)."""
     T, n, C = x.shape
-    p = params(n, T, C, x.dtype, t_max, eps)
+    p = params(n, T, C, x.dtype, t_max, eps, _ag(alpha))
     st = _lib.load().mhc_backward_map(ctypes.byref(p), _p(x), _p(phi), _p(b), _p(alpha), _p(f_out),
                                       _p(grad_x_next), _p(grad_h_in), _p(workspace),
                                       workspace.numel(), _p(dev_status), _stream(stream))
@@ -233,15 +239,17 @@ def mhc_backward_map(x, phi, b, alpha, f_out, grad_x_next, grad_h_in, workspace,
 
 
 def mhc_backward_apply(x, phi, grad_x_next, grad_h_in, workspace, *, t_max: int = 20,
-                       eps: float = 1e-6, out=None, dev_status=None, stream=None):
-    """Phase 2 of mhc_backward.  Returns (grad_x, grad_phi, grad_b, grad_alpha, grad_f_out)."""
+                       eps: float = 1e-6, alpha_groups: int = 1, out=None, dev_status=None,
+                       stream=None):
+    """Phase 2 of mhc_backward (alpha_groups as in the map phase).
+    Returns (grad_x, grad_phi, grad_b, grad_alpha, grad_f_out)."""
     T, n, C = x.shape
-    p = params(n, T, C, x.dtype, t_max, eps)
+    p = params(n, T, C, x.dtype, t_max, eps, alpha_groups)
     M = n * n + 2 * n
     if out is None:
         out = (torch.empty_like(x), torch.empty_like(phi),
                torch.empty(M, dtype=torch.float32, device=x.device),
-               torch.empty(1, dtype=torch.float32, device=x.device),
+               torch.empty(3 if alpha_groups == 3 else 1, dtype=torch.float32, device=x.device),
                torch.empty(T, C, dtype=x.dtype, device=x.device))
     gx, gphi, gb, ga, gf = out
     st = _lib.load().mhc_backward_apply(ctypes.byref(p), _p(x), _p(phi), _p(grad_x_next),

@@ -137,6 +137,7 @@ struct ApplyArgs {
   int* xcnt;      // [E]
   int* status;
   int write_gf;   // 0: grad_f_out is not produced (pre half of the split backward)
+  int ag;         // 3: grad_alpha per group (pre, post, res); else one shared alpha
 };
 
 // Walks one CTA's items: for every tile t its P owned slices, then the
@@ -198,7 +199,7 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* bcast = reinterpret_cast<int*>(tmem_slot + 2);
-  float* wsum = reinterpret_cast<float*>(smem + MISC_OFF + 256);  // [NEPI][M + 1], bias sums
+  float* wsum = reinterpret_cast<float*>(smem + MISC_OFF + 256);  // [NEPI + 1][M + 3], bias sums
   float* xch = reinterpret_cast<float*>(smem + XCH_OFF);           // [KR][M], u_lo halves
   auto bar = [&](int i) { return tc::smem_u32(bars + i); };
 
@@ -373,18 +374,25 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
 
     if (b == 0) {
       // grad_b / grad_alpha from the mapping kernel's per-CTA partials, in a fixed order
+      // columns: M dz sums, then dz . y over the pre, post and res logits
+      constexpr int NC = M + 3;
       const int ew = etid / 32;
       float sacc = 0.0f;
-      if (lane <= M)
+      if (lane < NC)
         for (int p = ew; p < a.nparts; p += NEPI) sacc += __ldg(a.part + (int64_t)p * CF::DZ_SIZE + lane);
-      if (lane <= M) wsum[ew * (M + 1) + lane] = sacc;
+      if (lane < NC) wsum[ew * NC + lane] = sacc;
       named_bar_sync(1, NEPI_T);
-      if (etid <= M) {
+      if (etid < NC) {
         float acc = 0.0f;
-        for (int w = 0; w < NEPI; ++w) acc += wsum[w * (M + 1) + etid];
+        for (int w = 0; w < NEPI; ++w) acc += wsum[w * NC + etid];
+        wsum[NEPI * NC + etid] = acc;
         if (etid < M) a.grad_b[etid] = acc;
-        else *a.grad_alpha = acc;
+        else if (a.ag == 3) a.grad_alpha[etid - M] = acc;
       }
+      named_bar_sync(1, NEPI_T);
+      // one shared alpha: its gradient is the sum of the three group sums
+      if (a.ag != 3 && etid == 0)
+        *a.grad_alpha = (wsum[NEPI * NC + M] + wsum[NEPI * NC + M + 1]) + wsum[NEPI * NC + M + 2];
     }
 
     // Read one M = 64 grad_phi accumulator (phi row 16q + l in lane 32q + l,
@@ -629,7 +637,8 @@ size_t apply_tc_scratch_bytes(int64_t T, int64_t C) {
 cudaError_t apply_tc_dispatch(int64_t T, int64_t C, const void* x, const void* phi_split,
                               const void* G, const void* g, const void* urec, const float* hrec,
                               const float* part, int nparts, void* gx, void* gf, float* gphi,
-                              float* gb, float* ga, void* scratch, int* st, cudaStream_t s) {
+                              float* gb, float* ga, int ag, void* scratch, int* st,
+                              cudaStream_t s) {
   using namespace tcap;
   const ApplyPlan pl = apply_plan(T, C, device_sms());
   CUtensorMap mx, mG, mg, mu, mp, mgx, mgf;
@@ -684,6 +693,7 @@ cudaError_t apply_tc_dispatch(int64_t T, int64_t C, const void* x, const void* p
   a.xcnt = (int*)((char*)scratch + (size_t)pl.E * pl.NTT * KR * M * 4);
   a.status = st;
   a.write_gf = gf != nullptr ? 1 : 0;
+  a.ag = ag;
   e = cudaFuncSetAttribute(k_apply_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (e != cudaSuccess) return e;
   if (pl.E > 0) {

@@ -44,7 +44,8 @@ __global__ void __launch_bounds__(bwdk::NT) k_bwd_apply(
     int64_t T, int64_t C, const TIO* __restrict__ x, const float* __restrict__ phi,
     const TIO* __restrict__ G, const TIO* __restrict__ g, const float* __restrict__ coef,
     const float* __restrict__ part, int nparts, TIO* __restrict__ grad_x, TIO* __restrict__ grad_f,
-    float* __restrict__ grad_phi, float* __restrict__ grad_b, float* __restrict__ grad_alpha) {
+    float* __restrict__ grad_phi, float* __restrict__ grad_b, float* __restrict__ grad_alpha,
+    int ag) {
   using S = ApplyShape<TIO, N>;
   using CF = Coef<N>;
   using namespace bwdk;
@@ -63,20 +64,27 @@ __global__ void __launch_bounds__(bwdk::NT) k_bwd_apply(
     // grad_b and grad_alpha: add the mapping kernel's per-CTA partial sums.
     // Warp w takes partials w, w + NW, ... in order; the NW results are then
     // added in warp order -- a fixed order, so repeated calls agree bitwise.
-    // (M + 1 columns can exceed a warp's 32 lanes: n = 8 has 81)
-    float* wsum = sm;  // [NW][M + 1]
-    for (int col = lane; col <= M; col += 32) {
+    // Columns: M dz sums, then dz . y over the pre, post and res logits (M + 3
+    // can exceed a warp's 32 lanes: n = 8 has 83).
+    constexpr int NC = M + 3;
+    float* wsum = sm;  // [NW][NC]
+    for (int col = lane; col < NC; col += 32) {
       float s = 0.0f;
       for (int q = warp; q < nparts; q += NW) s += __ldg(part + (int64_t)q * CF::DZ_SIZE + col);
-      wsum[warp * (M + 1) + col] = s;
+      wsum[warp * NC + col] = s;
     }
     __syncthreads();
-    for (int col = threadIdx.x; col <= M; col += NT) {
+    for (int col = threadIdx.x; col < NC; col += NT) {
       float a = 0.0f;
-      for (int w = 0; w < NW; ++w) a += wsum[w * (M + 1) + col];
+      for (int w = 0; w < NW; ++w) a += wsum[w * NC + col];
+      wsum[NW * NC + col] = a;
       if (col < M) grad_b[col] = a;
-      else *grad_alpha = a;
+      else if (ag == 3) grad_alpha[col - M] = a;
     }
+    __syncthreads();
+    // one shared alpha: its gradient is the sum of the three group sums
+    if (ag != 3 && threadIdx.x == 0)
+      *grad_alpha = (wsum[NW * NC + M] + wsum[NW * NC + M + 1]) + wsum[NW * NC + M + 2];
   }
 
   float ph[CPL][M], gp[CPL][M];
@@ -175,7 +183,7 @@ template <typename TIO, int N>
 static cudaError_t launch_apply_t(int64_t T, int64_t C, const void* x, const float* phi,
                                   const void* G, const void* g, const float* coef,
                                   const float* part, int nparts, void* gx, void* gf, float* gphi,
-                                  float* gb, float* ga, cudaStream_t s) {
+                                  float* gb, float* ga, int ag, cudaStream_t s) {
   using S = ApplyShape<TIO, N>;
   using CF = Coef<N>;
   const size_t smem_c = (size_t)bwdk::TB * CF::SIZE * 4;
@@ -187,21 +195,21 @@ static cudaError_t launch_apply_t(int64_t T, int64_t C, const void* x, const flo
   const int64_t grid = (C + S::CW - 1) / S::CW;
   kern<<<(unsigned)grid, bwdk::NT, smem, s>>>(T, C, (const TIO*)x, phi, (const TIO*)G,
                                              (const TIO*)g, coef, part, nparts, (TIO*)gx,
-                                             (TIO*)gf, gphi, gb, ga);
+                                             (TIO*)gf, gphi, gb, ga, ag);
   return cudaGetLastError();
 }
 
 cudaError_t apply_dispatch(int n, int dtype, int64_t T, int64_t C, const void* x, const float* phi,
                            const void* G, const void* g, const float* coef, const float* part,
                            int nparts, void* gx, void* gf, float* gphi, float* gb, float* ga,
-                           cudaStream_t s) {
+                           int ag, cudaStream_t s) {
 #define MHC_APPLY(NN)                                                                        \
   case NN:                                                                                   \
     return dtype == MHC_DTYPE_BF16                                                           \
                ? launch_apply_t<__nv_bfloat16, NN>(T, C, x, phi, G, g, coef, part, nparts, gx, gf, \
-                                                   gphi, gb, ga, s)                              \
+                                                   gphi, gb, ga, ag, s)                              \
                : launch_apply_t<float, NN>(T, C, x, phi, G, g, coef, part, nparts, gx, gf, gphi,  \
-                                           gb, ga, s);
+                                           gb, ga, ag, s);
   switch (n) {
     MHC_APPLY(1)
     MHC_APPLY(2)

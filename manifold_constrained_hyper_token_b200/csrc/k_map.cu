@@ -1,11 +1,12 @@
 // k_map.cu -- per-token mapping kernels on the CUDA cores (fp32 FMA):
 //
-//   forward   r = sqrt(mean x^2 + eps), y = (x . phi) / r, z = alpha y + b,
+//   forward   r = sqrt(mean x^2 + eps), y = (x . phi) / r, z = alpha_g y + b
+//             (alpha_g: the scale of the logit's group, pre / post / res),
 //             H_pre = sigmoid, H_post = 2 sigmoid, H_res = Sinkhorn(exp(z_res))
 //   backward  the same recompute, plus the C-reductions
 //               dH_pre[i] = <g, x_i>, dH_post[i] = <G_i, f>, dH_res[i][j] = <G_i, x_j>
 //             the Sinkhorn adjoint and the gate derivatives, giving
-//             dz, u = alpha dz / r and kappa = alpha (dz . y) / (K r^2).
+//             dz, u = alpha_g dz / r and kappa = sum_m alpha_g dz_m y_m / (K r^2).
 //
 // Sources: the RMSNorm/projection/gating operator of the chatgpz.de explainer
 // (section "Systemarbeit und Schulungsaufwand") and reportify.cn [17]-[19]:
@@ -48,7 +49,7 @@ static size_t map_smem_bytes() {
   constexpr int VPS = mapk::CC / Vec<TIO>::N;
   size_t stage = (size_t)S::STAGE_FLOATS * 4;
   size_t red = ((size_t)4 * mapk::TM * S::MP + (size_t)mapk::TM * (S::M + 1) +
-                (size_t)mapk::TM * N * VPS + (size_t)mapk::TM * (S::M + 1)) * 4;
+                (size_t)mapk::TM * N * VPS + (size_t)mapk::TM * (S::M + 3)) * 4;
   size_t two = 2 * stage;
   return two > red ? two : red;
 }
@@ -62,6 +63,7 @@ template <typename TIO, int N, int MODE>
 __global__ void __launch_bounds__(mapk::NT) k_map(
     int64_t T, int64_t C, int iters, float eps, const TIO* __restrict__ x,
     const float* __restrict__ phi, const float* __restrict__ bias, const float* __restrict__ alpha_p,
+    int ag,
     // forward outputs
     float* __restrict__ Hpre_o, float* __restrict__ Hpost_o, float* __restrict__ Hres_o,
     // backward inputs / outputs
@@ -229,7 +231,7 @@ __global__ void __launch_bounds__(mapk::NT) k_map(
   // sum of squares: slots of one token are spread over threads; gather them
   // into a [TM][N*VPS] table and add in slot order.
   float* sst = ssr + TM * (BWD ? M + 1 : 1);  // [TM][N*VPS]
-  float* dzs = sst + TM * N * VPS;            // [TM][M+1] (backward)
+  float* dzs = sst + TM * N * VPS;            // [TM][M+3] (backward)
 #pragma unroll
   for (int r = 0; r < NR; ++r) {
     const int v = tid + NT * r;
@@ -256,14 +258,15 @@ __global__ void __launch_bounds__(mapk::NT) k_map(
       float ss = 0.0f;
       for (int s = 0; s < N * VPS; ++s) ss += sst[tid * N * VPS + s];
       const float r = sqrtf(ss / (float)K + eps);
-      const float alpha = __ldg(alpha_p);
+      Alpha3 al;
+      al.load(alpha_p, ag);
       float y[M], z[M];
 #pragma unroll
       for (int m = 0; m < M; ++m) {
         const float yr = red[(0 * TM + tid) * MP + m] + red[(1 * TM + tid) * MP + m] +
                          red[(2 * TM + tid) * MP + m] + red[(3 * TM + tid) * MP + m];
         y[m] = yr / r;
-        z[m] = fmaf(alpha, y[m], __ldg(bias + m));
+        z[m] = fmaf(al.at<N>(m), y[m], __ldg(bias + m));
       }
       bool bad = !isfinite(r);
 #pragma unroll
@@ -303,9 +306,12 @@ __global__ void __launch_bounds__(mapk::NT) k_map(
         }
 #pragma unroll
         for (int e = 0; e < N * N; ++e) dz[2 * N + e] = dzres[e];
-        float dzy = 0.0f;
+        float dzy[3] = {0.0f, 0.0f, 0.0f};  // dz . y over the pre, post, res logits
 #pragma unroll
-        for (int m = 0; m < M; ++m) dzy = fmaf(dz[m], y[m], dzy);
+        for (int m = 0; m < M; ++m) {
+          const int grp = m < N ? 0 : (m < 2 * N ? 1 : 2);
+          dzy[grp] = fmaf(dz[m], y[m], dzy[grp]);
+        }
         using CF = Coef<N>;
         float* co = coef_o + t * CF::SIZE;
 #pragma unroll
@@ -315,25 +321,29 @@ __global__ void __launch_bounds__(mapk::NT) k_map(
           co[CF::PRE + i] = spre[i];
           co[CF::POST + i] = 2.0f * spost[i];
         }
-        const float ar = alpha / r;
+        float ar[3];
 #pragma unroll
-        for (int m = 0; m < M; ++m) co[CF::U + m] = ar * dz[m];
-        co[CF::KAPPA] = alpha * dzy / ((float)K * r * r);
+        for (int g = 0; g < 3; ++g) ar[g] = al.a[g] / r;
 #pragma unroll
-        for (int m = 0; m < M; ++m) dzs[tid * (M + 1) + m] = dz[m];
-        dzs[tid * (M + 1) + M] = dzy;
+        for (int m = 0; m < M; ++m) co[CF::U + m] = ar[m < N ? 0 : (m < 2 * N ? 1 : 2)] * dz[m];
+        const float wdzy = fmaf(al.a[2], dzy[2], fmaf(al.a[1], dzy[1], al.a[0] * dzy[0]));
+        co[CF::KAPPA] = wdzy / ((float)K * r * r);
+#pragma unroll
+        for (int m = 0; m < M; ++m) dzs[tid * (M + 3) + m] = dz[m];
+#pragma unroll
+        for (int g = 0; g < 3; ++g) dzs[tid * (M + 3) + M + g] = dzy[g];
       }
     } else if constexpr (BWD) {
 #pragma unroll
-      for (int m = 0; m <= M; ++m) dzs[tid * (M + 1) + m] = 0.0f;
+      for (int m = 0; m < M + 3; ++m) dzs[tid * (M + 3) + m] = 0.0f;
     }
   }
   if constexpr (BWD) {
-    // this CTA's share of grad_b and grad_alpha, summed in token order
+    // this CTA's share of grad_b and the three grad_alpha sums, in token order
     __syncthreads();
-    if (tid <= M) {
+    if (tid < M + 3) {
       float s = 0.0f;
-      for (int q = 0; q < TM; ++q) s += dzs[q * (M + 1) + tid];
+      for (int q = 0; q < TM; ++q) s += dzs[q * (M + 3) + tid];
       part_o[(int64_t)blockIdx.x * Coef<N>::DZ_SIZE + tid] = s;
     }
   }
@@ -341,7 +351,7 @@ __global__ void __launch_bounds__(mapk::NT) k_map(
 
 template <typename TIO, int N, int MODE>
 static cudaError_t launch_map_t(int64_t T, int64_t C, int iters, float eps, const void* x,
-                                const float* phi, const float* b, const float* alpha,
+                                const float* phi, const float* b, const float* alpha, int ag,
                                 float* Hpre, float* Hpost, float* Hres, const void* G,
                                 const void* g, const void* f, const float* red, float* coef,
                                 float* part, int* st, cudaStream_t s) {
@@ -350,7 +360,7 @@ static cudaError_t launch_map_t(int64_t T, int64_t C, int iters, float eps, cons
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int64_t grid = (T + mapk::TM - 1) / mapk::TM;
-  kern<<<(unsigned)grid, mapk::NT, smem, s>>>(T, C, iters, eps, (const TIO*)x, phi, b, alpha, Hpre,
+  kern<<<(unsigned)grid, mapk::NT, smem, s>>>(T, C, iters, eps, (const TIO*)x, phi, b, alpha, ag, Hpre,
                                              Hpost, Hres, (const TIO*)G, (const TIO*)g,
                                              (const TIO*)f, red, coef, part, st);
   return cudaGetLastError();
@@ -358,15 +368,16 @@ static cudaError_t launch_map_t(int64_t T, int64_t C, int iters, float eps, cons
 
 cudaError_t map_fwd_dispatch(int n, int dtype, int64_t T, int64_t C, int iters, float eps,
                              const void* x, const float* phi, const float* b, const float* alpha,
+                             int ag,
                              float* Hpre, float* Hpost, float* Hres, int* st, cudaStream_t s) {
 #define MHC_MAPF(NN)                                                                             \
   case NN:                                                                                       \
     return dtype == MHC_DTYPE_BF16                                                               \
-               ? launch_map_t<__nv_bfloat16, NN, MAP_FWD>(T, C, iters, eps, x, phi, b, alpha,    \
+               ? launch_map_t<__nv_bfloat16, NN, MAP_FWD>(T, C, iters, eps, x, phi, b, alpha, ag,    \
                                                           Hpre, Hpost, Hres, nullptr, nullptr,   \
                                                           nullptr, nullptr, nullptr, nullptr,    \
                                                           st, s)                                 \
-               : launch_map_t<float, NN, MAP_FWD>(T, C, iters, eps, x, phi, b, alpha, Hpre,      \
+               : launch_map_t<float, NN, MAP_FWD>(T, C, iters, eps, x, phi, b, alpha, ag, Hpre,      \
                                                   Hpost, Hres, nullptr, nullptr, nullptr,        \
                                                   nullptr, nullptr, nullptr, st, s);
   switch (n) {
@@ -381,27 +392,29 @@ cudaError_t map_fwd_dispatch(int n, int dtype, int64_t T, int64_t C, int iters, 
 
 template <typename TIO, int N>
 static cudaError_t map_bwd_n(int64_t T, int64_t C, int iters, float eps, const void* x,
-                             const float* phi, const float* b, const float* alpha, const void* G,
+                             const float* phi, const float* b, const float* alpha, int ag,
+                             const void* G,
                              const void* g, const void* f, const float* red, float* coef,
                              float* part, int* st, cudaStream_t s) {
   return red == nullptr
-             ? launch_map_t<TIO, N, MAP_BWD>(T, C, iters, eps, x, phi, b, alpha, nullptr, nullptr,
+             ? launch_map_t<TIO, N, MAP_BWD>(T, C, iters, eps, x, phi, b, alpha, ag, nullptr, nullptr,
                                              nullptr, G, g, f, nullptr, coef, part, st, s)
-             : launch_map_t<TIO, N, MAP_BWD_SPLIT>(T, C, iters, eps, x, phi, b, alpha, nullptr,
+             : launch_map_t<TIO, N, MAP_BWD_SPLIT>(T, C, iters, eps, x, phi, b, alpha, ag, nullptr,
                                                    nullptr, nullptr, nullptr, g, nullptr, red,
                                                    coef, part, st, s);
 }
 
 cudaError_t map_bwd_dispatch(int n, int dtype, int64_t T, int64_t C, int iters, float eps,
                              const void* x, const float* phi, const float* b, const float* alpha,
+                             int ag,
                              const void* G, const void* g, const void* f, const float* red,
                              float* coef, float* part, int* st, cudaStream_t s) {
 #define MHC_MAPB(NN)                                                                          \
   case NN:                                                                                    \
     return dtype == MHC_DTYPE_BF16                                                            \
-               ? map_bwd_n<__nv_bfloat16, NN>(T, C, iters, eps, x, phi, b, alpha, G, g, f, red, \
+               ? map_bwd_n<__nv_bfloat16, NN>(T, C, iters, eps, x, phi, b, alpha, ag, G, g, f, red, \
                                               coef, part, st, s)                              \
-               : map_bwd_n<float, NN>(T, C, iters, eps, x, phi, b, alpha, G, g, f, red, coef,   \
+               : map_bwd_n<float, NN>(T, C, iters, eps, x, phi, b, alpha, ag, G, g, f, red, coef,   \
                                       part, st, s);
   switch (n) {
     MHC_MAPB(1)

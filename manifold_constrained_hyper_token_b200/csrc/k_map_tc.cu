@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_phi,
     const __grid_constant__ CUtensorMap tm_G, const __grid_constant__ CUtensorMap tm_g,
     const __grid_constant__ CUtensorMap tm_f, int64_t T, int64_t C, int iters, float eps,
-    int ck_period, const float* __restrict__ bias, const float* __restrict__ alpha_p,
+    int ck_period, const float* __restrict__ bias, const float* __restrict__ alpha_p, int ag,
     float* __restrict__ Hpre_o, float* __restrict__ Hpost_o, float* __restrict__ Hres_o,
     __nv_bfloat16* __restrict__ urec_o, float* __restrict__ hrec_o, float* __restrict__ part_o,
     const float* __restrict__ red_in, const float* __restrict__ hpost_in,
@@ -406,8 +406,8 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
     ok = __all_sync(0xffffffffu, ok);  // the TMEM loads below are warp-collective
     float* red_ss = reinterpret_cast<float*>(smem);       // [2][TM]
     float* red_dt = red_ss + 2 * TM;                      // [2][M][TM]
-    float* dzs = red_dt + 2 * M * TM;                     // [M + 1][TM]
-    float* ck = dzs + (M + 1) * TM;                       // checkpoints [nck][16][TM]
+    float* dzs = red_dt + 2 * M * TM;                     // [M + 3][TM]
+    float* ck = dzs + (M + 3) * TM;                       // checkpoints [nck][16][TM]
     if (ok) {
       red_ss[h * TM + tok] = ss;
       if constexpr (BWD) {
@@ -497,12 +497,13 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
       // ------------------------------------------------- per-token epilogue
       const int64_t t = t0 + tok;
       const float r = sqrtf(sst / (float)K + eps);
-      const float alpha = __ldg(alpha_p);
+      Alpha3 al;
+      al.load(alpha_p, ag);
       float y[M], z[M];
 #pragma unroll
       for (int m = 0; m < M; ++m) {
         y[m] = yr[m] / r;
-        z[m] = fmaf(alpha, y[m], __ldg(bias + m));
+        z[m] = fmaf(al.at<N>(m), y[m], __ldg(bias + m));
       }
       float spre[N], spost[N];
 #pragma unroll
@@ -549,9 +550,12 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
         }
 #pragma unroll
         for (int e = 0; e < N * N; ++e) dz[2 * N + e] = dzres[e];
-        float dzy = 0.0f;
+        float dzy[3] = {0.0f, 0.0f, 0.0f};  // dz . y over the pre, post, res logits
 #pragma unroll
-        for (int m = 0; m < M; ++m) dzy = fmaf(dz[m], y[m], dzy);
+        for (int m = 0; m < M; ++m) {
+          const int grp = m < N ? 0 : (m < 2 * N ? 1 : 2);
+          dzy[grp] = fmaf(dz[m], y[m], dzy[grp]);
+        }
         const bool live = t < T;
         if (live) {
           float rec[TcRec::H_FLOATS];
@@ -562,17 +566,22 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
             rec[TcRec::H_PRE + i] = spre[i];
             rec[TcRec::H_POST + i] = 2.0f * spost[i];
           }
-          rec[TcRec::H_KAPPA] = alpha * dzy / ((float)K * r * r);
+          rec[TcRec::H_KAPPA] =
+              fmaf(al.a[2], dzy[2], fmaf(al.a[1], dzy[1], al.a[0] * dzy[0])) / ((float)K * r * r);
           rec[25] = rec[26] = rec[27] = 0.0f;
           float4* hd = reinterpret_cast<float4*>(hrec_o + t * TcRec::H_FLOATS);
 #pragma unroll
           for (int e = 0; e < TcRec::H_FLOATS / 4; ++e)
             hd[e] = make_float4(rec[4 * e], rec[4 * e + 1], rec[4 * e + 2], rec[4 * e + 3]);
-          const float ar = alpha / r;
+          float ar[3];
+#pragma unroll
+          for (int g = 0; g < 3; ++g) ar[g] = al.a[g] / r;
           uint32_t w[32];
 #pragma unroll
           for (int m2 = 0; m2 < 12; ++m2) {
-            const float u0 = ar * dz[2 * m2], u1 = ar * dz[2 * m2 + 1];
+            const int g0 = 2 * m2 < N ? 0 : (2 * m2 < 2 * N ? 1 : 2);
+            const int g1 = 2 * m2 + 1 < N ? 0 : (2 * m2 + 1 < 2 * N ? 1 : 2);
+            const float u0 = ar[g0] * dz[2 * m2], u1 = ar[g1] * dz[2 * m2 + 1];
             const __nv_bfloat162 hi = __floats2bfloat162_rn(u0, u1);
             const __nv_bfloat162 lo = __floats2bfloat162_rn(u0 - __low2float(hi), u1 - __high2float(hi));
             w[m2] = *reinterpret_cast<const uint32_t*>(&hi);
@@ -586,13 +595,14 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
         }
 #pragma unroll
         for (int m = 0; m < M; ++m) dzs[m * TM + tok] = live ? dz[m] : 0.0f;
-        dzs[M * TM + tok] = live ? dzy : 0.0f;
+#pragma unroll
+        for (int g = 0; g < 3; ++g) dzs[(M + g) * TM + tok] = live ? dzy[g] : 0.0f;
       }
     }
     if constexpr (BWD) {
       named_bar(1, 256);
-      if (epi && h == 0 && q == 0 && lane <= M) {
-        // this tile's share of grad_b / grad_alpha, summed in token order
+      if (epi && h == 0 && q == 0 && lane < M + 3) {
+        // this tile's share of grad_b and the three grad_alpha sums, in token order
         float a = 0.0f;
         for (int k = 0; k < TM; ++k) a += dzs[lane * TM + k];
         part_o[(int64_t)tile * Coef<N>::DZ_SIZE + lane] = a;
@@ -651,7 +661,7 @@ static cudaError_t encode_maps(int mode, int64_t T, int64_t C, const void* x, co
 // scratch in the freed stage memory.
 static int ck_period_for(int iters, size_t stage_bytes) {
   using namespace tcmap;
-  const size_t scratch = (size_t)(2 * TM + 2 * M * TM + (M + 1) * TM) * 4;
+  const size_t scratch = (size_t)(2 * TM + 2 * M * TM + (M + 3) * TM) * 4;
   const size_t per_ck = (size_t)N * N * TM * 4;
   const int max_ck = (int)((stage_bytes - scratch) / per_ck);  // >= 2 for the sizes used here
   const int steps = 2 * iters;
@@ -714,7 +724,7 @@ size_t map_tc_scratch_bytes(int64_t T, int64_t C) {
 template <int MODE>
 static cudaError_t launch_map_tc(const CUtensorMap& mx, const CUtensorMap& mp, const CUtensorMap& mG,
                                  const CUtensorMap& mg, const CUtensorMap& mf, int64_t T, int64_t C,
-                                 int iters, float eps, const float* b, const float* alpha,
+                                 int iters, float eps, const float* b, const float* alpha, int ag,
                                  float* Hpre, float* Hpost, float* Hres, void* urec, float* hrec,
                                  float* part, const float* red, void* kscratch, int* st,
                                  cudaStream_t s, const float* hpost_in = nullptr,
@@ -738,7 +748,7 @@ static cudaError_t launch_map_tc(const CUtensorMap& mx, const CUtensorMap& mp, c
   }
   const unsigned grid = (unsigned)(ntt * kp);
   const int P = (MODE == MAP_BWD || MODE == MAP_BWD_SPLIT) ? ck_period_for(iters, Cfg<MODE>::DATA) : 1;
-  kern<<<grid, NT, Cfg<MODE>::SMEM, s>>>(mx, mp, mG, mg, mf, T, C, iters, eps, P, b, alpha, Hpre,
+  kern<<<grid, NT, Cfg<MODE>::SMEM, s>>>(mx, mp, mG, mg, mf, T, C, iters, eps, P, b, alpha, ag, Hpre,
                                          Hpost, Hres, (__nv_bfloat16*)urec, hrec, part, red,
                                          hpost_in, hres_in, kp, kpart, kcnt, st);
   return cudaGetLastError();
@@ -746,6 +756,7 @@ static cudaError_t launch_map_tc(const CUtensorMap& mx, const CUtensorMap& mp, c
 
 cudaError_t map_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float eps, const void* x,
                             const float* phi, void* phi_split, const float* b, const float* alpha,
+                            int ag,
                             float* Hpre, float* Hpost, float* Hres, const void* G, const void* g,
                             const void* f, const float* red, void* urec, float* hrec, float* part,
                             void* kscratch, int* st, cudaStream_t s) {
@@ -759,13 +770,13 @@ cudaError_t map_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float eps
   if (e != cudaSuccess) return e;
   switch (mode) {
     case MAP_FWD:
-      return launch_map_tc<MAP_FWD>(mx, mp, mG, mg, mf, T, C, iters, eps, b, alpha, Hpre, Hpost,
+      return launch_map_tc<MAP_FWD>(mx, mp, mG, mg, mf, T, C, iters, eps, b, alpha, ag, Hpre, Hpost,
                                     Hres, nullptr, nullptr, nullptr, nullptr, kscratch, st, s);
     case MAP_BWD:
-      return launch_map_tc<MAP_BWD>(mx, mp, mG, mg, mf, T, C, iters, eps, b, alpha, nullptr,
+      return launch_map_tc<MAP_BWD>(mx, mp, mG, mg, mf, T, C, iters, eps, b, alpha, ag, nullptr,
                                     nullptr, nullptr, urec, hrec, part, nullptr, kscratch, st, s);
     case MAP_BWD_SPLIT:
-      return launch_map_tc<MAP_BWD_SPLIT>(mx, mp, mG, mg, mf, T, C, iters, eps, b, alpha, nullptr,
+      return launch_map_tc<MAP_BWD_SPLIT>(mx, mp, mG, mg, mf, T, C, iters, eps, b, alpha, ag, nullptr,
                                           nullptr, nullptr, urec, hrec, part, red, kscratch, st, s);
     default:
       return cudaErrorInvalidValue;
@@ -778,7 +789,8 @@ cudaError_t map_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float eps
 cudaError_t post_map_tc_dispatch(int64_t T, int64_t C, int iters, float eps, const void* x,
                                  const void* f, const float* Hpost_in, const float* Hres_in,
                                  const float* phi_next, void* phi_split, const float* b_next,
-                                 const float* alpha_next, void* x_next, float* Hpre, float* Hpost,
+                                 const float* alpha_next, int ag, void* x_next, float* Hpre,
+                                 float* Hpost,
                                  float* Hres, void* kscratch, int* st, cudaStream_t s) {
   using namespace tcmap;
   const int64_t K = (int64_t)N * C;
@@ -800,7 +812,7 @@ cudaError_t post_map_tc_dispatch(int64_t T, int64_t C, int iters, float eps, con
   const uint32_t b2[2] = {(uint32_t)Cfg<MAP_POSTFWD>::CH, TM};
   e = make_tmap_bf16(&mf, f, 2, d2, s2, b2, CU_TENSOR_MAP_SWIZZLE_64B);
   if (e != cudaSuccess) return e;
-  return launch_map_tc<MAP_POSTFWD>(mx, mp, mG, mg, mf, T, C, iters, eps, b_next, alpha_next, Hpre,
+  return launch_map_tc<MAP_POSTFWD>(mx, mp, mG, mg, mf, T, C, iters, eps, b_next, alpha_next, ag, Hpre,
                                     Hpost, Hres, nullptr, nullptr, nullptr, nullptr, kscratch, st,
                                     s, Hpost_in, Hres_in);
 }

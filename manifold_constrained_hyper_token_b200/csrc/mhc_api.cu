@@ -20,6 +20,8 @@ mhc_status check_params(const mhc_params* p) {
   if (!(p->eps >= 0.0f) || !isfinite(p->eps)) return MHC_ERR_INVALID_ARG;
   if (p->n != 1 && p->n != 2 && p->n != 4 && p->n != 8) return MHC_ERR_UNSUPPORTED;
   if (p->dtype != MHC_DTYPE_F32 && p->dtype != MHC_DTYPE_BF16) return MHC_ERR_UNSUPPORTED;
+  if (p->alpha_groups != 0 && p->alpha_groups != 1 && p->alpha_groups != 3)
+    return MHC_ERR_INVALID_ARG;
   // tile coordinates of the TMA copies are 32-bit signed: keep T (and a tile
   // past it) inside that range
   if (p->T > (int64_t)0x7fffffffLL - 256) return MHC_ERR_INVALID_ARG;
@@ -27,6 +29,9 @@ mhc_status check_params(const mhc_params* p) {
 }
 
 mhc_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MHC_OK : MHC_ERR_CUDA; }
+
+// 3: alpha = (alpha_pre, alpha_post, alpha_res); 0 or 1: one shared alpha
+int alpha_groups(const mhc_params* p) { return p->alpha_groups == 3 ? 3 : 1; }
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -137,13 +142,13 @@ mhc_status mhc_pre(const mhc_params* p, const void* x, const float* phi, const f
       return MHC_ERR_WORKSPACE;
     char* ws = (char*)workspace;
     st = from_cuda(mhc::map_tc_dispatch(mhc::MAP_FWD, p->T, p->C, p->t_max, p->eps, x, phi, ws, b,
-                                        alpha, H_pre, H_post, H_res, nullptr, nullptr, nullptr,
+                                        alpha, alpha_groups(p), H_pre, H_post, H_res, nullptr, nullptr, nullptr,
                                         nullptr, nullptr, nullptr, nullptr,
                                         ws + round_up(mhc::map_tc_phi_bytes(p->C), 256),
                                         dev_status, s));
   } else {
     st = from_cuda(mhc::map_fwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
-                                         alpha, H_pre, H_post, H_res, dev_status, s));
+                                         alpha, alpha_groups(p), H_pre, H_post, H_res, dev_status, s));
   }
   if (st != MHC_OK) return st;
   return from_cuda(mhc::hin_dispatch(p->n, p->dtype, p->T, p->C, x, H_pre, h_in, s));
@@ -182,13 +187,13 @@ mhc_status mhc_backward_map(const mhc_params* p, const void* x, const float* phi
   char* ws = (char*)workspace;
   if (use_tc(p))
     return from_cuda(mhc::map_tc_dispatch(mhc::MAP_BWD, p->T, p->C, p->t_max, p->eps, x, phi,
-                                          ws + w.phi_off, b, alpha, nullptr, nullptr, nullptr,
-                                          grad_x_next, grad_h_in, f_out, nullptr, ws + w.urec_off,
+                                          ws + w.phi_off, b, alpha, alpha_groups(p), nullptr,
+                                          nullptr, nullptr, grad_x_next, grad_h_in, f_out, nullptr, ws + w.urec_off,
                                           (float*)(ws + w.hrec_off), (float*)(ws + w.part_off),
                                           ws + w.kmap_off,
                                           dev_status, (cudaStream_t)stream));
   return from_cuda(mhc::map_bwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
-                                         alpha, grad_x_next, grad_h_in, f_out, nullptr,
+                                         alpha, alpha_groups(p), grad_x_next, grad_h_in, f_out, nullptr,
                                          (float*)(ws + w.coef_off), (float*)(ws + w.part_off),
                                          dev_status, (cudaStream_t)stream));
 }
@@ -214,13 +219,13 @@ mhc_status mhc_backward_apply(const mhc_params* p, const void* x, const float* p
                                             ws + w.urec_off, (const float*)(ws + w.hrec_off),
                                             (const float*)(ws + w.part_off), w.nparts, grad_x,
                                             grad_f_out, grad_phi, grad_b, grad_alpha,
-                                            (void*)(ws + w.apply_off), dev_status,
+                                            alpha_groups(p), (void*)(ws + w.apply_off), dev_status,
                                             (cudaStream_t)stream));
   return from_cuda(mhc::apply_dispatch(p->n, p->dtype, p->T, p->C, x, phi, grad_x_next, grad_h_in,
                                        (const float*)(ws + w.coef_off),
                                        (const float*)(ws + w.part_off), w.nparts, grad_x,
                                        grad_f_out, grad_phi, grad_b, grad_alpha,
-                                       (cudaStream_t)stream));
+                                       alpha_groups(p), (cudaStream_t)stream));
 }
 
 mhc_status mhc_backward(const mhc_params* p, const void* x, const float* phi, const float* b,
@@ -263,14 +268,15 @@ mhc_status mhc_post_fused(const mhc_params* p, const void* x, const void* f_out,
     char* ws = (char*)workspace;
     return from_cuda(mhc::post_map_tc_dispatch(
         p->T, p->C, p->t_max, p->eps, x, f_out, H_post, H_res, phi_next, ws, b_next, alpha_next,
-        x_next, H_pre_next, H_post_next, H_res_next,
+        alpha_groups(p), x_next, H_pre_next, H_post_next, H_res_next,
         ws + round_up(mhc::map_tc_phi_bytes(p->C), 256), dev_status, s));
   }
   // fp32 or n != 4: the post merge, then the mapping of x_next (both on the GPU)
   st = from_cuda(mhc::post_dispatch(p->n, p->dtype, p->T, p->C, x, f_out, H_post, H_res, x_next, s));
   if (st != MHC_OK) return st;
   return from_cuda(mhc::map_fwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x_next,
-                                         phi_next, b_next, alpha_next, H_pre_next, H_post_next,
+                                         phi_next, b_next, alpha_next, alpha_groups(p), H_pre_next,
+                                         H_post_next,
                                          H_res_next, dev_status, s));
 }
 
@@ -322,26 +328,26 @@ mhc_status mhc_pre_backward(const mhc_params* p, const void* x, const float* phi
   cudaStream_t s = (cudaStream_t)stream;
   if (use_tc(p)) {
     st = from_cuda(mhc::map_tc_dispatch(mhc::MAP_BWD_SPLIT, p->T, p->C, p->t_max, p->eps, x, phi,
-                                        ws + w.phi_off, b, alpha, nullptr, nullptr, nullptr,
-                                        nullptr, grad_h_in, nullptr, red, ws + w.urec_off,
+                                        ws + w.phi_off, b, alpha, alpha_groups(p), nullptr,
+                                        nullptr, nullptr, nullptr, grad_h_in, nullptr, red, ws + w.urec_off,
                                         (float*)(ws + w.hrec_off), (float*)(ws + w.part_off),
                                         ws + w.kmap_off, dev_status, s));
     if (st != MHC_OK) return st;
     return from_cuda(mhc::apply_tc_dispatch(p->T, p->C, x, ws + w.phi_off, grad_x_next, grad_h_in,
                                             ws + w.urec_off, (const float*)(ws + w.hrec_off),
                                             (const float*)(ws + w.part_off), w.nparts, grad_x,
-                                            nullptr, grad_phi, grad_b, grad_alpha,
+                                            nullptr, grad_phi, grad_b, grad_alpha, alpha_groups(p),
                                             (void*)(ws + w.apply_off), dev_status, s));
   }
   st = from_cuda(mhc::map_bwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
-                                       alpha, nullptr, grad_h_in, nullptr, red,
+                                       alpha, alpha_groups(p), nullptr, grad_h_in, nullptr, red,
                                        (float*)(ws + w.coef_off), (float*)(ws + w.part_off),
                                        dev_status, s));
   if (st != MHC_OK) return st;
   return from_cuda(mhc::apply_dispatch(p->n, p->dtype, p->T, p->C, x, phi, grad_x_next, grad_h_in,
                                        (const float*)(ws + w.coef_off),
                                        (const float*)(ws + w.part_off), w.nparts, grad_x, nullptr,
-                                       grad_phi, grad_b, grad_alpha, s));
+                                       grad_phi, grad_b, grad_alpha, alpha_groups(p), s));
 }
 
 mhc_status mhc_sinkhorn_knopp(int n, int iters, int64_t B, const float* logits, float* out,

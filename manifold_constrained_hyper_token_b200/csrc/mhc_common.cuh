@@ -249,8 +249,27 @@ template <int N> struct Coef {
   static constexpr int U = N * N + 2 * N;
   static constexpr int KAPPA = U + M;
   static constexpr int SIZE = ((KAPPA + 1) + 3) / 4 * 4;
-  // dz record for the bias / alpha sums: [0, M) dz, [M] dz . y, padded.
-  static constexpr int DZ_SIZE = ((M + 1) + 3) / 4 * 4;
+  // dz record for the bias / alpha sums: [0, M) dz, then dz . y over the
+  // pre, post and res logits ([M], [M + 1], [M + 2]), padded.
+  static constexpr int DZ_SIZE = ((M + 3) + 3) / 4 * 4;
+};
+
+// The logit scales: alpha_pre for the n pre logits, alpha_post for the n post
+// logits, alpha_res for the n*n residual logits; one shared alpha (ag != 3)
+// is three equal scales.
+struct Alpha3 {
+  float a[3];
+  __device__ __forceinline__ void load(const float* p, int ag) {
+    a[0] = __ldg(p);
+    a[1] = ag == 3 ? __ldg(p + 1) : a[0];
+    a[2] = ag == 3 ? __ldg(p + 2) : a[0];
+  }
+  // scale of logit m of a layer with N streams (m known at compile time in
+  // the unrolled loops, so this is a register choice)
+  template <int N>
+  __device__ __forceinline__ float at(int m) const {
+    return m < N ? a[0] : (m < 2 * N ? a[1] : a[2]);
+  }
 };
 
 // Per-token records of the tensor-core backward (n = 4), written by the

@@ -30,17 +30,21 @@ cudaError_t post_bwd_dispatch(int n, int dtype, int64_t T, int64_t C, const void
                               const float* Hpost, const void* G, void* gf, float* red,
                               cudaStream_t s);
 // k_map.cu (CUDA cores; red == nullptr selects MAP_BWD, else MAP_BWD_SPLIT)
+// ag: 3 = alpha holds the pre, post and res scales (and grad_alpha their three
+// gradients); otherwise one shared alpha.
 cudaError_t map_fwd_dispatch(int n, int dtype, int64_t T, int64_t C, int iters, float eps,
                              const void* x, const float* phi, const float* b, const float* alpha,
-                             float* Hpre, float* Hpost, float* Hres, int* st, cudaStream_t s);
+                             int ag, float* Hpre, float* Hpost, float* Hres, int* st,
+                             cudaStream_t s);
 cudaError_t map_bwd_dispatch(int n, int dtype, int64_t T, int64_t C, int iters, float eps,
                              const void* x, const float* phi, const float* b, const float* alpha,
-                             const void* G, const void* g, const void* f, const float* red,
+                             int ag, const void* G, const void* g, const void* f, const float* red,
                              float* coef, float* part, int* st, cudaStream_t s);
 // k_map_tc.cu (bf16, n = 4: projection on the tensor cores); mode is a MapMode
 cudaError_t map_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float eps, const void* x,
                             const float* phi, void* phi_split, const float* b, const float* alpha,
-                            float* Hpre, float* Hpost, float* Hres, const void* G, const void* g,
+                            int ag, float* Hpre, float* Hpost, float* Hres, const void* G,
+                            const void* g,
                             const void* f, const float* red, void* urec, float* hrec, float* part,
                             void* kscratch, int* st, cudaStream_t s);
 size_t map_tc_phi_bytes(int64_t C);
@@ -50,19 +54,20 @@ size_t map_tc_scratch_bytes(int64_t T, int64_t C);
 cudaError_t post_map_tc_dispatch(int64_t T, int64_t C, int iters, float eps, const void* x,
                                  const void* f, const float* Hpost_in, const float* Hres_in,
                                  const float* phi_next, void* phi_split, const float* b_next,
-                                 const float* alpha_next, void* x_next, float* Hpre, float* Hpost,
-                                 float* Hres, void* kscratch, int* st, cudaStream_t s);
+                                 const float* alpha_next, int ag, void* x_next, float* Hpre,
+                                 float* Hpost, float* Hres, void* kscratch, int* st, cudaStream_t s);
 // k_apply_tc.cu (bf16, n = 4: phi u and grad_phi on the tensor cores);
 // gf == nullptr skips grad_f_out
 cudaError_t apply_tc_dispatch(int64_t T, int64_t C, const void* x, const void* phi_split,
                               const void* G, const void* g, const void* urec, const float* hrec,
                               const float* part, int nparts, void* gx, void* gf, float* gphi,
-                              float* gb, float* ga, void* scratch, int* st, cudaStream_t s);
+                              float* gb, float* ga, int ag, void* scratch, int* st,
+                              cudaStream_t s);
 size_t apply_tc_scratch_bytes(int64_t T, int64_t C);
 // k_bwd.cu (CUDA cores); gf == nullptr skips grad_f_out
 cudaError_t apply_dispatch(int n, int dtype, int64_t T, int64_t C, const void* x, const float* phi,
                            const void* G, const void* g, const float* coef, const float* part,
                            int nparts, void* gx, void* gf, float* gphi, float* gb, float* ga,
-                           cudaStream_t s);
+                           int ag, cudaStream_t s);
 
 }  // namespace mhc

@@ -84,11 +84,12 @@ extern "C" mhc_status mhc_backward_noalloc(const mhc_params* p, const void* x, c
   float* part = (float*)(ws + round_up((size_t)p->T * coef_floats * 4, 256));
 
   cudaStream_t s = (cudaStream_t)stream;
+  const int ag = p->alpha_groups == 3 ? 3 : 1;
   cudaError_t e = mhc::map_bwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
-                                        alpha, grad_x_next, grad_h_in, f_out, nullptr, coef,
+                                        alpha, ag, grad_x_next, grad_h_in, f_out, nullptr, coef,
                                         part, dev_status, s);
   if (e != cudaSuccess) return MHC_ERR_CUDA;
   e = mhc::apply_dispatch(p->n, p->dtype, p->T, p->C, x, phi, grad_x_next, grad_h_in, coef, part,
-                          nparts, grad_x, grad_f_out, grad_phi, grad_b, grad_alpha, s);
+                          nparts, grad_x, grad_f_out, grad_phi, grad_b, grad_alpha, ag, s);
   return e == cudaSuccess ? MHC_OK : MHC_ERR_CUDA;
 }

@@ -368,6 +368,76 @@ def test_split_backward_chain(mhc, oracle_mod, dtype):
     assert _alpha_err(ga, ref["grad_alpha"], terms) < tol
 
 
+# ------------------------------------------ per-group alpha (pre, post, res)
+ALPHA3 = [0.02, -0.015, 0.03]
+
+
+def _alpha3_errs(ga, ref_ga, per_token):
+    """Each group's grad_alpha is a token sum that can cancel: measured against the
+    sum of its per-token magnitudes (as _alpha_err for one alpha)."""
+    got = _np(ga).reshape(-1)
+    out = []
+    for g in range(3):
+        scale = max(abs(ref_ga[g]), float(np.sum(np.abs(per_token[:, g]))))
+        out.append(abs(got[g] - ref_ga[g]) / scale if scale > 0 else 0.0)
+    return out
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("n,T,C", [(4, 130, 520), (2, 65, 24)])
+def test_pre_per_group_alpha(mhc, oracle_mod, dtype, n, T, C):
+    d = _inputs(T, n, C, dtype, seed=11 * T + n)
+    d["alpha"] = torch.tensor(ALPHA3, dtype=torch.float32)
+    dd = _dev(d)
+    h_in, Hpre, Hpost, Hres = mhc.mhc_pre(dd["x"], dd["phi"], dd["b"], dd["alpha"])
+    ref = oracle_mod.pre(d["x"], d["phi"], d["b"], np.array(ALPHA3))
+    for got, k in ((h_in, "h_in"), (Hpre, "H_pre"), (Hpost, "H_post"), (Hres, "H_res")):
+        assert rel_err(_np(got), ref[k]) < TOL[dtype], k
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("n,T,C", [(4, 130, 520), (2, 65, 24), (8, 33, 136)])
+def test_backward_per_group_alpha(mhc, oracle_mod, dtype, n, T, C):
+    d = _inputs(T, n, C, dtype, seed=13 * T + n)
+    d["alpha"] = torch.tensor(ALPHA3, dtype=torch.float32)
+    a3 = np.array(ALPHA3)
+    dd = _dev(d)
+    gx, gphi, gb, ga, gf = mhc.mhc_backward(dd["x"], dd["phi"], dd["b"], dd["alpha"], dd["f_out"],
+                                            dd["grad_x_next"], dd["grad_h_in"])
+    assert ga.numel() == 3
+    ref = oracle_mod.backward(d["x"], d["phi"], d["b"], a3, d["f_out"], d["grad_x_next"],
+                              d["grad_h_in"])
+    tol = TOL[dtype]
+    for got, k in ((gx, "grad_x"), (gphi, "grad_phi"), (gb, "grad_b"), (gf, "grad_f_out")):
+        assert rel_err(_np(got), ref[k]) < tol, k
+    terms = np.array([oracle_mod.backward(d["x"][t:t + 1], d["phi"], d["b"], a3, d["f_out"][t:t + 1],
+                                          d["grad_x_next"][t:t + 1], d["grad_h_in"][t:t + 1])["grad_alpha"]
+                      for t in range(T)])
+    assert max(_alpha3_errs(ga, ref["grad_alpha"], terms)) < tol
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_split_backward_per_group_alpha(mhc, oracle_mod, dtype):
+    T, n, C = 130, 4, 520
+    d = _inputs(T, n, C, dtype, seed=99)
+    d["alpha"] = torch.tensor(ALPHA3, dtype=torch.float32)
+    a3 = np.array(ALPHA3)
+    dd = _dev(d)
+    _, _, Hpost, _ = mhc.mhc_pre(dd["x"], dd["phi"], dd["b"], dd["alpha"])
+    gf, red = mhc.mhc_post_backward(dd["x"], dd["f_out"], Hpost, dd["grad_x_next"])
+    gx, gphi, gb, ga = mhc.mhc_pre_backward(dd["x"], dd["phi"], dd["b"], dd["alpha"],
+                                            dd["grad_x_next"], dd["grad_h_in"], red)
+    ref = oracle_mod.backward(d["x"], d["phi"], d["b"], a3, d["f_out"], d["grad_x_next"],
+                              d["grad_h_in"])
+    tol = TOL[dtype]
+    for got, k in ((gx, "grad_x"), (gphi, "grad_phi"), (gb, "grad_b"), (gf, "grad_f_out")):
+        assert rel_err(_np(got), ref[k]) < tol, k
+    terms = np.array([oracle_mod.backward(d["x"][t:t + 1], d["phi"], d["b"], a3, d["f_out"][t:t + 1],
+                                          d["grad_x_next"][t:t + 1], d["grad_h_in"][t:t + 1])["grad_alpha"]
+                      for t in range(T)])
+    assert max(_alpha3_errs(ga, ref["grad_alpha"], terms)) < tol
+
+
 def test_pre_backward_small_workspace_rejected(mhc):
     d = _dev(_inputs(64, 4, 256, torch.bfloat16, seed=5))
     red = torch.zeros(64, 20, dtype=torch.float32, device="cuda")
