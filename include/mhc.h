@@ -336,6 +336,34 @@ MHC_API mhc_status mhc_sinkhorn_knopp(int n, int iters, int64_t B, const float *
 MHC_API mhc_status mhc_depth_amax(int n, int64_t T, int L, const float *H, float *gain_fwd,
                           float *gain_bwd, int *dev_status, mhc_stream_t stream);
 
+/*
+ * mhc_recompute_plan -- block size for recomputing the depth stack (source:
+ * reportify.cn [21]: the mHC intermediates are dropped after the forward and
+ * rebuilt in the backward; [22]: the recompute block is chosen to make the
+ * total memory smallest.  The pages state the aim but not the cost; the cost
+ * below is this library's reading of it).
+ *
+ * The L layers are cut into consecutive blocks of at most `block` layers;
+ * the first block takes the remainder, so the last block is full.  The
+ * forward keeps only each block's input stream x [n][C] per token.  The
+ * backward handles the blocks last to first: it recomputes a block's forward
+ * and holds, for each of its layers, x_l [n][C], h_in_l [C] and f_out_l [C]
+ * while the block's backward runs, then drops that block's input.  At the
+ * peak (the last block) the resident activations per token are
+ *     R(B) = C * ( n * (ceil(L / B) - 1)  +  (n + 2) * B )   elements,
+ * the inputs of the other blocks plus one full block.  (Buffers that every
+ * B needs alike, the gradient being passed down and the layer being computed
+ * in the forward, are not counted.)  Over real B the minimum is at
+ * B = sqrt(n L / (n + 2)).
+ *
+ *   in : n >= 1 streams, L >= 1 layers
+ *   out: *block = the integer B in [1, L] with the smallest R(B) (the smallest
+ *        such B on a tie); *resident = R(block) / C (may be NULL).
+ *   MHC_ERR_INVALID_ARG for n < 1, L < 1 or block == NULL.  Host only: no
+ *   GPU work, no allocation.
+ */
+MHC_API mhc_status mhc_recompute_plan(int32_t n, int32_t L, int32_t *block, int64_t *resident);
+
 #ifdef __cplusplus
 }
 #endif

@@ -13,7 +13,7 @@ SYMBOLS = ("mhc_version", "mhc_status_string", "mhc_pre_workspace_size", "mhc_pr
            "mhc_backward_workspace_size", "mhc_backward", "mhc_backward_map", "mhc_backward_apply",
            "mhc_backward_noalloc", "mhc_post_backward", "mhc_pre_backward_workspace_size",
            "mhc_pre_backward", "mhc_post_fused_workspace_size", "mhc_post_fused",
-           "mhc_layer_input", "mhc_sinkhorn_knopp", "mhc_depth_amax")
+           "mhc_layer_input", "mhc_sinkhorn_knopp", "mhc_depth_amax", "mhc_recompute_plan")
 
 
 class MhcParams(ctypes.Structure):
@@ -73,5 +73,9 @@ def load() -> ctypes.CDLL:
     lib.mhc_sinkhorn_knopp.argtypes = [i32, i32, i64, vp, vp, vp, vp]
     lib.mhc_depth_amax.restype = i32
     lib.mhc_depth_amax.argtypes = [i32, i64, i32, vp, vp, vp, vp, vp]
+    lib.mhc_recompute_plan.restype = i32
+    lib.mhc_recompute_plan.argtypes = [ctypes.c_int32, ctypes.c_int32,
+                                       ctypes.POINTER(ctypes.c_int32),
+                                       ctypes.POINTER(ctypes.c_int64)]
     _lib = lib
     return lib

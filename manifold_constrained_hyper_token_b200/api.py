@@ -282,3 +282,12 @@ def mhc_depth_amax(H, *, out=None, dev_status=None, stream=None):
                                     _p(dev_status), _stream(stream))
     _check(st, "mhc_depth_amax")
     return gf, gb
+
+
+def mhc_recompute_plan(n: int, L: int):
+    """(block, resident): the recompute block size for an L-layer stack with n streams and
+    the resident activations per token at the backward's peak, in units of C elements."""
+    blk, res = ctypes.c_int32(0), ctypes.c_int64(0)
+    st = _lib.load().mhc_recompute_plan(int(n), int(L), ctypes.byref(blk), ctypes.byref(res))
+    _check(st, "mhc_recompute_plan")
+    return int(blk.value), int(res.value)

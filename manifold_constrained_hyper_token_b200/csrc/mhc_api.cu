@@ -370,4 +370,18 @@ mhc_status mhc_depth_amax(int n, int64_t T, int L, const float* H, float* gain_f
       mhc::depth_amax_dispatch(n, T, L, H, gain_fwd, gain_bwd, (cudaStream_t)stream));
 }
 
+mhc_status mhc_recompute_plan(int32_t n, int32_t L, int32_t* block, int64_t* resident) {
+  if (n < 1 || L < 1 || block == nullptr) return MHC_ERR_INVALID_ARG;
+  int32_t best = 1;
+  int64_t best_r = -1;
+  for (int32_t B = 1; B <= L; ++B) {
+    const int64_t blocks = ((int64_t)L + B - 1) / B;
+    const int64_t r = (int64_t)n * (blocks - 1) + (int64_t)(n + 2) * B;
+    if (best_r < 0 || r < best_r) { best_r = r; best = B; }
+  }
+  *block = best;
+  if (resident) *resident = best_r;
+  return MHC_OK;
+}
+
 }  // extern "C"
