@@ -287,9 +287,11 @@ MHC_API mhc_status mhc_pre_backward(const mhc_params *p, const void *x, const fl
  * Arguments, layouts, results and errors are those of mhc_backward, minus
  * the workspace.  The scratch is a library-owned device array of
  * MHC_NOALLOC_SCRATCH_BYTES that every GPU loading this library holds until
- * the process exits.  A problem whose mhc_backward_workspace_size() exceeds
- * MHC_NOALLOC_SCRATCH_BYTES is rejected with MHC_ERR_WORKSPACE before any
- * launch (n = 4: up to about 20,000 tokens per call).  The first call on a
+ * the process exits.  The call runs the CUDA-core kernels, whose scratch is
+ * a per-token record (n = 4: 208 bytes) and a partial sum per 64 tokens; a
+ * problem whose scratch exceeds MHC_NOALLOC_SCRATCH_BYTES is rejected with
+ * MHC_ERR_WORKSPACE before any launch (n = 4: up to about 20,000 tokens per
+ * call).  The first call on a
  * device looks up the array's device address (cudaGetSymbolAddress) with
  * that device current and caches it; make that first call before any stream
  * capture.  All calls share the one array and it keeps the last call's

@@ -59,8 +59,20 @@ extern "C" mhc_status mhc_backward_noalloc(const mhc_params* p, const void* x, c
   if (p == nullptr) return MHC_ERR_INVALID_ARG;
   if (p->n != 1 && p->n != 2 && p->n != 4 && p->n != 8) return MHC_ERR_UNSUPPORTED;
   if (p->dtype != MHC_DTYPE_F32 && p->dtype != MHC_DTYPE_BF16) return MHC_ERR_UNSUPPORTED;
-  const size_t need = mhc_backward_workspace_size(p);
-  if (need == 0) return MHC_ERR_INVALID_ARG;  // a size, t_max or eps out of range
+  if (mhc_backward_workspace_size(p) == 0) return MHC_ERR_INVALID_ARG;  // T, C, t_max or eps
+  // this entry point runs the CUDA-core kernels: per-token records, then the
+  // per-64-token partial sums
+  const int coef_floats = p->n == 1   ? mhc::Coef<1>::SIZE
+                          : p->n == 2 ? mhc::Coef<2>::SIZE
+                          : p->n == 8 ? mhc::Coef<8>::SIZE
+                                      : mhc::Coef<4>::SIZE;
+  const int dz_floats = p->n == 1   ? mhc::Coef<1>::DZ_SIZE
+                        : p->n == 2 ? mhc::Coef<2>::DZ_SIZE
+                        : p->n == 8 ? mhc::Coef<8>::DZ_SIZE
+                                    : mhc::Coef<4>::DZ_SIZE;
+  const int nparts = (int)((p->T + 63) / 64);
+  const size_t coef_bytes = round_up((size_t)p->T * coef_floats * 4, 256);
+  const size_t need = coef_bytes + (size_t)nparts * dz_floats * 4;
   if (need > (size_t)MHC_NOALLOC_SCRATCH_BYTES) return MHC_ERR_WORKSPACE;
   auto ok16 = [](const void* q) { return q != nullptr && ((uintptr_t)q & 15u) == 0; };
   if (!ok16(x) || !ok16(phi) || !ok16(b) || !ok16(alpha) || !ok16(f_out) || !ok16(grad_x_next) ||
@@ -71,17 +83,11 @@ extern "C" mhc_status mhc_backward_noalloc(const mhc_params* p, const void* x, c
   void* scratch = nullptr;
   if (scratch_address(&scratch) != cudaSuccess) return MHC_ERR_CUDA;
 
-  // Same carving as the caller-workspace path: per-token records, then the
-  // per-64-token partial sums.  Both are written in full by the first kernel
-  // before the second reads them, so no part of the scratch needs clearing.
-  const int coef_floats = p->n == 1   ? mhc::Coef<1>::SIZE
-                          : p->n == 2 ? mhc::Coef<2>::SIZE
-                          : p->n == 8 ? mhc::Coef<8>::SIZE
-                                      : mhc::Coef<4>::SIZE;
-  const int nparts = (int)((p->T + 63) / 64);
+  // Both parts are written in full by the first kernel before the second
+  // reads them, so no part of the scratch needs clearing.
   char* ws = (char*)scratch;
   float* coef = (float*)ws;
-  float* part = (float*)(ws + round_up((size_t)p->T * coef_floats * 4, 256));
+  float* part = (float*)(ws + coef_bytes);
 
   cudaStream_t s = (cudaStream_t)stream;
   const int ag = p->alpha_groups == 3 ? 3 : 1;
