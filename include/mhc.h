@@ -94,7 +94,10 @@ typedef enum mhc_dtype {
 
 /* Problem description shared by mhc_pre / mhc_post / mhc_backward. */
 typedef struct mhc_params {
-  int32_t n;      /* streams; this build supports n in {1, 2, 4, 8}           */
+  int32_t n;      /* streams; this build supports n in {1, 2, 4, 8, 16}; bf16
+                     with n = 4 runs the tensor-core kernels, n = 16 its own
+                     CUDA-core kernels (288 logits per token), the rest the
+                     CUDA-core kernels; mhc_backward_noalloc takes n <= 8    */
   int32_t t_max;  /* Sinkhorn-Knopp iterations (row then column pass), >= 0   */
   int64_t T;      /* tokens, 1 <= T <= 2^31 - 257 (32-bit tile coordinates)    */
   int64_t C;      /* channels per stream, >= 8 and a multiple of 8            */
@@ -285,7 +288,7 @@ MHC_API mhc_status mhc_pre_backward(const mhc_params *p, const void *x, const fl
  * method.
  *
  * Arguments, layouts, results and errors are those of mhc_backward, minus
- * the workspace.  The scratch is a library-owned device array of
+ * the workspace, and n = 16 is not taken (MHC_ERR_UNSUPPORTED).  The scratch is a library-owned device array of
  * MHC_NOALLOC_SCRATCH_BYTES that every GPU loading this library holds until
  * the process exits.  The call runs the CUDA-core kernels, whose scratch is
  * a per-token record (n = 4: 208 bytes) and a partial sum per 64 tokens; a

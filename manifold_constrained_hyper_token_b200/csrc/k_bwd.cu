@@ -203,6 +203,9 @@ cudaError_t apply_dispatch(int n, int dtype, int64_t T, int64_t C, const void* x
                            const void* G, const void* g, const float* coef, const float* part,
                            int nparts, void* gx, void* gf, float* gphi, float* gb, float* ga,
                            int ag, cudaStream_t s) {
+  if (n == 16)
+    return wide_apply_dispatch(dtype, T, C, x, phi, G, g, coef, part, nparts, gx, gf, gphi, gb, ga,
+                               ag, s);
 #define MHC_APPLY(NN)                                                                        \
   case NN:                                                                                   \
     return dtype == MHC_DTYPE_BF16                                                           \

@@ -370,6 +370,9 @@ cudaError_t map_fwd_dispatch(int n, int dtype, int64_t T, int64_t C, int iters, 
                              const void* x, const float* phi, const float* b, const float* alpha,
                              int ag,
                              float* Hpre, float* Hpost, float* Hres, int* st, cudaStream_t s) {
+  if (n == 16)
+    return wide_map_dispatch(MAP_FWD, dtype, T, C, iters, eps, x, phi, b, alpha, ag, Hpre, Hpost,
+                             Hres, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, st, s);
 #define MHC_MAPF(NN)                                                                             \
   case NN:                                                                                       \
     return dtype == MHC_DTYPE_BF16                                                               \
@@ -409,6 +412,10 @@ cudaError_t map_bwd_dispatch(int n, int dtype, int64_t T, int64_t C, int iters, 
                              int ag,
                              const void* G, const void* g, const void* f, const float* red,
                              float* coef, float* part, int* st, cudaStream_t s) {
+  if (n == 16)
+    return wide_map_dispatch(red == nullptr ? MAP_BWD : MAP_BWD_SPLIT, dtype, T, C, iters, eps, x,
+                             phi, b, alpha, ag, nullptr, nullptr, nullptr, G, g, f, red, coef,
+                             part, st, s);
 #define MHC_MAPB(NN)                                                                          \
   case NN:                                                                                    \
     return dtype == MHC_DTYPE_BF16                                                            \

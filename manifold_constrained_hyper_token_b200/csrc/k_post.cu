@@ -207,6 +207,7 @@ static cudaError_t launch_hin_t(int64_t T, int64_t C, const void* x, const float
 
 cudaError_t post_dispatch(int n, int dtype, int64_t T, int64_t C, const void* x, const void* f,
                           const float* Hpost, const float* Hres, void* xn, cudaStream_t s) {
+  if (n == 16) return wide_post_dispatch(dtype, T, C, x, f, Hpost, Hres, xn, s);
 #define MHC_POST_CASE(NN)                                                                   \
   case NN:                                                                                  \
     return dtype == MHC_DTYPE_BF16                                                          \
@@ -236,6 +237,7 @@ static cudaError_t launch_post_bwd_t(int64_t T, int64_t C, const void* x, const 
 cudaError_t post_bwd_dispatch(int n, int dtype, int64_t T, int64_t C, const void* x, const void* f,
                               const float* Hpost, const void* G, void* gf, float* red,
                               cudaStream_t s) {
+  if (n == 16) return wide_post_bwd_dispatch(dtype, T, C, x, f, Hpost, G, gf, red, s);
 #define MHC_PBWD_CASE(NN)                                                                      \
   case NN:                                                                                     \
     return dtype == MHC_DTYPE_BF16                                                             \
@@ -262,6 +264,7 @@ cudaError_t hin_dispatch(int n, int dtype, int64_t T, int64_t C, const void* x, 
     MHC_HIN_CASE(2)
     MHC_HIN_CASE(4)
     MHC_HIN_CASE(8)
+    MHC_HIN_CASE(16)
     default: return cudaErrorInvalidValue;
   }
 #undef MHC_HIN_CASE

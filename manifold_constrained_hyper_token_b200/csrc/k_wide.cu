@@ -1,0 +1,720 @@
+// k_wide.cu -- the mHC layer for a wide stream buffer (n = 16) on the CUDA cores.
+//
+// The same operators as k_map / k_post / k_bwd (the RMS-normalised
+// projection, the gates, Sinkhorn-Knopp and its adjoint, the post merge and
+// the backward apply; chatgpz.de explainer, sections "Von
+// Residualverbindungen zu Hyperverbindungen" and "Systemarbeit und
+// Schulungsaufwand"; reportify.cn [16]-[21]).  At n = 16 a token has M = 288
+// logits and a 16 x 16 residual mixer, so the per-thread register tiling of
+// those kernels does not fit.  Here:
+//
+//   k_wide_map        32 tokens per CTA: the projection y = x . phi as a
+//                     CUDA-core GEMM over the flattened k = i*C + c (with the
+//                     sum of squares), for the backward the 288 C-reductions
+//                     per token, then one thread per token for the gates,
+//                     Sinkhorn and (backward) its adjoint
+//   k_wide_post       x_next = H_res x + H_post^T f_out, coefficients in
+//                     shared memory
+//   k_wide_post_bwd   the post half of the backward in training order:
+//                     grad_f_out and <G_i, x_j>, <G_i, f_out>
+//   k_wide_apply_x    grad_x = phi u + H_res^T G + H_pre g - kappa x and
+//                     grad_f_out, the phi u term a GEMM over the logits
+//   k_wide_apply_phi  grad_phi = sum_t x_t u_t^T, a GEMM over the tokens
+//   k_wide_bias       grad_b and grad_alpha from the mapping CTAs' partials
+//
+// Every sum is taken in a fixed order, so repeated calls give identical bits.
+// The per-token Sinkhorn arrays (16 x 16) live in local memory.
+#include "mhc_common.cuh"
+#include "mhc_dispatch.h"
+
+namespace mhc {
+
+namespace widek {
+constexpr int N = 16;
+constexpr int M = N * N + 2 * N;   // 288 logits
+constexpr int TB = 32;             // tokens per mapping CTA
+constexpr int NT = 256;
+constexpr int KC = 32;             // projection: k rows per chunk
+constexpr int CPT = M / 32;        // logit columns (or dot products) per thread: 9
+constexpr int CQ = 8;              // reductions: channels per chunk
+constexpr int CQP = CQ + 1;        // padded stride of a (token, stream) row
+// shared memory of k_wide_map, in floats
+constexpr int STG = KC * TB + KC * M;             // 10240: staging (projection)
+constexpr int RED_STG = 2 * TB * N * CQP + 2 * TB * CQ;  // 9728: staging (reductions)
+constexpr int DZS = TB * (M + 3);                 // 9312: the epilogue's dz rows
+static_assert(RED_STG <= STG && DZS <= STG, "staging area");
+constexpr int YS_OFF = STG;                       // [TB][M] projections
+constexpr int DT_OFF = YS_OFF + TB * M;           // [TB][M] C-reductions
+constexpr int SS_OFF = DT_OFF + TB * M;           // [TB] sums of squares
+constexpr int SMEM_FLOATS = SS_OFF + TB;
+}  // namespace widek
+
+enum WideDots { WD_FULL = 0, WD_PRE = 1, WD_POST = 2 };
+
+// The C-reductions of one CTA's TB tokens, as dacc[token 4*ty + i][dot tx + 32q]:
+//   dot d < 256         <G_i, x_j>   (i = d / 16, j = d % 16)        WD_FULL, WD_POST
+//   256 <= d < 272      <g, x_i>     (i = d - 256)                    WD_FULL, WD_PRE
+//   272 <= d < 288      <G_i, f>     (i = d - 272)                    WD_FULL, WD_POST
+// Channels are taken in chunks of CQ, in order.  With WD_POST the chunk loop
+// also writes grad_f_out = sum_i H_post[i] G_i (hp: [TB][N] in shared memory).
+template <typename TIO, int WHICH>
+__device__ __forceinline__ void wide_dots(int64_t T, int64_t C, int64_t t0, const TIO* x,
+                                          const TIO* G, const TIO* g, const TIO* f,
+                                          const float* hp, TIO* gf, float* stg,
+                                          float (&dacc)[4][widek::CPT]) {
+  using namespace widek;
+  const int tid = threadIdx.x, ty = tid >> 5, tx = tid & 31;
+  float* xq = stg;                        // [TB][N][CQP]
+  float* Gq = xq + TB * N * CQP;          // [TB][N][CQP]
+  float* gq = Gq + TB * N * CQP;          // [TB][CQ]
+  float* fq = gq + TB * CQ;               // [TB][CQ]
+  constexpr bool USE_G = WHICH != WD_PRE;
+  constexpr bool USE_g = WHICH != WD_POST;
+  constexpr bool USE_f = WHICH != WD_PRE;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int q = 0; q < CPT; ++q) dacc[i][q] = 0.0f;
+  for (int64_t c0 = 0; c0 < C; c0 += CQ) {
+    // (token, stream, channel) elements: TB * N * CQ = 4096, 16 per thread
+#pragma unroll 4
+    for (int r = 0; r < TB * N * CQ / NT; ++r) {
+      const int e = tid + NT * r;
+      const int cc = e & (CQ - 1), j = (e >> 3) & (N - 1), tok = e >> 7;
+      const int64_t t = t0 + tok, c = c0 + cc;
+      const bool ok = t < T && c < C;
+      const int64_t gi = (t * N + j) * C + c;
+      xq[(tok * N + j) * CQP + cc] = ok ? to_f32(x[gi]) : 0.0f;
+      if constexpr (USE_G) Gq[(tok * N + j) * CQP + cc] = ok ? to_f32(G[gi]) : 0.0f;
+    }
+    {
+      // (token, channel) elements: TB * CQ = 256, one per thread
+      const int cc = tid & (CQ - 1), tok = tid >> 3;
+      const int64_t t = t0 + tok, c = c0 + cc;
+      const bool ok = t < T && c < C;
+      if constexpr (USE_g) gq[tid] = ok ? to_f32(g[t * C + c]) : 0.0f;
+      if constexpr (USE_f) fq[tid] = ok ? to_f32(f[t * C + c]) : 0.0f;
+    }
+    __syncthreads();
+    if constexpr (WHICH == WD_POST) {
+      // grad_f_out for (token tid / CQ, channel tid % CQ)
+      const int cc = tid & (CQ - 1), tok = tid >> 3;
+      const int64_t t = t0 + tok, c = c0 + cc;
+      if (t < T && c < C) {
+        float b = 0.0f;
+#pragma unroll
+        for (int i = 0; i < N; ++i) b = fmaf(hp[tok * N + i], Gq[(tok * N + i) * CQP + cc], b);
+        if constexpr (sizeof(TIO) == 2) gf[t * C + c] = __float2bfloat16_rn(b);
+        else gf[t * C + c] = b;
+      }
+    }
+#pragma unroll
+    for (int cc = 0; cc < CQ; ++cc) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int tok = 4 * ty + i;
+        const float* xr = xq + tok * N * CQP + cc;
+        const float* Gr = Gq + tok * N * CQP + cc;
+        if constexpr (WHICH != WD_PRE) {
+          // dots tx + 32 q < 256: <G_i, x_j>, j = tx % 16, i = tx / 16 + 2 q
+          const float xj = xr[(tx & (N - 1)) * CQP];
+#pragma unroll
+          for (int q = 0; q < CPT - 1; ++q)
+            dacc[i][q] = fmaf(Gr[((tx >> 4) + 2 * q) * CQP], xj, dacc[i][q]);
+        }
+        // dot 256 + tx: tx < 16 <g, x_tx>; tx >= 16 <G_(tx-16), f>
+        if (tx < N) {
+          if constexpr (USE_g) dacc[i][CPT - 1] = fmaf(gq[tok * CQ + cc], xr[tx * CQP], dacc[i][CPT - 1]);
+        } else {
+          if constexpr (USE_f)
+            dacc[i][CPT - 1] = fmaf(Gr[(tx - N) * CQP], fq[tok * CQ + cc], dacc[i][CPT - 1]);
+        }
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// The per-token epilogue for token t0 + tid: gates, Sinkhorn and, in the
+// backward, its adjoint, the coefficient record and the token's dz row.  Its
+// 16 x 16 arrays live in local memory: the forward runs it inside k_wide_map,
+// the backward in k_wide_bwd_epi, apart from the GEMM loops' registers.
+// yr: the token's M projections, dt: its M dot products (backward), ss: its
+// sum of squares.  In the backward yr and dt are the token's own coefficient
+// row, which is read in full before the record is written over it; the caller
+// runs the backward epilogue only for tokens t < T.
+template <int MODE>
+__device__ __forceinline__ void wide_epilogue(int tid, int64_t t, int64_t T, int64_t K, int iters,
+                                           float eps, const float* yr, const float* dt, float ss,
+                                           const float* bias, const float* alpha_p, int ag,
+                                           float* Hpre_o, float* Hpost_o, float* Hres_o,
+                                           const float* red_in, float* coef_o, float* dzs,
+                                           int* status) {
+  using namespace widek;
+  constexpr bool BWD = MODE != MAP_FWD;
+  constexpr bool SPLIT = MODE == MAP_BWD_SPLIT;
+  using CF = Coef<N>;
+  const bool mine = t < T;
+  const float r = sqrtf(ss / (float)K + eps);
+  Alpha3 al;
+  al.load(alpha_p, ag);
+  float spre[N], spost[N], zres[N * N];
+  bool bad = !isfinite(r);
+  for (int m = 0; m < M; ++m) {
+    const float y = yr[m] / r;
+    const float z = fmaf(al.at<N>(m), y, __ldg(bias + m));
+    bad |= !isfinite(z);
+    if (m < N) spre[m] = sigmoidf_(z);
+    else if (m < 2 * N) spost[m - N] = sigmoidf_(z);
+    else zres[m - 2 * N] = z;
+  }
+  if (mine && bad) flag_status(status, MHC_ERR_NONFINITE);
+  float H[N * N];
+  for (int e = 0; e < N * N; ++e) H[e] = zres[e];
+  sk_forward<N>(H, iters);
+  if constexpr (!BWD) {
+    if (mine) {
+      for (int i = 0; i < N; ++i) {
+        Hpre_o[t * N + i] = spre[i];
+        Hpost_o[t * N + i] = 2.0f * spost[i];
+      }
+      for (int e = 0; e < N * N; ++e) Hres_o[t * N * N + e] = H[e];
+    }
+  } else {
+    const float* rt = red_in + (SPLIT && mine ? t * (N * N + N) : 0);
+    float dA[N * N], dz[M];
+    for (int e = 0; e < N * N; ++e) dA[e] = !mine ? 0.0f : (SPLIT ? __ldg(rt + e) : dt[e]);
+    float dzres[N * N];
+    sk_adjoint<N>(zres, dA, dzres, iters);
+    for (int i = 0; i < N; ++i) {
+      dz[i] = dt[N * N + i] * spre[i] * (1.0f - spre[i]);
+      const float dpost = !mine ? 0.0f : (SPLIT ? __ldg(rt + N * N + i) : dt[N * N + N + i]);
+      dz[N + i] = dpost * 2.0f * spost[i] * (1.0f - spost[i]);
+    }
+    for (int e = 0; e < N * N; ++e) dz[2 * N + e] = dzres[e];
+    float dzy[3] = {0.0f, 0.0f, 0.0f};  // dz . y over the pre, post, res logits
+    for (int m = 0; m < M; ++m) {
+      const int grp = m < N ? 0 : (m < 2 * N ? 1 : 2);
+      dzy[grp] = fmaf(dz[m], yr[m] / r, dzy[grp]);
+    }
+    if (mine) {
+      float* co = coef_o + t * CF::SIZE;
+      for (int e = 0; e < N * N; ++e) co[CF::RES + e] = H[e];
+      for (int i = 0; i < N; ++i) {
+        co[CF::PRE + i] = spre[i];
+        co[CF::POST + i] = 2.0f * spost[i];
+      }
+      float ar[3];
+      for (int gr = 0; gr < 3; ++gr) ar[gr] = al.a[gr] / r;
+      for (int m = 0; m < M; ++m) co[CF::U + m] = ar[m < N ? 0 : (m < 2 * N ? 1 : 2)] * dz[m];
+      const float wdzy = fmaf(al.a[2], dzy[2], fmaf(al.a[1], dzy[1], al.a[0] * dzy[0]));
+      co[CF::KAPPA] = wdzy / ((float)K * r * r);
+      for (int e = CF::KAPPA + 1; e < CF::SIZE; ++e) co[e] = 0.0f;
+    }
+    for (int m = 0; m < M; ++m) dzs[tid * (M + 3) + m] = mine ? dz[m] : 0.0f;
+    for (int gr = 0; gr < 3; ++gr) dzs[tid * (M + 3) + M + gr] = mine ? dzy[gr] : 0.0f;
+  }
+  }
+
+// MAP_FWD: H_pre / H_post / H_res.  MAP_BWD: coef [T][Coef<16>::SIZE] and per
+// CTA the sums over its tokens of dz and dz . y (part [grid][DZ_SIZE]).
+// MAP_BWD_SPLIT: as MAP_BWD with <G_i, x_j> and <G_i, f_out> from `red`.
+template <typename TIO, int MODE>
+__global__ void __launch_bounds__(widek::NT) k_wide_map(
+    int64_t T, int64_t C, int iters, float eps, const TIO* __restrict__ x,
+    const float* __restrict__ phi, const float* __restrict__ bias,
+    const float* __restrict__ alpha_p, int ag, float* __restrict__ Hpre_o,
+    float* __restrict__ Hpost_o, float* __restrict__ Hres_o, const TIO* __restrict__ G,
+    const TIO* __restrict__ g, const TIO* __restrict__ f, const float* __restrict__ red_in,
+    float* __restrict__ coef_o, float* __restrict__ part_o, int* status) {
+  using namespace widek;
+  constexpr bool BWD = MODE != MAP_FWD;
+  constexpr bool SPLIT = MODE == MAP_BWD_SPLIT;
+  using CF = Coef<N>;
+  extern __shared__ __align__(16) float smem[];
+  float* stg = smem;
+  float* ys = smem + YS_OFF;
+  float* dts = smem + DT_OFF;
+  float* sss = smem + SS_OFF;
+  const int tid = threadIdx.x, ty = tid >> 5, tx = tid & 31;
+  const int64_t t0 = (int64_t)blockIdx.x * TB;
+  const int64_t K = (int64_t)N * C;
+
+  // ---- projection y[t][m] = sum_k x[t][k] phi[k][m], and the sums of squares
+  {
+    float* xs = stg;            // [KC][TB]
+    float* ps = stg + KC * TB;  // [KC][M]
+    float acc[4][CPT], ssp[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      ssp[i] = 0.0f;
+#pragma unroll
+      for (int q = 0; q < CPT; ++q) acc[i][q] = 0.0f;
+    }
+    for (int64_t k0 = 0; k0 < K; k0 += KC) {
+#pragma unroll
+      for (int r = 0; r < TB * KC / NT; ++r) {
+        const int tok = ty + 8 * r;
+        const int64_t t = t0 + tok, k = k0 + tx;
+        const float v = (t < T && k < K) ? to_f32(x[t * K + k]) : 0.0f;
+        xs[tx * TB + tok] = v;
+        ssp[r] = fmaf(v, v, ssp[r]);
+      }
+      for (int e = tid; e < KC * M; e += NT) {
+        const int kk = e / M;
+        ps[e] = (k0 + kk < K) ? __ldg(phi + (k0 + kk) * M + (e - kk * M)) : 0.0f;
+      }
+      __syncthreads();
+#pragma unroll 4
+      for (int kk = 0; kk < KC; ++kk) {
+        const float4 a = *reinterpret_cast<const float4*>(xs + kk * TB + 4 * ty);
+        const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int q = 0; q < CPT; ++q) {
+          const float bq = ps[kk * M + tx + 32 * q];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[i][q] = fmaf(av[i], bq, acc[i][q]);
+        }
+      }
+      __syncthreads();
+    }
+    // the backward stages y, the dot products and the sum of squares in the
+    // token's coefficient row: [0, M) y, [M, 2M) dots, [2M] sum of squares
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int64_t t = t0 + 4 * ty + i;
+#pragma unroll
+      for (int q = 0; q < CPT; ++q) {
+        if constexpr (BWD) {
+          if (t < T) coef_o[t * CF::SIZE + tx + 32 * q] = acc[i][q];
+        } else {
+          ys[(4 * ty + i) * M + tx + 32 * q] = acc[i][q];
+        }
+      }
+    }
+    // token ty + 8r: its 32 k-slots sit in the 32 lanes; xor tree, fixed order
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      float v = ssp[r];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (tx == 0) {
+        const int64_t t = t0 + ty + 8 * r;
+        if constexpr (BWD) {
+          if (t < T) coef_o[t * CF::SIZE + 2 * M] = v;
+        } else {
+          sss[ty + 8 * r] = v;
+        }
+      }
+    }
+  }
+
+  // ---- the C-reductions of the backward
+  if constexpr (BWD) {
+    float dacc[4][CPT];
+    if constexpr (SPLIT)
+      wide_dots<TIO, WD_PRE>(T, C, t0, x, nullptr, g, nullptr, nullptr, nullptr, stg, dacc);
+    else
+      wide_dots<TIO, WD_FULL>(T, C, t0, x, G, g, f, nullptr, nullptr, stg, dacc);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int64_t t = t0 + 4 * ty + i;
+      if (t >= T) continue;
+#pragma unroll
+      for (int q = 0; q < CPT; ++q) coef_o[t * CF::SIZE + M + tx + 32 * q] = dacc[i][q];
+    }
+    return;  // k_wide_bwd_epi finishes these tokens
+  }
+  __syncthreads();
+
+  // ---- the forward's per-token epilogue, one thread per token
+  if constexpr (!BWD) {
+    if (tid < TB)
+      wide_epilogue<MODE>(tid, t0 + tid, T, K, iters, eps, ys + tid * M, nullptr, sss[tid], bias,
+                          alpha_p, ag, Hpre_o, Hpost_o, Hres_o, red_in, coef_o, nullptr, status);
+  }
+}
+
+// The backward's per-token epilogue: one warp per TB tokens reads each token's
+// staged row (y, dot products, sum of squares) from coef, writes the
+// coefficient record over it, and adds the CTA's dz and dz . y rows in token
+// order into part [grid][DZ_SIZE].
+template <int MODE>
+__global__ void __launch_bounds__(32) k_wide_bwd_epi(int64_t T, int64_t C, int iters, float eps,
+                                                     const float* __restrict__ bias,
+                                                     const float* __restrict__ alpha_p, int ag,
+                                                     const float* __restrict__ red_in,
+                                                     float* __restrict__ coef,
+                                                     float* __restrict__ part_o, int* status) {
+  using namespace widek;
+  using CF = Coef<N>;
+  __shared__ float dzs[TB * (M + 3)];
+  const int tid = threadIdx.x;
+  const int64_t t = (int64_t)blockIdx.x * TB + tid;
+  if (t < T) {
+    const float* row = coef + t * CF::SIZE;
+    wide_epilogue<MODE>(tid, t, T, (int64_t)N * C, iters, eps, row, row + M, row[2 * M], bias,
+                        alpha_p, ag, nullptr, nullptr, nullptr, red_in, coef, dzs, status);
+  } else {
+    for (int m = 0; m < M + 3; ++m) dzs[tid * (M + 3) + m] = 0.0f;
+  }
+  __syncwarp();
+  for (int col = tid; col < M + 3; col += 32) {
+    float s = 0.0f;
+    for (int q = 0; q < TB; ++q) s += dzs[q * (M + 3) + col];
+    part_o[(int64_t)blockIdx.x * CF::DZ_SIZE + col] = s;
+  }
+}
+
+// x_next[i][c] = sum_j H_res[i][j] x[j][c] + H_post[i] f_out[c] (the k_post order)
+template <typename TIO>
+__global__ void __launch_bounds__(128) k_wide_post(int64_t T, int64_t C, const TIO* __restrict__ x,
+                                                   const TIO* __restrict__ f,
+                                                   const float* __restrict__ Hpost,
+                                                   const float* __restrict__ Hres,
+                                                   TIO* __restrict__ xn) {
+  using namespace widek;
+  using V = Vec<TIO>;
+  constexpr int W = V::N;
+  __shared__ float hr[N * N], hp[N];
+  const int64_t nv = C / W;
+  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < N * N; e += blockDim.x) hr[e] = __ldg(Hres + t * N * N + e);
+    if (threadIdx.x < N) hp[threadIdx.x] = __ldg(Hpost + t * N + threadIdx.x);
+    __syncthreads();
+    const TIO* xt = x + t * N * C;
+    TIO* ot = xn + t * N * C;
+    for (int64_t v = threadIdx.x; v < nv; v += blockDim.x) {
+      float xv[N][W], fv[W];
+#pragma unroll
+      for (int j = 0; j < N; ++j) V::load_stream(xt + j * C + v * W, xv[j]);
+      V::load_stream(f + t * C + v * W, fv);
+#pragma unroll 1
+      for (int i = 0; i < N; ++i) {
+        float o[W];
+#pragma unroll
+        for (int e = 0; e < W; ++e) {
+          float acc = hp[i] * fv[e];
+#pragma unroll
+          for (int j = 0; j < N; ++j) acc = fmaf(hr[i * N + j], xv[j][e], acc);
+          o[e] = acc;
+        }
+        V::store_stream(ot + i * C + v * W, o);
+      }
+    }
+  }
+}
+
+// The post half of the backward in training order: grad_f_out and
+// red [T][N*N + N] = (<G_i, x_j> row-major, then <G_i, f_out>).
+template <typename TIO>
+__global__ void __launch_bounds__(widek::NT) k_wide_post_bwd(int64_t T, int64_t C,
+                                                             const TIO* __restrict__ x,
+                                                             const TIO* __restrict__ f,
+                                                             const float* __restrict__ Hpost,
+                                                             const TIO* __restrict__ G,
+                                                             TIO* __restrict__ gf,
+                                                             float* __restrict__ red) {
+  using namespace widek;
+  extern __shared__ __align__(16) float smem[];
+  float* hp = smem;        // [TB][N]
+  float* stg = smem + TB * N;
+  const int tid = threadIdx.x, ty = tid >> 5, tx = tid & 31;
+  const int64_t t0 = (int64_t)blockIdx.x * TB;
+  for (int e = tid; e < TB * N; e += NT) {
+    const int64_t t = t0 + e / N;
+    hp[e] = t < T ? __ldg(Hpost + t * N + e % N) : 0.0f;
+  }
+  __syncthreads();
+  float dacc[4][CPT];
+  wide_dots<TIO, WD_POST>(T, C, t0, x, G, nullptr, f, hp, gf, stg, dacc);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t t = t0 + 4 * ty + i;
+    if (t >= T) continue;
+    float* rt = red + t * (N * N + N);
+#pragma unroll
+    for (int q = 0; q < CPT - 1; ++q) rt[tx + 32 * q] = dacc[i][q];
+    if (tx >= N) rt[N * N + tx - N] = dacc[i][CPT - 1];
+  }
+}
+
+// grad_x[t][k] (k = j*C + c) = sum_m phi[k][m] u[t][m] + H_pre[j] g[c]
+//                              + sum_i H_res[i][j] G[i][c] - kappa x[t][k]  (the k_bwd order)
+// grad_f_out[t][c] = sum_i H_post[i] G[i][c]   (when grad_f is not null)
+// A CTA owns 32 tokens x 64 k; the phi u term is a GEMM over the 288 logits.
+template <typename TIO>
+__global__ void __launch_bounds__(widek::NT) k_wide_apply_x(
+    int64_t T, int64_t C, const TIO* __restrict__ x, const float* __restrict__ phi,
+    const TIO* __restrict__ G, const TIO* __restrict__ g, const float* __restrict__ coef,
+    TIO* __restrict__ grad_x, TIO* __restrict__ grad_f) {
+  using namespace widek;
+  using CF = Coef<N>;
+  __shared__ __align__(16) float Us[32 * 32];   // [m][token]
+  __shared__ __align__(16) float ps[32 * 64];   // [m][k]
+  const int tid = threadIdx.x, ty = tid >> 5, tx = tid & 31;
+  const int64_t t0 = (int64_t)blockIdx.x * 32;
+  const int64_t k0 = (int64_t)blockIdx.y * 64;
+  const int64_t K = (int64_t)N * C;
+  float acc[4][2];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = 0.0f;
+  for (int m0 = 0; m0 < M; m0 += 32) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int e = tid + NT * r, tok = e >> 5, mm = e & 31;
+      const int64_t t = t0 + tok;
+      Us[mm * 32 + tok] = t < T ? __ldg(coef + t * CF::SIZE + CF::U + m0 + mm) : 0.0f;
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int e = tid + NT * r, kk = e >> 5, mm = e & 31;
+      const int64_t k = k0 + kk;
+      ps[mm * 64 + kk] = k < K ? __ldg(phi + k * M + m0 + mm) : 0.0f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int mm = 0; mm < 32; ++mm) {
+      const float4 a = *reinterpret_cast<const float4*>(Us + mm * 32 + 4 * ty);
+      const float av[4] = {a.x, a.y, a.z, a.w};
+      const float b0 = ps[mm * 64 + tx], b1 = ps[mm * 64 + tx + 32];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[i][0] = fmaf(b0, av[i], acc[i][0]);
+        acc[i][1] = fmaf(b1, av[i], acc[i][1]);
+      }
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t t = t0 + 4 * ty + i;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int64_t k = k0 + tx + 32 * h;
+      if (t >= T || k >= K) continue;
+      const int j = (int)(k / C);
+      const int64_t c = k - (int64_t)j * C;
+      const float* co = coef + t * CF::SIZE;
+      float a = fmaf(__ldg(co + CF::PRE + j), to_f32(g[t * C + c]), acc[i][h]);
+      float b = 0.0f;
+#pragma unroll 4
+      for (int i2 = 0; i2 < N; ++i2) {
+        const float Gv = to_f32(G[(t * N + i2) * C + c]);
+        a = fmaf(__ldg(co + CF::RES + i2 * N + j), Gv, a);
+        b = fmaf(__ldg(co + CF::POST + i2), Gv, b);
+      }
+      const float gx = fmaf(-__ldg(co + CF::KAPPA), to_f32(x[t * K + k]), a);
+      if constexpr (sizeof(TIO) == 2) {
+        grad_x[t * K + k] = __float2bfloat16_rn(gx);
+        if (j == 0 && grad_f != nullptr) grad_f[t * C + c] = __float2bfloat16_rn(b);
+      } else {
+        grad_x[t * K + k] = gx;
+        if (j == 0 && grad_f != nullptr) grad_f[t * C + c] = b;
+      }
+    }
+  }
+}
+
+// grad_phi[k][m] = sum_t x[t][k] u[t][m]: a CTA owns 32 rows k x 96 logits and
+// walks every token in order.
+template <typename TIO>
+__global__ void __launch_bounds__(widek::NT) k_wide_apply_phi(int64_t T, int64_t C,
+                                                              const TIO* __restrict__ x,
+                                                              const float* __restrict__ coef,
+                                                              float* __restrict__ grad_phi) {
+  using namespace widek;
+  using CF = Coef<N>;
+  __shared__ __align__(16) float xs[32 * 32];   // [token][k]
+  __shared__ __align__(16) float us[32 * 96];   // [token][m]
+  const int tid = threadIdx.x, ty = tid >> 5, tx = tid & 31;
+  const int64_t k0 = (int64_t)blockIdx.x * 32;
+  const int m0 = blockIdx.y * 96;
+  const int64_t K = (int64_t)N * C;
+  float acc[4][3];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = 0.0f;
+  for (int64_t t0 = 0; t0 < T; t0 += 32) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int e = tid + NT * r, tok = e >> 5, kk = e & 31;
+      const int64_t t = t0 + tok, k = k0 + kk;
+      xs[tok * 32 + kk] = (t < T && k < K) ? to_f32(x[t * K + k]) : 0.0f;
+    }
+#pragma unroll
+    for (int r = 0; r < 12; ++r) {
+      const int e = tid + NT * r, tok = e / 96, mm = e - tok * 96;
+      const int64_t t = t0 + tok;
+      us[e] = (t < T && m0 + mm < M) ? __ldg(coef + t * CF::SIZE + CF::U + m0 + mm) : 0.0f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int tok = 0; tok < 32; ++tok) {
+      const float4 a = *reinterpret_cast<const float4*>(xs + tok * 32 + 4 * ty);
+      const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+      for (int q = 0; q < 3; ++q) {
+        const float b = us[tok * 96 + tx + 32 * q];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i][q] = fmaf(av[i], b, acc[i][q]);
+      }
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t k = k0 + 4 * ty + i;
+#pragma unroll
+    for (int q = 0; q < 3; ++q) {
+      const int m = m0 + tx + 32 * q;
+      if (k < K && m < M) grad_phi[k * M + m] = acc[i][q];
+    }
+  }
+}
+
+// grad_b and grad_alpha: the mapping CTAs' partial sums added in a fixed
+// order (warp w takes partials w, w + 8, ...; the warps' results in order).
+__global__ void __launch_bounds__(widek::NT) k_wide_bias(const float* __restrict__ part,
+                                                         int nparts, float* __restrict__ grad_b,
+                                                         float* __restrict__ grad_alpha, int ag) {
+  using namespace widek;
+  constexpr int NC = M + 3, NW = NT / 32;
+  __shared__ float wsum[(NW + 1) * NC];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int col = lane; col < NC; col += 32) {
+    float s = 0.0f;
+    for (int q = warp; q < nparts; q += NW) s += __ldg(part + (int64_t)q * Coef<N>::DZ_SIZE + col);
+    wsum[warp * NC + col] = s;
+  }
+  __syncthreads();
+  for (int col = threadIdx.x; col < NC; col += NT) {
+    float a = 0.0f;
+    for (int w = 0; w < NW; ++w) a += wsum[w * NC + col];
+    wsum[NW * NC + col] = a;
+    if (col < M) grad_b[col] = a;
+    else if (ag == 3) grad_alpha[col - M] = a;
+  }
+  __syncthreads();
+  // one shared alpha: its gradient is the sum of the three group sums
+  if (ag != 3 && threadIdx.x == 0)
+    *grad_alpha = (wsum[NW * NC + M] + wsum[NW * NC + M + 1]) + wsum[NW * NC + M + 2];
+}
+
+// ------------------------------------------------------------------ host
+template <typename TIO, int MODE>
+static cudaError_t launch_wide_map(int64_t T, int64_t C, int iters, float eps, const void* x,
+                                   const float* phi, const float* b, const float* alpha, int ag,
+                                   float* Hpre, float* Hpost, float* Hres, const void* G,
+                                   const void* g, const void* f, const float* red, float* coef,
+                                   float* part, int* st, cudaStream_t s) {
+  const size_t smem = (size_t)widek::SMEM_FLOATS * 4;
+  auto kern = k_wide_map<TIO, MODE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int64_t grid = (T + widek::TB - 1) / widek::TB;
+  kern<<<(unsigned)grid, widek::NT, smem, s>>>(T, C, iters, eps, (const TIO*)x, phi, b, alpha, ag,
+                                              Hpre, Hpost, Hres, (const TIO*)G, (const TIO*)g,
+                                              (const TIO*)f, red, coef, part, st);
+  e = cudaGetLastError();
+  if constexpr (MODE != MAP_FWD) {
+    if (e != cudaSuccess) return e;
+    k_wide_bwd_epi<MODE><<<(unsigned)grid, 32, 0, s>>>(T, C, iters, eps, b, alpha, ag, red, coef,
+                                                       part, st);
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
+int wide_map_tokens_per_cta() { return widek::TB; }
+
+cudaError_t wide_map_dispatch(int mode, int dtype, int64_t T, int64_t C, int iters, float eps,
+                              const void* x, const float* phi, const float* b, const float* alpha,
+                              int ag, float* Hpre, float* Hpost, float* Hres, const void* G,
+                              const void* g, const void* f, const float* red, float* coef,
+                              float* part, int* st, cudaStream_t s) {
+  const bool bf = dtype == MHC_DTYPE_BF16;
+#define MHC_WMAP(MODE_)                                                                          \
+  return bf ? launch_wide_map<__nv_bfloat16, MODE_>(T, C, iters, eps, x, phi, b, alpha, ag, Hpre, \
+                                                    Hpost, Hres, G, g, f, red, coef, part, st, s) \
+            : launch_wide_map<float, MODE_>(T, C, iters, eps, x, phi, b, alpha, ag, Hpre, Hpost,  \
+                                            Hres, G, g, f, red, coef, part, st, s);
+  switch (mode) {
+    case MAP_FWD: MHC_WMAP(MAP_FWD)
+    case MAP_BWD: MHC_WMAP(MAP_BWD)
+    case MAP_BWD_SPLIT: MHC_WMAP(MAP_BWD_SPLIT)
+    default: return cudaErrorInvalidValue;
+  }
+#undef MHC_WMAP
+}
+
+cudaError_t wide_post_dispatch(int dtype, int64_t T, int64_t C, const void* x, const void* f,
+                               const float* Hpost, const float* Hres, void* xn, cudaStream_t s) {
+  const int64_t cap = 148 * 16;
+  const unsigned grid = (unsigned)(T < cap ? T : cap);
+  if (dtype == MHC_DTYPE_BF16)
+    k_wide_post<__nv_bfloat16><<<grid, 128, 0, s>>>(T, C, (const __nv_bfloat16*)x,
+                                                    (const __nv_bfloat16*)f, Hpost, Hres,
+                                                    (__nv_bfloat16*)xn);
+  else
+    k_wide_post<float><<<grid, 128, 0, s>>>(T, C, (const float*)x, (const float*)f, Hpost, Hres,
+                                            (float*)xn);
+  return cudaGetLastError();
+}
+
+cudaError_t wide_post_bwd_dispatch(int dtype, int64_t T, int64_t C, const void* x, const void* f,
+                                   const float* Hpost, const void* G, void* gf, float* red,
+                                   cudaStream_t s) {
+  using namespace widek;
+  const size_t smem = (size_t)(TB * N + RED_STG) * 4;
+  const unsigned grid = (unsigned)((T + TB - 1) / TB);
+  cudaError_t e;
+  if (dtype == MHC_DTYPE_BF16) {
+    e = cudaFuncSetAttribute(k_wide_post_bwd<__nv_bfloat16>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k_wide_post_bwd<__nv_bfloat16><<<grid, NT, smem, s>>>(
+        T, C, (const __nv_bfloat16*)x, (const __nv_bfloat16*)f, Hpost, (const __nv_bfloat16*)G,
+        (__nv_bfloat16*)gf, red);
+  } else {
+    e = cudaFuncSetAttribute(k_wide_post_bwd<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    k_wide_post_bwd<float><<<grid, NT, smem, s>>>(T, C, (const float*)x, (const float*)f, Hpost,
+                                                  (const float*)G, (float*)gf, red);
+  }
+  return cudaGetLastError();
+}
+
+template <typename TIO>
+static cudaError_t launch_wide_apply(int64_t T, int64_t C, const void* x, const float* phi,
+                                     const void* G, const void* g, const float* coef,
+                                     const float* part, int nparts, void* gx, void* gf,
+                                     float* gphi, float* gb, float* ga, int ag, cudaStream_t s) {
+  using namespace widek;
+  const int64_t K = (int64_t)N * C;
+  const dim3 gridx((unsigned)((T + 31) / 32), (unsigned)((K + 63) / 64));
+  k_wide_apply_x<TIO><<<gridx, NT, 0, s>>>(T, C, (const TIO*)x, phi, (const TIO*)G, (const TIO*)g,
+                                           coef, (TIO*)gx, (TIO*)gf);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const dim3 gridp((unsigned)((K + 31) / 32), (unsigned)((M + 95) / 96));
+  k_wide_apply_phi<TIO><<<gridp, NT, 0, s>>>(T, C, (const TIO*)x, coef, gphi);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  k_wide_bias<<<1, NT, 0, s>>>(part, nparts, gb, ga, ag);
+  return cudaGetLastError();
+}
+
+cudaError_t wide_apply_dispatch(int dtype, int64_t T, int64_t C, const void* x, const float* phi,
+                                const void* G, const void* g, const float* coef, const float* part,
+                                int nparts, void* gx, void* gf, float* gphi, float* gb, float* ga,
+                                int ag, cudaStream_t s) {
+  return dtype == MHC_DTYPE_BF16
+             ? launch_wide_apply<__nv_bfloat16>(T, C, x, phi, G, g, coef, part, nparts, gx, gf,
+                                                gphi, gb, ga, ag, s)
+             : launch_wide_apply<float>(T, C, x, phi, G, g, coef, part, nparts, gx, gf, gphi, gb,
+                                        ga, ag, s);
+}
+
+}  // namespace mhc

@@ -18,7 +18,7 @@ mhc_status check_params(const mhc_params* p) {
   if (!p) return MHC_ERR_INVALID_ARG;
   if (p->T < 1 || p->C < 8 || (p->C % 8) != 0 || p->t_max < 0) return MHC_ERR_INVALID_ARG;
   if (!(p->eps >= 0.0f) || !isfinite(p->eps)) return MHC_ERR_INVALID_ARG;
-  if (p->n != 1 && p->n != 2 && p->n != 4 && p->n != 8) return MHC_ERR_UNSUPPORTED;
+  if (p->n != 1 && p->n != 2 && p->n != 4 && p->n != 8 && p->n != 16) return MHC_ERR_UNSUPPORTED;
   if (p->dtype != MHC_DTYPE_F32 && p->dtype != MHC_DTYPE_BF16) return MHC_ERR_UNSUPPORTED;
   if (p->alpha_groups != 0 && p->alpha_groups != 1 && p->alpha_groups != 3)
     return MHC_ERR_INVALID_ARG;
@@ -40,6 +40,7 @@ int coef_size(int n) {
     case 1: return mhc::Coef<1>::SIZE;
     case 2: return mhc::Coef<2>::SIZE;
     case 8: return mhc::Coef<8>::SIZE;
+    case 16: return mhc::Coef<16>::SIZE;
     default: return mhc::Coef<4>::SIZE;
   }
 }
@@ -48,6 +49,7 @@ int dz_size(int n) {
     case 1: return mhc::Coef<1>::DZ_SIZE;
     case 2: return mhc::Coef<2>::DZ_SIZE;
     case 8: return mhc::Coef<8>::DZ_SIZE;
+    case 16: return mhc::Coef<16>::DZ_SIZE;
     default: return mhc::Coef<4>::DZ_SIZE;
   }
 }
@@ -69,7 +71,7 @@ struct BwdWorkspace {
 BwdWorkspace bwd_layout(const mhc_params* p) {
   BwdWorkspace w{};
   const bool tc = use_tc(p);
-  const int tokens_per_cta = tc ? 128 : 64;
+  const int tokens_per_cta = tc ? 128 : (p->n == 16 ? mhc::wide_map_tokens_per_cta() : 64);
   w.nparts = (int)((p->T + tokens_per_cta - 1) / tokens_per_cta);
   size_t off = 0;
   if (tc) {

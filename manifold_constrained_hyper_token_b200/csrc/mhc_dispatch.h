@@ -51,6 +51,23 @@ size_t map_tc_phi_bytes(int64_t C);
 // scratch of the channel-split mapping (part records, counters); kscratch
 // must hold this many bytes, 256-byte aligned (may be null when it is 0)
 size_t map_tc_scratch_bytes(int64_t T, int64_t C);
+
+// k_wide.cu (n = 16, CUDA cores); the mapping's mode is a MapMode
+int wide_map_tokens_per_cta();
+cudaError_t wide_map_dispatch(int mode, int dtype, int64_t T, int64_t C, int iters, float eps,
+                              const void* x, const float* phi, const float* b, const float* alpha,
+                              int ag, float* Hpre, float* Hpost, float* Hres, const void* G,
+                              const void* g, const void* f, const float* red, float* coef,
+                              float* part, int* st, cudaStream_t s);
+cudaError_t wide_post_dispatch(int dtype, int64_t T, int64_t C, const void* x, const void* f,
+                               const float* Hpost, const float* Hres, void* xn, cudaStream_t s);
+cudaError_t wide_post_bwd_dispatch(int dtype, int64_t T, int64_t C, const void* x, const void* f,
+                                   const float* Hpost, const void* G, void* gf, float* red,
+                                   cudaStream_t s);
+cudaError_t wide_apply_dispatch(int dtype, int64_t T, int64_t C, const void* x, const float* phi,
+                                const void* G, const void* g, const float* coef, const float* part,
+                                int nparts, void* gx, void* gf, float* gphi, float* gb, float* ga,
+                                int ag, cudaStream_t s);
 cudaError_t post_map_tc_dispatch(int64_t T, int64_t C, int iters, float eps, const void* x,
                                  const void* f, const float* Hpost_in, const float* Hres_in,
                                  const float* phi_next, void* phi_split, const float* b_next,

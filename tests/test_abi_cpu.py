@@ -67,7 +67,7 @@ ODD = ctypes.c_void_p(0x10004)
 @pytest.mark.parametrize("kw,code", [
     (dict(T=0), 1), (dict(T=2**31 - 256), 1), (dict(C=12), 1), (dict(C=0), 1), (dict(t_max=-1), 1),
     (dict(eps=-1.0), 1),
-    (dict(eps=float("nan")), 1), (dict(n=3), 2), (dict(n=16), 2), (dict(dtype=7), 2),
+    (dict(eps=float("nan")), 1), (dict(n=3), 2), (dict(n=32), 2), (dict(dtype=7), 2),
     (dict(alpha_groups=2), 1),
 ])
 def test_pre_rejects_bad_params(lib, kw, code):

@@ -125,7 +125,7 @@ def test_depth_amax_sinkhorn_batch(mhc, oracle_mod):
 
 # ----------------------------------------------------------------- post
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
-@pytest.mark.parametrize("n", [1, 2, 4, 8])
+@pytest.mark.parametrize("n", [1, 2, 4, 8, 16])
 @pytest.mark.parametrize("T,C", [(1, 8), (67, 24), (130, 256)])
 def test_post_parity(mhc, oracle_mod, dtype, n, T, C):
     d = _inputs(T, n, C, dtype, seed=T + C)
@@ -161,7 +161,7 @@ def _check_pre(mhc, oracle_mod, d, iters, dtype, eps=1e-6):
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
-@pytest.mark.parametrize("n", [1, 2, 4, 8])
+@pytest.mark.parametrize("n", [1, 2, 4, 8, 16])
 @pytest.mark.parametrize("T,C", [(1, 8), (65, 24), (130, 256)])
 @pytest.mark.parametrize("iters", [0, 1, 20])
 def test_pre_parity(mhc, oracle_mod, dtype, n, T, C, iters):
@@ -244,7 +244,7 @@ def _check_bwd(mhc, oracle_mod, d, iters, dtype, eps=1e-6, idx=None, chunk=None)
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
-@pytest.mark.parametrize("n", [1, 2, 4, 8])
+@pytest.mark.parametrize("n", [1, 2, 4, 8, 16])
 @pytest.mark.parametrize("T,C", [(1, 8), (65, 24), (130, 256)])
 @pytest.mark.parametrize("iters", [0, 1, 20])
 def test_backward_parity(mhc, oracle_mod, dtype, n, T, C, iters):
@@ -261,7 +261,7 @@ def test_backward_large_alpha_parity(mhc, oracle_mod, dtype):
 # ---------------------------- cross-layer fusion: post(l) + mapping(l+1)
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
 @pytest.mark.parametrize("n,T,C", [(1, 33, 24), (2, 70, 64), (4, 300, 520), (4, 1, 8), (4, 129, 4096),
-                                   (8, 65, 136)])
+                                   (8, 65, 136), (16, 33, 64)])
 def test_post_fused_parity(mhc, oracle_mod, dtype, n, T, C):
     """x_next and layer l+1's maps against the oracle's post then pre, and bit for bit
     against the unfused mhc_post -> mhc_pre (the fused kernel maps the stored x_next)."""
@@ -301,7 +301,8 @@ def _hpost(T, n, seed):
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
-@pytest.mark.parametrize("n,T,C", [(1, 33, 24), (2, 70, 64), (4, 300, 520), (4, 1, 8), (8, 65, 136)])
+@pytest.mark.parametrize("n,T,C", [(1, 33, 24), (2, 70, 64), (4, 300, 520), (4, 1, 8), (8, 65, 136),
+                                   (16, 40, 64)])
 def test_post_backward_parity(mhc, oracle_mod, dtype, n, T, C):
     """grad_f_out within the I/O tolerance; red (fp32 sums over C of exact products)
     within 1e-5."""
@@ -315,7 +316,8 @@ def test_post_backward_parity(mhc, oracle_mod, dtype, n, T, C):
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
-@pytest.mark.parametrize("n,T,C", [(1, 33, 24), (2, 70, 64), (4, 300, 520), (4, 1, 8), (8, 65, 136)])
+@pytest.mark.parametrize("n,T,C", [(1, 33, 24), (2, 70, 64), (4, 300, 520), (4, 1, 8), (8, 65, 136),
+                                   (16, 40, 64)])
 @pytest.mark.parametrize("iters", [1, 20])
 def test_pre_backward_parity(mhc, oracle_mod, dtype, n, T, C, iters):
     """The pre half on the same red as the oracle (the oracle's post-half red,
@@ -384,7 +386,7 @@ def _alpha3_errs(ga, ref_ga, per_token):
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
-@pytest.mark.parametrize("n,T,C", [(4, 130, 520), (2, 65, 24)])
+@pytest.mark.parametrize("n,T,C", [(4, 130, 520), (2, 65, 24), (16, 33, 64)])
 def test_pre_per_group_alpha(mhc, oracle_mod, dtype, n, T, C):
     d = _inputs(T, n, C, dtype, seed=11 * T + n)
     d["alpha"] = torch.tensor(ALPHA3, dtype=torch.float32)
@@ -396,7 +398,7 @@ def test_pre_per_group_alpha(mhc, oracle_mod, dtype, n, T, C):
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
-@pytest.mark.parametrize("n,T,C", [(4, 130, 520), (2, 65, 24), (8, 33, 136)])
+@pytest.mark.parametrize("n,T,C", [(4, 130, 520), (2, 65, 24), (8, 33, 136), (16, 33, 64)])
 def test_backward_per_group_alpha(mhc, oracle_mod, dtype, n, T, C):
     d = _inputs(T, n, C, dtype, seed=13 * T + n)
     d["alpha"] = torch.tensor(ALPHA3, dtype=torch.float32)
@@ -450,6 +452,18 @@ def test_pre_backward_small_workspace_rejected(mhc):
 
 def test_backward_is_deterministic(mhc):
     d = _dev(_inputs(300, 4, 512, torch.bfloat16, seed=4))
+    a = mhc.mhc_backward(d["x"], d["phi"], d["b"], d["alpha"], d["f_out"], d["grad_x_next"],
+                         d["grad_h_in"])
+    b = mhc.mhc_backward(d["x"], d["phi"], d["b"], d["alpha"], d["f_out"], d["grad_x_next"],
+                         d["grad_h_in"])
+    for u, v in zip(a, b):
+        assert torch.equal(u, v)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_wide_backward_is_deterministic(mhc, dtype):
+    """n = 16 runs its own kernels (k_wide.cu): fixed-order sums there too."""
+    d = _dev(_inputs(100, 16, 136, dtype, seed=6))
     a = mhc.mhc_backward(d["x"], d["phi"], d["b"], d["alpha"], d["f_out"], d["grad_x_next"],
                          d["grad_h_in"])
     b = mhc.mhc_backward(d["x"], d["phi"], d["b"], d["alpha"], d["f_out"], d["grad_x_next"],
