@@ -159,7 +159,7 @@ def _sig(v):
     return 1.0 / (1.0 + math.exp(-v))
 
 
-@pytest.mark.parametrize("n", [1, 2, 4])
+@pytest.mark.parametrize("n", [1, 2, 4, 8, 16])
 def test_pre_zero_projection_gives_bias_gates(oracle_mod, n):
     T, C = 3, 8
     M = n * n + 2 * n
@@ -279,9 +279,9 @@ def _loss(oracle_mod, x, phi, b, alpha, f, G, g, iters, eps):
     return float(np.sum(G * xn) + np.sum(g * o["h_in"]))
 
 
-@pytest.mark.parametrize("n,iters", [(1, 20), (2, 0), (2, 1), (4, 3), (4, 20)])
+@pytest.mark.parametrize("n,iters", [(1, 20), (2, 0), (2, 1), (4, 3), (4, 20), (8, 2), (16, 2)])
 def test_backward_matches_finite_differences(oracle_mod, n, iters):
-    T, C = 2, 8
+    T, C = 2, (8 if n <= 4 else 2)
     M = n * n + 2 * n
     eps = 1e-6
     rng = _rng(80 + 7 * n + iters)
@@ -333,7 +333,7 @@ def test_backward_parameter_sums_are_token_additive(oracle_mod):
 
 
 # ------------------------------------- the backward in training order (split)
-@pytest.mark.parametrize("n", [1, 2, 4])
+@pytest.mark.parametrize("n", [1, 2, 4, 8, 16])
 def test_post_backward_finite_differences(oracle_mod, n):
     """The post half against central differences of L = sum G . post(x, f, H_post, H_res):
     grad_f_out = dL/df_out, red = (dL/dH_res row-major, dL/dH_post).  post is linear
@@ -366,7 +366,7 @@ def test_post_backward_finite_differences(oracle_mod, n):
     np.testing.assert_allclose(red[:, n * n:], fd(hp, "hp_"), rtol=0, atol=1e-8)
 
 
-@pytest.mark.parametrize("n", [1, 2, 4])
+@pytest.mark.parametrize("n", [1, 2, 4, 8, 16])
 def test_split_backward_equals_whole(oracle_mod, n):
     """post half -> pre half (with grad_h_in given) reproduces the one-call backward,
     whose every gradient is pinned by finite differences above."""
