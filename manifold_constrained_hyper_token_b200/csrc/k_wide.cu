@@ -18,7 +18,8 @@
 //   k_wide_post_bwd   the post half of the backward in training order:
 //                     grad_f_out and <G_i, x_j>, <G_i, f_out>
 //   k_wide_apply_x    grad_x = phi u + H_res^T G + H_pre g - kappa x and
-//                     grad_f_out, the phi u term a GEMM over the logits
+//                     grad_f_out for 32 tokens x 4 channels of all streams,
+//                     the phi u term a GEMM over the logits
 //   k_wide_apply_phi  grad_phi = sum_t x_t u_t^T, a GEMM over the tokens
 //   k_wide_bias       grad_b and grad_alpha from the mapping CTAs' partials
 //
@@ -443,7 +444,21 @@ __global__ void __launch_bounds__(widek::NT) k_wide_post_bwd(int64_t T, int64_t 
 // grad_x[t][k] (k = j*C + c) = sum_m phi[k][m] u[t][m] + H_pre[j] g[c]
 //                              + sum_i H_res[i][j] G[i][c] - kappa x[t][k]  (the k_bwd order)
 // grad_f_out[t][c] = sum_i H_post[i] G[i][c]   (when grad_f is not null)
-// A CTA owns 32 tokens x 64 k; the phi u term is a GEMM over the 288 logits.
+// A CTA owns 32 tokens x 4 channels of all 16 streams (64 k, kk = 4 j + cc), so
+// the G values, grad_h_in and the tokens' coefficients are staged once and
+// shared by the 16 output streams; the phi u term is a GEMM over the logits.
+namespace widek {
+constexpr int AX_CC = 4;                       // channels per apply CTA
+constexpr int AX_K = N * AX_CC;                // 64 k per CTA
+constexpr int AX_H = N * N + 2 * N + 1;        // per token: H_res, H_pre, H_post, kappa
+constexpr int AX_US = 32 * 32;                 // [m][token]
+constexpr int AX_PS = 32 * AX_K;               // [m][kk]
+constexpr int AX_HS = 32 * AX_H;               // [token][AX_H]
+constexpr int AX_GS = 32 * N * AX_CC;          // [token][i][cc]
+constexpr int AX_GG = 32 * AX_CC;              // [token][cc]
+constexpr int AX_SMEM_FLOATS = AX_US + AX_PS + AX_HS + AX_GS + AX_GG;
+}  // namespace widek
+
 template <typename TIO>
 __global__ void __launch_bounds__(widek::NT) k_wide_apply_x(
     int64_t T, int64_t C, const TIO* __restrict__ x, const float* __restrict__ phi,
@@ -451,12 +466,32 @@ __global__ void __launch_bounds__(widek::NT) k_wide_apply_x(
     TIO* __restrict__ grad_x, TIO* __restrict__ grad_f) {
   using namespace widek;
   using CF = Coef<N>;
-  __shared__ __align__(16) float Us[32 * 32];   // [m][token]
-  __shared__ __align__(16) float ps[32 * 64];   // [m][k]
+  extern __shared__ __align__(16) float sm[];
+  float* Us = sm;
+  float* ps = Us + AX_US;
+  float* hs = ps + AX_PS;
+  float* Gs = hs + AX_HS;
+  float* gs = Gs + AX_GS;
   const int tid = threadIdx.x, ty = tid >> 5, tx = tid & 31;
   const int64_t t0 = (int64_t)blockIdx.x * 32;
-  const int64_t k0 = (int64_t)blockIdx.y * 64;
+  const int64_t c0 = (int64_t)blockIdx.y * AX_CC;   // C is a multiple of 8: whole groups
   const int64_t K = (int64_t)N * C;
+  // this CTA's coefficients, G and grad_h_in
+  for (int e = tid; e < AX_HS; e += NT) {
+    const int tok = e / AX_H, q = e - tok * AX_H;
+    const int64_t t = t0 + tok;
+    hs[e] = t < T ? __ldg(coef + t * CF::SIZE + (q < AX_H - 1 ? q : CF::KAPPA)) : 0.0f;
+  }
+  for (int e = tid; e < AX_GS; e += NT) {
+    const int cc = e & (AX_CC - 1), i = (e >> 2) & (N - 1), tok = e >> 6;
+    const int64_t t = t0 + tok;
+    Gs[e] = t < T ? to_f32(G[(t * N + i) * C + c0 + cc]) : 0.0f;
+  }
+  if (tid < AX_GG) {
+    const int cc = tid & (AX_CC - 1), tok = tid >> 2;
+    const int64_t t = t0 + tok;
+    gs[tid] = t < T ? to_f32(g[t * C + c0 + cc]) : 0.0f;
+  }
   float acc[4][2];
 #pragma unroll
   for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = 0.0f;
@@ -470,15 +505,15 @@ __global__ void __launch_bounds__(widek::NT) k_wide_apply_x(
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int e = tid + NT * r, kk = e >> 5, mm = e & 31;
-      const int64_t k = k0 + kk;
-      ps[mm * 64 + kk] = k < K ? __ldg(phi + k * M + m0 + mm) : 0.0f;
+      const int64_t k = (int64_t)(kk >> 2) * C + c0 + (kk & 3);
+      ps[mm * AX_K + kk] = __ldg(phi + k * M + m0 + mm);
     }
     __syncthreads();
 #pragma unroll 8
     for (int mm = 0; mm < 32; ++mm) {
       const float4 a = *reinterpret_cast<const float4*>(Us + mm * 32 + 4 * ty);
       const float av[4] = {a.x, a.y, a.z, a.w};
-      const float b0 = ps[mm * 64 + tx], b1 = ps[mm * 64 + tx + 32];
+      const float b0 = ps[mm * AX_K + tx], b1 = ps[mm * AX_K + tx + 32];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         acc[i][0] = fmaf(b0, av[i], acc[i][0]);
@@ -489,29 +524,28 @@ __global__ void __launch_bounds__(widek::NT) k_wide_apply_x(
   }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int64_t t = t0 + 4 * ty + i;
+    const int tok = 4 * ty + i;
+    const int64_t t = t0 + tok;
+    if (t >= T) continue;
+    const float* h = hs + tok * AX_H;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int64_t k = k0 + tx + 32 * h;
-      if (t >= T || k >= K) continue;
-      const int j = (int)(k / C);
-      const int64_t c = k - (int64_t)j * C;
-      const float* co = coef + t * CF::SIZE;
-      float a = fmaf(__ldg(co + CF::PRE + j), to_f32(g[t * C + c]), acc[i][h]);
-      float b = 0.0f;
-#pragma unroll 4
-      for (int i2 = 0; i2 < N; ++i2) {
-        const float Gv = to_f32(G[(t * N + i2) * C + c]);
-        a = fmaf(__ldg(co + CF::RES + i2 * N + j), Gv, a);
-        b = fmaf(__ldg(co + CF::POST + i2), Gv, b);
-      }
-      const float gx = fmaf(-__ldg(co + CF::KAPPA), to_f32(x[t * K + k]), a);
-      if constexpr (sizeof(TIO) == 2) {
-        grad_x[t * K + k] = __float2bfloat16_rn(gx);
-        if (j == 0 && grad_f != nullptr) grad_f[t * C + c] = __float2bfloat16_rn(b);
-      } else {
-        grad_x[t * K + k] = gx;
-        if (j == 0 && grad_f != nullptr) grad_f[t * C + c] = b;
+    for (int hh = 0; hh < 2; ++hh) {
+      const int kk = tx + 32 * hh, j = kk >> 2, cc = kk & 3;
+      const int64_t c = c0 + cc;
+      const float* Gt = Gs + tok * N * AX_CC + cc;
+      float a = fmaf(h[CF::PRE + j], gs[tok * AX_CC + cc], acc[i][hh]);
+#pragma unroll
+      for (int i2 = 0; i2 < N; ++i2) a = fmaf(h[CF::RES + i2 * N + j], Gt[i2 * AX_CC], a);
+      const int64_t k = (int64_t)j * C + c;
+      const float gx = fmaf(-h[AX_H - 1], to_f32(x[t * K + k]), a);
+      if constexpr (sizeof(TIO) == 2) grad_x[t * K + k] = __float2bfloat16_rn(gx);
+      else grad_x[t * K + k] = gx;
+      if (j == 0 && grad_f != nullptr) {
+        float b = 0.0f;
+#pragma unroll
+        for (int i2 = 0; i2 < N; ++i2) b = fmaf(h[CF::POST + i2], Gt[i2 * AX_CC], b);
+        if constexpr (sizeof(TIO) == 2) grad_f[t * C + c] = __float2bfloat16_rn(b);
+        else grad_f[t * C + c] = b;
       }
     }
   }
@@ -693,10 +727,14 @@ static cudaError_t launch_wide_apply(int64_t T, int64_t C, const void* x, const 
                                      float* gphi, float* gb, float* ga, int ag, cudaStream_t s) {
   using namespace widek;
   const int64_t K = (int64_t)N * C;
-  const dim3 gridx((unsigned)((T + 31) / 32), (unsigned)((K + 63) / 64));
-  k_wide_apply_x<TIO><<<gridx, NT, 0, s>>>(T, C, (const TIO*)x, phi, (const TIO*)G, (const TIO*)g,
-                                           coef, (TIO*)gx, (TIO*)gf);
-  cudaError_t e = cudaGetLastError();
+  const size_t smx = (size_t)AX_SMEM_FLOATS * 4;
+  cudaError_t e = cudaFuncSetAttribute(k_wide_apply_x<TIO>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smx);
+  if (e != cudaSuccess) return e;
+  const dim3 gridx((unsigned)((T + 31) / 32), (unsigned)(C / AX_CC));
+  k_wide_apply_x<TIO><<<gridx, NT, smx, s>>>(T, C, (const TIO*)x, phi, (const TIO*)G,
+                                             (const TIO*)g, coef, (TIO*)gx, (TIO*)gf);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const dim3 gridp((unsigned)((K + 31) / 32), (unsigned)((M + 95) / 96));
   k_wide_apply_phi<TIO><<<gridp, NT, 0, s>>>(T, C, (const TIO*)x, coef, gphi);
