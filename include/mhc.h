@@ -94,7 +94,7 @@ typedef enum mhc_dtype {
 
 /* Problem description shared by mhc_pre / mhc_post / mhc_backward. */
 typedef struct mhc_params {
-  int32_t n;      /* streams; this build supports n in {1, 2, 4, 8, 16}; bf16
+  int32_t n;      /* streams; the library supports n in {1, 2, 4, 8, 16}; bf16
                      with n = 4 runs the tensor-core kernels, n = 16 its own
                      CUDA-core kernels (288 logits per token), the rest the
                      CUDA-core kernels; mhc_backward_noalloc takes n <= 8    */
