@@ -37,6 +37,7 @@ constexpr int TB = 32;             // tokens per mapping CTA
 constexpr int NT = 256;
 constexpr int KC = 32;             // projection: k rows per chunk
 constexpr int CPT = M / 32;        // logit columns (or dot products) per thread: 9
+static_assert(KC * M % NT == 0, "phi chunk split over the threads");
 constexpr int CQ = 8;              // reductions: channels per chunk
 constexpr int CQP = CQ + 1;        // padded stride of a (token, stream) row
 // shared memory of k_wide_map, in floats
@@ -77,16 +78,26 @@ __device__ __forceinline__ void wide_dots(int64_t T, int64_t C, int64_t t0, cons
 #pragma unroll
     for (int q = 0; q < CPT; ++q) dacc[i][q] = 0.0f;
   for (int64_t c0 = 0; c0 < C; c0 += CQ) {
-    // (token, stream, channel) elements: TB * N * CQ = 4096, 16 per thread
-#pragma unroll 4
-    for (int r = 0; r < TB * N * CQ / NT; ++r) {
+    // (token, stream, channel) elements: TB * N * CQ = 4096, 16 per thread; all
+    // loads are issued before the first store, so their latencies overlap
+    constexpr int RX = TB * N * CQ / NT;
+    float xl[RX], Gl[RX];
+#pragma unroll
+    for (int r = 0; r < RX; ++r) {
       const int e = tid + NT * r;
       const int cc = e & (CQ - 1), j = (e >> 3) & (N - 1), tok = e >> 7;
       const int64_t t = t0 + tok, c = c0 + cc;
       const bool ok = t < T && c < C;
       const int64_t gi = (t * N + j) * C + c;
-      xq[(tok * N + j) * CQP + cc] = ok ? to_f32(x[gi]) : 0.0f;
-      if constexpr (USE_G) Gq[(tok * N + j) * CQP + cc] = ok ? to_f32(G[gi]) : 0.0f;
+      xl[r] = ok ? to_f32(x[gi]) : 0.0f;
+      if constexpr (USE_G) Gl[r] = ok ? to_f32(G[gi]) : 0.0f;
+    }
+#pragma unroll
+    for (int r = 0; r < RX; ++r) {
+      const int e = tid + NT * r;
+      const int cc = e & (CQ - 1), j = (e >> 3) & (N - 1), tok = e >> 7;
+      xq[(tok * N + j) * CQP + cc] = xl[r];
+      if constexpr (USE_G) Gq[(tok * N + j) * CQP + cc] = Gl[r];
     }
     {
       // (token, channel) elements: TB * CQ = 256, one per thread
@@ -253,18 +264,25 @@ __global__ void __launch_bounds__(widek::NT) k_wide_map(
       for (int q = 0; q < CPT; ++q) acc[i][q] = 0.0f;
     }
     for (int64_t k0 = 0; k0 < K; k0 += KC) {
+      // all loads are issued before the first store, so their latencies overlap
+      // (K is a multiple of 128: every phi chunk is whole)
+      constexpr int RP = KC * M / NT;  // 36
+      float xv[TB * KC / NT], pv[RP];
 #pragma unroll
       for (int r = 0; r < TB * KC / NT; ++r) {
-        const int tok = ty + 8 * r;
-        const int64_t t = t0 + tok, k = k0 + tx;
-        const float v = (t < T && k < K) ? to_f32(x[t * K + k]) : 0.0f;
-        xs[tx * TB + tok] = v;
-        ssp[r] = fmaf(v, v, ssp[r]);
+        const int64_t t = t0 + ty + 8 * r, k = k0 + tx;
+        xv[r] = (t < T && k < K) ? to_f32(x[t * K + k]) : 0.0f;
       }
-      for (int e = tid; e < KC * M; e += NT) {
-        const int kk = e / M;
-        ps[e] = (k0 + kk < K) ? __ldg(phi + (k0 + kk) * M + (e - kk * M)) : 0.0f;
+      const float* pc = phi + k0 * M;
+#pragma unroll
+      for (int r = 0; r < RP; ++r) pv[r] = __ldg(pc + tid + NT * r);
+#pragma unroll
+      for (int r = 0; r < TB * KC / NT; ++r) {
+        xs[tx * TB + ty + 8 * r] = xv[r];
+        ssp[r] = fmaf(xv[r], xv[r], ssp[r]);
       }
+#pragma unroll
+      for (int r = 0; r < RP; ++r) ps[tid + NT * r] = pv[r];
       __syncthreads();
 #pragma unroll 4
       for (int kk = 0; kk < KC; ++kk) {
@@ -457,6 +475,7 @@ constexpr int AX_HS = 32 * AX_H;               // [token][AX_H]
 constexpr int AX_GS = 32 * N * AX_CC;          // [token][i][cc]
 constexpr int AX_GG = 32 * AX_CC;              // [token][cc]
 constexpr int AX_SMEM_FLOATS = AX_US + AX_PS + AX_HS + AX_GS + AX_GG;
+static_assert(AX_GS % NT == 0, "G tile split over the threads");
 }  // namespace widek
 
 template <typename TIO>
@@ -476,16 +495,30 @@ __global__ void __launch_bounds__(widek::NT) k_wide_apply_x(
   const int64_t t0 = (int64_t)blockIdx.x * 32;
   const int64_t c0 = (int64_t)blockIdx.y * AX_CC;   // C is a multiple of 8: whole groups
   const int64_t K = (int64_t)N * C;
-  // this CTA's coefficients, G and grad_h_in
-  for (int e = tid; e < AX_HS; e += NT) {
-    const int tok = e / AX_H, q = e - tok * AX_H;
-    const int64_t t = t0 + tok;
-    hs[e] = t < T ? __ldg(coef + t * CF::SIZE + (q < AX_H - 1 ? q : CF::KAPPA)) : 0.0f;
-  }
-  for (int e = tid; e < AX_GS; e += NT) {
-    const int cc = e & (AX_CC - 1), i = (e >> 2) & (N - 1), tok = e >> 6;
-    const int64_t t = t0 + tok;
-    Gs[e] = t < T ? to_f32(G[(t * N + i) * C + c0 + cc]) : 0.0f;
+  // this CTA's coefficients, G and grad_h_in; loads are issued before stores
+  {
+    constexpr int RH = (AX_HS + NT - 1) / NT, RG = AX_GS / NT;
+    float hl[RH], gl[RG];
+#pragma unroll
+    for (int r = 0; r < RH; ++r) {
+      const int e = tid + NT * r;
+      const int tok = e / AX_H, q = e - tok * AX_H;
+      const int64_t t = t0 + tok;
+      hl[r] = (e < AX_HS && t < T) ? __ldg(coef + t * CF::SIZE + (q < AX_H - 1 ? q : CF::KAPPA))
+                                   : 0.0f;
+    }
+#pragma unroll
+    for (int r = 0; r < RG; ++r) {
+      const int e = tid + NT * r;
+      const int cc = e & (AX_CC - 1), i = (e >> 2) & (N - 1), tok = e >> 6;
+      const int64_t t = t0 + tok;
+      gl[r] = t < T ? to_f32(G[(t * N + i) * C + c0 + cc]) : 0.0f;
+    }
+#pragma unroll
+    for (int r = 0; r < RH; ++r)
+      if (tid + NT * r < AX_HS) hs[tid + NT * r] = hl[r];
+#pragma unroll
+    for (int r = 0; r < RG; ++r) Gs[tid + NT * r] = gl[r];
   }
   if (tid < AX_GG) {
     const int cc = tid & (AX_CC - 1), tok = tid >> 2;
@@ -496,17 +529,28 @@ __global__ void __launch_bounds__(widek::NT) k_wide_apply_x(
 #pragma unroll
   for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = 0.0f;
   for (int m0 = 0; m0 < M; m0 += 32) {
+    float ul[4], pl[8];
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const int e = tid + NT * r, tok = e >> 5, mm = e & 31;
       const int64_t t = t0 + tok;
-      Us[mm * 32 + tok] = t < T ? __ldg(coef + t * CF::SIZE + CF::U + m0 + mm) : 0.0f;
+      ul[r] = t < T ? __ldg(coef + t * CF::SIZE + CF::U + m0 + mm) : 0.0f;
     }
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int e = tid + NT * r, kk = e >> 5, mm = e & 31;
       const int64_t k = (int64_t)(kk >> 2) * C + c0 + (kk & 3);
-      ps[mm * AX_K + kk] = __ldg(phi + k * M + m0 + mm);
+      pl[r] = __ldg(phi + k * M + m0 + mm);
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int e = tid + NT * r;
+      Us[(e & 31) * 32 + (e >> 5)] = ul[r];
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int e = tid + NT * r;
+      ps[(e & 31) * AX_K + (e >> 5)] = pl[r];
     }
     __syncthreads();
 #pragma unroll 8
@@ -570,18 +614,23 @@ __global__ void __launch_bounds__(widek::NT) k_wide_apply_phi(int64_t T, int64_t
 #pragma unroll
   for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = 0.0f;
   for (int64_t t0 = 0; t0 < T; t0 += 32) {
+    float xl[4], ul[12];
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const int e = tid + NT * r, tok = e >> 5, kk = e & 31;
       const int64_t t = t0 + tok, k = k0 + kk;
-      xs[tok * 32 + kk] = (t < T && k < K) ? to_f32(x[t * K + k]) : 0.0f;
+      xl[r] = (t < T && k < K) ? to_f32(x[t * K + k]) : 0.0f;
     }
 #pragma unroll
     for (int r = 0; r < 12; ++r) {
       const int e = tid + NT * r, tok = e / 96, mm = e - tok * 96;
       const int64_t t = t0 + tok;
-      us[e] = (t < T && m0 + mm < M) ? __ldg(coef + t * CF::SIZE + CF::U + m0 + mm) : 0.0f;
+      ul[r] = (t < T && m0 + mm < M) ? __ldg(coef + t * CF::SIZE + CF::U + m0 + mm) : 0.0f;
     }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) xs[tid + NT * r] = xl[r];
+#pragma unroll
+    for (int r = 0; r < 12; ++r) us[tid + NT * r] = ul[r];
     __syncthreads();
 #pragma unroll 8
     for (int tok = 0; tok < 32; ++tok) {
