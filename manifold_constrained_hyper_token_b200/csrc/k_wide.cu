@@ -10,9 +10,15 @@
 //
 //   k_wide_map        32 tokens per CTA: the projection y = x . phi as a
 //                     CUDA-core GEMM over the flattened k = i*C + c (with the
-//                     sum of squares), for the backward the 288 C-reductions
-//                     per token, then one thread per token for the gates,
-//                     Sinkhorn and (backward) its adjoint
+//                     sum of squares); the forward then runs the gates and
+//                     Sinkhorn one thread per token; the backward adds the
+//                     288 C-reductions per token and stages y, the dot
+//                     products and the sum of squares in each token's
+//                     coefficient row
+//   k_wide_bwd_epi    the backward's per-token epilogue, one warp per 32
+//                     tokens: gates, Sinkhorn and its adjoint, the
+//                     coefficient record written over the staged row, and
+//                     the tile's grad_b / grad_alpha partial sums
 //   k_wide_post       x_next = H_res x + H_post^T f_out, coefficients in
 //                     shared memory
 //   k_wide_post_bwd   the post half of the backward in training order:
