@@ -34,6 +34,20 @@ constexpr int TMP = TM + 4;  // padded token stride of the staged x tile
 constexpr int NT = 256;      // threads
 }  // namespace mapk
 
+// Four consecutive activations widened to fp32 (8-byte bf16 or 16-byte fp32
+// load; the address is a multiple of 4 elements).
+__device__ __forceinline__ void ld4(const float* p, float (&v)[4]) {
+  const float4 q = *reinterpret_cast<const float4*>(p);
+  v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+}
+__device__ __forceinline__ void ld4(const __nv_bfloat16* p, float (&v)[4]) {
+  const uint2 q = *reinterpret_cast<const uint2*>(p);
+  v[0] = __uint_as_float(q.x << 16);
+  v[1] = __uint_as_float(q.x & 0xffff0000u);
+  v[2] = __uint_as_float(q.y << 16);
+  v[3] = __uint_as_float(q.y & 0xffff0000u);
+}
+
 template <int N> struct MapShape {
   static constexpr int M = N * N + 2 * N;
   static constexpr int MP = (M + 3) / 4 * 4;   // padded logit count
@@ -188,19 +202,38 @@ __global__ void __launch_bounds__(mapk::NT) k_map(
     if constexpr (BWD) {
       const int64_t t = t0 + dtok;
       const int64_t cb = ch * CC + dsub * DCH;
-      if (t < T) {
+      // C is a multiple of 8 and cb of 4: the DCH = 4 channels are all in range
+      // or all out, and each row's 4 values are one aligned vector load
+      static_assert(DCH == 4, "four channels per reduction thread");
+      if (t < T && cb < C) {
+        float Gq[N][DCH], gq[DCH], fq[DCH];
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+          if constexpr (SPLIT) {
+#pragma unroll
+            for (int e = 0; e < DCH; ++e) Gq[i][e] = 0.0f;
+          } else {
+            ld4(G + (t * N + i) * C + cb, Gq[i]);
+          }
+        }
+        ld4(g + t * C + cb, gq);
+        if constexpr (SPLIT) {
+#pragma unroll
+          for (int e = 0; e < DCH; ++e) fq[e] = 0.0f;
+        } else {
+          ld4(f + t * C + cb, fq);
+        }
 #pragma unroll
         for (int e = 0; e < DCH; ++e) {
-          const int64_t c = cb + e;
-          if (c < C) {
+          {
             float xv[N], Gv[N];
 #pragma unroll
             for (int i = 0; i < N; ++i) {
               xv[i] = xs[(i * CC + dsub * DCH + e) * TMP + dtok];
-              Gv[i] = SPLIT ? 0.0f : to_f32(G[(t * N + i) * C + c]);
+              Gv[i] = Gq[i][e];
             }
-            const float gv = to_f32(g[t * C + c]);
-            const float fv = SPLIT ? 0.0f : to_f32(f[t * C + c]);
+            const float gv = gq[e];
+            const float fv = fq[e];
             if constexpr (SPLIT) {
 #pragma unroll
               for (int i = 0; i < N; ++i) dots[N * N + i] = fmaf(gv, xv[i], dots[N * N + i]);
