@@ -23,6 +23,13 @@ for the longest single-kernel call.
 
 ``--impl reference`` times the fp64 CPU oracle (the reference arm of this
 library) on a bounded sample of the same workload instead.
+
+Two more workloads print their own line (the default line is the layer's):
+``--workload sinkhorn``: the standalone batched Sinkhorn-Knopp on 2^22
+matrices for n = 4, 8, 16 (20 iterations) and the depth-product Amax gain
+over L = 64 layers of 2^16 tokens; ``--workload depth``: a 24-layer stack
+(T = 65536 tokens per GPU, n = 4, C = 7168, F_l(h) = s_l h) forward and
+backward through ``DepthStack`` with block recompute.
 """
 from __future__ import annotations
 
@@ -42,6 +49,7 @@ sys.path.insert(0, ROOT)
 METRIC = "mHC layer tokens/s (fwd+bwd, n=4, C=7168) and achieved HBM GB/s vs B200 peak"
 T_TOK, N_STR, C_CH, T_MAX = 16384, 4, 7168, 20
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e, the spec figure
 
 
 def per_token_bytes(n=N_STR, C=C_CH, act=2):
@@ -182,9 +190,19 @@ def cpu_reference(seconds: float, seed: int = 0):
     while dt < seconds / 4 and S < 8192:
         S = min(8192, int(S * max(2.0, min(8.0, seconds / max(dt, 1e-3) / 2))))
         dt = run(S)
-    return {"value": S / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+    cores = oracle.num_threads()
+    # the plain cost: one host thread on a smaller sample of the same tokens
+    oracle.set_num_threads(1)
+    try:
+        S1 = 64
+        dt1 = run(S1)
+    finally:
+        oracle.set_num_threads(cores)
+    return {"value": S / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": f"first {S} tokens of the T={T_TOK}, n={N_STR}, C={C_CH} bf16 workload, "
-                      f"pre+post+backward in fp64, {dt:.2f} s"}
+                      f"pre+post+backward in fp64, {dt:.2f} s",
+            "single_thread": {"value": S1 / dt1, "unit": "tokens/s", "cores": 1,
+                              "sample": f"first {S1} tokens, {dt1:.2f} s"}}
 
 
 def run_reference(args, rank, world):
@@ -221,14 +239,17 @@ def run_reference(args, rank, world):
     cb = {"value": val, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
           "sample": f"{S} tokens per step of the T={T_TOK}, n={N_STR}, C={C_CH} bf16 workload, "
                     f"pre+post+backward in fp64"}
+    # a step here is the S-token sample the oracle ran, and ms_per_step its measured time
     line = {"metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": 1000.0 * T_TOK / val, "higher_is_better": True,
+            "warmup": args.warmup, "ms_per_step": 1000.0 * total / args.steps,
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": f"mHC layer fwd+bwd per GPU: T={T_TOK} tokens, n={N_STR}, "
-                                   f"C={C_CH}, t_max={T_MAX}, bf16 activations, fp32 maps",
-                       "T_per_gpu": T_TOK, "n": N_STR, "C": C_CH, "t_max": T_MAX,
-                       "parallelism": "host cores (oracle)"},
+            "config": {"workload": f"mHC layer fwd+bwd, oracle on a sample of S={S} tokens per "
+                                   f"step drawn from the T={T_TOK}, n={N_STR}, C={C_CH}, "
+                                   f"t_max={T_MAX} bf16 workload",
+                       "tokens_per_step": S, "T_sampled_from": T_TOK, "n": N_STR, "C": C_CH,
+                       "t_max": T_MAX, "parallelism": "host cores (oracle)"},
             "cpu_baseline": cb,
             "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -246,6 +267,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--tokens", type=int, default=T_TOK,
                     help="tokens per GPU (default 16384; smaller values for profiler captures)")
+    ap.add_argument("--workload", default="layer", choices=["layer", "sinkhorn", "depth"],
+                    help="layer: the fwd+bwd layer step (the default line); sinkhorn: batched "
+                         "Sinkhorn-Knopp and depth gain; depth: the 24-layer stack")
     ap.add_argument("--forward", default="unfused", choices=["fused", "unfused"],
                     help="fused: layer input + post merge fused with the next layer's mapping; "
                          "unfused: mhc_pre + mhc_post")
@@ -264,15 +288,39 @@ def main():
     import torch
     import torch.distributed as dist
 
-    import manifold_constrained_hyper_token_b200 as mhc
-    from manifold_constrained_hyper_token_b200 import parallel, synth
-
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
+    if args.workload == "sinkhorn":
+        run_sinkhorn(args, dev, rank, world, local_rank)
+    elif args.workload == "depth":
+        run_depth(args, dev, rank, world, local_rank)
+    else:
+        run_layer(args, dev, rank, world, local_rank)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def step_stats(ms):
+    """Median and spread of per-step device times (ms)."""
+    v = sorted(ms)
+    if not v:
+        return None
+    q = lambda f: v[min(len(v) - 1, int(round(f * (len(v) - 1))))]
+    return {"median": q(0.5), "p10": q(0.1), "p90": q(0.9), "min": v[0], "max": v[-1],
+            "n": len(v)}
+
+
+def run_layer(args, dev, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import manifold_constrained_hyper_token_b200 as mhc
+    from manifold_constrained_hyper_token_b200 import parallel, synth
 
     T, n, C = args.tokens, N_STR, C_CH
     K, M = n * C, n * n + 2 * n
@@ -294,7 +342,9 @@ def main():
     stream = torch.cuda.current_stream()
     fused = args.forward == "fused"
     calls = (["layer_input", "post_fused"] if fused else ["pre", "post"]) + ["bwd_map", "bwd_apply"]
-    launches_per_call = {"pre": 2, "post": 1, "layer_input": 1, "post_fused": 2, "bwd_map": 1,
+    # this library's kernels per call: pre = phi split + mapping + layer input;
+    # bwd_map = phi split + mapping; post_fused = phi split + fused kernel
+    launches_per_call = {"pre": 3, "post": 1, "layer_input": 1, "post_fused": 2, "bwd_map": 2,
                          "bwd_apply": 1}
     # the layer's maps; in a stack the previous layer's post_fused computes them
     mhc.mhc_pre(x, phi, b, alpha, t_max=T_MAX, out=(h_in, Hpre, Hpost, Hres), stream=stream)
@@ -355,6 +405,7 @@ def main():
         for i, c in enumerate(calls):
             per_call[c] += evs[s][i].elapsed_time(evs[s][i + 1])
     per_call = {c: v / args.steps for c, v in per_call.items()}
+    per_step = [evs[s][0].elapsed_time(evs[s][len(calls)]) for s in range(args.steps)]
     elapsed_ms = parallel.max_over_ranks(elapsed_ms, dev)
     ms_per_step = elapsed_ms / args.steps
     tokens_per_s = T * world / (ms_per_step / 1000.0)
@@ -364,7 +415,9 @@ def main():
     tb = per_token_bytes(n, C)
     pb = per_call_param_bytes(n, C)
     call_bytes = {c: T * tb[c] + pb[c] for c in calls}
-    single = [c for c in calls if launches_per_call[c] == 1]
+    # the roofline is read for a call whose time is one kernel's (the phi split
+    # ahead of the backward mapping is 5 us of its 0.5 ms and is counted in)
+    single = [c for c in calls if c in ("post", "bwd_map", "bwd_apply", "layer_input")]
     dom = max(single, key=lambda c: per_call[c])
     achieved = call_bytes[dom] / (per_call[dom] / 1000.0) / 1e9
     traffic = ncu_traffic(dom)
@@ -426,22 +479,177 @@ def main():
                        "parallelism": f"dp{world} over tokens",
                        "l2": "inputs larger than L2 (x and grad_x_next are 940 MB each); no flush"},
             "hbm": {"achieved_gbs": step_gbs, "peak_gbs": peak, "frac": step_gbs / peak,
-                    "peak_kind": peak_kind,
+                    "peak_kind": peak_kind, "frac_vs_nominal": step_gbs / NOMINAL_HBM_GBS,
                     "alg_bytes_per_step": step_alg_bytes},
             "per_call_ms": per_call,
+            "step_ms": step_stats(per_step),
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
                          "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                         "frac_vs_nominal": achieved / NOMINAL_HBM_GBS,
                          "alg_bytes_per_launch": call_bytes[dom], "peak_kind": peak_kind},
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": args.steps * sum(launches_per_call.values()),
+            "gpu_launches": args.steps * sum(launches_per_call[c] for c in calls),
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
 
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+
+def _timed(fn, steps, warmup, stream):
+    """Device times (ms) of `steps` calls of fn after `warmup` untimed ones."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for e0, e1 in evs:
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return [e0.elapsed_time(e1) for e0, e1 in evs]
+
+
+def sinkhorn_ops(n, iters):
+    """fp32 operations of one n x n Sinkhorn-Knopp estimate as the kernel runs it: the
+    row maxima, shift and exp (3 n^2), then per normalisation n^2 adds, n reciprocals
+    and n^2 multiplies."""
+    return 3 * n * n + 2 * iters * (2 * n * n + n)
+
+
+def run_sinkhorn(args, dev, rank, world, local_rank):
+    """Batched Sinkhorn-Knopp on 2^22 matrices (n = 4, 8, 16; logits N(0, 2); 20
+    iterations) and the depth-product Amax gain over L = 64 layers of 2^16 tokens.
+    Each rank runs its own batch (weak scaling)."""
+    import torch
+
+    import manifold_constrained_hyper_token_b200 as mhc
+    from manifold_constrained_hyper_token_b200 import parallel, synth
+
+    B, iters, Tdep, Ldep = 1 << 22, T_MAX, 1 << 16, 64
+    stream = torch.cuda.current_stream()
+    peak, peak_kind = load_peaks()
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    per_n = {}
+    total_ms, total_mat = 0.0, 0
+    for n in (4, 8, 16):
+        lg = synth.sinkhorn_logits(B, n, seed=100 + n + rank).to(dev)
+        out = torch.empty_like(lg)
+        ms = _timed(lambda: mhc.mhc_sinkhorn_knopp(lg, iters, out=out, stream=stream),
+                    args.steps, args.warmup, stream)
+        t = parallel.max_over_ranks(sum(ms) / len(ms), dev)
+        byts = B * 8 * n * n
+        ops = B * sinkhorn_ops(n, iters)
+        per_n[str(n)] = {"ms": t, "matrices_per_s": B * world / (t / 1e3),
+                         "hbm_gbs": byts / (t / 1e3) / 1e9, "hbm_frac": byts / (t / 1e3) / 1e9 / peak,
+                         "gops": ops / (t / 1e3) / 1e9, "step_ms": step_stats(ms)}
+        total_ms += t
+        total_mat += B
+        del lg, out
+    # depth product over 64 layers of 20-iteration Sinkhorn outputs (n = 4)
+    H = mhc.mhc_sinkhorn_knopp(synth.sinkhorn_logits(Tdep * Ldep, 4, seed=300 + rank).to(dev),
+                               iters).view(Tdep, Ldep, 4, 4)
+    gf = torch.empty(Tdep, device=dev)
+    gb = torch.empty(Tdep, device=dev)
+    ms = _timed(lambda: mhc.mhc_depth_amax(H, out=(gf, gb), stream=stream), args.steps,
+                args.warmup, stream)
+    td = parallel.max_over_ranks(sum(ms) / len(ms), dev)
+    dbytes = Tdep * Ldep * 16 * 4 + 2 * Tdep * 4
+    clocks = sampler.stop()
+    sm_mhz = clocks.get("sm_mhz") or 1965.0
+    # fp32 add / multiply issue rate: 128 lanes per SM per clock
+    alu_peak_gops = props.multi_processor_count * 128 * sm_mhz * 1e6 / 1e9
+    for v in per_n.values():
+        v["alu_frac"] = v["gops"] / alu_peak_gops
+    dom = max(per_n, key=lambda k: per_n[k]["ms"])
+    if rank == 0:
+        d = per_n[dom]
+        bound = "hbm" if d["hbm_frac"] >= d["alu_frac"] else "alu"
+        line = {
+            "metric": "batched Sinkhorn-Knopp matrices/s (2^22 matrices each for n=4,8,16, "
+                      "20 iterations)",
+            "value": total_mat * world / (total_ms / 1e3), "unit": "matrices/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "standalone Sinkhorn-Knopp: 2^22 matrices per n in {4, 8, 16}, "
+                                   "logits N(0, 2), 20 iterations; depth gain over L=64 layers "
+                                   "x 2^16 tokens (n=4)",
+                       "l2": "inputs larger than L2 (n=4: 268 MB of logits); no flush"},
+            "per_n": per_n,
+            "depth_amax": {"ms": td, "tokens_per_s": Tdep * world / (td / 1e3),
+                           "hbm_gbs": dbytes / (td / 1e3) / 1e9,
+                           "hbm_frac": dbytes / (td / 1e3) / 1e9 / peak},
+            "roofline": {"bound": bound, "kernel": f"k_sinkhorn n={dom}",
+                         "achieved": d["hbm_gbs"] if bound == "hbm" else d["gops"],
+                         "peak": peak if bound == "hbm" else alu_peak_gops,
+                         "unit": "GB/s" if bound == "hbm" else "Gop/s",
+                         "frac": d["hbm_frac"] if bound == "hbm" else d["alu_frac"],
+                         "traffic": None, "peak_kind": peak_kind if bound == "hbm" else
+                         "148 SMs x 128 fp32 lanes x median SM clock"},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def run_depth(args, dev, rank, world, local_rank):
+    """24 mHC layers, T tokens per GPU (default 65536), n = 4, C = 7168, bf16,
+    F_l(h) = s_l h, forward and backward through DepthStack (block recompute,
+    backward in training order)."""
+    import torch
+
+    from manifold_constrained_hyper_token_b200 import parallel, synth
+    from manifold_constrained_hyper_token_b200.depth import DepthStack
+
+    L, n, C = 24, N_STR, C_CH
+    T = args.tokens if args.tokens != T_TOK else 65536
+    layers = [{k: v.to(dev) for k, v in synth.layer_params(n, C, seed=l).items()}
+              for l in range(L)]
+    gains = [synth.depth_gain(l) for l in range(L)]
+    F = lambda l, h: h * gains[l]
+    Fb = lambda l, h, f, gfo: gfo * gains[l]
+    stack = DepthStack(layers, F, Fb, n)
+    d = synth.depth_stack_chunk(T, n, C, chunk=rank)
+    x0, GL = d["x0"].to(dev), d["G_last"].to(dev)
+    del d
+    stream = torch.cuda.current_stream()
+
+    def step():
+        stack.forward(x0)
+        stack.backward(GL)
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    ms = _timed(step, args.steps, args.warmup, stream)
+    clocks = sampler.stop()
+    t = parallel.max_over_ranks(sum(ms) / len(ms), dev)
+    peak, peak_kind = load_peaks()
+    tb = per_token_bytes(n, C)
+    alg = L * T * (tb["pre"] + tb["post"] + tb["bwd_min"])
+    if rank == 0:
+        line = {
+            "metric": "mHC depth-stack tokens/s (24 layers fwd+bwd with recompute, n=4, C=7168)",
+            "value": T * world / (t / 1e3), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": f"depth stack: L={L} layers, T={T} tokens per GPU, n={n}, "
+                                   f"C={C}, bf16, F_l(h)=s_l h, recompute block "
+                                   f"{stack.block}, backward in training order",
+                       "l2": "inputs larger than L2; no flush"},
+            "step_ms": step_stats(ms),
+            "hbm": {"alg_bytes_per_step": alg, "achieved_gbs": alg / (t / 1e3) / 1e9,
+                    "peak_gbs": peak, "frac": alg / (t / 1e3) / 1e9 / peak,
+                    "peak_kind": peak_kind,
+                    "note": "24 x 415,920 B/token (one forward and a one-pass backward per "
+                            "layer); the recompute forward and F are extra"},
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
 
 
 if __name__ == "__main__":

@@ -53,9 +53,10 @@
  *     (MHC_ERR_INVALID_ARG otherwise).
  *   - dev_status (optional, may be NULL): a device int the kernels set to a
  *     non-zero mhc_status when they detect a condition at run time
- *     (MHC_ERR_NONFINITE when an RMS value or a logit is not finite).  The
- *     library only ever writes error codes into it, never clears it; the
- *     caller zeroes it and reads it after synchronising.
+ *     (MHC_ERR_NONFINITE when an RMS value or a logit is not finite;
+ *     MHC_ERR_TIMEOUT when a bounded device-side wait ran out, see
+ *     mhc_params.wait_ns).  The library only ever writes error codes into it,
+ *     never clears it; the caller zeroes it and reads it after synchronising.
  */
 #ifndef MHC_H_
 #define MHC_H_
@@ -107,6 +108,16 @@ typedef struct mhc_params {
   int32_t alpha_groups; /* 0 or 1: one alpha scales all n^2+2n logits;
                            3: alpha = (alpha_pre, alpha_post, alpha_res), one
                            scale per logit group, and grad_alpha has 3 entries */
+  int64_t wait_ns;  /* limit, in ns, of every device-side wait of the
+                       tensor-core kernels on another warp's or the copy
+                       engine's progress; 0 = the default of 2 s.  When a wait
+                       runs out the kernel writes MHC_ERR_TIMEOUT to dev_status,
+                       finishes the copies and MMAs it already issued, frees
+                       its tensor memory and returns; the outputs of that call
+                       are undefined, and later calls are unaffected.  A small
+                       positive value makes the waits give up on purpose (how
+                       the timeout path is tested).  Kernels without such waits
+                       ignore it.  Must be >= 0.                               */
 } mhc_params;
 
 /* Library version, (major << 16) | minor. */
@@ -297,7 +308,10 @@ MHC_API mhc_status mhc_pre_backward(const mhc_params *p, const void *x, const fl
  * call).  The first call on a
  * device looks up the array's device address (cudaGetSymbolAddress) with
  * that device current and caches it; make that first call before any stream
- * capture.  All calls share the one array and it keeps the last call's
+ * capture.  The cached address belongs to the device's primary context: a
+ * process that destroys that context (cudaDeviceReset) must not call this
+ * entry point on that device afterwards, since the address would be stale.
+ * All calls share the one array and it keeps the last call's
  * contents (nothing in it needs to start at zero): calls whose work can
  * overlap on the GPU (on different streams, or from several threads without
  * ordering) race on it and must be serialised by the caller.  Allocates

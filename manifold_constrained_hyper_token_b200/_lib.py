@@ -20,7 +20,7 @@ class MhcParams(ctypes.Structure):
     """Mirror of ``mhc_params`` in include/mhc.h."""
     _fields_ = [("n", ctypes.c_int32), ("t_max", ctypes.c_int32), ("T", ctypes.c_int64),
                 ("C", ctypes.c_int64), ("eps", ctypes.c_float), ("dtype", ctypes.c_int32),
-                ("alpha_groups", ctypes.c_int32)]
+                ("alpha_groups", ctypes.c_int32), ("wait_ns", ctypes.c_int64)]
 
 
 _lib = None

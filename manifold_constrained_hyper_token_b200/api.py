@@ -55,12 +55,14 @@ def _stream(stream):
 
 
 def params(n: int, T: int, C: int, dtype: torch.dtype, t_max: int = 20, eps: float = 1e-6,
-           alpha_groups: int = 1):
-    """Build an ``mhc_params`` struct (alpha_groups 3: per-group alpha)."""
+           alpha_groups: int = 1, wait_ns: int = 0):
+    """Build an ``mhc_params`` struct (alpha_groups 3: per-group alpha; wait_ns: limit of
+    the tensor-core kernels' device-side waits, 0 = the library default)."""
     if dtype not in DTYPE_CODE:
         raise ValueError(f"unsupported activation dtype {dtype}")
     return _lib.MhcParams(n=int(n), t_max=int(t_max), T=int(T), C=int(C), eps=float(eps),
-                          dtype=DTYPE_CODE[dtype], alpha_groups=int(alpha_groups))
+                          dtype=DTYPE_CODE[dtype], alpha_groups=int(alpha_groups),
+                          wait_ns=int(wait_ns))
 
 
 def _ag(alpha) -> int:
@@ -88,11 +90,11 @@ def _workspace(nbytes: int, device, ws):
     return ws, ws.numel() * ws.element_size()
 
 
-def mhc_pre(x, phi, b, alpha, *, t_max: int = 20, eps: float = 1e-6, out=None, workspace=None,
-            dev_status=None, stream=None):
+def mhc_pre(x, phi, b, alpha, *, t_max: int = 20, eps: float = 1e-6, wait_ns: int = 0,
+            out=None, workspace=None, dev_status=None, stream=None):
     """x [T,n,C] -> (h_in [T,C], H_pre [T,n], H_post [T,n], H_res [T,n,n])."""
     T, n, C = x.shape
-    p = params(n, T, C, x.dtype, t_max, eps, _ag(alpha))
+    p = params(n, T, C, x.dtype, t_max, eps, _ag(alpha), wait_ns)
     if out is None:
         out = (torch.empty(T, C, dtype=x.dtype, device=x.device),
                torch.empty(T, n, dtype=torch.float32, device=x.device),
@@ -119,11 +121,12 @@ def mhc_post(x, f_out, H_post, H_res, *, out=None, dev_status=None, stream=None)
 
 
 def mhc_backward(x, phi, b, alpha, f_out, grad_x_next, grad_h_in, *, t_max: int = 20,
-                 eps: float = 1e-6, out=None, workspace=None, dev_status=None, stream=None):
+                 eps: float = 1e-6, wait_ns: int = 0, out=None, workspace=None, dev_status=None,
+                 stream=None):
     """Gradients of pre+post with recompute.
     Returns (grad_x, grad_phi, grad_b, grad_alpha, grad_f_out)."""
     T, n, C = x.shape
-    p = params(n, T, C, x.dtype, t_max, eps, _ag(alpha))
+    p = params(n, T, C, x.dtype, t_max, eps, _ag(alpha), wait_ns)
     if out is None:
         out = (torch.empty_like(x), torch.empty_like(phi), torch.empty_like(b),
                torch.empty_like(alpha), torch.empty_like(f_out))
@@ -139,13 +142,14 @@ def mhc_backward(x, phi, b, alpha, f_out, grad_x_next, grad_h_in, *, t_max: int 
 
 
 def mhc_backward_noalloc(x, phi, b, alpha, f_out, grad_x_next, grad_h_in, *, t_max: int = 20,
-                         eps: float = 1e-6, out=None, dev_status=None, stream=None):
+                         eps: float = 1e-6, wait_ns: int = 0, out=None, dev_status=None,
+                         stream=None):
     """mhc_backward without a workspace: the library's fixed device scratch array is used
     (for callers that cannot allocate device memory).  Output tensors must be passed in
     ``out`` by callers that cannot allocate; they are created here only as a convenience.
     Returns (grad_x, grad_phi, grad_b, grad_alpha, grad_f_out)."""
     T, n, C = x.shape
-    p = params(n, T, C, x.dtype, t_max, eps, _ag(alpha))
+    p = params(n, T, C, x.dtype, t_max, eps, _ag(alpha), wait_ns)
     if out is None:
         out = (torch.empty_like(x), torch.empty_like(phi), torch.empty_like(b),
                torch.empty_like(alpha), torch.empty_like(f_out))
@@ -159,11 +163,12 @@ def mhc_backward_noalloc(x, phi, b, alpha, f_out, grad_x_next, grad_h_in, *, t_m
 
 
 def mhc_post_fused(x, f_out, H_post, H_res, phi_next, b_next, alpha_next, *, t_max: int = 20,
-                   eps: float = 1e-6, out=None, workspace=None, dev_status=None, stream=None):
+                   eps: float = 1e-6, wait_ns: int = 0, out=None, workspace=None, dev_status=None,
+                 stream=None):
     """Layer l's post merge fused with layer l+1's mapping.
     Returns (x_next [T,n,C], H_pre_next [T,n], H_post_next [T,n], H_res_next [T,n,n])."""
     T, n, C = x.shape
-    p = params(n, T, C, x.dtype, t_max, eps, _ag(alpha_next))
+    p = params(n, T, C, x.dtype, t_max, eps, _ag(alpha_next), wait_ns)
     if out is None:
         out = (torch.empty_like(x), torch.empty(T, n, dtype=torch.float32, device=x.device),
                torch.empty(T, n, dtype=torch.float32, device=x.device),
@@ -207,11 +212,12 @@ def mhc_post_backward(x, f_out, H_post, grad_x_next, *, out=None, dev_status=Non
 
 
 def mhc_pre_backward(x, phi, b, alpha, grad_x_next, grad_h_in, red, *, t_max: int = 20,
-                     eps: float = 1e-6, out=None, workspace=None, dev_status=None, stream=None):
+                     eps: float = 1e-6, wait_ns: int = 0, out=None, workspace=None, dev_status=None,
+                 stream=None):
     """Second half of the layer backward in training order (after F's backward).
     Returns (grad_x, grad_phi, grad_b, grad_alpha)."""
     T, n, C = x.shape
-    p = params(n, T, C, x.dtype, t_max, eps, _ag(alpha))
+    p = params(n, T, C, x.dtype, t_max, eps, _ag(alpha), wait_ns)
     if out is None:
         out = (torch.empty_like(x), torch.empty_like(phi), torch.empty_like(b),
                torch.empty_like(alpha))
@@ -227,11 +233,12 @@ def mhc_pre_backward(x, phi, b, alpha, grad_x_next, grad_h_in, red, *, t_max: in
 
 
 def mhc_backward_map(x, phi, b, alpha, f_out, grad_x_next, grad_h_in, workspace, *,
-                     t_max: int = 20, eps: float = 1e-6, dev_status=None, stream=None):
+                     t_max: int = 20, eps: float = 1e-6, wait_ns: int = 0, dev_status=None,
+                     stream=None):
     """Phase 1 of mhc_backward: per-token records into ``workspace`` (uint8 tensor of at
     least mhc_backward_workspace_size bytes)."""
     T, n, C = x.shape
-    p = params(n, T, C, x.dtype, t_max, eps, _ag(alpha))
+    p = params(n, T, C, x.dtype, t_max, eps, _ag(alpha), wait_ns)
     st = _lib.load().mhc_backward_map(ctypes.byref(p), _p(x), _p(phi), _p(b), _p(alpha), _p(f_out),
                                       _p(grad_x_next), _p(grad_h_in), _p(workspace),
                                       workspace.numel(), _p(dev_status), _stream(stream))
@@ -239,12 +246,12 @@ def mhc_backward_map(x, phi, b, alpha, f_out, grad_x_next, grad_h_in, workspace,
 
 
 def mhc_backward_apply(x, phi, grad_x_next, grad_h_in, workspace, *, t_max: int = 20,
-                       eps: float = 1e-6, alpha_groups: int = 1, out=None, dev_status=None,
-                       stream=None):
+                       eps: float = 1e-6, wait_ns: int = 0, alpha_groups: int = 1, out=None,
+                       dev_status=None, stream=None):
     """Phase 2 of mhc_backward (alpha_groups as in the map phase).
     Returns (grad_x, grad_phi, grad_b, grad_alpha, grad_f_out)."""
     T, n, C = x.shape
-    p = params(n, T, C, x.dtype, t_max, eps, alpha_groups)
+    p = params(n, T, C, x.dtype, t_max, eps, alpha_groups, wait_ns)
     M = n * n + 2 * n
     if out is None:
         out = (torch.empty_like(x), torch.empty_like(phi),

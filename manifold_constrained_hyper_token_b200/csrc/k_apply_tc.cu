@@ -72,7 +72,6 @@ static_assert(STAGE % 1024 == 0 && U_OFF % 1024 == 0, "stage alignment");
 constexpr uint32_t TMEM_COLS = 512;             // D1 x2 | D2 primaries x PMAX | D2 extra
 constexpr uint32_t D2_COL = 2 * KR;             // 128
 constexpr uint32_t D2X_COL = D2_COL + PMAX * NU;  // 320
-constexpr uint64_t WAIT_NS = 2000000000ull;
 }  // namespace tcap
 
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
@@ -138,6 +137,7 @@ struct ApplyArgs {
   int* status;
   int write_gf;   // 0: grad_f_out is not produced (pre half of the split backward)
   int ag;         // 3: grad_alpha per group (pre, post, res); else one shared alpha
+  uint64_t wait_ns;  // limit of every wait on another warp's or the copy engine's progress
 };
 
 // Walks one CTA's items: for every tile t its P owned slices, then the
@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
       for (cur.start(a, b); cur.valid(a); cur.next(a, b), ++i) {
         const int s = i % NS;
         if (i >= NS && !tc::mbar_wait(bar(B_SFREE + s), (uint32_t)(i / NS - 1) & 1u, abort_flag,
-                                      WAIT_NS)) {
+                                      a.wait_ns)) {
           give_up();
           break;
         }
@@ -279,9 +279,10 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
         tc::bulk_load(base + H_OFF, a.hrec + (int64_t)tt0 * TcRec::H_FLOATS, hbytes, bar(B_FULL + s),
                       pol_keep);
       }
-      if (*abort_flag)
-        for (int k = (i > NS ? i - NS : 0); k < i; ++k)
-          tc::mbar_wait(bar(B_FULL + (k % NS)), (uint32_t)(k / NS) & 1u, nullptr, WAIT_NS / 4);
+      // every copy issued here has landed before the CTA can exit (after a normal
+      // run these waits return at once)
+      for (int k = (i > NS ? i - NS : 0); k < i; ++k)
+        tc::mbar_wait(bar(B_FULL + (k % NS)), (uint32_t)(k / NS) & 1u, nullptr, tc::kDrainWaitNs);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
@@ -296,10 +297,10 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
         const int s = i % NS, d = i & 1;
         const uint32_t sph = (uint32_t)(i / NS) & 1u, dph = (uint32_t)(i >> 1) & 1u;
         const bool extra = cur.is_extra(a);
-        bool ok = tc::mbar_wait(bar(B_FULL + s), sph, abort_flag, WAIT_NS);
-        if (ok && i >= 2) ok = tc::mbar_wait(bar(B_D1FREE + d), dph ^ 1u, abort_flag, WAIT_NS);
+        bool ok = tc::mbar_wait(bar(B_FULL + s), sph, abort_flag, a.wait_ns);
+        if (ok && i >= 2) ok = tc::mbar_wait(bar(B_D1FREE + d), dph ^ 1u, abort_flag, a.wait_ns);
         if (ok && extra && nx > 0)
-          ok = tc::mbar_wait(bar(B_XFREE), (uint32_t)(nx - 1) & 1u, abort_flag, WAIT_NS);
+          ok = tc::mbar_wait(bar(B_XFREE), (uint32_t)(nx - 1) & 1u, abort_flag, a.wait_ns);
         if (!ok) {
           give_up();
           break;
@@ -332,11 +333,11 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
           ++nx;
         }
       }
-      if (!*abort_flag) {
-        tc::mma_commit(bar(B_DONE));
-      } else if (any) {
+      if (!*abort_flag) tc::mma_commit(bar(B_DONE));
+      // every MMA issued here has finished before TMEM is freed
+      if (any) {
         tc::mma_commit(bar(B_FIN));
-        tc::mbar_wait(bar(B_FIN), 0, nullptr, WAIT_NS / 4);
+        tc::mbar_wait(bar(B_FIN), 0, nullptr, tc::kDrainWaitNs);
       }
     }
   } else if (warp == STORE_WARP) {
@@ -348,7 +349,7 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
       ItemCursor cur;
       for (cur.start(a, b); cur.valid(a); cur.next(a, b), ++i) {
         const int s = i % NS;
-        if (!tc::mbar_wait(bar(B_OUTREADY + s), (uint32_t)(i / NS) & 1u, abort_flag, WAIT_NS)) {
+        if (!tc::mbar_wait(bar(B_OUTREADY + s), (uint32_t)(i / NS) & 1u, abort_flag, a.wait_ns)) {
           give_up();
           break;
         }
@@ -430,7 +431,7 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
       const int s = i % NS, d = i & 1;
       const uint32_t sph = (uint32_t)(i / NS) & 1u, dph = (uint32_t)(i >> 1) & 1u;
       bool live = !*abort_flag;
-      if (live && !tc::mbar_wait(bar(B_FULL + s), sph, abort_flag, WAIT_NS)) {
+      if (live && !tc::mbar_wait(bar(B_FULL + s), sph, abort_flag, a.wait_ns)) {
         give_up();
         live = false;
       }
@@ -467,7 +468,7 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
         unpack_pairs(*reinterpret_cast<const uint4*>(st + GG_OFF + sw32(tok, chunk)), gp);
         // grad_f_out = sum_i H_post[i] G_i; it replaces this thread's grad_h_in
         // piece in the stage (same swizzled position) for the tile store
-        if (a.write_gf) {
+        if (a.write_gf && live) {
           uint32_t w[4];
 #pragma unroll
           for (int pr = 0; pr < 4; ++pr) {
@@ -492,7 +493,7 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
           }
         }
       }
-      if (live && !tc::mbar_wait(bar(B_D1READY + d), dph, abort_flag, WAIT_NS)) {
+      if (live && !tc::mbar_wait(bar(B_D1READY + d), dph, abort_flag, a.wait_ns)) {
         give_up();
         live = false;
       }
@@ -517,7 +518,9 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
             asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(acc[jj][pr]));
             w[pr] = pack2(lo + d1[jj][2 * pr], hi + d1[jj][2 * pr + 1]);
           }
-          *reinterpret_cast<uint4*>(st + X_OFF + jj * XB + sw32(tok, chunk)) = make_uint4(w[0], w[1], w[2], w[3]);
+          if (live)
+            *reinterpret_cast<uint4*>(st + X_OFF + jj * XB + sw32(tok, chunk)) =
+                make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
       tc::tc_fence_before();
@@ -531,7 +534,7 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
       if (cur.is_extra(a)) {
         // ---- a leftover slice's item: flush its partial; the last of the
         // slice's NTT partials to arrive adds them in tile order.
-        if (live && !tc::mbar_wait(bar(B_XDONE), (uint32_t)nx & 1u, abort_flag, WAIT_NS)) {
+        if (live && !tc::mbar_wait(bar(B_XDONE), (uint32_t)nx & 1u, abort_flag, a.wait_ns)) {
           give_up();
           live = false;
         }
@@ -575,7 +578,7 @@ __global__ void __launch_bounds__(tcap::NT, 1) k_apply_tc(
     }
 
     // ---- the owned slices' grad_phi rows, accumulated over every tile
-    bool live = !*abort_flag && tc::mbar_wait(bar(B_DONE), 0, abort_flag, WAIT_NS);
+    bool live = !*abort_flag && tc::mbar_wait(bar(B_DONE), 0, abort_flag, a.wait_ns);
     if (!live && !*abort_flag) give_up();
     live = __all_sync(0xffffffffu, live);
     named_bar_sync(1, NEPI_T);
@@ -638,7 +641,7 @@ cudaError_t apply_tc_dispatch(int64_t T, int64_t C, const void* x, const void* p
                               const void* G, const void* g, const void* urec, const float* hrec,
                               const float* part, int nparts, void* gx, void* gf, float* gphi,
                               float* gb, float* ga, int ag, void* scratch, int* st,
-                              cudaStream_t s) {
+                              int64_t wait_ns, cudaStream_t s) {
   using namespace tcap;
   const ApplyPlan pl = apply_plan(T, C, device_sms());
   CUtensorMap mx, mG, mg, mu, mp, mgx, mgf;
@@ -694,6 +697,7 @@ cudaError_t apply_tc_dispatch(int64_t T, int64_t C, const void* x, const void* p
   a.status = st;
   a.write_gf = gf != nullptr ? 1 : 0;
   a.ag = ag;
+  a.wait_ns = tc::wait_limit(wait_ns);
   e = cudaFuncSetAttribute(k_apply_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (e != cudaSuccess) return e;
   if (pl.E > 0) {

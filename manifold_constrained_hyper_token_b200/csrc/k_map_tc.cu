@@ -49,7 +49,6 @@ constexpr int STORE_WARP = 10;
 constexpr int NT = NWARPS * 32;
 constexpr uint32_t TMEM_COLS = 64;
 constexpr int KREC = 52;             // floats per part record: y[24] | ss | dots[24] | pad
-constexpr uint64_t WAIT_NS = 2000000000ull;  // 2 s per wait before giving up
 
 // MAP_FWD: the forward mapping.  MAP_BWD: the backward's recompute with all
 // 24 C-reductions.  MAP_BWD_SPLIT: the pre half of the backward in training
@@ -95,6 +94,11 @@ __global__ void k_phi_split(int64_t K, const float* __restrict__ phi, __nv_bfloa
   }
 }
 
+cudaError_t phi_split_dispatch(int64_t K, const float* phi, void* phi_split, cudaStream_t s) {
+  k_phi_split<<<(unsigned)((K + 255) / 256), 256, 0, s>>>(K, phi, (__nv_bfloat16*)phi_split);
+  return cudaGetLastError();
+}
+
 __device__ __forceinline__ void bf16x8_to_f32(uint4 q, float (&v)[8]) {
   const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
@@ -136,7 +140,7 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
     __nv_bfloat16* __restrict__ urec_o, float* __restrict__ hrec_o, float* __restrict__ part_o,
     const float* __restrict__ red_in, const float* __restrict__ hpost_in,
     const float* __restrict__ hres_in, int kp, float* __restrict__ kpart, int* __restrict__ kcnt,
-    int* status) {
+    int* status, uint64_t wait_ns) {
   using namespace tcmap;
   using CFG = Cfg<MODE>;
   constexpr bool BWD = MODE == MAP_BWD || MODE == MAP_BWD_SPLIT;
@@ -218,7 +222,7 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
       for (int cc = 0; cc < nch; ++cc) {
         const int s = cc % NS;
         const uint32_t ph = (uint32_t)(cc / NS) & 1u;
-        if (cc >= NS && !tc::mbar_wait(empty(s), ph ^ 1u, abort_flag, WAIT_NS)) {
+        if (cc >= NS && !tc::mbar_wait(empty(s), ph ^ 1u, abort_flag, wait_ns)) {
           give_up();
           break;
         }
@@ -239,11 +243,10 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
           tc::tma_load_2d(base + CFG::FN_OFF, &tm_f, full(s), c0, (int)t0, pol_stream);
         ++issued;
       }
-      if (*abort_flag) {
-        // drain: the last min(NS, issued) loads may still be landing
-        for (int cc = (issued > NS ? issued - NS : 0); cc < issued; ++cc)
-          tc::mbar_wait(full(cc % NS), (uint32_t)(cc / NS) & 1u, nullptr, WAIT_NS / 4);
-      }
+      // drain: the last min(NS, issued) loads may still be landing if a consumer
+      // gave up (after a normal run these waits return at once)
+      for (int cc = (issued > NS ? issued - NS : 0); cc < issued; ++cc)
+        tc::mbar_wait(full(cc % NS), (uint32_t)(cc / NS) & 1u, nullptr, tc::kDrainWaitNs);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
@@ -254,7 +257,7 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
         const int s = cc % NS;
         const uint32_t ph = (uint32_t)(cc / NS) & 1u;
         // with the post merge fused, the A operand is x_next, written by the math warps
-        if (!tc::mbar_wait(POST ? xready(s) : full(s), ph, abort_flag, WAIT_NS)) {
+        if (!tc::mbar_wait(POST ? xready(s) : full(s), ph, abort_flag, wait_ns)) {
           give_up();
           break;
         }
@@ -272,11 +275,12 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
         any = true;
         tc::mma_commit(empty(s));
       }
-      if (!*abort_flag) {
-        tc::mma_commit(done_bar);
-      } else if (any) {
+      if (!*abort_flag) tc::mma_commit(done_bar);
+      // every MMA issued here has finished before TMEM is freed, also when a
+      // consumer gave up after done_bar was committed
+      if (any) {
         tc::mma_commit(fin_bar);
-        tc::mbar_wait(fin_bar, 0, nullptr, WAIT_NS / 4);
+        tc::mbar_wait(fin_bar, 0, nullptr, tc::kDrainWaitNs);
       }
     }
   } else if (warp == STORE_WARP) {
@@ -284,7 +288,7 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
     if (POST && lane == 0) {
       for (int cc = 0; cc < nch; ++cc) {
         const int s = cc % NS;
-        if (!tc::mbar_wait(xready(s), (uint32_t)(cc / NS) & 1u, abort_flag, WAIT_NS)) {
+        if (!tc::mbar_wait(xready(s), (uint32_t)(cc / NS) & 1u, abort_flag, wait_ns)) {
           give_up();
           break;
         }
@@ -320,7 +324,7 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
     for (int cc = 0; cc < nch; ++cc) {
       const int s = cc % NS;
       const uint32_t ph = (uint32_t)(cc / NS) & 1u;
-      if (!tc::mbar_wait(full(s), ph, abort_flag, WAIT_NS)) {
+      if (!tc::mbar_wait(full(s), ph, abort_flag, wait_ns)) {
         give_up();
         break;
       }
@@ -400,14 +404,17 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
     // all MMAs (and so all reads of the stage buffers) finished before the
     // stage memory is reused for the epilogue; with the post merge fused, the
     // x_next stores as well
-    bool ok = !*abort_flag && tc::mbar_wait(done_bar, 0, abort_flag, WAIT_NS);
-    if (POST && ok) ok = tc::mbar_wait(sdone_bar, 0, abort_flag, WAIT_NS);
+    bool ok = !*abort_flag && tc::mbar_wait(done_bar, 0, abort_flag, wait_ns);
+    if (POST && ok) ok = tc::mbar_wait(sdone_bar, 0, abort_flag, wait_ns);
     if (!ok && !*abort_flag) give_up();
     ok = __all_sync(0xffffffffu, ok);  // the TMEM loads below are warp-collective
     float* red_ss = reinterpret_cast<float*>(smem);       // [2][TM]
     float* red_dt = red_ss + 2 * TM;                      // [2][M][TM]
     float* dzs = red_dt + 2 * M * TM;                     // [M + 3][TM]
     float* ck = dzs + (M + 3) * TM;                       // checkpoints [nck][16][TM]
+    // every math warp has finished reading its last stages before any of them
+    // reuses the stage memory (the MMA finishing does not imply that)
+    named_bar(1, 256);
     if (ok) {
       red_ss[h * TM + tok] = ss;
       if constexpr (BWD) {
@@ -727,7 +734,7 @@ static cudaError_t launch_map_tc(const CUtensorMap& mx, const CUtensorMap& mp, c
                                  int iters, float eps, const float* b, const float* alpha, int ag,
                                  float* Hpre, float* Hpost, float* Hres, void* urec, float* hrec,
                                  float* part, const float* red, void* kscratch, int* st,
-                                 cudaStream_t s, const float* hpost_in = nullptr,
+                                 int64_t wait_ns, cudaStream_t s, const float* hpost_in = nullptr,
                                  const float* hres_in = nullptr) {
   using namespace tcmap;
   auto kern = k_map_tc<MODE>;
@@ -750,7 +757,8 @@ static cudaError_t launch_map_tc(const CUtensorMap& mx, const CUtensorMap& mp, c
   const int P = (MODE == MAP_BWD || MODE == MAP_BWD_SPLIT) ? ck_period_for(iters, Cfg<MODE>::DATA) : 1;
   kern<<<grid, NT, Cfg<MODE>::SMEM, s>>>(mx, mp, mG, mg, mf, T, C, iters, eps, P, b, alpha, ag, Hpre,
                                          Hpost, Hres, (__nv_bfloat16*)urec, hrec, part, red,
-                                         hpost_in, hres_in, kp, kpart, kcnt, st);
+                                         hpost_in, hres_in, kp, kpart, kcnt, st,
+                                         tc::wait_limit(wait_ns));
   return cudaGetLastError();
 }
 
@@ -759,7 +767,7 @@ cudaError_t map_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float eps
                             int ag,
                             float* Hpre, float* Hpost, float* Hres, const void* G, const void* g,
                             const void* f, const float* red, void* urec, float* hrec, float* part,
-                            void* kscratch, int* st, cudaStream_t s) {
+                            void* kscratch, int* st, int64_t wait_ns, cudaStream_t s) {
   using namespace tcmap;
   const int64_t K = (int64_t)N * C;
   k_phi_split<<<(unsigned)((K + 255) / 256), 256, 0, s>>>(K, phi, (__nv_bfloat16*)phi_split);
@@ -771,13 +779,13 @@ cudaError_t map_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float eps
   switch (mode) {
     case MAP_FWD:
       return launch_map_tc<MAP_FWD>(mx, mp, mG, mg, mf, T, C, iters, eps, b, alpha, ag, Hpre, Hpost,
-                                    Hres, nullptr, nullptr, nullptr, nullptr, kscratch, st, s);
+                                    Hres, nullptr, nullptr, nullptr, nullptr, kscratch, st, wait_ns, s);
     case MAP_BWD:
       return launch_map_tc<MAP_BWD>(mx, mp, mG, mg, mf, T, C, iters, eps, b, alpha, ag, nullptr,
-                                    nullptr, nullptr, urec, hrec, part, nullptr, kscratch, st, s);
+                                    nullptr, nullptr, urec, hrec, part, nullptr, kscratch, st, wait_ns, s);
     case MAP_BWD_SPLIT:
       return launch_map_tc<MAP_BWD_SPLIT>(mx, mp, mG, mg, mf, T, C, iters, eps, b, alpha, ag, nullptr,
-                                          nullptr, nullptr, urec, hrec, part, red, kscratch, st, s);
+                                          nullptr, nullptr, urec, hrec, part, red, kscratch, st, wait_ns, s);
     default:
       return cudaErrorInvalidValue;
   }
@@ -791,7 +799,8 @@ cudaError_t post_map_tc_dispatch(int64_t T, int64_t C, int iters, float eps, con
                                  const float* phi_next, void* phi_split, const float* b_next,
                                  const float* alpha_next, int ag, void* x_next, float* Hpre,
                                  float* Hpost,
-                                 float* Hres, void* kscratch, int* st, cudaStream_t s) {
+                                 float* Hres, void* kscratch, int* st, int64_t wait_ns,
+                                 cudaStream_t s) {
   using namespace tcmap;
   const int64_t K = (int64_t)N * C;
   k_phi_split<<<(unsigned)((K + 255) / 256), 256, 0, s>>>(K, phi_next,
@@ -814,7 +823,7 @@ cudaError_t post_map_tc_dispatch(int64_t T, int64_t C, int iters, float eps, con
   if (e != cudaSuccess) return e;
   return launch_map_tc<MAP_POSTFWD>(mx, mp, mG, mg, mf, T, C, iters, eps, b_next, alpha_next, ag, Hpre,
                                     Hpost, Hres, nullptr, nullptr, nullptr, nullptr, kscratch, st,
-                                    s, Hpost_in, Hres_in);
+                                    wait_ns, s, Hpost_in, Hres_in);
 }
 
 }  // namespace mhc

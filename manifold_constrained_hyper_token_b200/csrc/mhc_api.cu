@@ -10,7 +10,7 @@
 namespace {
 
 constexpr int kVersionMajor = 0;
-constexpr int kVersionMinor = 1;
+constexpr int kVersionMinor = 2;
 
 bool aligned16(const void* p) { return p != nullptr && ((uintptr_t)p & 15u) == 0; }
 
@@ -22,6 +22,7 @@ mhc_status check_params(const mhc_params* p) {
   if (p->dtype != MHC_DTYPE_F32 && p->dtype != MHC_DTYPE_BF16) return MHC_ERR_UNSUPPORTED;
   if (p->alpha_groups != 0 && p->alpha_groups != 1 && p->alpha_groups != 3)
     return MHC_ERR_INVALID_ARG;
+  if (p->wait_ns < 0) return MHC_ERR_INVALID_ARG;
   // tile coordinates of the TMA copies are 32-bit signed: keep T (and a tile
   // past it) inside that range
   if (p->T > (int64_t)0x7fffffffLL - 256) return MHC_ERR_INVALID_ARG;
@@ -144,10 +145,10 @@ mhc_status mhc_pre(const mhc_params* p, const void* x, const float* phi, const f
       return MHC_ERR_WORKSPACE;
     char* ws = (char*)workspace;
     st = from_cuda(mhc::map_tc_dispatch(mhc::MAP_FWD, p->T, p->C, p->t_max, p->eps, x, phi, ws, b,
-                                        alpha, alpha_groups(p), H_pre, H_post, H_res, nullptr, nullptr, nullptr,
-                                        nullptr, nullptr, nullptr, nullptr,
+                                        alpha, alpha_groups(p), H_pre, H_post, H_res, nullptr,
+                                        nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                                         ws + round_up(mhc::map_tc_phi_bytes(p->C), 256),
-                                        dev_status, s));
+                                        dev_status, p->wait_ns, s));
   } else {
     st = from_cuda(mhc::map_fwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
                                          alpha, alpha_groups(p), H_pre, H_post, H_res, dev_status, s));
@@ -190,10 +191,10 @@ mhc_status mhc_backward_map(const mhc_params* p, const void* x, const float* phi
   if (use_tc(p))
     return from_cuda(mhc::map_tc_dispatch(mhc::MAP_BWD, p->T, p->C, p->t_max, p->eps, x, phi,
                                           ws + w.phi_off, b, alpha, alpha_groups(p), nullptr,
-                                          nullptr, nullptr, grad_x_next, grad_h_in, f_out, nullptr, ws + w.urec_off,
-                                          (float*)(ws + w.hrec_off), (float*)(ws + w.part_off),
-                                          ws + w.kmap_off,
-                                          dev_status, (cudaStream_t)stream));
+                                          nullptr, nullptr, grad_x_next, grad_h_in, f_out, nullptr,
+                                          ws + w.urec_off, (float*)(ws + w.hrec_off),
+                                          (float*)(ws + w.part_off), ws + w.kmap_off, dev_status,
+                                          p->wait_ns, (cudaStream_t)stream));
   return from_cuda(mhc::map_bwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
                                          alpha, alpha_groups(p), grad_x_next, grad_h_in, f_out, nullptr,
                                          (float*)(ws + w.coef_off), (float*)(ws + w.part_off),
@@ -222,7 +223,7 @@ mhc_status mhc_backward_apply(const mhc_params* p, const void* x, const float* p
                                             (const float*)(ws + w.part_off), w.nparts, grad_x,
                                             grad_f_out, grad_phi, grad_b, grad_alpha,
                                             alpha_groups(p), (void*)(ws + w.apply_off), dev_status,
-                                            (cudaStream_t)stream));
+                                            p->wait_ns, (cudaStream_t)stream));
   return from_cuda(mhc::apply_dispatch(p->n, p->dtype, p->T, p->C, x, phi, grad_x_next, grad_h_in,
                                        (const float*)(ws + w.coef_off),
                                        (const float*)(ws + w.part_off), w.nparts, grad_x,
@@ -271,7 +272,7 @@ mhc_status mhc_post_fused(const mhc_params* p, const void* x, const void* f_out,
     return from_cuda(mhc::post_map_tc_dispatch(
         p->T, p->C, p->t_max, p->eps, x, f_out, H_post, H_res, phi_next, ws, b_next, alpha_next,
         alpha_groups(p), x_next, H_pre_next, H_post_next, H_res_next,
-        ws + round_up(mhc::map_tc_phi_bytes(p->C), 256), dev_status, s));
+        ws + round_up(mhc::map_tc_phi_bytes(p->C), 256), dev_status, p->wait_ns, s));
   }
   // fp32 or n != 4: the post merge, then the mapping of x_next (both on the GPU)
   st = from_cuda(mhc::post_dispatch(p->n, p->dtype, p->T, p->C, x, f_out, H_post, H_res, x_next, s));
@@ -329,17 +330,18 @@ mhc_status mhc_pre_backward(const mhc_params* p, const void* x, const float* phi
   char* ws = (char*)workspace;
   cudaStream_t s = (cudaStream_t)stream;
   if (use_tc(p)) {
-    st = from_cuda(mhc::map_tc_dispatch(mhc::MAP_BWD_SPLIT, p->T, p->C, p->t_max, p->eps, x, phi,
-                                        ws + w.phi_off, b, alpha, alpha_groups(p), nullptr,
-                                        nullptr, nullptr, nullptr, grad_h_in, nullptr, red, ws + w.urec_off,
-                                        (float*)(ws + w.hrec_off), (float*)(ws + w.part_off),
-                                        ws + w.kmap_off, dev_status, s));
+    st = from_cuda(mhc::map_tc_dispatch(mhc::MAP_BWD_SPLIT, p->T, p->C, p->t_max, p->eps, x,
+                                        phi, ws + w.phi_off, b, alpha, alpha_groups(p), nullptr,
+                                        nullptr, nullptr, nullptr, grad_h_in, nullptr, red,
+                                        ws + w.urec_off, (float*)(ws + w.hrec_off),
+                                        (float*)(ws + w.part_off), ws + w.kmap_off, dev_status,
+                                        p->wait_ns, s));
     if (st != MHC_OK) return st;
     return from_cuda(mhc::apply_tc_dispatch(p->T, p->C, x, ws + w.phi_off, grad_x_next, grad_h_in,
                                             ws + w.urec_off, (const float*)(ws + w.hrec_off),
                                             (const float*)(ws + w.part_off), w.nparts, grad_x,
                                             nullptr, grad_phi, grad_b, grad_alpha, alpha_groups(p),
-                                            (void*)(ws + w.apply_off), dev_status, s));
+                                            (void*)(ws + w.apply_off), dev_status, p->wait_ns, s));
   }
   st = from_cuda(mhc::map_bwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
                                        alpha, alpha_groups(p), nullptr, grad_h_in, nullptr, red,

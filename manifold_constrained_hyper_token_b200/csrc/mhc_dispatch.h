@@ -40,18 +40,23 @@ cudaError_t map_bwd_dispatch(int n, int dtype, int64_t T, int64_t C, int iters, 
                              const void* x, const float* phi, const float* b, const float* alpha,
                              int ag, const void* G, const void* g, const void* f, const float* red,
                              float* coef, float* part, int* st, cudaStream_t s);
-// k_map_tc.cu (bf16, n = 4: projection on the tensor cores); mode is a MapMode
+// k_map_tc.cu (bf16, n = 4: projection on the tensor cores); mode is a MapMode.
+// wait_ns: limit of each wait on another warp's or the copy engine's progress
+// (0: the default 2 s); the tensor-core kernels take it, the CUDA-core ones
+// have no such waits.
 cudaError_t map_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float eps, const void* x,
                             const float* phi, void* phi_split, const float* b, const float* alpha,
                             int ag, float* Hpre, float* Hpost, float* Hres, const void* G,
                             const void* g,
                             const void* f, const float* red, void* urec, float* hrec, float* part,
-                            void* kscratch, int* st, cudaStream_t s);
+                            void* kscratch, int* st, int64_t wait_ns, cudaStream_t s);
 size_t map_tc_phi_bytes(int64_t C);
 // scratch of the channel-split mapping (part records, counters); kscratch
 // must hold this many bytes, 256-byte aligned (may be null when it is 0)
 size_t map_tc_scratch_bytes(int64_t T, int64_t C);
 
+// phi [K][24] fp32 -> the bf16 split copy of phi^T [48][K] the mapping MMAs read
+cudaError_t phi_split_dispatch(int64_t K, const float* phi, void* phi_split, cudaStream_t s);
 // k_wide.cu (n = 16, CUDA cores); the mapping's mode is a MapMode
 int wide_map_tokens_per_cta();
 cudaError_t wide_map_dispatch(int mode, int dtype, int64_t T, int64_t C, int iters, float eps,
@@ -72,14 +77,15 @@ cudaError_t post_map_tc_dispatch(int64_t T, int64_t C, int iters, float eps, con
                                  const void* f, const float* Hpost_in, const float* Hres_in,
                                  const float* phi_next, void* phi_split, const float* b_next,
                                  const float* alpha_next, int ag, void* x_next, float* Hpre,
-                                 float* Hpost, float* Hres, void* kscratch, int* st, cudaStream_t s);
+                                 float* Hpost, float* Hres, void* kscratch, int* st,
+                                 int64_t wait_ns, cudaStream_t s);
 // k_apply_tc.cu (bf16, n = 4: phi u and grad_phi on the tensor cores);
 // gf == nullptr skips grad_f_out
 cudaError_t apply_tc_dispatch(int64_t T, int64_t C, const void* x, const void* phi_split,
                               const void* G, const void* g, const void* urec, const float* hrec,
                               const float* part, int nparts, void* gx, void* gf, float* gphi,
                               float* gb, float* ga, int ag, void* scratch, int* st,
-                              cudaStream_t s);
+                              int64_t wait_ns, cudaStream_t s);
 size_t apply_tc_scratch_bytes(int64_t T, int64_t C);
 // k_bwd.cu (CUDA cores); gf == nullptr skips grad_f_out
 cudaError_t apply_dispatch(int n, int dtype, int64_t T, int64_t C, const void* x, const float* phi,

@@ -48,11 +48,43 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of phase `parity` (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Limits below this are counted in SM clock cycles (two per nanosecond) with
+// non-blocking tests, so that even a limit of a few nanoseconds gives up at
+// the first test that finds the phase incomplete; longer limits use the
+// global timer and the suspending try_wait.
+constexpr uint64_t kShortWaitNs = 1000000ull;
+
+// The short-limit wait, out of line: only a deliberately short limit takes it.
+static __device__ __noinline__ bool mbar_wait_short(uint32_t bar, uint32_t parity, volatile int* abort,
+                                             uint64_t limit_ns) {
+  const long long c0 = clock64();
+  const long long lim = (long long)(2 * limit_ns);
+  for (;;) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if (abort != nullptr && *abort) return false;
+    if (clock64() - c0 > lim) return false;
+  }
+}
+
 // Wait for phase `parity` of the barrier, giving up after `limit_ns` of wall
 // time or as soon as *abort becomes non-zero (abort may be null: time limit
 // only).  Returns false when it gave up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           uint64_t limit_ns) {
+  if (limit_ns < kShortWaitNs) return mbar_wait_short(bar, parity, abort, limit_ns);
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
@@ -62,6 +94,15 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       if (global_ns() - t0 > limit_ns) return false;
     }
   }
+}
+
+// Default limit of a wait on another warp's or the copy engine's progress, and
+// the fixed limit of the drain waits that run after a wait gave up (for copies
+// and MMAs this CTA already issued, which finish in microseconds).
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+constexpr uint64_t kDrainWaitNs = 500000000ull;
+__host__ __device__ __forceinline__ uint64_t wait_limit(int64_t requested_ns) {
+  return requested_ns > 0 ? (uint64_t)requested_ns : kDefaultWaitNs;
 }
 
 // -------------------------------------------------------------------- TMA

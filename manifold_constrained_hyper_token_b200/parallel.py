@@ -3,7 +3,8 @@
 Tokens are independent and the layer's parameters (phi, b, alpha) are shared,
 so a batch shards over ranks by tokens with no exchange in the forward pass;
 the backward's only exchange is a sum over ranks of the parameter gradients
-(grad_phi [nC, n^2+2n], grad_b [n^2+2n], grad_alpha [1]), kept in one flat
+(grad_phi [nC, n^2+2n], grad_b [n^2+2n], grad_alpha [1] or [3] with per-group
+alpha), kept in one flat
 buffer so that it is a single all-reduce.  These helpers are the host side of
 that scheme; the per-rank compute is the library's kernels.
 """
@@ -20,10 +21,12 @@ def token_shard(T: int, rank: int, world: int) -> tuple[int, int]:
     return start, start + base + (1 if rank < extra else 0)
 
 
-def param_grad_buffer(n: int, C: int, device, dtype=torch.float32):
-    """One flat buffer and its (grad_phi, grad_b, grad_alpha) views."""
+def param_grad_buffer(n: int, C: int, device, dtype=torch.float32, alpha_groups: int = 1):
+    """One flat buffer and its (grad_phi, grad_b, grad_alpha) views.  grad_alpha has
+    one entry for a shared alpha and three (pre, post, res) when alpha_groups == 3."""
     K, M = n * C, n * n + 2 * n
-    flat = torch.empty(K * M + M + 1, dtype=dtype, device=device)
+    na = 3 if alpha_groups == 3 else 1
+    flat = torch.empty(K * M + M + na, dtype=dtype, device=device)
     return flat, flat[:K * M].view(K, M), flat[K * M:K * M + M], flat[K * M + M:]
 
 

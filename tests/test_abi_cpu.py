@@ -45,6 +45,15 @@ def test_version(lib):
     assert lib.mhc_version() >= 1
 
 
+def test_params_struct_layout():
+    """The ctypes mirror of mhc_params has the C layout: three int32/int64 pairs,
+    eps, dtype, alpha_groups and the int64 wait limit (48 bytes)."""
+    from manifold_constrained_hyper_token_b200 import _lib
+    P = _lib.MhcParams
+    assert ctypes.sizeof(P) == 48
+    assert [P.T.offset, P.C.offset, P.eps.offset, P.wait_ns.offset] == [8, 16, 24, 40]
+
+
 def _params(**kw):
     from manifold_constrained_hyper_token_b200 import _lib
     d = dict(n=4, t_max=20, T=16, C=64, eps=1e-6, dtype=1)
@@ -68,7 +77,7 @@ ODD = ctypes.c_void_p(0x10004)
     (dict(T=0), 1), (dict(T=2**31 - 256), 1), (dict(C=12), 1), (dict(C=0), 1), (dict(t_max=-1), 1),
     (dict(eps=-1.0), 1),
     (dict(eps=float("nan")), 1), (dict(n=3), 2), (dict(n=32), 2), (dict(dtype=7), 2),
-    (dict(alpha_groups=2), 1),
+    (dict(alpha_groups=2), 1), (dict(wait_ns=-1), 1),
 ])
 def test_pre_rejects_bad_params(lib, kw, code):
     p = _params(**kw)

@@ -17,7 +17,7 @@ def _free_port() -> int:
         return s.getsockname()[1]
 
 
-def _worker(rank, world, port, result_dir):
+def _worker(rank, world, port, result_dir, alpha):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     import datetime
@@ -31,12 +31,13 @@ def _worker(rank, world, port, result_dir):
     T, n, C = 37, 4, 16
     d = synth.layer_inputs(T, n, C, seed=3, dtype=torch.float32, backward=True)
     lo, hi = parallel.token_shard(T, rank, world)
-    r = oracle.backward(d["x"][lo:hi], d["phi"], d["b"], 0.3, d["f_out"][lo:hi],
+    r = oracle.backward(d["x"][lo:hi], d["phi"], d["b"], alpha, d["f_out"][lo:hi],
                         d["grad_x_next"][lo:hi], d["grad_h_in"][lo:hi], iters=20)
-    flat, gphi, gb, ga = parallel.param_grad_buffer(n, C, "cpu", torch.float64)
+    flat, gphi, gb, ga = parallel.param_grad_buffer(n, C, "cpu", torch.float64,
+                                                    alpha_groups=len(alpha))
     gphi.copy_(torch.from_numpy(r["grad_phi"]))
     gb.copy_(torch.from_numpy(r["grad_b"]))
-    ga.fill_(r["grad_alpha"])
+    ga.copy_(torch.from_numpy(np.atleast_1d(np.asarray(r["grad_alpha"], dtype=np.float64))))
     parallel.allreduce_param_grads(flat)
     slowest = parallel.max_over_ranks(10.0 + rank, "cpu")
     np.save(os.path.join(result_dir, f"flat{rank}.npy"), flat.numpy())
@@ -57,23 +58,27 @@ def test_token_shard_covers_all_tokens():
             assert max(sizes) - min(sizes) <= 1
 
 
-def test_two_rank_backward_matches_single(tmp_path):
+@pytest.mark.parametrize("alpha", [[0.3], [0.3, -0.2, 0.5]], ids=["shared_alpha", "alpha_groups3"])
+def test_two_rank_backward_matches_single(tmp_path, alpha):
     import oracle
     from manifold_constrained_hyper_token_b200 import synth
     oracle.build()
     world = 2
-    mp.start_processes(_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+    mp.start_processes(_worker, args=(world, _free_port(), str(tmp_path), alpha), nprocs=world,
                        join=True, start_method="spawn")
     T, n, C = 37, 4, 16
     d = synth.layer_inputs(T, n, C, seed=3, dtype=torch.float32, backward=True)
-    full = oracle.backward(d["x"], d["phi"], d["b"], 0.3, d["f_out"], d["grad_x_next"],
+    full = oracle.backward(d["x"], d["phi"], d["b"], alpha, d["f_out"], d["grad_x_next"],
                            d["grad_h_in"], iters=20)
     K, M = n * C, n * n + 2 * n
     flats = [np.load(tmp_path / f"flat{r}.npy") for r in range(world)]
     np.testing.assert_array_equal(flats[0], flats[1])  # every rank holds the same sum
     np.testing.assert_allclose(flats[0][:K * M].reshape(K, M), full["grad_phi"], rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(flats[0][K * M:K * M + M], full["grad_b"], rtol=1e-12, atol=1e-12)
-    assert flats[0][-1] == pytest.approx(full["grad_alpha"], rel=1e-12, abs=1e-12)
+    na = len(alpha)
+    assert flats[0].size == K * M + M + na  # the buffer holds one grad_alpha per group
+    np.testing.assert_allclose(flats[0][K * M + M:], np.atleast_1d(full["grad_alpha"]),
+                               rtol=1e-12, atol=1e-12)
     gx = np.concatenate([np.load(tmp_path / f"gx{r}.npy") for r in range(world)])
     np.testing.assert_array_equal(gx, full["grad_x"])  # per-token outputs need no exchange
     assert all(np.load(tmp_path / f"max{r}.npy")[0] == 11.0 for r in range(world))

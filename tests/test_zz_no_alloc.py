@@ -13,7 +13,7 @@ import ctypes
 import pytest
 import torch
 
-from conftest import rel_err
+from conftest import assert_close, close_errs, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -36,12 +36,13 @@ def _case(T, n, C, dtype, seed):
     return {k: v.cuda() for k, v in d.items()}
 
 
-def _noalloc_via_abi(d, t_max=20, eps=1e-6):
+def _noalloc_via_abi(d, t_max=20, eps=1e-6, out=None):
     """Call the C entry point directly with caller-allocated outputs only."""
     from manifold_constrained_hyper_token_b200 import _lib, api
     T, n, C = d["x"].shape
-    out = (torch.empty_like(d["x"]), torch.empty_like(d["phi"]), torch.empty_like(d["b"]),
-           torch.empty_like(d["alpha"]), torch.empty_like(d["f_out"]))
+    if out is None:
+        out = (torch.empty_like(d["x"]), torch.empty_like(d["phi"]), torch.empty_like(d["b"]),
+               torch.empty_like(d["alpha"]), torch.empty_like(d["f_out"]))
     p = api.params(n, T, C, d["x"].dtype, t_max, eps)
     ptr = lambda t: ctypes.c_void_p(t.data_ptr())
     st = _lib.load().mhc_backward_noalloc(
@@ -51,11 +52,18 @@ def _noalloc_via_abi(d, t_max=20, eps=1e-6):
     return st, out
 
 
+# per stream count: two calls in a row with different sizes and inputs (the
+# second must not see anything the first left in the shared scratch); n = 8
+# with T = 6000 needs 3.9 MB of the 4 MiB array (656-byte records per token)
+CASES = {4: ((1000, 4, 1024, 1), (333, 4, 512, 2)),
+         8: ((6000, 8, 64, 3), (100, 8, 256, 4)),
+         2: ((2000, 2, 512, 5), (77, 2, 64, 6))}
+
+
+@pytest.mark.parametrize("n", [4, 8, 2])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-def test_noalloc_matches_backward_on_consecutive_calls(mhc, dtype):
-    # two calls in a row with different sizes and inputs: the second must not
-    # see anything the first left in the shared scratch
-    for T, n, C, seed in ((1000, 4, 1024, 1), (333, 4, 512, 2)):
+def test_noalloc_matches_backward_on_consecutive_calls(mhc, dtype, n):
+    for T, n, C, seed in CASES[n]:
         d = _case(T, n, C, dtype, seed)
         st, got = _noalloc_via_abi(d)
         assert st == 0, mhc.mhc_status_string(st)
@@ -76,3 +84,18 @@ def test_noalloc_rejects_sizes_beyond_scratch(mhc):
     fake = ctypes.c_void_p(0x10000)
     st = _lib.load().mhc_backward_noalloc(ctypes.byref(p), *([fake] * 12), None, None)
     assert st == 6  # MHC_ERR_WORKSPACE, returned before any launch
+
+
+def test_noalloc_allocates_nothing(mhc):
+    """After a first call on the device (which looks up the array's address),
+    further calls leave the device's free memory unchanged."""
+    d = _case(1000, 4, 1024, torch.bfloat16, seed=7)
+    st, out = _noalloc_via_abi(d)
+    assert st == 0
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for _ in range(3):
+        st, _ = _noalloc_via_abi(d, out=out)  # the same caller-owned outputs
+        assert st == 0
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
