@@ -1,0 +1,523 @@
+// k_map8_tc.cu -- per-token mapping for n = 8 streams with bf16 activations:
+// the logit projection y = x . phi (nC x 80) runs on the 5th-generation
+// tensor cores (tcgen05.mma, bf16 operands, fp32 accumulation in TMEM); the
+// sum of squares and, in the backward, the 80 C-reductions run on the CUDA
+// cores from the same shared-memory stages.  Sources: the fused RMSNorm /
+// projection / gating operator of the chatgpz.de explainer (section
+// "Systemarbeit und Schulungsaufwand"), the n-stream buffer of section "Von
+// Residualverbindungen zu Hyperverbindungen", and reportify.cn [17]-[19],
+// [21], [26] (RMS applied after the projection, Sinkhorn and its custom
+// backward in one operator, recompute, wider stream buffers).
+//
+// One CTA = 128 tokens (the MMA M).  The token's 8 C inputs stream through a
+// TMA ring in chunks of 16 channels x 8 streams (32-byte rows, 32-byte
+// swizzle): per stream an x tile [128 x 16] (the A operand, K-major) and the
+// rows of the bf16 split copy of phi^T as a [160 x 16] B operand -- the 80
+// logit columns' high parts, then their low parts (phi = hi + lo) -- so
+// y = D[:, m] + D[:, 80 + m] carries phi to ~16 bits while x is exact.
+//
+// Warp roles: warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs, warps
+// 2..9 reduce: warp 2 + 4h + q covers token rows 32q..32q+31 and stream half
+// h, i.e. the sum of squares of streams 4h..4h+3 and, in the backward,
+// <G_i, x_j> and <G_i, f_out> for i in 4h..4h+3 (all j) and <g, x_j> for j in
+// 4h..4h+3.  The h = 0 warps then run the per-token epilogue (gates,
+// Sinkhorn and its adjoint) with one thread per token and write the same
+// per-token records as the CUDA-core mapping, which the n = 8 apply reads.
+// Every wait is bounded; on timeout the kernel records MHC_ERR_TIMEOUT,
+// drains what it issued, frees TMEM and returns.
+#include "mhc_common.cuh"
+#include "mhc_dispatch.h"
+#include "tc_sm100.cuh"
+
+namespace mhc {
+
+namespace tcm8 {
+constexpr int N = 8;
+constexpr int M = N * N + 2 * N;     // 80 logits
+constexpr int TM = 128;              // tokens per CTA (MMA M)
+constexpr int NL = 2 * M;            // MMA N: 80 high + 80 low logit columns
+constexpr int CH = 16;               // channels per chunk: 32-byte rows
+constexpr int ROW = CH * 2;
+constexpr int XBOX = TM * ROW;       // one stream's x (or grad_x_next) tile: 4 KB
+constexpr int PBOX = NL * ROW;       // one stream's phi^T tile: 5 KB
+constexpr int NW = 10;
+constexpr int NT = NW * 32;
+constexpr uint32_t TMEM_COLS = 256;
+constexpr int NDH = 4 * N + 4 + 4;   // reductions per stream half: <G_i,x_j> 32, <G_i,f> 4, <g,x_j> 4
+
+template <int MODE> struct Cfg {
+  static constexpr bool FULLB = MODE == MAP_BWD;
+  static constexpr bool BWD = MODE == MAP_BWD || MODE == MAP_BWD_SPLIT;
+  static constexpr int X_OFF = 0;
+  static constexpr int P_OFF = N * XBOX;
+  static constexpr int G_OFF = P_OFF + N * PBOX;                 // grad_x_next (full backward)
+  static constexpr int GG_OFF = FULLB ? G_OFF + N * XBOX : G_OFF;  // grad_h_in (backward)
+  static constexpr int F_OFF = GG_OFF + XBOX;                     // f_out (full backward)
+  static constexpr int STAGE = FULLB ? F_OFF + XBOX : (BWD ? GG_OFF + XBOX : G_OFF);
+  static constexpr int NS = BWD ? 2 : 3;
+  // the stages, reused after the chunk loop by the epilogue; the backward
+  // epilogue keeps Sinkhorn checkpoints there, so the split backward (smaller
+  // stages) asks for the full backward's size
+  static constexpr int DATA = BWD && NS * STAGE < 229376 ? 229376 : NS * STAGE;
+  static constexpr int SMEM = DATA + 1024 /*align*/ + 256 /*barriers, flags*/;
+  static_assert(SMEM <= 232448, "shared memory");
+};
+}  // namespace tcm8
+
+namespace {
+
+__device__ __forceinline__ void unpack8(uint4 q, float (&v)[8]) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+// 16-byte piece `c` (0 or 1) of token row `tok` of a [128 x 16] bf16 tile
+// stored with the 32-byte swizzle.
+__device__ __forceinline__ uint4 ld32sw(const uint8_t* tile, int tok, int c) {
+  return *reinterpret_cast<const uint4*>(tile + tok * tcm8::ROW + ((c ^ ((tok >> 2) & 1)) << 4));
+}
+
+__device__ __forceinline__ void nbar8(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+}  // namespace
+
+template <int MODE>
+__global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
+    const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_phi,
+    const __grid_constant__ CUtensorMap tm_G, const __grid_constant__ CUtensorMap tm_g,
+    const __grid_constant__ CUtensorMap tm_f, int64_t T, int64_t C, int iters, float eps,
+    int ck_period, const float* __restrict__ bias, const float* __restrict__ alpha_p, int ag,
+    float* __restrict__ Hpre_o, float* __restrict__ Hpost_o, float* __restrict__ Hres_o,
+    float* __restrict__ coef_o, float* __restrict__ part_o, const float* __restrict__ red_in,
+    int* status, uint64_t wait_ns) {
+  using namespace tcm8;
+  using CFG = Cfg<MODE>;
+  using CF = Coef<N>;
+  constexpr bool BWD = CFG::BWD, FULLB = CFG::FULLB;
+  constexpr bool SPLIT = MODE == MAP_BWD_SPLIT;
+  constexpr int NS = CFG::NS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~(uintptr_t)1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + CFG::DATA);  // full[NS] empty[NS] done fin
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  auto full = [&](int s) { return tc::smem_u32(bars + s); };
+  auto empty = [&](int s) { return tc::smem_u32(bars + NS + s); };
+  const uint32_t done_bar = tc::smem_u32(bars + 2 * NS);
+  const uint32_t fin_bar = tc::smem_u32(bars + 2 * NS + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int64_t t0 = (int64_t)blockIdx.x * TM;
+  const int nch = (int)((C + CH - 1) / CH);
+  const int64_t K = (int64_t)N * C;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      tc::mbar_init(full(s), 1);
+      tc::mbar_init(empty(s), 1 + 8);  // the MMA commit + every math warp
+    }
+    tc::mbar_init(done_bar, 1);
+    tc::mbar_init(fin_bar, 1);
+    *abort_flag = 0;
+    tc::mbar_fence_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tc::tma_prefetch_desc(&tm_x);
+    tc::tma_prefetch_desc(&tm_phi);
+    if constexpr (BWD) tc::tma_prefetch_desc(&tm_g);
+    if constexpr (FULLB) {
+      tc::tma_prefetch_desc(&tm_G);
+      tc::tma_prefetch_desc(&tm_f);
+    }
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tc::smem_u32(tmem_slot), TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto give_up = [&]() {
+    *abort_flag = 1;
+    flag_status(status, MHC_ERR_TIMEOUT);
+  };
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA
+    if (lane == 0) {
+      const uint64_t pol_stream = tc::policy_evict_first();
+      const uint64_t pol_keep = tc::policy_evict_last();
+      int issued = 0;
+      for (int cc = 0; cc < nch; ++cc) {
+        const int s = cc % NS;
+        if (cc >= NS && !tc::mbar_wait(empty(s), ((uint32_t)(cc / NS) & 1u) ^ 1u, abort_flag,
+                                       wait_ns)) {
+          give_up();
+          break;
+        }
+        const uint32_t base = tc::smem_u32(smem + s * CFG::STAGE);
+        tc::mbar_arrive_expect_tx(full(s), CFG::STAGE);
+        const int c0 = cc * CH;
+        for (int i = 0; i < N; ++i) {
+          tc::tma_load_3d(base + CFG::X_OFF + i * XBOX, &tm_x, full(s), c0, i, (int)t0, pol_stream);
+          tc::tma_load_3d(base + CFG::P_OFF + i * PBOX, &tm_phi, full(s), c0, i, 0, pol_keep);
+          if constexpr (FULLB)
+            tc::tma_load_3d(base + CFG::G_OFF + i * XBOX, &tm_G, full(s), c0, i, (int)t0, pol_stream);
+        }
+        if constexpr (BWD) tc::tma_load_2d(base + CFG::GG_OFF, &tm_g, full(s), c0, (int)t0, pol_stream);
+        if constexpr (FULLB) tc::tma_load_2d(base + CFG::F_OFF, &tm_f, full(s), c0, (int)t0, pol_stream);
+        ++issued;
+      }
+      // every copy issued here has landed before the CTA can exit
+      for (int cc = (issued > NS ? issued - NS : 0); cc < issued; ++cc)
+        tc::mbar_wait(full(cc % NS), (uint32_t)(cc / NS) & 1u, nullptr, tc::kDrainWaitNs);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t idesc = tc::idesc_bf16(TM, NL);
+      bool any = false;
+      for (int cc = 0; cc < nch; ++cc) {
+        const int s = cc % NS;
+        if (!tc::mbar_wait(full(s), (uint32_t)(cc / NS) & 1u, abort_flag, wait_ns)) {
+          give_up();
+          break;
+        }
+        tc::tc_fence_after();
+        const uint32_t base = tc::smem_u32(smem + s * CFG::STAGE);
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+          const uint64_t a = tc::smem_desc(base + CFG::X_OFF + i * XBOX, 16, 8 * ROW, tc::SWZ_32B);
+          const uint64_t bd = tc::smem_desc(base + CFG::P_OFF + i * PBOX, 16, 8 * ROW, tc::SWZ_32B);
+          tc::mma_bf16(tmem, a, bd, idesc, (cc | i) != 0 ? 1u : 0u);
+        }
+        any = true;
+        tc::mma_commit(empty(s));
+      }
+      if (!*abort_flag) tc::mma_commit(done_bar);
+      // every MMA issued here has finished before TMEM is freed
+      if (any) {
+        tc::mma_commit(fin_bar);
+        tc::mbar_wait(fin_bar, 0, nullptr, tc::kDrainWaitNs);
+      }
+    }
+  } else {
+    // -------------------------------------------------- CUDA-core reductions
+    const int q = warp & 3;              // TMEM lane quarter this warp may read
+    const int h = (warp - 2) >> 2;       // stream half: streams 4h..4h+3
+    const int tok = 32 * q + lane;
+    float ss = 0.0f;
+    // [0, 32): <G_i, x_j> for i = 4h + r (r = 0..3), j = 0..7, at 8 r + j
+    // [32, 36): <G_i, f> for i = 4h + r;   [36, 40): <g, x_j> for j = 4h + r
+    float dots[BWD ? NDH : 1];
+#pragma unroll
+    for (int e = 0; e < (BWD ? NDH : 1); ++e) dots[e] = 0.0f;
+    for (int cc = 0; cc < nch; ++cc) {
+      const int s = cc % NS;
+      if (!tc::mbar_wait(full(s), (uint32_t)(cc / NS) & 1u, abort_flag, wait_ns)) {
+        give_up();
+        break;
+      }
+      const uint8_t* st = smem + s * CFG::STAGE;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {  // the two 8-channel halves of the chunk
+        float gv[8];
+        if constexpr (BWD) unpack8(ld32sw(st + CFG::GG_OFF, tok, c), gv);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          float xv[8];
+          unpack8(ld32sw(st + CFG::X_OFF + (4 * h + r) * XBOX, tok, c), xv);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            ss = fmaf(xv[e], xv[e], ss);
+            if constexpr (BWD) dots[36 + r] = fmaf(gv[e], xv[e], dots[36 + r]);
+          }
+        }
+        if constexpr (FULLB) {
+          float fv[8];
+          unpack8(ld32sw(st + CFG::F_OFF, tok, c), fv);
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            float Gv[8];
+            unpack8(ld32sw(st + CFG::G_OFF + (4 * h + r) * XBOX, tok, c), Gv);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) dots[32 + r] = fmaf(Gv[e], fv[e], dots[32 + r]);
+#pragma unroll
+            for (int j = 0; j < N; ++j) {
+              float xv[8];
+              unpack8(ld32sw(st + CFG::X_OFF + j * XBOX, tok, c), xv);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) dots[8 * r + j] = fmaf(Gv[e], xv[e], dots[8 * r + j]);
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(empty(s));
+    }
+
+    bool ok = !*abort_flag && tc::mbar_wait(done_bar, 0, abort_flag, wait_ns);
+    if (!ok && !*abort_flag) give_up();
+    ok = __all_sync(0xffffffffu, ok);  // the TMEM loads below are warp-collective
+    // stage memory is reused below: every math warp has finished reading it
+    nbar8(1, 256);
+    float* red_ss = reinterpret_cast<float*>(smem);   // [2][TM]
+    float* red_dt = red_ss + 2 * TM;                  // [2][NDH][TM]
+    float* dzs = red_dt + 2 * NDH * TM;               // [M + 3][TM]
+    float* ck = dzs + (M + 3) * TM;                   // checkpoints [nck][64][TM]
+    if (ok) {
+      red_ss[h * TM + tok] = ss;
+      if constexpr (BWD) {
+#pragma unroll
+        for (int e = 0; e < NDH; ++e) red_dt[(h * NDH + e) * TM + tok] = dots[e];
+      }
+    }
+    nbar8(1, 256);
+    if (ok && h == 0) {
+      // ------------------------------------------------- per-token epilogue
+      tc::tc_fence_after();
+      const int64_t t = t0 + tok;
+      const bool live = t < T;
+      const uint32_t lb = tmem + ((uint32_t)(32 * q) << 16);
+      float y[M];
+      {
+        float lo16[16], hi16[16];
+#pragma unroll
+        for (int b16 = 0; b16 < M / 16; ++b16) {
+          tc::tmem_ld16(lb + 16 * b16, hi16);
+          tc::tmem_ld16(lb + M + 16 * b16, lo16);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) y[16 * b16 + e] = hi16[e] + lo16[e];
+        }
+      }
+      const float r = sqrtf((red_ss[tok] + red_ss[TM + tok]) / (float)K + eps);
+      Alpha3 al;
+      al.load(alpha_p, ag);
+      float z[M];
+#pragma unroll
+      for (int m = 0; m < M; ++m) {
+        y[m] = y[m] / r;
+        z[m] = fmaf(al.at<N>(m), y[m], __ldg(bias + m));
+      }
+      if (live) {
+        bool bad = !isfinite(r);
+#pragma unroll
+        for (int m = 0; m < M; ++m) bad |= !isfinite(z[m]);
+        if (bad) flag_status(status, MHC_ERR_NONFINITE);
+      }
+      float spre[N], spost[N];
+#pragma unroll
+      for (int i = 0; i < N; ++i) {
+        spre[i] = sigmoidf_(z[i]);
+        spost[i] = sigmoidf_(z[N + i]);
+      }
+      float H[N * N];
+#pragma unroll
+      for (int e = 0; e < N * N; ++e) H[e] = z[2 * N + e];
+      if constexpr (!BWD) {
+        sk_forward<N>(H, iters);
+        if (live) {
+#pragma unroll
+          for (int i = 0; i < N; i += 4) {
+            *reinterpret_cast<float4*>(Hpre_o + t * N + i) =
+                make_float4(spre[i], spre[i + 1], spre[i + 2], spre[i + 3]);
+            *reinterpret_cast<float4*>(Hpost_o + t * N + i) = make_float4(
+                2.0f * spost[i], 2.0f * spost[i + 1], 2.0f * spost[i + 2], 2.0f * spost[i + 3]);
+          }
+#pragma unroll
+          for (int e = 0; e < N * N; e += 4)
+            *reinterpret_cast<float4*>(Hres_o + t * N * N + e) =
+                make_float4(H[e], H[e + 1], H[e + 2], H[e + 3]);
+        }
+      } else {
+        sk_forward_ckpt<N>(H, iters, ck + tok, TM, ck_period);
+        // dL/dH_res: <G_i, x_j> from the two stream halves, or the post half's
+        const float* rt = red_in + (live ? t : 0) * (N * N + N);
+        float dA[N * N];
+#pragma unroll
+        for (int i = 0; i < N; ++i)
+#pragma unroll
+          for (int j = 0; j < N; ++j)
+            dA[i * N + j] = SPLIT ? (live ? __ldg(rt + i * N + j) : 0.0f)
+                                  : red_dt[((i >> 2) * NDH + 8 * (i & 3) + j) * TM + tok];
+        float dzres[N * N];
+        sk_adjoint_ckpt<N>(dA, dzres, iters, ck + tok, TM, ck_period);
+        float dz[M];
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+          const float dpre = red_dt[((i >> 2) * NDH + 36 + (i & 3)) * TM + tok];
+          const float dpost = SPLIT ? (live ? __ldg(rt + N * N + i) : 0.0f)
+                                    : red_dt[((i >> 2) * NDH + 32 + (i & 3)) * TM + tok];
+          dz[i] = dpre * spre[i] * (1.0f - spre[i]);
+          dz[N + i] = dpost * 2.0f * spost[i] * (1.0f - spost[i]);
+        }
+#pragma unroll
+        for (int e = 0; e < N * N; ++e) dz[2 * N + e] = dzres[e];
+        float dzy[3] = {0.0f, 0.0f, 0.0f};  // dz . y over the pre, post, res logits
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+          const int g = m < N ? 0 : (m < 2 * N ? 1 : 2);
+          dzy[g] = fmaf(dz[m], y[m], dzy[g]);
+        }
+        if (live) {
+          // the per-token record of the n = 8 apply: H_res | H_pre | H_post | u | kappa
+          float* co = coef_o + t * CF::SIZE;
+#pragma unroll
+          for (int e = 0; e < N * N; ++e) co[CF::RES + e] = H[e];
+#pragma unroll
+          for (int i = 0; i < N; ++i) {
+            co[CF::PRE + i] = spre[i];
+            co[CF::POST + i] = 2.0f * spost[i];
+          }
+          float ar[3];
+#pragma unroll
+          for (int g = 0; g < 3; ++g) ar[g] = al.a[g] / r;
+#pragma unroll
+          for (int m = 0; m < M; ++m) co[CF::U + m] = ar[m < N ? 0 : (m < 2 * N ? 1 : 2)] * dz[m];
+          co[CF::KAPPA] =
+              fmaf(al.a[2], dzy[2], fmaf(al.a[1], dzy[1], al.a[0] * dzy[0])) / ((float)K * r * r);
+        }
+#pragma unroll
+        for (int m = 0; m < M; ++m) dzs[m * TM + tok] = live ? dz[m] : 0.0f;
+#pragma unroll
+        for (int g = 0; g < 3; ++g) dzs[(M + g) * TM + tok] = live ? dzy[g] : 0.0f;
+      }
+    }
+    if constexpr (BWD) {
+      nbar8(1, 256);
+      if (ok && h == 0 && tok < M + 3) {
+        // this tile's share of grad_b and the three grad_alpha sums, in token order
+        float a = 0.0f;
+        for (int k = 0; k < TM; ++k) a += dzs[tok * TM + k];
+        part_o[(int64_t)blockIdx.x * CF::DZ_SIZE + tok] = a;
+      }
+    }
+  }
+
+  __syncwarp();
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host
+namespace {
+// phi [K][80] fp32 -> phi^T split [160][K] bf16: rows 0..79 high parts, 80..159
+// the bf16 rounding of the remainder.
+__global__ void k_phi_split8(int64_t K, const float* __restrict__ phi,
+                             __nv_bfloat16* __restrict__ out) {
+  const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= K) return;
+#pragma unroll 4
+  for (int m = 0; m < tcm8::M; ++m) {
+    const float v = __ldg(phi + k * tcm8::M + m);
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+    out[(int64_t)m * K + k] = hi;
+    out[(int64_t)(tcm8::M + m) * K + k] = lo;
+  }
+}
+
+// Smallest checkpoint period whose checkpoints fit in the stage memory beside
+// the epilogue's reductions and dz sums.
+int map8_ck_period(int iters, size_t data_bytes) {
+  using namespace tcm8;
+  const size_t scratch = (size_t)(2 * TM + 2 * NDH * TM + (M + 3) * TM) * 4;
+  const size_t per_ck = (size_t)N * N * TM * 4;
+  const int max_ck = (int)((data_bytes - scratch) / per_ck);
+  const int steps = 2 * iters;
+  int P = 1;
+  while (steps / P + 1 > max_ck) ++P;
+  return P;
+}
+
+template <int MODE>
+cudaError_t launch_map8(const CUtensorMap& mx, const CUtensorMap& mp, const CUtensorMap& mG,
+                        const CUtensorMap& mg, const CUtensorMap& mf, int64_t T, int64_t C,
+                        int iters, float eps, const float* b, const float* alpha, int ag,
+                        float* Hpre, float* Hpost, float* Hres, float* coef, float* part,
+                        const float* red, int* st, int64_t wait_ns, cudaStream_t s) {
+  using namespace tcm8;
+  auto kern = k_map8_tc<MODE>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<MODE>::SMEM);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = (unsigned)((T + TM - 1) / TM);
+  const int P = map8_ck_period(iters, Cfg<MODE>::DATA);
+  kern<<<grid, NT, Cfg<MODE>::SMEM, s>>>(mx, mp, mG, mg, mf, T, C, iters, eps, P, b, alpha, ag,
+                                          Hpre, Hpost, Hres, coef, part, red, st,
+                                          tc::wait_limit(wait_ns));
+  return cudaGetLastError();
+}
+}  // namespace
+
+size_t map8_tc_phi_bytes(int64_t C) { return (size_t)tcm8::NL * tcm8::N * C * 2; }
+
+cudaError_t map8_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float eps, const void* x,
+                             const float* phi, void* phi_split, const float* b,
+                             const float* alpha, int ag, float* Hpre, float* Hpost, float* Hres,
+                             const void* G, const void* g, const void* f, const float* red,
+                             float* coef, float* part, int* st, int64_t wait_ns,
+                             cudaStream_t s) {
+  using namespace tcm8;
+  const int64_t K = (int64_t)N * C;
+  k_phi_split8<<<(unsigned)((K + 255) / 256), 256, 0, s>>>(K, phi, (__nv_bfloat16*)phi_split);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  CUtensorMap mx, mp, mG, mg, mf;
+  const CUtensorMapSwizzle SW = CU_TENSOR_MAP_SWIZZLE_32B;
+  const uint64_t dx[3] = {(uint64_t)C, (uint64_t)N, (uint64_t)T};
+  const uint64_t sx[2] = {(uint64_t)C * 2, (uint64_t)N * C * 2};
+  const uint32_t bx[3] = {CH, 1, TM};
+  e = make_tmap_bf16(&mx, x, 3, dx, sx, bx, SW);
+  if (e != cudaSuccess) return e;
+  const uint64_t dp[3] = {(uint64_t)C, (uint64_t)N, (uint64_t)NL};
+  const uint32_t bp[3] = {CH, 1, NL};
+  e = make_tmap_bf16(&mp, phi_split, 3, dp, sx, bp, SW);
+  if (e != cudaSuccess) return e;
+  // maps a mode does not read are copies of the x map (never dereferenced)
+  mG = mx;
+  mg = mx;
+  mf = mx;
+  const uint64_t d2[2] = {(uint64_t)C, (uint64_t)T};
+  const uint64_t s2[1] = {(uint64_t)C * 2};
+  const uint32_t b2[2] = {CH, TM};
+  if (mode != MAP_FWD) {
+    e = make_tmap_bf16(&mg, g, 2, d2, s2, b2, SW);
+    if (e != cudaSuccess) return e;
+  }
+  if (mode == MAP_BWD) {
+    e = make_tmap_bf16(&mG, G, 3, dx, sx, bx, SW);
+    if (e != cudaSuccess) return e;
+    e = make_tmap_bf16(&mf, f, 2, d2, s2, b2, SW);
+    if (e != cudaSuccess) return e;
+  }
+  switch (mode) {
+    case MAP_FWD:
+      return launch_map8<MAP_FWD>(mx, mp, mG, mg, mf, T, C, iters, eps, b, alpha, ag, Hpre, Hpost,
+                                  Hres, nullptr, nullptr, nullptr, st, wait_ns, s);
+    case MAP_BWD:
+      return launch_map8<MAP_BWD>(mx, mp, mG, mg, mf, T, C, iters, eps, b, alpha, ag, nullptr,
+                                  nullptr, nullptr, coef, part, nullptr, st, wait_ns, s);
+    case MAP_BWD_SPLIT:
+      return launch_map8<MAP_BWD_SPLIT>(mx, mp, mG, mg, mf, T, C, iters, eps, b, alpha, ag,
+                                        nullptr, nullptr, nullptr, coef, part, red, st, wait_ns, s);
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace mhc

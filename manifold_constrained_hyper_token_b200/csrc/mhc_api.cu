@@ -55,9 +55,12 @@ int dz_size(int n) {
   }
 }
 
-// bf16 activations with n = 4 take the tensor-core mapping kernel (128 tokens
-// per CTA); every other case the CUDA-core one (64 tokens per CTA).
+// bf16 activations with n = 4 take the tensor-core mapping and apply kernels
+// (128 tokens per mapping CTA); bf16 with n = 8 the tensor-core mapping (128
+// tokens per CTA) and the CUDA-core apply; every other case the CUDA-core
+// kernels (64 tokens per mapping CTA; n = 16 its own).
 bool use_tc(const mhc_params* p) { return p->dtype == MHC_DTYPE_BF16 && p->n == 4; }
+bool use_tc8(const mhc_params* p) { return p->dtype == MHC_DTYPE_BF16 && p->n == 8; }
 
 // Backward workspace.  CUDA-core path: per-token coefficient records, then one
 // partial-sum record (dz, dz . y) per 64-token mapping CTA.  Tensor-core path:
@@ -71,8 +74,9 @@ struct BwdWorkspace {
 
 BwdWorkspace bwd_layout(const mhc_params* p) {
   BwdWorkspace w{};
-  const bool tc = use_tc(p);
-  const int tokens_per_cta = tc ? 128 : (p->n == 16 ? mhc::wide_map_tokens_per_cta() : 64);
+  const bool tc = use_tc(p), tc8 = use_tc8(p);
+  const int tokens_per_cta =
+      (tc || tc8) ? 128 : (p->n == 16 ? mhc::wide_map_tokens_per_cta() : 64);
   w.nparts = (int)((p->T + tokens_per_cta - 1) / tokens_per_cta);
   size_t off = 0;
   if (tc) {
@@ -87,7 +91,8 @@ BwdWorkspace bwd_layout(const mhc_params* p) {
   w.part_off = off;
   off = round_up(off + (size_t)w.nparts * dz_size(p->n) * 4, 256);
   w.phi_off = off;
-  off = round_up(off + (tc ? mhc::map_tc_phi_bytes(p->C) : 0), 256);
+  off = round_up(off + (tc ? mhc::map_tc_phi_bytes(p->C) : (tc8 ? mhc::map8_tc_phi_bytes(p->C) : 0)),
+                 256);
   w.apply_off = off;
   off = round_up(off + (tc ? mhc::apply_tc_scratch_bytes(p->T, p->C) : 0), 256);
   w.kmap_off = off;
@@ -125,9 +130,10 @@ const char* mhc_status_string(int status) {
 size_t mhc_pre_workspace_size(const mhc_params* p) {
   if (check_params(p) != MHC_OK) return 0;
   // the bf16 split copy of phi, then the channel-split mapping's scratch
-  return use_tc(p) ? round_up(mhc::map_tc_phi_bytes(p->C), 256) +
-                         round_up(mhc::map_tc_scratch_bytes(p->T, p->C), 256)
-                   : 0;
+  if (use_tc(p))
+    return round_up(mhc::map_tc_phi_bytes(p->C), 256) +
+           round_up(mhc::map_tc_scratch_bytes(p->T, p->C), 256);
+  return use_tc8(p) ? round_up(mhc::map8_tc_phi_bytes(p->C), 256) : 0;
 }
 
 mhc_status mhc_pre(const mhc_params* p, const void* x, const float* phi, const float* b,
@@ -149,6 +155,14 @@ mhc_status mhc_pre(const mhc_params* p, const void* x, const float* phi, const f
                                         nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                                         ws + round_up(mhc::map_tc_phi_bytes(p->C), 256),
                                         dev_status, p->wait_ns, s));
+  } else if (use_tc8(p)) {
+    const size_t need = mhc_pre_workspace_size(p);
+    if (workspace == nullptr || workspace_bytes < need || ((uintptr_t)workspace & 255u) != 0)
+      return MHC_ERR_WORKSPACE;
+    st = from_cuda(mhc::map8_tc_dispatch(mhc::MAP_FWD, p->T, p->C, p->t_max, p->eps, x, phi,
+                                         workspace, b, alpha, alpha_groups(p), H_pre, H_post,
+                                         H_res, nullptr, nullptr, nullptr, nullptr, nullptr,
+                                         nullptr, dev_status, p->wait_ns, s));
   } else {
     st = from_cuda(mhc::map_fwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
                                          alpha, alpha_groups(p), H_pre, H_post, H_res, dev_status, s));
@@ -195,6 +209,13 @@ mhc_status mhc_backward_map(const mhc_params* p, const void* x, const float* phi
                                           ws + w.urec_off, (float*)(ws + w.hrec_off),
                                           (float*)(ws + w.part_off), ws + w.kmap_off, dev_status,
                                           p->wait_ns, (cudaStream_t)stream));
+  if (use_tc8(p))
+    return from_cuda(mhc::map8_tc_dispatch(mhc::MAP_BWD, p->T, p->C, p->t_max, p->eps, x, phi,
+                                           ws + w.phi_off, b, alpha, alpha_groups(p), nullptr,
+                                           nullptr, nullptr, grad_x_next, grad_h_in, f_out,
+                                           nullptr, (float*)(ws + w.coef_off),
+                                           (float*)(ws + w.part_off), dev_status, p->wait_ns,
+                                           (cudaStream_t)stream));
   return from_cuda(mhc::map_bwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
                                          alpha, alpha_groups(p), grad_x_next, grad_h_in, f_out, nullptr,
                                          (float*)(ws + w.coef_off), (float*)(ws + w.part_off),
@@ -274,9 +295,20 @@ mhc_status mhc_post_fused(const mhc_params* p, const void* x, const void* f_out,
         alpha_groups(p), x_next, H_pre_next, H_post_next, H_res_next,
         ws + round_up(mhc::map_tc_phi_bytes(p->C), 256), dev_status, p->wait_ns, s));
   }
-  // fp32 or n != 4: the post merge, then the mapping of x_next (both on the GPU)
+  // fp32 or n != 4: the post merge, then the mapping of x_next (both on the GPU),
+  // with the same mapping kernel mhc_pre runs
   st = from_cuda(mhc::post_dispatch(p->n, p->dtype, p->T, p->C, x, f_out, H_post, H_res, x_next, s));
   if (st != MHC_OK) return st;
+  if (use_tc8(p)) {
+    const size_t need = mhc_post_fused_workspace_size(p);
+    if (workspace == nullptr || workspace_bytes < need || ((uintptr_t)workspace & 255u) != 0)
+      return MHC_ERR_WORKSPACE;
+    return from_cuda(mhc::map8_tc_dispatch(mhc::MAP_FWD, p->T, p->C, p->t_max, p->eps, x_next,
+                                           phi_next, workspace, b_next, alpha_next,
+                                           alpha_groups(p), H_pre_next, H_post_next, H_res_next,
+                                           nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                                           dev_status, p->wait_ns, s));
+  }
   return from_cuda(mhc::map_fwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x_next,
                                          phi_next, b_next, alpha_next, alpha_groups(p), H_pre_next,
                                          H_post_next,
@@ -343,10 +375,17 @@ mhc_status mhc_pre_backward(const mhc_params* p, const void* x, const float* phi
                                             nullptr, grad_phi, grad_b, grad_alpha, alpha_groups(p),
                                             (void*)(ws + w.apply_off), dev_status, p->wait_ns, s));
   }
-  st = from_cuda(mhc::map_bwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
-                                       alpha, alpha_groups(p), nullptr, grad_h_in, nullptr, red,
-                                       (float*)(ws + w.coef_off), (float*)(ws + w.part_off),
-                                       dev_status, s));
+  if (use_tc8(p))
+    st = from_cuda(mhc::map8_tc_dispatch(mhc::MAP_BWD_SPLIT, p->T, p->C, p->t_max, p->eps, x,
+                                         phi, ws + w.phi_off, b, alpha, alpha_groups(p), nullptr,
+                                         nullptr, nullptr, nullptr, grad_h_in, nullptr, red,
+                                         (float*)(ws + w.coef_off), (float*)(ws + w.part_off),
+                                         dev_status, p->wait_ns, s));
+  else
+    st = from_cuda(mhc::map_bwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
+                                         alpha, alpha_groups(p), nullptr, grad_h_in, nullptr, red,
+                                         (float*)(ws + w.coef_off), (float*)(ws + w.part_off),
+                                         dev_status, s));
   if (st != MHC_OK) return st;
   return from_cuda(mhc::apply_dispatch(p->n, p->dtype, p->T, p->C, x, phi, grad_x_next, grad_h_in,
                                        (const float*)(ws + w.coef_off),

@@ -57,6 +57,18 @@ size_t map_tc_scratch_bytes(int64_t T, int64_t C);
 
 // phi [K][24] fp32 -> the bf16 split copy of phi^T [48][K] the mapping MMAs read
 cudaError_t phi_split_dispatch(int64_t K, const float* phi, void* phi_split, cudaStream_t s);
+// k_map8_tc.cu (bf16, n = 8: projection on the tensor cores); mode is MAP_FWD,
+// MAP_BWD or MAP_BWD_SPLIT.  Splits phi into phi_split (map8_tc_phi_bytes(C)
+// bytes); the backward modes write the CUDA-core apply's records (coef
+// [T][Coef<8>::SIZE]) and one partial-sum record per 128 tokens (part).
+cudaError_t map8_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float eps, const void* x,
+                             const float* phi, void* phi_split, const float* b,
+                             const float* alpha, int ag, float* Hpre, float* Hpost, float* Hres,
+                             const void* G, const void* g, const void* f, const float* red,
+                             float* coef, float* part, int* st, int64_t wait_ns,
+                             cudaStream_t s);
+size_t map8_tc_phi_bytes(int64_t C);
+
 // k_wide.cu (n = 16, CUDA cores); the mapping's mode is a MapMode
 int wide_map_tokens_per_cta();
 cudaError_t wide_map_dispatch(int mode, int dtype, int64_t T, int64_t C, int iters, float eps,

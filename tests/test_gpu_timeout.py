@@ -18,7 +18,7 @@ from conftest import assert_close
 pytestmark = pytest.mark.gpu
 
 TIMEOUT = 5
-TOL = 2e-2  # bf16 I/O (the tensor-core kernels run for bf16 with n = 4)
+TOL = 2e-2  # bf16 I/O (the tensor-core kernels run for bf16 with n = 4 and n = 8)
 
 
 @pytest.fixture(scope="module")
@@ -110,3 +110,36 @@ def test_fused_post_times_out_then_recovers(mhc, oracle_mod):
     assert int(st.item()) == 0
     ref_xn = oracle_mod.post(d["x"], d["f_out"], fwd["H_post"], fwd["H_res"])
     assert_close(_np(xn), ref_xn, TOL, "x_next")
+
+
+@pytest.mark.parametrize("phase", ["pre", "map"])
+def test_n8_mapping_times_out_then_recovers(mhc, oracle_mod, phase):
+    """The n = 8 tensor-core mapping (bf16) gives up the same way."""
+    from manifold_constrained_hyper_token_b200 import synth
+    T, n, C = 300, 8, 512
+    d = synth.layer_inputs(T, n, C, seed=17, dtype=torch.bfloat16, backward=True)
+    dd = {k: v.cuda() for k, v in d.items()}
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    if phase == "pre":
+        mhc.mhc_pre(dd["x"], dd["phi"], dd["b"], dd["alpha"], wait_ns=1, dev_status=st)
+    else:
+        ws = torch.empty(mhc.mhc_backward_workspace_size(n, T, C, torch.bfloat16),
+                         dtype=torch.uint8, device="cuda")
+        mhc.mhc_backward_map(dd["x"], dd["phi"], dd["b"], dd["alpha"], dd["f_out"],
+                             dd["grad_x_next"], dd["grad_h_in"], ws, wait_ns=1, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == TIMEOUT
+    st.zero_()
+    h_in, Hpre, Hpost, Hres = mhc.mhc_pre(dd["x"], dd["phi"], dd["b"], dd["alpha"], dev_status=st)
+    gx, gphi, gb, ga, gf = mhc.mhc_backward(dd["x"], dd["phi"], dd["b"], dd["alpha"], dd["f_out"],
+                                            dd["grad_x_next"], dd["grad_h_in"], dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    a = float(d["alpha"][0])
+    ref = oracle_mod.pre(d["x"], d["phi"], d["b"], a)
+    assert_close(_np(Hres), ref["H_res"], TOL, "H_res")
+    assert_close(_np(h_in), ref["h_in"], TOL, "h_in")
+    rb = oracle_mod.backward(d["x"], d["phi"], d["b"], a, d["f_out"], d["grad_x_next"],
+                             d["grad_h_in"])
+    assert_close(_np(gx), rb["grad_x"], TOL, "grad_x")
+    assert_close(_np(gphi), rb["grad_phi"], TOL, "grad_phi")
