@@ -22,7 +22,8 @@
 // <G_i, x_j> and <G_i, f_out> for i in 4h..4h+3 (all j) and <g, x_j> for j in
 // 4h..4h+3.  The h = 0 warps then run the per-token epilogue (gates,
 // Sinkhorn and its adjoint) with one thread per token and write the same
-// per-token records as the CUDA-core mapping, which the n = 8 apply reads.
+// per-token records as the CUDA-core mapping plus the U rows of the n = 8
+// tensor-core apply.
 // Every wait is bounded; on timeout the kernel records MHC_ERR_TIMEOUT,
 // drains what it issued, frees TMEM and returns.
 #include "mhc_common.cuh"
@@ -94,8 +95,8 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
     const __grid_constant__ CUtensorMap tm_f, int64_t T, int64_t C, int iters, float eps,
     int ck_period, const float* __restrict__ bias, const float* __restrict__ alpha_p, int ag,
     float* __restrict__ Hpre_o, float* __restrict__ Hpost_o, float* __restrict__ Hres_o,
-    float* __restrict__ coef_o, float* __restrict__ part_o, const float* __restrict__ red_in,
-    int* status, uint64_t wait_ns) {
+    float* __restrict__ coef_o, __nv_bfloat16* __restrict__ urec_o, float* __restrict__ part_o,
+    const float* __restrict__ red_in, int* status, uint64_t wait_ns) {
   using namespace tcm8;
   using CFG = Cfg<MODE>;
   using CF = Coef<N>;
@@ -386,6 +387,25 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
           for (int m = 0; m < M; ++m) co[CF::U + m] = ar[m < N ? 0 : (m < 2 * N ? 1 : 2)] * dz[m];
           co[CF::KAPPA] =
               fmaf(al.a[2], dzy[2], fmaf(al.a[1], dzy[1], al.a[0] * dzy[0])) / ((float)K * r * r);
+          // the MMA operand row: u to ~16 bits as bf16 high and low parts
+          uint4* ud = reinterpret_cast<uint4*>(urec_o + t * TcRec8::U_ELEMS);
+#pragma unroll
+          for (int v = 0; v < 12; ++v) {  // 8 u values per 16-byte vector, 10 of them used
+            uint32_t hw[4], lw[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+              const int m0 = 8 * v + 2 * p, m1 = m0 + 1;
+              const float u0 = m0 < M ? ar[m0 < N ? 0 : (m0 < 2 * N ? 1 : 2)] * dz[m0 < M ? m0 : 0] : 0.0f;
+              const float u1 = m1 < M ? ar[m1 < N ? 0 : (m1 < 2 * N ? 1 : 2)] * dz[m1 < M ? m1 : 0] : 0.0f;
+              const __nv_bfloat162 hi = __floats2bfloat162_rn(u0, u1);
+              const __nv_bfloat162 lo =
+                  __floats2bfloat162_rn(u0 - __low2float(hi), u1 - __high2float(hi));
+              hw[p] = *reinterpret_cast<const uint32_t*>(&hi);
+              lw[p] = *reinterpret_cast<const uint32_t*>(&lo);
+            }
+            ud[v] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            ud[TcRec8::LO / 8 + v] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+          }
         }
 #pragma unroll
         for (int m = 0; m < M; ++m) dzs[m * TM + tok] = live ? dz[m] : 0.0f;
@@ -448,8 +468,8 @@ template <int MODE>
 cudaError_t launch_map8(const CUtensorMap& mx, const CUtensorMap& mp, const CUtensorMap& mG,
                         const CUtensorMap& mg, const CUtensorMap& mf, int64_t T, int64_t C,
                         int iters, float eps, const float* b, const float* alpha, int ag,
-                        float* Hpre, float* Hpost, float* Hres, float* coef, float* part,
-                        const float* red, int* st, int64_t wait_ns, cudaStream_t s) {
+                        float* Hpre, float* Hpost, float* Hres, float* coef, void* urec,
+                        float* part, const float* red, int* st, int64_t wait_ns, cudaStream_t s) {
   using namespace tcm8;
   auto kern = k_map8_tc<MODE>;
   cudaError_t e =
@@ -458,8 +478,8 @@ cudaError_t launch_map8(const CUtensorMap& mx, const CUtensorMap& mp, const CUte
   const unsigned grid = (unsigned)((T + TM - 1) / TM);
   const int P = map8_ck_period(iters, Cfg<MODE>::DATA);
   kern<<<grid, NT, Cfg<MODE>::SMEM, s>>>(mx, mp, mG, mg, mf, T, C, iters, eps, P, b, alpha, ag,
-                                          Hpre, Hpost, Hres, coef, part, red, st,
-                                          tc::wait_limit(wait_ns));
+                                          Hpre, Hpost, Hres, coef, (__nv_bfloat16*)urec, part,
+                                          red, st, tc::wait_limit(wait_ns));
   return cudaGetLastError();
 }
 }  // namespace
@@ -470,7 +490,7 @@ cudaError_t map8_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float ep
                              const float* phi, void* phi_split, const float* b,
                              const float* alpha, int ag, float* Hpre, float* Hpost, float* Hres,
                              const void* G, const void* g, const void* f, const float* red,
-                             float* coef, float* part, int* st, int64_t wait_ns,
+                             float* coef, void* urec, float* part, int* st, int64_t wait_ns,
                              cudaStream_t s) {
   using namespace tcm8;
   const int64_t K = (int64_t)N * C;
@@ -508,13 +528,14 @@ cudaError_t map8_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float ep
   switch (mode) {
     case MAP_FWD:
       return launch_map8<MAP_FWD>(mx, mp, mG, mg, mf, T, C, iters, eps, b, alpha, ag, Hpre, Hpost,
-                                  Hres, nullptr, nullptr, nullptr, st, wait_ns, s);
+                                  Hres, nullptr, nullptr, nullptr, nullptr, st, wait_ns, s);
     case MAP_BWD:
       return launch_map8<MAP_BWD>(mx, mp, mG, mg, mf, T, C, iters, eps, b, alpha, ag, nullptr,
-                                  nullptr, nullptr, coef, part, nullptr, st, wait_ns, s);
+                                  nullptr, nullptr, coef, urec, part, nullptr, st, wait_ns, s);
     case MAP_BWD_SPLIT:
       return launch_map8<MAP_BWD_SPLIT>(mx, mp, mG, mg, mf, T, C, iters, eps, b, alpha, ag,
-                                        nullptr, nullptr, nullptr, coef, part, red, st, wait_ns, s);
+                                        nullptr, nullptr, nullptr, coef, urec, part, red, st,
+                                        wait_ns, s);
     default:
       return cudaErrorInvalidValue;
   }

@@ -15,6 +15,18 @@
 
 namespace mhc {
 
+// Reciprocal of a row or column sum by the approximate reciprocal instruction
+// (about one float32 ulp of error; subnormal inputs are not flushed).  The
+// correctly rounded division it replaces costs about as many instructions as
+// the rest of a normalisation; the standalone estimate is checked against the
+// fp64 oracle at 1e-5.  (The layer kernels keep the rounded division: their
+// forward and adjoint recompute the same iterates.)
+__device__ __forceinline__ float rcp_approx(float v) {
+  float r;
+  asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(v));
+  return r;
+}
+
 template <int N, int BR>
 __global__ void __launch_bounds__(256) k_sinkhorn(int iters, int64_t B, const float* __restrict__ logits,
                                                   float* __restrict__ out, int* status) {
@@ -73,7 +85,7 @@ __global__ void __launch_bounds__(256) k_sinkhorn(int iters, int64_t B, const fl
       for (int j = 0; j < BR; ++j) s += A[i][j];
 #pragma unroll
       for (int d = 1; d < NB; d <<= 1) s += __shfl_xor_sync(0xffffffffu, s, d);
-      const float inv = 1.0f / s;
+      const float inv = rcp_approx(s);
 #pragma unroll
       for (int j = 0; j < BR; ++j) A[i][j] *= inv;
     }
@@ -85,7 +97,7 @@ __global__ void __launch_bounds__(256) k_sinkhorn(int iters, int64_t B, const fl
       for (int i = 0; i < BR; ++i) s += A[i][j];
 #pragma unroll
       for (int d = NB; d < G; d <<= 1) s += __shfl_xor_sync(0xffffffffu, s, d);
-      const float inv = 1.0f / s;
+      const float inv = rcp_approx(s);
 #pragma unroll
       for (int i = 0; i < BR; ++i) A[i][j] *= inv;
     }

@@ -55,18 +55,19 @@ int dz_size(int n) {
   }
 }
 
-// bf16 activations with n = 4 take the tensor-core mapping and apply kernels
-// (128 tokens per mapping CTA); bf16 with n = 8 the tensor-core mapping (128
-// tokens per CTA) and the CUDA-core apply; every other case the CUDA-core
-// kernels (64 tokens per mapping CTA; n = 16 its own).
+// bf16 activations with n = 4 or n = 8 take the tensor-core mapping and apply
+// kernels (128 tokens per mapping CTA); every other case the CUDA-core kernels
+// (64 tokens per mapping CTA; n = 16 its own).
 bool use_tc(const mhc_params* p) { return p->dtype == MHC_DTYPE_BF16 && p->n == 4; }
 bool use_tc8(const mhc_params* p) { return p->dtype == MHC_DTYPE_BF16 && p->n == 8; }
 
 // Backward workspace.  CUDA-core path: per-token coefficient records, then one
-// partial-sum record (dz, dz . y) per 64-token mapping CTA.  Tensor-core path:
-// per-token U rows (bf16) and H records, the partial sums per 128-token CTA,
-// the bf16 split copy of phi^T that the mapping MMA reads, and the apply
-// kernel's grad_phi partials and slice counters.
+// partial-sum record (dz, dz . y) per 64-token mapping CTA.  Tensor-core path
+// (n = 4): per-token U rows (bf16) and H records, the partial sums per
+// 128-token CTA, the bf16 split copy of phi^T that the mapping MMA reads, and
+// the apply kernel's grad_phi partials and slice counters.  Tensor-core path
+// (n = 8): the coefficient records and the U rows, the partial sums, the phi
+// split copy, and the fp32 phi u scratch [T][8][C] of the apply.
 struct BwdWorkspace {
   size_t coef_off, urec_off, hrec_off, part_off, phi_off, apply_off, kmap_off, total;
   int nparts;
@@ -87,6 +88,10 @@ BwdWorkspace bwd_layout(const mhc_params* p) {
   } else {
     w.coef_off = off;
     off = round_up(off + (size_t)p->T * coef_size(p->n) * 4, 256);
+    if (tc8) {
+      w.urec_off = off;
+      off = round_up(off + (size_t)p->T * mhc::TcRec8::U_BYTES, 256);
+    }
   }
   w.part_off = off;
   off = round_up(off + (size_t)w.nparts * dz_size(p->n) * 4, 256);
@@ -94,7 +99,9 @@ BwdWorkspace bwd_layout(const mhc_params* p) {
   off = round_up(off + (tc ? mhc::map_tc_phi_bytes(p->C) : (tc8 ? mhc::map8_tc_phi_bytes(p->C) : 0)),
                  256);
   w.apply_off = off;
-  off = round_up(off + (tc ? mhc::apply_tc_scratch_bytes(p->T, p->C) : 0), 256);
+  off = round_up(off + (tc ? mhc::apply_tc_scratch_bytes(p->T, p->C)
+                           : (tc8 ? (size_t)p->T * 8 * p->C * 4 : 0)),
+                 256);
   w.kmap_off = off;
   off = round_up(off + (tc ? mhc::map_tc_scratch_bytes(p->T, p->C) : 0), 256);
   w.total = off;
@@ -162,7 +169,7 @@ mhc_status mhc_pre(const mhc_params* p, const void* x, const float* phi, const f
     st = from_cuda(mhc::map8_tc_dispatch(mhc::MAP_FWD, p->T, p->C, p->t_max, p->eps, x, phi,
                                          workspace, b, alpha, alpha_groups(p), H_pre, H_post,
                                          H_res, nullptr, nullptr, nullptr, nullptr, nullptr,
-                                         nullptr, dev_status, p->wait_ns, s));
+                                         nullptr, nullptr, dev_status, p->wait_ns, s));
   } else {
     st = from_cuda(mhc::map_fwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
                                          alpha, alpha_groups(p), H_pre, H_post, H_res, dev_status, s));
@@ -213,7 +220,7 @@ mhc_status mhc_backward_map(const mhc_params* p, const void* x, const float* phi
     return from_cuda(mhc::map8_tc_dispatch(mhc::MAP_BWD, p->T, p->C, p->t_max, p->eps, x, phi,
                                            ws + w.phi_off, b, alpha, alpha_groups(p), nullptr,
                                            nullptr, nullptr, grad_x_next, grad_h_in, f_out,
-                                           nullptr, (float*)(ws + w.coef_off),
+                                           nullptr, (float*)(ws + w.coef_off), ws + w.urec_off,
                                            (float*)(ws + w.part_off), dev_status, p->wait_ns,
                                            (cudaStream_t)stream));
   return from_cuda(mhc::map_bwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
@@ -245,6 +252,12 @@ mhc_status mhc_backward_apply(const mhc_params* p, const void* x, const float* p
                                             grad_f_out, grad_phi, grad_b, grad_alpha,
                                             alpha_groups(p), (void*)(ws + w.apply_off), dev_status,
                                             p->wait_ns, (cudaStream_t)stream));
+  if (use_tc8(p))
+    return from_cuda(mhc::apply8_tc_dispatch(
+        p->T, p->C, x, ws + w.phi_off, grad_x_next, grad_h_in, (const float*)(ws + w.coef_off),
+        ws + w.urec_off, (const float*)(ws + w.part_off), w.nparts, (float*)(ws + w.apply_off),
+        grad_x, grad_f_out, grad_phi, grad_b, grad_alpha, alpha_groups(p), dev_status, p->wait_ns,
+        (cudaStream_t)stream));
   return from_cuda(mhc::apply_dispatch(p->n, p->dtype, p->T, p->C, x, phi, grad_x_next, grad_h_in,
                                        (const float*)(ws + w.coef_off),
                                        (const float*)(ws + w.part_off), w.nparts, grad_x,
@@ -307,7 +320,7 @@ mhc_status mhc_post_fused(const mhc_params* p, const void* x, const void* f_out,
                                            phi_next, workspace, b_next, alpha_next,
                                            alpha_groups(p), H_pre_next, H_post_next, H_res_next,
                                            nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
-                                           dev_status, p->wait_ns, s));
+                                           nullptr, dev_status, p->wait_ns, s));
   }
   return from_cuda(mhc::map_fwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x_next,
                                          phi_next, b_next, alpha_next, alpha_groups(p), H_pre_next,
@@ -375,14 +388,19 @@ mhc_status mhc_pre_backward(const mhc_params* p, const void* x, const float* phi
                                             nullptr, grad_phi, grad_b, grad_alpha, alpha_groups(p),
                                             (void*)(ws + w.apply_off), dev_status, p->wait_ns, s));
   }
-  if (use_tc8(p))
+  if (use_tc8(p)) {
     st = from_cuda(mhc::map8_tc_dispatch(mhc::MAP_BWD_SPLIT, p->T, p->C, p->t_max, p->eps, x,
                                          phi, ws + w.phi_off, b, alpha, alpha_groups(p), nullptr,
                                          nullptr, nullptr, nullptr, grad_h_in, nullptr, red,
-                                         (float*)(ws + w.coef_off), (float*)(ws + w.part_off),
-                                         dev_status, p->wait_ns, s));
-  else
-    st = from_cuda(mhc::map_bwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
+                                         (float*)(ws + w.coef_off), ws + w.urec_off,
+                                         (float*)(ws + w.part_off), dev_status, p->wait_ns, s));
+    if (st != MHC_OK) return st;
+    return from_cuda(mhc::apply8_tc_dispatch(
+        p->T, p->C, x, ws + w.phi_off, grad_x_next, grad_h_in, (const float*)(ws + w.coef_off),
+        ws + w.urec_off, (const float*)(ws + w.part_off), w.nparts, (float*)(ws + w.apply_off),
+        grad_x, nullptr, grad_phi, grad_b, grad_alpha, alpha_groups(p), dev_status, p->wait_ns, s));
+  }
+  st = from_cuda(mhc::map_bwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
                                          alpha, alpha_groups(p), nullptr, grad_h_in, nullptr, red,
                                          (float*)(ws + w.coef_off), (float*)(ws + w.part_off),
                                          dev_status, s));

@@ -285,4 +285,13 @@ struct TcRec {
   static constexpr int H_RES = 0, H_PRE = 16, H_POST = 20, H_KAPPA = 24;
 };
 
+// The U row of the n = 8 tensor-core backward (written by the n = 8 mapping,
+// read by the phi u and grad_phi MMAs): [192] bf16 = u_hi (80) | 0 (16) |
+// u_lo (80) | 0 (16), three 64-element swizzle atoms, 384 bytes.
+struct TcRec8 {
+  static constexpr int U_ELEMS = 192;
+  static constexpr int U_BYTES = U_ELEMS * 2;
+  static constexpr int LO = 96;  // first column of u_lo
+};
+
 }  // namespace mhc

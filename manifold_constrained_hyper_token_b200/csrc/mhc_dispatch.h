@@ -59,14 +59,24 @@ size_t map_tc_scratch_bytes(int64_t T, int64_t C);
 cudaError_t phi_split_dispatch(int64_t K, const float* phi, void* phi_split, cudaStream_t s);
 // k_map8_tc.cu (bf16, n = 8: projection on the tensor cores); mode is MAP_FWD,
 // MAP_BWD or MAP_BWD_SPLIT.  Splits phi into phi_split (map8_tc_phi_bytes(C)
-// bytes); the backward modes write the CUDA-core apply's records (coef
-// [T][Coef<8>::SIZE]) and one partial-sum record per 128 tokens (part).
+// bytes); the backward modes write the per-token records (coef
+// [T][Coef<8>::SIZE]), the U rows (urec [T][TcRec8::U_ELEMS] bf16) and one
+// partial-sum record per 128 tokens (part).
 cudaError_t map8_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float eps, const void* x,
                              const float* phi, void* phi_split, const float* b,
                              const float* alpha, int ag, float* Hpre, float* Hpost, float* Hres,
                              const void* G, const void* g, const void* f, const float* red,
-                             float* coef, float* part, int* st, int64_t wait_ns,
+                             float* coef, void* urec, float* part, int* st, int64_t wait_ns,
                              cudaStream_t s);
+// k_apply8_tc.cu (bf16, n = 8): the apply as phi u on the tensor cores into
+// phiu (fp32 [T][8][C] scratch), grad_x / grad_f_out on the CUDA cores, and
+// grad_phi as a tensor-core contraction over the tokens; phi_split is the
+// mapping's bf16 split copy of phi^T.  gf == nullptr skips grad_f_out.
+cudaError_t apply8_tc_dispatch(int64_t T, int64_t C, const void* x, const void* phi_split,
+                               const void* G, const void* g, const float* coef, const void* urec,
+                               const float* part, int nparts, float* phiu, void* gx, void* gf,
+                               float* gphi, float* gb, float* ga, int ag, int* st,
+                               int64_t wait_ns, cudaStream_t s);
 size_t map8_tc_phi_bytes(int64_t C);
 
 // k_wide.cu (n = 16, CUDA cores); the mapping's mode is a MapMode
