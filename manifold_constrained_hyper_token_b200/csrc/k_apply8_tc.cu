@@ -44,10 +44,13 @@ constexpr int NU = TcRec8::U_ELEMS;     // 192
 constexpr int ATOM = 128 * 128;         // [128 rows][64 bf16] with the 128-byte swizzle: 16 KB
 // k_phiu8
 constexpr int KB = 256;                 // channels of one stream per item (MMA N)
-constexpr int PATOM = M * 128;          // [80 phi^T rows][64 channels]: 10 KB
+constexpr int CH = 16;                  // channels per block of the tiled phi^T copy
+constexpr int NL = 2 * M;               // rows per block (80 high, 80 low)
+constexpr int PHB = M * CH * 2;         // the 80 high rows of one block: 2.5 KB
 constexpr int A_U_OFF = 0;              // U tile: three atoms (48 KB)
-constexpr int A_P_OFF = 3 * ATOM;       // phi tile: four atoms (40 KB)
-constexpr int A_DATA = A_P_OFF + 4 * PATOM;
+constexpr int A_P_OFF = 3 * ATOM;       // phi tile: KB / CH blocks of high rows (40 KB)
+constexpr int A_DATA = A_P_OFF + (KB / CH) * PHB;
+constexpr int XT = 36;                  // row stride (floats) of the epilogue's transpose buffer
 constexpr int A_SMEM = A_DATA + 1024 + 64;
 constexpr int A_NT = 128;
 constexpr uint32_t A_TMEM = 256;
@@ -88,7 +91,7 @@ __device__ __forceinline__ uint4 pack8b(const float (&v)[8]) {
 
 // ------------------------------------------------------------------ phi u
 __global__ void __launch_bounds__(ap8::A_NT) k_phiu8(const __grid_constant__ CUtensorMap tm_u,
-                                                     const __grid_constant__ CUtensorMap tm_phi,
+                                                     const __nv_bfloat16* __restrict__ phi_t,
                                                      int64_t T, int64_t C, int ncb,
                                                      float* __restrict__ phiu, int* status,
                                                      uint64_t wait_ns) {
@@ -122,12 +125,17 @@ __global__ void __launch_bounds__(ap8::A_NT) k_phiu8(const __grid_constant__ CUt
 
   if (threadIdx.x == 0) {
     const uint64_t pol = tc::policy_evict_last();  // U and phi are read by many CTAs
-    tc::mbar_arrive_expect_tx(full, (uint32_t)A_DATA);
+    // phi: the high rows of the KB / CH channel blocks of stream j (blocks past
+    // the last channel are not loaded; the columns they feed are not stored)
+    const int64_t nblk = (C + CH - 1) / CH;
+    const int64_t q0 = (int64_t)c0 / CH;
+    const int nb = (int)(nblk - q0 < KB / CH ? nblk - q0 : KB / CH);
+    tc::mbar_arrive_expect_tx(full, (uint32_t)(3 * ATOM + nb * PHB));
     for (int a = 0; a < 3; ++a)
       tc::tma_load_2d(tc::smem_u32(smem + A_U_OFF + a * ATOM), &tm_u, full, 64 * a, (int)t0, pol);
-    for (int a = 0; a < 4; ++a)
-      tc::tma_load_3d(tc::smem_u32(smem + A_P_OFF + a * PATOM), &tm_phi, full, c0 + 64 * a, j, 0,
-                      pol);
+    for (int q = 0; q < nb; ++q)
+      tc::bulk_load(tc::smem_u32(smem + A_P_OFF + q * PHB), phi_t + ((q0 + q) * N + j) * (NL * CH),
+                    PHB, full, pol);
   }
   bool ok = true;
   if (warp == 1 && lane == 0) {
@@ -136,7 +144,8 @@ __global__ void __launch_bounds__(ap8::A_NT) k_phiu8(const __grid_constant__ CUt
       tc::tc_fence_after();
       // D[tok][k] = sum over m' of U[tok][m'] PHI[m'][k]: K-steps 0..4 take u_hi
       // against phi rows 0..79, steps 6..10 u_lo against the same rows; steps 5
-      // and 11 would only multiply U's zero padding
+      // and 11 would only multiply U's zero padding.  PHI is MN-major with the
+      // 32-byte swizzle: 16-channel atoms PHB bytes apart, 8-row groups 256 apart.
       constexpr uint32_t idesc = tc::idesc_bf16(TT, KB, false, true);
       const uint32_t ub = tc::smem_u32(smem + A_U_OFF), pb = tc::smem_u32(smem + A_P_OFF);
       int issued = 0;
@@ -145,7 +154,7 @@ __global__ void __launch_bounds__(ap8::A_NT) k_phiu8(const __grid_constant__ CUt
         if (s == 5 || s == 11) continue;
         const int r = s < 5 ? s : s - 6;  // 16-row block of phi^T
         const uint64_t da = tc::smem_desc(ub + (s / 4) * ATOM + (s % 4) * 32, 16, 1024, tc::SWZ_128B);
-        const uint64_t db = tc::smem_desc(pb + r * 16 * 128, PATOM, 1024, tc::SWZ_128B);
+        const uint64_t db = tc::smem_desc(pb + r * 16 * 32, PHB, 256, tc::SWZ_32B);
         tc::mma_bf16(tmem, da, db, idesc, issued > 0 ? 1u : 0u);
         ++issued;
       }
@@ -162,22 +171,36 @@ __global__ void __launch_bounds__(ap8::A_NT) k_phiu8(const __grid_constant__ CUt
   if (okall && !done) flag_status(status, MHC_ERR_TIMEOUT);
   done = __all_sync(0xffffffffu, done);
   if (done) {
+    // each warp turns its 32 token rows x 32 columns around in shared memory (the
+    // U tile, free once the MMAs are done), so that 8 lanes store one token's
+    // 128 contiguous bytes
     tc::tc_fence_after();
-    const int64_t t = t0 + 32 * warp + lane;
-    float* dst = phiu + (t * N + j) * C + c0;
+    float* xt = reinterpret_cast<float*>(smem + A_U_OFF) + warp * 32 * XT;
     const uint32_t lb = tmem + ((uint32_t)(32 * warp) << 16);
+    const int rr = lane >> 3, cq = lane & 7;
 #pragma unroll 1
-    for (int q = 0; q < KB / 16; ++q) {
-      float v[16];
-      tc::tmem_ld16(lb + 16 * q, v);
+    for (int q = 0; q < KB / 32; ++q) {
+      float v0[16], v1[16];
+      tc::tmem_ld16(lb + 32 * q, v0);
+      tc::tmem_ld16(lb + 32 * q + 16, v1);
       tc::tmem_ld_wait();
-      if (t < T) {
 #pragma unroll
-        for (int e = 0; e < 16; e += 4)
-          if (c0 + 16 * q + e < C)
-            __stcg(reinterpret_cast<float4*>(dst + 16 * q + e),
-                   make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]));
+      for (int e = 0; e < 4; ++e) {
+        *reinterpret_cast<float4*>(xt + lane * XT + 4 * e) =
+            make_float4(v0[4 * e], v0[4 * e + 1], v0[4 * e + 2], v0[4 * e + 3]);
+        *reinterpret_cast<float4*>(xt + lane * XT + 16 + 4 * e) =
+            make_float4(v1[4 * e], v1[4 * e + 1], v1[4 * e + 2], v1[4 * e + 3]);
       }
+      __syncwarp();
+      const int64_t c = (int64_t)c0 + 32 * q + 4 * cq;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = 4 * i + rr;
+        const int64_t t = t0 + 32 * warp + r;
+        const float4 val = *reinterpret_cast<const float4*>(xt + r * XT + 4 * cq);
+        if (t < T && c < C) __stcg(reinterpret_cast<float4*>(phiu + (t * N + j) * C + c), val);
+      }
+      __syncwarp();
     }
   }
   tc::tc_fence_before();
@@ -408,21 +431,16 @@ cudaError_t apply8_tc_dispatch(int64_t T, int64_t C, const void* x, const void* 
                                int64_t wait_ns, cudaStream_t s) {
   using namespace ap8;
   const uint64_t wl = tc::wait_limit(wait_ns);
-  CUtensorMap mu, mp, mx;
+  CUtensorMap mu, mx;
   // U rows [T][192] bf16, boxes of 64 columns x 128 tokens
   const uint64_t du[2] = {(uint64_t)NU, (uint64_t)T};
   const uint64_t su[1] = {(uint64_t)NU * 2};
   const uint32_t bu[2] = {64, TT};
   cudaError_t e = make_tmap_bf16(&mu, urec, 2, du, su, bu, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
-  // phi^T split [160][8][C] bf16: the 80 high rows, 64 channels of one stream
-  const uint64_t dp[3] = {(uint64_t)C, (uint64_t)N, (uint64_t)(2 * M)};
-  const uint64_t sx[2] = {(uint64_t)C * 2, (uint64_t)N * C * 2};
-  const uint32_t bp[3] = {64, 1, (uint32_t)M};
-  e = make_tmap_bf16(&mp, phi_split, 3, dp, sx, bp, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (e != cudaSuccess) return e;
   // x [T][8][C] bf16: 64 channels of one stream x 128 tokens
   const uint64_t dx[3] = {(uint64_t)C, (uint64_t)N, (uint64_t)T};
+  const uint64_t sx[2] = {(uint64_t)C * 2, (uint64_t)N * C * 2};
   const uint32_t bx[3] = {64, 1, TT};
   e = make_tmap_bf16(&mx, x, 3, dx, sx, bx, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
@@ -431,7 +449,7 @@ cudaError_t apply8_tc_dispatch(int64_t T, int64_t C, const void* x, const void* 
   const int ncb_a = (int)((C + KB - 1) / KB);
   e = cudaFuncSetAttribute(k_phiu8, cudaFuncAttributeMaxDynamicSharedMemorySize, A_SMEM);
   if (e != cudaSuccess) return e;
-  k_phiu8<<<(unsigned)((int64_t)ntt * N * ncb_a), A_NT, A_SMEM, s>>>(mu, mp, T, C, ncb_a, phiu, st,
+  k_phiu8<<<(unsigned)((int64_t)ntt * N * ncb_a), A_NT, A_SMEM, s>>>(mu, (const __nv_bfloat16*)phi_split, T, C, ncb_a, phiu, st,
                                                                     wl);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

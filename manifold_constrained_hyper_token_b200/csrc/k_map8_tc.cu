@@ -90,7 +90,7 @@ __device__ __forceinline__ void nbar8(int id, int count) {
 
 template <int MODE>
 __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
-    const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_phi,
+    const __grid_constant__ CUtensorMap tm_x, const __nv_bfloat16* __restrict__ phi_t,
     const __grid_constant__ CUtensorMap tm_G, const __grid_constant__ CUtensorMap tm_g,
     const __grid_constant__ CUtensorMap tm_f, int64_t T, int64_t C, int iters, float eps,
     int ck_period, const float* __restrict__ bias, const float* __restrict__ alpha_p, int ag,
@@ -131,7 +131,6 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
   }
   if (warp == 0 && lane == 0) {
     tc::tma_prefetch_desc(&tm_x);
-    tc::tma_prefetch_desc(&tm_phi);
     if constexpr (BWD) tc::tma_prefetch_desc(&tm_g);
     if constexpr (FULLB) {
       tc::tma_prefetch_desc(&tm_G);
@@ -168,9 +167,12 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
         const uint32_t base = tc::smem_u32(smem + s * CFG::STAGE);
         tc::mbar_arrive_expect_tx(full(s), CFG::STAGE);
         const int c0 = cc * CH;
+        // the chunk's phi^T tiles of all eight streams: one contiguous 40 KB block
+        // of the tiled copy, already in the 32-byte swizzled shared-memory order
+        tc::bulk_load(base + CFG::P_OFF, phi_t + (int64_t)cc * (N * NL * CH), N * PBOX, full(s),
+                      pol_keep);
         for (int i = 0; i < N; ++i) {
           tc::tma_load_3d(base + CFG::X_OFF + i * XBOX, &tm_x, full(s), c0, i, (int)t0, pol_stream);
-          tc::tma_load_3d(base + CFG::P_OFF + i * PBOX, &tm_phi, full(s), c0, i, 0, pol_keep);
           if constexpr (FULLB)
             tc::tma_load_3d(base + CFG::G_OFF + i * XBOX, &tm_G, full(s), c0, i, (int)t0, pol_stream);
         }
@@ -435,19 +437,30 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
 
 // ------------------------------------------------------------------ host
 namespace {
-// phi [K][80] fp32 -> phi^T split [160][K] bf16: rows 0..79 high parts, 80..159
-// the bf16 rounding of the remainder.
-__global__ void k_phi_split8(int64_t K, const float* __restrict__ phi,
+// phi [K][80] fp32 (k = j*C + c) -> the tiled bf16 split of phi^T the mapping
+// and apply MMAs read: block (chunk q of 16 channels, stream j) holds the 160
+// rows m (0..79 the high parts, 80..159 the bf16 rounding of the remainder) of
+// 16 channels, 32 bytes per row, with the two 16-byte halves of rows whose bit
+// 2 is set swapped -- the 32-byte swizzle of a 256-byte-aligned tile, so one
+// bulk copy of a block (or of the 8 blocks of a chunk) lands in shared memory
+// ready for the MMA.  Channels c >= C of the last chunk are zero.
+__global__ void k_phi_split8(int64_t C, int64_t ncp, const float* __restrict__ phi,
                              __nv_bfloat16* __restrict__ out) {
-  const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (k >= K) return;
+  using namespace tcm8;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // j * ncp + c
+  if (idx >= (int64_t)N * ncp) return;
+  const int64_t j = idx / ncp, c = idx % ncp;
+  const int64_t q = c / CH;
+  const int ci = (int)(c % CH), h = ci >> 3, e = ci & 7;
+  __nv_bfloat16* blk = out + (q * N + j) * (NL * CH);
 #pragma unroll 4
-  for (int m = 0; m < tcm8::M; ++m) {
-    const float v = __ldg(phi + k * tcm8::M + m);
+  for (int m = 0; m < M; ++m) {
+    const float v = c < C ? __ldg(phi + (j * C + c) * M + m) : 0.0f;
     const __nv_bfloat16 hi = __float2bfloat16_rn(v);
     const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
-    out[(int64_t)m * K + k] = hi;
-    out[(int64_t)(tcm8::M + m) * K + k] = lo;
+    const int m2 = M + m;
+    blk[m * CH + ((h ^ ((m >> 2) & 1)) << 3) + e] = hi;
+    blk[m2 * CH + ((h ^ ((m2 >> 2) & 1)) << 3) + e] = lo;
   }
 }
 
@@ -465,7 +478,7 @@ int map8_ck_period(int iters, size_t data_bytes) {
 }
 
 template <int MODE>
-cudaError_t launch_map8(const CUtensorMap& mx, const CUtensorMap& mp, const CUtensorMap& mG,
+cudaError_t launch_map8(const CUtensorMap& mx, const void* phi_t, const CUtensorMap& mG,
                         const CUtensorMap& mg, const CUtensorMap& mf, int64_t T, int64_t C,
                         int iters, float eps, const float* b, const float* alpha, int ag,
                         float* Hpre, float* Hpost, float* Hres, float* coef, void* urec,
@@ -477,14 +490,17 @@ cudaError_t launch_map8(const CUtensorMap& mx, const CUtensorMap& mp, const CUte
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)((T + TM - 1) / TM);
   const int P = map8_ck_period(iters, Cfg<MODE>::DATA);
-  kern<<<grid, NT, Cfg<MODE>::SMEM, s>>>(mx, mp, mG, mg, mf, T, C, iters, eps, P, b, alpha, ag,
+  kern<<<grid, NT, Cfg<MODE>::SMEM, s>>>(mx, (const __nv_bfloat16*)phi_t, mG, mg, mf, T, C, iters, eps, P, b, alpha, ag,
                                           Hpre, Hpost, Hres, coef, (__nv_bfloat16*)urec, part,
                                           red, st, tc::wait_limit(wait_ns));
   return cudaGetLastError();
 }
 }  // namespace
 
-size_t map8_tc_phi_bytes(int64_t C) { return (size_t)tcm8::NL * tcm8::N * C * 2; }
+size_t map8_tc_phi_bytes(int64_t C) {
+  const int64_t nch = (C + tcm8::CH - 1) / tcm8::CH;
+  return (size_t)nch * tcm8::N * tcm8::NL * tcm8::CH * 2;
+}
 
 cudaError_t map8_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float eps, const void* x,
                              const float* phi, void* phi_split, const float* b,
@@ -493,20 +509,17 @@ cudaError_t map8_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float ep
                              float* coef, void* urec, float* part, int* st, int64_t wait_ns,
                              cudaStream_t s) {
   using namespace tcm8;
-  const int64_t K = (int64_t)N * C;
-  k_phi_split8<<<(unsigned)((K + 255) / 256), 256, 0, s>>>(K, phi, (__nv_bfloat16*)phi_split);
+  const int64_t ncp = (C + CH - 1) / CH * CH;
+  k_phi_split8<<<(unsigned)((N * ncp + 255) / 256), 256, 0, s>>>(C, ncp, phi,
+                                                                  (__nv_bfloat16*)phi_split);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  CUtensorMap mx, mp, mG, mg, mf;
+  CUtensorMap mx, mG, mg, mf;
   const CUtensorMapSwizzle SW = CU_TENSOR_MAP_SWIZZLE_32B;
   const uint64_t dx[3] = {(uint64_t)C, (uint64_t)N, (uint64_t)T};
   const uint64_t sx[2] = {(uint64_t)C * 2, (uint64_t)N * C * 2};
   const uint32_t bx[3] = {CH, 1, TM};
   e = make_tmap_bf16(&mx, x, 3, dx, sx, bx, SW);
-  if (e != cudaSuccess) return e;
-  const uint64_t dp[3] = {(uint64_t)C, (uint64_t)N, (uint64_t)NL};
-  const uint32_t bp[3] = {CH, 1, NL};
-  e = make_tmap_bf16(&mp, phi_split, 3, dp, sx, bp, SW);
   if (e != cudaSuccess) return e;
   // maps a mode does not read are copies of the x map (never dereferenced)
   mG = mx;
@@ -527,13 +540,13 @@ cudaError_t map8_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float ep
   }
   switch (mode) {
     case MAP_FWD:
-      return launch_map8<MAP_FWD>(mx, mp, mG, mg, mf, T, C, iters, eps, b, alpha, ag, Hpre, Hpost,
+      return launch_map8<MAP_FWD>(mx, phi_split, mG, mg, mf, T, C, iters, eps, b, alpha, ag, Hpre, Hpost,
                                   Hres, nullptr, nullptr, nullptr, nullptr, st, wait_ns, s);
     case MAP_BWD:
-      return launch_map8<MAP_BWD>(mx, mp, mG, mg, mf, T, C, iters, eps, b, alpha, ag, nullptr,
+      return launch_map8<MAP_BWD>(mx, phi_split, mG, mg, mf, T, C, iters, eps, b, alpha, ag, nullptr,
                                   nullptr, nullptr, coef, urec, part, nullptr, st, wait_ns, s);
     case MAP_BWD_SPLIT:
-      return launch_map8<MAP_BWD_SPLIT>(mx, mp, mG, mg, mf, T, C, iters, eps, b, alpha, ag,
+      return launch_map8<MAP_BWD_SPLIT>(mx, phi_split, mG, mg, mf, T, C, iters, eps, b, alpha, ag,
                                         nullptr, nullptr, nullptr, coef, urec, part, red, st,
                                         wait_ns, s);
     default:

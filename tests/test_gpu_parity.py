@@ -536,15 +536,16 @@ def test_forward_backward_full_size(mhc, oracle_mod):
     assert_close(_np(ga), np.array([full["grad_alpha"]]), 2e-2)
 
 
-# ------------- bf16 n = 4 mapping: channel chunks spread evenly over the SMs
-# (T, C): tiles cut into several parts at arbitrary chunk boundaries, ranges
-# that cross tile boundaries, a ragged last chunk (C % 32 != 0) and a ragged
-# last tile, and the 16-part limit per tile.
+# ------------- bf16 n = 4 mapping with each 128-token tile cut into channel
+# parts (one CTA each, records added by the tile's last part in part order)
+# whenever one CTA per tile would leave SMs idle.  (T, C): several parts per
+# tile, a ragged last chunk (C % 32 != 0), a ragged last tile, and the 16-part
+# limit per tile.
 SPLIT_SHAPES = [(1000, 1024), (300, 7168), (777, 1000), (4096, 7168), (129, 4104)]
 
 
 @pytest.mark.parametrize("T,C", SPLIT_SHAPES)
-def test_balanced_mapping_pre(mhc, oracle_mod, T, C):
+def test_channel_split_mapping_pre(mhc, oracle_mod, T, C):
     d = _inputs(T, 4, C, torch.bfloat16, seed=T + 3 * C)
     idx = np.unique(np.concatenate([np.arange(0, T, max(1, T // 200)), [T - 1]]))
     dd = _dev(d)
@@ -559,13 +560,13 @@ def test_balanced_mapping_pre(mhc, oracle_mod, T, C):
 
 
 @pytest.mark.parametrize("T,C", SPLIT_SHAPES[:3] + SPLIT_SHAPES[4:])
-def test_balanced_mapping_backward(mhc, oracle_mod, T, C):
+def test_channel_split_mapping_backward(mhc, oracle_mod, T, C):
     d = _inputs(T, 4, C, torch.bfloat16, seed=2 * T + C)
     _check_bwd(mhc, oracle_mod, d, 20, torch.bfloat16)
 
 
 @pytest.mark.parametrize("T,C", [(1000, 1024), (300, 7168)])
-def test_balanced_mapping_pre_backward(mhc, oracle_mod, T, C):
+def test_channel_split_mapping_pre_backward(mhc, oracle_mod, T, C):
     d = _inputs(T, 4, C, torch.bfloat16, seed=5 * T + C)
     a = float(d["alpha"][0])
     fwd = oracle_mod.pre(d["x"], d["phi"], d["b"], a)
@@ -580,7 +581,7 @@ def test_balanced_mapping_pre_backward(mhc, oracle_mod, T, C):
         assert_close(_np(got), ref[k], 2e-2, k)
 
 
-def test_balanced_mapping_is_deterministic(mhc):
+def test_channel_split_mapping_is_deterministic(mhc):
     """Parts of a tile are added in part order: repeated calls give identical bits."""
     d = _dev(_inputs(4096, 4, 7168, torch.bfloat16, seed=8))
     outs = [mhc.mhc_backward(d["x"], d["phi"], d["b"], d["alpha"], d["f_out"], d["grad_x_next"],
