@@ -24,13 +24,26 @@ __global__ void __launch_bounds__(256) k_post(int64_t T, int64_t C, const TIO* _
                                               TIO* __restrict__ xn) {
   using V = Vec<TIO>;
   constexpr int W = V::N;
+  // n >= 8: the token's coefficients sit in shared memory (broadcast reads), so
+  // that the registers hold only the streams' values and two CTAs fit an SM
+  constexpr bool SH = N >= 8;
+  __shared__ float hs[SH ? N * N + N : 1];
   const int64_t nv = C / W;
   for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-    float hr[N * N], hp[N];
+    float hr[SH ? 1 : N * N], hp[SH ? 1 : N];
+    if constexpr (SH) {
+      __syncthreads();
+      for (int e = threadIdx.x; e < N * N + N; e += blockDim.x)
+        hs[e] = e < N * N ? __ldg(Hres + t * N * N + e) : __ldg(Hpost + t * N + (e - N * N));
+      __syncthreads();
+    } else {
 #pragma unroll
-    for (int e = 0; e < N * N; ++e) hr[e] = __ldg(Hres + t * N * N + e);
+      for (int e = 0; e < N * N; ++e) hr[e] = __ldg(Hres + t * N * N + e);
 #pragma unroll
-    for (int i = 0; i < N; ++i) hp[i] = __ldg(Hpost + t * N + i);
+      for (int i = 0; i < N; ++i) hp[i] = __ldg(Hpost + t * N + i);
+    }
+    auto HR = [&](int e) { return SH ? hs[e] : hr[e]; };
+    auto HP = [&](int i) { return SH ? hs[N * N + i] : hp[i]; };
     const TIO* xt = x + t * N * C;
     TIO* ot = xn + t * N * C;
     for (int64_t v = threadIdx.x; v < nv; v += blockDim.x) {
@@ -43,9 +56,9 @@ __global__ void __launch_bounds__(256) k_post(int64_t T, int64_t C, const TIO* _
         float o[W];
 #pragma unroll
         for (int e = 0; e < W; ++e) {
-          float acc = hp[i] * fv[e];
+          float acc = HP(i) * fv[e];
 #pragma unroll
-          for (int j = 0; j < N; ++j) acc = fmaf(hr[i * N + j], xv[j][e], acc);
+          for (int j = 0; j < N; ++j) acc = fmaf(HR(i * N + j), xv[j][e], acc);
           o[e] = acc;
         }
         V::store_stream(ot + i * C + v * W, o);
