@@ -94,6 +94,7 @@ def kernel_source_sha(files):
 
 
 # kernels behind each single-kernel call, for matching ncu traffic to sources
+# (keys: the call at n = 4; "<call>_n8" at n = 8)
 CALL_SOURCES = {
     "post": ["k_post.cu", "mhc_common.cuh"],
     "bwd_map": ["k_map_tc.cu", "tc_sm100.cuh", "mhc_common.cuh"],
@@ -101,18 +102,25 @@ CALL_SOURCES = {
     "pre": ["k_map_tc.cu", "k_post.cu", "tc_sm100.cuh", "mhc_common.cuh"],
     "layer_input": ["k_post.cu", "mhc_common.cuh"],
     "post_fused": ["k_map_tc.cu", "tc_sm100.cuh", "mhc_common.cuh"],
+    "post_n8": ["k_post.cu", "mhc_common.cuh"],
+    "bwd_map_n8": ["k_map8_tc.cu", "tc_sm100.cuh", "mhc_common.cuh"],
+    "layer_input_n8": ["k_post.cu", "mhc_common.cuh"],
 }
 
 
-def ncu_traffic(call):
+def traffic_key(call, n):
+    return call if n == N_STR else "%s_n%d" % (call, n)
+
+
+def ncu_traffic(key):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     the current source of that kernel; else None."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(p) as f:
             d = json.load(f)
-        e = d[call]
-        if e.get("source_sha") != kernel_source_sha(CALL_SOURCES[call]):
+        e = d[key]
+        if e.get("source_sha") != kernel_source_sha(CALL_SOURCES[key]):
             return None
         return float(e["bytes_per_launch"])
     except Exception:
@@ -346,9 +354,10 @@ def run_layer(args, dev, rank, world, local_rank):
     fused = args.forward == "fused"
     calls = (["layer_input", "post_fused"] if fused else ["pre", "post"]) + ["bwd_map", "bwd_apply"]
     # this library's kernels per call: pre = phi split + mapping + layer input;
-    # bwd_map = phi split + mapping; post_fused = phi split + fused kernel
+    # bwd_map = phi split + mapping; post_fused = phi split + fused kernel;
+    # bwd_apply = one kernel at n = 4, three at n = 8 (phi u, grad_x, grad_phi)
     launches_per_call = {"pre": 3, "post": 1, "layer_input": 1, "post_fused": 2, "bwd_map": 2,
-                         "bwd_apply": 1}
+                         "bwd_apply": 1 if n == N_STR else 3}
     # the layer's maps; in a stack the previous layer's post_fused computes them
     mhc.mhc_pre(x, phi, b, alpha, t_max=T_MAX, out=(h_in, Hpre, Hpost, Hres), stream=stream)
     nxt = (torch.empty_like(Hpre), torch.empty_like(Hpost), torch.empty_like(Hres))
@@ -419,11 +428,13 @@ def run_layer(args, dev, rank, world, local_rank):
     pb = per_call_param_bytes(n, C)
     call_bytes = {c: T * tb[c] + pb[c] for c in calls}
     # the roofline is read for a call whose time is one kernel's (the phi split
-    # ahead of the backward mapping is 5 us of its 0.5 ms and is counted in)
-    single = [c for c in calls if c in ("post", "bwd_map", "bwd_apply", "layer_input")]
+    # ahead of the backward mapping is 5 us of its 0.5 ms and is counted in; at
+    # n = 8 the apply is three kernels and is not such a call)
+    single = [c for c in calls
+              if c in ("post", "bwd_map", "layer_input") or (c == "bwd_apply" and n == N_STR)]
     dom = max(single, key=lambda c: per_call[c])
     achieved = call_bytes[dom] / (per_call[dom] / 1000.0) / 1e9
-    traffic = ncu_traffic(dom)
+    traffic = ncu_traffic(traffic_key(dom, n))
     fwd_calls = calls[:2]
     step_alg_bytes = (T * (sum(tb[c] for c in fwd_calls) + tb["bwd_min"]) +
                       sum(pb[c] for c in fwd_calls) + pb["bwd_apply"])
