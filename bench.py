@@ -213,6 +213,91 @@ def cpu_reference(seconds: float, seed: int = 0):
                               "sample": f"first {S1} tokens, {dt1:.2f} s"}}
 
 
+def _grow(run, seconds, start, cap):
+    """Grow the sample size from `start` until one timed pass takes about
+    `seconds` / 4 or more (or the cap is reached); returns (size, seconds)."""
+    S = start
+    dt = run(S)
+    while dt < seconds / 4 and S < cap:
+        S = min(cap, int(S * max(2.0, min(8.0, seconds / max(dt, 1e-3) / 2))))
+        dt = run(S)
+    return S, dt
+
+
+def _both_thread_counts(run, seconds, start, cap, small):
+    """The oracle with every host thread on a grown sample, then with one thread
+    on a `small` sample of the same workload."""
+    import oracle
+    S, dt = _grow(run, seconds, start, cap)
+    cores = oracle.num_threads()
+    oracle.set_num_threads(1)
+    try:
+        dt1 = run(small)
+    finally:
+        oracle.set_num_threads(cores)
+    return S, dt, cores, small, dt1
+
+
+def cpu_sinkhorn(seconds: float):
+    """The fp64 oracle's batched Sinkhorn on the first S matrices of each n's batch
+    (n = 4, 8, 16; the same seeded logits; 20 iterations): matrices/s."""
+    import oracle
+    from manifold_constrained_hyper_token_b200 import synth
+
+    def run(S):
+        lg = [synth.sinkhorn_logits(S, n, seed=100 + n) for n in (4, 8, 16)]
+        t0 = time.perf_counter()
+        for x in lg:
+            oracle.sinkhorn(x, T_MAX)
+        return time.perf_counter() - t0
+
+    S, dt, cores, S1, dt1 = _both_thread_counts(run, seconds, 1024, 1 << 22, 16384)
+    return {"value": 3 * S / dt, "unit": "matrices/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {S} matrices of each of the n=4, 8, 16 batches, 20 iterations "
+                      f"in fp64, {dt:.2f} s",
+            "single_thread": {"value": 3 * S1 / dt1, "unit": "matrices/s", "cores": 1,
+                              "sample": f"first {S1} matrices per n, {dt1:.2f} s"}}
+
+
+def cpu_depth(seconds: float, L: int = 24):
+    """The fp64 oracle through the L-layer stack (F_l(h) = s_l h) on the first S
+    tokens of chunk 0: forward, then each layer's backward with grad_h_in =
+    s_l grad_f_out, last layer first: tokens/s."""
+    import numpy as np
+    import oracle
+    from manifold_constrained_hyper_token_b200 import synth
+
+    prms = [synth.layer_params(N_STR, C_CH, seed=l) for l in range(L)]
+    gains = [synth.depth_gain(l) for l in range(L)]
+
+    def run(S):
+        d = synth.depth_stack_chunk(S, N_STR, C_CH, chunk=0)
+        t0 = time.perf_counter()
+        xs, fs = [d["x0"]], []
+        for l in range(L):
+            a = float(prms[l]["alpha"][0])
+            r = oracle.pre(xs[l], prms[l]["phi"], prms[l]["b"], a, iters=T_MAX)
+            fs.append(gains[l] * r["h_in"])
+            xs.append(oracle.post(xs[l], fs[l], r["H_post"], r["H_res"]))
+        G = d["G_last"]
+        for l in reversed(range(L)):
+            a = float(prms[l]["alpha"][0])
+            zero = np.zeros((S, C_CH))
+            gf = oracle.backward(xs[l], prms[l]["phi"], prms[l]["b"], a, fs[l], G, zero,
+                                 iters=T_MAX)["grad_f_out"]
+            G = oracle.backward(xs[l], prms[l]["phi"], prms[l]["b"], a, fs[l], G, gains[l] * gf,
+                                iters=T_MAX)["grad_x"]
+        return time.perf_counter() - t0
+
+    S, dt, cores, S1, dt1 = _both_thread_counts(run, seconds, 4, 4096, 8)
+    return {"value": S / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {S} tokens of the stack input, {L} layers forward and backward "
+                      f"(the per-layer backward run twice: grad_f_out, then grad_x) in fp64, "
+                      f"{dt:.2f} s",
+            "single_thread": {"value": S1 / dt1, "unit": "tokens/s", "cores": 1,
+                              "sample": f"first {S1} tokens, {dt1:.2f} s"}}
+
+
 def run_reference(args, rank, world):
     """Reference arm: the fp64 oracle on the host cores.  Each step runs
     pre + post + backward on a bounded sample of S tokens of the same
@@ -581,6 +666,9 @@ def run_sinkhorn(args, dev, rank, world, local_rank):
     for v in per_n.values():
         v["alu_frac"] = v["gops"] / alu_peak_gops
     dom = max(per_n, key=lambda k: per_n[k]["ms"])
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_sinkhorn(args.cpu_sample_seconds)
     if rank == 0:
         d = per_n[dom]
         bound = "hbm" if d["hbm_frac"] >= d["alu_frac"] else "alu"
@@ -606,6 +694,7 @@ def run_sinkhorn(args, dev, rank, world, local_rank):
                          "frac": d["hbm_frac"] if bound == "hbm" else d["alu_frac"],
                          "traffic": None, "peak_kind": peak_kind if bound == "hbm" else
                          "148 SMs x 128 fp32 lanes x median SM clock"},
+            "cpu_baseline": cpu,
             "gpu_launches": 4 * args.steps,
             "clocks": clocks,
         }
@@ -646,6 +735,16 @@ def run_depth(args, dev, rank, world, local_rank):
     peak, peak_kind = load_peaks()
     tb = per_token_bytes(n, C)
     alg = L * T * (tb["pre"] + tb["post"] + tb["bwd_min"])
+    # this library's launches per step: forward pre (phi split, mapping, layer
+    # input) + post per layer; backward: each recompute's pre (+ post when the
+    # next layer's input is rebuilt), then post_backward + pre_backward (phi
+    # split, split mapping, apply) per layer
+    rec = [st for st in stack.bwd_steps if st[0] == "recompute"]
+    launches = 4 * L + sum(3 + (1 if st[2] else 0) for st in rec) + 4 * L
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_depth(args.cpu_sample_seconds)
+    gbs = alg / (t / 1e3) / 1e9
     if rank == 0:
         line = {
             "metric": "mHC depth-stack tokens/s (24 layers fwd+bwd with recompute, n=4, C=7168)",
@@ -663,6 +762,11 @@ def run_depth(args, dev, rank, world, local_rank):
                     "peak_kind": peak_kind,
                     "note": "24 x 415,920 B/token (one forward and a one-pass backward per "
                             "layer); the recompute forward and F are extra"},
+            "roofline": {"bound": "hbm", "kernel": "whole step (24 layers, every kernel)",
+                         "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "traffic": None, "peak_kind": peak_kind},
+            "cpu_baseline": cpu,
+            "gpu_launches": launches * args.steps,
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

@@ -536,6 +536,62 @@ def test_forward_backward_full_size(mhc, oracle_mod):
     assert_close(_np(ga), np.array([full["grad_alpha"]]), 2e-2)
 
 
+# ------------- bf16 n = 8 on the tensor cores: several 128-token tiles with a
+# ragged last one, several 256-channel phi u blocks and 128-channel grad_phi
+# blocks with a ragged last one, and C % 16 == 8 (a half-filled last block of
+# the tiled phi copy)
+N8_SHAPES = [(300, 520), (129, 4104), (1000, 1024)]
+
+
+@pytest.mark.parametrize("T,C", N8_SHAPES)
+def test_n8_tensor_core_pre(mhc, oracle_mod, T, C):
+    d = _inputs(T, 8, C, torch.bfloat16, seed=11 * T + C)
+    dd = _dev(d)
+    st = _status()
+    h_in, Hpre, Hpost, Hres = mhc.mhc_pre(dd["x"], dd["phi"], dd["b"], dd["alpha"], dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ref = oracle_mod.pre(d["x"], d["phi"], d["b"], float(d["alpha"][0]))
+    for k, got in (("h_in", h_in), ("H_pre", Hpre), ("H_post", Hpost), ("H_res", Hres)):
+        assert_close(_np(got), ref[k], 2e-2, k)
+
+
+@pytest.mark.parametrize("T,C", N8_SHAPES)
+def test_n8_tensor_core_backward(mhc, oracle_mod, T, C):
+    d = _inputs(T, 8, C, torch.bfloat16, seed=13 * T + C)
+    _check_bwd(mhc, oracle_mod, d, 20, torch.bfloat16)
+
+
+@pytest.mark.slow
+def test_n8_forward_backward_large(mhc, oracle_mod):
+    """T=4096, n=8, C=7168 bf16 forward + backward (the n = 8 bench layer at a
+    quarter of its tokens): per-token outputs on a seeded sample of tokens;
+    grad_phi / grad_b / grad_alpha against the full-T oracle."""
+    from manifold_constrained_hyper_token_b200 import synth
+    T, n, C = 4096, 8, 7168
+    d = synth.layer_inputs(T, n, C, seed=3, dtype=torch.bfloat16, backward=True)
+    dd = _dev(d)
+    alpha = float(d["alpha"][0])
+    h_in, Hpre, Hpost, Hres = mhc.mhc_pre(dd["x"], dd["phi"], dd["b"], dd["alpha"])
+    gx, gphi, gb, ga, gf = mhc.mhc_backward(dd["x"], dd["phi"], dd["b"], dd["alpha"], dd["f_out"],
+                                            dd["grad_x_next"], dd["grad_h_in"])
+    torch.cuda.synchronize()
+    idx = synth.token_sample(T, 128, seed=4)
+    ic = idx.cuda()
+    ref = oracle_mod.pre(d["x"][idx], d["phi"], d["b"], alpha)
+    for got, r in ((h_in[ic], ref["h_in"]), (Hres[ic], ref["H_res"]), (Hpre[ic], ref["H_pre"])):
+        assert_close(_np(got), r, 2e-2)
+    rs = oracle_mod.backward(d["x"][idx], d["phi"], d["b"], alpha, d["f_out"][idx],
+                             d["grad_x_next"][idx], d["grad_h_in"][idx])
+    assert_close(_np(gx[ic]), rs["grad_x"], 2e-2)
+    assert_close(_np(gf[ic]), rs["grad_f_out"], 2e-2)
+    full = oracle_mod.backward(d["x"], d["phi"], d["b"], alpha, d["f_out"], d["grad_x_next"],
+                               d["grad_h_in"], chunk=512)
+    assert_close(_np(gphi), full["grad_phi"], 2e-2)
+    assert_close(_np(gb), full["grad_b"], 2e-2)
+    assert_close(_np(ga), np.array([full["grad_alpha"]]), 2e-2)
+
+
 # ------------- bf16 n = 4 mapping with each 128-token tile cut into channel
 # parts (one CTA each, records added by the tile's last part in part order)
 # whenever one CTA per tile would leave SMs idle.  (T, C): several parts per
