@@ -363,9 +363,10 @@ def main():
     ap.add_argument("--workload", default="layer", choices=["layer", "sinkhorn", "depth"],
                     help="layer: the fwd+bwd layer step (the default line); sinkhorn: batched "
                          "Sinkhorn-Knopp and depth gain; depth: the 24-layer stack")
-    ap.add_argument("--streams", type=int, default=N_STR, choices=[4, 8],
-                    help="layer workload stream count n (default 4, the headline; 8 runs the "
-                         "tensor-core mapping with the CUDA-core apply)")
+    ap.add_argument("--streams", type=int, default=N_STR, choices=[4, 8, 16],
+                    help="layer workload stream count n (default 4, the headline; 8 runs its "
+                         "tensor-core mapping and apply; 16 its tensor-core projection with the "
+                         "CUDA-core reductions, Sinkhorn and apply)")
     ap.add_argument("--forward", default="unfused", choices=["fused", "unfused"],
                     help="fused: layer input + post merge fused with the next layer's mapping; "
                          "unfused: mhc_pre + mhc_post")
@@ -441,8 +442,15 @@ def run_layer(args, dev, rank, world, local_rank):
     # this library's kernels per call: pre = phi split + mapping + layer input;
     # bwd_map = phi split + mapping; post_fused = phi split + fused kernel;
     # bwd_apply = one kernel at n = 4, three at n = 8 (phi u, grad_x, grad_phi)
+    # and n = 16 (grad_x, grad_phi, bias); n = 16: pre = phi split + projection +
+    # epilogue + layer input, bwd_map = phi split + projection + reductions +
+    # epilogue
     launches_per_call = {"pre": 3, "post": 1, "layer_input": 1, "post_fused": 2, "bwd_map": 2,
                          "bwd_apply": 1 if n == N_STR else 3}
+    if n == 8:  # the fused post is k_post, then the phi split and the mapping
+        launches_per_call["post_fused"] = 3
+    if n == 16:
+        launches_per_call.update({"pre": 4, "bwd_map": 4, "post_fused": 4})
     # the layer's maps; in a stack the previous layer's post_fused computes them
     mhc.mhc_pre(x, phi, b, alpha, t_max=T_MAX, out=(h_in, Hpre, Hpost, Hres), stream=stream)
     nxt = (torch.empty_like(Hpre), torch.empty_like(Hpost), torch.empty_like(Hres))
@@ -516,7 +524,8 @@ def run_layer(args, dev, rank, world, local_rank):
     # ahead of the backward mapping is 5 us of its 0.5 ms and is counted in; at
     # n = 8 the apply is three kernels and is not such a call)
     single = [c for c in calls
-              if c in ("post", "bwd_map", "layer_input") or (c == "bwd_apply" and n == N_STR)]
+              if c in ("post", "layer_input") or (c == "bwd_map" and n != 16) or
+              (c == "bwd_apply" and n == N_STR)]
     dom = max(single, key=lambda c: per_call[c])
     achieved = call_bytes[dom] / (per_call[dom] / 1000.0) / 1e9
     traffic = ncu_traffic(traffic_key(dom, n))

@@ -237,7 +237,10 @@ __device__ __forceinline__ void wide_epilogue(int tid, int64_t t, int64_t T, int
 // MAP_FWD: H_pre / H_post / H_res.  MAP_BWD: coef [T][Coef<16>::SIZE] and per
 // CTA the sums over its tokens of dz and dz . y (part [grid][DZ_SIZE]).
 // MAP_BWD_SPLIT: as MAP_BWD with <G_i, x_j> and <G_i, f_out> from `red`.
-template <typename TIO, int MODE>
+// PROJ = false (backward only): the projection and the sum of squares are
+// already in the rows (the tensor-core projection of bf16 inputs wrote them);
+// only the C-reductions run here.
+template <typename TIO, int MODE, bool PROJ = true>
 __global__ void __launch_bounds__(widek::NT) k_wide_map(
     int64_t T, int64_t C, int iters, float eps, const TIO* __restrict__ x,
     const float* __restrict__ phi, const float* __restrict__ bias,
@@ -259,7 +262,8 @@ __global__ void __launch_bounds__(widek::NT) k_wide_map(
   const int64_t K = (int64_t)N * C;
 
   // ---- projection y[t][m] = sum_k x[t][k] phi[k][m], and the sums of squares
-  {
+  static_assert(PROJ || BWD, "the forward projects");
+  if constexpr (PROJ) {
     float* xs = stg;            // [KC][TB]
     float* ps = stg + KC * TB;  // [KC][M]
     float acc[4][CPT], ssp[4];
@@ -389,6 +393,25 @@ __global__ void __launch_bounds__(32) k_wide_bwd_epi(int64_t T, int64_t C, int i
     for (int q = 0; q < TB; ++q) s += dzs[q * (M + 3) + col];
     part_o[(int64_t)blockIdx.x * CF::DZ_SIZE + col] = s;
   }
+}
+
+// The forward's per-token epilogue from rows written by the tensor-core
+// projection (y at [0, M), the sum of squares at [2M]): one thread per token.
+__global__ void __launch_bounds__(32) k_wide_fwd_epi(int64_t T, int64_t C, int iters, float eps,
+                                                     const float* __restrict__ bias,
+                                                     const float* __restrict__ alpha_p, int ag,
+                                                     const float* __restrict__ rows,
+                                                     float* __restrict__ Hpre_o,
+                                                     float* __restrict__ Hpost_o,
+                                                     float* __restrict__ Hres_o, int* status) {
+  using namespace widek;
+  using CF = Coef<N>;
+  const int tid = threadIdx.x;
+  const int64_t t = (int64_t)blockIdx.x * TB + tid;
+  if (t >= T) return;
+  const float* row = rows + t * CF::SIZE;
+  wide_epilogue<MAP_FWD>(tid, t, T, (int64_t)N * C, iters, eps, row, nullptr, row[2 * M], bias,
+                         alpha_p, ag, Hpre_o, Hpost_o, Hres_o, nullptr, nullptr, nullptr, status);
 }
 
 // x_next[i][c] = sum_j H_res[i][j] x[j][c] + H_post[i] f_out[c] (the k_post order)
@@ -716,6 +739,52 @@ static cudaError_t launch_wide_map(int64_t T, int64_t C, int iters, float eps, c
 }
 
 int wide_map_tokens_per_cta() { return widek::TB; }
+
+cudaError_t wide_map_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float eps,
+                                 const void* x, const float* phi, void* phi_t, const float* b,
+                                 const float* alpha, int ag, float* Hpre, float* Hpost,
+                                 float* Hres, const void* G, const void* g, const void* f,
+                                 const float* red, float* rows, float* part, int* st,
+                                 int64_t wait_ns, cudaStream_t s) {
+  using CF = Coef<widek::N>;
+  cudaError_t e = proj16_dispatch(T, C, x, phi, phi_t, rows, CF::SIZE, st, wait_ns, s);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = (unsigned)((T + widek::TB - 1) / widek::TB);
+  if (mode == MAP_FWD) {
+    k_wide_fwd_epi<<<grid, 32, 0, s>>>(T, C, iters, eps, b, alpha, ag, rows, Hpre, Hpost, Hres,
+                                       st);
+    return cudaGetLastError();
+  }
+  const size_t smem = (size_t)widek::SMEM_FLOATS * 4;
+  using BF = __nv_bfloat16;
+  if (mode == MAP_BWD) {
+    auto kern = k_wide_map<BF, MAP_BWD, false>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, widek::NT, smem, s>>>(T, C, iters, eps, (const BF*)x, phi, b, alpha, ag, nullptr,
+                                       nullptr, nullptr, (const BF*)G, (const BF*)g, (const BF*)f,
+                                       red, rows, part, st);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    k_wide_bwd_epi<MAP_BWD><<<grid, 32, 0, s>>>(T, C, iters, eps, b, alpha, ag, red, rows, part,
+                                                st);
+    return cudaGetLastError();
+  }
+  if (mode == MAP_BWD_SPLIT) {
+    auto kern = k_wide_map<BF, MAP_BWD_SPLIT, false>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, widek::NT, smem, s>>>(T, C, iters, eps, (const BF*)x, phi, b, alpha, ag, nullptr,
+                                       nullptr, nullptr, (const BF*)G, (const BF*)g, (const BF*)f,
+                                       red, rows, part, st);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    k_wide_bwd_epi<MAP_BWD_SPLIT><<<grid, 32, 0, s>>>(T, C, iters, eps, b, alpha, ag, red, rows,
+                                                      part, st);
+    return cudaGetLastError();
+  }
+  return cudaErrorInvalidValue;
+}
 
 cudaError_t wide_map_dispatch(int mode, int dtype, int64_t T, int64_t C, int iters, float eps,
                               const void* x, const float* phi, const float* b, const float* alpha,

@@ -60,6 +60,9 @@ int dz_size(int n) {
 // (64 tokens per mapping CTA; n = 16 its own).
 bool use_tc(const mhc_params* p) { return p->dtype == MHC_DTYPE_BF16 && p->n == 4; }
 bool use_tc8(const mhc_params* p) { return p->dtype == MHC_DTYPE_BF16 && p->n == 8; }
+// bf16 with n = 16: the projection on the tensor cores, the rest on k_wide
+bool use_tc16(const mhc_params* p) { return p->dtype == MHC_DTYPE_BF16 && p->n == 16; }
+size_t rows16_bytes(int64_t T) { return (size_t)T * mhc::Coef<16>::SIZE * 4; }
 
 // Backward workspace.  CUDA-core path: per-token coefficient records, then one
 // partial-sum record (dz, dz . y) per 64-token mapping CTA.  Tensor-core path
@@ -96,7 +99,9 @@ BwdWorkspace bwd_layout(const mhc_params* p) {
   w.part_off = off;
   off = round_up(off + (size_t)w.nparts * dz_size(p->n) * 4, 256);
   w.phi_off = off;
-  off = round_up(off + (tc ? mhc::map_tc_phi_bytes(p->C) : (tc8 ? mhc::map8_tc_phi_bytes(p->C) : 0)),
+  off = round_up(off + (tc    ? mhc::map_tc_phi_bytes(p->C)
+                        : tc8 ? mhc::map8_tc_phi_bytes(p->C)
+                              : (use_tc16(p) ? mhc::proj16_phi_bytes(p->C) : 0)),
                  256);
   w.apply_off = off;
   off = round_up(off + (tc ? mhc::apply_tc_scratch_bytes(p->T, p->C)
@@ -140,6 +145,8 @@ size_t mhc_pre_workspace_size(const mhc_params* p) {
   if (use_tc(p))
     return round_up(mhc::map_tc_phi_bytes(p->C), 256) +
            round_up(mhc::map_tc_scratch_bytes(p->T, p->C), 256);
+  if (use_tc16(p))  // the tiled phi copy, then the rows of projections
+    return round_up(mhc::proj16_phi_bytes(p->C), 256) + round_up(rows16_bytes(p->T), 256);
   return use_tc8(p) ? round_up(mhc::map8_tc_phi_bytes(p->C), 256) : 0;
 }
 
@@ -170,6 +177,16 @@ mhc_status mhc_pre(const mhc_params* p, const void* x, const float* phi, const f
                                          workspace, b, alpha, alpha_groups(p), H_pre, H_post,
                                          H_res, nullptr, nullptr, nullptr, nullptr, nullptr,
                                          nullptr, nullptr, dev_status, p->wait_ns, s));
+  } else if (use_tc16(p)) {
+    const size_t need = mhc_pre_workspace_size(p);
+    if (workspace == nullptr || workspace_bytes < need || ((uintptr_t)workspace & 255u) != 0)
+      return MHC_ERR_WORKSPACE;
+    char* ws = (char*)workspace;
+    st = from_cuda(mhc::wide_map_tc_dispatch(
+        mhc::MAP_FWD, p->T, p->C, p->t_max, p->eps, x, phi, ws, b, alpha, alpha_groups(p), H_pre,
+        H_post, H_res, nullptr, nullptr, nullptr, nullptr,
+        (float*)(ws + round_up(mhc::proj16_phi_bytes(p->C), 256)), nullptr, dev_status, p->wait_ns,
+        s));
   } else {
     st = from_cuda(mhc::map_fwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
                                          alpha, alpha_groups(p), H_pre, H_post, H_res, dev_status, s));
@@ -223,6 +240,12 @@ mhc_status mhc_backward_map(const mhc_params* p, const void* x, const float* phi
                                            nullptr, (float*)(ws + w.coef_off), ws + w.urec_off,
                                            (float*)(ws + w.part_off), dev_status, p->wait_ns,
                                            (cudaStream_t)stream));
+  if (use_tc16(p))
+    return from_cuda(mhc::wide_map_tc_dispatch(
+        mhc::MAP_BWD, p->T, p->C, p->t_max, p->eps, x, phi, ws + w.phi_off, b, alpha,
+        alpha_groups(p), nullptr, nullptr, nullptr, grad_x_next, grad_h_in, f_out, nullptr,
+        (float*)(ws + w.coef_off), (float*)(ws + w.part_off), dev_status, p->wait_ns,
+        (cudaStream_t)stream));
   return from_cuda(mhc::map_bwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
                                          alpha, alpha_groups(p), grad_x_next, grad_h_in, f_out, nullptr,
                                          (float*)(ws + w.coef_off), (float*)(ws + w.part_off),
@@ -322,6 +345,17 @@ mhc_status mhc_post_fused(const mhc_params* p, const void* x, const void* f_out,
                                            nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                                            nullptr, dev_status, p->wait_ns, s));
   }
+  if (use_tc16(p)) {
+    const size_t need = mhc_post_fused_workspace_size(p);
+    if (workspace == nullptr || workspace_bytes < need || ((uintptr_t)workspace & 255u) != 0)
+      return MHC_ERR_WORKSPACE;
+    char* ws = (char*)workspace;
+    return from_cuda(mhc::wide_map_tc_dispatch(
+        mhc::MAP_FWD, p->T, p->C, p->t_max, p->eps, x_next, phi_next, ws, b_next, alpha_next,
+        alpha_groups(p), H_pre_next, H_post_next, H_res_next, nullptr, nullptr, nullptr, nullptr,
+        (float*)(ws + round_up(mhc::proj16_phi_bytes(p->C), 256)), nullptr, dev_status, p->wait_ns,
+        s));
+  }
   return from_cuda(mhc::map_fwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x_next,
                                          phi_next, b_next, alpha_next, alpha_groups(p), H_pre_next,
                                          H_post_next,
@@ -400,7 +434,13 @@ mhc_status mhc_pre_backward(const mhc_params* p, const void* x, const float* phi
         ws + w.urec_off, (const float*)(ws + w.part_off), w.nparts, (float*)(ws + w.apply_off),
         grad_x, nullptr, grad_phi, grad_b, grad_alpha, alpha_groups(p), dev_status, p->wait_ns, s));
   }
-  st = from_cuda(mhc::map_bwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
+  if (use_tc16(p))
+    st = from_cuda(mhc::wide_map_tc_dispatch(
+        mhc::MAP_BWD_SPLIT, p->T, p->C, p->t_max, p->eps, x, phi, ws + w.phi_off, b, alpha,
+        alpha_groups(p), nullptr, nullptr, nullptr, nullptr, grad_h_in, nullptr, red,
+        (float*)(ws + w.coef_off), (float*)(ws + w.part_off), dev_status, p->wait_ns, s));
+  else
+    st = from_cuda(mhc::map_bwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
                                          alpha, alpha_groups(p), nullptr, grad_h_in, nullptr, red,
                                          (float*)(ws + w.coef_off), (float*)(ws + w.part_off),
                                          dev_status, s));

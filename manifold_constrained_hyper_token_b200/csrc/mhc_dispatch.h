@@ -79,6 +79,24 @@ cudaError_t apply8_tc_dispatch(int64_t T, int64_t C, const void* x, const void* 
                                int64_t wait_ns, cudaStream_t s);
 size_t map8_tc_phi_bytes(int64_t C);
 
+// k_proj16_tc.cu (bf16, n = 16): splits phi into the tiled bf16 copy phi_t
+// (proj16_phi_bytes(C) bytes) and writes each token's 288 projections y and
+// its sum of squares into rows [T][ostride] (y at [0, 288), ss at [576]).
+cudaError_t proj16_dispatch(int64_t T, int64_t C, const void* x, const float* phi, void* phi_t,
+                            float* rows, int64_t ostride, int* st, int64_t wait_ns,
+                            cudaStream_t s);
+size_t proj16_phi_bytes(int64_t C);
+// k_wide.cu, bf16 with n = 16: the mapping with the projection on the tensor
+// cores (proj16_dispatch) and the rest of the k_wide kernels: MAP_FWD writes
+// the maps (rows: [T][Coef<16>::SIZE] scratch); MAP_BWD / MAP_BWD_SPLIT write
+// the coefficient records into rows (= coef) and the partial sums.
+cudaError_t wide_map_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float eps,
+                                 const void* x, const float* phi, void* phi_t, const float* b,
+                                 const float* alpha, int ag, float* Hpre, float* Hpost,
+                                 float* Hres, const void* G, const void* g, const void* f,
+                                 const float* red, float* rows, float* part, int* st,
+                                 int64_t wait_ns, cudaStream_t s);
+
 // k_wide.cu (n = 16, CUDA cores); the mapping's mode is a MapMode
 int wide_map_tokens_per_cta();
 cudaError_t wide_map_dispatch(int mode, int dtype, int64_t T, int64_t C, int iters, float eps,
