@@ -29,6 +29,12 @@
 //   k_wide_apply_phi  grad_phi = sum_t x_t u_t^T, a GEMM over the tokens
 //   k_wide_bias       grad_b and grad_alpha from the mapping CTAs' partials
 //
+// With bf16 activations the projection runs on the tensor cores instead
+// (k_proj16_tc.cu writes y and the sum of squares into the rows; here
+// k_wide_fwd_epi runs the forward's epilogue from them, and k_wide_map in its
+// PROJ = false form adds only the backward's C-reductions), and so does the
+// apply (k_apply16_tc.cu; k_wide_bias supplies its grad_b and grad_alpha).
+//
 // Every sum is taken in a fixed order, so repeated calls give identical bits.
 // The per-token Sinkhorn arrays (16 x 16) live in local memory.
 #include "mhc_common.cuh"
@@ -865,6 +871,12 @@ static cudaError_t launch_wide_apply(int64_t T, int64_t C, const void* x, const 
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   k_wide_bias<<<1, NT, 0, s>>>(part, nparts, gb, ga, ag);
+  return cudaGetLastError();
+}
+
+cudaError_t wide_bias_dispatch(const float* part, int nparts, float* gb, float* ga, int ag,
+                               cudaStream_t s) {
+  k_wide_bias<<<1, widek::NT, 0, s>>>(part, nparts, gb, ga, ag);
   return cudaGetLastError();
 }
 

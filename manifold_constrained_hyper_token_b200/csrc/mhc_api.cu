@@ -56,8 +56,10 @@ int dz_size(int n) {
 }
 
 // bf16 activations with n = 4 or n = 8 take the tensor-core mapping and apply
-// kernels (128 tokens per mapping CTA); every other case the CUDA-core kernels
-// (64 tokens per mapping CTA; n = 16 its own).
+// kernels (128 tokens per mapping CTA); bf16 with n = 16 the tensor-core
+// projection and apply around the k_wide reductions, Sinkhorn and adjoint (32
+// tokens per epilogue CTA); every other case the CUDA-core kernels (64 tokens
+// per mapping CTA; n = 16 its own).
 bool use_tc(const mhc_params* p) { return p->dtype == MHC_DTYPE_BF16 && p->n == 4; }
 bool use_tc8(const mhc_params* p) { return p->dtype == MHC_DTYPE_BF16 && p->n == 8; }
 // bf16 with n = 16: the projection on the tensor cores, the rest on k_wide
@@ -95,6 +97,10 @@ BwdWorkspace bwd_layout(const mhc_params* p) {
       w.urec_off = off;
       off = round_up(off + (size_t)p->T * mhc::TcRec8::U_BYTES, 256);
     }
+    if (use_tc16(p)) {
+      w.urec_off = off;
+      off = round_up(off + mhc::apply16_urec_bytes(p->T), 256);
+    }
   }
   w.part_off = off;
   off = round_up(off + (size_t)w.nparts * dz_size(p->n) * 4, 256);
@@ -105,7 +111,7 @@ BwdWorkspace bwd_layout(const mhc_params* p) {
                  256);
   w.apply_off = off;
   off = round_up(off + (tc ? mhc::apply_tc_scratch_bytes(p->T, p->C)
-                           : (tc8 ? (size_t)p->T * 8 * p->C * 4 : 0)),
+                           : (tc8 || use_tc16(p) ? (size_t)p->T * p->n * p->C * 4 : 0)),
                  256);
   w.kmap_off = off;
   off = round_up(off + (tc ? mhc::map_tc_scratch_bytes(p->T, p->C) : 0), 256);
@@ -281,6 +287,12 @@ mhc_status mhc_backward_apply(const mhc_params* p, const void* x, const float* p
         ws + w.urec_off, (const float*)(ws + w.part_off), w.nparts, (float*)(ws + w.apply_off),
         grad_x, grad_f_out, grad_phi, grad_b, grad_alpha, alpha_groups(p), dev_status, p->wait_ns,
         (cudaStream_t)stream));
+  if (use_tc16(p))
+    return from_cuda(mhc::apply16_tc_dispatch(
+        p->T, p->C, x, ws + w.phi_off, grad_x_next, grad_h_in, (const float*)(ws + w.coef_off),
+        (const float*)(ws + w.part_off), w.nparts, (void*)(ws + w.urec_off),
+        (float*)(ws + w.apply_off), grad_x, grad_f_out, grad_phi, grad_b, grad_alpha,
+        alpha_groups(p), dev_status, p->wait_ns, (cudaStream_t)stream));
   return from_cuda(mhc::apply_dispatch(p->n, p->dtype, p->T, p->C, x, phi, grad_x_next, grad_h_in,
                                        (const float*)(ws + w.coef_off),
                                        (const float*)(ws + w.part_off), w.nparts, grad_x,
@@ -434,16 +446,22 @@ mhc_status mhc_pre_backward(const mhc_params* p, const void* x, const float* phi
         ws + w.urec_off, (const float*)(ws + w.part_off), w.nparts, (float*)(ws + w.apply_off),
         grad_x, nullptr, grad_phi, grad_b, grad_alpha, alpha_groups(p), dev_status, p->wait_ns, s));
   }
-  if (use_tc16(p))
+  if (use_tc16(p)) {
     st = from_cuda(mhc::wide_map_tc_dispatch(
         mhc::MAP_BWD_SPLIT, p->T, p->C, p->t_max, p->eps, x, phi, ws + w.phi_off, b, alpha,
         alpha_groups(p), nullptr, nullptr, nullptr, nullptr, grad_h_in, nullptr, red,
         (float*)(ws + w.coef_off), (float*)(ws + w.part_off), dev_status, p->wait_ns, s));
-  else
-    st = from_cuda(mhc::map_bwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
-                                         alpha, alpha_groups(p), nullptr, grad_h_in, nullptr, red,
-                                         (float*)(ws + w.coef_off), (float*)(ws + w.part_off),
-                                         dev_status, s));
+    if (st != MHC_OK) return st;
+    return from_cuda(mhc::apply16_tc_dispatch(
+        p->T, p->C, x, ws + w.phi_off, grad_x_next, grad_h_in, (const float*)(ws + w.coef_off),
+        (const float*)(ws + w.part_off), w.nparts, ws + w.urec_off, (float*)(ws + w.apply_off),
+        grad_x, nullptr, grad_phi, grad_b, grad_alpha, alpha_groups(p), dev_status, p->wait_ns,
+        s));
+  }
+  st = from_cuda(mhc::map_bwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
+                                       alpha, alpha_groups(p), nullptr, grad_h_in, nullptr, red,
+                                       (float*)(ws + w.coef_off), (float*)(ws + w.part_off),
+                                       dev_status, s));
   if (st != MHC_OK) return st;
   return from_cuda(mhc::apply_dispatch(p->n, p->dtype, p->T, p->C, x, phi, grad_x_next, grad_h_in,
                                        (const float*)(ws + w.coef_off),

@@ -97,6 +97,20 @@ cudaError_t wide_map_tc_dispatch(int mode, int64_t T, int64_t C, int iters, floa
                                  const float* red, float* rows, float* part, int* st,
                                  int64_t wait_ns, cudaStream_t s);
 
+// k_apply16_tc.cu (bf16, n = 16): the apply with phi u and grad_phi on the
+// tensor cores.  coef / part: the n = 16 mapping's records and partial sums;
+// phi_t: the tiled phi^T copy of proj16_dispatch; urec (apply16_urec_bytes(T))
+// and phiu (fp32 [T][16][C]) are scratch.  gf == nullptr skips grad_f_out.
+cudaError_t apply16_tc_dispatch(int64_t T, int64_t C, const void* x, const void* phi_t,
+                                const void* G, const void* g, const float* coef,
+                                const float* part, int nparts, void* urec, float* phiu, void* gx,
+                                void* gf, float* gphi, float* gb, float* ga, int ag, int* st,
+                                int64_t wait_ns, cudaStream_t s);
+size_t apply16_urec_bytes(int64_t T);
+// grad_b and grad_alpha of the n = 16 paths from the mapping's partial sums
+cudaError_t wide_bias_dispatch(const float* part, int nparts, float* gb, float* ga, int ag,
+                               cudaStream_t s);
+
 // k_wide.cu (n = 16, CUDA cores); the mapping's mode is a MapMode
 int wide_map_tokens_per_cta();
 cudaError_t wide_map_dispatch(int mode, int dtype, int64_t T, int64_t C, int iters, float eps,

@@ -18,7 +18,7 @@ from conftest import assert_close
 pytestmark = pytest.mark.gpu
 
 TIMEOUT = 5
-TOL = 2e-2  # bf16 I/O (the tensor-core kernels run for bf16 with n = 4 and n = 8)
+TOL = 2e-2  # bf16 I/O (the tensor-core kernels run for bf16 with n = 4, 8 and 16)
 
 
 @pytest.fixture(scope="module")
@@ -112,12 +112,15 @@ def test_fused_post_times_out_then_recovers(mhc, oracle_mod):
     assert_close(_np(xn), ref_xn, TOL, "x_next")
 
 
-@pytest.mark.parametrize("phase", ["pre", "map"])
-def test_n8_mapping_times_out_then_recovers(mhc, oracle_mod, phase):
-    """The n = 8 tensor-core mapping (bf16) gives up the same way."""
+@pytest.mark.parametrize("n", [8, 16])
+@pytest.mark.parametrize("phase", ["pre", "map", "apply"])
+def test_wide_tensor_core_paths_time_out_then_recover(mhc, oracle_mod, n, phase):
+    """The n = 8 and n = 16 tensor-core kernels (bf16) give up the same way: the
+    mapping / projection in the forward and the backward, and the apply's phi u and
+    grad_phi contractions."""
     from manifold_constrained_hyper_token_b200 import synth
-    T, n, C = 300, 8, 512
-    d = synth.layer_inputs(T, n, C, seed=17, dtype=torch.bfloat16, backward=True)
+    T, C = (300, 512) if n == 8 else (200, 256)
+    d = synth.layer_inputs(T, n, C, seed=17 + n, dtype=torch.bfloat16, backward=True)
     dd = {k: v.cuda() for k, v in d.items()}
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     if phase == "pre":
@@ -126,7 +129,13 @@ def test_n8_mapping_times_out_then_recovers(mhc, oracle_mod, phase):
         ws = torch.empty(mhc.mhc_backward_workspace_size(n, T, C, torch.bfloat16),
                          dtype=torch.uint8, device="cuda")
         mhc.mhc_backward_map(dd["x"], dd["phi"], dd["b"], dd["alpha"], dd["f_out"],
-                             dd["grad_x_next"], dd["grad_h_in"], ws, wait_ns=1, dev_status=st)
+                             dd["grad_x_next"], dd["grad_h_in"], ws,
+                             wait_ns=1 if phase == "map" else 0, dev_status=st)
+        if phase == "apply":
+            torch.cuda.synchronize()
+            assert int(st.item()) == 0
+            mhc.mhc_backward_apply(dd["x"], dd["phi"], dd["grad_x_next"], dd["grad_h_in"], ws,
+                                   wait_ns=1, dev_status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == TIMEOUT
     st.zero_()
