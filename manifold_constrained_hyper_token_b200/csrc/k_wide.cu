@@ -65,6 +65,11 @@ constexpr int SMEM_FLOATS = SS_OFF + TB;
 
 enum WideDots { WD_FULL = 0, WD_PRE = 1, WD_POST = 2 };
 
+// Sinkhorn checkpoints of the backward epilogue on the tensor-core path: every
+// second normalisation, iters + 1 iterates of N*N floats per token, laid out
+// per 32-token CTA as [iterate][element][token].
+constexpr int kWideCkPeriod = 2;
+
 // The C-reductions of one CTA's TB tokens, as dacc[token 4*ty + i][dot tx + 32q]:
 //   dot d < 256         <G_i, x_j>   (i = d / 16, j = d % 16)        WD_FULL, WD_POST
 //   256 <= d < 272      <g, x_i>     (i = d - 256)                    WD_FULL, WD_PRE
@@ -173,7 +178,7 @@ __device__ __forceinline__ void wide_epilogue(int tid, int64_t t, int64_t T, int
                                            const float* bias, const float* alpha_p, int ag,
                                            float* Hpre_o, float* Hpost_o, float* Hres_o,
                                            const float* red_in, float* coef_o, float* dzs,
-                                           int* status) {
+                                           int* status, float* ck = nullptr) {
   using namespace widek;
   constexpr bool BWD = MODE != MAP_FWD;
   constexpr bool SPLIT = MODE == MAP_BWD_SPLIT;
@@ -195,7 +200,13 @@ __device__ __forceinline__ void wide_epilogue(int tid, int64_t t, int64_t T, int
   if (mine && bad) flag_status(status, MHC_ERR_NONFINITE);
   float H[N * N];
   for (int e = 0; e < N * N; ++e) H[e] = zres[e];
-  sk_forward<N>(H, iters);
+  // with a checkpoint area (backward, tensor-core path) the forward keeps every
+  // second iterate there and the adjoint rebuilds each one from the nearest
+  // (the same iterates and results, a fraction of the recomputation)
+  if (BWD && ck != nullptr)
+    sk_forward_ckpt<N>(H, iters, ck, TB, kWideCkPeriod);
+  else
+    sk_forward<N>(H, iters);
   if constexpr (!BWD) {
     if (mine) {
       for (int i = 0; i < N; ++i) {
@@ -209,7 +220,10 @@ __device__ __forceinline__ void wide_epilogue(int tid, int64_t t, int64_t T, int
     float dA[N * N], dz[M];
     for (int e = 0; e < N * N; ++e) dA[e] = !mine ? 0.0f : (SPLIT ? __ldg(rt + e) : dt[e]);
     float dzres[N * N];
-    sk_adjoint<N>(zres, dA, dzres, iters);
+    if (ck != nullptr)
+      sk_adjoint_ckpt<N>(dA, dzres, iters, ck, TB, kWideCkPeriod);
+    else
+      sk_adjoint<N>(zres, dA, dzres, iters);
     for (int i = 0; i < N; ++i) {
       dz[i] = dt[N * N + i] * spre[i] * (1.0f - spre[i]);
       const float dpost = !mine ? 0.0f : (SPLIT ? __ldg(rt + N * N + i) : dt[N * N + N + i]);
@@ -380,7 +394,8 @@ __global__ void __launch_bounds__(32) k_wide_bwd_epi(int64_t T, int64_t C, int i
                                                      const float* __restrict__ alpha_p, int ag,
                                                      const float* __restrict__ red_in,
                                                      float* __restrict__ coef,
-                                                     float* __restrict__ part_o, int* status) {
+                                                     float* __restrict__ part_o, int* status,
+                                                     float* __restrict__ ck) {
   using namespace widek;
   using CF = Coef<N>;
   __shared__ float dzs[TB * (M + 3)];
@@ -388,8 +403,10 @@ __global__ void __launch_bounds__(32) k_wide_bwd_epi(int64_t T, int64_t C, int i
   const int64_t t = (int64_t)blockIdx.x * TB + tid;
   if (t < T) {
     const float* row = coef + t * CF::SIZE;
+    float* ckt = ck == nullptr ? nullptr
+                               : ck + (int64_t)blockIdx.x * ((int64_t)iters + 1) * N * N * TB + tid;
     wide_epilogue<MODE>(tid, t, T, (int64_t)N * C, iters, eps, row, row + M, row[2 * M], bias,
-                        alpha_p, ag, nullptr, nullptr, nullptr, red_in, coef, dzs, status);
+                        alpha_p, ag, nullptr, nullptr, nullptr, red_in, coef, dzs, status, ckt);
   } else {
     for (int m = 0; m < M + 3; ++m) dzs[tid * (M + 3) + m] = 0.0f;
   }
@@ -738,7 +755,7 @@ static cudaError_t launch_wide_map(int64_t T, int64_t C, int iters, float eps, c
   if constexpr (MODE != MAP_FWD) {
     if (e != cudaSuccess) return e;
     k_wide_bwd_epi<MODE><<<(unsigned)grid, 32, 0, s>>>(T, C, iters, eps, b, alpha, ag, red, coef,
-                                                       part, st);
+                                                       part, st, nullptr);
     e = cudaGetLastError();
   }
   return e;
@@ -746,11 +763,16 @@ static cudaError_t launch_wide_map(int64_t T, int64_t C, int iters, float eps, c
 
 int wide_map_tokens_per_cta() { return widek::TB; }
 
+size_t wide_ck_bytes(int64_t T, int iters) {
+  const int64_t ncta = (T + widek::TB - 1) / widek::TB;
+  return (size_t)ncta * ((size_t)iters + 1) * widek::N * widek::N * widek::TB * 4;
+}
+
 cudaError_t wide_map_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float eps,
                                  const void* x, const float* phi, void* phi_t, const float* b,
                                  const float* alpha, int ag, float* Hpre, float* Hpost,
                                  float* Hres, const void* G, const void* g, const void* f,
-                                 const float* red, float* rows, float* part, int* st,
+                                 const float* red, float* rows, float* part, float* ck, int* st,
                                  int64_t wait_ns, cudaStream_t s) {
   using CF = Coef<widek::N>;
   cudaError_t e = proj16_dispatch(T, C, x, phi, phi_t, rows, CF::SIZE, st, wait_ns, s);
@@ -773,7 +795,7 @@ cudaError_t wide_map_tc_dispatch(int mode, int64_t T, int64_t C, int iters, floa
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     k_wide_bwd_epi<MAP_BWD><<<grid, 32, 0, s>>>(T, C, iters, eps, b, alpha, ag, red, rows, part,
-                                                st);
+                                                st, ck);
     return cudaGetLastError();
   }
   if (mode == MAP_BWD_SPLIT) {
@@ -786,7 +808,7 @@ cudaError_t wide_map_tc_dispatch(int mode, int64_t T, int64_t C, int iters, floa
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     k_wide_bwd_epi<MAP_BWD_SPLIT><<<grid, 32, 0, s>>>(T, C, iters, eps, b, alpha, ag, red, rows,
-                                                      part, st);
+                                                      part, st, ck);
     return cudaGetLastError();
   }
   return cudaErrorInvalidValue;

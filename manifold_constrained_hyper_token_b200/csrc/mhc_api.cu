@@ -3,9 +3,10 @@
 // synchronises or keeps state between calls.
 #include <math.h>
 
+#include <algorithm>
+
 #include "mhc_common.cuh"
 #include "mhc_dispatch.h"
-
 
 namespace {
 
@@ -110,9 +111,14 @@ BwdWorkspace bwd_layout(const mhc_params* p) {
                               : (use_tc16(p) ? mhc::proj16_phi_bytes(p->C) : 0)),
                  256);
   w.apply_off = off;
-  off = round_up(off + (tc ? mhc::apply_tc_scratch_bytes(p->T, p->C)
-                           : (tc8 || use_tc16(p) ? (size_t)p->T * p->n * p->C * 4 : 0)),
-                 256);
+  // n = 16: the apply's phi u scratch, which the mapping first uses for its
+  // Sinkhorn checkpoints
+  size_t apply_bytes = 0;
+  if (tc) apply_bytes = mhc::apply_tc_scratch_bytes(p->T, p->C);
+  if (tc8) apply_bytes = (size_t)p->T * 8 * p->C * 4;
+  if (use_tc16(p))
+    apply_bytes = std::max((size_t)p->T * 16 * p->C * 4, mhc::wide_ck_bytes(p->T, p->t_max));
+  off = round_up(off + apply_bytes, 256);
   w.kmap_off = off;
   off = round_up(off + (tc ? mhc::map_tc_scratch_bytes(p->T, p->C) : 0), 256);
   w.total = off;
@@ -191,7 +197,8 @@ mhc_status mhc_pre(const mhc_params* p, const void* x, const float* phi, const f
     st = from_cuda(mhc::wide_map_tc_dispatch(
         mhc::MAP_FWD, p->T, p->C, p->t_max, p->eps, x, phi, ws, b, alpha, alpha_groups(p), H_pre,
         H_post, H_res, nullptr, nullptr, nullptr, nullptr,
-        (float*)(ws + round_up(mhc::proj16_phi_bytes(p->C), 256)), nullptr, dev_status, p->wait_ns,
+        (float*)(ws + round_up(mhc::proj16_phi_bytes(p->C), 256)), nullptr, nullptr, dev_status,
+        p->wait_ns,
         s));
   } else {
     st = from_cuda(mhc::map_fwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
@@ -250,8 +257,8 @@ mhc_status mhc_backward_map(const mhc_params* p, const void* x, const float* phi
     return from_cuda(mhc::wide_map_tc_dispatch(
         mhc::MAP_BWD, p->T, p->C, p->t_max, p->eps, x, phi, ws + w.phi_off, b, alpha,
         alpha_groups(p), nullptr, nullptr, nullptr, grad_x_next, grad_h_in, f_out, nullptr,
-        (float*)(ws + w.coef_off), (float*)(ws + w.part_off), dev_status, p->wait_ns,
-        (cudaStream_t)stream));
+        (float*)(ws + w.coef_off), (float*)(ws + w.part_off), (float*)(ws + w.apply_off),
+        dev_status, p->wait_ns, (cudaStream_t)stream));
   return from_cuda(mhc::map_bwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x, phi, b,
                                          alpha, alpha_groups(p), grad_x_next, grad_h_in, f_out, nullptr,
                                          (float*)(ws + w.coef_off), (float*)(ws + w.part_off),
@@ -365,7 +372,8 @@ mhc_status mhc_post_fused(const mhc_params* p, const void* x, const void* f_out,
     return from_cuda(mhc::wide_map_tc_dispatch(
         mhc::MAP_FWD, p->T, p->C, p->t_max, p->eps, x_next, phi_next, ws, b_next, alpha_next,
         alpha_groups(p), H_pre_next, H_post_next, H_res_next, nullptr, nullptr, nullptr, nullptr,
-        (float*)(ws + round_up(mhc::proj16_phi_bytes(p->C), 256)), nullptr, dev_status, p->wait_ns,
+        (float*)(ws + round_up(mhc::proj16_phi_bytes(p->C), 256)), nullptr, nullptr, dev_status,
+        p->wait_ns,
         s));
   }
   return from_cuda(mhc::map_fwd_dispatch(p->n, p->dtype, p->T, p->C, p->t_max, p->eps, x_next,
@@ -450,7 +458,8 @@ mhc_status mhc_pre_backward(const mhc_params* p, const void* x, const float* phi
     st = from_cuda(mhc::wide_map_tc_dispatch(
         mhc::MAP_BWD_SPLIT, p->T, p->C, p->t_max, p->eps, x, phi, ws + w.phi_off, b, alpha,
         alpha_groups(p), nullptr, nullptr, nullptr, nullptr, grad_h_in, nullptr, red,
-        (float*)(ws + w.coef_off), (float*)(ws + w.part_off), dev_status, p->wait_ns, s));
+        (float*)(ws + w.coef_off), (float*)(ws + w.part_off), (float*)(ws + w.apply_off),
+        dev_status, p->wait_ns, s));
     if (st != MHC_OK) return st;
     return from_cuda(mhc::apply16_tc_dispatch(
         p->T, p->C, x, ws + w.phi_off, grad_x_next, grad_h_in, (const float*)(ws + w.coef_off),

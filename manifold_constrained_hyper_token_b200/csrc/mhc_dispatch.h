@@ -89,13 +89,15 @@ size_t proj16_phi_bytes(int64_t C);
 // k_wide.cu, bf16 with n = 16: the mapping with the projection on the tensor
 // cores (proj16_dispatch) and the rest of the k_wide kernels: MAP_FWD writes
 // the maps (rows: [T][Coef<16>::SIZE] scratch); MAP_BWD / MAP_BWD_SPLIT write
-// the coefficient records into rows (= coef) and the partial sums.
+// the coefficient records into rows (= coef) and the partial sums, keeping the
+// Sinkhorn checkpoints in ck (wide_ck_bytes(T, iters) bytes; unused forward).
 cudaError_t wide_map_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float eps,
                                  const void* x, const float* phi, void* phi_t, const float* b,
                                  const float* alpha, int ag, float* Hpre, float* Hpost,
                                  float* Hres, const void* G, const void* g, const void* f,
-                                 const float* red, float* rows, float* part, int* st,
+                                 const float* red, float* rows, float* part, float* ck, int* st,
                                  int64_t wait_ns, cudaStream_t s);
+size_t wide_ck_bytes(int64_t T, int iters);
 
 // k_apply16_tc.cu (bf16, n = 16): the apply with phi u and grad_phi on the
 // tensor cores.  coef / part: the n = 16 mapping's records and partial sums;
