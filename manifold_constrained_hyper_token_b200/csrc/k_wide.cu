@@ -29,11 +29,11 @@
 //   k_wide_apply_phi  grad_phi = sum_t x_t u_t^T, a GEMM over the tokens
 //   k_wide_bias       grad_b and grad_alpha from the mapping CTAs' partials
 //
-// With bf16 activations the projection runs on the tensor cores instead
-// (k_proj16_tc.cu writes y and the sum of squares into the rows; here
-// k_wide_fwd_epi runs the forward's epilogue from them, and k_wide_map in its
-// PROJ = false form adds only the backward's C-reductions), and so does the
-// apply (k_apply16_tc.cu; k_wide_bias supplies its grad_b and grad_alpha).
+// With bf16 activations the projection, the backward's C-reductions and the
+// apply run on the tensor cores instead (k_proj16_tc.cu writes y and the sum of
+// squares into the rows, k_dots16_tc.cu the C-reductions; here k_wide_fwd_epi
+// and k_wide_bwd_epi run the epilogues from those rows; k_apply16_tc.cu is the
+// apply, with k_wide_bias for its grad_b and grad_alpha).
 //
 // Every sum is taken in a fixed order, so repeated calls give identical bits.
 // The per-token Sinkhorn arrays (16 x 16) live in local memory.
@@ -257,10 +257,7 @@ __device__ __forceinline__ void wide_epilogue(int tid, int64_t t, int64_t T, int
 // MAP_FWD: H_pre / H_post / H_res.  MAP_BWD: coef [T][Coef<16>::SIZE] and per
 // CTA the sums over its tokens of dz and dz . y (part [grid][DZ_SIZE]).
 // MAP_BWD_SPLIT: as MAP_BWD with <G_i, x_j> and <G_i, f_out> from `red`.
-// PROJ = false (backward only): the projection and the sum of squares are
-// already in the rows (the tensor-core projection of bf16 inputs wrote them);
-// only the C-reductions run here.
-template <typename TIO, int MODE, bool PROJ = true>
+template <typename TIO, int MODE>
 __global__ void __launch_bounds__(widek::NT) k_wide_map(
     int64_t T, int64_t C, int iters, float eps, const TIO* __restrict__ x,
     const float* __restrict__ phi, const float* __restrict__ bias,
@@ -282,8 +279,7 @@ __global__ void __launch_bounds__(widek::NT) k_wide_map(
   const int64_t K = (int64_t)N * C;
 
   // ---- projection y[t][m] = sum_k x[t][k] phi[k][m], and the sums of squares
-  static_assert(PROJ || BWD, "the forward projects");
-  if constexpr (PROJ) {
+  {
     float* xs = stg;            // [KC][TB]
     float* ps = stg + KC * TB;  // [KC][M]
     float acc[4][CPT], ssp[4];
@@ -783,35 +779,17 @@ cudaError_t wide_map_tc_dispatch(int mode, int64_t T, int64_t C, int iters, floa
                                        st);
     return cudaGetLastError();
   }
-  const size_t smem = (size_t)widek::SMEM_FLOATS * 4;
-  using BF = __nv_bfloat16;
-  if (mode == MAP_BWD) {
-    auto kern = k_wide_map<BF, MAP_BWD, false>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    kern<<<grid, widek::NT, smem, s>>>(T, C, iters, eps, (const BF*)x, phi, b, alpha, ag, nullptr,
-                                       nullptr, nullptr, (const BF*)G, (const BF*)g, (const BF*)f,
-                                       red, rows, part, st);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+  if (mode != MAP_BWD && mode != MAP_BWD_SPLIT) return cudaErrorInvalidValue;
+  // the C-reductions on the tensor cores (k_dots16_tc.cu), then the epilogue
+  e = dots16_dispatch(mode == MAP_BWD, T, C, x, G, g, f, rows, st, wait_ns, s);
+  if (e != cudaSuccess) return e;
+  if (mode == MAP_BWD)
     k_wide_bwd_epi<MAP_BWD><<<grid, 32, 0, s>>>(T, C, iters, eps, b, alpha, ag, red, rows, part,
                                                 st, ck);
-    return cudaGetLastError();
-  }
-  if (mode == MAP_BWD_SPLIT) {
-    auto kern = k_wide_map<BF, MAP_BWD_SPLIT, false>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    kern<<<grid, widek::NT, smem, s>>>(T, C, iters, eps, (const BF*)x, phi, b, alpha, ag, nullptr,
-                                       nullptr, nullptr, (const BF*)G, (const BF*)g, (const BF*)f,
-                                       red, rows, part, st);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+  else
     k_wide_bwd_epi<MAP_BWD_SPLIT><<<grid, 32, 0, s>>>(T, C, iters, eps, b, alpha, ag, red, rows,
                                                       part, st, ck);
-    return cudaGetLastError();
-  }
-  return cudaErrorInvalidValue;
+  return cudaGetLastError();
 }
 
 cudaError_t wide_map_dispatch(int mode, int dtype, int64_t T, int64_t C, int iters, float eps,
