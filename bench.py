@@ -446,8 +446,9 @@ def run_layer(args, dev, rank, world, local_rank):
     # phi split + projection + reductions + epilogue
     launches_per_call = {"pre": 3, "post": 1, "layer_input": 1, "post_fused": 2, "bwd_map": 2,
                          "bwd_apply": 1 if n == N_STR else 3}
-    if n == 8:  # the fused post is k_post, then the phi split and the mapping
-        launches_per_call["post_fused"] = 3
+    if n == 8:  # the fused post is k_post, then the phi split and the mapping; the
+        # backward mapping is the phi split, the tensor-core reductions, the mapping
+        launches_per_call.update({"post_fused": 3, "bwd_map": 3})
     if n == 16:  # the apply: U rows, phi u, grad_x, grad_phi, bias sums
         launches_per_call.update({"pre": 4, "bwd_map": 4, "post_fused": 4, "bwd_apply": 5})
     # the layer's maps; in a stack the previous layer's post_fused computes them

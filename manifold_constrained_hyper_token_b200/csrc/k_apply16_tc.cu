@@ -294,7 +294,7 @@ __global__ void __launch_bounds__(ap16::A_NT, 1) k_phiu16(
 // ------------------------------------------------------- grad_x, grad_f_out
 // One CTA visit per token: its coefficient record in shared memory, its
 // threads over 4-channel vectors of all sixteen streams.
-__global__ void __launch_bounds__(128) k_gx16(int64_t T, int64_t C,
+__global__ void __launch_bounds__(128, 4) k_gx16(int64_t T, int64_t C,
                                               const __nv_bfloat16* __restrict__ x,
                                               const __nv_bfloat16* __restrict__ G,
                                               const __nv_bfloat16* __restrict__ g,

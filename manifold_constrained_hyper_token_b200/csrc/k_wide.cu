@@ -31,7 +31,7 @@
 //
 // With bf16 activations the projection, the backward's C-reductions and the
 // apply run on the tensor cores instead (k_proj16_tc.cu writes y and the sum of
-// squares into the rows, k_dots16_tc.cu the C-reductions; here k_wide_fwd_epi
+// squares into the rows, k_dots_tc.cu the C-reductions; here k_wide_fwd_epi
 // and k_wide_bwd_epi run the epilogues from those rows; k_apply16_tc.cu is the
 // apply, with k_wide_bias for its grad_b and grad_alpha).
 //
@@ -780,7 +780,7 @@ cudaError_t wide_map_tc_dispatch(int mode, int64_t T, int64_t C, int iters, floa
     return cudaGetLastError();
   }
   if (mode != MAP_BWD && mode != MAP_BWD_SPLIT) return cudaErrorInvalidValue;
-  // the C-reductions on the tensor cores (k_dots16_tc.cu), then the epilogue
+  // the C-reductions on the tensor cores (k_dots_tc.cu), then the epilogue
   e = dots16_dispatch(mode == MAP_BWD, T, C, x, G, g, f, rows, st, wait_ns, s);
   if (e != cudaSuccess) return e;
   if (mode == MAP_BWD)

@@ -86,12 +86,16 @@ cudaError_t proj16_dispatch(int64_t T, int64_t C, const void* x, const float* ph
                             float* rows, int64_t ostride, int* st, int64_t wait_ns,
                             cudaStream_t s);
 size_t proj16_phi_bytes(int64_t C);
-// k_dots16_tc.cu (bf16, n = 16): the backward's C-reductions per token into
-// rows [T][Coef<16>::SIZE] at [288 + d]: full = all 288 (<G_i, x_j> on the
-// tensor cores, <g, x_i>, <G_i, f>); otherwise <g, x_i> only (split backward).
+// k_dots_tc.cu (bf16): the backward's C-reductions per token.  n = 16: into
+// rows [T][Coef<16>::SIZE] at [288 + d]; full = all 288 (<G_i, x_j> on the
+// tensor cores, <g, x_i>, <G_i, f>), otherwise <g, x_i> only (split backward).
+// n = 8: <G_i, x_j> (tensor cores) and <G_i, f> into red [T][72], the layout
+// the n = 8 mapping's split mode reads.
 cudaError_t dots16_dispatch(bool full, int64_t T, int64_t C, const void* x, const void* G,
                             const void* g, const void* f, float* rows, int* st, int64_t wait_ns,
                             cudaStream_t s);
+cudaError_t dots8_red_dispatch(int64_t T, int64_t C, const void* x, const void* G, const void* f,
+                               float* red, int* st, int64_t wait_ns, cudaStream_t s);
 // k_wide.cu, bf16 with n = 16: the mapping with the projection on the tensor
 // cores (proj16_dispatch) and the rest of the k_wide kernels: MAP_FWD writes
 // the maps (rows: [T][Coef<16>::SIZE] scratch); MAP_BWD / MAP_BWD_SPLIT write
