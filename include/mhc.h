@@ -195,11 +195,13 @@ MHC_API mhc_status mhc_backward(const mhc_params *p, const void *x, const float 
  * mhc_backward_map: recomputes the mapping and reduces the per-token
  *   C-contractions <grad_h_in, x_i>, <grad_x_next_i, f_out>,
  *   <grad_x_next_i, x_j>; runs the Sinkhorn adjoint and the gate derivatives
- *   (reportify.cn [19]); writes per-token coefficients and per-64-token
- *   partial sums of dz and dz . y into the workspace.
+ *   (reportify.cn [19]); writes per-token coefficient records and one
+ *   partial-sum record of dz and dz . y per mapping CTA into the workspace.
  * mhc_backward_apply: from those records writes grad_x, grad_f_out and
- *   grad_phi (each row of grad_phi summed over all T tokens by one CTA) and
- *   finishes grad_b and grad_alpha; all sums in a fixed order.
+ *   grad_phi (every row of grad_phi summed over all T tokens) and finishes
+ *   grad_b and grad_alpha; all sums in a fixed order.  It reads the records
+ *   and also uses the rest of the workspace as its own scratch (the const
+ *   qualifier states that the records are only read).
  * Arguments, layouts and errors are those of mhc_backward.
  */
 MHC_API mhc_status mhc_backward_map(const mhc_params *p, const void *x, const float *phi,
