@@ -9,10 +9,12 @@
 // recompute in the backward).
 //
 // One CTA = 128 tokens (the MMA M).  The token's n*C inputs stream through a
-// TMA ring in chunks of 32 channels x 4 streams (64-byte rows and swizzle; a
-// TMA row piece narrower than 64 bytes caps an SM's streaming rate): per
-// stream an x tile [128 x 32] (the MMA A operand, K-major) and the matching
-// rows of phi^T as a [48 x 32] B operand, whose 48 rows are the
+// TMA ring in chunks of 64 channels x 4 streams in the forward modes (128-byte
+// rows and swizzle, two stages) and of 32 channels x 4 streams in the backward
+// modes (64-byte rows; a TMA row piece narrower than 64 bytes caps an SM's
+// streaming rate): per stream an x tile [128 x CH] (the MMA A operand,
+// K-major) and the matching rows of phi^T as a [48 x CH] B operand, whose 48
+// rows are the
 // 24 logit columns split into a bf16 high part and a bf16 low part
 // (phi = hi + lo), so y = D[:, m] + D[:, 24 + m] carries phi to ~16 bits.
 // x itself is bf16, so the products are exact and only the fp32
@@ -59,11 +61,17 @@ constexpr int KREC = 52;             // floats per part record: y[24] | ss | dot
 // tensor cores project it, a store warp writes it out).
 template <int MODE> struct Cfg {
   static constexpr bool FULLB = MODE == MAP_BWD;
-  static constexpr int CH = 32;                 // channels per chunk: 64-byte rows
+  // channels per chunk: the forward modes stream 128-byte rows (half the row
+  // requests of 64-byte rows; the fused post merge also stores every row it
+  // loads), the backward modes 64-byte rows (their stages hold two or four
+  // tensors).  Both forward modes use the same chunks, so mhc_post_fused
+  // reproduces mhc_post -> mhc_pre bit for bit.
+  static constexpr int CH = MODE == MAP_FWD || MODE == MAP_POSTFWD ? 64 : 32;
   static constexpr int ROW = CH * 2;            // bytes per tile row = swizzle span
   static constexpr int XBOX = TM * CH * 2;      // one stream's x tile
   static constexpr int PBOX = NL * CH * 2;      // one stream's phi^T tile
-  static constexpr int NS = FULLB ? 2 : 4;      // pipeline stages (MAP_BWD stages 4 tensors)
+  // pipeline stages (MAP_BWD stages 4 tensors; the 128-byte-row stages are twice as big)
+  static constexpr int NS = FULLB || CH == 64 ? 2 : 4;
   static constexpr int X_OFF = 0;
   static constexpr int P_OFF = N * XBOX;
   static constexpr int G_OFF = P_OFF + N * PBOX;                 // grad_x_next tiles (MAP_BWD)
@@ -109,12 +117,15 @@ __device__ __forceinline__ void bf16x8_to_f32(uint4 q, float (&v)[8]) {
 }
 
 // Row `tok`, 16-byte chunk `chunk` of a bf16 tile whose rows are ROW bytes
-// and stored with the ROW-byte swizzle: 64-byte rows put chunk c at
-// c ^ ((tok >> 1) & 3), 32-byte rows at c ^ ((tok >> 2) & 1).
+// and stored with the ROW-byte swizzle: 128-byte rows put chunk c at
+// c ^ (tok & 7), 64-byte rows at c ^ ((tok >> 1) & 3), 32-byte rows at
+// c ^ ((tok >> 2) & 1).
 template <int ROW>
 __device__ __forceinline__ int sw_off(int tok, int chunk) {
-  static_assert(ROW == 32 || ROW == 64, "row width");
-  const int phys = ROW == 64 ? chunk ^ ((tok >> 1) & 3) : chunk ^ ((tok >> 2) & 1);
+  static_assert(ROW == 32 || ROW == 64 || ROW == 128, "row width");
+  const int phys = ROW == 128 ? chunk ^ (tok & 7)
+                   : ROW == 64 ? chunk ^ ((tok >> 1) & 3)
+                               : chunk ^ ((tok >> 2) & 1);
   return tok * ROW + phys * 16;
 }
 template <int ROW>
@@ -148,7 +159,7 @@ __global__ void __launch_bounds__(tcmap::NT, 1) k_map_tc(
   constexpr bool POST = MODE == MAP_POSTFWD;
   constexpr int NS = CFG::NS;
   constexpr int CH = CFG::CH, XBOX = CFG::XBOX, PBOX = CFG::PBOX, ROW = CFG::ROW;
-  constexpr tc::Swz SWZ = ROW == 64 ? tc::SWZ_64B : tc::SWZ_32B;
+  constexpr tc::Swz SWZ = ROW == 128 ? tc::SWZ_128B : (ROW == 64 ? tc::SWZ_64B : tc::SWZ_32B);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
@@ -631,10 +642,11 @@ static cudaError_t encode_maps(int mode, int64_t T, int64_t C, const void* x, co
                                const void* G, const void* g, const void* f, CUtensorMap* mx,
                                CUtensorMap* mp, CUtensorMap* mG, CUtensorMap* mg, CUtensorMap* mf) {
   using namespace tcmap;
-  const uint32_t CH = Cfg<MAP_FWD>::CH;
-  const CUtensorMapSwizzle SW = CU_TENSOR_MAP_SWIZZLE_64B;
-  static_assert(Cfg<MAP_FWD>::CH == Cfg<MAP_BWD>::CH && Cfg<MAP_BWD>::CH == Cfg<MAP_BWD_SPLIT>::CH,
-                "one chunk width for every mode");
+  static_assert(Cfg<MAP_FWD>::CH == Cfg<MAP_POSTFWD>::CH && Cfg<MAP_BWD>::CH == Cfg<MAP_BWD_SPLIT>::CH,
+                "one chunk width per direction");
+  const bool wide = mode == MAP_FWD || mode == MAP_POSTFWD;  // 128-byte rows (x and phi)
+  const uint32_t CH = wide ? Cfg<MAP_FWD>::CH : Cfg<MAP_BWD>::CH;
+  const CUtensorMapSwizzle SW = wide ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   const uint64_t dx[3] = {(uint64_t)C, (uint64_t)N, (uint64_t)T};
   const uint64_t sx[2] = {(uint64_t)C * 2, (uint64_t)N * C * 2};
   const uint32_t bx[3] = {CH, 1, TM};
@@ -651,7 +663,7 @@ static cudaError_t encode_maps(int mode, int64_t T, int64_t C, const void* x, co
   const uint64_t d2[2] = {(uint64_t)C, (uint64_t)T};
   const uint64_t s2[1] = {(uint64_t)C * 2};
   const uint32_t b2[2] = {CH, TM};
-  if (mode != MAP_FWD) {
+  if (mode != MAP_FWD && mode != MAP_POSTFWD) {
     e = make_tmap_bf16(mg, g, 2, d2, s2, b2, SW);
     if (e != cudaSuccess) return e;
   }
@@ -697,7 +709,8 @@ static int map_device_sms() {
 static int map_tc_kp(int64_t T, int64_t C) {
   using namespace tcmap;
   const int64_t ntt = (T + TM - 1) / TM;
-  const int nch = (int)((C + Cfg<MAP_FWD>::CH - 1) / Cfg<MAP_FWD>::CH);
+  constexpr int kModelCh = 32;  // the cost model counts 32-channel chunks
+  const int nch = (int)((C + kModelCh - 1) / kModelCh);
   const int sms = map_device_sms();
   constexpr double kFixedChunks = 8.0;
   int kmax = nch / 4;
@@ -809,17 +822,18 @@ cudaError_t post_map_tc_dispatch(int64_t T, int64_t C, int iters, float eps, con
   if (e != cudaSuccess) return e;
   CUtensorMap mx, mp, mG, mg, mf;
   // the forward maps for x and phi, then x_next (store) and f_out
-  e = encode_maps(MAP_FWD, T, C, x, phi_split, nullptr, nullptr, nullptr, &mx, &mp, &mG, &mg, &mf);
+  e = encode_maps(MAP_POSTFWD, T, C, x, phi_split, nullptr, nullptr, nullptr, &mx, &mp, &mG, &mg,
+                  &mf);
   if (e != cudaSuccess) return e;
   const uint64_t dx[3] = {(uint64_t)C, (uint64_t)N, (uint64_t)T};
   const uint64_t sx[2] = {(uint64_t)C * 2, (uint64_t)N * C * 2};
   const uint32_t bx[3] = {(uint32_t)Cfg<MAP_POSTFWD>::CH, 1, TM};
-  e = make_tmap_bf16(&mG, x_next, 3, dx, sx, bx, CU_TENSOR_MAP_SWIZZLE_64B);
+  e = make_tmap_bf16(&mG, x_next, 3, dx, sx, bx, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
   const uint64_t d2[2] = {(uint64_t)C, (uint64_t)T};
   const uint64_t s2[1] = {(uint64_t)C * 2};
   const uint32_t b2[2] = {(uint32_t)Cfg<MAP_POSTFWD>::CH, TM};
-  e = make_tmap_bf16(&mf, f, 2, d2, s2, b2, CU_TENSOR_MAP_SWIZZLE_64B);
+  e = make_tmap_bf16(&mf, f, 2, d2, s2, b2, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
   return launch_map_tc<MAP_POSTFWD>(mx, mp, mG, mg, mf, T, C, iters, eps, b_next, alpha_next, ag, Hpre,
                                     Hpost, Hres, nullptr, nullptr, nullptr, nullptr, kscratch, st,
