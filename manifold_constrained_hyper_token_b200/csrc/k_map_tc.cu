@@ -9,10 +9,10 @@
 // recompute in the backward).
 //
 // One CTA = 128 tokens (the MMA M).  The token's n*C inputs stream through a
-// TMA ring in chunks of 64 channels x 4 streams in the forward modes (128-byte
-// rows and swizzle, two stages) and of 32 channels x 4 streams in the backward
-// modes (64-byte rows; a TMA row piece narrower than 64 bytes caps an SM's
-// streaming rate): per stream an x tile [128 x CH] (the MMA A operand,
+// TMA ring in chunks of 64 channels x 4 streams in the forward and split
+// backward modes (128-byte rows and swizzle, two stages) and of 32 channels x 4
+// streams in the full backward (64-byte rows; a TMA row piece narrower than 64
+// bytes caps an SM's streaming rate): per stream an x tile [128 x CH] (the MMA A operand,
 // K-major) and the matching rows of phi^T as a [48 x CH] B operand, whose 48
 // rows are the
 // 24 logit columns split into a bf16 high part and a bf16 low part
@@ -61,12 +61,12 @@ constexpr int KREC = 52;             // floats per part record: y[24] | ss | dot
 // tensor cores project it, a store warp writes it out).
 template <int MODE> struct Cfg {
   static constexpr bool FULLB = MODE == MAP_BWD;
-  // channels per chunk: the forward modes stream 128-byte rows (half the row
-  // requests of 64-byte rows; the fused post merge also stores every row it
-  // loads), the backward modes 64-byte rows (their stages hold two or four
-  // tensors).  Both forward modes use the same chunks, so mhc_post_fused
-  // reproduces mhc_post -> mhc_pre bit for bit.
-  static constexpr int CH = MODE == MAP_FWD || MODE == MAP_POSTFWD ? 64 : 32;
+  // channels per chunk: the forward modes and the split backward stream
+  // 128-byte rows (half the row requests of 64-byte rows; the fused post merge
+  // also stores every row it loads), the full backward 64-byte rows (its
+  // stages hold four tensors).  Both forward modes use the same chunks, so
+  // mhc_post_fused reproduces mhc_post -> mhc_pre bit for bit.
+  static constexpr int CH = MODE == MAP_BWD ? 32 : 64;
   static constexpr int ROW = CH * 2;            // bytes per tile row = swizzle span
   static constexpr int XBOX = TM * CH * 2;      // one stream's x tile
   static constexpr int PBOX = NL * CH * 2;      // one stream's phi^T tile
@@ -642,9 +642,10 @@ static cudaError_t encode_maps(int mode, int64_t T, int64_t C, const void* x, co
                                const void* G, const void* g, const void* f, CUtensorMap* mx,
                                CUtensorMap* mp, CUtensorMap* mG, CUtensorMap* mg, CUtensorMap* mf) {
   using namespace tcmap;
-  static_assert(Cfg<MAP_FWD>::CH == Cfg<MAP_POSTFWD>::CH && Cfg<MAP_BWD>::CH == Cfg<MAP_BWD_SPLIT>::CH,
-                "one chunk width per direction");
-  const bool wide = mode == MAP_FWD || mode == MAP_POSTFWD;  // 128-byte rows (x and phi)
+  static_assert(Cfg<MAP_FWD>::CH == Cfg<MAP_POSTFWD>::CH &&
+                    Cfg<MAP_FWD>::CH == Cfg<MAP_BWD_SPLIT>::CH,
+                "one chunk width for the 128-byte-row modes");
+  const bool wide = mode != MAP_BWD;  // 128-byte rows
   const uint32_t CH = wide ? Cfg<MAP_FWD>::CH : Cfg<MAP_BWD>::CH;
   const CUtensorMapSwizzle SW = wide ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   const uint64_t dx[3] = {(uint64_t)C, (uint64_t)N, (uint64_t)T};
