@@ -69,6 +69,28 @@ def test_workspace_size_query(lib):
     assert lib.mhc_pre_workspace_size(ctypes.byref(p)) >= 0
 
 
+@pytest.mark.parametrize("n", [8, 16])
+def test_wide_tensor_core_workspaces(lib, n):
+    """bf16 with n = 8 or 16 takes the tensor-core paths: mhc_pre needs the split phi^T
+    copy (2M rows of nC bf16; at n = 16 also the per-token rows of projections, 580
+    floats each), and the backward holds the apply's fp32 phi u scratch [T][n][C] on
+    top of the per-token records.  fp32 activations take the CUDA-core paths, whose
+    forward needs no workspace."""
+    T, C = 4096, 7168
+    M = n * n + 2 * n
+    bf = _params(n=n, T=T, C=C, dtype=1)
+    pre = lib.mhc_pre_workspace_size(ctypes.byref(bf))
+    assert pre >= 2 * M * n * C * 2 and pre % 256 == 0
+    if n == 16:
+        assert pre >= 2 * M * n * C * 2 + T * 580 * 4
+    assert lib.mhc_post_fused_workspace_size(ctypes.byref(bf)) == pre
+    bwd = lib.mhc_backward_workspace_size(ctypes.byref(bf))
+    assert bwd >= T * n * C * 4 + 2 * M * n * C * 2 and bwd % 256 == 0
+    f32 = _params(n=n, T=T, C=C, dtype=0)
+    assert lib.mhc_pre_workspace_size(ctypes.byref(f32)) == 0
+    assert 0 < lib.mhc_backward_workspace_size(ctypes.byref(f32)) < bwd
+
+
 FAKE = ctypes.c_void_p(0x10000)   # 16-byte aligned, never dereferenced (validation fails first)
 ODD = ctypes.c_void_p(0x10004)
 
