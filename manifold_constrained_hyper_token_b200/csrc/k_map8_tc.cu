@@ -14,7 +14,12 @@
 // swizzle): per stream an x tile [128 x 16] (the A operand, K-major) and the
 // rows of the bf16 split copy of phi^T as a [160 x 16] B operand -- the 80
 // logit columns' high parts, then their low parts (phi = hi + lo) -- so
-// y = D[:, m] + D[:, 80 + m] carries phi to ~16 bits while x is exact.
+// y = D[:, m] + D[:, 80 + m] carries phi to ~16 bits while x is exact.  The
+// split copy is tiled and pre-swizzled, so a chunk's eight phi tiles (40 KB)
+// arrive as one bulk copy.  The library runs the whole backward in the split
+// mode: <G_i, x_j> and <G_i, f_out> come from the tensor-core reductions of
+// k_dots_tc.cu (or the post half of the training-order backward), and this
+// kernel adds <g, x_j>.
 //
 // Warp roles: warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs, warps
 // 2..9 reduce: warp 2 + 4h + q covers token rows 32q..32q+31 and stream half
