@@ -592,6 +592,33 @@ def test_n8_forward_backward_large(mhc, oracle_mod):
     assert_close(_np(ga), np.array([full["grad_alpha"]]), 2e-2)
 
 
+@pytest.mark.slow
+def test_n16_forward_backward_large(mhc, oracle_mod):
+    """T=200, n=16, C=7168 bf16 forward + backward: the n = 16 tensor-core kernels at
+    the bench's channel count (112 projection chunks, 28 phi u channel blocks, 56
+    grad_phi blocks, C-reduction slabs of 8 tokens) and a ragged second token tile,
+    every output against the oracle."""
+    from manifold_constrained_hyper_token_b200 import synth
+    T, n, C = 200, 16, 7168
+    d = synth.layer_inputs(T, n, C, seed=6, dtype=torch.bfloat16, backward=True)
+    dd = _dev(d)
+    alpha = float(d["alpha"][0])
+    st = _status()
+    h_in, Hpre, Hpost, Hres = mhc.mhc_pre(dd["x"], dd["phi"], dd["b"], dd["alpha"], dev_status=st)
+    gx, gphi, gb, ga, gf = mhc.mhc_backward(dd["x"], dd["phi"], dd["b"], dd["alpha"], dd["f_out"],
+                                            dd["grad_x_next"], dd["grad_h_in"], dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ref = oracle_mod.pre(d["x"], d["phi"], d["b"], alpha)
+    for k, got in (("h_in", h_in), ("H_pre", Hpre), ("H_post", Hpost), ("H_res", Hres)):
+        assert_close(_np(got), ref[k], 2e-2, k)
+    rb = oracle_mod.backward(d["x"], d["phi"], d["b"], alpha, d["f_out"], d["grad_x_next"],
+                             d["grad_h_in"])
+    for k, got in (("grad_x", gx), ("grad_f_out", gf), ("grad_phi", gphi), ("grad_b", gb)):
+        assert_close(_np(got), rb[k], 2e-2, k)
+    assert_close(_np(ga), np.array([rb["grad_alpha"]]), 2e-2, "grad_alpha")
+
+
 # ------------- bf16 n = 4 mapping with each 128-token tile cut into channel
 # parts (one CTA each, records added by the tile's last part in part order)
 # whenever one CTA per tile would leave SMs idle.  (T, C): several parts per
