@@ -96,9 +96,10 @@ typedef enum mhc_dtype {
 /* Problem description shared by mhc_pre / mhc_post / mhc_backward. */
 typedef struct mhc_params {
   int32_t n;      /* streams; the library supports n in {1, 2, 4, 8, 16}; bf16
-                     with n = 4 runs the tensor-core kernels, n = 16 its own
-                     CUDA-core kernels (288 logits per token), the rest the
-                     CUDA-core kernels; mhc_backward_noalloc takes n <= 8    */
+                     with n = 4, 8 or 16 runs tensor-core kernels (n = 16 with
+                     its own CUDA-core epilogues, 288 logits per token), fp32
+                     and n <= 2 the CUDA-core kernels; mhc_backward_noalloc
+                     takes n <= 8 and runs the CUDA-core kernels             */
   int32_t t_max;  /* Sinkhorn-Knopp iterations (row then column pass), >= 0   */
   int64_t T;      /* tokens, 1 <= T <= 2^31 - 257 (32-bit tile coordinates)    */
   int64_t C;      /* channels per stream, >= 8 and a multiple of 8            */

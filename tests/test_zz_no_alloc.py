@@ -56,7 +56,7 @@ def _noalloc_via_abi(d, t_max=20, eps=1e-6, out=None):
 # second must not see anything the first left in the shared scratch); n = 8
 # with T = 6000 needs 3.9 MB of the 4 MiB array (656-byte records per token)
 CASES = {4: ((1000, 4, 1024, 1), (333, 4, 512, 2)),
-         8: ((1000, 8, 64, 3), (100, 8, 256, 4)),
+         8: ((6000, 8, 64, 3), (100, 8, 256, 4)),
          2: ((2000, 2, 512, 5), (77, 2, 64, 6))}
 
 
