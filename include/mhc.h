@@ -101,7 +101,8 @@ typedef struct mhc_params {
                      and n <= 2 the CUDA-core kernels; mhc_backward_noalloc
                      takes n <= 8 and runs the CUDA-core kernels             */
   int32_t t_max;  /* Sinkhorn-Knopp iterations (row then column pass), >= 0   */
-  int64_t T;      /* tokens, 1 <= T <= 2^31 - 257 (32-bit tile coordinates)    */
+  int64_t T;      /* tokens, 1 <= T <= 2^31 - 257 (32-bit tile coordinates;
+                     bf16 with n >= 8: T * n <= 2^31 - 257)                  */
   int64_t C;      /* channels per stream, >= 8 and a multiple of 8            */
   float eps;      /* RMS epsilon added to the mean square, >= 0               */
   int32_t dtype;  /* mhc_dtype of x, f_out, h_in, x_next and the activation

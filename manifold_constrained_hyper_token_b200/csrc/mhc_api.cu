@@ -25,8 +25,11 @@ mhc_status check_params(const mhc_params* p) {
     return MHC_ERR_INVALID_ARG;
   if (p->wait_ns < 0) return MHC_ERR_INVALID_ARG;
   // tile coordinates of the TMA copies are 32-bit signed: keep T (and a tile
-  // past it) inside that range
+  // past it) inside that range; the bf16 n = 8 and n = 16 backward reductions
+  // address x and grad_x_next as T*n rows
   if (p->T > (int64_t)0x7fffffffLL - 256) return MHC_ERR_INVALID_ARG;
+  if (p->dtype == MHC_DTYPE_BF16 && p->n >= 8 && p->T * p->n > (int64_t)0x7fffffffLL - 256)
+    return MHC_ERR_INVALID_ARG;
   return MHC_OK;
 }
 

@@ -100,6 +100,7 @@ ODD = ctypes.c_void_p(0x10004)
     (dict(eps=-1.0), 1),
     (dict(eps=float("nan")), 1), (dict(n=3), 2), (dict(n=32), 2), (dict(dtype=7), 2),
     (dict(alpha_groups=2), 1), (dict(wait_ns=-1), 1),
+    (dict(n=16, T=2**31 // 16), 1), (dict(n=8, T=2**31 // 8), 1),
 ])
 def test_pre_rejects_bad_params(lib, kw, code):
     p = _params(**kw)
