@@ -10,9 +10,9 @@
 //           (d < 256: i = d / 16, j = d % 16; then <g, x_i>, then <G_i, f>),
 //           where the backward epilogue of k_wide.cu reads them; the split
 //           backward (training order) needs only <g, x_i>;
-//   n = 8:  <G_i, x_j> and <G_i, f> into rows [T][72] in the layout of the post
-//           half's reductions (i*8 + j, then 64 + i), which the n = 8 mapping
-//           reads in its split mode; it adds <g, x_j> itself.
+//   n = 8:  all 80 into rows [T][80] (<G_i, x_j> at i*8 + j, <G_i, f> at
+//           64 + i, <g, x_j> at 72 + j), which the n = 8 mapping reads in its
+//           MAP_BWD_DOTS mode.
 //
 // The n*n products <G_i, x_j> of a token are an n x n matrix product over the
 // channels.  128 / n consecutive tokens' stream rows are 128 consecutive rows
@@ -33,14 +33,14 @@
 namespace mhc {
 
 // Modes: DOTS_FULL16 (n = 16, all 288), DOTS_GX16 (n = 16, <g, x_i> only),
-// DOTS_RED8 (n = 8, <G_i, x_j> and <G_i, f>).
+// DOTS_RED8 (n = 8, all 80).
 enum DotsMode { DOTS_FULL16 = 0, DOTS_GX16 = 1, DOTS_RED8 = 2 };
 
 template <int MODE> struct DotsCfg {
   static constexpr int N = MODE == DOTS_RED8 ? 8 : 16;
   static constexpr bool MMA = MODE != DOTS_GX16;    // <G_i, x_j> on the tensor cores
   static constexpr bool USE_G = MODE != DOTS_GX16;
-  static constexpr bool USE_g = MODE != DOTS_RED8;  // <g, x_i>
+  static constexpr bool USE_g = true;               // <g, x_i>
   static constexpr bool USE_f = MODE != DOTS_GX16;  // <G_i, f>
   static constexpr int TG = 128 / N;                // tokens per slab
   static constexpr int NG = 2;                      // slabs per CTA
@@ -80,7 +80,7 @@ __device__ __forceinline__ void dot8(uint4 a, uint4 b, float& acc) {
 }
 }  // namespace
 
-// rows: n = 16, [T][Coef<16>::SIZE] coefficient rows; n = 8, [T][72].
+// rows: n = 16, [T][Coef<16>::SIZE] coefficient rows; n = 8, [T][80].
 template <int MODE>
 __global__ void __launch_bounds__(DotsCfg<MODE>::NT, 1) k_dots_tc(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_G,
@@ -90,9 +90,9 @@ __global__ void __launch_bounds__(DotsCfg<MODE>::NT, 1) k_dots_tc(
   constexpr int N = D::N, NS = D::NS;
   // destination of token t's products: <G_i, x_j> at GX + i*N + j, <g, x_i> at
   // GV + i, <G_i, f> at GF + i in a row of RS floats
-  constexpr int RS = N == 16 ? Coef<16>::SIZE : N * N + N;
+  constexpr int RS = N == 16 ? Coef<16>::SIZE : N * N + 2 * N;
   constexpr int GX = N == 16 ? Coef<16>::M : 0;
-  constexpr int GV = GX + N * N;
+  constexpr int GV = N == 16 ? GX + N * N : N * N + N;
   constexpr int GF = N == 16 ? GX + N * N + N : N * N;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -331,9 +331,10 @@ cudaError_t dots16_dispatch(bool full, int64_t T, int64_t C, const void* x, cons
               : launch_dots<DOTS_GX16>(T, C, x, G, g, f, rows, st, wait_ns, s);
 }
 
-cudaError_t dots8_red_dispatch(int64_t T, int64_t C, const void* x, const void* G, const void* f,
-                               float* red, int* st, int64_t wait_ns, cudaStream_t s) {
-  return launch_dots<DOTS_RED8>(T, C, x, G, nullptr, f, red, st, wait_ns, s);
+cudaError_t dots8_red_dispatch(int64_t T, int64_t C, const void* x, const void* G, const void* g,
+                               const void* f, float* red, int* st, int64_t wait_ns,
+                               cudaStream_t s) {
+  return launch_dots<DOTS_RED8>(T, C, x, G, g, f, red, st, wait_ns, s);
 }
 
 }  // namespace mhc

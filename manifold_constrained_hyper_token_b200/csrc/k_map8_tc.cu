@@ -16,10 +16,11 @@
 // logit columns' high parts, then their low parts (phi = hi + lo) -- so
 // y = D[:, m] + D[:, 80 + m] carries phi to ~16 bits while x is exact.  The
 // split copy is tiled and pre-swizzled, so a chunk's eight phi tiles (40 KB)
-// arrive as one bulk copy.  The library runs the whole backward in the split
-// mode: <G_i, x_j> and <G_i, f_out> come from the tensor-core reductions of
-// k_dots_tc.cu (or the post half of the training-order backward), and this
-// kernel adds <g, x_j>.
+// arrive as one bulk copy.  The library's whole backward runs this kernel in
+// the MAP_BWD_DOTS mode (only x staged, three stages): every C-reduction comes
+// from the tensor-core reductions of k_dots_tc.cu.  The training-order
+// backward runs the split mode: <G_i, x_j> and <G_i, f_out> from the post
+// half, <g, x_j> here.
 //
 // Warp roles: warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs, warps
 // 2..9 reduce: warp 2 + 4h + q covers token rows 32q..32q+31 and stream half
@@ -53,14 +54,15 @@ constexpr int NDH = 4 * N + 4 + 4;   // reductions per stream half: <G_i,x_j> 32
 
 template <int MODE> struct Cfg {
   static constexpr bool FULLB = MODE == MAP_BWD;
-  static constexpr bool BWD = MODE == MAP_BWD || MODE == MAP_BWD_SPLIT;
+  static constexpr bool BWD = MODE == MAP_BWD || MODE == MAP_BWD_SPLIT || MODE == MAP_BWD_DOTS;
+  static constexpr bool STAGE_G = MODE == MAP_BWD || MODE == MAP_BWD_SPLIT;  // grad_h_in staged
   static constexpr int X_OFF = 0;
   static constexpr int P_OFF = N * XBOX;
   static constexpr int G_OFF = P_OFF + N * PBOX;                 // grad_x_next (full backward)
   static constexpr int GG_OFF = FULLB ? G_OFF + N * XBOX : G_OFF;  // grad_h_in (backward)
   static constexpr int F_OFF = GG_OFF + XBOX;                     // f_out (full backward)
-  static constexpr int STAGE = FULLB ? F_OFF + XBOX : (BWD ? GG_OFF + XBOX : G_OFF);
-  static constexpr int NS = BWD ? 2 : 3;
+  static constexpr int STAGE = FULLB ? F_OFF + XBOX : (STAGE_G ? GG_OFF + XBOX : G_OFF);
+  static constexpr int NS = STAGE_G ? 2 : 3;
   // the stages, reused after the chunk loop by the epilogue; the backward
   // epilogue keeps Sinkhorn checkpoints there, so the split backward (smaller
   // stages) asks for the full backward's size
@@ -107,6 +109,8 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
   using CF = Coef<N>;
   constexpr bool BWD = CFG::BWD, FULLB = CFG::FULLB;
   constexpr bool SPLIT = MODE == MAP_BWD_SPLIT;
+  constexpr bool DOTS = MODE == MAP_BWD_DOTS;  // every C-reduction from red_in
+  constexpr bool STAGE_G = CFG::STAGE_G;
   constexpr int NS = CFG::NS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -136,7 +140,7 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
   }
   if (warp == 0 && lane == 0) {
     tc::tma_prefetch_desc(&tm_x);
-    if constexpr (BWD) tc::tma_prefetch_desc(&tm_g);
+    if constexpr (STAGE_G) tc::tma_prefetch_desc(&tm_g);
     if constexpr (FULLB) {
       tc::tma_prefetch_desc(&tm_G);
       tc::tma_prefetch_desc(&tm_f);
@@ -181,7 +185,8 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
           if constexpr (FULLB)
             tc::tma_load_3d(base + CFG::G_OFF + i * XBOX, &tm_G, full(s), c0, i, (int)t0, pol_stream);
         }
-        if constexpr (BWD) tc::tma_load_2d(base + CFG::GG_OFF, &tm_g, full(s), c0, (int)t0, pol_stream);
+        if constexpr (STAGE_G)
+          tc::tma_load_2d(base + CFG::GG_OFF, &tm_g, full(s), c0, (int)t0, pol_stream);
         if constexpr (FULLB) tc::tma_load_2d(base + CFG::F_OFF, &tm_f, full(s), c0, (int)t0, pol_stream);
         ++issued;
       }
@@ -239,7 +244,7 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
 #pragma unroll
       for (int c = 0; c < 2; ++c) {  // the two 8-channel halves of the chunk
         float gv[8];
-        if constexpr (BWD) unpack8(ld32sw(st + CFG::GG_OFF, tok, c), gv);
+        if constexpr (STAGE_G) unpack8(ld32sw(st + CFG::GG_OFF, tok, c), gv);
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
           float xv[8];
@@ -247,7 +252,7 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             ss = fmaf(xv[e], xv[e], ss);
-            if constexpr (BWD) dots[36 + r] = fmaf(gv[e], xv[e], dots[36 + r]);
+            if constexpr (STAGE_G) dots[36 + r] = fmaf(gv[e], xv[e], dots[36 + r]);
           }
         }
         if constexpr (FULLB) {
@@ -349,23 +354,26 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
         }
       } else {
         sk_forward_ckpt<N>(H, iters, ck + tok, TM, ck_period);
-        // dL/dH_res: <G_i, x_j> from the two stream halves, or the post half's
-        const float* rt = red_in + (live ? t : 0) * (N * N + N);
+        // dL/dH_res: <G_i, x_j> from the two stream halves, or the post half's,
+        // or (DOTS) the tensor-core reductions' rows
+        constexpr int RSTRIDE = DOTS ? N * N + 2 * N : N * N + N;
+        const float* rt = red_in + (live ? t : 0) * RSTRIDE;
         float dA[N * N];
 #pragma unroll
         for (int i = 0; i < N; ++i)
 #pragma unroll
           for (int j = 0; j < N; ++j)
-            dA[i * N + j] = SPLIT ? (live ? __ldg(rt + i * N + j) : 0.0f)
-                                  : red_dt[((i >> 2) * NDH + 8 * (i & 3) + j) * TM + tok];
+            dA[i * N + j] = SPLIT || DOTS ? (live ? __ldg(rt + i * N + j) : 0.0f)
+                                          : red_dt[((i >> 2) * NDH + 8 * (i & 3) + j) * TM + tok];
         float dzres[N * N];
         sk_adjoint_ckpt<N>(dA, dzres, iters, ck + tok, TM, ck_period);
         float dz[M];
 #pragma unroll
         for (int i = 0; i < N; ++i) {
-          const float dpre = red_dt[((i >> 2) * NDH + 36 + (i & 3)) * TM + tok];
-          const float dpost = SPLIT ? (live ? __ldg(rt + N * N + i) : 0.0f)
-                                    : red_dt[((i >> 2) * NDH + 32 + (i & 3)) * TM + tok];
+          const float dpre = DOTS ? (live ? __ldg(rt + N * N + N + i) : 0.0f)
+                                  : red_dt[((i >> 2) * NDH + 36 + (i & 3)) * TM + tok];
+          const float dpost = SPLIT || DOTS ? (live ? __ldg(rt + N * N + i) : 0.0f)
+                                            : red_dt[((i >> 2) * NDH + 32 + (i & 3)) * TM + tok];
           dz[i] = dpre * spre[i] * (1.0f - spre[i]);
           dz[N + i] = dpost * 2.0f * spost[i] * (1.0f - spost[i]);
         }
@@ -533,7 +541,7 @@ cudaError_t map8_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float ep
   const uint64_t d2[2] = {(uint64_t)C, (uint64_t)T};
   const uint64_t s2[1] = {(uint64_t)C * 2};
   const uint32_t b2[2] = {CH, TM};
-  if (mode != MAP_FWD) {
+  if (mode == MAP_BWD || mode == MAP_BWD_SPLIT) {
     e = make_tmap_bf16(&mg, g, 2, d2, s2, b2, SW);
     if (e != cudaSuccess) return e;
   }
@@ -554,6 +562,10 @@ cudaError_t map8_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float ep
       return launch_map8<MAP_BWD_SPLIT>(mx, phi_split, mG, mg, mf, T, C, iters, eps, b, alpha, ag,
                                         nullptr, nullptr, nullptr, coef, urec, part, red, st,
                                         wait_ns, s);
+    case MAP_BWD_DOTS:
+      return launch_map8<MAP_BWD_DOTS>(mx, phi_split, mG, mg, mf, T, C, iters, eps, b, alpha, ag,
+                                       nullptr, nullptr, nullptr, coef, urec, part, red, st,
+                                       wait_ns, s);
     default:
       return cudaErrorInvalidValue;
   }

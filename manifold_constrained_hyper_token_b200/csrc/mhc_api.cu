@@ -100,10 +100,10 @@ BwdWorkspace bwd_layout(const mhc_params* p) {
     if (tc8) {
       w.urec_off = off;
       off = round_up(off + (size_t)p->T * mhc::TcRec8::U_BYTES, 256);
-      // the whole backward's <G_i, x_j>, <G_i, f_out> from the tensor-core
-      // reductions, read by the mapping in its split mode
+      // the whole backward's C-reductions from the tensor-core kernel, read
+      // by the mapping in its MAP_BWD_DOTS mode
       w.red_off = off;
-      off = round_up(off + (size_t)p->T * (8 * 8 + 8) * 4, 256);
+      off = round_up(off + (size_t)p->T * (8 * 8 + 2 * 8) * 4, 256);
     }
     if (use_tc16(p)) {
       w.urec_off = off;
@@ -254,15 +254,15 @@ mhc_status mhc_backward_map(const mhc_params* p, const void* x, const float* phi
                                           (float*)(ws + w.part_off), ws + w.kmap_off, dev_status,
                                           p->wait_ns, (cudaStream_t)stream));
   if (use_tc8(p)) {
-    // <G_i, x_j> and <G_i, f_out> on the tensor cores, then the mapping in the
-    // split mode (x and grad_h_in staged; <g, x_j>, the projection, the adjoint)
-    st = from_cuda(mhc::dots8_red_dispatch(p->T, p->C, x, grad_x_next, f_out,
+    // the C-reductions (<G_i, x_j> on the tensor cores), then the mapping with
+    // only x staged (the projection, the gates, the adjoint)
+    st = from_cuda(mhc::dots8_red_dispatch(p->T, p->C, x, grad_x_next, grad_h_in, f_out,
                                            (float*)(ws + w.red_off), dev_status, p->wait_ns,
                                            (cudaStream_t)stream));
     if (st != MHC_OK) return st;
-    return from_cuda(mhc::map8_tc_dispatch(mhc::MAP_BWD_SPLIT, p->T, p->C, p->t_max, p->eps, x,
+    return from_cuda(mhc::map8_tc_dispatch(mhc::MAP_BWD_DOTS, p->T, p->C, p->t_max, p->eps, x,
                                            phi, ws + w.phi_off, b, alpha, alpha_groups(p), nullptr,
-                                           nullptr, nullptr, nullptr, grad_h_in, nullptr,
+                                           nullptr, nullptr, nullptr, nullptr, nullptr,
                                            (const float*)(ws + w.red_off),
                                            (float*)(ws + w.coef_off), ws + w.urec_off,
                                            (float*)(ws + w.part_off), dev_status, p->wait_ns,

@@ -14,7 +14,9 @@ namespace mhc {
 // C-reduction; or the pre half of the backward in training order, which takes
 // <G_i, x_j> and <G_i, f_out> from the post half (`red`, [T][n*n + n]).
 // MAP_POSTFWD: layer l's post merge fused with layer l+1's forward mapping.
-enum MapMode { MAP_FWD = 0, MAP_BWD = 1, MAP_BWD_SPLIT = 2, MAP_POSTFWD = 3 };
+// MAP_BWD_DOTS (n = 8): the backward's recompute with every C-reduction read
+// from `red` ([T][n*n + 2n]: <G_i, x_j>, <G_i, f_out>, <g, x_j>).
+enum MapMode { MAP_FWD = 0, MAP_BWD = 1, MAP_BWD_SPLIT = 2, MAP_POSTFWD = 3, MAP_BWD_DOTS = 4 };
 
 // k_sinkhorn.cu
 cudaError_t sinkhorn_dispatch(int n, int iters, int64_t B, const float* logits, float* out,
@@ -58,7 +60,7 @@ size_t map_tc_scratch_bytes(int64_t T, int64_t C);
 // phi [K][24] fp32 -> the bf16 split copy of phi^T [48][K] the mapping MMAs read
 cudaError_t phi_split_dispatch(int64_t K, const float* phi, void* phi_split, cudaStream_t s);
 // k_map8_tc.cu (bf16, n = 8: projection on the tensor cores); mode is MAP_FWD,
-// MAP_BWD or MAP_BWD_SPLIT.  Splits phi into phi_split (map8_tc_phi_bytes(C)
+// MAP_BWD, MAP_BWD_SPLIT or MAP_BWD_DOTS.  Splits phi into phi_split (map8_tc_phi_bytes(C)
 // bytes); the backward modes write the per-token records (coef
 // [T][Coef<8>::SIZE]), the U rows (urec [T][TcRec8::U_ELEMS] bf16) and one
 // partial-sum record per 128 tokens (part).
@@ -89,13 +91,14 @@ size_t proj16_phi_bytes(int64_t C);
 // k_dots_tc.cu (bf16): the backward's C-reductions per token.  n = 16: into
 // rows [T][Coef<16>::SIZE] at [288 + d]; full = all 288 (<G_i, x_j> on the
 // tensor cores, <g, x_i>, <G_i, f>), otherwise <g, x_i> only (split backward).
-// n = 8: <G_i, x_j> (tensor cores) and <G_i, f> into red [T][72], the layout
-// the n = 8 mapping's split mode reads.
+// n = 8: <G_i, x_j> (tensor cores), <G_i, f> and <g, x_j> into red [T][80],
+// the layout the n = 8 mapping's MAP_BWD_DOTS mode reads.
 cudaError_t dots16_dispatch(bool full, int64_t T, int64_t C, const void* x, const void* G,
                             const void* g, const void* f, float* rows, int* st, int64_t wait_ns,
                             cudaStream_t s);
-cudaError_t dots8_red_dispatch(int64_t T, int64_t C, const void* x, const void* G, const void* f,
-                               float* red, int* st, int64_t wait_ns, cudaStream_t s);
+cudaError_t dots8_red_dispatch(int64_t T, int64_t C, const void* x, const void* G, const void* g,
+                               const void* f, float* red, int* st, int64_t wait_ns,
+                               cudaStream_t s);
 // k_wide.cu, bf16 with n = 16: the mapping with the projection on the tensor
 // cores (proj16_dispatch) and the rest of the k_wide kernels: MAP_FWD writes
 // the maps (rows: [T][Coef<16>::SIZE] scratch); MAP_BWD / MAP_BWD_SPLIT write
