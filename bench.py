@@ -103,7 +103,6 @@ CALL_SOURCES = {
     "layer_input": ["k_post.cu", "mhc_common.cuh"],
     "post_fused": ["k_map_tc.cu", "tc_sm100.cuh", "mhc_common.cuh"],
     "post_n8": ["k_post.cu", "mhc_common.cuh"],
-    "bwd_map_n8": ["k_map8_tc.cu", "tc_sm100.cuh", "mhc_common.cuh"],
     "layer_input_n8": ["k_post.cu", "mhc_common.cuh"],
 }
 
@@ -521,11 +520,11 @@ def run_layer(args, dev, rank, world, local_rank):
     pb = per_call_param_bytes(n, C)
     call_bytes = {c: T * tb[c] + pb[c] for c in calls}
     # the roofline is read for a call whose time is one kernel's (the phi split
-    # ahead of the backward mapping is 5 us of its 0.5 ms and is counted in; at
-    # n = 8 the apply is three kernels and is not such a call)
+    # ahead of the n = 4 backward mapping is 5 us of its 0.5 ms and is counted
+    # in; at n = 8 and 16 the backward mapping and the apply are several
+    # kernels each and are not such calls)
     single = [c for c in calls
-              if c in ("post", "layer_input") or (c == "bwd_map" and n != 16) or
-              (c == "bwd_apply" and n == N_STR)]
+              if c in ("post", "layer_input") or (c in ("bwd_map", "bwd_apply") and n == N_STR)]
     dom = max(single, key=lambda c: per_call[c])
     achieved = call_bytes[dom] / (per_call[dom] / 1000.0) / 1e9
     traffic = ncu_traffic(traffic_key(dom, n))
