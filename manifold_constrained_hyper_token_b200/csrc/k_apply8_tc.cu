@@ -8,22 +8,23 @@
 //   grad_phi[k][m] = sum_t x_t[k] u_t[m]
 //
 // (reverse mode of the update equation of the chatgpz.de explainer and of the
-// RMS-normalised projection; reportify.cn [19]-[21]).  At n = 8 an item of the fused
-// n = 4 design (x, grad_x_next and grad_h_in of 16 channels x 8 streams x 128
-// tokens, the tile's U rows and H records, the slice's phi rows) needs about
-// 170 KB of shared memory, and the grad_phi accumulators of three slices do
-// not fit beside the phi u accumulators in TMEM, so the two contractions run
-// as their own tensor-core kernels:
+// RMS-normalised projection; reportify.cn [19]-[21]).  At n = 8 the grad_phi
+// accumulators of the channels a CTA covers do not fit beside the phi u
+// accumulators in TMEM, so the two contractions run as two tensor-core kernels:
 //
-//   k_phiu8   phi u for a (128-token tile, 256 channels of one stream) item:
+//   k_gxu8    grad_x and grad_f_out for (128-token tile, 32 channels of all 8
+//             streams) items, one persistent CTA per SM: phi u as
 //             D[128 x 256] = U[128 x 192] . PHI[192 x 256] (tcgen05, bf16
-//             operands, fp32 in TMEM), written to an fp32 scratch [T][8][C];
-//   k_gx8     grad_x and grad_f_out from that scratch, x, grad_x_next and
-//             grad_h_in with coalesced 16-byte loads and stores (CUDA cores),
-//             and grad_b / grad_alpha from the mapping's partial sums;
+//             operands, fp32 in TMEM, two accumulators so that one item's MMAs
+//             overlap the previous item's epilogue); the epilogue warps turn
+//             8 tokens' rows of D around in shared memory and add the CUDA-core
+//             terms from x, grad_x_next and grad_h_in, which they load with
+//             coalesced 16-byte loads (4 lanes cover one token's 64-byte row
+//             piece), so phi u never leaves the chip;
 //   k_gphi8   grad_phi for 128 rows of phi: D[128 x 192] += X^T[128 x 128] .
 //             U[128 x 192] over every token tile (tcgen05), then
-//             grad_phi = D[:, m] + D[:, 96 + m].
+//             grad_phi = D[:, m] + D[:, 96 + m];
+//   k_bias8   grad_b and grad_alpha from the mapping's per-tile partial sums.
 //
 // U is [u_hi (80) | 0 (16) | u_lo (80) | 0 (16)]: phi u = (u_hi + u_lo) . phi_hi
 // and x . u carries u to ~16 bits (x is exact).  All sums are in a fixed order:
@@ -42,18 +43,32 @@ constexpr int M = N * N + 2 * N;        // 80 logits
 constexpr int TT = 128;                 // tokens per tile
 constexpr int NU = TcRec8::U_ELEMS;     // 192
 constexpr int ATOM = 128 * 128;         // [128 rows][64 bf16] with the 128-byte swizzle: 16 KB
-// k_phiu8
-constexpr int KB = 256;                 // channels of one stream per item (MMA N)
 constexpr int CH = 16;                  // channels per block of the tiled phi^T copy
 constexpr int NL = 2 * M;               // rows per block (80 high, 80 low)
 constexpr int PHB = M * CH * 2;         // the 80 high rows of one block: 2.5 KB
-constexpr int A_U_OFF = 0;              // U tile: three atoms (48 KB)
-constexpr int A_P_OFF = 3 * ATOM;       // phi tile: KB / CH blocks of high rows (40 KB)
-constexpr int A_DATA = A_P_OFF + (KB / CH) * PHB;
-constexpr int XT = 36;                  // row stride (floats) of the epilogue's transpose buffer
-constexpr int A_SMEM = A_DATA + 1024 + 64;
-constexpr int A_NT = 128;
-constexpr uint32_t A_TMEM = 256;
+// k_gxu8
+constexpr int FS = 32;                  // channels per item (all 8 streams)
+constexpr int FN = N * FS;              // MMA N: 256 columns, column 32 j + channel
+constexpr int F_U_OFF = 0;              // U tile: three atoms (48 KB)
+constexpr int F_P_OFF = 3 * ATOM;       // phi: 16 atoms (stream j, 16-channel half) of PHB
+constexpr int F_W_OFF = F_P_OFF + 2 * N * PHB;  // the epilogue warps' areas
+constexpr int NEPI = 4;                 // epilogue warps, one per TMEM lane quarter
+constexpr int CK = 8;                   // tokens per epilogue step
+constexpr int XTS = 260;                // row stride (floats) of the transpose buffer
+constexpr int RS = (N + 1) * 64;        // a token's staged rows (grad_x_next x 8, grad_h_in)
+constexpr int HS = 84;                  // H record in shared memory: res, pre, post, kappa
+constexpr int SL_H = CK * RS;           // ring slot: [CK][RS] rows, then [CK][HS] records
+constexpr int SLOT = SL_H + CK * HS * 4;
+constexpr int NSLOT = 3;                // steps staged: the current one and two ahead
+constexpr int W_RING = CK * XTS * 4;
+constexpr int W_BYTES = W_RING + NSLOT * SLOT;
+constexpr int F_DATA = F_W_OFF + NEPI * W_BYTES;
+constexpr int F_SMEM = F_DATA + 1024 + 128;
+constexpr int F_NT = (2 + NEPI) * 32;   // TMA, MMA, epilogue x4
+constexpr uint32_t F_TMEM = 512;
+static_assert(F_P_OFF % 1024 == 0 && F_W_OFF % 1024 == 0, "operand alignment");
+static_assert(W_BYTES % 16 == 0 && SLOT % 16 == 0 && W_RING % 16 == 0, "alignment");
+static_assert((XTS * 4) % 128 == 16 && RS % 128 == 64 && (HS * 4) % 16 == 0, "bank spread");
 // k_gphi8
 constexpr int CB = 128;                 // phi rows (channels of one stream) per CTA (MMA M)
 constexpr int C_X_OFF = 0;              // x tile [128 tokens][128 channels]: two atoms
@@ -64,235 +79,382 @@ constexpr int C_DATA = C_NS * C_STAGE;
 constexpr int C_SMEM = C_DATA + 1024 + 64;
 constexpr int C_NT = 128;
 constexpr uint32_t C_TMEM = 256;
-// k_gx8
+// k_bias8
 constexpr int B_NT = 128;
-static_assert(A_SMEM <= 232448 && C_SMEM <= 232448, "shared memory");
+static_assert(F_SMEM <= 232448 && C_SMEM <= 232448, "shared memory");
 }  // namespace ap8
 
 namespace {
-__device__ __forceinline__ void unpack8b(uint4 q, float (&v)[8]) {
-  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    v[2 * i] = __uint_as_float(w[i] << 16);
-    v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-  }
+// 16-byte asynchronous global -> shared copies (L2 only), in commit groups
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
-__device__ __forceinline__ uint4 pack8b(const float (&v)[8]) {
-  uint32_t w[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-    w[i] = *reinterpret_cast<uint32_t*>(&h);
-  }
-  return make_uint4(w[0], w[1], w[2], w[3]);
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait0() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+// wait until at most two committed groups of this thread are still in flight
+__device__ __forceinline__ void cp_async_wait2() {
+  asm volatile("cp.async.wait_group 2;" ::: "memory");
+}
+// Paired fp32 arithmetic (one fma.rn.f32x2 = two IEEE fp32 FMAs).
+__device__ __forceinline__ uint64_t f2pack(float x, float y) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(x), "f"(y));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+// two bf16 (one 32-bit word) widened to an fp32 pair, and back
+__device__ __forceinline__ uint64_t bf2_to_f2(uint32_t w) {
+  return f2pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+__device__ __forceinline__ uint32_t f2_to_bf2(uint64_t v) {
+  float x, y;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(x), "=f"(y) : "l"(v));
+  __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+  return *reinterpret_cast<uint32_t*>(&h);
 }
 }  // namespace
 
-// ------------------------------------------------------------------ phi u
-__global__ void __launch_bounds__(ap8::A_NT) k_phiu8(const __grid_constant__ CUtensorMap tm_u,
-                                                     const __nv_bfloat16* __restrict__ phi_t,
-                                                     int64_t T, int64_t C, int ncb,
-                                                     float* __restrict__ phiu, int* status,
-                                                     uint64_t wait_ns) {
+// ------------------------------------------------------- grad_x, grad_f_out
+// Items it = blockIdx.x + k * gridDim.x in (tile, 32-channel slice) order, so
+// the CTAs work on neighbouring slices of the same token rows at any time.
+// Warp 0 loads each item's U tile (when the tile changes) and the 16 phi atoms
+// of its slice into single-buffered operands; warp 1 issues the MMAs into the
+// item's accumulator (columns 256 (k & 1)..); warps 2..5 each take the 32
+// tokens of their TMEM lane quarter in four steps of 8 tokens.  A step's
+// grad_x_next and grad_h_in rows and H records are copied into a three-slot
+// ring two steps ahead (cp.async, 16 bytes per lane, 4 lanes per 64-byte row
+// piece); x is loaded into registers at the start of the step; the 8 tokens'
+// D rows go through a transpose buffer, and the lanes then work as 8 tokens
+// x 4 groups of 8 channels over all 8 streams.
+__global__ void __launch_bounds__(ap8::F_NT, 1) k_gxu8(
+    const __grid_constant__ CUtensorMap tm_u, const __nv_bfloat16* __restrict__ phi_t, int64_t T,
+    int64_t C, int nsl, int64_t nitems, const __nv_bfloat16* __restrict__ x,
+    const __nv_bfloat16* __restrict__ G, const __nv_bfloat16* __restrict__ g,
+    const float* __restrict__ coef, __nv_bfloat16* __restrict__ gx,
+    __nv_bfloat16* __restrict__ gf, int* status, uint64_t wait_ns) {
   using namespace ap8;
+  using CF = Coef<N>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + A_DATA);  // full, mma, fin
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
-  const uint32_t full = tc::smem_u32(bars), mma_bar = tc::smem_u32(bars + 1);
+  // op_full op_empty dfull[2] dempty[2] fin
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + F_DATA);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 7);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const uint32_t op_full = tc::smem_u32(bars), op_empty = tc::smem_u32(bars + 1);
+  auto dfull = [&](int d) { return tc::smem_u32(bars + 2 + d); };
+  auto dempty = [&](int d) { return tc::smem_u32(bars + 4 + d); };
+  const uint32_t fin_bar = tc::smem_u32(bars + 6);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int item = blockIdx.x;
-  const int tile = item / (N * ncb), rem = item % (N * ncb);
-  const int j = rem / ncb, cb = rem % ncb;
-  const int64_t t0 = (int64_t)tile * TT;
-  const int c0 = cb * KB;
+  const int64_t nblk = (C + CH - 1) / CH;
 
   if (threadIdx.x == 0) {
-    tc::mbar_init(full, 1);
-    tc::mbar_init(mma_bar, 1);
+    tc::mbar_init(op_full, 1);
+    tc::mbar_init(op_empty, 1);
+    for (int d = 0; d < 2; ++d) {
+      tc::mbar_init(dfull(d), 1);
+      tc::mbar_init(dempty(d), NEPI);
+    }
+    tc::mbar_init(fin_bar, 1);
+    *abort_flag = 0;
     tc::mbar_fence_init();
   }
+  if (warp == 0 && lane == 0) tc::tma_prefetch_desc(&tm_u);
   if (warp == 1) {
-    tc::tmem_alloc(tc::smem_u32(tmem_slot), A_TMEM);
+    tc::tmem_alloc(tc::smem_u32(tmem_slot), F_TMEM);
     tc::tmem_relinquish();
   }
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  auto give_up = [&]() {
+    *abort_flag = 1;
+    flag_status(status, MHC_ERR_TIMEOUT);
+  };
 
-  if (threadIdx.x == 0) {
-    const uint64_t pol = tc::policy_evict_last();  // U and phi are read by many CTAs
-    // phi: the high rows of the KB / CH channel blocks of stream j (blocks past
-    // the last channel are not loaded; the columns they feed are not stored)
-    const int64_t nblk = (C + CH - 1) / CH;
-    const int64_t q0 = (int64_t)c0 / CH;
-    const int nb = (int)(nblk - q0 < KB / CH ? nblk - q0 : KB / CH);
-    tc::mbar_arrive_expect_tx(full, (uint32_t)(3 * ATOM + nb * PHB));
-    for (int a = 0; a < 3; ++a)
-      tc::tma_load_2d(tc::smem_u32(smem + A_U_OFF + a * ATOM), &tm_u, full, 64 * a, (int)t0, pol);
-    for (int q = 0; q < nb; ++q)
-      tc::bulk_load(tc::smem_u32(smem + A_P_OFF + q * PHB), phi_t + ((q0 + q) * N + j) * (NL * CH),
-                    PHB, full, pol);
-  }
-  bool ok = true;
-  if (warp == 1 && lane == 0) {
-    ok = tc::mbar_wait(full, 0, nullptr, wait_ns);
-    if (ok) {
-      tc::tc_fence_after();
-      // D[tok][k] = sum over m' of U[tok][m'] PHI[m'][k]: K-steps 0..4 take u_hi
-      // against phi rows 0..79, steps 6..10 u_lo against the same rows; steps 5
-      // and 11 would only multiply U's zero padding.  PHI is MN-major with the
-      // 32-byte swizzle: 16-channel atoms PHB bytes apart, 8-row groups 256 apart.
-      constexpr uint32_t idesc = tc::idesc_bf16(TT, KB, false, true);
-      const uint32_t ub = tc::smem_u32(smem + A_U_OFF), pb = tc::smem_u32(smem + A_P_OFF);
-      int issued = 0;
-#pragma unroll
-      for (int s = 0; s < NU / 16; ++s) {
-        if (s == 5 || s == 11) continue;
-        const int r = s < 5 ? s : s - 6;  // 16-row block of phi^T
-        const uint64_t da = tc::smem_desc(ub + (s / 4) * ATOM + (s % 4) * 32, 16, 1024, tc::SWZ_128B);
-        const uint64_t db = tc::smem_desc(pb + r * 16 * 32, PHB, 256, tc::SWZ_32B);
-        tc::mma_bf16(tmem, da, db, idesc, issued > 0 ? 1u : 0u);
-        ++issued;
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA
+    if (lane == 0) {
+      const uint64_t pol = tc::policy_evict_last();  // U and phi are read by many CTAs
+      int64_t prev_tile = -1;
+      int li = 0;
+      for (int64_t it = blockIdx.x; it < nitems; it += gridDim.x, ++li) {
+        const int64_t tile = it / nsl;
+        const int64_t q0 = (it % nsl) * (FS / CH);
+        // the phi blocks past the last channel are not loaded (their columns
+        // are not stored)
+        const int nb = (int)(nblk - q0 < FS / CH ? nblk - q0 : FS / CH);
+        if (li >= 1 && !tc::mbar_wait(op_empty, (uint32_t)(li - 1) & 1u, abort_flag, wait_ns)) {
+          give_up();
+          break;
+        }
+        const bool new_u = tile != prev_tile;
+        tc::mbar_arrive_expect_tx(op_full, (uint32_t)((new_u ? 3 * ATOM : 0) + nb * N * PHB));
+        if (new_u)
+          for (int a = 0; a < 3; ++a)
+            tc::tma_load_2d(tc::smem_u32(smem + F_U_OFF + a * ATOM), &tm_u, op_full, 64 * a,
+                            (int)(tile * TT), pol);
+        for (int h = 0; h < nb; ++h)
+          for (int j = 0; j < N; ++j)
+            tc::bulk_load(tc::smem_u32(smem + F_P_OFF + (2 * j + h) * PHB),
+                          phi_t + ((q0 + h) * N + j) * (NL * CH), PHB, op_full, pol);
+        prev_tile = tile;
       }
-      tc::mma_commit(mma_bar);
-    } else {
-      flag_status(status, MHC_ERR_TIMEOUT);
-      // the copies already issued land before the CTA exits
-      tc::mbar_wait(full, 0, nullptr, tc::kDrainWaitNs);
+      // every copy issued here has landed before the CTA can exit
+      if (li > 0) tc::mbar_wait(op_full, (uint32_t)(li - 1) & 1u, nullptr, tc::kDrainWaitNs);
     }
-  }
-  // the epilogue: warp w reads TMEM lanes 32w..32w+31 (tokens), 256 columns
-  const bool okall = __syncthreads_or(!ok) == 0;
-  bool done = okall && tc::mbar_wait(mma_bar, 0, nullptr, wait_ns);
-  if (okall && !done) flag_status(status, MHC_ERR_TIMEOUT);
-  done = __all_sync(0xffffffffu, done);
-  if (done) {
-    // each warp turns its 32 token rows x 32 columns around in shared memory (the
-    // U tile, free once the MMAs are done), so that 8 lanes store one token's
-    // 128 contiguous bytes
-    tc::tc_fence_after();
-    float* xt = reinterpret_cast<float*>(smem + A_U_OFF) + warp * 32 * XT;
-    const uint32_t lb = tmem + ((uint32_t)(32 * warp) << 16);
-    const int rr = lane >> 3, cq = lane & 7;
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      // D[tok][32 j + c] = sum over m' of U[tok][m'] PHI[m'][32 j + c]: K-steps
+      // 0..4 take u_hi against phi rows 0..79, steps 6..10 u_lo against the
+      // same rows (5 and 11 would only multiply U's zero padding).  PHI is
+      // MN-major with the 32-byte swizzle: 16-channel atoms PHB bytes apart,
+      // 8-row groups 256 apart.
+      constexpr uint32_t idesc = tc::idesc_bf16(TT, FN, false, true);
+      const uint32_t ub = tc::smem_u32(smem + F_U_OFF), pb = tc::smem_u32(smem + F_P_OFF);
+      bool any = false;
+      int li = 0;
+      for (int64_t it = blockIdx.x; it < nitems; it += gridDim.x, ++li) {
+        const int d = li & 1;
+        if (li >= 2 &&
+            !tc::mbar_wait(dempty(d), ((uint32_t)(li >> 1) & 1u) ^ 1u, abort_flag, wait_ns)) {
+          give_up();
+          break;
+        }
+        if (!tc::mbar_wait(op_full, (uint32_t)li & 1u, abort_flag, wait_ns)) {
+          give_up();
+          break;
+        }
+        tc::tc_fence_after();
+        const uint32_t dt = tmem + (uint32_t)(d * FN);
+        int issued = 0;
+#pragma unroll
+        for (int s = 0; s < NU / 16; ++s) {
+          if (s == 5 || s == 11) continue;
+          const int r = s < 5 ? s : s - 6;  // 16-row block of phi^T
+          const uint64_t da =
+              tc::smem_desc(ub + (s / 4) * ATOM + (s % 4) * 32, 16, 1024, tc::SWZ_128B);
+          const uint64_t db = tc::smem_desc(pb + r * 16 * 32, PHB, 256, tc::SWZ_32B);
+          tc::mma_bf16(dt, da, db, idesc, issued > 0 ? 1u : 0u);
+          ++issued;
+        }
+        any = true;
+        tc::mma_commit(op_empty);
+        tc::mma_commit(dfull(d));
+      }
+      // every MMA issued here has finished before TMEM is freed
+      if (any) {
+        tc::mma_commit(fin_bar);
+        tc::mbar_wait(fin_bar, 0, nullptr, tc::kDrainWaitNs);
+      }
+    }
+  } else {
+    // ----------------------------------------------------------- epilogue
+    const int ew = warp - 2;
+    const int qd = warp & 3;             // TMEM lane quarter: tokens 32 qd .. 32 qd + 31
+    uint8_t* wbase = smem + F_W_OFF + ew * W_BYTES;
+    float* xt = reinterpret_cast<float*>(wbase);
+    const uint32_t ring = tc::smem_u32(wbase + W_RING);
+    const int r = lane >> 2, q = lane & 3;  // token of the step, 8-channel group
+    // this lane's share of a step's H records: chunks f = lane + 32 k of the
+    // 8 x 21 16-byte chunks (rows [0, 80) and kappa of each token)
+    int h_tok[6], h_src[6], h_dst[6];
+#pragma unroll
+    for (int k = 0; k < 6; ++k) {
+      const int f = lane + 32 * k;
+      const int tk = f / 21, kk = f % 21;
+      h_tok[k] = f < CK * 21 ? tk : CK;
+      h_src[k] = tk * CF::SIZE + (kk < 20 ? 4 * kk : CF::KAPPA);
+      h_dst[k] = SL_H + (tk * HS + 4 * kk) * 4;
+    }
+    // stage step s (4 steps of 8 tokens per item) into ring slot s % 3: the
+    // step's grad_x_next and grad_h_in rows and its H records
+    auto stage = [&](int64_t s) {
+      const int64_t it = blockIdx.x + (s >> 2) * (int64_t)gridDim.x;
+      if (it < nitems) {
+        const uint32_t dst = ring + (uint32_t)((s % NSLOT) * SLOT);
+        const int64_t tb = (it / nsl) * TT + 32 * qd + CK * (int)(s & 3);
+        const int64_t t = tb + r, c = (it % nsl) * FS + 8 * q;
+        if (t < T && c < C) {
+          const uint32_t rd = dst + (uint32_t)(r * RS + 16 * q);
+#pragma unroll
+          for (int i = 0; i < N; ++i) cp_async16(rd + 64 * i, G + (t * N + i) * C + c);
+          cp_async16(rd + 64 * N, g + t * C + c);
+        }
+#pragma unroll
+        for (int k = 0; k < 6; ++k)
+          if (h_tok[k] < CK && tb + h_tok[k] < T)
+            cp_async16(dst + (uint32_t)h_dst[k], coef + tb * CF::SIZE + h_src[k]);
+      }
+      cp_async_commit();
+    };
+    stage(0);
+    stage(1);
+    int64_t s = 0;
+    bool ok = true;
+    int li = 0;
+    for (int64_t it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++li) {
+      const int d = li & 1;
+      const int64_t c = (it % nsl) * FS + 8 * q;
+      const int64_t tile0 = (it / nsl) * TT + 32 * qd;
+      const uint32_t taddr = tmem + (uint32_t)(d * FN) + ((uint32_t)(32 * qd) << 16);
 #pragma unroll 1
-    for (int q = 0; q < KB / 32; ++q) {
-      float v0[16], v1[16];
-      tc::tmem_ld16(lb + 32 * q, v0);
-      tc::tmem_ld16(lb + 32 * q + 16, v1);
-      tc::tmem_ld_wait();
+      for (int ci = 0; ci < 4; ++ci, ++s) {
+        stage(s + 2);
+        const int64_t t = tile0 + CK * ci + r;
+        const bool vld = t < T && c < C;
+        // x is needed last: its loads fly while D is turned around
+        uint4 Xp[N];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        *reinterpret_cast<float4*>(xt + lane * XT + 4 * e) =
-            make_float4(v0[4 * e], v0[4 * e + 1], v0[4 * e + 2], v0[4 * e + 3]);
-        *reinterpret_cast<float4*>(xt + lane * XT + 16 + 4 * e) =
-            make_float4(v1[4 * e], v1[4 * e + 1], v1[4 * e + 2], v1[4 * e + 3]);
-      }
-      __syncwarp();
-      const int64_t c = (int64_t)c0 + 32 * q + 4 * cq;
+        for (int i = 0; i < N; ++i) Xp[i] = make_uint4(0, 0, 0, 0);
+        if (vld) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = 4 * i + rr;
-        const int64_t t = t0 + 32 * warp + r;
-        const float4 val = *reinterpret_cast<const float4*>(xt + r * XT + 4 * cq);
-        if (t < T && c < C) __stcg(reinterpret_cast<float4*>(phiu + (t * N + j) * C + c), val);
+          for (int i = 0; i < N; ++i)
+            Xp[i] = __ldcs(reinterpret_cast<const uint4*>(x + (t * N + i) * C + c));
+        }
+        if (ci == 0) {
+          bool okw = tc::mbar_wait(dfull(d), (uint32_t)(li >> 1) & 1u, abort_flag, wait_ns);
+          if (!okw && !*abort_flag) give_up();
+          ok = __all_sync(0xffffffffu, okw);
+          if (!ok) break;
+          tc::tc_fence_after();
+        }
+        // D rows of the step's 8 tokens (lanes 8 ci .. 8 ci + 7 of the quarter)
+        // into the transpose buffer, 64 columns per TMEM wait
+        const int row = lane - CK * ci;
+        const bool mine = row >= 0 && row < CK;
+#pragma unroll 1
+        for (int kb = 0; kb < FN / 64; ++kb) {
+          float v[4][16];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) tc::tmem_ld16(taddr + 64 * kb + 16 * u, v[u]);
+          tc::tmem_ld_wait();
+          if (mine) {
+            float* dst = xt + row * XTS + 64 * kb;
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                *reinterpret_cast<float4*>(dst + 16 * u + 4 * e) =
+                    make_float4(v[u][4 * e], v[u][4 * e + 1], v[u][4 * e + 2], v[u][4 * e + 3]);
+          }
+        }
+        cp_async_wait2();  // this step's staged rows and records
+        __syncwarp();
+        const uint8_t* slot = wbase + W_RING + (s % NSLOT) * SLOT;
+        const uint8_t* rows = slot + r * RS + 16 * q;
+        const float* hr = reinterpret_cast<const float*>(slot + SL_H) + r * HS;
+        // acc[j][p]: channels 2p, 2p + 1 of stream j, starting from phi u
+        uint64_t acc[N][4];
+#pragma unroll
+        for (int j = 0; j < N; ++j) {
+          const ulonglong2 a0 = *reinterpret_cast<const ulonglong2*>(xt + r * XTS + 32 * j + 8 * q);
+          const ulonglong2 a1 =
+              *reinterpret_cast<const ulonglong2*>(xt + r * XTS + 32 * j + 8 * q + 4);
+          acc[j][0] = a0.x;
+          acc[j][1] = a0.y;
+          acc[j][2] = a1.x;
+          acc[j][3] = a1.y;
+        }
+        {
+          const uint4 gw = *reinterpret_cast<const uint4*>(rows + 64 * N);
+          const uint64_t gp[4] = {bf2_to_f2(gw.x), bf2_to_f2(gw.y), bf2_to_f2(gw.z),
+                                  bf2_to_f2(gw.w)};
+#pragma unroll
+          for (int j = 0; j < N; ++j) {
+            const float h = hr[CF::PRE + j];
+            const uint64_t hh = f2pack(h, h);
+#pragma unroll
+            for (int p = 0; p < 4; ++p) acc[j][p] = f2fma(hh, gp[p], acc[j][p]);
+          }
+        }
+        uint64_t gfa[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+          const uint4 w = *reinterpret_cast<const uint4*>(rows + 64 * i);
+          const uint64_t Gp[4] = {bf2_to_f2(w.x), bf2_to_f2(w.y), bf2_to_f2(w.z), bf2_to_f2(w.w)};
+          const float hpo = hr[CF::POST + i];
+          const uint64_t hh = f2pack(hpo, hpo);
+#pragma unroll
+          for (int p = 0; p < 4; ++p) gfa[p] = f2fma(hh, Gp[p], gfa[p]);
+          const float4 h0 = *reinterpret_cast<const float4*>(hr + CF::RES + N * i);
+          const float4 h1 = *reinterpret_cast<const float4*>(hr + CF::RES + N * i + 4);
+          const float hres[N] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+#pragma unroll
+          for (int j = 0; j < N; ++j) {
+            const uint64_t hj = f2pack(hres[j], hres[j]);
+#pragma unroll
+            for (int p = 0; p < 4; ++p) acc[j][p] = f2fma(hj, Gp[p], acc[j][p]);
+          }
+        }
+        if (vld) {
+          const float nk = -hr[M];
+          const uint64_t kk = f2pack(nk, nk);
+#pragma unroll
+          for (int j = 0; j < N; ++j) {
+            const uint32_t xw[4] = {Xp[j].x, Xp[j].y, Xp[j].z, Xp[j].w};
+            uint32_t o[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) o[p] = f2_to_bf2(f2fma(kk, bf2_to_f2(xw[p]), acc[j][p]));
+            __stcs(reinterpret_cast<uint4*>(gx + (t * N + j) * C + c),
+                   make_uint4(o[0], o[1], o[2], o[3]));
+          }
+          if (gf != nullptr)
+            __stcs(reinterpret_cast<uint4*>(gf + t * C + c),
+                   make_uint4(f2_to_bf2(gfa[0]), f2_to_bf2(gfa[1]), f2_to_bf2(gfa[2]),
+                              f2_to_bf2(gfa[3])));
+        }
+        __syncwarp();  // the transpose buffer and the slot are rewritten later
       }
+      if (!ok) break;
+      tc::tc_fence_before();
       __syncwarp();
+      if (lane == 0) tc::mbar_arrive(dempty(d));
     }
+    cp_async_wait0();
   }
   tc::tc_fence_before();
   __syncthreads();
   if (warp == 1) {
-    // an MMA still running after a failed wait finishes before TMEM is freed
-    if (!done && lane == 0 && okall) tc::mbar_wait(mma_bar, 0, nullptr, tc::kDrainWaitNs);
-    __syncwarp();
     tc::tc_fence_after();
-    tc::tmem_dealloc(tmem, A_TMEM);
+    tc::tmem_dealloc(tmem, F_TMEM);
   }
 }
 
-// ------------------------------------------------------- grad_x, grad_f_out
-// One CTA visit per token: the token's H record in shared memory, its threads
-// over 8-channel vectors of all eight streams.  CTA 0 also finishes grad_b
-// and grad_alpha from the mapping's per-tile partial sums in a fixed order.
-__global__ void __launch_bounds__(ap8::B_NT) k_gx8(int64_t T, int64_t C,
-                                                   const __nv_bfloat16* __restrict__ x,
-                                                   const __nv_bfloat16* __restrict__ G,
-                                                   const __nv_bfloat16* __restrict__ g,
-                                                   const float* __restrict__ phiu,
-                                                   const float* __restrict__ coef,
-                                                   const float* __restrict__ part, int nparts,
-                                                   __nv_bfloat16* __restrict__ gx,
-                                                   __nv_bfloat16* __restrict__ gf,
-                                                   float* __restrict__ grad_b,
-                                                   float* __restrict__ grad_alpha, int ag) {
+// grad_b and grad_alpha: the mapping's per-tile partial sums in a fixed order
+// (warp w adds partials w, w + 4, ...; then the four warps' sums in order).
+__global__ void __launch_bounds__(ap8::B_NT) k_bias8(const float* __restrict__ part, int nparts,
+                                                     float* __restrict__ grad_b,
+                                                     float* __restrict__ grad_alpha, int ag) {
   using namespace ap8;
   using CF = Coef<N>;
-  __shared__ float hs[CF::SIZE];
-  __shared__ float wsum[4][M + 3];
+  constexpr int NC = M + 3;
+  __shared__ float wsum[4][NC];
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  if (blockIdx.x == 0) {
-    constexpr int NC = M + 3;
-    for (int col = lane; col < NC; col += 32) {
-      float s = 0.0f;
-      for (int q = warp; q < nparts; q += 4) s += __ldg(part + (int64_t)q * CF::DZ_SIZE + col);
-      wsum[warp][col] = s;
-    }
-    __syncthreads();
-    for (int col = tid; col < NC; col += B_NT) {
-      const float a = ((wsum[0][col] + wsum[1][col]) + wsum[2][col]) + wsum[3][col];
-      if (col < M) grad_b[col] = a;
-      else if (ag == 3) grad_alpha[col - M] = a;
-      wsum[0][col] = a;
-    }
-    __syncthreads();
-    if (ag != 3 && tid == 0) *grad_alpha = (wsum[0][M] + wsum[0][M + 1]) + wsum[0][M + 2];
+  for (int col = lane; col < NC; col += 32) {
+    float s = 0.0f;
+    for (int q = warp; q < nparts; q += 4) s += __ldg(part + (int64_t)q * CF::DZ_SIZE + col);
+    wsum[warp][col] = s;
   }
-  const int64_t nv = C / 8;
-  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-    __syncthreads();
-    for (int e = tid; e < CF::SIZE; e += B_NT) hs[e] = __ldg(coef + t * CF::SIZE + e);
-    __syncthreads();
-    const float kappa = hs[CF::KAPPA];
-    for (int64_t v = tid; v < nv; v += B_NT) {
-      const int64_t c = v * 8;
-      float Gv[N][8], gv[8];
-#pragma unroll
-      for (int i = 0; i < N; ++i)
-        unpack8b(__ldcs(reinterpret_cast<const uint4*>(G + (t * N + i) * C + c)), Gv[i]);
-      unpack8b(__ldcs(reinterpret_cast<const uint4*>(g + t * C + c)), gv);
-      if (gf != nullptr) {
-        float o[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          float a = 0.0f;
-#pragma unroll
-          for (int i = 0; i < N; ++i) a = fmaf(hs[CF::POST + i], Gv[i][e], a);
-          o[e] = a;
-        }
-        __stcs(reinterpret_cast<uint4*>(gf + t * C + c), pack8b(o));
-      }
-#pragma unroll 1
-      for (int jj = 0; jj < N; ++jj) {
-        float xv[8], o[8];
-        unpack8b(__ldcs(reinterpret_cast<const uint4*>(x + (t * N + jj) * C + c)), xv);
-        const float4* pu = reinterpret_cast<const float4*>(phiu + (t * N + jj) * C + c);
-        const float4 p0 = __ldcs(pu), p1 = __ldcs(pu + 1);
-        const float pv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          float a = fmaf(hs[CF::PRE + jj], gv[e], pv[e]);
-#pragma unroll
-          for (int i = 0; i < N; ++i) a = fmaf(hs[CF::RES + i * N + jj], Gv[i][e], a);
-          o[e] = fmaf(-kappa, xv[e], a);
-        }
-        __stcs(reinterpret_cast<uint4*>(gx + (t * N + jj) * C + c), pack8b(o));
-      }
-    }
+  __syncthreads();
+  for (int col = tid; col < NC; col += B_NT) {
+    const float a = ((wsum[0][col] + wsum[1][col]) + wsum[2][col]) + wsum[3][col];
+    if (col < M) grad_b[col] = a;
+    else if (ag == 3) grad_alpha[col - M] = a;
+    wsum[0][col] = a;
   }
+  __syncthreads();
+  if (ag != 3 && tid == 0) *grad_alpha = (wsum[0][M] + wsum[0][M + 1]) + wsum[0][M + 2];
 }
 
 // --------------------------------------------------------------- grad_phi
@@ -426,9 +588,9 @@ __global__ void __launch_bounds__(ap8::C_NT) k_gphi8(const __grid_constant__ CUt
 // ------------------------------------------------------------------ host
 cudaError_t apply8_tc_dispatch(int64_t T, int64_t C, const void* x, const void* phi_split,
                                const void* G, const void* g, const float* coef, const void* urec,
-                               const float* part, int nparts, float* phiu, void* gx, void* gf,
-                               float* gphi, float* gb, float* ga, int ag, int* st,
-                               int64_t wait_ns, cudaStream_t s) {
+                               const float* part, int nparts, void* gx, void* gf, float* gphi,
+                               float* gb, float* ga, int ag, int* st, int64_t wait_ns,
+                               cudaStream_t s) {
   using namespace ap8;
   const uint64_t wl = tc::wait_limit(wait_ns);
   CUtensorMap mu, mx;
@@ -445,19 +607,23 @@ cudaError_t apply8_tc_dispatch(int64_t T, int64_t C, const void* x, const void* 
   e = make_tmap_bf16(&mx, x, 3, dx, sx, bx, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
 
-  const int ntt = (int)((T + TT - 1) / TT);
-  const int ncb_a = (int)((C + KB - 1) / KB);
-  e = cudaFuncSetAttribute(k_phiu8, cudaFuncAttributeMaxDynamicSharedMemorySize, A_SMEM);
+  const int64_t ntt = (T + TT - 1) / TT;
+  const int nsl = (int)((C + FS - 1) / FS);
+  const int64_t nitems = ntt * nsl;
+  int dev = 0, nsm = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t grid_a = nitems < nsm ? nitems : nsm;
+  e = cudaFuncSetAttribute(k_gxu8, cudaFuncAttributeMaxDynamicSharedMemorySize, F_SMEM);
   if (e != cudaSuccess) return e;
-  k_phiu8<<<(unsigned)((int64_t)ntt * N * ncb_a), A_NT, A_SMEM, s>>>(mu, (const __nv_bfloat16*)phi_split, T, C, ncb_a, phiu, st,
-                                                                    wl);
+  k_gxu8<<<(unsigned)grid_a, F_NT, F_SMEM, s>>>(
+      mu, (const __nv_bfloat16*)phi_split, T, C, nsl, nitems, (const __nv_bfloat16*)x,
+      (const __nv_bfloat16*)G, (const __nv_bfloat16*)g, coef, (__nv_bfloat16*)gx,
+      (__nv_bfloat16*)gf, st, wl);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
-  const int64_t grid_b = T < 148 * 8 ? T : 148 * 8;
-  k_gx8<<<(unsigned)grid_b, B_NT, 0, s>>>(T, C, (const __nv_bfloat16*)x, (const __nv_bfloat16*)G,
-                                          (const __nv_bfloat16*)g, phiu, coef, part, nparts,
-                                          (__nv_bfloat16*)gx, (__nv_bfloat16*)gf, gb, ga, ag);
+  k_bias8<<<1, B_NT, 0, s>>>(part, nparts, gb, ga, ag);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 

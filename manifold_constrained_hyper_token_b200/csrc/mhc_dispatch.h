@@ -70,15 +70,15 @@ cudaError_t map8_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float ep
                              const void* G, const void* g, const void* f, const float* red,
                              float* coef, void* urec, float* part, int* st, int64_t wait_ns,
                              cudaStream_t s);
-// k_apply8_tc.cu (bf16, n = 8): the apply as phi u on the tensor cores into
-// phiu (fp32 [T][8][C] scratch), grad_x / grad_f_out on the CUDA cores, and
-// grad_phi as a tensor-core contraction over the tokens; phi_split is the
-// mapping's bf16 split copy of phi^T.  gf == nullptr skips grad_f_out.
+// k_apply8_tc.cu (bf16, n = 8): grad_x / grad_f_out with phi u on the tensor
+// cores (the accumulators stay on chip), grad_phi as a tensor-core contraction
+// over the tokens, and grad_b / grad_alpha from the partial sums; phi_split is
+// the mapping's bf16 split copy of phi^T.  gf == nullptr skips grad_f_out.
 cudaError_t apply8_tc_dispatch(int64_t T, int64_t C, const void* x, const void* phi_split,
                                const void* G, const void* g, const float* coef, const void* urec,
-                               const float* part, int nparts, float* phiu, void* gx, void* gf,
-                               float* gphi, float* gb, float* ga, int ag, int* st,
-                               int64_t wait_ns, cudaStream_t s);
+                               const float* part, int nparts, void* gx, void* gf, float* gphi,
+                               float* gb, float* ga, int ag, int* st, int64_t wait_ns,
+                               cudaStream_t s);
 size_t map8_tc_phi_bytes(int64_t C);
 
 // k_proj16_tc.cu (bf16, n = 16): splits phi into the tiled bf16 copy phi_t
