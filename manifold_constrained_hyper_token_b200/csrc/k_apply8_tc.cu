@@ -52,19 +52,21 @@ constexpr int FN = N * FS;              // MMA N: 256 columns, column 32 j + cha
 constexpr int F_U_OFF = 0;              // U tile: three atoms (48 KB)
 constexpr int F_P_OFF = 3 * ATOM;       // phi: 16 atoms (stream j, 16-channel half) of PHB
 constexpr int F_W_OFF = F_P_OFF + 2 * N * PHB;  // the epilogue warps' areas
-constexpr int NEPI = 4;                 // epilogue warps, one per TMEM lane quarter
+constexpr int NEPI = 8;                 // epilogue warps: two per TMEM lane quarter
 constexpr int CK = 8;                   // tokens per epilogue step
 constexpr int XTS = 260;                // row stride (floats) of the transpose buffer
-constexpr int RS = (N + 1) * 64;        // a token's staged rows (grad_x_next x 8, grad_h_in)
+constexpr int RS = (2 * N + 1) * 64;    // a token's staged rows: grad_x_next x 8, x x 8, grad_h_in
+constexpr int RX = N * 64;              // offset of the x rows in them
+constexpr int RG = 2 * N * 64;          // and of the grad_h_in row
 constexpr int HS = 84;                  // H record in shared memory: res, pre, post, kappa
 constexpr int SL_H = CK * RS;           // ring slot: [CK][RS] rows, then [CK][HS] records
 constexpr int SLOT = SL_H + CK * HS * 4;
-constexpr int NSLOT = 3;                // steps staged: the current one and two ahead
+constexpr int NSLOT = 2;                // steps staged: the current one and the next
 constexpr int W_RING = CK * XTS * 4;
 constexpr int W_BYTES = W_RING + NSLOT * SLOT;
-constexpr int F_DATA = F_W_OFF + NEPI * W_BYTES;
+constexpr int F_DATA = F_W_OFF + 4 * W_BYTES;   // one area per lane quarter
 constexpr int F_SMEM = F_DATA + 1024 + 128;
-constexpr int F_NT = (2 + NEPI) * 32;   // TMA, MMA, epilogue x4
+constexpr int F_NT = (2 + NEPI) * 32;   // TMA, MMA, epilogue x8
 constexpr uint32_t F_TMEM = 512;
 static_assert(F_P_OFF % 1024 == 0 && F_W_OFF % 1024 == 0, "operand alignment");
 static_assert(W_BYTES % 16 == 0 && SLOT % 16 == 0 && W_RING % 16 == 0, "alignment");
@@ -92,12 +94,15 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 __device__ __forceinline__ void cp_async_wait0() {
   asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
-// wait until at most two committed groups of this thread are still in flight
-__device__ __forceinline__ void cp_async_wait2() {
-  asm volatile("cp.async.wait_group 2;" ::: "memory");
+// wait until at most one committed group of this thread is still in flight
+__device__ __forceinline__ void cp_async_wait1() {
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
 }
 // Paired fp32 arithmetic (one fma.rn.f32x2 = two IEEE fp32 FMAs).
 __device__ __forceinline__ uint64_t f2pack(float x, float y) {
@@ -127,13 +132,14 @@ __device__ __forceinline__ uint32_t f2_to_bf2(uint64_t v) {
 // the CTAs work on neighbouring slices of the same token rows at any time.
 // Warp 0 loads each item's U tile (when the tile changes) and the 16 phi atoms
 // of its slice into single-buffered operands; warp 1 issues the MMAs into the
-// item's accumulator (columns 256 (k & 1)..); warps 2..5 each take the 32
-// tokens of their TMEM lane quarter in four steps of 8 tokens.  A step's
-// grad_x_next and grad_h_in rows and H records are copied into a three-slot
-// ring two steps ahead (cp.async, 16 bytes per lane, 4 lanes per 64-byte row
-// piece); x is loaded into registers at the start of the step; the 8 tokens'
-// D rows go through a transpose buffer, and the lanes then work as 8 tokens
-// x 4 groups of 8 channels over all 8 streams.
+// item's accumulator (columns 256 (k & 1)..); warps 2..9 work in pairs, one
+// pair per TMEM lane quarter, on its 32 tokens in four steps of 8 tokens,
+// each warp of a pair on four of the eight streams.  A step's x, grad_x_next
+// and grad_h_in rows and H records are copied into the pair's two-slot ring
+// one step ahead (cp.async, 16 bytes per lane, 4 lanes per 64-byte row piece);
+// the 8 tokens' D rows go through the pair's transpose buffer, and the lanes
+// then work as 8 tokens x 4 groups of 8 channels.  A 64-thread named barrier orders the pair's shared
+// buffers.
 __global__ void __launch_bounds__(ap8::F_NT, 1) k_gxu8(
     const __grid_constant__ CUtensorMap tm_u, const __nv_bfloat16* __restrict__ phi_t, int64_t T,
     int64_t C, int nsl, int64_t nitems, const __nv_bfloat16* __restrict__ x,
@@ -145,10 +151,12 @@ __global__ void __launch_bounds__(ap8::F_NT, 1) k_gxu8(
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
-  // op_full op_empty dfull[2] dempty[2] fin
+  // op_full op_empty dfull[2] dempty[2] fin, the TMEM address, the abort flag
+  // and the epilogue pairs' wait results
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + F_DATA);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 7);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* pair_ok = reinterpret_cast<volatile int*>(tmem_slot + 2);  // [4][2]
   const uint32_t op_full = tc::smem_u32(bars), op_empty = tc::smem_u32(bars + 1);
   auto dfull = [&](int d) { return tc::smem_u32(bars + 2 + d); };
   auto dempty = [&](int d) { return tc::smem_u32(bars + 4 + d); };
@@ -260,87 +268,99 @@ __global__ void __launch_bounds__(ap8::F_NT, 1) k_gxu8(
     }
   } else {
     // ----------------------------------------------------------- epilogue
+    // warps qd + 2 and qd + 6 (mod 4 = qd) share TMEM lane quarter qd, its
+    // transpose buffer and its ring; warp half hw takes streams 4 hw .. 4 hw + 3
     const int ew = warp - 2;
     const int qd = warp & 3;             // TMEM lane quarter: tokens 32 qd .. 32 qd + 31
-    uint8_t* wbase = smem + F_W_OFF + ew * W_BYTES;
+    const int hw = ew >> 2;
+    const int pbar = 1 + qd;             // named barrier of the pair
+    uint8_t* wbase = smem + F_W_OFF + qd * W_BYTES;
     float* xt = reinterpret_cast<float*>(wbase);
     const uint32_t ring = tc::smem_u32(wbase + W_RING);
     const int r = lane >> 2, q = lane & 3;  // token of the step, 8-channel group
-    // this lane's share of a step's H records: chunks f = lane + 32 k of the
-    // 8 x 21 16-byte chunks (rows [0, 80) and kappa of each token)
-    int h_tok[6], h_src[6], h_dst[6];
+    // this warp's share of a step's H records: chunks f = lane + 32 k
+    // (k = 3 hw .. 3 hw + 2) of the 8 x 21 16-byte chunks (rows [0, 80) and
+    // kappa of each token)
+    int h_tok[3], h_src[3], h_dst[3];
 #pragma unroll
-    for (int k = 0; k < 6; ++k) {
-      const int f = lane + 32 * k;
+    for (int k = 0; k < 3; ++k) {
+      const int f = lane + 32 * (3 * hw + k);
       const int tk = f / 21, kk = f % 21;
       h_tok[k] = f < CK * 21 ? tk : CK;
       h_src[k] = tk * CF::SIZE + (kk < 20 ? 4 * kk : CF::KAPPA);
       h_dst[k] = SL_H + (tk * HS + 4 * kk) * 4;
     }
-    // stage step s (4 steps of 8 tokens per item) into ring slot s % 3: the
-    // step's grad_x_next and grad_h_in rows and its H records
-    auto stage = [&](int64_t s) {
-      const int64_t it = blockIdx.x + (s >> 2) * (int64_t)gridDim.x;
-      if (it < nitems) {
-        const uint32_t dst = ring + (uint32_t)((s % NSLOT) * SLOT);
-        const int64_t tb = (it / nsl) * TT + 32 * qd + CK * (int)(s & 3);
-        const int64_t t = tb + r, c = (it % nsl) * FS + 8 * q;
+    // stage this warp's half of step s = (item (tile, slice), ci) into ring
+    // slot s % 2: grad_x_next and x rows 4 hw .. 4 hw + 3 (and grad_h_in for
+    // hw = 1) and a third of the H records
+    auto stage = [&](int s, int tile, int sl, int ci) {
+      if (tile >= 0) {
+        const uint32_t dst = ring + (uint32_t)((s & 1) * SLOT);
+        const int64_t tb = (int64_t)tile * TT + 32 * qd + CK * ci;
+        const int64_t t = tb + r, c = (int64_t)sl * FS + 8 * q;
         if (t < T && c < C) {
           const uint32_t rd = dst + (uint32_t)(r * RS + 16 * q);
+          const int64_t off = (t * N + 4 * hw) * C + c;
+          const __nv_bfloat16* pG = G + off;
+          const __nv_bfloat16* pX = x + off;
 #pragma unroll
-          for (int i = 0; i < N; ++i) cp_async16(rd + 64 * i, G + (t * N + i) * C + c);
-          cp_async16(rd + 64 * N, g + t * C + c);
+          for (int i = 0; i < 4; ++i) {
+            cp_async16(rd + 64 * (4 * hw + i), pG + i * C);
+            cp_async16(rd + RX + 64 * (4 * hw + i), pX + i * C);
+          }
+          if (hw == 1) cp_async16(rd + RG, g + t * C + c);
         }
+        const float* hsrc = coef + tb * CF::SIZE;
 #pragma unroll
-        for (int k = 0; k < 6; ++k)
-          if (h_tok[k] < CK && tb + h_tok[k] < T)
-            cp_async16(dst + (uint32_t)h_dst[k], coef + tb * CF::SIZE + h_src[k]);
+        for (int k = 0; k < 3; ++k)
+          if (h_tok[k] < CK && tb + h_tok[k] < T) cp_async16(dst + (uint32_t)h_dst[k], hsrc + h_src[k]);
       }
       cp_async_commit();
     };
-    stage(0);
-    stage(1);
-    int64_t s = 0;
+    const int nit = (int)nitems, grid = (int)gridDim.x;
+    int it = (int)blockIdx.x;
+    int tile = it / nsl, sl = it - tile * nsl;
+    stage(0, tile, sl, 0);
+    int s = 0;
     bool ok = true;
     int li = 0;
-    for (int64_t it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++li) {
+    for (; it < nit && ok; it += grid, ++li) {
       const int d = li & 1;
-      const int64_t c = (it % nsl) * FS + 8 * q;
-      const int64_t tile0 = (it / nsl) * TT + 32 * qd;
+      const int itn = it + grid;
+      const int tilen = itn < nit ? itn / nsl : -1, sln = itn - (itn / nsl) * nsl;
+      const int64_t c = (int64_t)sl * FS + 8 * q;
+      const int64_t tile0 = (int64_t)tile * TT + 32 * qd;
       const uint32_t taddr = tmem + (uint32_t)(d * FN) + ((uint32_t)(32 * qd) << 16);
 #pragma unroll 1
       for (int ci = 0; ci < 4; ++ci, ++s) {
-        stage(s + 2);
+        if (ci < 3) stage(s + 1, tile, sl, ci + 1);
+        else stage(s + 1, tilen, sln, 0);
         const int64_t t = tile0 + CK * ci + r;
         const bool vld = t < T && c < C;
-        // x is needed last: its loads fly while D is turned around
-        uint4 Xp[N];
-#pragma unroll
-        for (int i = 0; i < N; ++i) Xp[i] = make_uint4(0, 0, 0, 0);
-        if (vld) {
-#pragma unroll
-          for (int i = 0; i < N; ++i)
-            Xp[i] = __ldcs(reinterpret_cast<const uint4*>(x + (t * N + i) * C + c));
-        }
         if (ci == 0) {
+          // both warps of the pair take the same decision
           bool okw = tc::mbar_wait(dfull(d), (uint32_t)(li >> 1) & 1u, abort_flag, wait_ns);
+          okw = __all_sync(0xffffffffu, okw);
           if (!okw && !*abort_flag) give_up();
-          ok = __all_sync(0xffffffffu, okw);
+          if (lane == 0) pair_ok[2 * qd + hw] = okw ? 1 : 0;
+          named_bar_sync(pbar, 64);
+          ok = pair_ok[2 * qd] != 0 && pair_ok[2 * qd + 1] != 0;
           if (!ok) break;
           tc::tc_fence_after();
         }
-        // D rows of the step's 8 tokens (lanes 8 ci .. 8 ci + 7 of the quarter)
-        // into the transpose buffer, 64 columns per TMEM wait
+        // this warp's 128 D columns of the step's 8 tokens (lanes 8 ci ..
+        // 8 ci + 7 of the quarter) into the transpose buffer
         const int row = lane - CK * ci;
         const bool mine = row >= 0 && row < CK;
 #pragma unroll 1
-        for (int kb = 0; kb < FN / 64; ++kb) {
+        for (int kb = 0; kb < 2; ++kb) {
+          const int col = 128 * hw + 64 * kb;
           float v[4][16];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) tc::tmem_ld16(taddr + 64 * kb + 16 * u, v[u]);
+          for (int u = 0; u < 4; ++u) tc::tmem_ld16(taddr + col + 16 * u, v[u]);
           tc::tmem_ld_wait();
           if (mine) {
-            float* dst = xt + row * XTS + 64 * kb;
+            float* dst = xt + row * XTS + col;
 #pragma unroll
             for (int u = 0; u < 4; ++u)
 #pragma unroll
@@ -349,33 +369,39 @@ __global__ void __launch_bounds__(ap8::F_NT, 1) k_gxu8(
                     make_float4(v[u][4 * e], v[u][4 * e + 1], v[u][4 * e + 2], v[u][4 * e + 3]);
           }
         }
-        cp_async_wait2();  // this step's staged rows and records
-        __syncwarp();
-        const uint8_t* slot = wbase + W_RING + (s % NSLOT) * SLOT;
+        if (ci == 3) {
+          // the item's accumulator is free for the MMAs two items on
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(dempty(d));
+        }
+        cp_async_wait1();           // this warp's copies of the step
+        named_bar_sync(pbar, 64);   // and the other warp's, and both halves of D
+        const uint8_t* slot = wbase + W_RING + (s & 1) * SLOT;
         const uint8_t* rows = slot + r * RS + 16 * q;
         const float* hr = reinterpret_cast<const float*>(slot + SL_H) + r * HS;
-        // acc[j][p]: channels 2p, 2p + 1 of stream j, starting from phi u
-        uint64_t acc[N][4];
+        // acc[jj][p]: channels 2p, 2p + 1 of stream 4 hw + jj, from phi u
+        uint64_t acc[4][4];
 #pragma unroll
-        for (int j = 0; j < N; ++j) {
-          const ulonglong2 a0 = *reinterpret_cast<const ulonglong2*>(xt + r * XTS + 32 * j + 8 * q);
-          const ulonglong2 a1 =
-              *reinterpret_cast<const ulonglong2*>(xt + r * XTS + 32 * j + 8 * q + 4);
-          acc[j][0] = a0.x;
-          acc[j][1] = a0.y;
-          acc[j][2] = a1.x;
-          acc[j][3] = a1.y;
+        for (int jj = 0; jj < 4; ++jj) {
+          const float* a = xt + r * XTS + 32 * (4 * hw + jj) + 8 * q;
+          const ulonglong2 a0 = *reinterpret_cast<const ulonglong2*>(a);
+          const ulonglong2 a1 = *reinterpret_cast<const ulonglong2*>(a + 4);
+          acc[jj][0] = a0.x;
+          acc[jj][1] = a0.y;
+          acc[jj][2] = a1.x;
+          acc[jj][3] = a1.y;
         }
         {
-          const uint4 gw = *reinterpret_cast<const uint4*>(rows + 64 * N);
+          const uint4 gw = *reinterpret_cast<const uint4*>(rows + RG);
           const uint64_t gp[4] = {bf2_to_f2(gw.x), bf2_to_f2(gw.y), bf2_to_f2(gw.z),
                                   bf2_to_f2(gw.w)};
 #pragma unroll
-          for (int j = 0; j < N; ++j) {
-            const float h = hr[CF::PRE + j];
+          for (int jj = 0; jj < 4; ++jj) {
+            const float h = hr[CF::PRE + 4 * hw + jj];
             const uint64_t hh = f2pack(h, h);
 #pragma unroll
-            for (int p = 0; p < 4; ++p) acc[j][p] = f2fma(hh, gp[p], acc[j][p]);
+            for (int p = 0; p < 4; ++p) acc[jj][p] = f2fma(hh, gp[p], acc[jj][p]);
           }
         }
         uint64_t gfa[4] = {0, 0, 0, 0};
@@ -383,43 +409,43 @@ __global__ void __launch_bounds__(ap8::F_NT, 1) k_gxu8(
         for (int i = 0; i < N; ++i) {
           const uint4 w = *reinterpret_cast<const uint4*>(rows + 64 * i);
           const uint64_t Gp[4] = {bf2_to_f2(w.x), bf2_to_f2(w.y), bf2_to_f2(w.z), bf2_to_f2(w.w)};
-          const float hpo = hr[CF::POST + i];
-          const uint64_t hh = f2pack(hpo, hpo);
+          if (hw == 0) {
+            const float hpo = hr[CF::POST + i];
+            const uint64_t hh = f2pack(hpo, hpo);
 #pragma unroll
-          for (int p = 0; p < 4; ++p) gfa[p] = f2fma(hh, Gp[p], gfa[p]);
-          const float4 h0 = *reinterpret_cast<const float4*>(hr + CF::RES + N * i);
-          const float4 h1 = *reinterpret_cast<const float4*>(hr + CF::RES + N * i + 4);
-          const float hres[N] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+            for (int p = 0; p < 4; ++p) gfa[p] = f2fma(hh, Gp[p], gfa[p]);
+          }
+          const float4 h = *reinterpret_cast<const float4*>(hr + CF::RES + N * i + 4 * hw);
+          const float hres[4] = {h.x, h.y, h.z, h.w};
 #pragma unroll
-          for (int j = 0; j < N; ++j) {
-            const uint64_t hj = f2pack(hres[j], hres[j]);
+          for (int jj = 0; jj < 4; ++jj) {
+            const uint64_t hj = f2pack(hres[jj], hres[jj]);
 #pragma unroll
-            for (int p = 0; p < 4; ++p) acc[j][p] = f2fma(hj, Gp[p], acc[j][p]);
+            for (int p = 0; p < 4; ++p) acc[jj][p] = f2fma(hj, Gp[p], acc[jj][p]);
           }
         }
         if (vld) {
           const float nk = -hr[M];
           const uint64_t kk = f2pack(nk, nk);
 #pragma unroll
-          for (int j = 0; j < N; ++j) {
-            const uint32_t xw[4] = {Xp[j].x, Xp[j].y, Xp[j].z, Xp[j].w};
+          for (int jj = 0; jj < 4; ++jj) {
+            const uint4 xq = *reinterpret_cast<const uint4*>(rows + RX + 64 * (4 * hw + jj));
+            const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
             uint32_t o[4];
 #pragma unroll
-            for (int p = 0; p < 4; ++p) o[p] = f2_to_bf2(f2fma(kk, bf2_to_f2(xw[p]), acc[j][p]));
-            __stcs(reinterpret_cast<uint4*>(gx + (t * N + j) * C + c),
+            for (int p = 0; p < 4; ++p) o[p] = f2_to_bf2(f2fma(kk, bf2_to_f2(xw[p]), acc[jj][p]));
+            __stcs(reinterpret_cast<uint4*>(gx + (t * N + 4 * hw + jj) * C + c),
                    make_uint4(o[0], o[1], o[2], o[3]));
           }
-          if (gf != nullptr)
+          if (hw == 0 && gf != nullptr)
             __stcs(reinterpret_cast<uint4*>(gf + t * C + c),
                    make_uint4(f2_to_bf2(gfa[0]), f2_to_bf2(gfa[1]), f2_to_bf2(gfa[2]),
                               f2_to_bf2(gfa[3])));
         }
-        __syncwarp();  // the transpose buffer and the slot are rewritten later
+        named_bar_sync(pbar, 64);  // the transpose buffer and the slot are rewritten later
       }
-      if (!ok) break;
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(dempty(d));
+      tile = tilen;
+      sl = sln;
     }
     cp_async_wait0();
   }
@@ -614,6 +640,7 @@ cudaError_t apply8_tc_dispatch(int64_t T, int64_t C, const void* x, const void* 
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   const int64_t grid_a = nitems < nsm ? nitems : nsm;
+  if (nitems > 0x7fffffff - grid_a) return cudaErrorInvalidValue;  // 32-bit item indices
   e = cudaFuncSetAttribute(k_gxu8, cudaFuncAttributeMaxDynamicSharedMemorySize, F_SMEM);
   if (e != cudaSuccess) return e;
   k_gxu8<<<(unsigned)grid_a, F_NT, F_SMEM, s>>>(
