@@ -73,9 +73,11 @@ def test_workspace_size_query(lib):
 def test_wide_tensor_core_workspaces(lib, n):
     """bf16 with n = 8 or 16 takes the tensor-core paths: mhc_pre needs the split phi^T
     copy (2M rows of nC bf16; at n = 16 also the per-token rows of projections, 580
-    floats each), and the backward holds the apply's fp32 phi u scratch [T][n][C] on
-    top of the per-token records.  fp32 activations take the CUDA-core paths, whose
-    forward needs no workspace."""
+    floats each).  At n = 16 the backward holds the apply's fp32 phi u scratch
+    [T][n][C] on top of the per-token records; at n = 8 phi u stays in the apply
+    kernel's tensor memory, so the backward holds the records (coefficients, U rows,
+    C-reductions) and the phi copy only.  fp32 activations take the CUDA-core paths,
+    whose forward needs no workspace."""
     T, C = 4096, 7168
     M = n * n + 2 * n
     bf = _params(n=n, T=T, C=C, dtype=1)
@@ -85,7 +87,13 @@ def test_wide_tensor_core_workspaces(lib, n):
         assert pre >= 2 * M * n * C * 2 + T * 580 * 4
     assert lib.mhc_post_fused_workspace_size(ctypes.byref(bf)) == pre
     bwd = lib.mhc_backward_workspace_size(ctypes.byref(bf))
-    assert bwd >= T * n * C * 4 + 2 * M * n * C * 2 and bwd % 256 == 0
+    records = T * (M + M + 4) * 4   # coefficient records: H, u, kappa (padded)
+    if n == 16:
+        assert bwd >= T * n * C * 4 + 2 * M * n * C * 2 and bwd % 256 == 0
+    else:
+        u_rows, dots = T * 192 * 2, T * M * 4
+        assert bwd >= records + u_rows + dots + 2 * M * n * C * 2 and bwd % 256 == 0
+        assert bwd < T * n * C * 4   # no [T][n][C] fp32 scratch
     f32 = _params(n=n, T=T, C=C, dtype=0)
     assert lib.mhc_pre_workspace_size(ctypes.byref(f32)) == 0
     assert 0 < lib.mhc_backward_workspace_size(ctypes.byref(f32)) < bwd
