@@ -17,7 +17,8 @@
 //             ring; phi_hi comes from the tiled, pre-swizzled phi^T copy the
 //             projection reads; two TMEM accumulators, so one item's epilogue
 //             overlaps the next item's MMAs; fp32 scratch [T][16][C]
-//   k_gx16    grad_x and grad_f_out from that scratch (CUDA cores, 8-byte vectors)
+//   k_gx16    grad_x and grad_f_out from that scratch (CUDA cores, 8-byte vectors,
+//             paired fp32 FMAs)
 //   k_gphi16  grad_phi for 128 rows of phi: D[128 x 288] += X^T (u_hi + u_lo)
 //             over every token tile (tcgen05)
 //
@@ -70,18 +71,6 @@ static_assert(A_STAGE % 1024 == 0 && A_XT_OFF % 1024 == 0, "stage alignment");
 }  // namespace ap16
 
 namespace {
-__device__ __forceinline__ void unpack4b(uint2 q, float (&v)[4]) {
-  v[0] = __uint_as_float(q.x << 16);
-  v[1] = __uint_as_float(q.x & 0xffff0000u);
-  v[2] = __uint_as_float(q.y << 16);
-  v[3] = __uint_as_float(q.y & 0xffff0000u);
-}
-__device__ __forceinline__ uint2 pack4b(const float (&v)[4]) {
-  __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
-  __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
-  return make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b));
-}
-
 // u (fp32, in the coefficient records) -> the bf16 U rows
 __global__ void k_urec16(int64_t T, const float* __restrict__ coef,
                          __nv_bfloat16* __restrict__ urec) {
@@ -293,7 +282,11 @@ __global__ void __launch_bounds__(ap16::A_NT, 1) k_phiu16(
 
 // ------------------------------------------------------- grad_x, grad_f_out
 // One CTA visit per token: its coefficient record in shared memory, its
-// threads over 4-channel vectors of all sixteen streams.
+// threads over 4-channel vectors of all sixteen streams.  A thread keeps the
+// sixteen output streams' sums as fp32 pairs, starting from phi u, and walks
+// the input streams i once: H_res row i comes as four 16-byte shared-memory
+// reads and each grad_x_next vector is widened once.  Per element the terms
+// are added in the order phi u, H_pre g, H_res[0..15] G, -kappa x.
 __global__ void __launch_bounds__(128, 4) k_gx16(int64_t T, int64_t C,
                                               const __nv_bfloat16* __restrict__ x,
                                               const __nv_bfloat16* __restrict__ G,
@@ -304,46 +297,64 @@ __global__ void __launch_bounds__(128, 4) k_gx16(int64_t T, int64_t C,
                                               __nv_bfloat16* __restrict__ gf) {
   using namespace ap16;
   using CF = Coef<N>;
-  __shared__ float hs[CF::SIZE];
+  static_assert(CF::RES % 4 == 0 && N % 4 == 0, "16-byte rows of H_res");
+  __shared__ __align__(16) float hs[CF::SIZE];
   const int tid = threadIdx.x;
   const int64_t nv = C / 4;
   for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
     __syncthreads();
     for (int e = tid; e < CF::SIZE; e += blockDim.x) hs[e] = __ldg(coef + t * CF::SIZE + e);
     __syncthreads();
-    const float kappa = hs[CF::KAPPA];
+    const float nk = -hs[CF::KAPPA];
     for (int64_t v = tid; v < nv; v += blockDim.x) {
       const int64_t c = v * 4;
-      float Gv[N][4], gv[4];
+      uint64_t acc[N][2];
 #pragma unroll
-      for (int i = 0; i < N; ++i)
-        unpack4b(__ldcs(reinterpret_cast<const uint2*>(G + (t * N + i) * C + c)), Gv[i]);
-      unpack4b(__ldcs(reinterpret_cast<const uint2*>(g + t * C + c)), gv);
-      if (gf != nullptr) {
-        float o[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float a = 0.0f;
-#pragma unroll
-          for (int i = 0; i < N; ++i) a = fmaf(hs[CF::POST + i], Gv[i][e], a);
-          o[e] = a;
-        }
-        __stcs(reinterpret_cast<uint2*>(gf + t * C + c), pack4b(o));
+      for (int j = 0; j < N; ++j) {
+        const ulonglong2 p = __ldcs(reinterpret_cast<const ulonglong2*>(phiu + (t * N + j) * C + c));
+        acc[j][0] = p.x;
+        acc[j][1] = p.y;
       }
-#pragma unroll 2
-      for (int jj = 0; jj < N; ++jj) {
-        float xv[4], o[4];
-        unpack4b(__ldcs(reinterpret_cast<const uint2*>(x + (t * N + jj) * C + c)), xv);
-        const float4 p = __ldcs(reinterpret_cast<const float4*>(phiu + (t * N + jj) * C + c));
-        const float pv[4] = {p.x, p.y, p.z, p.w};
+      {
+        const uint2 gw = __ldcs(reinterpret_cast<const uint2*>(g + t * C + c));
+        const uint64_t gp[2] = {bf2_to_f2(gw.x), bf2_to_f2(gw.y)};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float a = fmaf(hs[CF::PRE + jj], gv[e], pv[e]);
-#pragma unroll
-          for (int i = 0; i < N; ++i) a = fmaf(hs[CF::RES + i * N + jj], Gv[i][e], a);
-          o[e] = fmaf(-kappa, xv[e], a);
+        for (int j = 0; j < N; ++j) {
+          const uint64_t h = f2pack(hs[CF::PRE + j], hs[CF::PRE + j]);
+          acc[j][0] = f2fma(h, gp[0], acc[j][0]);
+          acc[j][1] = f2fma(h, gp[1], acc[j][1]);
         }
-        __stcs(reinterpret_cast<uint2*>(gx + (t * N + jj) * C + c), pack4b(o));
+      }
+      uint64_t gfa[2] = {0, 0};
+#pragma unroll
+      for (int i = 0; i < N; ++i) {
+        const uint2 w = __ldcs(reinterpret_cast<const uint2*>(G + (t * N + i) * C + c));
+        const uint64_t Gp[2] = {bf2_to_f2(w.x), bf2_to_f2(w.y)};
+        const uint64_t hpo = f2pack(hs[CF::POST + i], hs[CF::POST + i]);
+        gfa[0] = f2fma(hpo, Gp[0], gfa[0]);
+        gfa[1] = f2fma(hpo, Gp[1], gfa[1]);
+#pragma unroll
+        for (int q4 = 0; q4 < N / 4; ++q4) {
+          const float4 h = *reinterpret_cast<const float4*>(hs + CF::RES + N * i + 4 * q4);
+          const float hr[4] = {h.x, h.y, h.z, h.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t hh = f2pack(hr[k], hr[k]);
+            acc[4 * q4 + k][0] = f2fma(hh, Gp[0], acc[4 * q4 + k][0]);
+            acc[4 * q4 + k][1] = f2fma(hh, Gp[1], acc[4 * q4 + k][1]);
+          }
+        }
+      }
+      if (gf != nullptr)
+        __stcs(reinterpret_cast<uint2*>(gf + t * C + c),
+               make_uint2(f2_to_bf2(gfa[0]), f2_to_bf2(gfa[1])));
+      const uint64_t kk = f2pack(nk, nk);
+#pragma unroll
+      for (int j = 0; j < N; ++j) {
+        const uint2 xw = __ldcs(reinterpret_cast<const uint2*>(x + (t * N + j) * C + c));
+        __stcs(reinterpret_cast<uint2*>(gx + (t * N + j) * C + c),
+               make_uint2(f2_to_bf2(f2fma(kk, bf2_to_f2(xw.x), acc[j][0])),
+                          f2_to_bf2(f2fma(kk, bf2_to_f2(xw.y), acc[j][1]))));
       }
     }
   }

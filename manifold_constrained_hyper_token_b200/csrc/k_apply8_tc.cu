@@ -104,27 +104,6 @@ __device__ __forceinline__ void cp_async_wait0() {
 __device__ __forceinline__ void cp_async_wait1() {
   asm volatile("cp.async.wait_group 1;" ::: "memory");
 }
-// Paired fp32 arithmetic (one fma.rn.f32x2 = two IEEE fp32 FMAs).
-__device__ __forceinline__ uint64_t f2pack(float x, float y) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(x), "f"(y));
-  return r;
-}
-__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-// two bf16 (one 32-bit word) widened to an fp32 pair, and back
-__device__ __forceinline__ uint64_t bf2_to_f2(uint32_t w) {
-  return f2pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-}
-__device__ __forceinline__ uint32_t f2_to_bf2(uint64_t v) {
-  float x, y;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(x), "=f"(y) : "l"(v));
-  __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
 }  // namespace
 
 // ------------------------------------------------------- grad_x, grad_f_out

@@ -89,26 +89,6 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
 }
-// Paired fp32 arithmetic (one fma.rn.f32x2 = two IEEE fp32 FMAs).
-__device__ __forceinline__ uint64_t f2pack(float x, float y) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(x), "f"(y));
-  return r;
-}
-__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-// two bf16 (one 32-bit word) widened to an fp32 pair
-__device__ __forceinline__ uint64_t bf2_to_f2(uint32_t w) {
-  return f2pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-}
-__device__ __forceinline__ uint32_t f2_to_bf2(uint64_t v) {
-  float x, y;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(x), "=f"(y) : "l"(v));
-  return pack2(x, y);
-}
 __device__ __forceinline__ void unpack_pairs(uint4 q, uint64_t (&v)[4]) {
   v[0] = bf2_to_f2(q.x);
   v[1] = bf2_to_f2(q.y);

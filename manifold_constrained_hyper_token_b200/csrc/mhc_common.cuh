@@ -294,4 +294,29 @@ struct TcRec8 {
   static constexpr int LO = 96;  // first column of u_lo
 };
 
+// ------------------------------------------------- paired fp32 arithmetic
+// One fma.rn.f32x2 is two IEEE fp32 FMAs on a pair of values held in one
+// 64-bit register (element 0 in the low half).
+__device__ __forceinline__ uint64_t f2pack(float x, float y) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(x), "f"(y));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+// two bf16 (one 32-bit word, element 0 in the low half) widened to an fp32
+// pair, and an fp32 pair rounded back to two bf16
+__device__ __forceinline__ uint64_t bf2_to_f2(uint32_t w) {
+  return f2pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+__device__ __forceinline__ uint32_t f2_to_bf2(uint64_t v) {
+  float x, y;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(x), "=f"(y) : "l"(v));
+  __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
 }  // namespace mhc
