@@ -309,12 +309,10 @@ MHC_API mhc_status mhc_pre_backward(const mhc_params *p, const void *x, const fl
  * a per-token record (n = 4: 208 bytes) and a partial sum per 64 tokens; a
  * problem whose scratch exceeds MHC_NOALLOC_SCRATCH_BYTES is rejected with
  * MHC_ERR_WORKSPACE before any launch (n = 4: up to about 20,000 tokens per
- * call).  The first call on a
- * device looks up the array's device address (cudaGetSymbolAddress) with
- * that device current and caches it; make that first call before any stream
- * capture.  The cached address belongs to the device's primary context: a
- * process that destroys that context (cudaDeviceReset) must not call this
- * entry point on that device afterwards, since the address would be stale.
+ * call).  Every call looks up the array's device address
+ * (cudaGetSymbolAddress) on the current device; nothing is cached, so calls
+ * made after a device reset use the array of the new context.  The first call
+ * on a device may load the module: make it before any stream capture.
  * All calls share the one array and it keeps the last call's
  * contents (nothing in it needs to start at zero): calls whose work can
  * overlap on the GPU (on different streams, or from several threads without

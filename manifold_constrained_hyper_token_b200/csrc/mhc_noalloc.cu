@@ -12,11 +12,10 @@
 // The scratch is one file-scope __device__ array of MHC_NOALLOC_SCRATCH_BYTES
 // (4 MiB).  Every GPU that loads this library holds it until the process
 // exits.  Host code cannot use the array's name as a device address (in host
-// code it names a host-side shadow), so the device address is looked up with
-// cudaGetSymbolAddress once per device, with that device current, on the first
-// call made on it, and cached.
-#include <mutex>
-
+// code it names a host-side shadow), so every call looks the device address up
+// with cudaGetSymbolAddress on the current device.  Nothing is cached: after a
+// device reset, or once the module is loaded again, the next call gets the
+// array's new address.
 #include "mhc_common.cuh"
 #include "mhc_dispatch.h"
 
@@ -25,24 +24,12 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[MHC_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_setup_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
-
-// Device address of g_noalloc_scratch on the current device (set up on first use).
+// Device address of g_noalloc_scratch on the current device.
 cudaError_t scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return cudaSuccess;
 }
 
