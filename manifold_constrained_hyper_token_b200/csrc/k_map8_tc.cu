@@ -10,26 +10,27 @@
 // backward in one operator, recompute, wider stream buffers).
 //
 // One CTA = 128 tokens (the MMA M).  The token's 8 C inputs stream through a
-// TMA ring in chunks of 16 channels x 8 streams (32-byte rows, 32-byte
-// swizzle): per stream an x tile [128 x 16] (the A operand, K-major) and the
-// rows of the bf16 split copy of phi^T as a [160 x 16] B operand -- the 80
-// logit columns' high parts, then their low parts (phi = hi + lo) -- so
+// TMA ring in chunks of 64 channels x 2 streams (128-byte rows, 128-byte
+// swizzle; chunk cc covers channel group cc / 4 and streams 2 (cc % 4) and
+// 2 (cc % 4) + 1): per stream an x tile [128 x 64] (the A operand, K-major,
+// four K-steps of 16 channels) and, per 16 channels and stream, the rows of the
+// bf16 split copy of phi^T as a [160 x 16] B operand -- the 80 logit columns'
+// high parts, then their low parts (phi = hi + lo) -- so
 // y = D[:, m] + D[:, 80 + m] carries phi to ~16 bits while x is exact.  The
 // split copy is tiled and pre-swizzled, so a chunk's eight phi tiles (40 KB)
-// arrive as one bulk copy.  The library's whole backward runs this kernel in
+// arrive as four bulk copies.  The library's whole backward runs this kernel in
 // the MAP_BWD_DOTS mode (only x staged, three stages): every C-reduction comes
 // from the tensor-core reductions of k_dots_tc.cu.  The training-order
 // backward runs the split mode: <G_i, x_j> and <G_i, f_out> from the post
-// half, <g, x_j> here.
+// half, <g, x_j> here (grad_h_in staged with each chunk).
 //
 // Warp roles: warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs, warps
-// 2..9 reduce: warp 2 + 4h + q covers token rows 32q..32q+31 and stream half
-// h, i.e. the sum of squares of streams 4h..4h+3 and, in the backward,
-// <G_i, x_j> and <G_i, f_out> for i in 4h..4h+3 (all j) and <g, x_j> for j in
-// 4h..4h+3.  The h = 0 warps then run the per-token epilogue (gates,
-// Sinkhorn and its adjoint) with one thread per token and write the same
-// per-token records as the CUDA-core mapping plus the U rows of the n = 8
-// tensor-core apply.
+// 2..9 reduce: warp 2 + 4h + q covers token rows 32q..32q+31 and stream h of
+// each chunk's pair, i.e. the sum of squares of streams h, h + 2, h + 4, h + 6
+// and, in the split backward, <g, x_j> for those streams.  The h = 0 warps
+// then run the per-token epilogue (gates, Sinkhorn and its adjoint) with one
+// thread per token and write the same per-token records as the CUDA-core
+// mapping plus the U rows of the n = 8 tensor-core apply.
 // Every wait is bounded; on timeout the kernel records MHC_ERR_TIMEOUT,
 // drains what it issued, frees TMEM and returns.
 #include "mhc_common.cuh"
@@ -43,30 +44,32 @@ constexpr int N = 8;
 constexpr int M = N * N + 2 * N;     // 80 logits
 constexpr int TM = 128;              // tokens per CTA (MMA M)
 constexpr int NL = 2 * M;            // MMA N: 80 high + 80 low logit columns
-constexpr int CH = 16;               // channels per chunk: 32-byte rows
+constexpr int CH = 64;               // channels per chunk: 128-byte rows
 constexpr int ROW = CH * 2;
-constexpr int XBOX = TM * ROW;       // one stream's x (or grad_x_next) tile: 4 KB
-constexpr int PBOX = NL * ROW;       // one stream's phi^T tile: 5 KB
+constexpr int XBOX = TM * ROW;       // one stream's x (or grad_h_in) tile: 16 KB
+constexpr int SPC = 2;               // streams per chunk
+constexpr int PB = 16;               // channels per block of the tiled phi^T copy
+constexpr int PROW = PB * 2;         // its 32-byte rows
+constexpr int PBOX = NL * PROW;      // one (16-channel block, stream) phi^T tile: 5 KB
 constexpr int NW = 10;
 constexpr int NT = NW * 32;
 constexpr uint32_t TMEM_COLS = 256;
 constexpr int NDH = 4 * N + 4 + 4;   // reductions per stream half: <G_i,x_j> 32, <G_i,f> 4, <g,x_j> 4
 
 template <int MODE> struct Cfg {
-  static constexpr bool FULLB = MODE == MAP_BWD;
-  static constexpr bool BWD = MODE == MAP_BWD || MODE == MAP_BWD_SPLIT || MODE == MAP_BWD_DOTS;
-  static constexpr bool STAGE_G = MODE == MAP_BWD || MODE == MAP_BWD_SPLIT;  // grad_h_in staged
-  static constexpr int X_OFF = 0;
-  static constexpr int P_OFF = N * XBOX;
-  static constexpr int G_OFF = P_OFF + N * PBOX;                 // grad_x_next (full backward)
-  static constexpr int GG_OFF = FULLB ? G_OFF + N * XBOX : G_OFF;  // grad_h_in (backward)
-  static constexpr int F_OFF = GG_OFF + XBOX;                     // f_out (full backward)
-  static constexpr int STAGE = FULLB ? F_OFF + XBOX : (STAGE_G ? GG_OFF + XBOX : G_OFF);
+  static_assert(MODE == MAP_FWD || MODE == MAP_BWD_SPLIT || MODE == MAP_BWD_DOTS, "mode");
+  static constexpr bool BWD = MODE == MAP_BWD_SPLIT || MODE == MAP_BWD_DOTS;
+  static constexpr bool STAGE_G = MODE == MAP_BWD_SPLIT;  // grad_h_in staged
+  static constexpr int X_OFF = 0;                         // x tiles of the chunk's two streams
+  static constexpr int P_OFF = SPC * XBOX;                // phi^T tiles: (16-channel step k, stream) at (2k + s)
+  static constexpr int GG_OFF = P_OFF + SPC * (CH / PB) * PBOX;  // grad_h_in (split backward)
+  static constexpr int STAGE = STAGE_G ? GG_OFF + XBOX : GG_OFF;
   static constexpr int NS = STAGE_G ? 2 : 3;
   // the stages, reused after the chunk loop by the epilogue; the backward
-  // epilogue keeps Sinkhorn checkpoints there, so the split backward (smaller
-  // stages) asks for the full backward's size
+  // epilogue keeps Sinkhorn checkpoints there, so the backward asks for at
+  // least 224 KB
   static constexpr int DATA = BWD && NS * STAGE < 229376 ? 229376 : NS * STAGE;
+  static_assert(STAGE % 1024 == 0 && GG_OFF % 1024 == 0, "128-byte swizzle atoms");
   static constexpr int SMEM = DATA + 1024 /*align*/ + 256 /*barriers, flags*/;
   static_assert(SMEM <= 232448, "shared memory");
 };
@@ -83,10 +86,10 @@ __device__ __forceinline__ void unpack8(uint4 q, float (&v)[8]) {
   }
 }
 
-// 16-byte piece `c` (0 or 1) of token row `tok` of a [128 x 16] bf16 tile
-// stored with the 32-byte swizzle.
-__device__ __forceinline__ uint4 ld32sw(const uint8_t* tile, int tok, int c) {
-  return *reinterpret_cast<const uint4*>(tile + tok * tcm8::ROW + ((c ^ ((tok >> 2) & 1)) << 4));
+// 16-byte piece `c` (0..7) of token row `tok` of a [128 x 64] bf16 tile
+// stored with the 128-byte swizzle.
+__device__ __forceinline__ uint4 ld128sw(const uint8_t* tile, int tok, int c) {
+  return *reinterpret_cast<const uint4*>(tile + tok * tcm8::ROW + ((c ^ (tok & 7)) << 4));
 }
 
 __device__ __forceinline__ void nbar8(int id, int count) {
@@ -98,8 +101,7 @@ __device__ __forceinline__ void nbar8(int id, int count) {
 template <int MODE>
 __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
     const __grid_constant__ CUtensorMap tm_x, const __nv_bfloat16* __restrict__ phi_t,
-    const __grid_constant__ CUtensorMap tm_G, const __grid_constant__ CUtensorMap tm_g,
-    const __grid_constant__ CUtensorMap tm_f, int64_t T, int64_t C, int iters, float eps,
+    const __grid_constant__ CUtensorMap tm_g, int64_t T, int64_t C, int iters, float eps,
     int ck_period, const float* __restrict__ bias, const float* __restrict__ alpha_p, int ag,
     float* __restrict__ Hpre_o, float* __restrict__ Hpost_o, float* __restrict__ Hres_o,
     float* __restrict__ coef_o, __nv_bfloat16* __restrict__ urec_o, float* __restrict__ part_o,
@@ -107,8 +109,7 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
   using namespace tcm8;
   using CFG = Cfg<MODE>;
   using CF = Coef<N>;
-  constexpr bool BWD = CFG::BWD, FULLB = CFG::FULLB;
-  constexpr bool SPLIT = MODE == MAP_BWD_SPLIT;
+  constexpr bool BWD = CFG::BWD;
   constexpr bool DOTS = MODE == MAP_BWD_DOTS;  // every C-reduction from red_in
   constexpr bool STAGE_G = CFG::STAGE_G;
   constexpr int NS = CFG::NS;
@@ -125,7 +126,7 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t t0 = (int64_t)blockIdx.x * TM;
-  const int nch = (int)((C + CH - 1) / CH);
+  const int nch = (int)((C + CH - 1) / CH) * (N / SPC);  // chunks: channel groups x stream pairs
   const int64_t K = (int64_t)N * C;
 
   if (threadIdx.x == 0) {
@@ -141,10 +142,6 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
   if (warp == 0 && lane == 0) {
     tc::tma_prefetch_desc(&tm_x);
     if constexpr (STAGE_G) tc::tma_prefetch_desc(&tm_g);
-    if constexpr (FULLB) {
-      tc::tma_prefetch_desc(&tm_G);
-      tc::tma_prefetch_desc(&tm_f);
-    }
   }
   if (warp == 1) {
     tc::tmem_alloc(tc::smem_u32(tmem_slot), TMEM_COLS);
@@ -175,19 +172,19 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
         }
         const uint32_t base = tc::smem_u32(smem + s * CFG::STAGE);
         tc::mbar_arrive_expect_tx(full(s), CFG::STAGE);
-        const int c0 = cc * CH;
-        // the chunk's phi^T tiles of all eight streams: one contiguous 40 KB block
-        // of the tiled copy, already in the 32-byte swizzled shared-memory order
-        tc::bulk_load(base + CFG::P_OFF, phi_t + (int64_t)cc * (N * NL * CH), N * PBOX, full(s),
-                      pol_keep);
-        for (int i = 0; i < N; ++i) {
-          tc::tma_load_3d(base + CFG::X_OFF + i * XBOX, &tm_x, full(s), c0, i, (int)t0, pol_stream);
-          if constexpr (FULLB)
-            tc::tma_load_3d(base + CFG::G_OFF + i * XBOX, &tm_G, full(s), c0, i, (int)t0, pol_stream);
-        }
+        const int c0 = (cc >> 2) * CH, j0 = SPC * (cc & 3);
+        // the chunk's phi^T tiles: for each of its four 16-channel blocks, the
+        // tiles of streams j0 and j0 + 1 are one contiguous 10 KB piece of the
+        // tiled copy, already in the 32-byte swizzled shared-memory order
+        for (int k = 0; k < CH / PB; ++k)
+          tc::bulk_load(base + CFG::P_OFF + SPC * k * PBOX,
+                        phi_t + ((int64_t)((cc >> 2) * (CH / PB) + k) * N + j0) * (NL * PB),
+                        SPC * PBOX, full(s), pol_keep);
+        for (int i = 0; i < SPC; ++i)
+          tc::tma_load_3d(base + CFG::X_OFF + i * XBOX, &tm_x, full(s), c0, j0 + i, (int)t0,
+                          pol_stream);
         if constexpr (STAGE_G)
           tc::tma_load_2d(base + CFG::GG_OFF, &tm_g, full(s), c0, (int)t0, pol_stream);
-        if constexpr (FULLB) tc::tma_load_2d(base + CFG::F_OFF, &tm_f, full(s), c0, (int)t0, pol_stream);
         ++issued;
       }
       // every copy issued here has landed before the CTA can exit
@@ -208,10 +205,17 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
         tc::tc_fence_after();
         const uint32_t base = tc::smem_u32(smem + s * CFG::STAGE);
 #pragma unroll
-        for (int i = 0; i < N; ++i) {
-          const uint64_t a = tc::smem_desc(base + CFG::X_OFF + i * XBOX, 16, 8 * ROW, tc::SWZ_32B);
-          const uint64_t bd = tc::smem_desc(base + CFG::P_OFF + i * PBOX, 16, 8 * ROW, tc::SWZ_32B);
-          tc::mma_bf16(tmem, a, bd, idesc, (cc | i) != 0 ? 1u : 0u);
+        for (int i = 0; i < SPC; ++i) {
+#pragma unroll
+          for (int k = 0; k < CH / PB; ++k) {
+            // A: x tile i, 16-channel step k (32 bytes into each 128-byte row);
+            // B: the phi^T tile of block k and stream j0 + i
+            const uint64_t a =
+                tc::smem_desc(base + CFG::X_OFF + i * XBOX + 32 * k, 16, 8 * ROW, tc::SWZ_128B);
+            const uint64_t bd = tc::smem_desc(base + CFG::P_OFF + (SPC * k + i) * PBOX, 16,
+                                              8 * PROW, tc::SWZ_32B);
+            tc::mma_bf16(tmem, a, bd, idesc, (cc | i | k) != 0 ? 1u : 0u);
+          }
         }
         any = true;
         tc::mma_commit(empty(s));
@@ -226,56 +230,47 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
   } else {
     // -------------------------------------------------- CUDA-core reductions
     const int q = warp & 3;              // TMEM lane quarter this warp may read
-    const int h = (warp - 2) >> 2;       // stream half: streams 4h..4h+3
+    const int h = (warp - 2) >> 2;       // stream h of each chunk's pair (streams h, h + 2, ..)
     const int tok = 32 * q + lane;
     float ss = 0.0f;
-    // [0, 32): <G_i, x_j> for i = 4h + r (r = 0..3), j = 0..7, at 8 r + j
-    // [32, 36): <G_i, f> for i = 4h + r;   [36, 40): <g, x_j> for j = 4h + r
+    // split backward: <g, x_j> for j = 2p + h (p = chunk % 4) at [36 + p], the
+    // layout of the reductions buffer below
     float dots[BWD ? NDH : 1];
 #pragma unroll
     for (int e = 0; e < (BWD ? NDH : 1); ++e) dots[e] = 0.0f;
-    for (int cc = 0; cc < nch; ++cc) {
-      const int s = cc % NS;
-      if (!tc::mbar_wait(full(s), (uint32_t)(cc / NS) & 1u, abort_flag, wait_ns)) {
-        give_up();
-        break;
-      }
-      const uint8_t* st = smem + s * CFG::STAGE;
+    bool run = true;
+    for (int cc4 = 0; cc4 < nch && run; cc4 += N / SPC) {
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {  // the two 8-channel halves of the chunk
-        float gv[8];
-        if constexpr (STAGE_G) unpack8(ld32sw(st + CFG::GG_OFF, tok, c), gv);
+      for (int p = 0; p < N / SPC; ++p) {
+        const int cc = cc4 + p;
+        const int s = cc % NS;
+        if (!tc::mbar_wait(full(s), (uint32_t)(cc / NS) & 1u, abort_flag, wait_ns)) {
+          give_up();
+          run = false;
+          break;
+        }
+        const uint8_t* st = smem + s * CFG::STAGE;
+        const uint8_t* xt = st + CFG::X_OFF + h * XBOX;
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
+        for (int c = 0; c < CH / 8; ++c) {  // the 8-channel pieces of the chunk
           float xv[8];
-          unpack8(ld32sw(st + CFG::X_OFF + (4 * h + r) * XBOX, tok, c), xv);
+          unpack8(ld128sw(xt, tok, c), xv);
+          if constexpr (STAGE_G) {
+            float gv[8];
+            unpack8(ld128sw(st + CFG::GG_OFF, tok, c), gv);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            ss = fmaf(xv[e], xv[e], ss);
-            if constexpr (STAGE_G) dots[36 + r] = fmaf(gv[e], xv[e], dots[36 + r]);
-          }
-        }
-        if constexpr (FULLB) {
-          float fv[8];
-          unpack8(ld32sw(st + CFG::F_OFF, tok, c), fv);
-#pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            float Gv[8];
-            unpack8(ld32sw(st + CFG::G_OFF + (4 * h + r) * XBOX, tok, c), Gv);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) dots[32 + r] = fmaf(Gv[e], fv[e], dots[32 + r]);
-#pragma unroll
-            for (int j = 0; j < N; ++j) {
-              float xv[8];
-              unpack8(ld32sw(st + CFG::X_OFF + j * XBOX, tok, c), xv);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) dots[8 * r + j] = fmaf(Gv[e], xv[e], dots[8 * r + j]);
+            for (int e = 0; e < 8; ++e) {
+              ss = fmaf(xv[e], xv[e], ss);
+              dots[36 + p] = fmaf(gv[e], xv[e], dots[36 + p]);
             }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ss = fmaf(xv[e], xv[e], ss);
           }
         }
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(empty(s));
       }
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(empty(s));
     }
 
     bool ok = !*abort_flag && tc::mbar_wait(done_bar, 0, abort_flag, wait_ns);
@@ -354,26 +349,24 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
         }
       } else {
         sk_forward_ckpt<N>(H, iters, ck + tok, TM, ck_period);
-        // dL/dH_res: <G_i, x_j> from the two stream halves, or the post half's,
-        // or (DOTS) the tensor-core reductions' rows
+        // dL/dH_res: <G_i, x_j> from the post half's reductions (split) or the
+        // tensor-core reductions' rows (DOTS)
         constexpr int RSTRIDE = DOTS ? N * N + 2 * N : N * N + N;
         const float* rt = red_in + (live ? t : 0) * RSTRIDE;
         float dA[N * N];
 #pragma unroll
         for (int i = 0; i < N; ++i)
 #pragma unroll
-          for (int j = 0; j < N; ++j)
-            dA[i * N + j] = SPLIT || DOTS ? (live ? __ldg(rt + i * N + j) : 0.0f)
-                                          : red_dt[((i >> 2) * NDH + 8 * (i & 3) + j) * TM + tok];
+          for (int j = 0; j < N; ++j) dA[i * N + j] = live ? __ldg(rt + i * N + j) : 0.0f;
         float dzres[N * N];
         sk_adjoint_ckpt<N>(dA, dzres, iters, ck + tok, TM, ck_period);
         float dz[M];
 #pragma unroll
         for (int i = 0; i < N; ++i) {
+          // <g, x_i>: stream i was reduced by the warps of pair member i & 1
           const float dpre = DOTS ? (live ? __ldg(rt + N * N + N + i) : 0.0f)
-                                  : red_dt[((i >> 2) * NDH + 36 + (i & 3)) * TM + tok];
-          const float dpost = SPLIT || DOTS ? (live ? __ldg(rt + N * N + i) : 0.0f)
-                                            : red_dt[((i >> 2) * NDH + 32 + (i & 3)) * TM + tok];
+                                  : red_dt[((i & 1) * NDH + 36 + (i >> 1)) * TM + tok];
+          const float dpost = live ? __ldg(rt + N * N + i) : 0.0f;
           dz[i] = dpre * spre[i] * (1.0f - spre[i]);
           dz[N + i] = dpost * 2.0f * spost[i] * (1.0f - spost[i]);
         }
@@ -455,25 +448,26 @@ namespace {
 // rows m (0..79 the high parts, 80..159 the bf16 rounding of the remainder) of
 // 16 channels, 32 bytes per row, with the two 16-byte halves of rows whose bit
 // 2 is set swapped -- the 32-byte swizzle of a 256-byte-aligned tile, so one
-// bulk copy of a block (or of the 8 blocks of a chunk) lands in shared memory
-// ready for the MMA.  Channels c >= C of the last chunk are zero.
+// bulk copy of a block (or of consecutive streams' blocks) lands in shared
+// memory ready for the MMA.  The copy covers whole 64-channel groups (the
+// mapping's chunks); channels c >= C are zero.
 __global__ void k_phi_split8(int64_t C, int64_t ncp, const float* __restrict__ phi,
                              __nv_bfloat16* __restrict__ out) {
   using namespace tcm8;
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // j * ncp + c
   if (idx >= (int64_t)N * ncp) return;
   const int64_t j = idx / ncp, c = idx % ncp;
-  const int64_t q = c / CH;
-  const int ci = (int)(c % CH), h = ci >> 3, e = ci & 7;
-  __nv_bfloat16* blk = out + (q * N + j) * (NL * CH);
+  const int64_t q = c / PB;
+  const int ci = (int)(c % PB), h = ci >> 3, e = ci & 7;
+  __nv_bfloat16* blk = out + (q * N + j) * (NL * PB);
 #pragma unroll 4
   for (int m = 0; m < M; ++m) {
     const float v = c < C ? __ldg(phi + (j * C + c) * M + m) : 0.0f;
     const __nv_bfloat16 hi = __float2bfloat16_rn(v);
     const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
     const int m2 = M + m;
-    blk[m * CH + ((h ^ ((m >> 2) & 1)) << 3) + e] = hi;
-    blk[m2 * CH + ((h ^ ((m2 >> 2) & 1)) << 3) + e] = lo;
+    blk[m * PB + ((h ^ ((m >> 2) & 1)) << 3) + e] = hi;
+    blk[m2 * PB + ((h ^ ((m2 >> 2) & 1)) << 3) + e] = lo;
   }
 }
 
@@ -491,8 +485,8 @@ int map8_ck_period(int iters, size_t data_bytes) {
 }
 
 template <int MODE>
-cudaError_t launch_map8(const CUtensorMap& mx, const void* phi_t, const CUtensorMap& mG,
-                        const CUtensorMap& mg, const CUtensorMap& mf, int64_t T, int64_t C,
+cudaError_t launch_map8(const CUtensorMap& mx, const void* phi_t, const CUtensorMap& mg,
+                        int64_t T, int64_t C,
                         int iters, float eps, const float* b, const float* alpha, int ag,
                         float* Hpre, float* Hpost, float* Hres, float* coef, void* urec,
                         float* part, const float* red, int* st, int64_t wait_ns, cudaStream_t s) {
@@ -503,7 +497,7 @@ cudaError_t launch_map8(const CUtensorMap& mx, const void* phi_t, const CUtensor
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)((T + TM - 1) / TM);
   const int P = map8_ck_period(iters, Cfg<MODE>::DATA);
-  kern<<<grid, NT, Cfg<MODE>::SMEM, s>>>(mx, (const __nv_bfloat16*)phi_t, mG, mg, mf, T, C, iters, eps, P, b, alpha, ag,
+  kern<<<grid, NT, Cfg<MODE>::SMEM, s>>>(mx, (const __nv_bfloat16*)phi_t, mg, T, C, iters, eps, P, b, alpha, ag,
                                           Hpre, Hpost, Hres, coef, (__nv_bfloat16*)urec, part,
                                           red, st, tc::wait_limit(wait_ns));
   return cudaGetLastError();
@@ -511,8 +505,8 @@ cudaError_t launch_map8(const CUtensorMap& mx, const void* phi_t, const CUtensor
 }  // namespace
 
 size_t map8_tc_phi_bytes(int64_t C) {
-  const int64_t nch = (C + tcm8::CH - 1) / tcm8::CH;
-  return (size_t)nch * tcm8::N * tcm8::NL * tcm8::CH * 2;
+  const int64_t nblk = (C + tcm8::CH - 1) / tcm8::CH * (tcm8::CH / tcm8::PB);
+  return (size_t)nblk * tcm8::N * tcm8::NL * tcm8::PB * 2;
 }
 
 cudaError_t map8_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float eps, const void* x,
@@ -527,45 +521,31 @@ cudaError_t map8_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float ep
                                                                   (__nv_bfloat16*)phi_split);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  CUtensorMap mx, mG, mg, mf;
-  const CUtensorMapSwizzle SW = CU_TENSOR_MAP_SWIZZLE_32B;
+  CUtensorMap mx, mg;
+  const CUtensorMapSwizzle SW = CU_TENSOR_MAP_SWIZZLE_128B;
   const uint64_t dx[3] = {(uint64_t)C, (uint64_t)N, (uint64_t)T};
   const uint64_t sx[2] = {(uint64_t)C * 2, (uint64_t)N * C * 2};
   const uint32_t bx[3] = {CH, 1, TM};
   e = make_tmap_bf16(&mx, x, 3, dx, sx, bx, SW);
   if (e != cudaSuccess) return e;
-  // maps a mode does not read are copies of the x map (never dereferenced)
-  mG = mx;
-  mg = mx;
-  mf = mx;
-  const uint64_t d2[2] = {(uint64_t)C, (uint64_t)T};
-  const uint64_t s2[1] = {(uint64_t)C * 2};
-  const uint32_t b2[2] = {CH, TM};
-  if (mode == MAP_BWD || mode == MAP_BWD_SPLIT) {
+  mg = mx;  // read only by the split backward (otherwise a copy, never dereferenced)
+  if (mode == MAP_BWD_SPLIT) {
+    const uint64_t d2[2] = {(uint64_t)C, (uint64_t)T};
+    const uint64_t s2[1] = {(uint64_t)C * 2};
+    const uint32_t b2[2] = {CH, TM};
     e = make_tmap_bf16(&mg, g, 2, d2, s2, b2, SW);
-    if (e != cudaSuccess) return e;
-  }
-  if (mode == MAP_BWD) {
-    e = make_tmap_bf16(&mG, G, 3, dx, sx, bx, SW);
-    if (e != cudaSuccess) return e;
-    e = make_tmap_bf16(&mf, f, 2, d2, s2, b2, SW);
     if (e != cudaSuccess) return e;
   }
   switch (mode) {
     case MAP_FWD:
-      return launch_map8<MAP_FWD>(mx, phi_split, mG, mg, mf, T, C, iters, eps, b, alpha, ag, Hpre, Hpost,
+      return launch_map8<MAP_FWD>(mx, phi_split, mg, T, C, iters, eps, b, alpha, ag, Hpre, Hpost,
                                   Hres, nullptr, nullptr, nullptr, nullptr, st, wait_ns, s);
-    case MAP_BWD:
-      return launch_map8<MAP_BWD>(mx, phi_split, mG, mg, mf, T, C, iters, eps, b, alpha, ag, nullptr,
-                                  nullptr, nullptr, coef, urec, part, nullptr, st, wait_ns, s);
     case MAP_BWD_SPLIT:
-      return launch_map8<MAP_BWD_SPLIT>(mx, phi_split, mG, mg, mf, T, C, iters, eps, b, alpha, ag,
-                                        nullptr, nullptr, nullptr, coef, urec, part, red, st,
-                                        wait_ns, s);
+      return launch_map8<MAP_BWD_SPLIT>(mx, phi_split, mg, T, C, iters, eps, b, alpha, ag, nullptr,
+                                        nullptr, nullptr, coef, urec, part, red, st, wait_ns, s);
     case MAP_BWD_DOTS:
-      return launch_map8<MAP_BWD_DOTS>(mx, phi_split, mG, mg, mf, T, C, iters, eps, b, alpha, ag,
-                                       nullptr, nullptr, nullptr, coef, urec, part, red, st,
-                                       wait_ns, s);
+      return launch_map8<MAP_BWD_DOTS>(mx, phi_split, mg, T, C, iters, eps, b, alpha, ag, nullptr,
+                                       nullptr, nullptr, coef, urec, part, red, st, wait_ns, s);
     default:
       return cudaErrorInvalidValue;
   }
