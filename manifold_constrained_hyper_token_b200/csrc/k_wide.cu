@@ -442,9 +442,12 @@ __global__ void __launch_bounds__(128) k_wide_post(int64_t T, int64_t C, const T
                                                    TIO* __restrict__ xn) {
   using namespace widek;
   using V = Vec<TIO>;
-  constexpr int W = V::N;
-  __shared__ float hr[N * N], hp[N];
+  constexpr int W = V::N, P = W / 2;  // channels per vector, fp32 pairs per vector
+  __shared__ __align__(16) float hr[N * N];
+  __shared__ float hp[N];
   const int64_t nv = C / W;
+  // -0 as the addend makes fma(h, f, -0) the plain product h f, sign of zero included
+  const uint64_t nz = f2pack(-0.0f, -0.0f);
   for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
     __syncthreads();
     for (int e = threadIdx.x; e < N * N; e += blockDim.x) hr[e] = __ldg(Hres + t * N * N + e);
@@ -453,19 +456,45 @@ __global__ void __launch_bounds__(128) k_wide_post(int64_t T, int64_t C, const T
     const TIO* xt = x + t * N * C;
     TIO* ot = xn + t * N * C;
     for (int64_t v = threadIdx.x; v < nv; v += blockDim.x) {
-      float xv[N][W], fv[W];
+      // the vector's channels of every stream as fp32 pairs
+      uint64_t xv[N][P], fv[P];
+      {
+        float tmp[W];
 #pragma unroll
-      for (int j = 0; j < N; ++j) V::load_stream(xt + j * C + v * W, xv[j]);
-      V::load_stream(f + t * C + v * W, fv);
+        for (int j = 0; j < N; ++j) {
+          V::load_stream(xt + j * C + v * W, tmp);
+#pragma unroll
+          for (int p = 0; p < P; ++p) xv[j][p] = f2pack(tmp[2 * p], tmp[2 * p + 1]);
+        }
+        V::load_stream(f + t * C + v * W, tmp);
+#pragma unroll
+        for (int p = 0; p < P; ++p) fv[p] = f2pack(tmp[2 * p], tmp[2 * p + 1]);
+      }
+      // x_next[i] = H_post[i] f + sum_j H_res[i][j] x[j], the terms added in j order
 #pragma unroll 1
       for (int i = 0; i < N; ++i) {
+        uint64_t acc[P];
+        const uint64_t h0 = f2pack(hp[i], hp[i]);
+#pragma unroll
+        for (int p = 0; p < P; ++p) acc[p] = f2fma(h0, fv[p], nz);
+#pragma unroll
+        for (int j4 = 0; j4 < N / 4; ++j4) {
+          const float4 h = *reinterpret_cast<const float4*>(hr + i * N + 4 * j4);
+          const float hv[4] = {h.x, h.y, h.z, h.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t hh = f2pack(hv[k], hv[k]);
+#pragma unroll
+            for (int p = 0; p < P; ++p) acc[p] = f2fma(hh, xv[4 * j4 + k][p], acc[p]);
+          }
+        }
         float o[W];
 #pragma unroll
-        for (int e = 0; e < W; ++e) {
-          float acc = hp[i] * fv[e];
-#pragma unroll
-          for (int j = 0; j < N; ++j) acc = fmaf(hr[i * N + j], xv[j][e], acc);
-          o[e] = acc;
+        for (int p = 0; p < P; ++p) {
+          float a, b;
+          asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(acc[p]));
+          o[2 * p] = a;
+          o[2 * p + 1] = b;
         }
         V::store_stream(ot + i * C + v * W, o);
       }
