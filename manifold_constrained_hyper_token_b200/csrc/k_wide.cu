@@ -67,8 +67,104 @@ enum WideDots { WD_FULL = 0, WD_PRE = 1, WD_POST = 2 };
 
 // Sinkhorn checkpoints of the backward epilogue on the tensor-core path: every
 // second normalisation, iters + 1 iterates of N*N floats per token, laid out
-// per 32-token CTA as [iterate][element][token].
+// per token as [iterate][row][column].
 constexpr int kWideCkPeriod = 2;
+
+namespace widek {
+constexpr int EPI_NT = TB * N;     // the tensor-core path's epilogues: 16 lanes per token
+constexpr int TBS = N * N + N;     // floats per token of their transpose buffers (272)
+}  // namespace widek
+
+// ------------------------------------------------- 16 lanes per 16 x 16 matrix
+// Sinkhorn-Knopp and its adjoint for one token's 16 x 16 matrix spread over
+// 16 lanes of a warp: lane i of the half-warp holds row i in registers.  A row
+// pass is local to the lane; a column pass goes through the half-warp's
+// transpose buffer tb (256 floats; row r stored rotated by r, so that both the
+// row writes and the column reads hit 16 different banks) and the 16 floats
+// vb that follow it (a token's area is TBS = 272 floats).  Both
+// half-warps of a warp run the same steps (the __syncwarp calls are
+// warp-wide).  Every sum runs in a fixed order (a row's columns, a column's
+// rows, in index order).
+__device__ __forceinline__ void sk16_init(float (&a)[widek::N], int iters) {
+  constexpr int N = widek::N;
+  float mx = 0.0f;
+  if (iters > 0) {
+    mx = a[0];
+#pragma unroll
+    for (int j = 1; j < N; ++j) mx = fmaxf(mx, a[j]);
+  }
+#pragma unroll
+  for (int j = 0; j < N; ++j) a[j] = expf(a[j] - mx);
+}
+
+// Normalisation q (odd: rows, even: columns); returns the sum this lane's row
+// (odd q) or column i (even q) was divided by.
+__device__ __forceinline__ float sk16_step(float (&a)[widek::N], int q, int i, float* tb,
+                                           float* vb) {
+  constexpr int N = widek::N;
+  if (q & 1) {
+    float acc = 0.0f;
+#pragma unroll
+    for (int j = 0; j < N; ++j) acc += a[j];
+    const float inv = 1.0f / acc;
+#pragma unroll
+    for (int j = 0; j < N; ++j) a[j] *= inv;
+    return acc;
+  }
+#pragma unroll
+  for (int j = 0; j < N; ++j) tb[i * N + ((j + i) & (N - 1))] = a[j];
+  __syncwarp();
+  float acc = 0.0f;
+#pragma unroll
+  for (int r = 0; r < N; ++r) acc += tb[r * N + ((i + r) & (N - 1))];
+  vb[i] = 1.0f / acc;
+  __syncwarp();
+#pragma unroll
+  for (int j = 0; j < N; ++j) a[j] *= vb[j];
+  __syncwarp();  // tb and vb are rewritten by the next column pass
+  return acc;
+}
+
+// One step of the adjoint: a is the iterate after normalisation q, s the sum
+// this lane's row (odd q) or column i (even q) was divided by, g the gradient
+// with respect to that iterate (this lane's row), turned into the gradient
+// with respect to the iterate before the step:
+//   rows:    g_ij <- (g_ij - sum_k g_ik a_ik) / s_i
+//   columns: g_ij <- (g_ij - sum_k g_kj a_kj) / s_j
+__device__ __forceinline__ void sk16_adjoint_step(const float (&a)[widek::N], float s,
+                                                  float (&g)[widek::N], int q, int i, float* tb,
+                                                  float* vb) {
+  constexpr int N = widek::N;
+  if (q & 1) {
+    float d = 0.0f;
+#pragma unroll
+    for (int j = 0; j < N; ++j) d = fmaf(g[j], a[j], d);
+    const float inv = 1.0f / s;
+#pragma unroll
+    for (int j = 0; j < N; ++j) g[j] = (g[j] - d) * inv;
+    return;
+  }
+#pragma unroll
+  for (int j = 0; j < N; ++j) tb[i * N + ((j + i) & (N - 1))] = g[j] * a[j];
+  __syncwarp();
+  float d = 0.0f;
+#pragma unroll
+  for (int r = 0; r < N; ++r) d += tb[r * N + ((i + r) & (N - 1))];
+  __syncwarp();  // every column is read: tb's first row takes the reciprocals
+  vb[i] = d;
+  tb[i] = 1.0f / s;
+  __syncwarp();
+#pragma unroll
+  for (int j = 0; j < N; ++j) g[j] = (g[j] - vb[j]) * tb[j];
+  __syncwarp();
+}
+
+// sum over the 16 lanes of a half-warp, the same bits in every lane
+__device__ __forceinline__ float half_sum(float v) {
+#pragma unroll
+  for (int o = 8; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
 
 // The C-reductions of one CTA's TB tokens, as dacc[token 4*ty + i][dot tx + 32q]:
 //   dot d < 256         <G_i, x_j>   (i = d / 16, j = d % 16)        WD_FULL, WD_POST
@@ -380,18 +476,17 @@ __global__ void __launch_bounds__(widek::NT) k_wide_map(
   }
 }
 
-// The backward's per-token epilogue: one warp per TB tokens reads each token's
-// staged row (y, dot products, sum of squares) from coef, writes the
-// coefficient record over it, and adds the CTA's dz and dz . y rows in token
-// order into part [grid][DZ_SIZE].
+// The CUDA-core path's backward epilogue (no checkpoint scratch): one thread
+// per token reads the token's staged row (y, dot products, sum of squares)
+// from coef, writes the coefficient record over it, and adds the CTA's dz and
+// dz . y rows in token order into part [grid][DZ_SIZE].
 template <int MODE>
-__global__ void __launch_bounds__(32) k_wide_bwd_epi(int64_t T, int64_t C, int iters, float eps,
+__global__ void __launch_bounds__(32) k_wide_bwd_epi_thread(int64_t T, int64_t C, int iters, float eps,
                                                      const float* __restrict__ bias,
                                                      const float* __restrict__ alpha_p, int ag,
                                                      const float* __restrict__ red_in,
                                                      float* __restrict__ coef,
-                                                     float* __restrict__ part_o, int* status,
-                                                     float* __restrict__ ck) {
+                                                     float* __restrict__ part_o, int* status) {
   using namespace widek;
   using CF = Coef<N>;
   __shared__ float dzs[TB * (M + 3)];
@@ -399,10 +494,8 @@ __global__ void __launch_bounds__(32) k_wide_bwd_epi(int64_t T, int64_t C, int i
   const int64_t t = (int64_t)blockIdx.x * TB + tid;
   if (t < T) {
     const float* row = coef + t * CF::SIZE;
-    float* ckt = ck == nullptr ? nullptr
-                               : ck + (int64_t)blockIdx.x * ((int64_t)iters + 1) * N * N * TB + tid;
     wide_epilogue<MODE>(tid, t, T, (int64_t)N * C, iters, eps, row, row + M, row[2 * M], bias,
-                        alpha_p, ag, nullptr, nullptr, nullptr, red_in, coef, dzs, status, ckt);
+                        alpha_p, ag, nullptr, nullptr, nullptr, red_in, coef, dzs, status);
   } else {
     for (int m = 0; m < M + 3; ++m) dzs[tid * (M + 3) + m] = 0.0f;
   }
@@ -414,23 +507,195 @@ __global__ void __launch_bounds__(32) k_wide_bwd_epi(int64_t T, int64_t C, int i
   }
 }
 
-// The forward's per-token epilogue from rows written by the tensor-core
-// projection (y at [0, M), the sum of squares at [2M]): one thread per token.
-__global__ void __launch_bounds__(32) k_wide_fwd_epi(int64_t T, int64_t C, int iters, float eps,
-                                                     const float* __restrict__ bias,
-                                                     const float* __restrict__ alpha_p, int ag,
-                                                     const float* __restrict__ rows,
-                                                     float* __restrict__ Hpre_o,
-                                                     float* __restrict__ Hpost_o,
-                                                     float* __restrict__ Hres_o, int* status) {
+// The per-token epilogues of the tensor-core path, 16 lanes per token (lane i
+// of a half-warp: row i of H_res, pre and post logit i), TB tokens per CTA.
+// From the token's row (y at [0, M), the backward's dot products at [M, 2M),
+// the sum of squares at [2M]) they compute the gates and Sinkhorn (forward), or
+// the record of the apply and the token's dz (backward: the record is written
+// over the row once every lane has read it).
+template <int MODE>
+__global__ void __launch_bounds__(widek::EPI_NT) k_wide_bwd_epi(
+    int64_t T, int64_t C, int iters, float eps, const float* __restrict__ bias,
+    const float* __restrict__ alpha_p, int ag, const float* __restrict__ red_in,
+    float* __restrict__ coef, float* __restrict__ part_o, int* status, float* __restrict__ ck) {
   using namespace widek;
   using CF = Coef<N>;
-  const int tid = threadIdx.x;
-  const int64_t t = (int64_t)blockIdx.x * TB + tid;
-  if (t >= T) return;
-  const float* row = rows + t * CF::SIZE;
-  wide_epilogue<MAP_FWD>(tid, t, T, (int64_t)N * C, iters, eps, row, nullptr, row[2 * M], bias,
-                         alpha_p, ag, Hpre_o, Hpost_o, Hres_o, nullptr, nullptr, nullptr, status);
+  constexpr bool SPLIT = MODE == MAP_BWD_SPLIT;
+  // the transpose buffers during Sinkhorn, then the CTA's dz rows
+  static_assert(TB * TBS <= TB * (M + 3), "overlay");
+  __shared__ __align__(16) float sbuf[TB * (M + 3)];
+  float* tbs = sbuf;
+  float* dzs = sbuf;
+  const int lt = threadIdx.x >> 4, i = threadIdx.x & 15;  // token of the CTA, row
+  const int64_t t = (int64_t)blockIdx.x * TB + lt;
+  const bool live = t < T;
+  float* tb = tbs + lt * TBS;
+  float* vb = tb + N * N;
+  const float* row = coef + (live ? t : 0) * CF::SIZE;
+  const int64_t K = (int64_t)N * C;
+  // ---- the row's inputs (every lane reads before any lane writes the record)
+  const float r = sqrtf((live ? row[2 * M] : 1.0f) / (float)K + eps);
+  Alpha3 al;
+  al.load(alpha_p, ag);
+  float yres[N], a[N], g[N];
+  float ypre = 0.0f, ypost = 0.0f, zpre = 0.0f, zpost = 0.0f;
+  bool bad = !isfinite(r);
+  {
+    const float y0 = live ? row[i] / r : 0.0f, y1 = live ? row[N + i] / r : 0.0f;
+    ypre = y0;
+    ypost = y1;
+    zpre = fmaf(al.at<N>(i), y0, __ldg(bias + i));
+    zpost = fmaf(al.at<N>(N + i), y1, __ldg(bias + N + i));
+    bad |= !isfinite(zpre) || !isfinite(zpost);
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+      const int m = 2 * N + i * N + j;
+      yres[j] = live ? row[m] / r : 0.0f;
+      a[j] = fmaf(al.a[2], yres[j], __ldg(bias + m));
+      bad |= !isfinite(a[j]);
+    }
+  }
+  const float* rt = red_in + (SPLIT && live ? t * (N * N + N) : 0);
+#pragma unroll
+  for (int j = 0; j < N; ++j)
+    g[j] = !live ? 0.0f : (SPLIT ? __ldg(rt + i * N + j) : row[M + i * N + j]);
+  const float dpre_in = live ? row[M + N * N + i] : 0.0f;
+  const float dpost_in = !live ? 0.0f : (SPLIT ? __ldg(rt + N * N + i) : row[M + N * N + N + i]);
+  if (__any_sync(0xffffffffu, live && bad) && live && bad) flag_status(status, MHC_ERR_NONFINITE);
+  __syncwarp();
+  // ---- Sinkhorn with checkpoints, then its adjoint from them
+  float* ckt = ck + (live ? t : 0) * ((int64_t)iters + 1) * N * N + i * N;
+  auto ck_store = [&](int c, const float (&v)[N]) {
+    if (live) {
+      float4* d = reinterpret_cast<float4*>(ckt + (int64_t)c * N * N);
+#pragma unroll
+      for (int j4 = 0; j4 < N / 4; ++j4) d[j4] = make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
+    }
+  };
+  auto ck_load = [&](int c, float (&v)[N]) {
+    if (live) {
+      const float4* src = reinterpret_cast<const float4*>(ckt + (int64_t)c * N * N);
+#pragma unroll
+      for (int j4 = 0; j4 < N / 4; ++j4) {
+        const float4 q = src[j4];
+        v[4 * j4] = q.x;
+        v[4 * j4 + 1] = q.y;
+        v[4 * j4 + 2] = q.z;
+        v[4 * j4 + 3] = q.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < N; ++j) v[j] = 1.0f;
+    }
+  };
+  constexpr int P = kWideCkPeriod;
+  sk16_init(a, iters);
+  ck_store(0, a);
+  for (int q = 1; q <= 2 * iters; ++q) {
+    sk16_step(a, q, i, tb, vb);
+    if (q % P == 0) ck_store(q / P, a);
+  }
+  float H[N];  // this lane's row of H_res
+#pragma unroll
+  for (int j = 0; j < N; ++j) H[j] = a[j];
+  for (int step = 2 * iters; step >= 1; --step) {
+    const int c = (step - 1) / P;
+    ck_load(c, a);
+    for (int q = c * P + 1; q < step; ++q) sk16_step(a, q, i, tb, vb);
+    const float sq = sk16_step(a, step, i, tb, vb);
+    sk16_adjoint_step(a, sq, g, step, i, tb, vb);
+  }
+  ck_load(0, a);  // the exponentiated logits
+  float dzres[N];
+#pragma unroll
+  for (int j = 0; j < N; ++j) dzres[j] = g[j] * a[j];
+  // ---- gates, dz, the record
+  const float spre = sigmoidf_(zpre), spost = sigmoidf_(zpost);
+  const float dzpre = dpre_in * spre * (1.0f - spre);
+  const float dzpost = dpost_in * 2.0f * spost * (1.0f - spost);
+  float pres = 0.0f;
+#pragma unroll
+  for (int j = 0; j < N; ++j) pres = fmaf(dzres[j], yres[j], pres);
+  const float dzy0 = half_sum(dzpre * ypre), dzy1 = half_sum(dzpost * ypost);
+  const float dzy2 = half_sum(pres);
+  if (live) {
+    float* co = coef + t * CF::SIZE;
+    float4* hr = reinterpret_cast<float4*>(co + CF::RES + i * N);
+#pragma unroll
+    for (int j4 = 0; j4 < N / 4; ++j4) hr[j4] = make_float4(H[4 * j4], H[4 * j4 + 1], H[4 * j4 + 2], H[4 * j4 + 3]);
+    co[CF::PRE + i] = spre;
+    co[CF::POST + i] = 2.0f * spost;
+    const float ar0 = al.a[0] / r, ar1 = al.a[1] / r, ar2 = al.a[2] / r;
+    co[CF::U + i] = ar0 * dzpre;
+    co[CF::U + N + i] = ar1 * dzpost;
+    float4* ur = reinterpret_cast<float4*>(co + CF::U + 2 * N + i * N);
+#pragma unroll
+    for (int j4 = 0; j4 < N / 4; ++j4)
+      ur[j4] = make_float4(ar2 * dzres[4 * j4], ar2 * dzres[4 * j4 + 1], ar2 * dzres[4 * j4 + 2],
+                           ar2 * dzres[4 * j4 + 3]);
+    if (i == 0) {
+      const float wdzy = fmaf(al.a[2], dzy2, fmaf(al.a[1], dzy1, al.a[0] * dzy0));
+      co[CF::KAPPA] = wdzy / ((float)K * r * r);
+      for (int e = CF::KAPPA + 1; e < CF::SIZE; ++e) co[e] = 0.0f;
+    }
+  }
+  __syncthreads();  // every token's Sinkhorn is done with the transpose buffers
+  float* dz = dzs + lt * (M + 3);
+  dz[i] = live ? dzpre : 0.0f;
+  dz[N + i] = live ? dzpost : 0.0f;
+#pragma unroll
+  for (int j = 0; j < N; ++j) dz[2 * N + i * N + j] = live ? dzres[j] : 0.0f;
+  if (i == 0) {
+    dz[M] = live ? dzy0 : 0.0f;
+    dz[M + 1] = live ? dzy1 : 0.0f;
+    dz[M + 2] = live ? dzy2 : 0.0f;
+  }
+  __syncthreads();
+  // this CTA's sums of dz and dz . y, in token order
+  for (int col = threadIdx.x; col < M + 3; col += EPI_NT) {
+    float sum = 0.0f;
+    for (int q = 0; q < TB; ++q) sum += dzs[q * (M + 3) + col];
+    part_o[(int64_t)blockIdx.x * CF::DZ_SIZE + col] = sum;
+  }
+}
+
+__global__ void __launch_bounds__(widek::EPI_NT) k_wide_fwd_epi(
+    int64_t T, int64_t C, int iters, float eps, const float* __restrict__ bias,
+    const float* __restrict__ alpha_p, int ag, const float* __restrict__ rows,
+    float* __restrict__ Hpre_o, float* __restrict__ Hpost_o, float* __restrict__ Hres_o,
+    int* status) {
+  using namespace widek;
+  using CF = Coef<N>;
+  __shared__ __align__(16) float tbs[TB * TBS];
+  const int lt = threadIdx.x >> 4, i = threadIdx.x & 15;
+  const int64_t t = (int64_t)blockIdx.x * TB + lt;
+  const bool live = t < T;
+  float* tb = tbs + lt * TBS;
+  float* vb = tb + N * N;
+  const float* row = rows + (live ? t : 0) * CF::SIZE;
+  const float r = sqrtf((live ? row[2 * M] : 1.0f) / (float)(N * C) + eps);
+  Alpha3 al;
+  al.load(alpha_p, ag);
+  const float zpre = fmaf(al.at<N>(i), live ? row[i] / r : 0.0f, __ldg(bias + i));
+  const float zpost = fmaf(al.at<N>(N + i), live ? row[N + i] / r : 0.0f, __ldg(bias + N + i));
+  bool bad = !isfinite(r) || !isfinite(zpre) || !isfinite(zpost);
+  float a[N];
+#pragma unroll
+  for (int j = 0; j < N; ++j) {
+    const int m = 2 * N + i * N + j;
+    a[j] = fmaf(al.a[2], live ? row[m] / r : 0.0f, __ldg(bias + m));
+    bad |= !isfinite(a[j]);
+  }
+  if (__any_sync(0xffffffffu, live && bad) && live && bad) flag_status(status, MHC_ERR_NONFINITE);
+  sk16_init(a, iters);
+  for (int q = 1; q <= 2 * iters; ++q) sk16_step(a, q, i, tb, vb);
+  if (live) {
+    Hpre_o[t * N + i] = sigmoidf_(zpre);
+    Hpost_o[t * N + i] = 2.0f * sigmoidf_(zpost);
+    float4* hr = reinterpret_cast<float4*>(Hres_o + t * N * N + i * N);
+#pragma unroll
+    for (int j4 = 0; j4 < N / 4; ++j4) hr[j4] = make_float4(a[4 * j4], a[4 * j4 + 1], a[4 * j4 + 2], a[4 * j4 + 3]);
+  }
 }
 
 // x_next[i][c] = sum_j H_res[i][j] x[j][c] + H_post[i] f_out[c] (the k_post order)
@@ -779,8 +1044,8 @@ static cudaError_t launch_wide_map(int64_t T, int64_t C, int iters, float eps, c
   e = cudaGetLastError();
   if constexpr (MODE != MAP_FWD) {
     if (e != cudaSuccess) return e;
-    k_wide_bwd_epi<MODE><<<(unsigned)grid, 32, 0, s>>>(T, C, iters, eps, b, alpha, ag, red, coef,
-                                                       part, st, nullptr);
+    k_wide_bwd_epi_thread<MODE><<<(unsigned)grid, 32, 0, s>>>(T, C, iters, eps, b, alpha, ag, red,
+                                                              coef, part, st);
     e = cudaGetLastError();
   }
   return e;
@@ -804,8 +1069,8 @@ cudaError_t wide_map_tc_dispatch(int mode, int64_t T, int64_t C, int iters, floa
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)((T + widek::TB - 1) / widek::TB);
   if (mode == MAP_FWD) {
-    k_wide_fwd_epi<<<grid, 32, 0, s>>>(T, C, iters, eps, b, alpha, ag, rows, Hpre, Hpost, Hres,
-                                       st);
+    k_wide_fwd_epi<<<grid, widek::EPI_NT, 0, s>>>(T, C, iters, eps, b, alpha, ag, rows, Hpre,
+                                                  Hpost, Hres, st);
     return cudaGetLastError();
   }
   if (mode != MAP_BWD && mode != MAP_BWD_SPLIT) return cudaErrorInvalidValue;
@@ -813,11 +1078,11 @@ cudaError_t wide_map_tc_dispatch(int mode, int64_t T, int64_t C, int iters, floa
   e = dots16_dispatch(mode == MAP_BWD, T, C, x, G, g, f, rows, st, wait_ns, s);
   if (e != cudaSuccess) return e;
   if (mode == MAP_BWD)
-    k_wide_bwd_epi<MAP_BWD><<<grid, 32, 0, s>>>(T, C, iters, eps, b, alpha, ag, red, rows, part,
-                                                st, ck);
+    k_wide_bwd_epi<MAP_BWD><<<grid, widek::EPI_NT, 0, s>>>(T, C, iters, eps, b, alpha, ag, red,
+                                                           rows, part, st, ck);
   else
-    k_wide_bwd_epi<MAP_BWD_SPLIT><<<grid, 32, 0, s>>>(T, C, iters, eps, b, alpha, ag, red, rows,
-                                                      part, st, ck);
+    k_wide_bwd_epi<MAP_BWD_SPLIT><<<grid, widek::EPI_NT, 0, s>>>(T, C, iters, eps, b, alpha, ag,
+                                                                 red, rows, part, st, ck);
   return cudaGetLastError();
 }
 
