@@ -15,10 +15,11 @@
 //                     288 C-reductions per token and stages y, the dot
 //                     products and the sum of squares in each token's
 //                     coefficient row
-//   k_wide_bwd_epi    the backward's per-token epilogue, one warp per 32
-//                     tokens: gates, Sinkhorn and its adjoint, the
-//                     coefficient record written over the staged row, and
-//                     the tile's grad_b / grad_alpha partial sums
+//   k_wide_bwd_epi_thread  the backward's per-token epilogue, one thread per
+//                     token in a one-warp CTA of 32 tokens: gates, Sinkhorn
+//                     and its adjoint, the coefficient record written over the
+//                     staged row, and the tile's grad_b / grad_alpha partial
+//                     sums
 //   k_wide_post       x_next = H_res x + H_post^T f_out, coefficients in
 //                     shared memory
 //   k_wide_post_bwd   the post half of the backward in training order:
@@ -32,11 +33,14 @@
 // With bf16 activations the projection, the backward's C-reductions and the
 // apply run on the tensor cores instead (k_proj16_tc.cu writes y and the sum of
 // squares into the rows, k_dots_tc.cu the C-reductions; here k_wide_fwd_epi
-// and k_wide_bwd_epi run the epilogues from those rows; k_apply16_tc.cu is the
-// apply, with k_wide_bias for its grad_b and grad_alpha).
+// and k_wide_bwd_epi run the epilogues from those rows with 16 lanes per
+// token, one row of the 16 x 16 Sinkhorn matrix per lane, the adjoint from
+// every second iterate kept in a global scratch; k_apply16_tc.cu is the apply,
+// with k_wide_bias for its grad_b and grad_alpha).
 //
 // Every sum is taken in a fixed order, so repeated calls give identical bits.
-// The per-token Sinkhorn arrays (16 x 16) live in local memory.
+// On the fp32 path the per-token Sinkhorn arrays (16 x 16) live in local
+// memory, one token per thread.
 #include "mhc_common.cuh"
 #include "mhc_dispatch.h"
 
