@@ -23,7 +23,9 @@
 //             piece), so phi u never leaves the chip;
 //   k_gphi8   grad_phi for 128 rows of phi: D[128 x 192] += X^T[128 x 128] .
 //             U[128 x 192] over every token tile (tcgen05), then
-//             grad_phi = D[:, m] + D[:, 96 + m];
+//             grad_phi = D[:, m] + D[:, 96 + m]; the (block, tile) units are
+//             split evenly over persistent CTAs, and k_gphi8_fin adds the
+//             parts of blocks that two or more CTAs share;
 //   k_bias8   grad_b and grad_alpha from the mapping's per-tile partial sums.
 //
 // U is [u_hi (80) | 0 (16) | u_lo (80) | 0 (16)]: phi u = (u_hi + u_lo) . phi_hi
@@ -78,9 +80,10 @@ constexpr int C_U_OFF = 2 * ATOM;       // U tile: three atoms
 constexpr int C_STAGE = 5 * ATOM;       // 80 KB
 constexpr int C_NS = 2;
 constexpr int C_DATA = C_NS * C_STAGE;
-constexpr int C_SMEM = C_DATA + 1024 + 64;
-constexpr int C_NT = 128;
-constexpr uint32_t C_TMEM = 256;
+constexpr int C_SMEM = C_DATA + 1024 + 128;
+constexpr int C_NT = 6 * 32;            // TMA, MMA, four epilogue warps
+constexpr uint32_t C_TMEM = 512;        // two accumulators of NU columns
+constexpr int C_MAXGRID = 256;          // partial-sum slots are sized for this many CTAs
 // k_bias8
 constexpr int B_NT = 128;
 static_assert(F_SMEM <= 232448 && C_SMEM <= 232448, "shared memory");
@@ -463,33 +466,50 @@ __global__ void __launch_bounds__(ap8::B_NT) k_bias8(const float* __restrict__ p
 }
 
 // --------------------------------------------------------------- grad_phi
-__global__ void __launch_bounds__(ap8::C_NT) k_gphi8(const __grid_constant__ CUtensorMap tm_x,
-                                                     const __grid_constant__ CUtensorMap tm_u,
-                                                     int64_t T, int64_t C, int ncb,
-                                                     float* __restrict__ grad_phi, int* status,
-                                                     uint64_t wait_ns) {
+// The (128-channel block of one stream, 128-token tile) units, block-major,
+// are split evenly over the CTAs (a contiguous range each), so that every SM
+// has the same number of tiles.  A CTA's range cuts into segments, one per
+// block it touches; a segment accumulates D[128 x 192] += X^T U over its tiles
+// (two TMEM accumulators, alternating, so one segment's epilogue overlaps the
+// next segment's MMAs).  A segment that covers its whole block writes grad_phi;
+// the first and last segments of a range can be parts of a block, and write
+// the CTA's partial slots 0 and 1 instead, which k_gphi8_fin adds in CTA
+// order.  The owner of unit u is the CTA b with lo_b <= u < lo_{b+1},
+// lo_b = floor(b * units / grid).
+__global__ void __launch_bounds__(ap8::C_NT, 1) k_gphi8(const __grid_constant__ CUtensorMap tm_x,
+                                                        const __grid_constant__ CUtensorMap tm_u,
+                                                        int64_t T, int64_t C, int ncb,
+                                                        int64_t nunits,
+                                                        float* __restrict__ grad_phi,
+                                                        float* __restrict__ partial, int* status,
+                                                        uint64_t wait_ns) {
   using namespace ap8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C_DATA);  // full[2] empty[2] done fin
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C_NS + 2);
+  // full[2] empty[2] dfull[2] dempty[2] fin
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C_DATA);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C_NS + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   auto full = [&](int s) { return tc::smem_u32(bars + s); };
   auto empty = [&](int s) { return tc::smem_u32(bars + C_NS + s); };
-  const uint32_t done_bar = tc::smem_u32(bars + 2 * C_NS);
-  const uint32_t fin_bar = tc::smem_u32(bars + 2 * C_NS + 1);
+  auto dfull = [&](int d) { return tc::smem_u32(bars + 2 * C_NS + d); };
+  auto dempty = [&](int d) { return tc::smem_u32(bars + 2 * C_NS + 2 + d); };
+  const uint32_t fin_bar = tc::smem_u32(bars + 2 * C_NS + 4);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int j = blockIdx.x / ncb, cb = blockIdx.x % ncb;
-  const int c0 = cb * CB;
-  const int ntt = (int)((T + TT - 1) / TT);
+  const int64_t ntt = (T + TT - 1) / TT;
+  const int64_t lo = (int64_t)blockIdx.x * nunits / gridDim.x;
+  const int64_t hi = ((int64_t)blockIdx.x + 1) * nunits / gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C_NS; ++s) {
       tc::mbar_init(full(s), 1);
       tc::mbar_init(empty(s), 1);
     }
-    tc::mbar_init(done_bar, 1);
+    for (int d = 0; d < 2; ++d) {
+      tc::mbar_init(dfull(d), 1);
+      tc::mbar_init(dempty(d), 4);  // the four epilogue warps
+    }
     tc::mbar_init(fin_bar, 1);
     *abort_flag = 0;
     tc::mbar_fence_init();
@@ -507,81 +527,118 @@ __global__ void __launch_bounds__(ap8::C_NT) k_gphi8(const __grid_constant__ CUt
     flag_status(status, MHC_ERR_TIMEOUT);
   };
 
-  if (warp == 0 && lane == 0) {
+  if (warp == 0) {
     // ---------------------------------------------------------------- TMA
-    const uint64_t pol_x = tc::policy_evict_first(), pol_u = tc::policy_evict_last();
-    int issued = 0;
-    for (int it = 0; it < ntt; ++it) {
-      const int s = it % C_NS;
-      if (it >= C_NS && !tc::mbar_wait(empty(s), ((uint32_t)(it / C_NS) & 1u) ^ 1u, abort_flag,
-                                       wait_ns)) {
-        give_up();
-        break;
+    if (lane == 0) {
+      const uint64_t pol_x = tc::policy_evict_first(), pol_u = tc::policy_evict_last();
+      int64_t k = 0;
+      for (int64_t u = lo; u < hi; ++u, ++k) {
+        const int s = (int)(k % C_NS);
+        if (k >= C_NS && !tc::mbar_wait(empty(s), ((uint32_t)(k / C_NS) & 1u) ^ 1u, abort_flag,
+                                        wait_ns)) {
+          give_up();
+          break;
+        }
+        const int64_t blk = u / ntt, tile = u % ntt;
+        const int j = (int)(blk / ncb), c0 = (int)(blk % ncb) * CB;
+        const uint32_t base = tc::smem_u32(smem + s * C_STAGE);
+        tc::mbar_arrive_expect_tx(full(s), (uint32_t)C_STAGE);
+        for (int a = 0; a < 2; ++a)
+          tc::tma_load_3d(base + C_X_OFF + a * ATOM, &tm_x, full(s), c0 + 64 * a, j,
+                          (int)(tile * TT), pol_x);
+        for (int a = 0; a < 3; ++a)
+          tc::tma_load_2d(base + C_U_OFF + a * ATOM, &tm_u, full(s), 64 * a, (int)(tile * TT),
+                          pol_u);
       }
-      const uint32_t base = tc::smem_u32(smem + s * C_STAGE);
-      tc::mbar_arrive_expect_tx(full(s), (uint32_t)C_STAGE);
-      for (int a = 0; a < 2; ++a)
-        tc::tma_load_3d(base + C_X_OFF + a * ATOM, &tm_x, full(s), c0 + 64 * a, j, it * TT, pol_x);
-      for (int a = 0; a < 3; ++a)
-        tc::tma_load_2d(base + C_U_OFF + a * ATOM, &tm_u, full(s), 64 * a, it * TT, pol_u);
-      ++issued;
+      // every copy issued here has landed before the CTA can exit
+      for (int64_t q = (k > C_NS ? k - C_NS : 0); q < k; ++q)
+        tc::mbar_wait(full((int)(q % C_NS)), (uint32_t)(q / C_NS) & 1u, nullptr, tc::kDrainWaitNs);
     }
-    for (int it = (issued > C_NS ? issued - C_NS : 0); it < issued; ++it)
-      tc::mbar_wait(full(it % C_NS), (uint32_t)(it / C_NS) & 1u, nullptr, tc::kDrainWaitNs);
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
     // D[k][m'] += sum over 16 tokens of X[tok][k] U[tok][m']: A = X^T (MN-major,
     // two 64-channel atoms), B = U (MN-major, three 64-column atoms)
-    constexpr uint32_t idesc = tc::idesc_bf16(CB, NU, true, true);
-    bool any = false;
-    for (int it = 0; it < ntt; ++it) {
-      const int s = it % C_NS;
-      if (!tc::mbar_wait(full(s), (uint32_t)(it / C_NS) & 1u, abort_flag, wait_ns)) {
-        give_up();
-        break;
+    if (lane == 0) {
+      constexpr uint32_t idesc = tc::idesc_bf16(CB, NU, true, true);
+      bool any = false;
+      int seg = 0;
+      int64_t k = 0;
+      for (int64_t u = lo; u < hi; ++u, ++k) {
+        const int s = (int)(k % C_NS);
+        const int64_t tile = u % ntt;
+        const bool first = u == lo || tile == 0, last = u == hi - 1 || tile == ntt - 1;
+        const int d = seg & 1;
+        if (first && seg >= 2 &&
+            !tc::mbar_wait(dempty(d), ((uint32_t)(seg >> 1) & 1u) ^ 1u, abort_flag, wait_ns)) {
+          give_up();
+          break;
+        }
+        if (!tc::mbar_wait(full(s), (uint32_t)(k / C_NS) & 1u, abort_flag, wait_ns)) {
+          give_up();
+          break;
+        }
+        tc::tc_fence_after();
+        const uint32_t base = tc::smem_u32(smem + s * C_STAGE);
+#pragma unroll
+        for (int kk = 0; kk < TT / 16; ++kk) {
+          const uint64_t da = tc::smem_desc(base + C_X_OFF + kk * 2048, ATOM, 1024, tc::SWZ_128B);
+          const uint64_t db = tc::smem_desc(base + C_U_OFF + kk * 2048, ATOM, 1024, tc::SWZ_128B);
+          tc::mma_bf16(tmem + (uint32_t)(d * NU), da, db, idesc, (first && kk == 0) ? 0u : 1u);
+        }
+        any = true;
+        tc::mma_commit(empty(s));
+        if (last) {
+          tc::mma_commit(dfull(d));
+          ++seg;
+        }
       }
+      // every MMA issued here has finished before TMEM is freed
+      if (any) {
+        tc::mma_commit(fin_bar);
+        tc::mbar_wait(fin_bar, 0, nullptr, tc::kDrainWaitNs);
+      }
+    }
+  } else {
+    // ----------------------------------------------------------- epilogue
+    // warp w holds phi rows (channels) 32 (w % 4).. of the segment's block
+    const int q = warp & 3;
+    const int64_t b0 = lo / ntt, b1 = hi > lo ? (hi - 1) / ntt : b0 - 1;
+    bool ok = true;
+    for (int64_t blk = b0; blk <= b1 && ok; ++blk) {
+      const int si = (int)(blk - b0), d = si & 1;
+      bool okw = tc::mbar_wait(dfull(d), (uint32_t)(si >> 1) & 1u, abort_flag, wait_ns);
+      if (!okw && !*abort_flag) give_up();
+      ok = __all_sync(0xffffffffu, okw);
+      if (!ok) break;
       tc::tc_fence_after();
-      const uint32_t base = tc::smem_u32(smem + s * C_STAGE);
-#pragma unroll
-      for (int k = 0; k < TT / 16; ++k) {
-        const uint64_t da = tc::smem_desc(base + C_X_OFF + k * 2048, ATOM, 1024, tc::SWZ_128B);
-        const uint64_t db = tc::smem_desc(base + C_U_OFF + k * 2048, ATOM, 1024, tc::SWZ_128B);
-        tc::mma_bf16(tmem, da, db, idesc, (it | k) != 0 ? 1u : 0u);
-      }
-      any = true;
-      tc::mma_commit(empty(s));
-    }
-    if (!*abort_flag) tc::mma_commit(done_bar);
-    if (any) {
-      tc::mma_commit(fin_bar);
-      tc::mbar_wait(fin_bar, 0, nullptr, tc::kDrainWaitNs);
-    }
-  }
-  // ---- epilogue: warp w holds phi rows (channels) 32w..32w+31 of this block
-  bool ok = !*abort_flag && tc::mbar_wait(done_bar, 0, abort_flag, wait_ns);
-  if (!ok && !*abort_flag) give_up();
-  ok = __all_sync(0xffffffffu, ok);
-  if (ok) {
-    tc::tc_fence_after();
-    const int64_t c = (int64_t)c0 + 32 * warp + lane;
-    float* dst = grad_phi + ((int64_t)j * C + c) * M;
-    const uint32_t lb = tmem + ((uint32_t)(32 * warp) << 16);
+      const int64_t s_lo = blk * ntt > lo ? blk * ntt : lo;
+      const int64_t s_hi = (blk + 1) * ntt < hi ? (blk + 1) * ntt : hi;
+      const bool whole = s_lo == blk * ntt && s_hi == (blk + 1) * ntt;
+      const int j = (int)(blk / ncb);
+      const int64_t c = (blk % ncb) * CB + 32 * q + lane;
+      float* dst = whole ? grad_phi + ((int64_t)j * C + c) * M
+                         : partial + (((int64_t)blockIdx.x * 2 + (si == 0 ? 0 : 1)) * CB +
+                                      32 * q + lane) * M;
+      const uint32_t lb = tmem + (uint32_t)(d * NU) + ((uint32_t)(32 * q) << 16);
 #pragma unroll 1
-    for (int q = 0; q < M / 16; ++q) {
-      float hi[16], lo[16];
-      tc::tmem_ld16(lb + 16 * q, hi);
-      tc::tmem_ld16(lb + TcRec8::LO + 16 * q, lo);
-      tc::tmem_ld_wait();
-      if (c < C) {
+      for (int qq = 0; qq < M / 16; ++qq) {
+        float hv[16], lv[16];
+        tc::tmem_ld16(lb + 16 * qq, hv);
+        tc::tmem_ld16(lb + TcRec8::LO + 16 * qq, lv);
+        tc::tmem_ld_wait();
+        if (c < C) {
 #pragma unroll
-        for (int e = 0; e < 16; e += 4)
-          *reinterpret_cast<float4*>(dst + 16 * q + e) =
-              make_float4(hi[e] + lo[e], hi[e + 1] + lo[e + 1], hi[e + 2] + lo[e + 2],
-                          hi[e + 3] + lo[e + 3]);
+          for (int e = 0; e < 16; e += 4)
+            *reinterpret_cast<float4*>(dst + 16 * qq + e) =
+                make_float4(hv[e] + lv[e], hv[e + 1] + lv[e + 1], hv[e + 2] + lv[e + 2],
+                            hv[e + 3] + lv[e + 3]);
+        }
       }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(dempty(d));
     }
   }
-  __syncwarp();
   tc::tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -590,12 +647,50 @@ __global__ void __launch_bounds__(ap8::C_NT) k_gphi8(const __grid_constant__ CUt
   }
 }
 
+// grad_phi rows of the blocks that several CTAs share: the CTAs' partial
+// slots added in CTA order.  One thread per (block, row).
+__global__ void k_gphi8_fin(int64_t C, int ncb, int64_t ntt, int64_t nunits, int grid,
+                            const float* __restrict__ partial, float* __restrict__ grad_phi) {
+  using namespace ap8;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // blk * CB + row
+  const int64_t blk = idx / CB;
+  const int row = (int)(idx % CB);
+  if (blk >= nunits / ntt) return;
+  auto owner = [&](int64_t u) { return ((u + 1) * grid - 1) / nunits; };
+  const int64_t bfirst = owner(blk * ntt), blast = owner((blk + 1) * ntt - 1);
+  if (bfirst == blast) return;  // one CTA covered the block and wrote it
+  const int64_t c = (blk % ncb) * CB + row;
+  if (c >= C) return;
+  float acc[M];
+#pragma unroll
+  for (int m = 0; m < M; ++m) acc[m] = 0.0f;
+  for (int64_t b = bfirst; b <= blast; ++b) {
+    const int64_t lo_b = b * nunits / grid;
+    const int slot = lo_b / ntt == blk ? 0 : 1;
+    const float* p = partial + ((b * 2 + slot) * CB + row) * M;
+#pragma unroll
+    for (int m = 0; m < M; m += 4) {
+      const float4 v = *reinterpret_cast<const float4*>(p + m);
+      acc[m] += v.x;
+      acc[m + 1] += v.y;
+      acc[m + 2] += v.z;
+      acc[m + 3] += v.w;
+    }
+  }
+  float* dst = grad_phi + ((blk / ncb) * C + c) * M;
+#pragma unroll
+  for (int m = 0; m < M; m += 4)
+    *reinterpret_cast<float4*>(dst + m) = make_float4(acc[m], acc[m + 1], acc[m + 2], acc[m + 3]);
+}
+
 // ------------------------------------------------------------------ host
+size_t apply8_tc_scratch_bytes() { return (size_t)ap8::C_MAXGRID * 2 * ap8::CB * ap8::M * 4; }
+
 cudaError_t apply8_tc_dispatch(int64_t T, int64_t C, const void* x, const void* phi_split,
                                const void* G, const void* g, const float* coef, const void* urec,
                                const float* part, int nparts, void* gx, void* gf, float* gphi,
-                               float* gb, float* ga, int ag, int* st, int64_t wait_ns,
-                               cudaStream_t s) {
+                               float* gb, float* ga, int ag, float* gpart, int* st,
+                               int64_t wait_ns, cudaStream_t s) {
   using namespace ap8;
   const uint64_t wl = tc::wait_limit(wait_ns);
   CUtensorMap mu, mx;
@@ -634,9 +729,18 @@ cudaError_t apply8_tc_dispatch(int64_t T, int64_t C, const void* x, const void* 
   if (e != cudaSuccess) return e;
 
   const int ncb_c = (int)((C + CB - 1) / CB);
+  const int64_t nunits_c = (int64_t)N * ncb_c * ntt;
+  int grid_c = (int)(nunits_c < nsm ? nunits_c : nsm);
+  if (grid_c > C_MAXGRID) grid_c = C_MAXGRID;
   e = cudaFuncSetAttribute(k_gphi8, cudaFuncAttributeMaxDynamicSharedMemorySize, C_SMEM);
   if (e != cudaSuccess) return e;
-  k_gphi8<<<(unsigned)(N * ncb_c), C_NT, C_SMEM, s>>>(mx, mu, T, C, ncb_c, gphi, st, wl);
+  k_gphi8<<<(unsigned)grid_c, C_NT, C_SMEM, s>>>(mx, mu, T, C, ncb_c, nunits_c, gphi, gpart, st,
+                                                 wl);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t nrows = (int64_t)N * ncb_c * CB;
+  k_gphi8_fin<<<(unsigned)((nrows + 127) / 128), 128, 0, s>>>(C, ncb_c, ntt, nunits_c, grid_c,
+                                                               gpart, gphi);
   return cudaGetLastError();
 }
 

@@ -76,7 +76,8 @@ size_t rows16_bytes(int64_t T) { return (size_t)T * mhc::Coef<16>::SIZE * 4; }
 // 128-token CTA, the bf16 split copy of phi^T that the mapping MMA reads, and
 // the apply kernel's grad_phi partials and slice counters.  Tensor-core path
 // (n = 8): the coefficient records, the U rows, the C-reductions of the
-// backward mapping, the partial sums and the phi split copy.
+// backward mapping, the partial sums, the phi split copy and the grad_phi
+// parts of the blocks that the apply's CTAs share.
 struct BwdWorkspace {
   size_t coef_off, urec_off, hrec_off, part_off, phi_off, apply_off, kmap_off, red_off, total;
   int nparts;
@@ -122,6 +123,7 @@ BwdWorkspace bwd_layout(const mhc_params* p) {
   // Sinkhorn checkpoints
   size_t apply_bytes = 0;
   if (tc) apply_bytes = mhc::apply_tc_scratch_bytes(p->T, p->C);
+  if (tc8) apply_bytes = mhc::apply8_tc_scratch_bytes();
   if (use_tc16(p))
     apply_bytes = std::max((size_t)p->T * 16 * p->C * 4, mhc::wide_ck_bytes(p->T, p->t_max));
   off = round_up(off + apply_bytes, 256);
@@ -306,8 +308,8 @@ mhc_status mhc_backward_apply(const mhc_params* p, const void* x, const float* p
     return from_cuda(mhc::apply8_tc_dispatch(
         p->T, p->C, x, ws + w.phi_off, grad_x_next, grad_h_in, (const float*)(ws + w.coef_off),
         ws + w.urec_off, (const float*)(ws + w.part_off), w.nparts, grad_x, grad_f_out,
-        grad_phi, grad_b, grad_alpha, alpha_groups(p), dev_status, p->wait_ns,
-        (cudaStream_t)stream));
+        grad_phi, grad_b, grad_alpha, alpha_groups(p), (float*)(ws + w.apply_off), dev_status,
+        p->wait_ns, (cudaStream_t)stream));
   if (use_tc16(p))
     return from_cuda(mhc::apply16_tc_dispatch(
         p->T, p->C, x, ws + w.phi_off, grad_x_next, grad_h_in, (const float*)(ws + w.coef_off),
@@ -466,7 +468,8 @@ mhc_status mhc_pre_backward(const mhc_params* p, const void* x, const float* phi
     return from_cuda(mhc::apply8_tc_dispatch(
         p->T, p->C, x, ws + w.phi_off, grad_x_next, grad_h_in, (const float*)(ws + w.coef_off),
         ws + w.urec_off, (const float*)(ws + w.part_off), w.nparts, grad_x, nullptr, grad_phi,
-        grad_b, grad_alpha, alpha_groups(p), dev_status, p->wait_ns, s));
+        grad_b, grad_alpha, alpha_groups(p), (float*)(ws + w.apply_off), dev_status, p->wait_ns,
+        s));
   }
   if (use_tc16(p)) {
     st = from_cuda(mhc::wide_map_tc_dispatch(

@@ -73,12 +73,15 @@ cudaError_t map8_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float ep
 // k_apply8_tc.cu (bf16, n = 8): grad_x / grad_f_out with phi u on the tensor
 // cores (the accumulators stay on chip), grad_phi as a tensor-core contraction
 // over the tokens, and grad_b / grad_alpha from the partial sums; phi_split is
-// the mapping's bf16 split copy of phi^T.  gf == nullptr skips grad_f_out.
+// the mapping's bf16 split copy of phi^T; gpart is scratch of
+// apply8_tc_scratch_bytes() bytes (grad_phi parts of blocks that CTAs share).
+// gf == nullptr skips grad_f_out.
 cudaError_t apply8_tc_dispatch(int64_t T, int64_t C, const void* x, const void* phi_split,
                                const void* G, const void* g, const float* coef, const void* urec,
                                const float* part, int nparts, void* gx, void* gf, float* gphi,
-                               float* gb, float* ga, int ag, int* st, int64_t wait_ns,
-                               cudaStream_t s);
+                               float* gb, float* ga, int ag, float* gpart, int* st,
+                               int64_t wait_ns, cudaStream_t s);
+size_t apply8_tc_scratch_bytes();
 size_t map8_tc_phi_bytes(int64_t C);
 
 // k_proj16_tc.cu (bf16, n = 16): splits phi into the tiled bf16 copy phi_t
