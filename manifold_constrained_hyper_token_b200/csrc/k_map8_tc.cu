@@ -65,10 +65,11 @@ template <int MODE> struct Cfg {
   static constexpr int GG_OFF = P_OFF + SPC * (CH / PB) * PBOX;  // grad_h_in (split backward)
   static constexpr int STAGE = STAGE_G ? GG_OFF + XBOX : GG_OFF;
   static constexpr int NS = STAGE_G ? 2 : 3;
-  // the stages, reused after the chunk loop by the epilogue; the backward
-  // epilogue keeps Sinkhorn checkpoints there, so the backward asks for at
-  // least 224 KB
-  static constexpr int DATA = BWD && NS * STAGE < 229376 ? 229376 : NS * STAGE;
+  // the stages, reused after the chunk loop by the epilogue's reductions, dz
+  // rows and per-token logits
+  static constexpr int DATA = NS * STAGE;
+  static_assert((2 * TM + 2 * NDH * TM + (M + 3) * TM + TM * (2 * M + 4)) * 4 <= DATA,
+                "epilogue scratch");
   static_assert(STAGE % 1024 == 0 && GG_OFF % 1024 == 0, "128-byte swizzle atoms");
   static constexpr int SMEM = DATA + 1024 /*align*/ + 256 /*barriers, flags*/;
   static_assert(SMEM <= 232448, "shared memory");
@@ -96,13 +97,76 @@ __device__ __forceinline__ void nbar8(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// ---------------------------------------------- 8 lanes per 8 x 8 matrix
+// Sinkhorn-Knopp and its adjoint for one token's 8 x 8 matrix on an aligned
+// group of 8 lanes, lane i holding row i.  Column sums are butterflies over
+// the group (xor 4, 2, 1), so every lane of the group gets every column's sum,
+// with the same bits.  The four groups of a warp run the same steps.
+__device__ __forceinline__ float sum8(float v) {
+  v += __shfl_xor_sync(0xffffffffu, v, 4);
+  v += __shfl_xor_sync(0xffffffffu, v, 2);
+  v += __shfl_xor_sync(0xffffffffu, v, 1);
+  return v;
+}
+
+__device__ __forceinline__ void sk8_init(float (&a)[8], int iters) {
+  float mx = 0.0f;
+  if (iters > 0) {
+    mx = a[0];
+#pragma unroll
+    for (int j = 1; j < 8; ++j) mx = fmaxf(mx, a[j]);
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) a[j] = expf(a[j] - mx);
+}
+
+// Normalisation q (odd: rows, even: columns); s receives the sums divided out
+// (odd q: s[0] = this lane's row sum; even q: s[j] = column j's sum).
+__device__ __forceinline__ void sk8_step(float (&a)[8], int q, float (&s)[8]) {
+  if (q & 1) {
+    float acc = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc += a[j];
+    const float inv = 1.0f / acc;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) a[j] *= inv;
+    s[0] = acc;
+    return;
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) s[j] = sum8(a[j]);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) a[j] *= 1.0f / s[j];
+}
+
+// One adjoint step: a is the iterate after normalisation q, s its sums, g the
+// gradient with respect to it (this lane's row), turned into the gradient with
+// respect to the iterate before the step.
+__device__ __forceinline__ void sk8_adjoint_step(const float (&a)[8], const float (&s)[8],
+                                                 float (&g)[8], int q) {
+  if (q & 1) {
+    float d = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) d = fmaf(g[j], a[j], d);
+    const float inv = 1.0f / s[0];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) g[j] = (g[j] - d) * inv;
+    return;
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float d = sum8(g[j] * a[j]);
+    g[j] = (g[j] - d) * (1.0f / s[j]);
+  }
+}
+
 }  // namespace
 
 template <int MODE>
 __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
     const __grid_constant__ CUtensorMap tm_x, const __nv_bfloat16* __restrict__ phi_t,
     const __grid_constant__ CUtensorMap tm_g, int64_t T, int64_t C, int iters, float eps,
-    int ck_period, const float* __restrict__ bias, const float* __restrict__ alpha_p, int ag,
+    float* __restrict__ ck, const float* __restrict__ bias, const float* __restrict__ alpha_p, int ag,
     float* __restrict__ Hpre_o, float* __restrict__ Hpost_o, float* __restrict__ Hres_o,
     float* __restrict__ coef_o, __nv_bfloat16* __restrict__ urec_o, float* __restrict__ part_o,
     const float* __restrict__ red_in, int* status, uint64_t wait_ns) {
@@ -281,7 +345,8 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
     float* red_ss = reinterpret_cast<float*>(smem);   // [2][TM]
     float* red_dt = red_ss + 2 * TM;                  // [2][NDH][TM]
     float* dzs = red_dt + 2 * NDH * TM;               // [M + 3][TM]
-    float* ck = dzs + (M + 3) * TM;                   // checkpoints [nck][64][TM]
+    constexpr int ZS = 2 * M + 4;                     // a token's z (M), then y / r (M)
+    float* zs = dzs + (M + 3) * TM;                   // [TM][ZS]
     if (ok) {
       red_ss[h * TM + tok] = ss;
       if constexpr (BWD) {
@@ -291,134 +356,202 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
     }
     nbar8(1, 256);
     if (ok && h == 0) {
-      // ------------------------------------------------- per-token epilogue
+      // ---------------------------------- the logits, one thread per token
       tc::tc_fence_after();
-      const int64_t t = t0 + tok;
-      const bool live = t < T;
+      const bool live = t0 + tok < T;
       const uint32_t lb = tmem + ((uint32_t)(32 * q) << 16);
-      float y[M];
-      {
-        float lo16[16], hi16[16];
-#pragma unroll
-        for (int b16 = 0; b16 < M / 16; ++b16) {
-          tc::tmem_ld16(lb + 16 * b16, hi16);
-          tc::tmem_ld16(lb + M + 16 * b16, lo16);
-          tc::tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) y[16 * b16 + e] = hi16[e] + lo16[e];
-        }
-      }
       const float r = sqrtf((red_ss[tok] + red_ss[TM + tok]) / (float)K + eps);
       Alpha3 al;
       al.load(alpha_p, ag);
-      float z[M];
+      float* zt = zs + tok * ZS;
+      float zf[BWD ? 1 : M];  // the forward keeps its logits in registers
+      bool bad = !isfinite(r);
+      float lo16[16], hi16[16];
 #pragma unroll
-      for (int m = 0; m < M; ++m) {
-        y[m] = y[m] / r;
-        z[m] = fmaf(al.at<N>(m), y[m], __ldg(bias + m));
+      for (int b16 = 0; b16 < M / 16; ++b16) {
+        tc::tmem_ld16(lb + 16 * b16, hi16);
+        tc::tmem_ld16(lb + M + 16 * b16, lo16);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int m = 16 * b16 + e;
+          const float yv = (hi16[e] + lo16[e]) / r;
+          const float z = fmaf(al.at<N>(m), yv, __ldg(bias + m));
+          bad |= !isfinite(z);
+          if constexpr (BWD) {
+            zt[m] = z;
+            zt[M + m] = yv;
+          } else {
+            zf[m] = z;
+          }
+        }
       }
-      if (live) {
-        bool bad = !isfinite(r);
-#pragma unroll
-        for (int m = 0; m < M; ++m) bad |= !isfinite(z[m]);
-        if (bad) flag_status(status, MHC_ERR_NONFINITE);
-      }
-      float spre[N], spost[N];
-#pragma unroll
-      for (int i = 0; i < N; ++i) {
-        spre[i] = sigmoidf_(z[i]);
-        spost[i] = sigmoidf_(z[N + i]);
-      }
-      float H[N * N];
-#pragma unroll
-      for (int e = 0; e < N * N; ++e) H[e] = z[2 * N + e];
+      if (live && bad) flag_status(status, MHC_ERR_NONFINITE);
       if constexpr (!BWD) {
+        // the forward: gates and Sinkhorn in this thread's registers
+        const int64_t t = t0 + tok;
+        float H[N * N];
+#pragma unroll
+        for (int e = 0; e < N * N; ++e) H[e] = zf[2 * N + e];
         sk_forward<N>(H, iters);
         if (live) {
 #pragma unroll
           for (int i = 0; i < N; i += 4) {
             *reinterpret_cast<float4*>(Hpre_o + t * N + i) =
-                make_float4(spre[i], spre[i + 1], spre[i + 2], spre[i + 3]);
+                make_float4(sigmoidf_(zf[i]), sigmoidf_(zf[i + 1]), sigmoidf_(zf[i + 2]),
+                            sigmoidf_(zf[i + 3]));
             *reinterpret_cast<float4*>(Hpost_o + t * N + i) = make_float4(
-                2.0f * spost[i], 2.0f * spost[i + 1], 2.0f * spost[i + 2], 2.0f * spost[i + 3]);
+                2.0f * sigmoidf_(zf[N + i]), 2.0f * sigmoidf_(zf[N + i + 1]),
+                2.0f * sigmoidf_(zf[N + i + 2]), 2.0f * sigmoidf_(zf[N + i + 3]));
           }
 #pragma unroll
           for (int e = 0; e < N * N; e += 4)
             *reinterpret_cast<float4*>(Hres_o + t * N * N + e) =
                 make_float4(H[e], H[e + 1], H[e + 2], H[e + 3]);
         }
-      } else {
-        sk_forward_ckpt<N>(H, iters, ck + tok, TM, ck_period);
-        // dL/dH_res: <G_i, x_j> from the post half's reductions (split) or the
-        // tensor-core reductions' rows (DOTS)
-        constexpr int RSTRIDE = DOTS ? N * N + 2 * N : N * N + N;
-        const float* rt = red_in + (live ? t : 0) * RSTRIDE;
-        float dA[N * N];
+      }
+    }
+    if constexpr (BWD) nbar8(1, 256);
+    if (BWD && ok) {
+      // ------------- gates, Sinkhorn and its adjoint: 8 lanes per token, lane
+      // i on row i of H_res and on pre / post logit i; 4 tokens per warp, the
+      // 8 math warps take the 128 tokens in 4 rounds
+      const int i = lane & 7, sub = lane >> 3, mw = warp - 2;
+      Alpha3 al;
+      al.load(alpha_p, ag);
+#pragma unroll 1
+      for (int rd = 0; rd < TM / 32; ++rd) {
+        const int tk = 32 * rd + 4 * mw + sub;
+        const int64_t t = t0 + tk;
+        const bool live = t < T;
+        const float* zt = zs + tk * ZS;
+        float a[N], sq[N];
 #pragma unroll
-        for (int i = 0; i < N; ++i)
+        for (int j = 0; j < N; ++j) a[j] = zt[2 * N + N * i + j];
+        const float spre = sigmoidf_(zt[i]), spost = sigmoidf_(zt[N + i]);
+        sk8_init(a, iters);
+        {
+          // checkpoints: the iterate after every second normalisation (and the
+          // start), row i of each at ckt + c * 64
+          float* ckt = ck + (live ? t : 0) * ((int64_t)iters + 1) * N * N + N * i;
+          auto ck_store = [&](int c) {
+            if (live) {
+              float4* d4 = reinterpret_cast<float4*>(ckt + (int64_t)c * N * N);
+              d4[0] = make_float4(a[0], a[1], a[2], a[3]);
+              d4[1] = make_float4(a[4], a[5], a[6], a[7]);
+            }
+          };
+          auto ck_load = [&](int c) {
+            if (live) {
+              const float4* s4 = reinterpret_cast<const float4*>(ckt + (int64_t)c * N * N);
+              const float4 v0 = s4[0], v1 = s4[1];
+              a[0] = v0.x; a[1] = v0.y; a[2] = v0.z; a[3] = v0.w;
+              a[4] = v1.x; a[5] = v1.y; a[6] = v1.z; a[7] = v1.w;
+            } else {
 #pragma unroll
-          for (int j = 0; j < N; ++j) dA[i * N + j] = live ? __ldg(rt + i * N + j) : 0.0f;
-        float dzres[N * N];
-        sk_adjoint_ckpt<N>(dA, dzres, iters, ck + tok, TM, ck_period);
-        float dz[M];
-#pragma unroll
-        for (int i = 0; i < N; ++i) {
-          // <g, x_i>: stream i was reduced by the warps of pair member i & 1
-          const float dpre = DOTS ? (live ? __ldg(rt + N * N + N + i) : 0.0f)
-                                  : red_dt[((i & 1) * NDH + 36 + (i >> 1)) * TM + tok];
-          const float dpost = live ? __ldg(rt + N * N + i) : 0.0f;
-          dz[i] = dpre * spre[i] * (1.0f - spre[i]);
-          dz[N + i] = dpost * 2.0f * spost[i] * (1.0f - spost[i]);
-        }
-#pragma unroll
-        for (int e = 0; e < N * N; ++e) dz[2 * N + e] = dzres[e];
-        float dzy[3] = {0.0f, 0.0f, 0.0f};  // dz . y over the pre, post, res logits
-#pragma unroll
-        for (int m = 0; m < M; ++m) {
-          const int g = m < N ? 0 : (m < 2 * N ? 1 : 2);
-          dzy[g] = fmaf(dz[m], y[m], dzy[g]);
-        }
-        if (live) {
-          // the per-token record of the n = 8 apply: H_res | H_pre | H_post | u | kappa
-          float* co = coef_o + t * CF::SIZE;
-#pragma unroll
-          for (int e = 0; e < N * N; ++e) co[CF::RES + e] = H[e];
-#pragma unroll
-          for (int i = 0; i < N; ++i) {
-            co[CF::PRE + i] = spre[i];
-            co[CF::POST + i] = 2.0f * spost[i];
+              for (int j = 0; j < N; ++j) a[j] = 1.0f;
+            }
+          };
+          ck_store(0);
+          for (int qn = 1; qn <= 2 * iters; ++qn) {
+            sk8_step(a, qn, sq);
+            if ((qn & 1) == 0) ck_store(qn >> 1);
           }
-          float ar[3];
+          float H[N];
 #pragma unroll
-          for (int g = 0; g < 3; ++g) ar[g] = al.a[g] / r;
+          for (int j = 0; j < N; ++j) H[j] = a[j];
+          // dL/dH_res: <G_i, x_j> from the post half's reductions (split) or the
+          // tensor-core reductions' rows (DOTS)
+          constexpr int RSTRIDE = DOTS ? N * N + 2 * N : N * N + N;
+          const float* rt = red_in + (live ? t : 0) * RSTRIDE;
+          float g[N];
 #pragma unroll
-          for (int m = 0; m < M; ++m) co[CF::U + m] = ar[m < N ? 0 : (m < 2 * N ? 1 : 2)] * dz[m];
-          co[CF::KAPPA] =
-              fmaf(al.a[2], dzy[2], fmaf(al.a[1], dzy[1], al.a[0] * dzy[0])) / ((float)K * r * r);
-          // the MMA operand row: u to ~16 bits as bf16 high and low parts
-          uint4* ud = reinterpret_cast<uint4*>(urec_o + t * TcRec8::U_ELEMS);
+          for (int j = 0; j < N; ++j) g[j] = live ? __ldg(rt + N * i + j) : 0.0f;
+          for (int step = 2 * iters; step >= 1; --step) {
+            const int c = (step - 1) >> 1;
+            ck_load(c);
+            for (int qn = 2 * c + 1; qn < step; ++qn) sk8_step(a, qn, sq);
+            sk8_step(a, step, sq);
+            sk8_adjoint_step(a, sq, g, step);
+          }
+          ck_load(0);  // the exponentiated logits
+          float dzres[N];
 #pragma unroll
-          for (int v = 0; v < 12; ++v) {  // 8 u values per 16-byte vector, 10 of them used
+          for (int j = 0; j < N; ++j) dzres[j] = g[j] * a[j];
+          // <g, x_i>: stream i was reduced by the warps of pair member i & 1 (split)
+          const float dpre = DOTS ? (live ? __ldg(rt + N * N + N + i) : 0.0f)
+                                  : red_dt[((i & 1) * NDH + 36 + (i >> 1)) * TM + tk];
+          const float dpost = live ? __ldg(rt + N * N + i) : 0.0f;
+          const float dzpre = dpre * spre * (1.0f - spre);
+          const float dzpost = dpost * 2.0f * spost * (1.0f - spost);
+          float pres = 0.0f;
+#pragma unroll
+          for (int j = 0; j < N; ++j) pres = fmaf(dzres[j], zt[M + 2 * N + N * i + j], pres);
+          const float dzy0 = sum8(dzpre * zt[M + i]), dzy1 = sum8(dzpost * zt[M + N + i]);
+          const float dzy2 = sum8(pres);
+          const float r = sqrtf((red_ss[tk] + red_ss[TM + tk]) / (float)K + eps);
+          const float ar0 = al.a[0] / r, ar1 = al.a[1] / r, ar2 = al.a[2] / r;
+          if (live) {
+            // the per-token record of the n = 8 apply: H_res | H_pre | H_post | u | kappa
+            float* co = coef_o + t * CF::SIZE;
+            float4* hr = reinterpret_cast<float4*>(co + CF::RES + N * i);
+            hr[0] = make_float4(H[0], H[1], H[2], H[3]);
+            hr[1] = make_float4(H[4], H[5], H[6], H[7]);
+            co[CF::PRE + i] = spre;
+            co[CF::POST + i] = 2.0f * spost;
+            const float upre = ar0 * dzpre, upost = ar1 * dzpost;
+            co[CF::U + i] = upre;
+            co[CF::U + N + i] = upost;
+            float ures[N];
+#pragma unroll
+            for (int j = 0; j < N; ++j) ures[j] = ar2 * dzres[j];
+            float4* ur = reinterpret_cast<float4*>(co + CF::U + 2 * N + N * i);
+            ur[0] = make_float4(ures[0], ures[1], ures[2], ures[3]);
+            ur[1] = make_float4(ures[4], ures[5], ures[6], ures[7]);
+            if (i == 0)
+              co[CF::KAPPA] = fmaf(al.a[2], dzy2, fmaf(al.a[1], dzy1, al.a[0] * dzy0)) /
+                              ((float)K * r * r);
+            // the MMA operand row: u to ~16 bits as bf16 high and low parts,
+            // [u_hi (80) | 0 (16) | u_lo (80) | 0 (16)]
+            __nv_bfloat16* ud = urec_o + t * TcRec8::U_ELEMS;
+            auto split = [&](float u, __nv_bfloat16& hi, __nv_bfloat16& lo) {
+              hi = __float2bfloat16_rn(u);
+              lo = __float2bfloat16_rn(u - __bfloat162float(hi));
+            };
+            __nv_bfloat16 h0, l0;
+            split(upre, h0, l0);
+            ud[i] = h0;
+            ud[TcRec8::LO + i] = l0;
+            split(upost, h0, l0);
+            ud[N + i] = h0;
+            ud[TcRec8::LO + N + i] = l0;
             uint32_t hw[4], lw[4];
 #pragma unroll
-            for (int p = 0; p < 4; ++p) {
-              const int m0 = 8 * v + 2 * p, m1 = m0 + 1;
-              const float u0 = m0 < M ? ar[m0 < N ? 0 : (m0 < 2 * N ? 1 : 2)] * dz[m0 < M ? m0 : 0] : 0.0f;
-              const float u1 = m1 < M ? ar[m1 < N ? 0 : (m1 < 2 * N ? 1 : 2)] * dz[m1 < M ? m1 : 0] : 0.0f;
-              const __nv_bfloat162 hi = __floats2bfloat162_rn(u0, u1);
-              const __nv_bfloat162 lo =
-                  __floats2bfloat162_rn(u0 - __low2float(hi), u1 - __high2float(hi));
-              hw[p] = *reinterpret_cast<const uint32_t*>(&hi);
-              lw[p] = *reinterpret_cast<const uint32_t*>(&lo);
+            for (int p2 = 0; p2 < 4; ++p2) {
+              const __nv_bfloat162 hi = __floats2bfloat162_rn(ures[2 * p2], ures[2 * p2 + 1]);
+              const __nv_bfloat162 lo = __floats2bfloat162_rn(ures[2 * p2] - __low2float(hi),
+                                                              ures[2 * p2 + 1] - __high2float(hi));
+              hw[p2] = *reinterpret_cast<const uint32_t*>(&hi);
+              lw[p2] = *reinterpret_cast<const uint32_t*>(&lo);
             }
-            ud[v] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-            ud[TcRec8::LO / 8 + v] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            *reinterpret_cast<uint4*>(ud + 2 * N + N * i) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            *reinterpret_cast<uint4*>(ud + TcRec8::LO + 2 * N + N * i) =
+                make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            if (i < 2) {  // the zero padding after u_hi and after u_lo
+              *reinterpret_cast<uint4*>(ud + M + 8 * i) = make_uint4(0, 0, 0, 0);
+              *reinterpret_cast<uint4*>(ud + TcRec8::LO + M + 8 * i) = make_uint4(0, 0, 0, 0);
+            }
+          }
+          dzs[i * TM + tk] = live ? dzpre : 0.0f;
+          dzs[(N + i) * TM + tk] = live ? dzpost : 0.0f;
+#pragma unroll
+          for (int j = 0; j < N; ++j) dzs[(2 * N + N * i + j) * TM + tk] = live ? dzres[j] : 0.0f;
+          if (i == 0) {
+            dzs[M * TM + tk] = live ? dzy0 : 0.0f;
+            dzs[(M + 1) * TM + tk] = live ? dzy1 : 0.0f;
+            dzs[(M + 2) * TM + tk] = live ? dzy2 : 0.0f;
           }
         }
-#pragma unroll
-        for (int m = 0; m < M; ++m) dzs[m * TM + tok] = live ? dz[m] : 0.0f;
-#pragma unroll
-        for (int g = 0; g < 3; ++g) dzs[(M + g) * TM + tok] = live ? dzy[g] : 0.0f;
       }
     }
     if constexpr (BWD) {
@@ -471,38 +604,29 @@ __global__ void k_phi_split8(int64_t C, int64_t ncp, const float* __restrict__ p
   }
 }
 
-// Smallest checkpoint period whose checkpoints fit in the stage memory beside
-// the epilogue's reductions and dz sums.
-int map8_ck_period(int iters, size_t data_bytes) {
-  using namespace tcm8;
-  const size_t scratch = (size_t)(2 * TM + 2 * NDH * TM + (M + 3) * TM) * 4;
-  const size_t per_ck = (size_t)N * N * TM * 4;
-  const int max_ck = (int)((data_bytes - scratch) / per_ck);
-  const int steps = 2 * iters;
-  int P = 1;
-  while (steps / P + 1 > max_ck) ++P;
-  return P;
-}
-
 template <int MODE>
 cudaError_t launch_map8(const CUtensorMap& mx, const void* phi_t, const CUtensorMap& mg,
                         int64_t T, int64_t C,
                         int iters, float eps, const float* b, const float* alpha, int ag,
                         float* Hpre, float* Hpost, float* Hres, float* coef, void* urec,
-                        float* part, const float* red, int* st, int64_t wait_ns, cudaStream_t s) {
+                        float* part, const float* red, float* ck, int* st, int64_t wait_ns,
+                        cudaStream_t s) {
   using namespace tcm8;
   auto kern = k_map8_tc<MODE>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<MODE>::SMEM);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)((T + TM - 1) / TM);
-  const int P = map8_ck_period(iters, Cfg<MODE>::DATA);
-  kern<<<grid, NT, Cfg<MODE>::SMEM, s>>>(mx, (const __nv_bfloat16*)phi_t, mg, T, C, iters, eps, P, b, alpha, ag,
+  kern<<<grid, NT, Cfg<MODE>::SMEM, s>>>(mx, (const __nv_bfloat16*)phi_t, mg, T, C, iters, eps, ck, b, alpha, ag,
                                           Hpre, Hpost, Hres, coef, (__nv_bfloat16*)urec, part,
                                           red, st, tc::wait_limit(wait_ns));
   return cudaGetLastError();
 }
 }  // namespace
+
+size_t map8_ck_bytes(int64_t T, int iters) {
+  return (size_t)T * ((size_t)iters + 1) * tcm8::N * tcm8::N * 4;
+}
 
 size_t map8_tc_phi_bytes(int64_t C) {
   const int64_t nblk = (C + tcm8::CH - 1) / tcm8::CH * (tcm8::CH / tcm8::PB);
@@ -513,8 +637,8 @@ cudaError_t map8_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float ep
                              const float* phi, void* phi_split, const float* b,
                              const float* alpha, int ag, float* Hpre, float* Hpost, float* Hres,
                              const void* G, const void* g, const void* f, const float* red,
-                             float* coef, void* urec, float* part, int* st, int64_t wait_ns,
-                             cudaStream_t s) {
+                             float* coef, void* urec, float* part, float* ck, int* st,
+                             int64_t wait_ns, cudaStream_t s) {
   using namespace tcm8;
   const int64_t ncp = (C + CH - 1) / CH * CH;
   k_phi_split8<<<(unsigned)((N * ncp + 255) / 256), 256, 0, s>>>(C, ncp, phi,
@@ -539,13 +663,16 @@ cudaError_t map8_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float ep
   switch (mode) {
     case MAP_FWD:
       return launch_map8<MAP_FWD>(mx, phi_split, mg, T, C, iters, eps, b, alpha, ag, Hpre, Hpost,
-                                  Hres, nullptr, nullptr, nullptr, nullptr, st, wait_ns, s);
+                                  Hres, nullptr, nullptr, nullptr, nullptr, nullptr, st, wait_ns,
+                                  s);
     case MAP_BWD_SPLIT:
       return launch_map8<MAP_BWD_SPLIT>(mx, phi_split, mg, T, C, iters, eps, b, alpha, ag, nullptr,
-                                        nullptr, nullptr, coef, urec, part, red, st, wait_ns, s);
+                                        nullptr, nullptr, coef, urec, part, red, ck, st, wait_ns,
+                                        s);
     case MAP_BWD_DOTS:
       return launch_map8<MAP_BWD_DOTS>(mx, phi_split, mg, T, C, iters, eps, b, alpha, ag, nullptr,
-                                       nullptr, nullptr, coef, urec, part, red, st, wait_ns, s);
+                                       nullptr, nullptr, coef, urec, part, red, ck, st, wait_ns,
+                                       s);
     default:
       return cudaErrorInvalidValue;
   }

@@ -76,8 +76,9 @@ size_t rows16_bytes(int64_t T) { return (size_t)T * mhc::Coef<16>::SIZE * 4; }
 // 128-token CTA, the bf16 split copy of phi^T that the mapping MMA reads, and
 // the apply kernel's grad_phi partials and slice counters.  Tensor-core path
 // (n = 8): the coefficient records, the U rows, the C-reductions of the
-// backward mapping, the partial sums, the phi split copy and the grad_phi
-// parts of the blocks that the apply's CTAs share.
+// backward mapping, the partial sums, the phi split copy, the grad_phi parts
+// of the blocks that the apply's CTAs share, and the mapping's Sinkhorn
+// checkpoints.
 struct BwdWorkspace {
   size_t coef_off, urec_off, hrec_off, part_off, phi_off, apply_off, kmap_off, red_off, total;
   int nparts;
@@ -127,8 +128,13 @@ BwdWorkspace bwd_layout(const mhc_params* p) {
   if (use_tc16(p))
     apply_bytes = std::max((size_t)p->T * 16 * p->C * 4, mhc::wide_ck_bytes(p->T, p->t_max));
   off = round_up(off + apply_bytes, 256);
+  // the mapping's scratch: n = 4, its channel-split records; n = 8, its Sinkhorn
+  // checkpoints
   w.kmap_off = off;
-  off = round_up(off + (tc ? mhc::map_tc_scratch_bytes(p->T, p->C) : 0), 256);
+  off = round_up(off + (tc    ? mhc::map_tc_scratch_bytes(p->T, p->C)
+                        : tc8 ? mhc::map8_ck_bytes(p->T, p->t_max)
+                              : 0),
+                 256);
   w.total = off;
   return w;
 }
@@ -196,7 +202,7 @@ mhc_status mhc_pre(const mhc_params* p, const void* x, const float* phi, const f
     st = from_cuda(mhc::map8_tc_dispatch(mhc::MAP_FWD, p->T, p->C, p->t_max, p->eps, x, phi,
                                          workspace, b, alpha, alpha_groups(p), H_pre, H_post,
                                          H_res, nullptr, nullptr, nullptr, nullptr, nullptr,
-                                         nullptr, nullptr, dev_status, p->wait_ns, s));
+                                         nullptr, nullptr, nullptr, dev_status, p->wait_ns, s));
   } else if (use_tc16(p)) {
     const size_t need = mhc_pre_workspace_size(p);
     if (workspace == nullptr || workspace_bytes < need || ((uintptr_t)workspace & 255u) != 0)
@@ -266,8 +272,8 @@ mhc_status mhc_backward_map(const mhc_params* p, const void* x, const float* phi
                                            nullptr, nullptr, nullptr, nullptr, nullptr,
                                            (const float*)(ws + w.red_off),
                                            (float*)(ws + w.coef_off), ws + w.urec_off,
-                                           (float*)(ws + w.part_off), dev_status, p->wait_ns,
-                                           (cudaStream_t)stream));
+                                           (float*)(ws + w.part_off), (float*)(ws + w.kmap_off),
+                                           dev_status, p->wait_ns, (cudaStream_t)stream));
   }
   if (use_tc16(p))
     return from_cuda(mhc::wide_map_tc_dispatch(
@@ -378,7 +384,7 @@ mhc_status mhc_post_fused(const mhc_params* p, const void* x, const void* f_out,
                                            phi_next, workspace, b_next, alpha_next,
                                            alpha_groups(p), H_pre_next, H_post_next, H_res_next,
                                            nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
-                                           nullptr, dev_status, p->wait_ns, s));
+                                           nullptr, nullptr, dev_status, p->wait_ns, s));
   }
   if (use_tc16(p)) {
     const size_t need = mhc_post_fused_workspace_size(p);
@@ -463,7 +469,8 @@ mhc_status mhc_pre_backward(const mhc_params* p, const void* x, const float* phi
                                          phi, ws + w.phi_off, b, alpha, alpha_groups(p), nullptr,
                                          nullptr, nullptr, nullptr, grad_h_in, nullptr, red,
                                          (float*)(ws + w.coef_off), ws + w.urec_off,
-                                         (float*)(ws + w.part_off), dev_status, p->wait_ns, s));
+                                         (float*)(ws + w.part_off), (float*)(ws + w.kmap_off),
+                                         dev_status, p->wait_ns, s));
     if (st != MHC_OK) return st;
     return from_cuda(mhc::apply8_tc_dispatch(
         p->T, p->C, x, ws + w.phi_off, grad_x_next, grad_h_in, (const float*)(ws + w.coef_off),

@@ -63,13 +63,17 @@ cudaError_t phi_split_dispatch(int64_t K, const float* phi, void* phi_split, cud
 // MAP_BWD_SPLIT or MAP_BWD_DOTS (G and f are not read).  Splits phi into phi_split (map8_tc_phi_bytes(C)
 // bytes); the backward modes write the per-token records (coef
 // [T][Coef<8>::SIZE]), the U rows (urec [T][TcRec8::U_ELEMS] bf16) and one
-// partial-sum record per 128 tokens (part).
+// partial-sum record per 128 tokens (part); the backward modes keep Sinkhorn
+// checkpoints in ck (map8_ck_bytes(T, iters) bytes; unused forward).
 cudaError_t map8_tc_dispatch(int mode, int64_t T, int64_t C, int iters, float eps, const void* x,
                              const float* phi, void* phi_split, const float* b,
                              const float* alpha, int ag, float* Hpre, float* Hpost, float* Hres,
                              const void* G, const void* g, const void* f, const float* red,
-                             float* coef, void* urec, float* part, int* st, int64_t wait_ns,
-                             cudaStream_t s);
+                             float* coef, void* urec, float* part, float* ck, int* st,
+                             int64_t wait_ns, cudaStream_t s);
+// Sinkhorn checkpoints of the n = 8 backward mapping (ck, global scratch):
+// iters + 1 iterates of 64 floats per token
+size_t map8_ck_bytes(int64_t T, int iters);
 // k_apply8_tc.cu (bf16, n = 8): grad_x / grad_f_out with phi u on the tensor
 // cores (the accumulators stay on chip), grad_phi as a tensor-core contraction
 // over the tokens, and grad_b / grad_alpha from the partial sums; phi_split is
