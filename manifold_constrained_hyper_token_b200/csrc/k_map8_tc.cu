@@ -97,69 +97,6 @@ __device__ __forceinline__ void nbar8(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-// ---------------------------------------------- 8 lanes per 8 x 8 matrix
-// Sinkhorn-Knopp and its adjoint for one token's 8 x 8 matrix on an aligned
-// group of 8 lanes, lane i holding row i.  Column sums are butterflies over
-// the group (xor 4, 2, 1), so every lane of the group gets every column's sum,
-// with the same bits.  The four groups of a warp run the same steps.
-__device__ __forceinline__ float sum8(float v) {
-  v += __shfl_xor_sync(0xffffffffu, v, 4);
-  v += __shfl_xor_sync(0xffffffffu, v, 2);
-  v += __shfl_xor_sync(0xffffffffu, v, 1);
-  return v;
-}
-
-__device__ __forceinline__ void sk8_init(float (&a)[8], int iters) {
-  float mx = 0.0f;
-  if (iters > 0) {
-    mx = a[0];
-#pragma unroll
-    for (int j = 1; j < 8; ++j) mx = fmaxf(mx, a[j]);
-  }
-#pragma unroll
-  for (int j = 0; j < 8; ++j) a[j] = expf(a[j] - mx);
-}
-
-// Normalisation q (odd: rows, even: columns); s receives the sums divided out
-// (odd q: s[0] = this lane's row sum; even q: s[j] = column j's sum).
-__device__ __forceinline__ void sk8_step(float (&a)[8], int q, float (&s)[8]) {
-  if (q & 1) {
-    float acc = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc += a[j];
-    const float inv = 1.0f / acc;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) a[j] *= inv;
-    s[0] = acc;
-    return;
-  }
-#pragma unroll
-  for (int j = 0; j < 8; ++j) s[j] = sum8(a[j]);
-#pragma unroll
-  for (int j = 0; j < 8; ++j) a[j] *= 1.0f / s[j];
-}
-
-// One adjoint step: a is the iterate after normalisation q, s its sums, g the
-// gradient with respect to it (this lane's row), turned into the gradient with
-// respect to the iterate before the step.
-__device__ __forceinline__ void sk8_adjoint_step(const float (&a)[8], const float (&s)[8],
-                                                 float (&g)[8], int q) {
-  if (q & 1) {
-    float d = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) d = fmaf(g[j], a[j], d);
-    const float inv = 1.0f / s[0];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) g[j] = (g[j] - d) * inv;
-    return;
-  }
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const float d = sum8(g[j] * a[j]);
-    g[j] = (g[j] - d) * (1.0f / s[j]);
-  }
-}
-
 }  // namespace
 
 template <int MODE>
@@ -429,7 +366,7 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
 #pragma unroll
         for (int j = 0; j < N; ++j) a[j] = zt[2 * N + N * i + j];
         const float spre = sigmoidf_(zt[i]), spost = sigmoidf_(zt[N + i]);
-        sk8_init(a, iters);
+        skl_init<N>(a, iters);
         {
           // checkpoints: the iterate after every second normalisation (and the
           // start), row i of each at ckt + c * 64
@@ -454,7 +391,7 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
           };
           ck_store(0);
           for (int qn = 1; qn <= 2 * iters; ++qn) {
-            sk8_step(a, qn, sq);
+            skl_step<N>(a, qn, sq);
             if ((qn & 1) == 0) ck_store(qn >> 1);
           }
           float H[N];
@@ -470,9 +407,9 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
           for (int step = 2 * iters; step >= 1; --step) {
             const int c = (step - 1) >> 1;
             ck_load(c);
-            for (int qn = 2 * c + 1; qn < step; ++qn) sk8_step(a, qn, sq);
-            sk8_step(a, step, sq);
-            sk8_adjoint_step(a, sq, g, step);
+            for (int qn = 2 * c + 1; qn < step; ++qn) skl_step<N>(a, qn, sq);
+            skl_step<N>(a, step, sq);
+            skl_adjoint_step<N>(a, sq, g, step);
           }
           ck_load(0);  // the exponentiated logits
           float dzres[N];
@@ -487,8 +424,8 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
           float pres = 0.0f;
 #pragma unroll
           for (int j = 0; j < N; ++j) pres = fmaf(dzres[j], zt[M + 2 * N + N * i + j], pres);
-          const float dzy0 = sum8(dzpre * zt[M + i]), dzy1 = sum8(dzpost * zt[M + N + i]);
-          const float dzy2 = sum8(pres);
+          const float dzy0 = group_sum<N>(dzpre * zt[M + i]), dzy1 = group_sum<N>(dzpost * zt[M + N + i]);
+          const float dzy2 = group_sum<N>(pres);
           const float r = sqrtf((red_ss[tk] + red_ss[TM + tk]) / (float)K + eps);
           const float ar0 = al.a[0] / r, ar1 = al.a[1] / r, ar2 = al.a[2] / r;
           if (live) {

@@ -319,4 +319,73 @@ __device__ __forceinline__ uint32_t f2_to_bf2(uint64_t v) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// ------------------------------------------- N lanes per N x N Sinkhorn matrix
+// Sinkhorn-Knopp and its adjoint for one token's N x N matrix on an aligned
+// group of N lanes (N = 4 or 8), lane i holding row i.  Column sums are
+// butterflies over the group (xor N/2, .., 1), so every lane of the group gets
+// every column's sum, with the same bits.  All groups of a warp run the same
+// steps (the shuffles are warp-wide).
+template <int N>
+__device__ __forceinline__ float group_sum(float v) {
+#pragma unroll
+  for (int o = N / 2; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <int N>
+__device__ __forceinline__ void skl_init(float (&a)[N], int iters) {
+  float mx = 0.0f;
+  if (iters > 0) {
+    mx = a[0];
+#pragma unroll
+    for (int j = 1; j < N; ++j) mx = fmaxf(mx, a[j]);
+  }
+#pragma unroll
+  for (int j = 0; j < N; ++j) a[j] = expf(a[j] - mx);
+}
+
+// Normalisation q (odd: rows, even: columns); s receives the sums divided out
+// (odd q: s[0] = this lane's row sum; even q: s[j] = column j's sum).
+template <int N>
+__device__ __forceinline__ void skl_step(float (&a)[N], int q, float (&s)[N]) {
+  if (q & 1) {
+    float acc = 0.0f;
+#pragma unroll
+    for (int j = 0; j < N; ++j) acc += a[j];
+    const float inv = 1.0f / acc;
+#pragma unroll
+    for (int j = 0; j < N; ++j) a[j] *= inv;
+    s[0] = acc;
+    return;
+  }
+#pragma unroll
+  for (int j = 0; j < N; ++j) s[j] = group_sum<N>(a[j]);
+#pragma unroll
+  for (int j = 0; j < N; ++j) a[j] *= 1.0f / s[j];
+}
+
+// One adjoint step: a is the iterate after normalisation q, s its sums, g the
+// gradient with respect to it (this lane's row), turned into the gradient with
+// respect to the iterate before the step:
+//   rows:    g_ij <- (g_ij - sum_k g_ik a_ik) / s_i
+//   columns: g_ij <- (g_ij - sum_k g_kj a_kj) / s_j
+template <int N>
+__device__ __forceinline__ void skl_adjoint_step(const float (&a)[N], const float (&s)[N],
+                                                 float (&g)[N], int q) {
+  if (q & 1) {
+    float d = 0.0f;
+#pragma unroll
+    for (int j = 0; j < N; ++j) d = fmaf(g[j], a[j], d);
+    const float inv = 1.0f / s[0];
+#pragma unroll
+    for (int j = 0; j < N; ++j) g[j] = (g[j] - d) * inv;
+    return;
+  }
+#pragma unroll
+  for (int j = 0; j < N; ++j) {
+    const float d = group_sum<N>(g[j] * a[j]);
+    g[j] = (g[j] - d) * (1.0f / s[j]);
+  }
+}
+
 }  // namespace mhc
