@@ -372,7 +372,6 @@ __global__ void __launch_bounds__(widek::NT) k_wide_map(
   extern __shared__ __align__(16) float smem[];
   float* stg = smem;
   float* ys = smem + YS_OFF;
-  float* dts = smem + DT_OFF;
   float* sss = smem + SS_OFF;
   const int tid = threadIdx.x, ty = tid >> 5, tx = tid & 31;
   const int64_t t0 = (int64_t)blockIdx.x * TB;
