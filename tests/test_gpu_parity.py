@@ -475,6 +475,20 @@ def test_wide_backward_is_deterministic(mhc, dtype):
         assert torch.equal(u, v)
 
 
+@pytest.mark.parametrize("T,C", [(1000, 1024), (2048, 7168)])
+def test_n8_backward_is_deterministic(mhc, T, C):
+    """n = 8 with bf16 runs the tensor-core kernels, whose grad_phi is split over
+    persistent CTAs (shared blocks added in CTA order) and whose Sinkhorn sums run
+    as butterflies over 8 lanes: repeated calls give identical bits."""
+    d = _dev(_inputs(T, 8, C, torch.bfloat16, seed=10))
+    a = mhc.mhc_backward(d["x"], d["phi"], d["b"], d["alpha"], d["f_out"], d["grad_x_next"],
+                         d["grad_h_in"])
+    b = mhc.mhc_backward(d["x"], d["phi"], d["b"], d["alpha"], d["f_out"], d["grad_x_next"],
+                         d["grad_h_in"])
+    for u, v in zip(a, b):
+        assert torch.equal(u, v)
+
+
 def test_backward_small_workspace_rejected(mhc):
     d = _dev(_inputs(64, 4, 64, torch.bfloat16))
     need = mhc.mhc_backward_workspace_size(4, 64, 64, torch.bfloat16)
