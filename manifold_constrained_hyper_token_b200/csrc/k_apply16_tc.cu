@@ -20,7 +20,9 @@
 //   k_gx16    grad_x and grad_f_out from that scratch (CUDA cores, 8-byte vectors,
 //             paired fp32 FMAs)
 //   k_gphi16  grad_phi for 128 rows of phi: D[128 x 288] += X^T (u_hi + u_lo)
-//             over every token tile (tcgen05)
+//             over every token tile (tcgen05), the (block, tile) units split
+//             evenly over persistent CTAs; k_gphi16_fin adds the parts of
+//             blocks that two or more CTAs share
 //
 // grad_b and grad_alpha come from the mapping's partial sums (k_wide.cu).  All
 // sums run in a fixed order, so repeated calls give identical bits.  Waits are
@@ -66,6 +68,7 @@ constexpr int G_DATA = G_NS * G_STAGE;
 constexpr int G_SMEM = G_DATA + 1024 + 128;
 constexpr int G_NT = 6 * 32;
 constexpr uint32_t G_TMEM = 512;
+constexpr int G_MAXGRID = 256;          // partial-sum slots are sized for this many CTAs
 static_assert(A_SMEM <= 232448 && G_SMEM <= 232448, "shared memory");
 static_assert(A_STAGE % 1024 == 0 && A_XT_OFF % 1024 == 0, "stage alignment");
 }  // namespace ap16
@@ -360,35 +363,47 @@ __global__ void __launch_bounds__(128, 4) k_gx16(int64_t T, int64_t C,
   }
 }
 
-// --------------------------------------------------------------- grad_phi
+// grad_phi for 128 rows of phi (128 channels of one stream) per (block, token
+// tile) unit: D[128 x 288] += X^T (u_hi + u_lo), the u_hi half of a tile then
+// its u_lo half through the stage ring.  The units, block-major, are split
+// evenly over persistent CTAs (a contiguous range each); a range cuts into one
+// segment per block it touches.  D (288 TMEM columns) is single: before a
+// segment's first MMA the MMA warp waits for the previous segment's epilogue.
+// A segment that covers its whole block writes grad_phi; the first and last
+// segments of a range can be parts of a block and write the CTA's partial
+// slots 0 and 1, which k_gphi16_fin adds in CTA order.
 __global__ void __launch_bounds__(ap16::G_NT, 1) k_gphi16(const __grid_constant__ CUtensorMap tm_x,
                                                          const __grid_constant__ CUtensorMap tm_u,
                                                          int64_t T, int64_t C, int ncb,
+                                                         int64_t nunits,
                                                          float* __restrict__ grad_phi,
+                                                         float* __restrict__ partial,
                                                          int* status, uint64_t wait_ns) {
   using namespace ap16;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + G_DATA);  // full[2] empty[2] done fin
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * G_NS + 2);
+  // full[2] empty[2] dfull dempty fin
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + G_DATA);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * G_NS + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   auto full = [&](int s) { return tc::smem_u32(bars + s); };
   auto empty = [&](int s) { return tc::smem_u32(bars + G_NS + s); };
-  const uint32_t done_bar = tc::smem_u32(bars + 2 * G_NS);
-  const uint32_t fin_bar = tc::smem_u32(bars + 2 * G_NS + 1);
+  const uint32_t dfull = tc::smem_u32(bars + 2 * G_NS);
+  const uint32_t dempty = tc::smem_u32(bars + 2 * G_NS + 1);
+  const uint32_t fin_bar = tc::smem_u32(bars + 2 * G_NS + 2);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int j = blockIdx.x / ncb, cb = blockIdx.x % ncb;
-  const int c0 = cb * CB;
-  const int ntt = (int)((T + TT - 1) / TT);
-  const int nst = 2 * ntt;  // per token tile: the u_hi half, then the u_lo half
+  const int64_t ntt = (T + TT - 1) / TT;
+  const int64_t lo = (int64_t)blockIdx.x * nunits / gridDim.x;
+  const int64_t hi = ((int64_t)blockIdx.x + 1) * nunits / gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < G_NS; ++s) {
       tc::mbar_init(full(s), 1);
       tc::mbar_init(empty(s), 1);
     }
-    tc::mbar_init(done_bar, 1);
+    tc::mbar_init(dfull, 1);
+    tc::mbar_init(dempty, 4);  // the four epilogue warps
     tc::mbar_init(fin_bar, 1);
     *abort_flag = 0;
     tc::mbar_fence_init();
@@ -409,25 +424,31 @@ __global__ void __launch_bounds__(ap16::G_NT, 1) k_gphi16(const __grid_constant_
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------------- TMA
     const uint64_t pol_x = tc::policy_evict_normal(), pol_u = tc::policy_evict_last();
-    int issued = 0;
-    for (int g = 0; g < nst; ++g) {
-      const int s = g % G_NS;
-      if (g >= G_NS &&
-          !tc::mbar_wait(empty(s), ((uint32_t)(g / G_NS) & 1u) ^ 1u, abort_flag, wait_ns)) {
-        give_up();
-        break;
+    int64_t g = 0;
+    bool stop = false;
+    for (int64_t u = lo; u < hi && !stop; ++u) {
+      const int64_t blk = u / ntt, tile = u % ntt;
+      const int j = (int)(blk / ncb), c0 = (int)(blk % ncb) * CB;
+      for (int hh = 0; hh < 2; ++hh, ++g) {  // the u_hi half, then the u_lo half
+        const int s = (int)(g % G_NS);
+        if (g >= G_NS &&
+            !tc::mbar_wait(empty(s), ((uint32_t)(g / G_NS) & 1u) ^ 1u, abort_flag, wait_ns)) {
+          give_up();
+          stop = true;
+          break;
+        }
+        const uint32_t base = tc::smem_u32(smem + s * G_STAGE);
+        tc::mbar_arrive_expect_tx(full(s), (uint32_t)G_STAGE);
+        for (int a = 0; a < 2; ++a)
+          tc::tma_load_3d(base + G_X + a * ATOM, &tm_x, full(s), c0 + 64 * a, j,
+                          (int)(tile * TT), pol_x);
+        for (int a = 0; a < 5; ++a)
+          tc::tma_load_2d(base + G_U + a * ATOM, &tm_u, full(s), hh * MP + 64 * a,
+                          (int)(tile * TT), pol_u);
       }
-      const int it = g >> 1, hh = g & 1;
-      const uint32_t base = tc::smem_u32(smem + s * G_STAGE);
-      tc::mbar_arrive_expect_tx(full(s), (uint32_t)G_STAGE);
-      for (int a = 0; a < 2; ++a)
-        tc::tma_load_3d(base + G_X + a * ATOM, &tm_x, full(s), c0 + 64 * a, j, it * TT, pol_x);
-      for (int a = 0; a < 5; ++a)
-        tc::tma_load_2d(base + G_U + a * ATOM, &tm_u, full(s), hh * MP + 64 * a, it * TT, pol_u);
-      ++issued;
     }
-    for (int g = (issued > G_NS ? issued - G_NS : 0); g < issued; ++g)
-      tc::mbar_wait(full(g % G_NS), (uint32_t)(g / G_NS) & 1u, nullptr, tc::kDrainWaitNs);
+    for (int64_t q = (g > G_NS ? g - G_NS : 0); q < g; ++q)
+      tc::mbar_wait(full((int)(q % G_NS)), (uint32_t)(q / G_NS) & 1u, nullptr, tc::kDrainWaitNs);
   } else if (warp == 1 && lane == 0) {
     // ---------------------------------------------------------------- MMA
     // D[k][m] += sum over 16 tokens of X[tok][k] U[tok][m]: A = X^T (MN-major,
@@ -435,43 +456,69 @@ __global__ void __launch_bounds__(ap16::G_NT, 1) k_gphi16(const __grid_constant_
     // 128..287 (N = 160) of the half, into D columns 0..127 and 128..287
     constexpr uint32_t id1 = tc::idesc_bf16(CB, 128, true, true);
     constexpr uint32_t id2 = tc::idesc_bf16(CB, 160, true, true);
-    bool any = false;
-    for (int g = 0; g < nst; ++g) {
-      const int s = g % G_NS;
-      if (!tc::mbar_wait(full(s), (uint32_t)(g / G_NS) & 1u, abort_flag, wait_ns)) {
+    bool any = false, stop = false;
+    int seg = 0;
+    int64_t g = 0;
+    for (int64_t u = lo; u < hi && !stop; ++u) {
+      const int64_t tile = u % ntt;
+      const bool first = u == lo || tile == 0, last = u == hi - 1 || tile == ntt - 1;
+      if (first && seg >= 1 &&
+          !tc::mbar_wait(dempty, ((uint32_t)(seg - 1) & 1u), abort_flag, wait_ns)) {
         give_up();
         break;
       }
-      tc::tc_fence_after();
-      const uint32_t base = tc::smem_u32(smem + s * G_STAGE);
+      for (int hh = 0; hh < 2; ++hh, ++g) {
+        const int s = (int)(g % G_NS);
+        if (!tc::mbar_wait(full(s), (uint32_t)(g / G_NS) & 1u, abort_flag, wait_ns)) {
+          give_up();
+          stop = true;
+          break;
+        }
+        tc::tc_fence_after();
+        const uint32_t base = tc::smem_u32(smem + s * G_STAGE);
 #pragma unroll
-      for (int k = 0; k < TT / 16; ++k) {
-        const uint64_t da = tc::smem_desc(base + G_X + k * 2048, ATOM, 1024, tc::SWZ_128B);
-        const uint64_t b1 = tc::smem_desc(base + G_U + k * 2048, ATOM, 1024, tc::SWZ_128B);
-        const uint64_t b2 =
-            tc::smem_desc(base + G_U + 2 * ATOM + k * 2048, ATOM, 1024, tc::SWZ_128B);
-        const uint32_t acc = (g | k) != 0 ? 1u : 0u;
-        tc::mma_bf16(tmem, da, b1, id1, acc);
-        tc::mma_bf16(tmem + 128, da, b2, id2, acc);
+        for (int k = 0; k < TT / 16; ++k) {
+          const uint64_t da = tc::smem_desc(base + G_X + k * 2048, ATOM, 1024, tc::SWZ_128B);
+          const uint64_t b1 = tc::smem_desc(base + G_U + k * 2048, ATOM, 1024, tc::SWZ_128B);
+          const uint64_t b2 =
+              tc::smem_desc(base + G_U + 2 * ATOM + k * 2048, ATOM, 1024, tc::SWZ_128B);
+          const uint32_t acc = (first && hh == 0 && k == 0) ? 0u : 1u;
+          tc::mma_bf16(tmem, da, b1, id1, acc);
+          tc::mma_bf16(tmem + 128, da, b2, id2, acc);
+        }
+        any = true;
+        tc::mma_commit(empty(s));
       }
-      any = true;
-      tc::mma_commit(empty(s));
+      if (stop) break;
+      if (last) {
+        tc::mma_commit(dfull);
+        ++seg;
+      }
     }
-    if (!*abort_flag) tc::mma_commit(done_bar);
     if (any) {
       tc::mma_commit(fin_bar);
       tc::mbar_wait(fin_bar, 0, nullptr, tc::kDrainWaitNs);
     }
   } else if (warp >= 2) {
-    // ----- epilogue: warp w holds phi rows (channels) 32(w % 4).. of this block
-    bool ok = !*abort_flag && tc::mbar_wait(done_bar, 0, abort_flag, wait_ns);
-    if (!ok && !*abort_flag) give_up();
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok) {
+    // ----- epilogue: warp w holds phi rows (channels) 32(w % 4).. of the segment's block
+    const int qd = warp & 3;
+    const int64_t b0 = lo / ntt, b1 = hi > lo ? (hi - 1) / ntt : b0 - 1;
+    bool ok = true;
+    for (int64_t blk = b0; blk <= b1 && ok; ++blk) {
+      const int si = (int)(blk - b0);
+      bool okw = tc::mbar_wait(dfull, (uint32_t)si & 1u, abort_flag, wait_ns);
+      if (!okw && !*abort_flag) give_up();
+      ok = __all_sync(0xffffffffu, okw);
+      if (!ok) break;
       tc::tc_fence_after();
-      const int qd = warp & 3;
-      const int64_t c = (int64_t)c0 + 32 * qd + lane;
-      float* dst = grad_phi + ((int64_t)j * C + c) * M;
+      const int64_t s_lo = blk * ntt > lo ? blk * ntt : lo;
+      const int64_t s_hi = (blk + 1) * ntt < hi ? (blk + 1) * ntt : hi;
+      const bool whole = s_lo == blk * ntt && s_hi == (blk + 1) * ntt;
+      const int j = (int)(blk / ncb);
+      const int64_t c = (blk % ncb) * CB + 32 * qd + lane;
+      float* dst = whole ? grad_phi + ((int64_t)j * C + c) * M
+                         : partial + (((int64_t)blockIdx.x * 2 + (si == 0 ? 0 : 1)) * CB +
+                                      32 * qd + lane) * M;
       const uint32_t lb = tmem + ((uint32_t)(32 * qd) << 16);
 #pragma unroll 1
       for (int b16 = 0; b16 < M / 16; ++b16) {
@@ -485,6 +532,9 @@ __global__ void __launch_bounds__(ap16::G_NT, 1) k_gphi16(const __grid_constant_
                 make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
         }
       }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(dempty);
     }
   }
   __syncwarp();
@@ -496,8 +546,39 @@ __global__ void __launch_bounds__(ap16::G_NT, 1) k_gphi16(const __grid_constant_
   }
 }
 
+// grad_phi rows of the blocks that several CTAs share: the CTAs' partial
+// slots added in CTA order.  One thread per (block, row).
+__global__ void k_gphi16_fin(int64_t C, int ncb, int64_t ntt, int64_t nunits, int grid,
+                             const float* __restrict__ partial, float* __restrict__ grad_phi) {
+  using namespace ap16;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // blk * CB + row
+  const int64_t blk = idx / CB;
+  const int row = (int)(idx % CB);
+  if (blk >= nunits / ntt) return;
+  auto owner = [&](int64_t u) { return ((u + 1) * grid - 1) / nunits; };
+  const int64_t bfirst = owner(blk * ntt), blast = owner((blk + 1) * ntt - 1);
+  if (bfirst == blast) return;  // one CTA covered the block and wrote it
+  const int64_t c = (blk % ncb) * CB + row;
+  if (c >= C) return;
+  float* dst = grad_phi + ((blk / ncb) * C + c) * M;
+  for (int m4 = 0; m4 < M; m4 += 4) {
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int64_t b = bfirst; b <= blast; ++b) {
+      const int64_t lo_b = b * nunits / grid;
+      const int slot = lo_b / ntt == blk ? 0 : 1;
+      const float4 v = *reinterpret_cast<const float4*>(partial + ((b * 2 + slot) * CB + row) * M + m4);
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    *reinterpret_cast<float4*>(dst + m4) = acc;
+  }
+}
+
 // ------------------------------------------------------------------ host
 size_t apply16_urec_bytes(int64_t T) { return (size_t)T * ap16::NU * 2; }
+size_t apply16_gphi_part_bytes() { return (size_t)ap16::G_MAXGRID * 2 * ap16::CB * ap16::M * 4; }
 
 cudaError_t apply16_tc_dispatch(int64_t T, int64_t C, const void* x, const void* phi_t,
                                 const void* G, const void* g, const float* coef,
@@ -543,9 +624,20 @@ cudaError_t apply16_tc_dispatch(int64_t T, int64_t C, const void* x, const void*
   if (e != cudaSuccess) return e;
 
   const int ncb_c = (int)((C + CB - 1) / CB);
+  const int64_t nunits_c = (int64_t)N * ncb_c * ntt;
+  int grid_c = (int)(nunits_c < nsm ? nunits_c : nsm);
+  if (grid_c > G_MAXGRID) grid_c = G_MAXGRID;
+  // the partial slots reuse the phi u scratch (k_gx16 has read it by now)
+  float* gpart = phiu;
   e = cudaFuncSetAttribute(k_gphi16, cudaFuncAttributeMaxDynamicSharedMemorySize, G_SMEM);
   if (e != cudaSuccess) return e;
-  k_gphi16<<<(unsigned)(N * ncb_c), G_NT, G_SMEM, s>>>(mx, mu, T, C, ncb_c, gphi, st, wl);
+  k_gphi16<<<(unsigned)grid_c, G_NT, G_SMEM, s>>>(mx, mu, T, C, ncb_c, nunits_c, gphi, gpart, st,
+                                                  wl);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t nrows = (int64_t)N * ncb_c * CB;
+  k_gphi16_fin<<<(unsigned)((nrows + 127) / 128), 128, 0, s>>>(C, ncb_c, ntt, nunits_c, grid_c,
+                                                                gpart, gphi);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return wide_bias_dispatch(part, nparts, gb, ga, ag, s);

@@ -126,7 +126,8 @@ BwdWorkspace bwd_layout(const mhc_params* p) {
   if (tc) apply_bytes = mhc::apply_tc_scratch_bytes(p->T, p->C);
   if (tc8) apply_bytes = mhc::apply8_tc_scratch_bytes();
   if (use_tc16(p))
-    apply_bytes = std::max((size_t)p->T * 16 * p->C * 4, mhc::wide_ck_bytes(p->T, p->t_max));
+    apply_bytes = std::max({(size_t)p->T * 16 * p->C * 4, mhc::wide_ck_bytes(p->T, p->t_max),
+                            mhc::apply16_gphi_part_bytes()});
   off = round_up(off + apply_bytes, 256);
   // the mapping's scratch: n = 4, its channel-split records; n = 8, its Sinkhorn
   // checkpoints

@@ -129,6 +129,8 @@ cudaError_t apply16_tc_dispatch(int64_t T, int64_t C, const void* x, const void*
                                 void* gf, float* gphi, float* gb, float* ga, int ag, int* st,
                                 int64_t wait_ns, cudaStream_t s);
 size_t apply16_urec_bytes(int64_t T);
+// the phi u scratch also holds grad_phi's partial slots: at least this many bytes
+size_t apply16_gphi_part_bytes();
 // grad_b and grad_alpha of the n = 16 paths from the mapping's partial sums
 cudaError_t wide_bias_dispatch(const float* part, int nparts, float* gb, float* ga, int ag,
                                cudaStream_t s);
