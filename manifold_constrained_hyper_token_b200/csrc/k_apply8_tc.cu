@@ -18,9 +18,9 @@
 //             operands, fp32 in TMEM, two accumulators so that one item's MMAs
 //             overlap the previous item's epilogue); the epilogue warps turn
 //             8 tokens' rows of D around in shared memory and add the CUDA-core
-//             terms from x, grad_x_next and grad_h_in, which they load with
-//             coalesced 16-byte loads (4 lanes cover one token's 64-byte row
-//             piece), so phi u never leaves the chip;
+//             terms from x, grad_x_next and grad_h_in, which they stage one
+//             step ahead with 16-byte cp.async copies (4 lanes cover one
+//             token's 64-byte row piece), so phi u never leaves the chip;
 //   k_gphi8   grad_phi for 128 rows of phi: D[128 x 192] += X^T[128 x 128] .
 //             U[128 x 192] over every token tile (tcgen05), then
 //             grad_phi = D[:, m] + D[:, 96 + m]; the (block, tile) units are
