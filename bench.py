@@ -440,16 +440,17 @@ def run_layer(args, dev, rank, world, local_rank):
     calls = (["layer_input", "post_fused"] if fused else ["pre", "post"]) + ["bwd_map", "bwd_apply"]
     # this library's kernels per call: pre = phi split + mapping + layer input;
     # bwd_map = phi split + mapping; post_fused = phi split + fused kernel;
-    # bwd_apply = one kernel at n = 4, three at n = 8 (phi u, grad_x, grad_phi);
+    # bwd_apply = one kernel at n = 4; n = 8: grad_x with phi u, bias sums,
+    # grad_phi and its finish (k_gxu8, k_bias8, k_gphi8, k_gphi8_fin);
     # n = 16: pre = phi split + projection + epilogue + layer input, bwd_map =
     # phi split + projection + reductions + epilogue
     launches_per_call = {"pre": 3, "post": 1, "layer_input": 1, "post_fused": 2, "bwd_map": 2,
-                         "bwd_apply": 1 if n == N_STR else 3}
+                         "bwd_apply": 1 if n == N_STR else 4}
     if n == 8:  # the fused post is k_post, then the phi split and the mapping; the
         # backward mapping is the phi split, the tensor-core reductions, the mapping
         launches_per_call.update({"post_fused": 3, "bwd_map": 3})
-    if n == 16:  # the apply: U rows, phi u, grad_x, grad_phi, bias sums
-        launches_per_call.update({"pre": 4, "bwd_map": 4, "post_fused": 4, "bwd_apply": 5})
+    if n == 16:  # the apply: U rows, phi u, grad_x, grad_phi and its finish, bias sums
+        launches_per_call.update({"pre": 4, "bwd_map": 4, "post_fused": 4, "bwd_apply": 6})
     # the layer's maps; in a stack the previous layer's post_fused computes them
     mhc.mhc_pre(x, phi, b, alpha, t_max=T_MAX, out=(h_in, Hpre, Hpost, Hres), stream=stream)
     nxt = (torch.empty_like(Hpre), torch.empty_like(Hpost), torch.empty_like(Hres))
