@@ -648,39 +648,32 @@ __global__ void __launch_bounds__(ap8::C_NT, 1) k_gphi8(const __grid_constant__ 
 }
 
 // grad_phi rows of the blocks that several CTAs share: the CTAs' partial
-// slots added in CTA order.  One thread per (block, row).
-__global__ void k_gphi8_fin(int64_t C, int ncb, int64_t ntt, int64_t nunits, int grid,
-                            const float* __restrict__ partial, float* __restrict__ grad_phi) {
+// slots added in CTA order.  One CTA per block (it returns at once when one CTA
+// covered the block), its threads along the rows' 16-byte pieces.
+__global__ void __launch_bounds__(256) k_gphi8_fin(int64_t C, int ncb, int64_t ntt, int64_t nunits,
+                                            int grid, const float* __restrict__ partial,
+                                            float* __restrict__ grad_phi) {
   using namespace ap8;
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // blk * CB + row
-  const int64_t blk = idx / CB;
-  const int row = (int)(idx % CB);
-  if (blk >= nunits / ntt) return;
+  const int64_t blk = blockIdx.x;
   auto owner = [&](int64_t u) { return ((u + 1) * grid - 1) / nunits; };
   const int64_t bfirst = owner(blk * ntt), blast = owner((blk + 1) * ntt - 1);
-  if (bfirst == blast) return;  // one CTA covered the block and wrote it
-  const int64_t c = (blk % ncb) * CB + row;
-  if (c >= C) return;
-  float acc[M];
-#pragma unroll
-  for (int m = 0; m < M; ++m) acc[m] = 0.0f;
-  for (int64_t b = bfirst; b <= blast; ++b) {
-    const int64_t lo_b = b * nunits / grid;
-    const int slot = lo_b / ntt == blk ? 0 : 1;
-    const float* p = partial + ((b * 2 + slot) * CB + row) * M;
-#pragma unroll
-    for (int m = 0; m < M; m += 4) {
-      const float4 v = *reinterpret_cast<const float4*>(p + m);
-      acc[m] += v.x;
-      acc[m + 1] += v.y;
-      acc[m + 2] += v.z;
-      acc[m + 3] += v.w;
+  if (bfirst == blast) return;
+  for (int e = threadIdx.x; e < CB * (M / 4); e += blockDim.x) {
+    const int row = e / (M / 4), m = 4 * (e % (M / 4));
+    const int64_t c = (blk % ncb) * CB + row;
+    if (c >= C) continue;
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int64_t b = bfirst; b <= blast; ++b) {
+      const int64_t lo_b = b * nunits / grid;
+      const int slot = lo_b / ntt == blk ? 0 : 1;
+      const float4 v = *reinterpret_cast<const float4*>(partial + ((b * 2 + slot) * CB + row) * M + m);
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
     }
+    *reinterpret_cast<float4*>(grad_phi + ((blk / ncb) * C + c) * M + m) = acc;
   }
-  float* dst = grad_phi + ((blk / ncb) * C + c) * M;
-#pragma unroll
-  for (int m = 0; m < M; m += 4)
-    *reinterpret_cast<float4*>(dst + m) = make_float4(acc[m], acc[m + 1], acc[m + 2], acc[m + 3]);
 }
 
 // ------------------------------------------------------------------ host
@@ -738,9 +731,8 @@ cudaError_t apply8_tc_dispatch(int64_t T, int64_t C, const void* x, const void* 
                                                  wl);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int64_t nrows = (int64_t)N * ncb_c * CB;
-  k_gphi8_fin<<<(unsigned)((nrows + 127) / 128), 128, 0, s>>>(C, ncb_c, ntt, nunits_c, grid_c,
-                                                               gpart, gphi);
+  k_gphi8_fin<<<(unsigned)(N * ncb_c), 256, 0, s>>>(C, ncb_c, ntt, nunits_c, grid_c, gpart,
+                                                     gphi);
   return cudaGetLastError();
 }
 
