@@ -99,6 +99,16 @@ def test_wide_tensor_core_workspaces(lib, n):
     assert 0 < lib.mhc_backward_workspace_size(ctypes.byref(f32)) < bwd
 
 
+@pytest.mark.parametrize("n,slot_floats", [(8, 128 * 80), (16, 128 * 288)])
+def test_small_problem_workspace_holds_grad_phi_slots(lib, n, slot_floats):
+    """The tensor-core apply at n = 8 and 16 splits grad_phi over up to 256
+    persistent CTAs, each with two partial slots of 128 rows; the backward
+    workspace holds them even when the problem itself is tiny."""
+    bf = _params(n=n, T=1, C=8, dtype=1)
+    bwd = lib.mhc_backward_workspace_size(ctypes.byref(bf))
+    assert bwd >= 256 * 2 * slot_floats * 4
+
+
 FAKE = ctypes.c_void_p(0x10000)   # 16-byte aligned, never dereferenced (validation fails first)
 ODD = ctypes.c_void_p(0x10004)
 
