@@ -314,7 +314,8 @@ __global__ void __launch_bounds__(128, 4) k_gx16(int64_t T, int64_t C,
       uint64_t acc[N][2];
 #pragma unroll
       for (int j = 0; j < N; ++j) {
-        const ulonglong2 p = __ldcs(reinterpret_cast<const ulonglong2*>(phiu + (t * N + j) * C + c));
+        const ulonglong2 p =
+            __ldcs(reinterpret_cast<const ulonglong2*>(phiu + (t * N + j) * C + c));
         acc[j][0] = p.x;
         acc[j][1] = p.y;
       }
@@ -565,7 +566,8 @@ __global__ void __launch_bounds__(256) k_gphi16_fin(int64_t C, int ncb, int64_t 
     for (int64_t b = bfirst; b <= blast; ++b) {
       const int64_t lo_b = b * nunits / grid;
       const int slot = lo_b / ntt == blk ? 0 : 1;
-      const float4 v = *reinterpret_cast<const float4*>(partial + ((b * 2 + slot) * CB + row) * M + m);
+      const float4 v =
+          *reinterpret_cast<const float4*>(partial + ((b * 2 + slot) * CB + row) * M + m);
       acc.x += v.x;
       acc.y += v.y;
       acc.z += v.z;

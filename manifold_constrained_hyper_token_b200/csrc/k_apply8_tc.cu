@@ -120,8 +120,8 @@ __device__ __forceinline__ void cp_async_wait1() {
 // and grad_h_in rows and H records are copied into the pair's two-slot ring
 // one step ahead (cp.async, 16 bytes per lane, 4 lanes per 64-byte row piece);
 // the 8 tokens' D rows go through the pair's transpose buffer, and the lanes
-// then work as 8 tokens x 4 groups of 8 channels.  A 64-thread named barrier orders the pair's shared
-// buffers.
+// then work as 8 tokens x 4 groups of 8 channels.  A 64-thread named barrier
+// orders the pair's shared buffers.
 __global__ void __launch_bounds__(ap8::F_NT, 1) k_gxu8(
     const __grid_constant__ CUtensorMap tm_u, const __nv_bfloat16* __restrict__ phi_t, int64_t T,
     int64_t C, int nsl, int64_t nitems, const __nv_bfloat16* __restrict__ x,
@@ -295,7 +295,8 @@ __global__ void __launch_bounds__(ap8::F_NT, 1) k_gxu8(
         const float* hsrc = coef + tb * CF::SIZE;
 #pragma unroll
         for (int k = 0; k < 3; ++k)
-          if (h_tok[k] < CK && tb + h_tok[k] < T) cp_async16(dst + (uint32_t)h_dst[k], hsrc + h_src[k]);
+          if (h_tok[k] < CK && tb + h_tok[k] < T)
+            cp_async16(dst + (uint32_t)h_dst[k], hsrc + h_src[k]);
       }
       cp_async_commit();
     };
@@ -666,7 +667,8 @@ __global__ void __launch_bounds__(256) k_gphi8_fin(int64_t C, int ncb, int64_t n
     for (int64_t b = bfirst; b <= blast; ++b) {
       const int64_t lo_b = b * nunits / grid;
       const int slot = lo_b / ntt == blk ? 0 : 1;
-      const float4 v = *reinterpret_cast<const float4*>(partial + ((b * 2 + slot) * CB + row) * M + m);
+      const float4 v =
+          *reinterpret_cast<const float4*>(partial + ((b * 2 + slot) * CB + row) * M + m);
       acc.x += v.x;
       acc.y += v.y;
       acc.z += v.z;

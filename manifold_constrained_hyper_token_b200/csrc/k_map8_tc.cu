@@ -54,14 +54,17 @@ constexpr int PBOX = NL * PROW;      // one (16-channel block, stream) phi^T til
 constexpr int NW = 10;
 constexpr int NT = NW * 32;
 constexpr uint32_t TMEM_COLS = 256;
-constexpr int NDH = 4 * N + 4 + 4;   // reductions per stream half: <G_i,x_j> 32, <G_i,f> 4, <g,x_j> 4
+// reductions per stream half: <G_i,x_j> 32, <G_i,f> 4, <g,x_j> 4 (the split
+// backward fills only the last four)
+constexpr int NDH = 4 * N + 4 + 4;
 
 template <int MODE> struct Cfg {
   static_assert(MODE == MAP_FWD || MODE == MAP_BWD_SPLIT || MODE == MAP_BWD_DOTS, "mode");
   static constexpr bool BWD = MODE == MAP_BWD_SPLIT || MODE == MAP_BWD_DOTS;
   static constexpr bool STAGE_G = MODE == MAP_BWD_SPLIT;  // grad_h_in staged
   static constexpr int X_OFF = 0;                         // x tiles of the chunk's two streams
-  static constexpr int P_OFF = SPC * XBOX;                // phi^T tiles: (16-channel step k, stream) at (2k + s)
+  // phi^T tiles: the one of 16-channel step k and stream s of the pair at 2k + s
+  static constexpr int P_OFF = SPC * XBOX;
   static constexpr int GG_OFF = P_OFF + SPC * (CH / PB) * PBOX;  // grad_h_in (split backward)
   static constexpr int STAGE = STAGE_G ? GG_OFF + XBOX : GG_OFF;
   static constexpr int NS = STAGE_G ? 2 : 3;
@@ -103,7 +106,8 @@ template <int MODE>
 __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
     const __grid_constant__ CUtensorMap tm_x, const __nv_bfloat16* __restrict__ phi_t,
     const __grid_constant__ CUtensorMap tm_g, int64_t T, int64_t C, int iters, float eps,
-    float* __restrict__ ck, const float* __restrict__ bias, const float* __restrict__ alpha_p, int ag,
+    float* __restrict__ ck, const float* __restrict__ bias, const float* __restrict__ alpha_p,
+    int ag,
     float* __restrict__ Hpre_o, float* __restrict__ Hpost_o, float* __restrict__ Hres_o,
     float* __restrict__ coef_o, __nv_bfloat16* __restrict__ urec_o, float* __restrict__ part_o,
     const float* __restrict__ red_in, int* status, uint64_t wait_ns) {
@@ -424,7 +428,8 @@ __global__ void __launch_bounds__(tcm8::NT, 1) k_map8_tc(
           float pres = 0.0f;
 #pragma unroll
           for (int j = 0; j < N; ++j) pres = fmaf(dzres[j], zt[M + 2 * N + N * i + j], pres);
-          const float dzy0 = group_sum<N>(dzpre * zt[M + i]), dzy1 = group_sum<N>(dzpost * zt[M + N + i]);
+          const float dzy0 = group_sum<N>(dzpre * zt[M + i]);
+          const float dzy1 = group_sum<N>(dzpost * zt[M + N + i]);
           const float dzy2 = group_sum<N>(pres);
           const float r = sqrtf((red_ss[tk] + red_ss[TM + tk]) / (float)K + eps);
           const float ar0 = al.a[0] / r, ar1 = al.a[1] / r, ar2 = al.a[2] / r;
@@ -554,7 +559,8 @@ cudaError_t launch_map8(const CUtensorMap& mx, const void* phi_t, const CUtensor
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<MODE>::SMEM);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)((T + TM - 1) / TM);
-  kern<<<grid, NT, Cfg<MODE>::SMEM, s>>>(mx, (const __nv_bfloat16*)phi_t, mg, T, C, iters, eps, ck, b, alpha, ag,
+  kern<<<grid, NT, Cfg<MODE>::SMEM, s>>>(mx, (const __nv_bfloat16*)phi_t, mg, T, C, iters, eps,
+                                          ck, b, alpha, ag,
                                           Hpre, Hpost, Hres, coef, (__nv_bfloat16*)urec, part,
                                           red, st, tc::wait_limit(wait_ns));
   return cudaGetLastError();

@@ -253,7 +253,8 @@ __device__ __forceinline__ void wide_dots(int64_t T, int64_t C, int64_t t0, cons
         }
         // dot 256 + tx: tx < 16 <g, x_tx>; tx >= 16 <G_(tx-16), f>
         if (tx < N) {
-          if constexpr (USE_g) dacc[i][CPT - 1] = fmaf(gq[tok * CQ + cc], xr[tx * CQP], dacc[i][CPT - 1]);
+          if constexpr (USE_g)
+            dacc[i][CPT - 1] = fmaf(gq[tok * CQ + cc], xr[tx * CQP], dacc[i][CPT - 1]);
         } else {
           if constexpr (USE_f)
             dacc[i][CPT - 1] = fmaf(Gr[(tx - N) * CQP], fq[tok * CQ + cc], dacc[i][CPT - 1]);
@@ -484,7 +485,8 @@ __global__ void __launch_bounds__(widek::NT) k_wide_map(
 // from coef, writes the coefficient record over it, and adds the CTA's dz and
 // dz . y rows in token order into part [grid][DZ_SIZE].
 template <int MODE>
-__global__ void __launch_bounds__(32) k_wide_bwd_epi_thread(int64_t T, int64_t C, int iters, float eps,
+__global__ void __launch_bounds__(32) k_wide_bwd_epi_thread(int64_t T, int64_t C, int iters,
+                                                            float eps,
                                                      const float* __restrict__ bias,
                                                      const float* __restrict__ alpha_p, int ag,
                                                      const float* __restrict__ red_in,
@@ -572,7 +574,8 @@ __global__ void __launch_bounds__(widek::EPI_NT) k_wide_bwd_epi(
     if (live) {
       float4* d = reinterpret_cast<float4*>(ckt + (int64_t)c * N * N);
 #pragma unroll
-      for (int j4 = 0; j4 < N / 4; ++j4) d[j4] = make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
+      for (int j4 = 0; j4 < N / 4; ++j4)
+        d[j4] = make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
     }
   };
   auto ck_load = [&](int c, float (&v)[N]) {
@@ -625,7 +628,8 @@ __global__ void __launch_bounds__(widek::EPI_NT) k_wide_bwd_epi(
     float* co = coef + t * CF::SIZE;
     float4* hr = reinterpret_cast<float4*>(co + CF::RES + i * N);
 #pragma unroll
-    for (int j4 = 0; j4 < N / 4; ++j4) hr[j4] = make_float4(H[4 * j4], H[4 * j4 + 1], H[4 * j4 + 2], H[4 * j4 + 3]);
+    for (int j4 = 0; j4 < N / 4; ++j4)
+      hr[j4] = make_float4(H[4 * j4], H[4 * j4 + 1], H[4 * j4 + 2], H[4 * j4 + 3]);
     co[CF::PRE + i] = spre;
     co[CF::POST + i] = 2.0f * spost;
     const float ar0 = al.a[0] / r, ar1 = al.a[1] / r, ar2 = al.a[2] / r;
@@ -697,7 +701,8 @@ __global__ void __launch_bounds__(widek::EPI_NT) k_wide_fwd_epi(
     Hpost_o[t * N + i] = 2.0f * sigmoidf_(zpost);
     float4* hr = reinterpret_cast<float4*>(Hres_o + t * N * N + i * N);
 #pragma unroll
-    for (int j4 = 0; j4 < N / 4; ++j4) hr[j4] = make_float4(a[4 * j4], a[4 * j4 + 1], a[4 * j4 + 2], a[4 * j4 + 3]);
+    for (int j4 = 0; j4 < N / 4; ++j4)
+      hr[j4] = make_float4(a[4 * j4], a[4 * j4 + 1], a[4 * j4 + 2], a[4 * j4 + 3]);
   }
 }
 
@@ -1038,7 +1043,8 @@ static cudaError_t launch_wide_map(int64_t T, int64_t C, int iters, float eps, c
                                    float* part, int* st, cudaStream_t s) {
   const size_t smem = (size_t)widek::SMEM_FLOATS * 4;
   auto kern = k_wide_map<TIO, MODE>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int64_t grid = (T + widek::TB - 1) / widek::TB;
   kern<<<(unsigned)grid, widek::NT, smem, s>>>(T, C, iters, eps, (const TIO*)x, phi, b, alpha, ag,

@@ -60,8 +60,8 @@ size_t map_tc_scratch_bytes(int64_t T, int64_t C);
 // phi [K][24] fp32 -> the bf16 split copy of phi^T [48][K] the mapping MMAs read
 cudaError_t phi_split_dispatch(int64_t K, const float* phi, void* phi_split, cudaStream_t s);
 // k_map8_tc.cu (bf16, n = 8: projection on the tensor cores); mode is MAP_FWD,
-// MAP_BWD_SPLIT or MAP_BWD_DOTS (G and f are not read).  Splits phi into phi_split (map8_tc_phi_bytes(C)
-// bytes); the backward modes write the per-token records (coef
+// MAP_BWD_SPLIT or MAP_BWD_DOTS (G and f are not read).  Splits phi into
+// phi_split (map8_tc_phi_bytes(C) bytes); the backward modes write the per-token records (coef
 // [T][Coef<8>::SIZE]), the U rows (urec [T][TcRec8::U_ELEMS] bf16) and one
 // partial-sum record per 128 tokens (part); the backward modes keep Sinkhorn
 // checkpoints in ck (map8_ck_bytes(T, iters) bytes; unused forward).
