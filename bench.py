@@ -48,8 +48,16 @@ sys.path.insert(0, ROOT)
 
 METRIC = "mHC layer tokens/s (fwd+bwd, n=4, C=7168) and achieved HBM GB/s vs B200 peak"
 T_TOK, N_STR, C_CH, T_MAX = 16384, 4, 7168, 20
+SINKHORN_METRIC = ("batched Sinkhorn-Knopp matrices/s (2^22 matrices each for n=4,8,16, "
+                   "20 iterations)")
+DEPTH_METRIC = "mHC depth-stack tokens/s (24 layers fwd+bwd with recompute, n=4, C=7168)"
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e, the spec figure
+
+
+def layer_metric(n: int) -> str:
+    """The layer line's metric for n streams."""
+    return METRIC if n == N_STR else METRIC.replace("n=4", f"n={n}")
 
 
 def per_token_bytes(n=N_STR, C=C_CH, act=2):
@@ -172,19 +180,25 @@ class ClockSampler:
         return {"sm_mhz": med, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def cpu_reference(seconds: float, seed: int = 0):
-    """The fp64 oracle, as it stands, on the first S tokens of the same workload:
-    pre + post + backward.  S is grown until one pass takes about `seconds`."""
+def oracle_layer_pass(n: int = N_STR, seed: int = 0, pool: int = 0):
+    """One timed pass of the fp64 oracle over the layer: pre + post + backward on
+    the first S tokens of the seeded workload with n streams.  Returns
+    run(S) -> seconds (the inputs are drawn before the clock starts).  With
+    pool > 0 the tokens come from one pool of that many, drawn once."""
     import torch
 
     import oracle
     from manifold_constrained_hyper_token_b200 import synth
 
-    params = synth.layer_params(N_STR, C_CH, seed)
+    params = synth.layer_params(n, C_CH, seed)
     alpha = float(params["alpha"][0])
+    held = synth.activations(pool, n, C_CH, seed, torch.bfloat16, backward=True) if pool else None
 
     def run(S):
-        d = synth.activations(S, N_STR, C_CH, seed, torch.bfloat16, backward=True)
+        if held is not None:
+            d = {k: v[:S] for k, v in held.items()}
+        else:
+            d = synth.activations(S, n, C_CH, seed, torch.bfloat16, backward=True)
         t0 = time.perf_counter()
         o = oracle.pre(d["x"], params["phi"], params["b"], alpha, iters=T_MAX)
         oracle.post(d["x"], d["f_out"], o["H_post"], o["H_res"])
@@ -192,24 +206,57 @@ def cpu_reference(seconds: float, seed: int = 0):
                         d["grad_h_in"], iters=T_MAX)
         return time.perf_counter() - t0
 
-    S = 32
-    dt = run(S)
-    while dt < seconds / 4 and S < 8192:
-        S = min(8192, int(S * max(2.0, min(8.0, seconds / max(dt, 1e-3) / 2))))
-        dt = run(S)
-    cores = oracle.num_threads()
-    # the plain cost: one host thread on a smaller sample of the same tokens
-    oracle.set_num_threads(1)
-    try:
-        S1 = 64
-        dt1 = run(S1)
-    finally:
-        oracle.set_num_threads(cores)
-    return {"value": S / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"first {S} tokens of the T={T_TOK}, n={N_STR}, C={C_CH} bf16 workload, "
-                      f"pre+post+backward in fp64, {dt:.2f} s",
-            "single_thread": {"value": S1 / dt1, "unit": "tokens/s", "cores": 1,
-                              "sample": f"first {S1} tokens, {dt1:.2f} s"}}
+    return run
+
+
+def oracle_sinkhorn_pass():
+    """One timed pass of the fp64 oracle's batched Sinkhorn on the first S
+    matrices of each n's seeded batch (n = 4, 8, 16; 20 iterations): run(S) ->
+    seconds for 3 S matrices."""
+    import oracle
+    from manifold_constrained_hyper_token_b200 import synth
+
+    def run(S):
+        lg = [synth.sinkhorn_logits(S, n, seed=100 + n) for n in (4, 8, 16)]
+        t0 = time.perf_counter()
+        for x in lg:
+            oracle.sinkhorn(x, T_MAX)
+        return time.perf_counter() - t0
+
+    return run
+
+
+def oracle_depth_pass(L: int = 24):
+    """One timed pass of the fp64 oracle through the L-layer stack (F_l(h) = s_l
+    h) on the first S tokens of chunk 0: forward, then each layer's backward
+    with grad_h_in = s_l grad_f_out, last layer first.  run(S) -> seconds."""
+    import numpy as np
+    import oracle
+    from manifold_constrained_hyper_token_b200 import synth
+
+    prms = [synth.layer_params(N_STR, C_CH, seed=l) for l in range(L)]
+    gains = [synth.depth_gain(l) for l in range(L)]
+
+    def run(S):
+        d = synth.depth_stack_chunk(S, N_STR, C_CH, chunk=0)
+        t0 = time.perf_counter()
+        xs, fs = [d["x0"]], []
+        for l in range(L):
+            a = float(prms[l]["alpha"][0])
+            r = oracle.pre(xs[l], prms[l]["phi"], prms[l]["b"], a, iters=T_MAX)
+            fs.append(gains[l] * r["h_in"])
+            xs.append(oracle.post(xs[l], fs[l], r["H_post"], r["H_res"]))
+        G = d["G_last"]
+        for l in reversed(range(L)):
+            a = float(prms[l]["alpha"][0])
+            zero = np.zeros((S, C_CH))
+            gf = oracle.backward(xs[l], prms[l]["phi"], prms[l]["b"], a, fs[l], G, zero,
+                                 iters=T_MAX)["grad_f_out"]
+            G = oracle.backward(xs[l], prms[l]["phi"], prms[l]["b"], a, fs[l], G, gains[l] * gf,
+                                iters=T_MAX)["grad_x"]
+        return time.perf_counter() - t0
+
+    return run
 
 
 def _grow(run, seconds, start, cap):
@@ -237,20 +284,23 @@ def _both_thread_counts(run, seconds, start, cap, small):
     return S, dt, cores, small, dt1
 
 
+def cpu_reference(seconds: float, seed: int = 0):
+    """The fp64 oracle, as it stands, on the first S tokens of the layer workload:
+    pre + post + backward.  S is grown until one pass takes about `seconds`."""
+    S, dt, cores, S1, dt1 = _both_thread_counts(oracle_layer_pass(N_STR, seed), seconds, 32,
+                                                8192, 64)
+    return {"value": S / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {S} tokens of the T={T_TOK}, n={N_STR}, C={C_CH} bf16 workload, "
+                      f"pre+post+backward in fp64, {dt:.2f} s",
+            "single_thread": {"value": S1 / dt1, "unit": "tokens/s", "cores": 1,
+                              "sample": f"first {S1} tokens, {dt1:.2f} s"}}
+
+
 def cpu_sinkhorn(seconds: float):
     """The fp64 oracle's batched Sinkhorn on the first S matrices of each n's batch
     (n = 4, 8, 16; the same seeded logits; 20 iterations): matrices/s."""
-    import oracle
-    from manifold_constrained_hyper_token_b200 import synth
-
-    def run(S):
-        lg = [synth.sinkhorn_logits(S, n, seed=100 + n) for n in (4, 8, 16)]
-        t0 = time.perf_counter()
-        for x in lg:
-            oracle.sinkhorn(x, T_MAX)
-        return time.perf_counter() - t0
-
-    S, dt, cores, S1, dt1 = _both_thread_counts(run, seconds, 1024, 1 << 22, 16384)
+    S, dt, cores, S1, dt1 = _both_thread_counts(oracle_sinkhorn_pass(), seconds, 1024, 1 << 22,
+                                                16384)
     return {"value": 3 * S / dt, "unit": "matrices/s", "cores": cores, "kind": "oracle",
             "sample": f"first {S} matrices of each of the n=4, 8, 16 batches, 20 iterations "
                       f"in fp64, {dt:.2f} s",
@@ -259,36 +309,9 @@ def cpu_sinkhorn(seconds: float):
 
 
 def cpu_depth(seconds: float, L: int = 24):
-    """The fp64 oracle through the L-layer stack (F_l(h) = s_l h) on the first S
-    tokens of chunk 0: forward, then each layer's backward with grad_h_in =
-    s_l grad_f_out, last layer first: tokens/s."""
-    import numpy as np
-    import oracle
-    from manifold_constrained_hyper_token_b200 import synth
-
-    prms = [synth.layer_params(N_STR, C_CH, seed=l) for l in range(L)]
-    gains = [synth.depth_gain(l) for l in range(L)]
-
-    def run(S):
-        d = synth.depth_stack_chunk(S, N_STR, C_CH, chunk=0)
-        t0 = time.perf_counter()
-        xs, fs = [d["x0"]], []
-        for l in range(L):
-            a = float(prms[l]["alpha"][0])
-            r = oracle.pre(xs[l], prms[l]["phi"], prms[l]["b"], a, iters=T_MAX)
-            fs.append(gains[l] * r["h_in"])
-            xs.append(oracle.post(xs[l], fs[l], r["H_post"], r["H_res"]))
-        G = d["G_last"]
-        for l in reversed(range(L)):
-            a = float(prms[l]["alpha"][0])
-            zero = np.zeros((S, C_CH))
-            gf = oracle.backward(xs[l], prms[l]["phi"], prms[l]["b"], a, fs[l], G, zero,
-                                 iters=T_MAX)["grad_f_out"]
-            G = oracle.backward(xs[l], prms[l]["phi"], prms[l]["b"], a, fs[l], G, gains[l] * gf,
-                                iters=T_MAX)["grad_x"]
-        return time.perf_counter() - t0
-
-    S, dt, cores, S1, dt1 = _both_thread_counts(run, seconds, 4, 4096, 8)
+    """The fp64 oracle through the L-layer stack on the first S tokens of chunk 0,
+    forward and backward: tokens/s."""
+    S, dt, cores, S1, dt1 = _both_thread_counts(oracle_depth_pass(L), seconds, 4, 4096, 8)
     return {"value": S / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": f"first {S} tokens of the stack input, {L} layers forward and backward "
                       f"(the per-layer backward run twice: grad_f_out, then grad_x) in fp64, "
@@ -297,53 +320,74 @@ def cpu_depth(seconds: float, L: int = 24):
                               "sample": f"first {S1} tokens, {dt1:.2f} s"}}
 
 
+def _reference_sample(run, start, cap, warmup, steps, budget_s):
+    """Reference-arm sample size: one calibration pass of at least one unit per
+    host thread (the oracle spreads tokens or matrices over its threads), then
+    the S (at most `cap`) for which the warm-up and timed passes together take
+    about budget_s.  Returns S, the seconds of the `steps` timed passes and the
+    threads the oracle kept busy."""
+    import oracle
+    threads = oracle.num_threads()
+    start = min(cap, max(start, threads))
+    rate = start / run(start)
+    S = int(max(start, min(cap, budget_s * rate / (warmup + steps))))
+    for _ in range(warmup):
+        run(S)
+    return S, sum(run(S) for _ in range(steps)), min(S, threads)
+
+
 def run_reference(args, rank, world):
-    """Reference arm: the fp64 oracle on the host cores.  Each step runs
-    pre + post + backward on a bounded sample of S tokens of the same
-    workload; S is chosen from a short calibration so that the whole
-    W + K step run takes about two minutes."""
+    """Reference arm: the fp64 oracle on the host cores, for the workload the
+    arguments name (the layer with --streams n, the batched Sinkhorn, or the
+    depth stack), with that arm's metric and unit.  Each step runs the oracle
+    on a bounded sample of S units of the workload; S comes from a short
+    calibration so that the W + K steps take about --reference-seconds."""
     if rank != 0:
         return
-    import torch
-
-    import oracle
-    from manifold_constrained_hyper_token_b200 import synth
-
-    params = synth.layer_params(N_STR, C_CH, 0)
-    alpha = float(params["alpha"][0])
-    pool = synth.activations(256, N_STR, C_CH, 0, torch.bfloat16, backward=True)
-
-    def one(S):
-        d = {k: v[:S] for k, v in pool.items()}
-        t0 = time.perf_counter()
-        o = oracle.pre(d["x"], params["phi"], params["b"], alpha, iters=T_MAX)
-        oracle.post(d["x"], d["f_out"], o["H_post"], o["H_res"])
-        oracle.backward(d["x"], params["phi"], params["b"], alpha, d["f_out"], d["grad_x_next"],
-                        d["grad_h_in"], iters=T_MAX)
-        return time.perf_counter() - t0
-
-    rate = 32 / one(32)
-    S = int(max(1, min(256, 120.0 * rate / (args.warmup + args.steps))))
-    for _ in range(args.warmup):
-        one(S)
-    total = sum(one(S) for _ in range(args.steps))
-    val = args.steps * S / total
-    cb = {"value": val, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
-          "sample": f"{S} tokens per step of the T={T_TOK}, n={N_STR}, C={C_CH} bf16 workload, "
-                    f"pre+post+backward in fp64"}
-    # a step here is the S-token sample the oracle ran, and ms_per_step its measured time
-    line = {"metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": 1000.0 * total / args.steps,
-            "higher_is_better": True,
+    W, K, budget = args.warmup, args.steps, args.reference_seconds
+    if args.workload == "sinkhorn":
+        S, total, cores = _reference_sample(oracle_sinkhorn_pass(), 1024, 1 << 22, W, K,
+                                            budget)
+        metric, unit, units = SINKHORN_METRIC, "matrices/s", 3 * S
+        sample = (f"first {S} matrices of each of the n=4, 8, 16 batches per step, 20 "
+                  f"iterations in fp64")
+        cfg = {"workload": f"standalone Sinkhorn-Knopp, oracle on the first {S} matrices per n "
+                           f"of the 2^22-matrix batches (n in {{4, 8, 16}}, logits N(0, 2), "
+                           f"{T_MAX} iterations) per step",
+               "matrices_per_step": units, "B_sampled_from": 1 << 22, "t_max": T_MAX}
+    elif args.workload == "depth":
+        L = 24
+        T = args.tokens if args.tokens != T_TOK else 65536
+        S, total, cores = _reference_sample(oracle_depth_pass(L), 4, 4096, W, K, budget)
+        metric, unit, units = DEPTH_METRIC, "tokens/s", S
+        sample = (f"first {S} tokens of the stack input per step, {L} layers forward and "
+                  f"backward in fp64")
+        cfg = {"workload": f"depth stack, oracle on the first {S} tokens of the L={L}, "
+                           f"T={T}, n={N_STR}, C={C_CH}, F_l(h)=s_l h workload per step",
+               "tokens_per_step": S, "T_sampled_from": T, "L": L, "n": N_STR, "C": C_CH,
+               "t_max": T_MAX}
+    else:
+        n = args.streams
+        S, total, cores = _reference_sample(oracle_layer_pass(n, 0, pool=256), 32, 256, W, K,
+                                            budget)
+        metric, unit, units = layer_metric(n), "tokens/s", S
+        sample = (f"{S} tokens per step of the T={args.tokens}, n={n}, C={C_CH} bf16 "
+                  f"workload, pre+post+backward in fp64")
+        cfg = {"workload": f"mHC layer fwd+bwd, oracle on a sample of S={S} tokens per step "
+                           f"drawn from the T={args.tokens}, n={n}, C={C_CH}, t_max={T_MAX} "
+                           f"bf16 workload",
+               "tokens_per_step": S, "T_sampled_from": args.tokens, "n": n, "C": C_CH,
+               "t_max": T_MAX}
+    cfg["parallelism"] = "host cores (oracle)"
+    val = K * units / total
+    # a step here is the sample the oracle ran, and ms_per_step its measured time
+    line = {"metric": metric, "value": val, "unit": unit, "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": 1000.0 * total / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "impl": "reference",
-            "config": {"workload": f"mHC layer fwd+bwd, oracle on a sample of S={S} tokens per "
-                                   f"step drawn from the T={T_TOK}, n={N_STR}, C={C_CH}, "
-                                   f"t_max={T_MAX} bf16 workload",
-                       "tokens_per_step": S, "T_sampled_from": T_TOK, "n": N_STR, "C": C_CH,
-                       "t_max": T_MAX, "parallelism": "host cores (oracle)"},
-            "cpu_baseline": cb,
-            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+            "impl": "reference", "config": cfg,
+            "cpu_baseline": {"value": val, "unit": unit, "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -355,6 +399,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-sample-seconds", type=float, default=12.0)
+    ap.add_argument("--reference-seconds", type=float, default=120.0,
+                    help="--impl reference: host seconds for the warm-up and timed steps together")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--tokens", type=int, default=T_TOK,
@@ -573,7 +619,7 @@ def run_layer(args, dev, rank, world, local_rank):
 
     if rank == 0:
         line = {
-            "metric": METRIC if n == N_STR else METRIC.replace("n=4", f"n={n}"),
+            "metric": layer_metric(n),
             "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -682,8 +728,7 @@ def run_sinkhorn(args, dev, rank, world, local_rank):
         d = per_n[dom]
         bound = "hbm" if d["hbm_frac"] >= d["alu_frac"] else "alu"
         line = {
-            "metric": "batched Sinkhorn-Knopp matrices/s (2^22 matrices each for n=4,8,16, "
-                      "20 iterations)",
+            "metric": SINKHORN_METRIC,
             "value": total_mat * world / (total_ms / 1e3), "unit": "matrices/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": total_ms, "higher_is_better": True, "scaling": "weak",
@@ -756,7 +801,7 @@ def run_depth(args, dev, rank, world, local_rank):
     gbs = alg / (t / 1e3) / 1e9
     if rank == 0:
         line = {
-            "metric": "mHC depth-stack tokens/s (24 layers fwd+bwd with recompute, n=4, C=7168)",
+            "metric": DEPTH_METRIC,
             "value": T * world / (t / 1e3), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
