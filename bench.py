@@ -70,9 +70,12 @@ def per_token_bytes(n=N_STR, C=C_CH, act=2):
         "post": nC * act + C * act + 4 * (n + n * n) + nC * act,           # x, f, H in; x_next out
         "layer_input": nC * act + C * act + 4 * n,                         # x, H_pre in; h_in out
         "post_fused": nC * act + C * act + 4 * (n + n * n) + nC * act + 4 * (2 * n + n * n),
-        "bwd_map": 2 * nC * act + 2 * C * act + coef,                      # x, G, g, f in; records out
-        "bwd_apply": 2 * nC * act + C * act + coef + nC * act + C * act,   # x, G, g, records in; grads out
-        "bwd_min": 2 * nC * act + 2 * C * act + nC * act + C * act,        # one pass: x, G, g, f in; grads out
+        # x, G, g, f in; records out
+        "bwd_map": 2 * nC * act + 2 * C * act + coef,
+        # x, G, g, records in; grads out
+        "bwd_apply": 2 * nC * act + C * act + coef + nC * act + C * act,
+        # one pass: x, G, g, f in; grads out
+        "bwd_min": 2 * nC * act + 2 * C * act + nC * act + C * act,
     }
 
 
@@ -96,7 +99,8 @@ def load_peaks():
 def kernel_source_sha(files):
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "manifold_constrained_hyper_token_b200", "csrc", f), "rb") as fh:
+        path = os.path.join(ROOT, "manifold_constrained_hyper_token_b200", "csrc", f)
+        with open(path, "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
@@ -632,8 +636,8 @@ def run_layer(args, dev, rank, world, local_rank):
                        "forward": args.forward,
                        "T_per_gpu": T, "n": n, "C": C, "t_max": T_MAX,
                        "parallelism": f"dp{world} over tokens",
-                       "l2": f"inputs larger than L2 (x and grad_x_next are {T * n * C * 2 / 1e6:.0f} "
-                             "MB each); no flush"},
+                       "l2": f"inputs larger than L2 (x and grad_x_next are "
+                             f"{T * n * C * 2 / 1e6:.0f} MB each); no flush"},
             "hbm": {"achieved_gbs": step_gbs, "peak_gbs": peak, "frac": step_gbs / peak,
                     "peak_kind": peak_kind, "frac_vs_nominal": step_gbs / NOMINAL_HBM_GBS,
                     "alg_bytes_per_step": step_alg_bytes},
@@ -700,7 +704,8 @@ def run_sinkhorn(args, dev, rank, world, local_rank):
         byts = B * 8 * n * n
         ops = B * sinkhorn_ops(n, iters)
         per_n[str(n)] = {"ms": t, "matrices_per_s": B * world / (t / 1e3),
-                         "hbm_gbs": byts / (t / 1e3) / 1e9, "hbm_frac": byts / (t / 1e3) / 1e9 / peak,
+                         "hbm_gbs": byts / (t / 1e3) / 1e9,
+                         "hbm_frac": byts / (t / 1e3) / 1e9 / peak,
                          "gops": ops / (t / 1e3) / 1e9, "step_ms": step_stats(ms)}
         total_ms += t
         total_mat += B

@@ -159,8 +159,9 @@ MHC_API mhc_status mhc_pre(const mhc_params *p, const void *x, const float *phi,
  *        x_next[i][c] = sum_j H_res[i][j] x[j][c] + H_post[i] f_out[c]
  * x_next must not alias x or f_out.
  */
-MHC_API mhc_status mhc_post(const mhc_params *p, const void *x, const void *f_out, const float *H_post,
-                    const float *H_res, void *x_next, int *dev_status, mhc_stream_t stream);
+MHC_API mhc_status mhc_post(const mhc_params *p, const void *x, const void *f_out,
+                            const float *H_post, const float *H_res, void *x_next,
+                            int *dev_status, mhc_stream_t stream);
 
 /* Bytes of workspace mhc_backward needs for these params. */
 MHC_API size_t mhc_backward_workspace_size(const mhc_params *p);
@@ -183,11 +184,12 @@ MHC_API size_t mhc_backward_workspace_size(const mhc_params *p);
  * bits.  workspace: at least mhc_backward_workspace_size(p) bytes, 256-byte
  * aligned; its contents on entry do not matter.
  */
-MHC_API mhc_status mhc_backward(const mhc_params *p, const void *x, const float *phi, const float *b,
-                        const float *alpha, const void *f_out, const void *grad_x_next,
-                        const void *grad_h_in, void *grad_x, float *grad_phi, float *grad_b,
-                        float *grad_alpha, void *grad_f_out, void *workspace,
-                        size_t workspace_bytes, int *dev_status, mhc_stream_t stream);
+MHC_API mhc_status mhc_backward(const mhc_params *p, const void *x, const float *phi,
+                                const float *b, const float *alpha, const void *f_out,
+                                const void *grad_x_next, const void *grad_h_in, void *grad_x,
+                                float *grad_phi, float *grad_b, float *grad_alpha,
+                                void *grad_f_out, void *workspace, size_t workspace_bytes,
+                                int *dev_status, mhc_stream_t stream);
 
 /*
  * mhc_backward_map / mhc_backward_apply -- the two phases mhc_backward runs,
@@ -303,21 +305,21 @@ MHC_API mhc_status mhc_pre_backward(const mhc_params *p, const void *x, const fl
  * method.
  *
  * Arguments, layouts, results and errors are those of mhc_backward, minus
- * the workspace, and n = 16 is not taken (MHC_ERR_UNSUPPORTED).  The scratch is a library-owned device array of
- * MHC_NOALLOC_SCRATCH_BYTES that every GPU loading this library holds until
- * the process exits.  The call runs the CUDA-core kernels, whose scratch is
- * a per-token record (n = 4: 208 bytes) and a partial sum per 64 tokens; a
- * problem whose scratch exceeds MHC_NOALLOC_SCRATCH_BYTES is rejected with
- * MHC_ERR_WORKSPACE before any launch (n = 4: up to about 20,000 tokens per
- * call).  Every call looks up the array's device address
- * (cudaGetSymbolAddress) on the current device; nothing is cached, so calls
- * made after a device reset use the array of the new context.  The first call
- * on a device may load the module: make it before any stream capture.
- * All calls share the one array and it keeps the last call's
- * contents (nothing in it needs to start at zero): calls whose work can
- * overlap on the GPU (on different streams, or from several threads without
- * ordering) race on it and must be serialised by the caller.  Allocates
- * nothing: no cudaMalloc, cudaFree or allocating library routine.
+ * the workspace, and n = 16 is not taken (MHC_ERR_UNSUPPORTED).  The scratch
+ * is a library-owned device array of MHC_NOALLOC_SCRATCH_BYTES that every
+ * GPU loading this library holds until the process exits.  The call runs the
+ * CUDA-core kernels, whose scratch is a per-token record (n = 4: 208 bytes)
+ * and a partial sum per 64 tokens; a problem whose scratch exceeds
+ * MHC_NOALLOC_SCRATCH_BYTES is rejected with MHC_ERR_WORKSPACE before any
+ * launch (n = 4: up to about 20,000 tokens per call).  Every call looks up
+ * the array's device address (cudaGetSymbolAddress) on the current device;
+ * nothing is cached, so calls made after a device reset use the array of the
+ * new context.  The first call on a device may load the module: make it
+ * before any stream capture.  All calls share the one array and it keeps the
+ * last call's contents (nothing in it needs to start at zero): calls whose
+ * work can overlap on the GPU (on different streams, or from several threads
+ * without ordering) race on it and must be serialised by the caller.
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
  */
 #define MHC_NOALLOC_SCRATCH_BYTES (4u * 1024u * 1024u)
 MHC_API mhc_status mhc_backward_noalloc(const mhc_params *p, const void *x, const float *phi,
