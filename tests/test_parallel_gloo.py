@@ -17,7 +17,7 @@ def _free_port() -> int:
         return s.getsockname()[1]
 
 
-def _worker(rank, world, port, result_dir, alpha):
+def _worker(rank, world, port, result_dir, alpha, n):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     import datetime
@@ -28,7 +28,7 @@ def _worker(rank, world, port, result_dir, alpha):
     from manifold_constrained_hyper_token_b200 import parallel, synth
     dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=60))
-    T, n, C = 37, 4, 16
+    T, C = 37, 16
     d = synth.layer_inputs(T, n, C, seed=3, dtype=torch.float32, backward=True)
     lo, hi = parallel.token_shard(T, rank, world)
     r = oracle.backward(d["x"][lo:hi], d["phi"], d["b"], alpha, d["f_out"][lo:hi],
@@ -58,22 +58,26 @@ def test_token_shard_covers_all_tokens():
             assert max(sizes) - min(sizes) <= 1
 
 
-@pytest.mark.parametrize("alpha", [[0.3], [0.3, -0.2, 0.5]], ids=["shared_alpha", "alpha_groups3"])
-def test_two_rank_backward_matches_single(tmp_path, alpha):
+@pytest.mark.parametrize("n,alpha", [(4, [0.3]), (4, [0.3, -0.2, 0.5]), (8, [0.3, -0.2, 0.5]),
+                                     (16, [0.3])],
+                         ids=["n4_shared_alpha", "n4_alpha_groups3", "n8_alpha_groups3",
+                              "n16_shared_alpha"])
+def test_two_rank_backward_matches_single(tmp_path, n, alpha):
     import oracle
     from manifold_constrained_hyper_token_b200 import synth
     oracle.build()
     world = 2
-    mp.start_processes(_worker, args=(world, _free_port(), str(tmp_path), alpha), nprocs=world,
-                       join=True, start_method="spawn")
-    T, n, C = 37, 4, 16
+    mp.start_processes(_worker, args=(world, _free_port(), str(tmp_path), alpha, n),
+                       nprocs=world, join=True, start_method="spawn")
+    T, C = 37, 16
     d = synth.layer_inputs(T, n, C, seed=3, dtype=torch.float32, backward=True)
     full = oracle.backward(d["x"], d["phi"], d["b"], alpha, d["f_out"], d["grad_x_next"],
                            d["grad_h_in"], iters=20)
     K, M = n * C, n * n + 2 * n
     flats = [np.load(tmp_path / f"flat{r}.npy") for r in range(world)]
     np.testing.assert_array_equal(flats[0], flats[1])  # every rank holds the same sum
-    np.testing.assert_allclose(flats[0][:K * M].reshape(K, M), full["grad_phi"], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(flats[0][:K * M].reshape(K, M), full["grad_phi"], rtol=1e-12,
+                               atol=1e-12)
     np.testing.assert_allclose(flats[0][K * M:K * M + M], full["grad_b"], rtol=1e-12, atol=1e-12)
     na = len(alpha)
     assert flats[0].size == K * M + M + na  # the buffer holds one grad_alpha per group
