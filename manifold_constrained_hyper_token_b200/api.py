@@ -5,7 +5,11 @@ arguments: tensors become device pointers, shapes become an ``mhc_params``,
 the stream is the current torch stream unless one is given.  Output tensors
 are allocated with torch when the caller does not pass them.  Every step of
 the computation runs in the library's CUDA kernels; a non-zero status raises
-``MhcError``.  Tensors must be contiguous CUDA tensors.
+``MhcError``.  Tensors must be contiguous CUDA tensors on x's device.  Before
+any launch every tensor is checked against the problem's sizes: the element
+type the call reads or writes, and at least as many elements as it touches, so
+that a mis-sized argument raises ValueError here instead of sending a kernel
+past the end of an allocation.
 """
 from __future__ import annotations
 
@@ -16,6 +20,7 @@ import torch
 from . import _lib
 
 DTYPE_CODE = {torch.float32: 0, torch.bfloat16: 1}
+F32 = torch.float32
 
 
 class MhcError(RuntimeError):
@@ -47,6 +52,59 @@ def _p(t):
     if not t.is_contiguous():
         raise ValueError("libmhc takes contiguous tensors only")
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _fits(t, numel, dtype, device, what):
+    """Reject a tensor that the call would reinterpret (another element type),
+    run past the end of (fewer elements than it reads or writes) or reach on
+    another device.  None passes: the library rejects a missing required
+    pointer itself."""
+    if t is None:
+        return
+    if t.dtype != dtype:
+        raise ValueError(f"{what}: dtype {t.dtype}, the call takes {dtype}")
+    if t.numel() < numel:
+        raise ValueError(f"{what}: {t.numel()} elements, the call touches {numel}")
+    if t.device != device:
+        raise ValueError(f"{what}: on {t.device}, the call runs on {device}")
+
+
+def _on(t, device, what):
+    """A workspace (any element type; the library checks its byte count) on the
+    call's device."""
+    if t is not None and t.device != device:
+        raise ValueError(f"{what}: on {t.device}, the call runs on {device}")
+
+
+def _maps_in(x, phi, b, alpha):
+    """phi [nC, n^2+2n], b [n^2+2n], alpha [1] or [3]: fp32 on x's device."""
+    T, n, C = x.shape
+    M = n * n + 2 * n
+    _fits(phi, n * C * M, F32, x.device, "phi")
+    _fits(b, M, F32, x.device, "b")
+    _fits(alpha, 1, F32, x.device, "alpha")
+
+
+def _upstream(x, f_out, grad_x_next, grad_h_in):
+    """The backward's activations: f_out and grad_h_in [T, C], grad_x_next
+    [T, n, C], all of x's dtype (f_out may be None where the call takes none)."""
+    T, n, C = x.shape
+    _fits(f_out, T * C, x.dtype, x.device, "f_out")
+    _fits(grad_x_next, T * n * C, x.dtype, x.device, "grad_x_next")
+    _fits(grad_h_in, T * C, x.dtype, x.device, "grad_h_in")
+
+
+def _grads_out(x, ag, gx, gphi, gb, ga, gf):
+    """The backward's outputs: grad_x [T, n, C] and grad_f_out [T, C] of x's
+    dtype; grad_phi, grad_b and grad_alpha (3 entries with per-group alpha)
+    fp32."""
+    T, n, C = x.shape
+    M = n * n + 2 * n
+    _fits(gx, T * n * C, x.dtype, x.device, "grad_x")
+    _fits(gphi, n * C * M, F32, x.device, "grad_phi")
+    _fits(gb, M, F32, x.device, "grad_b")
+    _fits(ga, 3 if ag == 3 else 1, F32, x.device, "grad_alpha")
+    _fits(gf, T * C, x.dtype, x.device, "grad_f_out")
 
 
 def _stream(stream):
@@ -101,6 +159,13 @@ def mhc_pre(x, phi, b, alpha, *, t_max: int = 20, eps: float = 1e-6, wait_ns: in
                torch.empty(T, n, dtype=torch.float32, device=x.device),
                torch.empty(T, n, n, dtype=torch.float32, device=x.device))
     h_in, H_pre, H_post, H_res = out
+    _maps_in(x, phi, b, alpha)
+    _fits(h_in, T * C, x.dtype, x.device, "h_in")
+    _fits(H_pre, T * n, F32, x.device, "H_pre")
+    _fits(H_post, T * n, F32, x.device, "H_post")
+    _fits(H_res, T * n * n, F32, x.device, "H_res")
+    _fits(dev_status, 1, torch.int32, x.device, "dev_status")
+    _on(workspace, x.device, "workspace")
     lib = _lib.load()
     ws, wsb = _workspace(int(lib.mhc_pre_workspace_size(ctypes.byref(p))), x.device, workspace)
     st = lib.mhc_pre(ctypes.byref(p), _p(x), _p(phi), _p(b), _p(alpha), _p(h_in), _p(H_pre),
@@ -114,6 +179,11 @@ def mhc_post(x, f_out, H_post, H_res, *, out=None, dev_status=None, stream=None)
     T, n, C = x.shape
     p = params(n, T, C, x.dtype)
     x_next = torch.empty_like(x) if out is None else out
+    _fits(f_out, T * C, x.dtype, x.device, "f_out")
+    _fits(H_post, T * n, F32, x.device, "H_post")
+    _fits(H_res, T * n * n, F32, x.device, "H_res")
+    _fits(x_next, T * n * C, x.dtype, x.device, "x_next")
+    _fits(dev_status, 1, torch.int32, x.device, "dev_status")
     st = _lib.load().mhc_post(ctypes.byref(p), _p(x), _p(f_out), _p(H_post), _p(H_res),
                               _p(x_next), _p(dev_status), _stream(stream))
     _check(st, "mhc_post")
@@ -131,6 +201,11 @@ def mhc_backward(x, phi, b, alpha, f_out, grad_x_next, grad_h_in, *, t_max: int 
         out = (torch.empty_like(x), torch.empty_like(phi), torch.empty_like(b),
                torch.empty_like(alpha), torch.empty_like(f_out))
     gx, gphi, gb, ga, gf = out
+    _maps_in(x, phi, b, alpha)
+    _upstream(x, f_out, grad_x_next, grad_h_in)
+    _grads_out(x, _ag(alpha), gx, gphi, gb, ga, gf)
+    _fits(dev_status, 1, torch.int32, x.device, "dev_status")
+    _on(workspace, x.device, "workspace")
     lib = _lib.load()
     ws, wsb = _workspace(int(lib.mhc_backward_workspace_size(ctypes.byref(p))), x.device,
                          workspace)
@@ -154,6 +229,10 @@ def mhc_backward_noalloc(x, phi, b, alpha, f_out, grad_x_next, grad_h_in, *, t_m
         out = (torch.empty_like(x), torch.empty_like(phi), torch.empty_like(b),
                torch.empty_like(alpha), torch.empty_like(f_out))
     gx, gphi, gb, ga, gf = out
+    _maps_in(x, phi, b, alpha)
+    _upstream(x, f_out, grad_x_next, grad_h_in)
+    _grads_out(x, _ag(alpha), gx, gphi, gb, ga, gf)
+    _fits(dev_status, 1, torch.int32, x.device, "dev_status")
     st = _lib.load().mhc_backward_noalloc(ctypes.byref(p), _p(x), _p(phi), _p(b), _p(alpha),
                                           _p(f_out), _p(grad_x_next), _p(grad_h_in), _p(gx),
                                           _p(gphi), _p(gb), _p(ga), _p(gf), _p(dev_status),
@@ -174,6 +253,16 @@ def mhc_post_fused(x, f_out, H_post, H_res, phi_next, b_next, alpha_next, *, t_m
                torch.empty(T, n, dtype=torch.float32, device=x.device),
                torch.empty(T, n, n, dtype=torch.float32, device=x.device))
     xn, hpre, hpost, hres = out
+    _fits(f_out, T * C, x.dtype, x.device, "f_out")
+    _fits(H_post, T * n, F32, x.device, "H_post")
+    _fits(H_res, T * n * n, F32, x.device, "H_res")
+    _maps_in(x, phi_next, b_next, alpha_next)
+    _fits(xn, T * n * C, x.dtype, x.device, "x_next")
+    _fits(hpre, T * n, F32, x.device, "H_pre_next")
+    _fits(hpost, T * n, F32, x.device, "H_post_next")
+    _fits(hres, T * n * n, F32, x.device, "H_res_next")
+    _fits(dev_status, 1, torch.int32, x.device, "dev_status")
+    _on(workspace, x.device, "workspace")
     lib = _lib.load()
     ws, wsb = _workspace(int(lib.mhc_post_fused_workspace_size(ctypes.byref(p))), x.device,
                          workspace)
@@ -189,6 +278,9 @@ def mhc_layer_input(x, H_pre, *, out=None, dev_status=None, stream=None):
     T, n, C = x.shape
     p = params(n, T, C, x.dtype)
     h_in = torch.empty(T, C, dtype=x.dtype, device=x.device) if out is None else out
+    _fits(H_pre, T * n, F32, x.device, "H_pre")
+    _fits(h_in, T * C, x.dtype, x.device, "h_in")
+    _fits(dev_status, 1, torch.int32, x.device, "dev_status")
     st = _lib.load().mhc_layer_input(ctypes.byref(p), _p(x), _p(H_pre), _p(h_in),
                                      _p(dev_status), _stream(stream))
     _check(st, "mhc_layer_input")
@@ -204,6 +296,12 @@ def mhc_post_backward(x, f_out, H_post, grad_x_next, *, out=None, dev_status=Non
         out = (torch.empty_like(f_out),
                torch.empty(T, n * n + n, dtype=torch.float32, device=x.device))
     gf, red = out
+    _fits(f_out, T * C, x.dtype, x.device, "f_out")
+    _fits(H_post, T * n, F32, x.device, "H_post")
+    _fits(grad_x_next, T * n * C, x.dtype, x.device, "grad_x_next")
+    _fits(gf, T * C, x.dtype, x.device, "grad_f_out")
+    _fits(red, T * (n * n + n), F32, x.device, "red")
+    _fits(dev_status, 1, torch.int32, x.device, "dev_status")
     st = _lib.load().mhc_post_backward(ctypes.byref(p), _p(x), _p(f_out), _p(H_post),
                                        _p(grad_x_next), _p(gf), _p(red), _p(dev_status),
                                        _stream(stream))
@@ -222,6 +320,12 @@ def mhc_pre_backward(x, phi, b, alpha, grad_x_next, grad_h_in, red, *, t_max: in
         out = (torch.empty_like(x), torch.empty_like(phi), torch.empty_like(b),
                torch.empty_like(alpha))
     gx, gphi, gb, ga = out
+    _maps_in(x, phi, b, alpha)
+    _upstream(x, None, grad_x_next, grad_h_in)
+    _fits(red, T * (n * n + n), F32, x.device, "red")
+    _grads_out(x, _ag(alpha), gx, gphi, gb, ga, None)
+    _fits(dev_status, 1, torch.int32, x.device, "dev_status")
+    _on(workspace, x.device, "workspace")
     lib = _lib.load()
     ws, wsb = _workspace(int(lib.mhc_pre_backward_workspace_size(ctypes.byref(p))), x.device,
                          workspace)
@@ -239,6 +343,10 @@ def mhc_backward_map(x, phi, b, alpha, f_out, grad_x_next, grad_h_in, workspace,
     least mhc_backward_workspace_size bytes)."""
     T, n, C = x.shape
     p = params(n, T, C, x.dtype, t_max, eps, _ag(alpha), wait_ns)
+    _maps_in(x, phi, b, alpha)
+    _upstream(x, f_out, grad_x_next, grad_h_in)
+    _fits(dev_status, 1, torch.int32, x.device, "dev_status")
+    _on(workspace, x.device, "workspace")
     st = _lib.load().mhc_backward_map(ctypes.byref(p), _p(x), _p(phi), _p(b), _p(alpha), _p(f_out),
                                       _p(grad_x_next), _p(grad_h_in), _p(workspace),
                                       workspace.numel(), _p(dev_status), _stream(stream))
@@ -259,6 +367,11 @@ def mhc_backward_apply(x, phi, grad_x_next, grad_h_in, workspace, *, t_max: int 
                torch.empty(3 if alpha_groups == 3 else 1, dtype=torch.float32, device=x.device),
                torch.empty(T, C, dtype=x.dtype, device=x.device))
     gx, gphi, gb, ga, gf = out
+    _fits(phi, n * C * M, F32, x.device, "phi")
+    _upstream(x, None, grad_x_next, grad_h_in)
+    _grads_out(x, alpha_groups, gx, gphi, gb, ga, gf)
+    _fits(dev_status, 1, torch.int32, x.device, "dev_status")
+    _on(workspace, x.device, "workspace")
     st = _lib.load().mhc_backward_apply(ctypes.byref(p), _p(x), _p(phi), _p(grad_x_next),
                                         _p(grad_h_in), _p(gx), _p(gphi), _p(gb), _p(ga), _p(gf),
                                         _p(workspace), workspace.numel(), _p(dev_status),
@@ -272,6 +385,9 @@ def mhc_sinkhorn_knopp(logits, iters: int = 20, *, out=None, dev_status=None, st
     n = logits.shape[-1]
     B = logits.numel() // (n * n)
     res = torch.empty_like(logits) if out is None else out
+    _fits(logits, B * n * n, F32, logits.device, "logits")
+    _fits(res, B * n * n, F32, logits.device, "out")
+    _fits(dev_status, 1, torch.int32, logits.device, "dev_status")
     st = _lib.load().mhc_sinkhorn_knopp(int(n), int(iters), int(B), _p(logits), _p(res),
                                         _p(dev_status), _stream(stream))
     _check(st, "mhc_sinkhorn_knopp")
@@ -285,6 +401,10 @@ def mhc_depth_amax(H, *, out=None, dev_status=None, stream=None):
         out = (torch.empty(T, dtype=torch.float32, device=H.device),
                torch.empty(T, dtype=torch.float32, device=H.device))
     gf, gb = out
+    _fits(H, T * L * n * n, F32, H.device, "H")
+    _fits(gf, T, F32, H.device, "gain_fwd")
+    _fits(gb, T, F32, H.device, "gain_bwd")
+    _fits(dev_status, 1, torch.int32, H.device, "dev_status")
     st = _lib.load().mhc_depth_amax(int(n), int(T), int(L), _p(H), _p(gf), _p(gb),
                                     _p(dev_status), _stream(stream))
     _check(st, "mhc_depth_amax")
