@@ -47,11 +47,13 @@
  *   red (the post half's reductions, backward in training order):
  *                   [T][n*n + n] = <G_i, x_j> (row-major i, j) then <G_i, f_out>
  *
- * Parity pins (tests/test_oracle_pins.py): hand-worked and closed-form
- * Sinkhorn cases, diagonal-scaling and permutation invariants, the gate and
- * RMS special cases, the standard residual at n = 1, finite differences of
- * every backward gradient (the whole backward and the post half), and the
- * split backward against the one-call backward.
+ * Parity pins (tests/test_oracle_pins.py, fixtures in tests/golden/):
+ * hand-worked and closed-form Sinkhorn cases, diagonal-scaling and
+ * permutation invariants, the gate and RMS special cases, the standard
+ * residual at n = 1, finite differences of every backward gradient (the whole
+ * backward, the post half, and per-group alpha), three equal group scales
+ * against one shared alpha, the split backward against the one-call backward,
+ * and a hand-multiplied 2 x 2 depth product for the Amax gains.
  */
 #include <math.h>
 #include <stdint.h>
